@@ -1,0 +1,157 @@
+"""Parity oracle for the selective state-space block core (test infrastructure).
+
+Thin ctypes wrapper around ``ssm_oracle.c``, the plain double-precision CPU
+definition of the method. Only the test suite, the package smoke check and the
+benchmark's CPU-baseline leg may import this package; the product path never
+does, and nothing here is shared with the CUDA sources.
+
+Arrays are widened exactly to float64 before the call (bf16/fp32 -> f64 is
+exact), so the oracle sees the very values the kernels read.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "ssm_oracle.c")
+LIB = os.path.join(HERE, "libssm_oracle.so")
+
+EULER_B = 0
+ZOH = 1
+_DISC = {"euler": EULER_B, "euler_b": EULER_B, "zoh": ZOH}
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ssm_oracle.c into libssm_oracle.so (gcc, OpenMP, IEEE math)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", SRC, "-o", LIB, "-lm"]
+        subprocess.run(cmd, check=True)
+    return LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(LIB)
+        d, i64, i32 = ctypes.c_double, ctypes.c_int64, ctypes.c_int
+        p = ctypes.c_void_p
+        lib.oracle_scan.argtypes = [i64, i32, i32, p, p, p, p, p, d, p, p, p]
+        lib.oracle_scan.restype = None
+        lib.oracle_channels.argtypes = [i64, i64, i32, i32, i32, d, d] + [p] * 5 + [p] * 7 + [p, p] + [p, p, p] + [i32]
+        lib.oracle_channels.restype = None
+        lib.oracle_causal_conv.argtypes = [i64, i32, p, p, p, d, p]
+        lib.oracle_causal_conv.restype = None
+        for name in ("oracle_silu", "oracle_softplus", "oracle_A"):
+            getattr(lib, name).argtypes = [d]
+            getattr(lib, name).restype = d
+        lib.oracle_dt.argtypes = [d, d, d, d, d]
+        lib.oracle_dt.restype = d
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = i32
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def silu(v: float) -> float:
+    return _load().oracle_silu(float(v))
+
+
+def softplus(v: float) -> float:
+    return _load().oracle_softplus(float(v))
+
+
+def dt_of(dt_raw: float, w_dt: float, dt_bias: float, lo: float, hi: float) -> float:
+    return _load().oracle_dt(float(dt_raw), float(w_dt), float(dt_bias), float(lo), float(hi))
+
+
+def A_of(A_log: float) -> float:
+    return _load().oracle_A(float(A_log))
+
+
+def causal_conv(x, w, bias=0.0, hist=None):
+    """Causal depthwise conv of one channel: returns c[L]."""
+    x, w, hist = _f64(x), _f64(w), _f64(hist)
+    L, K = x.shape[0], w.shape[0]
+    c = np.empty(max(L, 1))
+    _load().oracle_causal_conv(L, K, _ptr(hist), _ptr(x), _ptr(w), float(bias), _ptr(c))
+    return c[:L]
+
+
+def scan(u, dt, A, B, C, D=0.0, h0=None, disc="euler"):
+    """Selective scan of one channel. u, dt: [L]; A: [N]; B, C: [L, N].
+    Returns (y_pre_gate[L], h_final[N])."""
+    u, dt, A, B, C, h0 = map(_f64, (u, dt, A, B, C, h0))
+    L, N = u.shape[0], A.shape[0]
+    assert B.shape == (L, N) and C.shape == (L, N) and dt.shape == (L,)
+    y = np.empty(max(L, 1))
+    h = np.empty(N)
+    _load().oracle_scan(L, N, _DISC[disc], _ptr(u), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), float(D), _ptr(h0), _ptr(y), _ptr(h))
+    return y[:L], h
+
+
+def channels(x, z, B, C, dt_raw, bidx, conv_w, conv_b, w_dt, dt_bias, A_log, D,
+             hist=None, h0=None, lo=1e-4, hi=1.0, disc="euler", threads=0):
+    """Run the block core on n independent channels.
+
+    x, z: [n, L] (the channel's columns); B, C: [nseq, L, N]; dt_raw: [nseq, L];
+    bidx: [n] sequence index of each channel; conv_w: [n, K]; conv_b, w_dt,
+    dt_bias, D: [n]; A_log: [n, N]; hist: [n, K-1] or None; h0: [n, N] or None.
+    Returns (out[n, L], h_out[n, N], hist_out[n, K-1]) in float64."""
+    x, z, B, C, dt_raw = map(_f64, (x, z, B, C, dt_raw))
+    conv_w, conv_b, w_dt, dt_bias, A_log, D, hist, h0 = map(_f64, (conv_w, conv_b, w_dt, dt_bias, A_log, D, hist, h0))
+    bidx = np.ascontiguousarray(np.asarray(bidx, dtype=np.int64))
+    n, L = x.shape
+    N, K = A_log.shape[1], conv_w.shape[1]
+    assert z.shape == (n, L) and B.shape[1:] == (L, N) and C.shape == B.shape and dt_raw.shape == B.shape[:2]
+    assert bidx.shape == (n,) and (n == 0 or (bidx.min() >= 0 and bidx.max() < B.shape[0]))
+    out = np.empty((n, max(L, 1)))
+    h_out = np.empty((n, N))
+    hist_out = np.empty((n, max(K - 1, 1)))
+    _load().oracle_channels(n, L, N, K, _DISC[disc], float(lo), float(hi), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
+                            _ptr(bidx), _ptr(conv_w), _ptr(conv_b), _ptr(w_dt), _ptr(dt_bias), _ptr(A_log), _ptr(D),
+                            _ptr(hist), _ptr(h0), _ptr(out), _ptr(h_out), _ptr(hist_out), int(threads))
+    return out[:, :L], h_out, hist_out[:, : K - 1]
+
+
+def prefill_sampled(x, z, B, C, dt_raw, conv_w, conv_b, w_dt, dt_bias, A_log, D, chans,
+                    conv_cache_in=None, ssm_state_in=None, lo=1e-4, hi=1.0, disc="euler", threads=0):
+    """Oracle prefill on selected channels of dense inputs.
+
+    x, z: [b, L, E] (any row stride); B, C: [b, L, N]; dt_raw: [b, L];
+    parameters [E] / [E, K] / [E, N]; conv_cache_in: [b, K-1, E] or None;
+    ssm_state_in: [b, E, N] or None; chans: list of (batch, channel) pairs.
+    Returns (out[n, L], state[n, N], conv_cache[n, K-1]) for those channels."""
+    bs = np.array([c[0] for c in chans], dtype=np.int64)
+    es = np.array([c[1] for c in chans], dtype=np.int64)
+
+    def cols(t):  # [b, L, E] -> [n, L]
+        return np.stack([_f64(t[b, :, e]) for b, e in zip(bs, es)]) if len(bs) else np.empty((0, t.shape[1]))
+
+    hist = None if conv_cache_in is None else np.stack([_f64(conv_cache_in[b, :, e]) for b, e in zip(bs, es)])
+    h0 = None if ssm_state_in is None else np.stack([_f64(ssm_state_in[b, e, :]) for b, e in zip(bs, es)])
+    conv_w, conv_b, w_dt, dt_bias, A_log, D = map(_f64, (conv_w, conv_b, w_dt, dt_bias, A_log, D))
+    return channels(cols(x), cols(z), B, C, dt_raw, bs, conv_w[es], conv_b[es], w_dt[es], dt_bias[es], A_log[es], D[es],
+                    hist=hist, h0=h0, lo=lo, hi=hi, disc=disc, threads=threads)
