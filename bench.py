@@ -1,0 +1,432 @@
+"""Benchmark of the selective-scan block core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one prefill (conv, SiLU, dt, discretisation, scan, D skip, gate,
+final state and conv cache) over one batch of the workload, inputs resident in
+HBM. Default workload: long-context prefill, b=1, L=65536, E=7680, N=16, K=4,
+bf16 x/z/y, fp32 B/C/dt_raw/state (3 GB of inputs: larger than L2, so no
+flush is needed between steps). The JSON line also carries the decode
+workload (prompt 512, then 1024 one-token steps at b=256, E=7680), the
+roofline of the dominant kernel, the oracle timed on the host cores, and an
+end-to-end figure through the API with host buffers.
+
+With N > 1 (torchrun, one process per GPU) every rank runs the same per-GPU
+workload on its own channels (weak scaling; channels shard with no collective
+on the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_depthwise_b200 import workloads as W  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+PROFILES = os.path.join(ROOT, "profiles")
+FALLBACK_HBM_GBS = 6650.0
+
+# SM resources used to derive the ALU roofline (B200, sm_100a): 148 SMs,
+# 16 SFU lanes and 128 FP32 lanes per SM per clock (the SFU and FFMA rates
+# were confirmed by a throughput probe on this GPU model).
+SMS, SFU_PER_CLK, FMA_PER_CLK = 148, 16, 128
+# Per channel-token the method needs 16 exp (dA) + 2 sigmoid (exp + reciprocal)
+# + 1 softplus (exp + log1p) = 22 SFU-class evaluations, and 4 FP32 ops per
+# state (dt*A, dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 84 FP32-pipe ops.
+SFU_OPS_PER_CT, FMA_OPS_PER_CT, POLY_EXP_FMA_OPS = 22, 84, 8
+
+
+def alu_peak_ct_per_s(sm_mhz: float) -> float:
+    """Best channel-tokens/s the SM pipes allow when k of the 22 SFU
+    evaluations move to an FMA-pipe polynomial (~8 FP32 ops each): minimise
+    max((22-k)/16, (84+8k)/128) clocks per channel-token per SM."""
+    best = math.inf
+    for i in range(0, 2201):
+        k = i / 100.0
+        best = min(best, max((SFU_OPS_PER_CT - k) / SFU_PER_CLK, (FMA_OPS_PER_CT + POLY_EXP_FMA_OPS * k) / FMA_PER_CLK))
+    return SMS * sm_mhz * 1e6 / best
+
+
+def min_bytes_prefill(w: W.Workload) -> float:
+    """Algorithmic bytes of one prefill: read x, z, B, C, dt_raw and the
+    parameters once, write y, the final state and conv cache once."""
+    io = 2 if w.io_dtype == torch.bfloat16 else 4
+    b, L, E, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    act = b * L * E * io * 3 + b * L * (2 * N + 1) * 4
+    params = E * (4 + 1 + 1 + 1 + N + 1) * 4
+    caches = b * E * N * 4 + b * 3 * E * io
+    return float(act + params + caches)
+
+
+def min_bytes_decode_step(w: W.Workload) -> float:
+    """One decode step: state read + write, cache read + write, x, z, y, B, C,
+    dt_raw, parameters."""
+    io = 2 if w.io_dtype == torch.bfloat16 else 4
+    b, E, N = w.batch, w.d_inner, w.d_state
+    return float(2 * b * E * N * 4 + 2 * b * 3 * E * io + 3 * b * E * io + b * (2 * N + 1) * 4
+                 + E * (4 + 1 + 1 + 1 + N + 1) * 4)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "selective_state_space_depthwise_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, n), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(PROFILES, "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[f"{kernel}:{workload}"]
+        if e.get("source_hash") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- oracle ---
+def cpu_baseline(w: W.Workload, target_s: float = 10.0):
+    """The oracle, as it stands, on the host cores: n channels of sequence 0
+    over the workload's full length, n sized for about `target_s` of wall time."""
+    import oracle
+
+    oracle.build()
+    params = W.make_params(w)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    L, N = w.seqlen, w.d_state
+    threads = oracle.max_threads()
+
+    def run(n):
+        x = torch.randn((n, L), generator=g).to(w.io_dtype).double().numpy()
+        z = torch.randn((n, L), generator=g).to(w.io_dtype).double().numpy()
+        B = torch.randn((1, L, N), generator=g).double().numpy()
+        C = torch.randn((1, L, N), generator=g).double().numpy()
+        dt = torch.randn((1, L), generator=g).double().numpy()
+        e = slice(0, n)
+        p = {k: v[e].double().numpy() for k, v in params.items()}
+        t0 = time.perf_counter()
+        oracle.channels(x, z, B, C, dt, [0] * n, p["conv_w"], p["conv_b"], p["w_dt"], p["dt_bias"], p["A_log"],
+                        p["D"], lo=w.dt_min, hi=w.dt_max, threads=threads)
+        return time.perf_counter() - t0
+
+    cal_n = max(threads, 1)
+    cal = run(cal_n)
+    n = int(min(w.d_inner, max(cal_n, cal_n * target_s / max(cal, 1e-3))))
+    n = max(threads, (n // threads) * threads)
+    dt_s = run(n)
+    return {"value": n * L / dt_s, "unit": "channel-tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} channels x L={L} of the {w.name} workload, float64, OpenMP over channels",
+            "seconds": round(dt_s, 3)}
+
+
+# ------------------------------------------------------------------- GPU ---
+def make_device_inputs(w: W.Workload, rank: int):
+    wr = w.scaled(seed=w.seed + 1000 * rank) if rank else w
+    return W.make_inputs(wr, device="cuda", gen_device="cuda")
+
+
+def timed_prefill(inp, steps, warmup, dist):
+    from selective_state_space_depthwise_b200 import api
+
+    args = (inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp)
+    y, cc, st = api.prefill(*args)
+    for _ in range(warmup):
+        api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(stream)
+        for _ in range(steps):
+            api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        torch.distributed.barrier()
+    ms = ev0.elapsed_time(ev1)
+    return ms, clk.summary()
+
+
+def e2e_prefill(w: W.Workload, inp, steps):
+    """Same metric through the public API with host buffers: every step copies
+    the step's inputs from pinned host memory, runs the prefill and reads the
+    outputs back."""
+    from selective_state_space_depthwise_b200 import api
+
+    names = ("x", "z", "B", "C", "dt_raw")
+    host = {k: inp[k].to("cpu").pin_memory() for k in names}
+    dev = {k: torch.empty_like(inp[k]) for k in names}
+    params = {k: inp[k] for k in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")}
+    b, L, E = w.batch, w.seqlen, w.d_inner
+    y = torch.empty((b, L, E), dtype=w.io_dtype, device="cuda")
+    cc = torch.empty((b, 3, E), dtype=w.io_dtype, device="cuda")
+    st = torch.empty((b, E, 16), dtype=torch.float32, device="cuda")
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    cc_h = torch.empty(cc.shape, dtype=cc.dtype).pin_memory()
+    st_h = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = y.numel() * y.element_size() + cc.numel() * cc.element_size() + st.numel() * st.element_size()
+
+    def step():
+        for k in names:
+            dev[k].copy_(host[k], non_blocking=True)
+        api.prefill(dev["x"], dev["z"], dev["B"], dev["C"], dev["dt_raw"], params, y=y, conv_cache_out=cc,
+                    ssm_state_out=st)
+        y_h.copy_(y, non_blocking=True)
+        cc_h.copy_(cc, non_blocking=True)
+        st_h.copy_(st, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    return {"value": b * L * E / (ms * 1e-3), "unit": "channel-tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
+
+
+def decode_bench(w: W.Workload, rank: int, hbm_peak: float, peak_kind: str):
+    """Prompt prefill (untimed), then the workload's one-token steps, each a
+    separate C call; per-step device time from CUDA events."""
+    from selective_state_space_depthwise_b200 import api
+
+    inp = make_device_inputs(w, rank)
+    L0, steps = w.seqlen, w.decode_steps
+    pre = {**inp, **{k: inp[k][:, :L0] for k in ("x", "z", "B", "C", "dt_raw")}}
+    _, cc, st = api.prefill(pre["x"], pre["z"], pre["B"], pre["C"], pre["dt_raw"], pre)
+    y = torch.empty((w.batch, w.d_inner), dtype=w.io_dtype, device="cuda")
+    cc0, st0 = cc.clone(), st.clone()
+
+    def step(t):
+        api.decode_step(inp["x"][:, t], inp["z"][:, t], inp["B"][:, t], inp["C"][:, t], inp["dt_raw"][:, t], inp,
+                        cc, st, y=y)
+
+    for t in range(L0, L0 + 8):  # warm-up on the first tokens, then restore the caches
+        step(t)
+    cc.copy_(cc0)
+    st.copy_(st0)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for t in range(L0, L0 + steps):
+        step(t)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    us = ev0.elapsed_time(ev1) * 1e3 / steps
+    ct = w.batch * w.d_inner
+    gbs = min_bytes_decode_step(w) / (us * 1e-6) / 1e9
+    return {"workload": f"decode b={w.batch} E={w.d_inner} N=16 K=4 bf16 x/z/y, fp32 state; prompt {L0}, "
+                        f"{steps} one-token steps",
+            "us_per_step": round(us, 2), "value": ct / (us * 1e-6), "unit": "channel-tokens/s",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4), "peak_kind": peak_kind,
+                         "traffic": ncu_traffic("decode", "decode"),
+                         "algorithmic_bytes_per_launch": min_bytes_decode_step(w)},
+            "gpu_launches": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long_context", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode sub-benchmark")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = W.WORKLOADS[args.workload]
+    if w.decode_steps:
+        ap.error("the step workload must be a prefill shape; the decode workload is reported alongside")
+
+    if args.impl == "reference":
+        # The oracle is the reference arm: rank 0 alone runs it on the host cores.
+        if rank != 0:
+            return
+        per_step = []
+        cb = None
+        for i in range(args.warmup + args.steps):
+            cb = cpu_baseline(w, target_s=2.0)
+            if i >= args.warmup:
+                per_step.append(cb["value"])
+        value = statistics.median(per_step)
+        cb["value"] = value
+        print(json.dumps({"impl": "reference", "metric": "selective-scan channel-tokens/s", "value": value,
+                          "unit": "channel-tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+                          "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64", "data": "synthetic", "config": {"workload": w.note, "batch": w.batch,
+                                                                          "seq_len": w.seqlen, "d_inner": w.d_inner},
+                          "cpu_baseline": cb,
+                          "e2e": {"value": value, "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+
+    dist = world > 1
+    if dist:
+        import datetime
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    from selective_state_space_depthwise_b200 import _lib
+
+    _lib.load()
+    hbm_peak, peak_kind = load_peaks()
+
+    inp = make_device_inputs(w, rank)
+    ms, clocks = timed_prefill(inp, args.steps, args.warmup, dist)
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    ct_step = w.batch * w.seqlen * w.d_inner
+    value = ct_step * world / (ms_step * 1e-3)
+    per_gpu = ct_step / (ms_step * 1e-3)
+    gbs = min_bytes_prefill(w) / (ms_step * 1e-3) / 1e9
+    sm_mhz = clocks["sm_mhz"] if clocks else 1965.0
+    peak_ct = alu_peak_ct_per_s(1965.0)
+
+    extra = {}
+    if rank == 0:
+        if not args.no_e2e:
+            extra["e2e"] = e2e_prefill(w, inp, steps=3)
+            extra["e2e"]["value"] *= world
+        del inp
+        torch.cuda.empty_cache()
+        if not args.no_decode:
+            extra["decode"] = decode_bench(W.WORKLOADS["decode"], rank, hbm_peak, peak_kind)
+        if not args.no_cpu and world == 1:
+            extra["cpu_baseline"] = cpu_baseline(w)
+    if dist:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    line = {
+        "metric": "selective-scan channel-tokens/s (prefill); achieved HBM GB/s vs B200 peak",
+        "value": value, "unit": "channel-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "io_dtype": "bf16" if w.io_dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.note}; b={w.batch} L={w.seqlen} E={w.d_inner} N=16 K=4",
+                   "batch": w.batch, "seq_len": w.seqlen, "d_inner": w.d_inner, "d_state": 16, "d_conv": 4,
+                   "parallelism": f"dp{world} (channel shards, no collective)" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (no flush)" if min_bytes_prefill(w) > 126e6 else "inputs fit in L2"},
+        "roofline": {"bound": "alu", "achieved": per_gpu, "peak": peak_ct, "unit": "channel-tokens/s",
+                     "frac": round(per_gpu / peak_ct, 4),
+                     "peak_basis": "SFU 16 + FP32 128 lanes/clk/SM x 148 SMs at 1965 MHz, 22 SFU-class + 84 FP32 "
+                                   "ops per channel-token, best SFU/FMA split",
+                     "traffic": ncu_traffic("prefill", w.name),
+                     "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                             "frac": round(gbs / hbm_peak, 4), "peak_kind": peak_kind,
+                             "algorithmic_bytes_per_launch": min_bytes_prefill(w)}},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    line.update(extra)
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

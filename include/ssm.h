@@ -1,0 +1,173 @@
+/*
+ * ssm.h -- C ABI of the B200 (sm_100a) selective state-space block core.
+ *
+ * The block core computes, per channel e of every sequence (Mamba-style,
+ * diagonal A, one B/C group shared by all channels):
+ *
+ *   c_t   = conv_b[e] + sum_{k<4} conv_w[e,k] * xh[t+k]    causal depthwise conv,
+ *           xh = [3 history rows, x_0 .. x_{L-1}]           weight 3 = current token
+ *   u_t   = SiLU(c_t)
+ *   dt_t  = clip(softplus(dt_raw_t * w_dt[e] + dt_bias[e]), dt_min, dt_max)
+ *   A_n   = -exp(A_log[e,n])
+ *   h_n   <- exp(dt_t A_n) h_n + dt_t B_{t,n} u_t          (Euler-B, default)
+ *            exp(dt_t A_n) h_n + (exp(dt_t A_n)-1)/A_n B_{t,n} u_t   (ZOH)
+ *   y_t   = (sum_n C_{t,n} h_n + D[e] u_t) * SiLU(z_t)
+ *
+ * Sources: "Axon-SSM: selective state space model" (Bit-Axon docs), the block
+ * diagram under "Algorithm" (conv1d causal kernel=4 groups=E, SiLU, x_proj to
+ * B, C, dt_raw, dt_proj 1->E with softplus and clip, scan, y*SiLU(z)),
+ * "State initialization" (A = -exp(A_log)), "JIT-compiled kernels"
+ * (_ssm_fma: dA*h + dB*x_t; _compute_dt: clip(softplus(dt+dt_bias),lo,hi)) and
+ * "Autoregressive decoding" (prefill from cache=None with a zero state that
+ * builds conv_cache from the last K-1 positions; decode = one scan step that
+ * carries [conv_cache, ssm_state]). The zero-order-hold option follows "Mamba/
+ * SSM basics" (molayo insights), "Technical details"; the D skip on the scan
+ * input follows "What is the Mamba model?" (velog), "chunkscan". Two entry
+ * points, one per mode, as "Understanding the selective state space model from
+ * the implementation side" (molayo insights) recommends in its reading
+ * checklist (separate full-sequence scan and incremental update).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    allocates no device memory and keeps no per-call state.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = the
+ *    legacy default stream); nothing synchronises the host. Launch failures
+ *    return SSM_ERR_CUDA; faults during execution surface at the caller's next
+ *    synchronisation.
+ *  - Argument checks happen on the host before any launch: a NULL required
+ *    pointer, a non-positive size, a misaligned pointer or stride returns
+ *    SSM_ERR_INVALID_ARG; d_state != 16 or d_conv != 4 returns
+ *    SSM_ERR_UNSUPPORTED. ssm_last_error() then describes the failure.
+ *  - Strides are in elements; 0 selects the dense default. x, z, y and
+ *    conv_cache use `io_dtype`; B, C, dt_raw, the parameters and ssm_state are
+ *    fp32. Pointers of x, z, y, B, C, dt_raw must be 16-byte aligned and the
+ *    non-zero strides of x, z, y multiples of 8 elements (16 bytes at bf16),
+ *    those of B, C multiples of 4 elements; d_inner must be a multiple of 8.
+ */
+#ifndef SSM_B200_H
+#define SSM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SSM_OK = 0,
+  SSM_ERR_INVALID_ARG = 1,
+  SSM_ERR_UNSUPPORTED = 2,
+  SSM_ERR_CUDA = 3,
+  SSM_ERR_DEVICE = 4 /* a kernel reported a failure through the error word */
+} ssm_status;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+typedef enum { SSM_DISC_EULER_B = 0, SSM_DISC_ZOH = 1 } ssm_discretization;
+
+/* Problem shape, options and tensor strides (elements; 0 = dense default). */
+typedef struct {
+  int64_t batch;          /* b: independent sequences (> 0) */
+  int64_t seqlen;         /* L: tokens per sequence for prefill (>= 0); decode ignores it */
+  int64_t d_inner;        /* E: channels (> 0, multiple of 8) */
+  int32_t d_state;        /* N: must be 16 */
+  int32_t d_conv;         /* K: must be 4 */
+  float dt_min, dt_max;   /* clip bounds of dt, 0 < dt_min <= dt_max */
+  int32_t io_dtype;       /* ssm_dtype of x, z, y, conv_cache */
+  int32_t discretization; /* ssm_discretization */
+  /* x, z, y: element (s, t, e) lives at s*seq_stride + t*tok_stride + e.
+   * Dense defaults: tok_stride = E, seq_stride = L*tok_stride (prefill) or
+   * tok_stride (decode, where t is absent). A fused in_proj buffer [b, L, 2E]
+   * passes x = buf, z = buf + E with tok_stride = 2E. */
+  int64_t x_tok_stride, x_seq_stride;
+  int64_t z_tok_stride, z_seq_stride;
+  int64_t y_tok_stride, y_seq_stride;
+  /* B, C: element (s, t, n) at s*bc_seq_stride + t*bc_tok_stride + n.
+   * Dense: bc_tok_stride = 16, bc_seq_stride = L*16 (decode: 16).
+   * dt_raw: element (s, t) at s*dt_seq_stride + t. Dense: L (decode: 1). */
+  int64_t bc_tok_stride, bc_seq_stride;
+  int64_t dt_seq_stride;
+} ssm_dims;
+
+/* Per-channel parameters, fp32, dense, device pointers (all required).
+ * conv_w [E][4], conv_b [E], w_dt [E], dt_bias [E], A_log [E][16], D [E]. */
+typedef struct {
+  const float *conv_w, *conv_b, *w_dt, *dt_bias, *A_log, *D;
+} ssm_weights;
+
+/* Launch shape overrides for tests and tuning; pass NULL for the defaults. */
+typedef struct {
+  int32_t threads_per_channel; /* 0 = auto, else 1, 2, 4, 8 or 16 */
+  int32_t channels_per_cta;    /* 0 = auto, else 8, 16, 32 or 64 */
+} ssm_tuning;
+
+/*
+ * ssm_prefill -- full-sequence mode ("Autoregressive decoding", first call).
+ *
+ *   x, z            [b, L, *] io_dtype (strides above)
+ *   B, C            [b, L, 16] fp32; dt_raw [b, L] fp32
+ *   conv_cache_in   [b, 3, E] io_dtype, dense, or NULL = zero history
+ *   ssm_state_in    [b, E, 16] fp32, dense, or NULL = zero state
+ *   y               [b, L, *] io_dtype (strides above); must not overlap x or z
+ *   conv_cache_out  [b, 3, E] io_dtype: the last 3 raw x rows of [history, x]
+ *   ssm_state_out   [b, E, 16] fp32: the state after the last token
+ *   workspace       device scratch of ssm_prefill_workspace_bytes() bytes, or
+ *                   NULL when that size is 0
+ * conv_cache_out may alias conv_cache_in and ssm_state_out may alias
+ * ssm_state_in (each channel reads its cache before writing it). The non-NULL
+ * *_in pointers let a long sequence be processed in pieces: feeding one call's
+ * caches to the next gives the result of one call over the whole sequence.
+ * L == 0 copies the incoming caches (or zeros) to the outputs; x, z, B, C,
+ * dt_raw and y are then not read and may be NULL.
+ */
+ssm_status ssm_prefill(const ssm_dims *dims, const ssm_weights *w, const void *x, const void *z,
+                       const float *B, const float *C, const float *dt_raw, const void *conv_cache_in,
+                       const float *ssm_state_in, void *y, void *conv_cache_out, float *ssm_state_out,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* ssm_prefill with launch-shape overrides (tuning may be NULL). */
+ssm_status ssm_prefill_ex(const ssm_dims *dims, const ssm_weights *w, const void *x, const void *z,
+                          const float *B, const float *C, const float *dt_raw, const void *conv_cache_in,
+                          const float *ssm_state_in, void *y, void *conv_cache_out, float *ssm_state_out,
+                          void *workspace, size_t workspace_bytes, const ssm_tuning *tuning, void *stream);
+
+/* Device scratch bytes ssm_prefill needs for `dims` (0 for every shape the
+ * single-pass kernel covers). Returns 0 for invalid dims as well. */
+size_t ssm_prefill_workspace_bytes(const ssm_dims *dims);
+
+/*
+ * ssm_decode_step -- one-token mode ("Autoregressive decoding", later calls):
+ * concatenates conv_cache with the new token, runs the conv for that token and
+ * exactly one scan step from ssm_state, and updates both caches IN PLACE.
+ *
+ *   x, z        [b, *] io_dtype, token of sequence s at s*x_seq_stride (dense: E)
+ *   B, C        [b, 16] fp32 at s*bc_seq_stride (dense: 16); dt_raw [b] at s*dt_seq_stride (dense: 1)
+ *   y           [b, *] io_dtype at s*y_seq_stride (dense: E)
+ *   conv_cache  [b, 3, E] io_dtype, dense, in-out
+ *   ssm_state   [b, E, 16] fp32, dense, in-out
+ * dims->seqlen is ignored. Consecutive calls on one stream continue the
+ * sequence: prefill(L) followed by k calls equals prefill(L + k).
+ */
+ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const void *x, const void *z,
+                           const float *B, const float *C, const float *dt_raw, void *y, void *conv_cache,
+                           float *ssm_state, void *stream);
+
+/* Reads and clears the device error word that kernels set when a bounded
+ * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed. */
+ssm_status ssm_check_device_error(void *stream);
+
+/* Static description of a status code. */
+const char *ssm_status_string(ssm_status s);
+
+/* Message of the last failure on the calling host thread ("" if none). */
+const char *ssm_last_error(void);
+
+/* Library version as "major.minor.patch". */
+const char *ssm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_B200_H */

@@ -1,0 +1,154 @@
+"""PyTorch-facing calls of the C ABI (include/ssm.h).
+
+Each function reads sizes and strides off the tensors, allocates missing
+outputs with torch (device memory is PyTorch's job here), and makes exactly
+one C call on the current CUDA stream. Every step of the block core runs in
+the library's CUDA kernels; tensors that are not on a CUDA device are
+rejected -- there is no CPU path.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.float32: _lib.SSM_F32, torch.bfloat16: _lib.SSM_BF16}
+_DISC = {"euler": _lib.SSM_DISC_EULER_B, "euler_b": _lib.SSM_DISC_EULER_B, "zoh": _lib.SSM_DISC_ZOH}
+PARAM_NAMES = ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(name, t, device):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise RuntimeError(f"{name} must be a CUDA tensor: the block core has no CPU path")
+    if t.device != device:
+        raise RuntimeError(f"{name} is on {t.device}, expected {device}")
+
+
+def _weights(params, E, device):
+    for n in PARAM_NAMES:
+        t = params[n]
+        _need_cuda(n, t, device)
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous float32")
+    if params["conv_w"].shape != (E, 4) or params["A_log"].shape != (E, 16):
+        raise ValueError("conv_w must be [E, 4] and A_log [E, 16]")
+    for n in ("conv_b", "w_dt", "dt_bias", "D"):
+        if params[n].shape != (E,):
+            raise ValueError(f"{n} must be [E]")
+    w = _lib.SsmWeights()
+    for n in PARAM_NAMES:
+        setattr(w, n, params[n].data_ptr())
+    return w
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_dims(batch, seqlen, E, io_dtype, dt_min=1e-4, dt_max=1.0, discretization="euler", **strides):
+    d = _lib.SsmDims()
+    d.batch, d.seqlen, d.d_inner, d.d_state, d.d_conv = batch, seqlen, E, 16, 4
+    d.dt_min, d.dt_max = dt_min, dt_max
+    d.io_dtype = _DTYPES[io_dtype] if isinstance(io_dtype, torch.dtype) else int(io_dtype)
+    d.discretization = _DISC[discretization]
+    for k, v in strides.items():
+        setattr(d, k, int(v))
+    return d
+
+
+def workspace_bytes(batch, seqlen, E, io_dtype=torch.bfloat16) -> int:
+    lib = _lib.load()
+    return int(lib.ssm_prefill_workspace_bytes(ctypes.byref(make_dims(batch, seqlen, E, io_dtype))))
+
+
+def prefill(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None, y=None, conv_cache_out=None,
+            ssm_state_out=None, dt_min=1e-4, dt_max=1.0, discretization="euler", tuning=None, stream=None):
+    """Full-sequence block core. x, z: [b, L, E] (last dim contiguous; token and
+    sequence strides are passed through); B, C: [b, L, 16]; dt_raw: [b, L].
+    Returns (y [b, L, E], conv_cache_out [b, 3, E], ssm_state_out [b, E, 16])."""
+    lib = _lib.load()
+    b, L, E = x.shape
+    dev = x.device
+    for n, t in (("x", x), ("z", z), ("B", B), ("C", C), ("dt_raw", dt_raw), ("conv_cache_in", conv_cache_in),
+                 ("ssm_state_in", ssm_state_in), ("y", y), ("conv_cache_out", conv_cache_out),
+                 ("ssm_state_out", ssm_state_out)):
+        _need_cuda(n, t, dev)
+    if x.dtype not in _DTYPES or z.dtype != x.dtype:
+        raise ValueError("x and z must share an io dtype (float32 or bfloat16)")
+    if z.shape != (b, L, E) or B.shape != (b, L, 16) or C.shape != (b, L, 16) or dt_raw.shape != (b, L):
+        raise ValueError("shape mismatch: z [b,L,E], B/C [b,L,16], dt_raw [b,L]")
+    if x.stride(2) != 1 or z.stride(2) != 1 or B.stride(2) != 1 or dt_raw.stride(1) != 1:
+        raise ValueError("the innermost dimension of x, z, B, C, dt_raw must be contiguous")
+    if B.stride() != C.stride():
+        raise ValueError("B and C must share strides")
+    if y is None:
+        y = torch.empty((b, L, E), dtype=x.dtype, device=dev)
+    if conv_cache_out is None:
+        conv_cache_out = torch.empty((b, 3, E), dtype=x.dtype, device=dev)
+    if ssm_state_out is None:
+        ssm_state_out = torch.empty((b, E, 16), dtype=torch.float32, device=dev)
+    for n, t, shp, dt in (("conv_cache_out", conv_cache_out, (b, 3, E), x.dtype),
+                          ("ssm_state_out", ssm_state_out, (b, E, 16), torch.float32),
+                          ("conv_cache_in", conv_cache_in, (b, 3, E), x.dtype),
+                          ("ssm_state_in", ssm_state_in, (b, E, 16), torch.float32)):
+        if t is not None and (t.shape != shp or t.dtype != dt or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous {dt} tensor of shape {shp}")
+    if y.shape != (b, L, E) or y.dtype != x.dtype or y.stride(2) != 1:
+        raise ValueError("y must be [b, L, E] in the io dtype with a contiguous last dim")
+    dims = make_dims(b, L, E, x.dtype, dt_min, dt_max, discretization,
+                     x_tok_stride=x.stride(1), x_seq_stride=x.stride(0), z_tok_stride=z.stride(1),
+                     z_seq_stride=z.stride(0), y_tok_stride=y.stride(1), y_seq_stride=y.stride(0),
+                     bc_tok_stride=B.stride(1), bc_seq_stride=B.stride(0), dt_seq_stride=dt_raw.stride(0))
+    w = _weights(params, E, dev)
+    ws = int(lib.ssm_prefill_workspace_bytes(ctypes.byref(dims)))
+    work = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
+    tun = None
+    if tuning:
+        tun = _lib.SsmTuning(int(tuning.get("threads_per_channel", 0)), int(tuning.get("channels_per_cta", 0)))
+    st = lib.ssm_prefill_ex(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
+                            _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(y), _ptr(conv_cache_out),
+                            _ptr(ssm_state_out), _ptr(work), ws, ctypes.byref(tun) if tun else None, _stream(stream))
+    _lib.check(st)
+    return y, conv_cache_out, ssm_state_out
+
+
+def decode_step(x, z, B, C, dt_raw, params, conv_cache, ssm_state, *, y=None, dt_min=1e-4, dt_max=1.0,
+                discretization="euler", stream=None):
+    """One-token block core. x, z: [b, E] (last dim contiguous); B, C: [b, 16];
+    dt_raw: [b]; conv_cache [b, 3, E] and ssm_state [b, E, 16] are updated in
+    place. Returns y [b, E]."""
+    lib = _lib.load()
+    b, E = x.shape
+    dev = x.device
+    for n, t in (("x", x), ("z", z), ("B", B), ("C", C), ("dt_raw", dt_raw), ("conv_cache", conv_cache),
+                 ("ssm_state", ssm_state), ("y", y)):
+        _need_cuda(n, t, dev)
+    if x.dtype not in _DTYPES or z.dtype != x.dtype or conv_cache.dtype != x.dtype:
+        raise ValueError("x, z and conv_cache must share an io dtype")
+    if z.shape != (b, E) or B.shape != (b, 16) or C.shape != (b, 16) or dt_raw.shape != (b,):
+        raise ValueError("shape mismatch: z [b,E], B/C [b,16], dt_raw [b]")
+    if x.stride(1) != 1 or z.stride(1) != 1 or B.stride(1) != 1 or B.stride() != C.stride():
+        raise ValueError("innermost dims must be contiguous and B, C share strides")
+    if conv_cache.shape != (b, 3, E) or not conv_cache.is_contiguous():
+        raise ValueError("conv_cache must be a contiguous [b, 3, E] tensor")
+    if ssm_state.shape != (b, E, 16) or ssm_state.dtype != torch.float32 or not ssm_state.is_contiguous():
+        raise ValueError("ssm_state must be a contiguous float32 [b, E, 16] tensor")
+    if y is None:
+        y = torch.empty((b, E), dtype=x.dtype, device=dev)
+    dims = make_dims(b, 1, E, x.dtype, dt_min, dt_max, discretization, x_seq_stride=x.stride(0),
+                     z_seq_stride=z.stride(0), y_seq_stride=y.stride(0), bc_seq_stride=B.stride(0),
+                     dt_seq_stride=dt_raw.stride(0))
+    w = _weights(params, E, dev)
+    st = lib.ssm_decode_step(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
+                             _ptr(y), _ptr(conv_cache), _ptr(ssm_state), _stream(stream))
+    _lib.check(st)
+    return y

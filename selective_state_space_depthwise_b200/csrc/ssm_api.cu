@@ -1,0 +1,251 @@
+// ssm_api.cu -- the extern "C" boundary declared in include/ssm.h.
+//
+// Host-side only: argument checks, stride resolution, launch-shape choice and
+// one kernel launch per call on the caller's stream. No device memory is
+// allocated and no host synchronisation happens on the compute entry points.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "ssm.h"
+#include "ssm_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+ssm_status fail(ssm_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+ssm_status ok() {
+  g_last_error[0] = '\0';
+  return SSM_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Checks shared by both modes. `prefill` selects the dense stride defaults.
+ssm_status check_dims(const ssm_dims* d, bool prefill, ssm::Strides* s) {
+  if (!d) return fail(SSM_ERR_INVALID_ARG, "dims is NULL");
+  if (d->d_state != 16) return fail(SSM_ERR_UNSUPPORTED, "d_state=%d: only 16 is built", d->d_state);
+  if (d->d_conv != 4) return fail(SSM_ERR_UNSUPPORTED, "d_conv=%d: only 4 is built", d->d_conv);
+  if (d->batch <= 0) return fail(SSM_ERR_INVALID_ARG, "batch=%lld must be > 0", (long long)d->batch);
+  if (prefill && d->seqlen < 0) return fail(SSM_ERR_INVALID_ARG, "seqlen=%lld must be >= 0", (long long)d->seqlen);
+  if (d->d_inner <= 0 || d->d_inner % 8 != 0)
+    return fail(SSM_ERR_INVALID_ARG, "d_inner=%lld must be a positive multiple of 8", (long long)d->d_inner);
+  if (!(d->dt_min > 0.0f) || !(d->dt_max >= d->dt_min))
+    return fail(SSM_ERR_INVALID_ARG, "need 0 < dt_min <= dt_max (got %g, %g)", d->dt_min, d->dt_max);
+  if (d->io_dtype != SSM_F32 && d->io_dtype != SSM_BF16)
+    return fail(SSM_ERR_INVALID_ARG, "io_dtype=%d unknown", d->io_dtype);
+  if (d->discretization != SSM_DISC_EULER_B && d->discretization != SSM_DISC_ZOH)
+    return fail(SSM_ERR_INVALID_ARG, "discretization=%d unknown", d->discretization);
+  const int64_t E = d->d_inner;
+  const int64_t L = prefill ? d->seqlen : 1;
+  s->x_tok = d->x_tok_stride ? d->x_tok_stride : E;
+  s->z_tok = d->z_tok_stride ? d->z_tok_stride : E;
+  s->y_tok = d->y_tok_stride ? d->y_tok_stride : E;
+  s->x_seq = d->x_seq_stride ? d->x_seq_stride : (prefill ? L * s->x_tok : s->x_tok);
+  s->z_seq = d->z_seq_stride ? d->z_seq_stride : (prefill ? L * s->z_tok : s->z_tok);
+  s->y_seq = d->y_seq_stride ? d->y_seq_stride : (prefill ? L * s->y_tok : s->y_tok);
+  s->bc_tok = d->bc_tok_stride ? d->bc_tok_stride : 16;
+  s->bc_seq = d->bc_seq_stride ? d->bc_seq_stride : (prefill ? L * s->bc_tok : s->bc_tok);
+  s->dt_seq = d->dt_seq_stride ? d->dt_seq_stride : (prefill ? L : 1);
+  const int64_t io[6] = {s->x_tok, s->x_seq, s->z_tok, s->z_seq, s->y_tok, s->y_seq};
+  for (int i = 0; i < 6; ++i)
+    if (io[i] < 0 || io[i] % 8 != 0)
+      return fail(SSM_ERR_INVALID_ARG, "x/z/y strides must be non-negative multiples of 8 elements");
+  if (s->x_tok < E || s->z_tok < E || s->y_tok < E)
+    return fail(SSM_ERR_INVALID_ARG, "x/z/y token strides must be >= d_inner");
+  if (s->bc_tok < 16 || s->bc_tok % 4 != 0 || s->bc_seq < 0 || s->bc_seq % 4 != 0)
+    return fail(SSM_ERR_INVALID_ARG, "B/C strides: token stride >= 16 and both multiples of 4");
+  if (s->dt_seq < 0) return fail(SSM_ERR_INVALID_ARG, "dt_raw sequence stride must be >= 0");
+  return SSM_OK;
+}
+
+ssm_status check_weights(const ssm_weights* w) {
+  if (!w) return fail(SSM_ERR_INVALID_ARG, "weights is NULL");
+  const float* p[6] = {w->conv_w, w->conv_b, w->w_dt, w->dt_bias, w->A_log, w->D};
+  const char* names[6] = {"conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D"};
+  for (int i = 0; i < 6; ++i) {
+    if (!p[i]) return fail(SSM_ERR_INVALID_ARG, "weights.%s is NULL", names[i]);
+    if (!aligned(p[i], 4)) return fail(SSM_ERR_INVALID_ARG, "weights.%s is not 4-byte aligned", names[i]);
+  }
+  return SSM_OK;
+}
+
+ssm_status check_io_ptr(const void* p, const char* name, size_t align) {
+  if (!p) return fail(SSM_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(SSM_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return SSM_OK;
+}
+
+int num_sms_current() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+void fill_weights(ssm::KernelArgs& a, const ssm_weights* w) {
+  a.conv_w = w->conv_w;
+  a.conv_b = w->conv_b;
+  a.w_dt = w->w_dt;
+  a.dt_bias = w->dt_bias;
+  a.A_log = w->A_log;
+  a.D = w->D;
+}
+
+__device__ int g_device_error = 0;
+
+}  // namespace
+
+extern "C" {
+
+size_t ssm_prefill_workspace_bytes(const ssm_dims* dims) {
+  (void)dims;
+  return 0;
+}
+
+ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                          const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
+                          void* y, void* conv_cache_out, float* ssm_state_out, void* workspace, size_t workspace_bytes,
+                          const ssm_tuning* tuning, void* stream) {
+  ssm::Strides s;
+  ssm_status st = check_dims(dims, true, &s);
+  if (st != SSM_OK) return st;
+  if ((st = check_weights(w)) != SSM_OK) return st;
+  if (dims->seqlen > 0) {  // with L == 0 the token tensors are not read and may be NULL
+    if ((st = check_io_ptr(x, "x", 16)) != SSM_OK) return st;
+    if ((st = check_io_ptr(z, "z", 16)) != SSM_OK) return st;
+    if ((st = check_io_ptr(y, "y", 16)) != SSM_OK) return st;
+    if ((st = check_io_ptr(B, "B", 16)) != SSM_OK) return st;
+    if ((st = check_io_ptr(C, "C", 16)) != SSM_OK) return st;
+    if ((st = check_io_ptr(dt_raw, "dt_raw", 4)) != SSM_OK) return st;
+    if (y == x || y == z) return fail(SSM_ERR_INVALID_ARG, "y must not alias x or z");
+  }
+  if ((st = check_io_ptr(conv_cache_out, "conv_cache_out", 16)) != SSM_OK) return st;
+  if ((st = check_io_ptr(ssm_state_out, "ssm_state_out", 16)) != SSM_OK) return st;
+  if (conv_cache_in && !aligned(conv_cache_in, 16)) return fail(SSM_ERR_INVALID_ARG, "conv_cache_in not 16-byte aligned");
+  if (ssm_state_in && !aligned(ssm_state_in, 4)) return fail(SSM_ERR_INVALID_ARG, "ssm_state_in not 4-byte aligned");
+  if (workspace_bytes < ssm_prefill_workspace_bytes(dims))
+    return fail(SSM_ERR_INVALID_ARG, "workspace too small");
+  (void)workspace;
+
+  ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current());
+  if (tuning) {
+    if (tuning->threads_per_channel) sh.G = tuning->threads_per_channel;
+    if (tuning->channels_per_cta) sh.NCH = tuning->channels_per_cta;
+    if (!ssm::prefill_shape_supported(sh))
+      return fail(SSM_ERR_INVALID_ARG, "tuning: unsupported shape G=%d NCH=%d", sh.G, sh.NCH);
+  }
+
+  ssm::KernelArgs a{};
+  a.x = x;
+  a.z = z;
+  a.B = B;
+  a.C = C;
+  a.dt_raw = dt_raw;
+  fill_weights(a, w);
+  a.conv_cache_in = conv_cache_in;
+  a.ssm_state_in = ssm_state_in;
+  a.y = y;
+  a.conv_cache_out = conv_cache_out;
+  a.ssm_state_out = ssm_state_out;
+  a.batch = dims->batch;
+  a.L = dims->seqlen;
+  a.E = dims->d_inner;
+  a.s = s;
+  a.dt_min = dims->dt_min;
+  a.dt_max = dims->dt_max;
+  cudaError_t err = ssm::launch_prefill(a, dims->io_dtype == SSM_BF16, dims->discretization == SSM_DISC_ZOH, sh,
+                                        static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+ssm_status ssm_prefill(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                       const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
+                       void* y, void* conv_cache_out, float* ssm_state_out, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  return ssm_prefill_ex(dims, w, x, z, B, C, dt_raw, conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out,
+                        workspace, workspace_bytes, nullptr, stream);
+}
+
+ssm_status ssm_decode_step(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                           const float* C, const float* dt_raw, void* y, void* conv_cache, float* ssm_state,
+                           void* stream) {
+  ssm::Strides s;
+  ssm_status st = check_dims(dims, false, &s);
+  if (st != SSM_OK) return st;
+  if ((st = check_weights(w)) != SSM_OK) return st;
+  const size_t io_size = dims->io_dtype == SSM_BF16 ? 2 : 4;
+  if ((st = check_io_ptr(x, "x", io_size)) != SSM_OK) return st;
+  if ((st = check_io_ptr(z, "z", io_size)) != SSM_OK) return st;
+  if ((st = check_io_ptr(y, "y", io_size)) != SSM_OK) return st;
+  if ((st = check_io_ptr(B, "B", 16)) != SSM_OK) return st;
+  if ((st = check_io_ptr(C, "C", 16)) != SSM_OK) return st;
+  if ((st = check_io_ptr(dt_raw, "dt_raw", 4)) != SSM_OK) return st;
+  if ((st = check_io_ptr(conv_cache, "conv_cache", io_size)) != SSM_OK) return st;
+  if ((st = check_io_ptr(ssm_state, "ssm_state", 16)) != SSM_OK) return st;
+  if (y == x || y == z) return fail(SSM_ERR_INVALID_ARG, "y must not alias x or z");
+
+  ssm::KernelArgs a{};
+  a.x = x;
+  a.z = z;
+  a.B = B;
+  a.C = C;
+  a.dt_raw = dt_raw;
+  fill_weights(a, w);
+  a.conv_cache_in = conv_cache;
+  a.ssm_state_in = ssm_state;
+  a.y = y;
+  a.conv_cache_out = conv_cache;
+  a.ssm_state_out = ssm_state;
+  a.batch = dims->batch;
+  a.L = 1;
+  a.E = dims->d_inner;
+  a.s = s;
+  a.dt_min = dims->dt_min;
+  a.dt_max = dims->dt_max;
+  cudaError_t err = ssm::launch_decode(a, dims->io_dtype == SSM_BF16, dims->discretization == SSM_DISC_ZOH,
+                                       static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+  return ok();
+}
+
+ssm_status ssm_check_device_error(void* stream) {
+  int v = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(st);
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "device error check: %s", cudaGetErrorString(err));
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    cudaStreamSynchronize(st);
+    return fail(SSM_ERR_DEVICE, "a kernel reported device error code %d", v);
+  }
+  return ok();
+}
+
+const char* ssm_status_string(ssm_status s) {
+  switch (s) {
+    case SSM_OK: return "ok";
+    case SSM_ERR_INVALID_ARG: return "invalid argument";
+    case SSM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SSM_ERR_CUDA: return "CUDA error";
+    case SSM_ERR_DEVICE: return "device-side failure";
+  }
+  return "unknown status";
+}
+
+const char* ssm_last_error(void) { return g_last_error; }
+
+const char* ssm_version(void) { return "0.1.0"; }
+
+}  // extern "C"

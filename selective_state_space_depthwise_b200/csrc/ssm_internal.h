@@ -1,0 +1,52 @@
+// ssm_internal.h -- launch interface between the C ABI and the CUDA kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Element strides of every strided tensor (already resolved from the ABI's
+// "0 = dense" convention).
+struct Strides {
+  int64_t x_tok, x_seq, z_tok, z_seq, y_tok, y_seq;
+  int64_t bc_tok, bc_seq, dt_seq;
+};
+
+// Arguments of both modes. For decode, L is 1 and the *_in / *_out cache
+// pointers are the same in-out buffers.
+struct KernelArgs {
+  const void* x;
+  const void* z;
+  const float* B;
+  const float* C;
+  const float* dt_raw;
+  const float* conv_w;
+  const float* conv_b;
+  const float* w_dt;
+  const float* dt_bias;
+  const float* A_log;
+  const float* D;
+  const void* conv_cache_in;
+  const float* ssm_state_in;
+  void* y;
+  void* conv_cache_out;
+  float* ssm_state_out;
+  int64_t batch, L, E;
+  Strides s;
+  float dt_min, dt_max;
+};
+
+// Prefill launch shape: G threads per channel (each holding 16/G states) and
+// NCH channels per CTA.
+struct PrefillShape {
+  int G;
+  int NCH;
+};
+
+PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t L, int num_sms);
+bool prefill_shape_supported(PrefillShape sh);
+cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st);
+cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStream_t st);
+
+}  // namespace ssm

@@ -94,6 +94,8 @@ def _randn_chunked(shape, g, device, dtype, chunk_elems=1 << 28):
     """N(0,1) drawn in fp32 and rounded (RNE) to `dtype`, in bounded chunks
     along the leading dimension to cap the fp32 temporary."""
     out = torch.empty(shape, dtype=dtype, device=device)
+    if out.numel() == 0:
+        return out
     flat = out.view(shape[0], -1)
     per_row = flat.shape[1]
     rows = max(1, chunk_elems // max(per_row, 1))

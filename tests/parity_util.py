@@ -1,0 +1,74 @@
+"""Helpers shared by the GPU parity tests: oracle runs over chosen channels and
+the comparison metrics (relative L2 per tensor, bit-exact caches)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+TOL = {torch.float32: 1e-5, torch.bfloat16: 2e-3}  # relative L2 of outputs and final states, per io dtype
+
+
+def rel_l2(got, want) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    den = np.linalg.norm(want)
+    num = np.linalg.norm(got - want)
+    return float(num / den) if den > 0 else float(num)
+
+
+def round_io(a, dtype) -> np.ndarray:
+    """Round oracle values once to the io dtype (RNE), back to float64."""
+    return torch.from_numpy(np.asarray(a, dtype=np.float64)).to(dtype).double().numpy()
+
+
+def all_channels(b, E):
+    return [(s, e) for s in range(b) for e in range(E)]
+
+
+def oracle_prefill(inp, chans, *, L=None, conv_cache_in=None, ssm_state_in=None, dt_min=1e-4, dt_max=1.0,
+                   disc="euler", threads=0):
+    """Oracle over `chans` of inputs shaped like the kernel's (CPU or GPU
+    tensors; the stored values are read back exactly). L limits the tokens."""
+    x, z, B, C, dt = inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"]
+    if L is not None:
+        x, z, B, C, dt = x[:, :L], z[:, :L], B[:, :L], C[:, :L], dt[:, :L]
+    seqs = sorted({s for s, _ in chans})
+    remap = {s: i for i, s in enumerate(seqs)}
+    Bn = B[seqs].detach().to("cpu").double().numpy()
+    Cn = C[seqs].detach().to("cpu").double().numpy()
+    dtn = dt[seqs].detach().to("cpu").double().numpy()
+    xs = np.stack([x[s, :, e].detach().to("cpu").double().numpy() for s, e in chans])
+    zs = np.stack([z[s, :, e].detach().to("cpu").double().numpy() for s, e in chans])
+    es = [e for _, e in chans]
+    p = {k: inp[k].detach().to("cpu").double().numpy() for k in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")}
+    hist = None if conv_cache_in is None else np.stack(
+        [conv_cache_in[s, :, e].detach().to("cpu").double().numpy() for s, e in chans])
+    h0 = None if ssm_state_in is None else np.stack(
+        [ssm_state_in[s, e, :].detach().to("cpu").double().numpy() for s, e in chans])
+    return oracle.channels(xs, zs, Bn, Cn, dtn, [remap[s] for s, _ in chans], p["conv_w"][es], p["conv_b"][es],
+                           p["w_dt"][es], p["dt_bias"][es], p["A_log"][es], p["D"][es], hist=hist, h0=h0,
+                           lo=dt_min, hi=dt_max, disc=disc, threads=threads)
+
+
+def gather(y, cache, state, chans):
+    """Kernel outputs of the chosen channels as float64 arrays."""
+    ys = np.stack([y[s, :, e].detach().to("cpu").double().numpy() for s, e in chans])
+    cs = np.stack([cache[s, :, e].detach().to("cpu").double().numpy() for s, e in chans])
+    hs = np.stack([state[s, e, :].detach().to("cpu").double().numpy() for s, e in chans])
+    return ys, cs, hs
+
+
+def compare(io_dtype, got, want, label=""):
+    """Assert the parity tolerances: y and state by relative L2, the conv
+    cache bit-exact. Returns the measured errors."""
+    ys, cs, hs = got
+    out_o, h_o, c_o = want
+    e_y = rel_l2(ys, round_io(out_o, io_dtype))
+    e_h = rel_l2(hs, h_o)
+    assert np.array_equal(cs, c_o), f"{label}: conv_cache differs"
+    assert e_y <= TOL[io_dtype], f"{label}: y rel-L2 {e_y:.3e} > {TOL[io_dtype]:.0e}"
+    assert e_h <= TOL[io_dtype], f"{label}: state rel-L2 {e_h:.3e} > {TOL[io_dtype]:.0e}"
+    assert np.isfinite(ys).all() and np.isfinite(hs).all(), f"{label}: non-finite output"
+    return e_y, e_h

@@ -1,0 +1,132 @@
+"""CPU checks of the C ABI: the library builds and loads, exports every
+function include/ssm.h declares, and rejects bad arguments on the host before
+any CUDA call (no kernel runs here)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from selective_state_space_depthwise_b200 import _lib, api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(ssm_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_surface():
+    assert declared_functions() == sorted(_lib.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings_and_version(lib):
+    assert lib.ssm_status_string(0) == b"ok"
+    assert b"invalid" in lib.ssm_status_string(1)
+    assert b"unsupported" in lib.ssm_status_string(2)
+    assert lib.ssm_status_string(99) == b"unknown status"
+    assert re.fullmatch(rb"\d+\.\d+\.\d+", lib.ssm_version())
+
+
+def valid_dims(**kw):
+    d = api.make_dims(2, 64, 32, torch.bfloat16)
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+FAKE = 0x10000  # a 16-byte-aligned non-null address; never dereferenced on the host
+
+
+def fake_weights():
+    w = _lib.SsmWeights()
+    for n in api.PARAM_NAMES:
+        setattr(w, n, FAKE)
+    return w
+
+
+def call_prefill(lib, dims, weights, ptrs=None):
+    p = dict(x=FAKE, z=FAKE, B=FAKE, C=FAKE, dt=FAKE, cin=None, sin=None, y=FAKE + 4096, cout=FAKE, sout=FAKE)
+    p.update(ptrs or {})
+    return lib.ssm_prefill(ctypes.byref(dims) if dims is not None else None,
+                           ctypes.byref(weights) if weights is not None else None, p["x"], p["z"], p["B"], p["C"],
+                           p["dt"], p["cin"], p["sin"], p["y"], p["cout"], p["sout"], None, 0, None)
+
+
+@pytest.mark.parametrize("case,field,value,status", [
+    ("d_state", "d_state", 8, _lib.SSM_ERR_UNSUPPORTED),
+    ("d_conv", "d_conv", 3, _lib.SSM_ERR_UNSUPPORTED),
+    ("batch", "batch", 0, _lib.SSM_ERR_INVALID_ARG),
+    ("seqlen", "seqlen", -1, _lib.SSM_ERR_INVALID_ARG),
+    ("d_inner", "d_inner", 12, _lib.SSM_ERR_INVALID_ARG),
+    ("dt_min", "dt_min", 0.0, _lib.SSM_ERR_INVALID_ARG),
+    ("dt_order", "dt_max", 1e-5, _lib.SSM_ERR_INVALID_ARG),
+    ("io_dtype", "io_dtype", 7, _lib.SSM_ERR_INVALID_ARG),
+    ("disc", "discretization", 5, _lib.SSM_ERR_INVALID_ARG),
+    ("x_tok", "x_tok_stride", 36, _lib.SSM_ERR_INVALID_ARG),
+    ("x_tok_small", "x_tok_stride", 16, _lib.SSM_ERR_INVALID_ARG),
+    ("bc_tok", "bc_tok_stride", 8, _lib.SSM_ERR_INVALID_ARG),
+    ("bc_seq", "bc_seq_stride", 18, _lib.SSM_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_bad_dims(lib, case, field, value, status):
+    assert call_prefill(lib, valid_dims(**{field: value}), fake_weights()) == status
+    assert lib.ssm_last_error() != b""
+
+
+def test_prefill_rejects_bad_pointers(lib):
+    d, w = valid_dims(), fake_weights()
+    assert call_prefill(lib, None, w) == _lib.SSM_ERR_INVALID_ARG
+    assert call_prefill(lib, d, None) == _lib.SSM_ERR_INVALID_ARG
+    for k in ("x", "z", "B", "C", "dt", "y", "cout", "sout"):
+        assert call_prefill(lib, d, w, {k: None}) == _lib.SSM_ERR_INVALID_ARG, k
+        assert b"NULL" in lib.ssm_last_error(), k
+    for k in ("x", "z", "B", "C", "y", "cout"):
+        assert call_prefill(lib, d, w, {k: FAKE + 2}) == _lib.SSM_ERR_INVALID_ARG, k
+    assert call_prefill(lib, d, w, {"y": FAKE}) == _lib.SSM_ERR_INVALID_ARG  # y aliases x
+    w2 = fake_weights()
+    w2.A_log = None
+    assert call_prefill(lib, d, w2) == _lib.SSM_ERR_INVALID_ARG
+    assert b"A_log" in lib.ssm_last_error()
+
+
+def test_decode_rejects_bad_arguments(lib):
+    w = fake_weights()
+    d = valid_dims(d_state=32)
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4096, FAKE, FAKE, None]
+    assert lib.ssm_decode_step(ctypes.byref(d), ctypes.byref(w), *args) == _lib.SSM_ERR_UNSUPPORTED
+    d = valid_dims()
+    bad = list(args)
+    bad[7] = FAKE + 4  # ssm_state must be 16-byte aligned
+    assert lib.ssm_decode_step(ctypes.byref(d), ctypes.byref(w), *bad) == _lib.SSM_ERR_INVALID_ARG
+    bad = list(args)
+    bad[5] = FAKE  # y aliases x
+    assert lib.ssm_decode_step(ctypes.byref(d), ctypes.byref(w), *bad) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_workspace_is_zero_for_the_single_pass_kernel(lib):
+    assert lib.ssm_prefill_workspace_bytes(ctypes.byref(valid_dims())) == 0
+    assert lib.ssm_prefill_workspace_bytes(None) == 0
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    x = torch.zeros(1, 8, 8, dtype=torch.bfloat16)
+    p = {n: torch.zeros(8, 4) if n == "conv_w" else torch.zeros(8, 16) if n == "A_log" else torch.zeros(8)
+         for n in api.PARAM_NAMES}
+    with pytest.raises(RuntimeError, match="no CPU path"):
+        api.prefill(x, x, torch.zeros(1, 8, 16), torch.zeros(1, 8, 16), torch.zeros(1, 8), p)
