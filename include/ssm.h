@@ -91,15 +91,23 @@ typedef struct {
 } ssm_dims;
 
 /* Per-channel parameters, fp32, dense, device pointers (all required).
- * conv_w [E][4], conv_b [E], w_dt [E], dt_bias [E], A_log [E][16], D [E]. */
+ * conv_w [E][4], conv_b [E], w_dt [E], dt_bias [E], A_log [E][16], D [E].
+ * conv_w and A_log must be 16-byte aligned, the others 4-byte aligned. */
 typedef struct {
   const float *conv_w, *conv_b, *w_dt, *dt_bias, *A_log, *D;
 } ssm_weights;
 
-/* Launch shape overrides for tests and tuning; pass NULL for the defaults. */
+/* Launch shape overrides for tests and tuning; pass NULL for the defaults.
+ * kernel 1 (channel tiles): G = threads_per_channel lanes of one warp share a
+ *   channel; channels_per_cta: G=1: 32/64/128, G=2: 16/32/64, G=4 or 8: 8/16/32.
+ * kernel 2 (state slices): a CTA of G warps covers 32 channels and warp j owns
+ *   state slice j of each; threads_per_channel = G in {2, 4, 8}. */
 typedef struct {
-  int32_t threads_per_channel; /* 0 = auto, else 1, 2, 4, 8 or 16 */
-  int32_t channels_per_cta;    /* 0 = auto, else 8, 16, 32 or 64 */
+  int32_t threads_per_channel; /* 0 = auto, else 1, 2, 4 or 8 */
+  int32_t channels_per_cta;    /* 0 = auto (kernel 1 only) */
+  int32_t kernel;              /* 0 = auto, 1 = channel tiles, 2 = state slices */
+  int32_t poly_pairs;          /* -1 = auto; else state pairs per thread and token whose
+                                  exp2 runs as an FMA-pipe polynomial instead of on the SFU */
 } ssm_tuning;
 
 /*

@@ -57,7 +57,8 @@ class SsmWeights(ctypes.Structure):
 
 
 class SsmTuning(ctypes.Structure):
-    _fields_ = [("threads_per_channel", ctypes.c_int32), ("channels_per_cta", ctypes.c_int32)]
+    _fields_ = [("threads_per_channel", ctypes.c_int32), ("channels_per_cta", ctypes.c_int32),
+                ("kernel", ctypes.c_int32), ("poly_pairs", ctypes.c_int32)]
 
 
 class SsmError(RuntimeError):

@@ -113,7 +113,8 @@ def prefill(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None
     work = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
     tun = None
     if tuning:
-        tun = _lib.SsmTuning(int(tuning.get("threads_per_channel", 0)), int(tuning.get("channels_per_cta", 0)))
+        tun = _lib.SsmTuning(int(tuning.get("threads_per_channel", 0)), int(tuning.get("channels_per_cta", 0)),
+                             int(tuning.get("kernel", 0)), int(tuning.get("poly_pairs", -1)))
     st = lib.ssm_prefill_ex(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
                             _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(y), _ptr(conv_cache_out),
                             _ptr(ssm_state_out), _ptr(work), ws, ctypes.byref(tun) if tun else None, _stream(stream))

@@ -5,86 +5,102 @@
 // one output, and exactly one scan step runs from the carried ssm_state; both
 // caches are updated in place.
 //
-// The step is bound by the fp32 state stream (64 B read + 64 B written per
-// channel). Four lanes share a channel and each moves a 16-byte quarter of its
-// state, so a warp covers 8 channels x 64 B = 512 contiguous bytes per access.
-// The per-channel scalar work (conv, SiLU, dt, SiLU(z)) is repeated by the
-// four lanes rather than exchanged: the SM has ample ALU slack at this
-// arithmetic intensity.
+// The step is bound by the fp32 state stream: 64 B read + 64 B written per
+// channel against ~12 B of everything else. One thread owns a channel: it
+// issues its four 16-byte state loads first, so every thread has its whole
+// state in flight while the per-channel work (conv, SiLU, dt, SiLU(z)) runs,
+// then advances the 16 states with packed f32x2 arithmetic and writes them
+// back as four 16-byte stores. Across a warp the state accesses cover 32
+// consecutive channels (2 KB) and x, z, y, the cache rows 64 contiguous bytes.
 #include <cuda_bf16.h>
 
+#include "sm100_ptx.cuh"
 #include "ssm_internal.h"
 #include "ssm_math.cuh"
 
 namespace ssm {
 namespace {
 
-constexpr int kDecodeThreads = 256;
+constexpr int kDecodeThreads = 128;
 
 template <typename T, bool ZOH>
 __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const KernelArgs a) {
-  const int64_t gid = static_cast<int64_t>(blockIdx.x) * kDecodeThreads + threadIdx.x;
-  const int q = static_cast<int>(gid & 3);  // state quarter
-  const int64_t ch = gid >> 2;              // seq * E + e
-  // b*E*4 is a multiple of 32 (E % 8 == 0), so whole warps leave together.
+  const int64_t ch = static_cast<int64_t>(blockIdx.x) * kDecodeThreads + threadIdx.x;  // seq * E + e
   if (ch >= a.batch * a.E) return;
   const int64_t seq = ch / a.E;
   const int64_t e = ch - seq * a.E;
 
+  float4* hp = reinterpret_cast<float4*>(a.ssm_state_out + ch * 16);
+  float4 hv[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) hv[q] = hp[q];
+
   T* cache = static_cast<T*>(a.conv_cache_out);  // in-out
-  const T* x = static_cast<const T*>(a.x);
-  const T* z = static_cast<const T*>(a.z);
   const T c0 = cache[(seq * 3 + 0) * a.E + e];
   const T c1 = cache[(seq * 3 + 1) * a.E + e];
   const T c2 = cache[(seq * 3 + 2) * a.E + e];
-  const T xt = x[seq * a.s.x_seq + e];
-  const float zt = IO<T>::to_f(z[seq * a.s.z_seq + e]);
+  const T xt = static_cast<const T*>(a.x)[seq * a.s.x_seq + e];
+  const float zt = IO<T>::to_f(static_cast<const T*>(a.z)[seq * a.s.z_seq + e]);
+  const float4 cw = *reinterpret_cast<const float4*>(a.conv_w + e * 4);
+  const float4* Al = reinterpret_cast<const float4*>(a.A_log + e * 16);
+  const float4* Bq = reinterpret_cast<const float4*>(a.B + seq * a.s.bc_seq);
+  const float4* Cq = reinterpret_cast<const float4*>(a.C + seq * a.s.bc_seq);
 
-  const float conv = fmaf(a.conv_w[e * 4 + 3], IO<T>::to_f(xt),
-                          fmaf(a.conv_w[e * 4 + 2], IO<T>::to_f(c2),
-                               fmaf(a.conv_w[e * 4 + 1], IO<T>::to_f(c1),
-                                    fmaf(a.conv_w[e * 4 + 0], IO<T>::to_f(c0), a.conv_b[e]))));
+  const float conv = fmaf(cw.w, IO<T>::to_f(xt),
+                          fmaf(cw.z, IO<T>::to_f(c2), fmaf(cw.y, IO<T>::to_f(c1), fmaf(cw.x, IO<T>::to_f(c0), a.conv_b[e]))));
   const float u = silu(conv);
   const float dt = dt_of(fmaf(a.dt_raw[seq * a.s.dt_seq], a.w_dt[e], a.dt_bias[e]), a.dt_min, a.dt_max);
   const float zg = silu(zt);
 
-  float4* hp = reinterpret_cast<float4*>(a.ssm_state_out + ch * 16 + 4 * q);
-  float4 hv = *hp;
-  const float4 Bv = *reinterpret_cast<const float4*>(a.B + seq * a.s.bc_seq + 4 * q);
-  const float4 Cv = *reinterpret_cast<const float4*>(a.C + seq * a.s.bc_seq + 4 * q);
-  float h[4] = {hv.x, hv.y, hv.z, hv.w};
-  const float bb[4] = {Bv.x, Bv.y, Bv.z, Bv.w};
-  const float cc[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
-  float yp = 0.0f;
+  float yl = 0.0f, yh = 0.0f;
+  if constexpr (ZOH) {
 #pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const float A = -expf(a.A_log[e * 16 + 4 * q + s]);
-    float dA, coef;
-    if constexpr (ZOH) {
-      const float xa = dt * A;
-      dA = ex2_approx(xa * kLog2e);
-      coef = expm1_nonpos(xa, dA) / A * u;
-    } else {
-      dA = ex2_approx(dt * (A * kLog2e));
-      coef = dt * u;
+    for (int q = 0; q < 4; ++q) {
+      const float4 al = Al[q], b = Bq[q], cc = Cq[q];
+      const float alv[4] = {al.x, al.y, al.z, al.w}, bv[4] = {b.x, b.y, b.z, b.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
+      float hs[4] = {hv[q].x, hv[q].y, hv[q].z, hv[q].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float A = -expf(alv[i]);
+        const float xa = dt * A;
+        const float dA = ex2_approx(xa * kLog2e);
+        hs[i] = fmaf(dA, hs[i], expm1_nonpos(xa, dA) / A * u * bv[i]);
+        yl = fmaf(cv[i], hs[i], yl);
+      }
+      hv[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
     }
-    h[s] = fmaf(dA, h[s], coef * bb[s]);
-    yp = fmaf(cc[s], h[s], yp);
+  } else {
+    const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
+    uint64_t acc = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 al = Al[q], b = Bq[q], cc = Cq[q];
+      // a2 = A * log2(e) = -exp(A_log) * log2(e)
+      const float a0 = -expf(al.x) * kLog2e, a1 = -expf(al.y) * kLog2e;
+      const float a2v = -expf(al.z) * kLog2e, a3 = -expf(al.w) * kLog2e;
+      float x0, x1, x2, x3;
+      upk2(fmul2(dt2, pk2(a0, a1)), x0, x1);
+      upk2(fmul2(dt2, pk2(a2v, a3)), x2, x3);
+      const uint64_t h01 = ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(hv[q].x, hv[q].y), fmul2(dtu2, pk2(b.x, b.y)));
+      const uint64_t h23 = ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(hv[q].z, hv[q].w), fmul2(dtu2, pk2(b.z, b.w)));
+      acc = q == 0 ? fmul2(pk2(cc.x, cc.y), h01) : ffma2(pk2(cc.x, cc.y), h01, acc);
+      acc = ffma2(pk2(cc.z, cc.w), h23, acc);
+      upk2(h01, hv[q].x, hv[q].y);
+      upk2(h23, hv[q].z, hv[q].w);
+    }
+    upk2(acc, yl, yh);
   }
-  yp += __shfl_xor_sync(0xffffffffu, yp, 1);
-  yp += __shfl_xor_sync(0xffffffffu, yp, 2);
-  *hp = make_float4(h[0], h[1], h[2], h[3]);
-  __syncwarp();  // every lane of the channel has read the old cache rows
-  if (q == 0) static_cast<T*>(a.y)[seq * a.s.y_seq + e] = IO<T>::from_f((yp + a.D[e] * u) * zg);
-  if (q == 1) cache[(seq * 3 + 0) * a.E + e] = c1;
-  if (q == 2) cache[(seq * 3 + 1) * a.E + e] = c2;
-  if (q == 3) cache[(seq * 3 + 2) * a.E + e] = xt;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) hp[q] = hv[q];
+  static_cast<T*>(a.y)[seq * a.s.y_seq + e] = IO<T>::from_f((yl + yh + a.D[e] * u) * zg);
+  cache[(seq * 3 + 0) * a.E + e] = c1;
+  cache[(seq * 3 + 1) * a.E + e] = c2;
+  cache[(seq * 3 + 2) * a.E + e] = xt;
 }
 
 template <typename T, bool ZOH>
 cudaError_t launch(const KernelArgs& a, cudaStream_t st) {
-  const int64_t threads = a.batch * a.E * 4;
-  const int64_t blocks = (threads + kDecodeThreads - 1) / kDecodeThreads;
+  const int64_t blocks = (a.batch * a.E + kDecodeThreads - 1) / kDecodeThreads;
   if (blocks > 0x7fffffff) return cudaErrorInvalidConfiguration;
   decode_kernel<T, ZOH><<<static_cast<unsigned>(blocks), kDecodeThreads, 0, st>>>(a);
   return cudaGetLastError();

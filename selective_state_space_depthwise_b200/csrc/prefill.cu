@@ -6,179 +6,180 @@
 // clip(softplus(dt_raw*w_dt + dt_bias)), dA = exp(dt*A) with A = -exp(A_log),
 // the scan h = dA*h + dt*B*u (the _ssm_fma leaf of "JIT-compiled kernels"),
 // y = C.h + D*u and the gate y*SiLU(z). dA, dB and h never reach HBM: the 16
-// states of a channel stay in registers for the whole walk over L.
+// states of a channel live in registers for the whole walk over L.
 //
-// Work split. G threads share a channel and hold 16/G states each. Tokens are
-// processed in rounds of G: in a round, thread j does the per-token work (conv,
-// SiLU, dt, SiLU(z)) of token j, the group exchanges dt and dt*u by shuffles,
-// every thread advances its states through the G tokens in order, and the
-// partial readouts are reduce-scattered so that thread j ends with the full
-// C.h of token j. G > 1 gives more warps when b*E is small (b = 1 shapes)
-// without splitting L.
+// Pipeline. L is walked in stages of kTok tokens through a kStages-deep ring
+// in shared memory filled by TMA tile loads: the x tile carries a 3-row halo
+// for the conv (rows before token 0 come back zero-filled and are replaced by
+// conv_cache_in when one is given), B and C (shared by all channels) come as
+// [token][16] tiles, and warp 0 stages dt_raw one stage ahead. Thread 0
+// re-arms a slot right after the CTA has finished with it; every wait on the
+// ring's mbarriers is bounded.
 //
-// Data movement. L is walked in stages of kTok tokens through a kStages-deep
-// ring in shared memory filled by cp.async: the x tile carries a 3-row halo
-// (the conv history; zeros or conv_cache_in before token 0), B and C (shared by
-// all channels) and dt_raw are staged once per CTA. Output tiles go through
-// shared memory and leave as 16-byte stores. Tokens past L are zero-filled and
-// given dt = 0, which leaves the states unchanged.
+// Work split. G threads share a channel and hold 16/G states each (G is
+// chosen from b*E so that small batches still fill the GPU without splitting
+// L). With G == 1 one thread does everything for its channel token by token.
+// With G > 1 each stage runs three phases:
+//  A. per-token work for a contiguous run of kTok/G tokens of the thread's
+//     channel (conv with a sliding window of x, SiLU, dt), written to shared
+//     memory as (dt, dt, dt*u, dt*u); D*u and SiLU(z) stay in registers;
+//  B. every thread advances its states through all kTok tokens (packed f32x2
+//     multiplies/FMAs, SFU exp2 for the decays) and writes the partial
+//     readout C.h of each token -- a stream whose only carried dependency is
+//     the state;
+//  C. each thread sums the G partials of its phase-A tokens, applies the D
+//     skip and the gate, and fills an output tile that leaves by TMA store.
+#include <cuda.h>
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
+#include "sm100_ptx.cuh"
 #include "ssm_internal.h"
 #include "ssm_math.cuh"
 
 namespace ssm {
 namespace {
 
-constexpr int kTok = 64;    // tokens per pipeline stage
+constexpr int kTok = 32;    // tokens per pipeline stage (= lanes of the dt_raw stager)
 constexpr int kStages = 3;  // ring depth
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
+struct Maps {
+  CUtensorMap x, z, B, C, y;
+};
 
-// 16-byte async copy global -> shared; src_bytes < 16 zero-fills the rest.
-__device__ __forceinline__ void cp_async_16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
+constexpr int align128(int v) { return (v + 127) / 128 * 128; }
 
-__device__ __forceinline__ void cp_async_4(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-
-// Shared-memory layout of one pipeline stage (byte offsets, all 16-aligned).
-template <typename T, int NCH>
-struct Stage {
-  static constexpr int kXRows = kTok + 3;
-  static constexpr int kRow = NCH * static_cast<int>(sizeof(T));  // bytes per token row
-  static_assert(kRow % 16 == 0, "a channel tile row must be a whole number of 16-byte chunks");
+// Shared-memory layout (byte offsets from a 128-aligned base).
+template <typename T, int NCH, int G>
+struct Smem {
+  static constexpr int kEs = static_cast<int>(sizeof(T));
+  static constexpr int kXBytes = (kTok + 3) * NCH * kEs;  // TMA box {NCH, kTok + 3}
+  static constexpr int kZBytes = kTok * NCH * kEs;        // TMA box {NCH, kTok}
+  static constexpr int kBCBytes = kTok * 16 * 4;          // TMA box {16, kTok}
   static constexpr int kX = 0;
-  static constexpr int kZ = kX + kXRows * kRow;
-  static constexpr int kB = kZ + kTok * kRow;
-  static constexpr int kC = kB + kTok * 16 * 4;
-  static constexpr int kD = kC + kTok * 16 * 4;
-  static constexpr int kBytes = kD + kTok * 4;
-  static constexpr int kYBytes = kTok * kRow;
-  static constexpr int kTotal = kStages * kBytes + kYBytes;
+  static constexpr int kZ = align128(kX + kXBytes);
+  static constexpr int kB = align128(kZ + kZBytes);
+  static constexpr int kC = kB + kBCBytes;
+  static constexpr int kSlot = kC + kBCBytes;
+  // Phase-A outputs (G > 1): a row per channel, one pad entry after every
+  // thread's run of kTok/G tokens so that the runs of a warp hit distinct banks.
+  static constexpr int kRow = kTok + G;
+  // Partial readouts (G > 1): [channel][state slice][token], rows padded by 4
+  // floats and channels by a further 4 x G floats for bank spread.
+  static constexpr int kPRow = kTok + 4;
+  static constexpr int kPCh = G * kPRow + 4 * G;
+  static constexpr int kDT = kStages * kSlot;                           // float4 (dt, dt, dt*u, dt*u)
+  static constexpr int kP = kDT + (G > 1 ? NCH * kRow * 16 : 0);       // float partials
+  static constexpr int kDr = kP + (G > 1 ? NCH * kPCh * 4 : 0);        // dt_raw, 2 stages
+  static constexpr int kY = align128(kDr + 2 * kTok * 4);              // output tiles (G > 1)
+  static constexpr int kYBytes = G > 1 ? align128(kTok * NCH * kEs) : 0;
+  static constexpr int kBar = kY + 2 * kYBytes;
+  static constexpr int kTotal = kBar + kStages * 8;
+  static constexpr uint32_t kTxBytes = static_cast<uint32_t>(kXBytes + kZBytes + 2 * kBCBytes);
+  static_assert((NCH * kEs) % 16 == 0, "TMA rows must be whole 16-byte chunks");
 };
 
-// Issue the cp.async copies of stage [t0, t0 + kTok) of sequence `seq`,
-// channels [e0, e0 + NCH).
-template <typename T, int NCH, int NT>
-__device__ __forceinline__ void load_stage(unsigned char* st, const KernelArgs& a, int64_t seq, int64_t e0,
-                                           int64_t t0, int tid) {
-  using S = Stage<T, NCH>;
-  constexpr int EPC = 16 / static_cast<int>(sizeof(T));  // elements per 16-byte chunk
-  constexpr int CPR = NCH / EPC;                          // chunks per token row
-  const T* x = static_cast<const T*>(a.x);
-  const T* z = static_cast<const T*>(a.z);
-  const T* hist = static_cast<const T*>(a.conv_cache_in);
-  for (int i = tid; i < S::kXRows * CPR; i += NT) {
-    const int r = i / CPR, q = i % CPR;
-    const int64_t t = t0 - 3 + r;
-    const int64_t e = e0 + q * EPC;
-    const void* src = a.x;
-    int bytes = 0;
-    if (e < a.E) {
-      if (t >= 0 && t < a.L) {
-        src = x + seq * a.s.x_seq + t * a.s.x_tok + e;
-        bytes = 16;
-      } else if (t < 0 && hist != nullptr) {
-        src = hist + (seq * 3 + (3 + t)) * a.E + e;
-        bytes = 16;
-      }
+// Advance KP packed state pairs through one token; returns C.h over the pairs.
+// dt2 = {dt, dt}, inj2 = {dt*u, dt*u}; B, C point at this thread's states.
+template <int KP, int NPOLY = 0>
+__device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const float* a2, float* h, const float* Bp,
+                                            const float* Cp) {
+  uint64_t acc = 0;
+#pragma unroll
+  for (int q = 0; q < KP; ++q) {
+    float b0, b1, c0, c1;
+    if constexpr (KP >= 2) {
+      const float4 bq = *reinterpret_cast<const float4*>(Bp + 4 * (q / 2));
+      const float4 cq = *reinterpret_cast<const float4*>(Cp + 4 * (q / 2));
+      b0 = (q & 1) ? bq.z : bq.x, b1 = (q & 1) ? bq.w : bq.y;
+      c0 = (q & 1) ? cq.z : cq.x, c1 = (q & 1) ? cq.w : cq.y;
+    } else {
+      const float2 bq = *reinterpret_cast<const float2*>(Bp);
+      const float2 cq = *reinterpret_cast<const float2*>(Cp);
+      b0 = bq.x, b1 = bq.y, c0 = cq.x, c1 = cq.y;
     }
-    cp_async_16(st + S::kX + r * S::kRow + q * 16, src, bytes);
+    float x0, x1;
+    upk2(fmul2(dt2, pk2(a2[2 * q], a2[2 * q + 1])), x0, x1);
+    // the last NPOLY pairs take the FMA-pipe exp2, the others the SFU
+    const uint64_t dA = q >= KP - NPOLY ? ex2_poly2(x0, x1) : pk2(ex2_approx(x0), ex2_approx(x1));
+    const uint64_t hb = ffma2(dA, pk2(h[2 * q], h[2 * q + 1]), fmul2(inj2, pk2(b0, b1)));
+    upk2(hb, h[2 * q], h[2 * q + 1]);
+    acc = q == 0 ? fmul2(pk2(c0, c1), hb) : ffma2(pk2(c0, c1), hb, acc);
   }
-  for (int i = tid; i < kTok * CPR; i += NT) {
-    const int r = i / CPR, q = i % CPR;
-    const int64_t t = t0 + r;
-    const int64_t e = e0 + q * EPC;
-    const bool ok = t < a.L && e < a.E;
-    cp_async_16(st + S::kZ + r * S::kRow + q * 16, ok ? z + seq * a.s.z_seq + t * a.s.z_tok + e : a.z, ok ? 16 : 0);
-  }
-  for (int i = tid; i < kTok * 4; i += NT) {
-    const int r = i >> 2, q = i & 3;
-    const int64_t t = t0 + r;
-    const bool ok = t < a.L;
-    const int64_t off = seq * a.s.bc_seq + t * a.s.bc_tok + 4 * q;
-    cp_async_16(st + S::kB + (r * 16 + 4 * q) * 4, ok ? a.B + off : a.B, ok ? 16 : 0);
-    cp_async_16(st + S::kC + (r * 16 + 4 * q) * 4, ok ? a.C + off : a.C, ok ? 16 : 0);
-  }
-  for (int i = tid; i < kTok; i += NT) {
-    const int64_t t = t0 + i;
-    const bool ok = t < a.L;
-    cp_async_4(st + S::kD + 4 * i, ok ? a.dt_raw + seq * a.s.dt_seq + t : a.dt_raw, ok ? 4 : 0);
-  }
+  float lo, hi;
+  upk2(acc, lo, hi);
+  return lo + hi;
 }
 
-// Reduce-scatter over the G lanes of a group: on entry v[i] is this lane's
-// partial for token i; on exit v[0] of lane j holds the group sum for token j.
-template <int G, int H>
-struct ReduceScatter {
-  static __device__ __forceinline__ void run(float* v, int j) {
-    const bool up = (j & H) != 0;
-#pragma unroll
-    for (int i = 0; i < H; ++i) {
-      const float send = up ? v[i] : v[i + H];
-      const float keep = up ? v[i + H] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, H);
-    }
-    ReduceScatter<G, H / 2>::run(v, j);
-  }
-};
-
-template <int G>
-struct ReduceScatter<G, 0> {
-  static __device__ __forceinline__ void run(float*, int) {}
-};
-
+// Zero-order-hold variant (scalar): h = e^{dt A} h + (e^{dt A} - 1)/A * u * B.
 template <int K>
-__device__ __forceinline__ void load_k(const float* p, float (&v)[K]) {
-  if constexpr (K % 4 == 0) {
+__device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* Av, float* h, const float* Bp,
+                                                const float* Cp) {
+  float acc = 0.0f;
 #pragma unroll
-    for (int s = 0; s < K; s += 4) {
-      const float4 q = *reinterpret_cast<const float4*>(p + s);
-      v[s] = q.x;
-      v[s + 1] = q.y;
-      v[s + 2] = q.z;
-      v[s + 3] = q.w;
-    }
-  } else if constexpr (K == 2) {
-    const float2 q = *reinterpret_cast<const float2*>(p);
-    v[0] = q.x;
-    v[1] = q.y;
-  } else {
-    v[0] = *p;
+  for (int q = 0; q < K; ++q) {
+    const float xa = dt * Av[q];
+    const float dA = ex2_approx(xa * kLog2e);
+    h[q] = fmaf(dA, h[q], expm1_nonpos(xa, dA) / Av[q] * u * Bp[q]);
+    acc = fmaf(Cp[q], h[q], acc);
   }
+  return acc;
 }
 
-template <typename T, int G, int NCH, bool ZOH>
-__global__ void __launch_bounds__(NCH* G) prefill_kernel(const KernelArgs a) {
-  constexpr int NT = NCH * G;
-  constexpr int K = 16 / G;  // states per thread
-  using S = Stage<T, NCH>;
-  constexpr int EPC = 16 / static_cast<int>(sizeof(T));
-  constexpr int CPR = NCH / EPC;
-  extern __shared__ __align__(128) unsigned char smem[];
-  T* ys = reinterpret_cast<T*>(smem + kStages * S::kBytes);
+template <typename T, int G, int NCH, bool ZOH, int NPOLY>
+__global__ void __launch_bounds__(NCH* G) prefill_kernel(const __grid_constant__ Maps maps, const KernelArgs a) {
+  constexpr int NT = NCH * G;  // threads
+  constexpr int K = 16 / G;    // states per thread
+  constexpr int KP = K / 2;    // packed state pairs
+  constexpr int TA = kTok / G;  // phase-A tokens per thread (G > 1)
+  using S = Smem<T, NCH, G>;
+  static_assert(kTok % G == 0 && NT % 32 == 0 && K >= 2, "bad shape");
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t full0 = sb + S::kBar;
+  float* Dr = reinterpret_cast<float*>(smem + S::kDr);  // [2][kTok]
 
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int64_t tiles = (a.E + NCH - 1) / NCH;
+  const int seq = static_cast<int>(blockIdx.x / tiles);
+  const int e0 = static_cast<int>(blockIdx.x % tiles) * NCH;
+  const int64_t L = a.L;
+  const int64_t n_stages = (L + kTok - 1) / kTok;
+  const float* dtr = a.dt_raw + static_cast<int64_t>(seq) * a.s.dt_seq;
+
+  auto issue_stage = [&](int64_t st_idx) {  // thread 0 only
+    const int slot = static_cast<int>(st_idx % kStages);
+    const uint32_t base = sb + slot * S::kSlot, bar = full0 + 8 * slot;
+    const int t0 = static_cast<int>(st_idx * kTok);
+    mbar_arrive_expect_tx(bar, S::kTxBytes);
+    tma_load_3d(base + S::kX, &maps.x, e0, t0 - 3, seq, bar);
+    tma_load_3d(base + S::kZ, &maps.z, e0, t0, seq, bar);
+    tma_load_3d(base + S::kB, &maps.B, 0, t0, seq, bar);
+    tma_load_3d(base + S::kC, &maps.C, 0, t0, seq, bar);
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(full0 + 8 * i, 1);
+    mbar_fence_init();
+    prefetch_tensormap(&maps.x);
+    prefetch_tensormap(&maps.z);
+    prefetch_tensormap(&maps.B);
+    prefetch_tensormap(&maps.C);
+    for (int64_t i = 0; i < kStages && i < n_stages; ++i) issue_stage(i);
+  }
+  float d_next = 0.0f;  // warp 0 stages dt_raw one stage ahead
+  if (tid < 32) {
+    Dr[lane] = lane < L ? dtr[lane] : 0.0f;
+    d_next = kTok + lane < L ? dtr[kTok + lane] : 0.0f;
+  }
+  __syncthreads();
+
   const int c = tid / G;  // channel within the tile
   const int j = tid % G;  // state slice; also the token this lane owns in a round
-  const int64_t tiles_per_seq = (a.E + NCH - 1) / NCH;
-  const int64_t seq = blockIdx.x / tiles_per_seq;
-  const int64_t e0 = (blockIdx.x % tiles_per_seq) * NCH;
-  const int64_t e = e0 + c;
+  const int e = e0 + c;
   const bool ch_ok = e < a.E;
   const int64_t ec = ch_ok ? e : a.E - 1;  // clamped index for parameter loads
 
@@ -186,107 +187,183 @@ __global__ void __launch_bounds__(NCH* G) prefill_kernel(const KernelArgs a) {
   const float cw2 = a.conv_w[ec * 4 + 2], cw3 = a.conv_w[ec * 4 + 3];
   const float cb = a.conv_b[ec], wdt = a.w_dt[ec], dtb = a.dt_bias[ec], Dd = a.D[ec];
   const float lo = a.dt_min, hi = a.dt_max;
-  float a2[K];  // A_n * log2(e), so that exp(dt*A_n) = 2^(dt*a2_n)
+  float hx0 = 0.0f, hx1 = 0.0f, hx2 = 0.0f;  // conv history before token 0
+  if (a.conv_cache_in) {
+    const T* hist = static_cast<const T*>(a.conv_cache_in) + static_cast<int64_t>(seq) * 3 * a.E + ec;
+    hx0 = IO<T>::to_f(hist[0]);
+    hx1 = IO<T>::to_f(hist[a.E]);
+    hx2 = IO<T>::to_f(hist[2 * a.E]);
+  }
+  float a2[K];  // A_n * log2(e): exp(dt*A_n) = 2^(dt*a2_n)
   float Av[K];  // A_n (ZOH only)
   float h[K];
 #pragma unroll
-  for (int s = 0; s < K; ++s) {
-    const float A = -expf(a.A_log[ec * 16 + j * K + s]);
-    Av[s] = A;
-    a2[s] = A * kLog2e;
-    h[s] = a.ssm_state_in ? a.ssm_state_in[(seq * a.E + ec) * 16 + j * K + s] : 0.0f;
+  for (int q = 0; q < K; ++q) {
+    const float A = -expf(a.A_log[ec * 16 + j * K + q]);
+    Av[q] = A;
+    a2[q] = A * kLog2e;
+    h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + j * K + q] : 0.0f;
   }
   (void)Av;
 
-  const int64_t L = a.L;
-  const int64_t n_stages = (L + kTok - 1) / kTok;
-#pragma unroll
-  for (int s = 0; s < kStages - 1; ++s) {
-    if (s < n_stages) load_stage<T, NCH, NT>(smem + s * S::kBytes, a, seq, e0, static_cast<int64_t>(s) * kTok, tid);
-    cp_async_commit();
-  }
+  for (int64_t s = 0; s < n_stages; ++s) {
+    const int slot = static_cast<int>(s % kStages);
+    const unsigned char* st = smem + slot * S::kSlot;
+    mbar_wait_bounded(full0 + 8 * slot, static_cast<uint32_t>((s / kStages) & 1), a.err, 1);
+    const T* X = reinterpret_cast<const T*>(st + S::kX);
+    const T* Z = reinterpret_cast<const T*>(st + S::kZ);
+    const float* Bt = reinterpret_cast<const float*>(st + S::kB);
+    const float* Ct = reinterpret_cast<const float*>(st + S::kC);
+    const float* D_ = Dr + (s & 1) * kTok;
+    const int64_t t0 = s * kTok;
+    const bool first = s == 0;
+    // Tile row r of x holds token t0 + r - 3.
+    auto xrow = [&](int r) {
+      if (first && r < 3) return r == 0 ? hx0 : (r == 1 ? hx1 : hx2);
+      return IO<T>::to_f(X[r * NCH + c]);
+    };
 
-  for (int64_t it = 0; it < n_stages; ++it) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();  // stage `it` landed for everyone; previous output tile drained
-    {
-      const int64_t nx = it + kStages - 1;
-      if (nx < n_stages) load_stage<T, NCH, NT>(smem + (nx % kStages) * S::kBytes, a, seq, e0, nx * kTok, tid);
-      cp_async_commit();
-    }
-    const unsigned char* st = smem + (it % kStages) * S::kBytes;
-    const T* xs = reinterpret_cast<const T*>(st + S::kX);
-    const T* zs = reinterpret_cast<const T*>(st + S::kZ);
-    const float* Bs = reinterpret_cast<const float*>(st + S::kB);
-    const float* Cs = reinterpret_cast<const float*>(st + S::kC);
-    const float* Ds = reinterpret_cast<const float*>(st + S::kD);
-    const int64_t t0 = it * kTok;
-
+    if constexpr (G == 1) {
+      // One thread owns every token of its channel: per-token work and the
+      // scan fuse; y goes straight to global memory (a warp writes 32
+      // consecutive channels of a token).
+      T* yrow = static_cast<T*>(a.y) + static_cast<int64_t>(seq) * a.s.y_seq + e;
+      float w0 = xrow(0), w1 = xrow(1), w2 = xrow(2);
+      constexpr int kChunk = 8;  // tokens computed before their outputs are stored
 #pragma unroll 1
-    for (int r = 0; r < kTok; r += G) {
-      // Per-token work for the token this lane owns (row tl of the stage).
-      const int tl = r + j;
-      const float x0 = IO<T>::to_f(xs[(tl + 0) * NCH + c]);
-      const float x1 = IO<T>::to_f(xs[(tl + 1) * NCH + c]);
-      const float x2 = IO<T>::to_f(xs[(tl + 2) * NCH + c]);
-      const float x3 = IO<T>::to_f(xs[(tl + 3) * NCH + c]);
-      const float conv = fmaf(cw3, x3, fmaf(cw2, x2, fmaf(cw1, x1, fmaf(cw0, x0, cb))));
-      const float u = silu(conv);
-      float dt = dt_of(fmaf(Ds[tl], wdt, dtb), lo, hi);
-      if (t0 + tl >= L) dt = 0.0f;  // past the end: keep the state
-      const float inj = ZOH ? u : dt * u;
-      const float zg = silu(IO<T>::to_f(zs[tl * NCH + c]));
-
-      float dtv[G], injv[G], yp[G];
+      for (int tc = 0; tc < kTok; tc += kChunk) {
+        float yv[kChunk];
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        dtv[i] = __shfl_sync(0xffffffffu, dt, i, G);
-        injv[i] = __shfl_sync(0xffffffffu, inj, i, G);
-      }
-#pragma unroll
-      for (int i = 0; i < G; ++i) {
-        float bv[K], cv[K];
-        load_k<K>(Bs + (r + i) * 16 + j * K, bv);
-        load_k<K>(Cs + (r + i) * 16 + j * K, cv);
-        float acc = 0.0f;
-#pragma unroll
-        for (int s = 0; s < K; ++s) {
-          float dA, coef;
-          if constexpr (ZOH) {
-            const float xa = dtv[i] * Av[s];
-            dA = ex2_approx(xa * kLog2e);
-            coef = expm1_nonpos(xa, dA) / Av[s] * injv[i];  // (e^{dt A} - 1)/A * u
-          } else {
-            dA = ex2_approx(dtv[i] * a2[s]);
-            coef = injv[i];  // dt * u
-          }
-          h[s] = fmaf(dA, h[s], coef * bv[s]);
-          acc = fmaf(cv[s], h[s], acc);
+        for (int k = 0; k < kChunk; ++k) {
+          const int tl = tc + k;
+          const float w3 = xrow(tl + 3);
+          const float conv = fmaf(cw3, w3, fmaf(cw2, w2, fmaf(cw1, w1, fmaf(cw0, w0, cb))));
+          w0 = w1;
+          w1 = w2;
+          w2 = w3;
+          const float u = silu(conv);
+          float dt = dt_of(fmaf(D_[tl], wdt, dtb), lo, hi);
+          if (t0 + tl >= L) dt = 0.0f;  // past the end: keep the state
+          const float zg = silu(IO<T>::to_f(Z[tl * NCH + c]));
+          float yc;
+          if constexpr (ZOH)
+            yc = scan_token_zoh<K>(dt, u, Av, h, Bt + tl * 16, Ct + tl * 16);
+          else
+            yc = scan_token<KP, NPOLY>(pk2(dt, dt), pk2(dt * u, dt * u), a2, h, Bt + tl * 16, Ct + tl * 16);
+          yv[k] = (yc + Dd * u) * zg;
         }
-        yp[i] = acc;
+        if (ch_ok) {
+#pragma unroll
+          for (int k = 0; k < kChunk; ++k)
+            if (t0 + tc + k < L) yrow[(t0 + tc + k) * a.s.y_tok] = IO<T>::from_f(yv[k]);
+        }
       }
-      ReduceScatter<G, G / 2>::run(yp, j);
-      ys[tl * NCH + c] = IO<T>::from_f((yp[0] + Dd * u) * zg);
+    } else {
+      float4* DT = reinterpret_cast<float4*>(smem + S::kDT) + c * S::kRow;
+      float* P = reinterpret_cast<float*>(smem + S::kP) + c * S::kPCh;
+      auto pos = [](int tl) { return tl + tl / TA; };
+      // Phase A: tokens [j*TA, (j+1)*TA) of channel c. All inputs are read
+      // first and the (dt, dt, dt*u, dt*u) rows written last; D*u and SiLU(z)
+      // stay in registers for phase C.
+      float du[TA], zg[TA];
+      {
+        const int tb = j * TA;
+        float xw[TA + 3], zr[TA], dr[TA];
+#pragma unroll
+        for (int i = 0; i < TA + 3; ++i) xw[i] = xrow(tb + i);
+#pragma unroll
+        for (int i = 0; i < TA; ++i) {
+          zr[i] = IO<T>::to_f(Z[(tb + i) * NCH + c]);
+          dr[i] = D_[tb + i];
+        }
+        float4 dtv[TA];
+#pragma unroll
+        for (int i = 0; i < TA; ++i) {
+          const float conv = fmaf(cw3, xw[i + 3], fmaf(cw2, xw[i + 2], fmaf(cw1, xw[i + 1], fmaf(cw0, xw[i], cb))));
+          const float u = silu(conv);
+          float dt = dt_of(fmaf(dr[i], wdt, dtb), lo, hi);
+          if (t0 + tb + i >= L) dt = 0.0f;  // past the end: keep the state
+          const float inj = ZOH ? u : dt * u;
+          dtv[i] = make_float4(dt, dt, inj, inj);
+          du[i] = Dd * u;
+          zg[i] = silu(zr[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < TA; ++i) DT[pos(tb + i)] = dtv[i];
+      }
+      if (tid == 0) bulk_wait_read<1>();  // output tile (s & 1) no longer read by the store of stage s - 2
+      named_bar_sync(1, NT);
+
+      // Phase B: this thread's K states through all kTok tokens of the stage.
+      // Partial readouts C.h stay in registers until the stream is done.
+      float pr[kTok];
+#pragma unroll
+      for (int tl = 0; tl < kTok; ++tl) {
+        const float4 dd = DT[pos(tl)];
+        const float* Bp = Bt + tl * 16 + j * K;
+        const float* Cp = Ct + tl * 16 + j * K;
+        if constexpr (ZOH)
+          pr[tl] = scan_token_zoh<K>(dd.x, dd.z, Av, h, Bp, Cp);
+        else
+          pr[tl] = scan_token<KP>(pk2(dd.x, dd.y), pk2(dd.z, dd.w), a2, h, Bp, Cp);
+      }
+      {
+        float* Pj = P + j * S::kPRow;
+#pragma unroll
+        for (int tl = 0; tl < kTok; tl += 4)
+          *reinterpret_cast<float4*>(Pj + tl) = make_float4(pr[tl], pr[tl + 1], pr[tl + 2], pr[tl + 3]);
+      }
+      __syncwarp();  // the G slices of a channel live in one warp
+
+      // Phase C: sum the G partials of this thread's phase-A tokens, gate, write the tile.
+      {
+        const int tb = j * TA;
+        float ys[TA];
+#pragma unroll
+        for (int q = 0; q < TA; q += 4) {
+          float4 acc = *reinterpret_cast<const float4*>(P + tb + q);
+#pragma unroll
+          for (int jj = 1; jj < G; ++jj) {
+            const float4 v = *reinterpret_cast<const float4*>(P + jj * S::kPRow + tb + q);
+            acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+          }
+          ys[q + 0] = (acc.x + du[q + 0]) * zg[q + 0];
+          ys[q + 1] = (acc.y + du[q + 1]) * zg[q + 1];
+          ys[q + 2] = (acc.z + du[q + 2]) * zg[q + 2];
+          ys[q + 3] = (acc.w + du[q + 3]) * zg[q + 3];
+        }
+        T* Y = reinterpret_cast<T*>(smem + S::kY + (s & 1) * S::kYBytes);
+#pragma unroll
+        for (int i = 0; i < TA; ++i) Y[(tb + i) * NCH + c] = IO<T>::from_f(ys[i]);
+      }
+      fence_proxy_async_smem();
     }
-    __syncthreads();  // output tile complete
-    for (int i = tid; i < kTok * CPR; i += NT) {
-      const int rr = i / CPR, q = i % CPR;
-      const int64_t t = t0 + rr;
-      const int64_t eo = e0 + q * EPC;
-      if (t < L && eo < a.E) {
-        T* dst = static_cast<T*>(a.y) + seq * a.s.y_seq + t * a.s.y_tok + eo;
-        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ys + rr * NCH + q * EPC);
+
+    // End of stage: stage dt_raw two ahead, then release the ring slot.
+    if (tid < 32) {
+      Dr[((s + 1) & 1) * kTok + lane] = d_next;
+      const int64_t tn = t0 + 2 * kTok + lane;
+      d_next = tn < L ? dtr[tn] : 0.0f;
+    }
+    named_bar_sync(1, NT);
+    if (tid == 0) {
+      if constexpr (G > 1) {
+        tma_store_3d(&maps.y, sb + S::kY + (s & 1) * S::kYBytes, e0, static_cast<int>(t0), seq);
+        bulk_commit();
       }
+      if (s + kStages < n_stages) issue_stage(s + kStages);
     }
   }
-  cp_async_wait<0>();
+  if constexpr (G > 1) {
+    if (tid == 0) bulk_wait<0>();
+  }
 
   if (ch_ok) {
 #pragma unroll
-    for (int s = 0; s < K; ++s) a.ssm_state_out[(seq * a.E + e) * 16 + j * K + s] = h[s];
+    for (int q = 0; q < K; ++q) a.ssm_state_out[(static_cast<int64_t>(seq) * a.E + e) * 16 + j * K + q] = h[q];
     if (j == 0) {
-      // conv_cache_out = last 3 raw rows of [history, x]; read all before writing
-      // (the output may alias conv_cache_in).
+      // conv_cache_out = last 3 raw rows of [history, x]; read all before
+      // writing (the output may alias conv_cache_in).
       const T* x = static_cast<const T*>(a.x);
       const T* hist = static_cast<const T*>(a.conv_cache_in);
       T keep[3];
@@ -296,74 +373,406 @@ __global__ void __launch_bounds__(NCH* G) prefill_kernel(const KernelArgs a) {
         if (t >= 0)
           keep[k] = x[seq * a.s.x_seq + t * a.s.x_tok + e];
         else
-          keep[k] = hist ? hist[(seq * 3 + (3 + t)) * a.E + e] : IO<T>::from_f(0.0f);
+          keep[k] = hist ? hist[(static_cast<int64_t>(seq) * 3 + (3 + t)) * a.E + e] : IO<T>::from_f(0.0f);
       }
       T* out = static_cast<T*>(a.conv_cache_out);
 #pragma unroll
-      for (int k = 0; k < 3; ++k) out[(seq * 3 + k) * a.E + e] = keep[k];
+      for (int k = 0; k < 3; ++k) out[(static_cast<int64_t>(seq) * 3 + k) * a.E + e] = keep[k];
     }
   }
 }
 
-template <typename T, int G, int NCH, bool ZOH>
+// ------------------------------------------------ slice-per-warp kernel ---
+// G > 1: a CTA covers 32 channels with G warps; warp J owns states
+// [J*16/G, (J+1)*16/G) of every channel (lane = channel). B and C are then
+// identical across a warp (broadcast loads), and x, z, the phase-A rows, the
+// partial readouts and y are all lane-contiguous (conflict-free).
+template <typename T, int G>
+struct SliceSmem {
+  static constexpr int kEs = static_cast<int>(sizeof(T));
+  static constexpr int kXBytes = (kTok + 3) * 32 * kEs;
+  static constexpr int kZBytes = kTok * 32 * kEs;
+  static constexpr int kBCBytes = kTok * 16 * 4;
+  static constexpr int kX = 0;
+  static constexpr int kZ = align128(kX + kXBytes);
+  static constexpr int kB = align128(kZ + kZBytes);
+  static constexpr int kC = kB + kBCBytes;
+  static constexpr int kSlot = kC + kBCBytes;
+  static constexpr int kDT = kStages * kSlot;               // float2 (dt, dt*u) [token][channel]
+  static constexpr int kPR = kTok + 4;                      // partial row (padded)
+  static constexpr int kP = kDT + kTok * 32 * 8;            // float [slice][channel][kPR]
+  static constexpr int kDr = kP + G * 32 * kPR * 4;         // dt_raw, 2 stages
+  static constexpr int kY = align128(kDr + 2 * kTok * 4);   // output tiles [token][channel]
+  static constexpr int kYBytes = align128(kTok * 32 * kEs);
+  static constexpr int kBar = kY + 2 * kYBytes;
+  static constexpr int kTotal = kBar + kStages * 8;
+  static constexpr uint32_t kTxBytes = static_cast<uint32_t>(kXBytes + kZBytes + 2 * kBCBytes);
+};
+
+// Phase B for one state slice: advance the slice's K states through kTok
+// tokens, writing the partial readouts C.h to P[slice][lane][*] eight tokens
+// at a time. The pointers do not alias (distinct shared-memory regions).
+template <int K, bool ZOH, int NPOLY>
+__device__ __forceinline__ void slice_phase_b(const float2* __restrict__ DT, const float* __restrict__ Bs,
+                                              const float* __restrict__ Cs, const float* a2, const float* Av, float* h,
+                                              float* __restrict__ Pj, int lane) {
+#pragma unroll 1
+  for (int tc = 0; tc < kTok; tc += 8) {
+    float pr[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int tl = tc + k;
+      const float2 dd = DT[tl * 32 + lane];
+      if constexpr (ZOH)
+        pr[k] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
+      else
+        pr[k] = scan_token<K / 2, NPOLY>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
+    }
+    *reinterpret_cast<float4*>(Pj + tc) = make_float4(pr[0], pr[1], pr[2], pr[3]);
+    *reinterpret_cast<float4*>(Pj + tc + 4) = make_float4(pr[4], pr[5], pr[6], pr[7]);
+  }
+}
+
+template <typename T, int G, bool ZOH, int NPOLY>
+__global__ void __launch_bounds__(32 * G) prefill_slice_kernel(const __grid_constant__ Maps maps, const KernelArgs a) {
+  constexpr int NT = 32 * G;
+  constexpr int K = 16 / G;
+  constexpr int TA = kTok / G;  // phase-A and phase-C tokens per warp
+  using S = SliceSmem<T, G>;
+  static_assert(TA % 4 == 0 && K >= 2, "bad slice shape");
+
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t full0 = sb + S::kBar;
+  float* Dr = reinterpret_cast<float*>(smem + S::kDr);
+  float2* DT = reinterpret_cast<float2*>(smem + S::kDT);
+  float* P = reinterpret_cast<float*>(smem + S::kP);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int64_t tiles = (a.E + 31) / 32;
+  const int seq = static_cast<int>(blockIdx.x / tiles);
+  const int e0 = static_cast<int>(blockIdx.x % tiles) * 32;
+  const int64_t L = a.L;
+  const int64_t n_stages = (L + kTok - 1) / kTok;
+  const float* dtr = a.dt_raw + static_cast<int64_t>(seq) * a.s.dt_seq;
+
+  auto issue_stage = [&](int64_t st_idx) {  // thread 0 only
+    const int slot = static_cast<int>(st_idx % kStages);
+    const uint32_t base = sb + slot * S::kSlot, bar = full0 + 8 * slot;
+    const int t0 = static_cast<int>(st_idx * kTok);
+    mbar_arrive_expect_tx(bar, S::kTxBytes);
+    tma_load_3d(base + S::kX, &maps.x, e0, t0 - 3, seq, bar);
+    tma_load_3d(base + S::kZ, &maps.z, e0, t0, seq, bar);
+    tma_load_3d(base + S::kB, &maps.B, 0, t0, seq, bar);
+    tma_load_3d(base + S::kC, &maps.C, 0, t0, seq, bar);
+  };
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(full0 + 8 * i, 1);
+    mbar_fence_init();
+    prefetch_tensormap(&maps.x);
+    prefetch_tensormap(&maps.z);
+    prefetch_tensormap(&maps.B);
+    prefetch_tensormap(&maps.C);
+    for (int64_t i = 0; i < kStages && i < n_stages; ++i) issue_stage(i);
+  }
+  float d_next = 0.0f;
+  if (tid < 32) {
+    Dr[lane] = lane < L ? dtr[lane] : 0.0f;
+    d_next = kTok + lane < L ? dtr[kTok + lane] : 0.0f;
+  }
+  __syncthreads();
+
+  const int e = e0 + lane;
+  const bool ch_ok = e < a.E;
+  const int64_t ec = ch_ok ? e : a.E - 1;
+  const float cw0 = a.conv_w[ec * 4 + 0], cw1 = a.conv_w[ec * 4 + 1];
+  const float cw2 = a.conv_w[ec * 4 + 2], cw3 = a.conv_w[ec * 4 + 3];
+  const float cb = a.conv_b[ec], wdt = a.w_dt[ec], dtb = a.dt_bias[ec], Dd = a.D[ec];
+  const float lo = a.dt_min, hi = a.dt_max;
+  float hx0 = 0.0f, hx1 = 0.0f, hx2 = 0.0f;
+  if (a.conv_cache_in) {
+    const T* hist = static_cast<const T*>(a.conv_cache_in) + static_cast<int64_t>(seq) * 3 * a.E + ec;
+    hx0 = IO<T>::to_f(hist[0]);
+    hx1 = IO<T>::to_f(hist[a.E]);
+    hx2 = IO<T>::to_f(hist[2 * a.E]);
+  }
+  float a2[K], Av[K], h[K];
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    const float A = -expf(a.A_log[ec * 16 + warp * K + q]);
+    Av[q] = A;
+    a2[q] = A * kLog2e;
+    h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + warp * K + q] : 0.0f;
+  }
+
+  for (int64_t s = 0; s < n_stages; ++s) {
+    const int slot = static_cast<int>(s % kStages);
+    const unsigned char* st = smem + slot * S::kSlot;
+    mbar_wait_bounded(full0 + 8 * slot, static_cast<uint32_t>((s / kStages) & 1), a.err, 1);
+    const T* X = reinterpret_cast<const T*>(st + S::kX);
+    const T* Z = reinterpret_cast<const T*>(st + S::kZ);
+    const float* Bt = reinterpret_cast<const float*>(st + S::kB);
+    const float* Ct = reinterpret_cast<const float*>(st + S::kC);
+    const float* D_ = Dr + (s & 1) * kTok;
+    const int64_t t0 = s * kTok;
+    const bool first = s == 0;
+    const int tb = warp * TA;
+
+    // Phase A: tokens [tb, tb + TA) of this lane's channel. Inputs first, then
+    // the (dt, dt*u) rows; D*u and SiLU(z) stay in registers for phase C.
+    float du[TA], zg[TA];
+    {
+      float xw[TA + 3], zr[TA], dr[TA];
+#pragma unroll
+      for (int i = 0; i < TA + 3; ++i) {
+        const int r = tb + i;
+        xw[i] = (first && r < 3) ? (r == 0 ? hx0 : (r == 1 ? hx1 : hx2)) : IO<T>::to_f(X[r * 32 + lane]);
+      }
+#pragma unroll
+      for (int i = 0; i < TA; ++i) {
+        zr[i] = IO<T>::to_f(Z[(tb + i) * 32 + lane]);
+        dr[i] = D_[tb + i];
+      }
+      float2 dtv[TA];
+#pragma unroll
+      for (int i = 0; i < TA; ++i) {
+        const float conv = fmaf(cw3, xw[i + 3], fmaf(cw2, xw[i + 2], fmaf(cw1, xw[i + 1], fmaf(cw0, xw[i], cb))));
+        const float u = silu(conv);
+        float dt = dt_of(fmaf(dr[i], wdt, dtb), lo, hi);
+        if (t0 + tb + i >= L) dt = 0.0f;  // past the end: keep the state
+        dtv[i] = make_float2(dt, ZOH ? u : dt * u);
+        du[i] = Dd * u;
+        zg[i] = silu(zr[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < TA; ++i) DT[(tb + i) * 32 + lane] = dtv[i];
+    }
+    if (tid == 0) bulk_wait_read<1>();  // output tile (s & 1) no longer read by the store of stage s - 2
+    named_bar_sync(1, NT);
+
+    // Phase B: this warp's state slice through all kTok tokens.
+    slice_phase_b<K, ZOH, NPOLY>(DT, Bt + warp * K, Ct + warp * K, a2, Av, h, P + (warp * 32 + lane) * S::kPR, lane);
+    named_bar_sync(1, NT);
+
+    // Phase C: tokens [tb, tb + TA): sum the G slices, skip, gate, output tile.
+    {
+      float ys[TA];
+#pragma unroll
+      for (int q = 0; q < TA; q += 4) {
+        float4 acc = *reinterpret_cast<const float4*>(P + lane * S::kPR + tb + q);
+#pragma unroll
+        for (int jj = 1; jj < G; ++jj) {
+          const float4 v = *reinterpret_cast<const float4*>(P + (jj * 32 + lane) * S::kPR + tb + q);
+          acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+        }
+        ys[q + 0] = (acc.x + du[q + 0]) * zg[q + 0];
+        ys[q + 1] = (acc.y + du[q + 1]) * zg[q + 1];
+        ys[q + 2] = (acc.z + du[q + 2]) * zg[q + 2];
+        ys[q + 3] = (acc.w + du[q + 3]) * zg[q + 3];
+      }
+      T* Y = reinterpret_cast<T*>(smem + S::kY + (s & 1) * S::kYBytes);
+#pragma unroll
+      for (int i = 0; i < TA; ++i) Y[(tb + i) * 32 + lane] = IO<T>::from_f(ys[i]);
+      fence_proxy_async_smem();
+    }
+
+    if (tid < 32) {
+      Dr[((s + 1) & 1) * kTok + lane] = d_next;
+      const int64_t tn = t0 + 2 * kTok + lane;
+      d_next = tn < L ? dtr[tn] : 0.0f;
+    }
+    named_bar_sync(1, NT);
+    if (tid == 0) {
+      tma_store_3d(&maps.y, sb + S::kY + (s & 1) * S::kYBytes, e0, static_cast<int>(t0), seq);
+      bulk_commit();
+      if (s + kStages < n_stages) issue_stage(s + kStages);
+    }
+  }
+  if (tid == 0) bulk_wait<0>();
+
+  if (ch_ok) {
+#pragma unroll
+    for (int q = 0; q < K; ++q) a.ssm_state_out[(static_cast<int64_t>(seq) * a.E + e) * 16 + warp * K + q] = h[q];
+    if (warp == 0) {
+      const T* x = static_cast<const T*>(a.x);
+      const T* hist = static_cast<const T*>(a.conv_cache_in);
+      T keep[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const int64_t t = L - 3 + k;
+        if (t >= 0)
+          keep[k] = x[seq * a.s.x_seq + t * a.s.x_tok + e];
+        else
+          keep[k] = hist ? hist[(static_cast<int64_t>(seq) * 3 + (3 + t)) * a.E + e] : IO<T>::from_f(0.0f);
+      }
+      T* out = static_cast<T*>(a.conv_cache_out);
+#pragma unroll
+      for (int k = 0; k < 3; ++k) out[(static_cast<int64_t>(seq) * 3 + k) * a.E + e] = keep[k];
+    }
+  }
+}
+
+// L == 0: the outputs are the incoming caches (or zeros).
+template <typename T>
+__global__ void caches_only_kernel(const KernelArgs a) {
+  const int64_t ch = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (ch >= a.batch * a.E) return;
+  const int64_t seq = ch / a.E, e = ch - seq * a.E;
+  for (int n = 0; n < 16; ++n) a.ssm_state_out[ch * 16 + n] = a.ssm_state_in ? a.ssm_state_in[ch * 16 + n] : 0.0f;
+  const T* hist = static_cast<const T*>(a.conv_cache_in);
+  T* out = static_cast<T*>(a.conv_cache_out);
+  T keep[3];
+  for (int k = 0; k < 3; ++k) keep[k] = hist ? hist[(seq * 3 + k) * a.E + e] : IO<T>::from_f(0.0f);
+  for (int k = 0; k < 3; ++k) out[(seq * 3 + k) * a.E + e] = keep[k];
+}
+
+// ------------------------------------------------------------------ host ---
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// Rank-3 tiled map over (inner, rows, seqs) with element strides in bytes.
+bool map3(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+          uint64_t s1_bytes, uint64_t s2_bytes, uint32_t b0, uint32_t b1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes ? s2_bytes : s1_bytes * d1};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int NCH>
+bool make_maps(const KernelArgs& a, Maps* m) {
+  const CUtensorMapDataType dt =
+      sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const uint64_t es = sizeof(T), E = a.E, L = a.L, b = a.batch;
+  return map3(&m->x, dt, a.x, E, L, b, a.s.x_tok * es, a.s.x_seq * es, NCH, kTok + 3) &&
+         map3(&m->z, dt, a.z, E, L, b, a.s.z_tok * es, a.s.z_seq * es, NCH, kTok) &&
+         map3(&m->y, dt, a.y, E, L, b, a.s.y_tok * es, a.s.y_seq * es, NCH, kTok) &&
+         map3(&m->B, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.B, 16, L, b, a.s.bc_tok * 4, a.s.bc_seq * 4, 16, kTok) &&
+         map3(&m->C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.C, 16, L, b, a.s.bc_tok * 4, a.s.bc_seq * 4, 16, kTok);
+}
+
+template <typename T, int G, int NCH, bool ZOH, int NPOLY>
 cudaError_t launch_one(const KernelArgs& a, cudaStream_t st) {
-  using S = Stage<T, NCH>;
-  auto kern = prefill_kernel<T, G, NCH, ZOH>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+  using S = Smem<T, NCH, G>;
+  Maps maps;
+  if (!make_maps<T, NCH>(a, &maps)) return cudaErrorInvalidValue;
+  auto kern = prefill_kernel<T, G, NCH, ZOH, NPOLY>;
+  const int smem = S::kTotal + 128;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  const int64_t tiles = a.batch * ((a.E + NCH - 1) / NCH);
-  if (tiles > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(tiles), NCH * G, S::kTotal, st>>>(a);
+  const int64_t grid = a.batch * ((a.E + NCH - 1) / NCH);
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), NCH * G, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
 
+template <typename T, int G, bool ZOH, int NPOLY>
+cudaError_t launch_slice(const KernelArgs& a, cudaStream_t st) {
+  using S = SliceSmem<T, G>;
+  Maps maps;
+  if (!make_maps<T, 32>(a, &maps)) return cudaErrorInvalidValue;
+  auto kern = prefill_slice_kernel<T, G, ZOH, NPOLY>;
+  const int smem = S::kTotal + 128;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  const int64_t grid = a.batch * ((a.E + 31) / 32);
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<unsigned>(grid), 32 * G, smem, st>>>(maps, a);
+  return cudaGetLastError();
+}
+
+// Every instantiated launch shape. ZOH runs its scalar scan (npoly 0 only).
 template <typename T, bool ZOH>
 cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st) {
-#define SSM_CASE(G_, N_) \
-  if (sh.G == G_ && sh.NCH == N_) return launch_one<T, G_, N_, ZOH>(a, st);
-  SSM_CASE(1, 32)
-  SSM_CASE(1, 64)
-  SSM_CASE(2, 16)
-  SSM_CASE(2, 32)
-  SSM_CASE(2, 64)
-  SSM_CASE(4, 8)
-  SSM_CASE(4, 16)
-  SSM_CASE(4, 32)
-  SSM_CASE(8, 8)
-  SSM_CASE(8, 16)
-  SSM_CASE(8, 32)
-  SSM_CASE(16, 8)
-  SSM_CASE(16, 16)
-  SSM_CASE(16, 32)
-#undef SSM_CASE
+#define SSM_SLICE(G_, P_) \
+  if (sh.kernel == 2 && sh.G == G_ && sh.npoly == P_) return launch_slice<T, G_, ZOH, P_>(a, st);
+#define SSM_TILE(G_, N_, P_) \
+  if (sh.kernel == 1 && sh.G == G_ && sh.NCH == N_ && sh.npoly == P_) return launch_one<T, G_, N_, ZOH, P_>(a, st);
+  SSM_SLICE(2, 0)
+  SSM_SLICE(4, 0)
+  SSM_SLICE(8, 0)
+  SSM_TILE(1, 32, 0)
+  SSM_TILE(1, 64, 0)
+  SSM_TILE(1, 128, 0)
+  SSM_TILE(2, 16, 0)
+  SSM_TILE(2, 32, 0)
+  SSM_TILE(2, 64, 0)
+  SSM_TILE(4, 8, 0)
+  SSM_TILE(4, 16, 0)
+  SSM_TILE(4, 32, 0)
+  SSM_TILE(8, 8, 0)
+  SSM_TILE(8, 16, 0)
+  SSM_TILE(8, 32, 0)
+  if constexpr (!ZOH) {
+    SSM_SLICE(2, 1)
+    SSM_SLICE(2, 2)
+    SSM_SLICE(4, 1)
+    SSM_TILE(1, 32, 1)
+    SSM_TILE(1, 32, 2)
+    SSM_TILE(1, 32, 3)
+    SSM_TILE(1, 64, 1)
+    SSM_TILE(1, 64, 2)
+    SSM_TILE(1, 128, 1)
+    SSM_TILE(1, 128, 2)
+  }
+#undef SSM_SLICE
+#undef SSM_TILE
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 bool prefill_shape_supported(PrefillShape sh) {
-  const int g = sh.G, n = sh.NCH;
-  const bool g_ok = g == 1 || g == 2 || g == 4 || g == 8 || g == 16;
-  const bool n_ok = n == 8 || n == 16 || n == 32 || n == 64;
-  return g_ok && n_ok && g * n >= 32 && g * n <= 512;
+  const int g = sh.G, n = sh.NCH, p = sh.npoly;
+  if (sh.kernel == 2) return (g == 2 && p >= 0 && p <= 2) || (g == 4 && p >= 0 && p <= 1) || (g == 8 && p == 0);
+  if (sh.kernel != 1) return false;
+  if (p != 0) {  // FMA-pipe exp2 variants exist for G == 1 tiles only
+    if (g != 1 || p < 0) return false;
+    return n == 32 ? p <= 3 : ((n == 64 || n == 128) && p <= 2);
+  }
+  if (g == 1) return n == 32 || n == 64 || n == 128;
+  if (g == 2) return n == 16 || n == 32 || n == 64;
+  if (g == 4 || g == 8) return n == 8 || n == 16 || n == 32;
+  return false;
 }
 
-// Enough warps to give every SM sub-partition about two, without splitting L:
-// grow G (threads per channel) until b*E*G/32 reaches that, then pick the
-// widest channel tile that still leaves every SM a tile.
+// Launch shape from the parallelism b*E offers (measured on B200 for the
+// long-context, layer-shape and batched workloads): state slices of 2 when
+// b*E/32 CTAs of 2 warps still leave at most ~one warp per SM sub-partition,
+// state slices of 4 otherwise. The SFU carries every exp2 (npoly 0): the
+// FMA-pipe polynomial measured slower in every shape.
 PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int num_sms) {
-  const int64_t ch = batch * E;
-  const int64_t want_threads = static_cast<int64_t>(num_sms) * 4 * 2 * 32;
-  int g = 1;
-  while (g < 16 && ch * g < want_threads) g *= 2;
-  int n = 32;
-  while (n > 8 && batch * ((E + n - 1) / n) < num_sms && n * g > 32) n /= 2;
-  if (n * g < 32) n = 32 / g;
-  if (n * g > 512) n = 512 / g;
-  return PrefillShape{g, n};
+  const int64_t warps_g2 = batch * ((E + 31) / 32) * 2;
+  if (warps_g2 <= static_cast<int64_t>(num_sms) * 4 * 6 / 5) return PrefillShape{2, 32, 2, 0};
+  return PrefillShape{4, 32, 2, 0};
 }
 
 cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st) {
+  if (a.L == 0) {
+    const int64_t n = a.batch * a.E;
+    const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+    if (io_bf16)
+      caches_only_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(a);
+    else
+      caches_only_kernel<float><<<blocks, 256, 0, st>>>(a);
+    return cudaGetLastError();
+  }
   if (!prefill_shape_supported(sh)) return cudaErrorInvalidValue;
   if (io_bf16) return zoh ? dispatch<__nv_bfloat16, true>(a, sh, st) : dispatch<__nv_bfloat16, false>(a, sh, st);
   return zoh ? dispatch<float, true>(a, sh, st) : dispatch<float, false>(a, sh, st);

@@ -74,7 +74,8 @@ ssm_status check_weights(const ssm_weights* w) {
   const char* names[6] = {"conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D"};
   for (int i = 0; i < 6; ++i) {
     if (!p[i]) return fail(SSM_ERR_INVALID_ARG, "weights.%s is NULL", names[i]);
-    if (!aligned(p[i], 4)) return fail(SSM_ERR_INVALID_ARG, "weights.%s is not 4-byte aligned", names[i]);
+    const size_t need = (i == 0 || i == 4) ? 16 : 4;  // conv_w and A_log rows are read as 16-byte vectors
+    if (!aligned(p[i], need)) return fail(SSM_ERR_INVALID_ARG, "weights.%s is not %zu-byte aligned", names[i], need);
   }
   return SSM_OK;
 }
@@ -101,6 +102,19 @@ void fill_weights(ssm::KernelArgs& a, const ssm_weights* w) {
 }
 
 __device__ int g_device_error = 0;
+
+// Device address of the error word on the current device (looked up once per
+// device; host code must not pass the symbol itself to a kernel).
+int* device_error_ptr() {
+  static int* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  if (dev >= 0 && dev < 64) cache[dev] = static_cast<int*>(p);
+  return static_cast<int*>(p);
+}
 
 }  // namespace
 
@@ -138,10 +152,13 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
 
   ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current());
   if (tuning) {
+    if (tuning->kernel) sh.kernel = tuning->kernel;
+    if (tuning->poly_pairs >= 0) sh.npoly = tuning->poly_pairs;
     if (tuning->threads_per_channel) sh.G = tuning->threads_per_channel;
     if (tuning->channels_per_cta) sh.NCH = tuning->channels_per_cta;
+    if (sh.kernel == 1 && !tuning->channels_per_cta && sh.G > 1) sh.NCH = 32;
     if (!ssm::prefill_shape_supported(sh))
-      return fail(SSM_ERR_INVALID_ARG, "tuning: unsupported shape G=%d NCH=%d", sh.G, sh.NCH);
+      return fail(SSM_ERR_INVALID_ARG, "tuning: unsupported shape kernel=%d G=%d NCH=%d", sh.kernel, sh.G, sh.NCH);
   }
 
   ssm::KernelArgs a{};
@@ -162,6 +179,8 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
   a.s = s;
   a.dt_min = dims->dt_min;
   a.dt_max = dims->dt_max;
+  a.err = device_error_ptr();
+  if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   cudaError_t err = ssm::launch_prefill(a, dims->io_dtype == SSM_BF16, dims->discretization == SSM_DISC_ZOH, sh,
                                         static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
@@ -212,6 +231,8 @@ ssm_status ssm_decode_step(const ssm_dims* dims, const ssm_weights* w, const voi
   a.s = s;
   a.dt_min = dims->dt_min;
   a.dt_max = dims->dt_max;
+  a.err = device_error_ptr();
+  if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   cudaError_t err = ssm::launch_decode(a, dims->io_dtype == SSM_BF16, dims->discretization == SSM_DISC_ZOH,
                                        static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));

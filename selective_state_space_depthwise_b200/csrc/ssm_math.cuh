@@ -67,6 +67,45 @@ __device__ __forceinline__ float expm1_nonpos(float x, float ex) {
   return x > -0.125f ? series : ex - 1.0f;
 }
 
+// 2^x for x <= 0 on the FMA pipe, for a pair of arguments (packed f32x2):
+// x = n + f with n = round(x), f in [-1/2, 1/2]; 2^f by a degree-5 polynomial
+// whose maximum relative error on [-1/2, 1/2] was minimised by the Remez
+// exchange algorithm (fit_exp2_poly.py; 2.4e-7 in float32, on par with
+// ex2.approx); 2^n is added to the exponent field. Arguments below -125 are
+// clamped there (2^-125 ~ 2e-38, where the SFU version flushes to zero).
+__device__ __forceinline__ uint64_t ex2_poly2(float x0, float x1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer in the low bits
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  uint64_t x;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  uint64_t sh, t, n, f, p;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(sh) : "f"(kShift));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(sh));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(sh));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(n));
+  uint64_t c;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(p) : "f"(1.327647245e-03f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(9.675540961e-03f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(5.550713092e-02f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(2.402212024e-01f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(6.931469440e-01f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(1.000000119e+00f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c));
+  uint32_t t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+  p0 += t0 << 23;  // t's low mantissa bits hold n; shifted, they add n to p's exponent
+  p1 += t1 << 23;
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(p0), "r"(p1));
+  return r;
+}
+
 template <typename T>
 struct IO;
 

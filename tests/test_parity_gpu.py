@@ -15,8 +15,9 @@ from selective_state_space_depthwise_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-SHAPES = [(1, 32), (1, 64), (2, 16), (2, 32), (4, 8), (4, 16), (4, 32), (8, 8), (8, 16), (8, 32), (16, 8), (16, 16),
-          (16, 32)]
+# (kernel, G, channels per CTA): kernel 1 = channel tiles, kernel 2 = state slices (32 channels per CTA)
+SHAPES = [(1, 1, 32), (1, 1, 64), (1, 1, 128), (1, 2, 16), (1, 2, 32), (1, 2, 64), (1, 4, 8), (1, 4, 16), (1, 4, 32),
+          (1, 8, 8), (1, 8, 16), (1, 8, 32), (2, 2, 0), (2, 4, 0), (2, 8, 0)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -41,14 +42,46 @@ def device_inputs(w, gen_device="cpu"):
 
 
 @pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("shape", SHAPES, ids=[f"G{g}_N{n}" for g, n in SHAPES])
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"k{k}_G{g}_N{n}" for k, g, n in SHAPES])
 def test_prefill_every_launch_shape(io_dtype, shape):
-    # E = 48 leaves a ragged channel tile for N = 32; L = 200 leaves a ragged stage.
+    # E = 48 leaves a ragged channel tile for N >= 32; L = 200 leaves a ragged stage.
     w = small_workload(io_dtype)
     inp = device_inputs(w)
-    y, cc, st = run_prefill(inp, tuning={"threads_per_channel": shape[0], "channels_per_cta": shape[1]})
+    k, g, n = shape
+    y, cc, st = run_prefill(inp, tuning={"kernel": k, "threads_per_channel": g, "channels_per_cta": n})
     chans = all_channels(w.batch, w.d_inner)
-    compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"G{shape[0]} N{shape[1]}")
+    compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"kernel {k} G{g} N{n}")
+
+
+POLY = [(1, 1, 32, 1), (1, 1, 32, 3), (1, 1, 64, 2), (1, 1, 128, 1), (2, 2, 0, 1), (2, 2, 0, 2), (2, 4, 0, 1)]
+
+
+@pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", POLY, ids=[f"k{k}_G{g}_N{n}_p{p}" for k, g, n, p in POLY])
+def test_prefill_fma_pipe_exp2_variants(io_dtype, shape):
+    """Launch shapes where some decays use the FMA-pipe exp2 polynomial."""
+    w = small_workload(io_dtype, b=2, L=150, E=64, seed=13)
+    inp = device_inputs(w)
+    k, g, n, p = shape
+    y, cc, st = run_prefill(inp, tuning={"kernel": k, "threads_per_channel": g, "channels_per_cta": n, "poly_pairs": p})
+    chans = all_channels(w.batch, w.d_inner)
+    compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"poly {shape}")
+
+
+@pytest.mark.parametrize("g", [2, 4, 8])
+def test_slice_kernel_lengths_history_and_zoh(g):
+    """The state-slice kernel on short sequences, with incoming caches, and ZOH."""
+    for L, E, disc in ((1, 32, "euler"), (3, 40, "euler"), (33, 64, "zoh"), (97, 32, "euler")):
+        w = small_workload(torch.bfloat16, b=2, L=L, E=E, seed=90 + L)
+        inp = device_inputs(w)
+        gen = torch.Generator(device="cpu").manual_seed(5)
+        cc_in = torch.randn((2, 3, E), generator=gen).to(torch.bfloat16).cuda()
+        st_in = torch.randn((2, E, 16), generator=gen).cuda()
+        y, cc, st = run_prefill(inp, conv_cache_in=cc_in, ssm_state_in=st_in, discretization=disc,
+                                tuning={"kernel": 2, "threads_per_channel": g})
+        chans = all_channels(2, E)
+        want = oracle_prefill(inp, chans, conv_cache_in=cc_in, ssm_state_in=st_in, disc=disc)
+        compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"slice G{g} L{L} {disc}")
 
 
 def test_tiny_workload_fp32_full():
