@@ -41,6 +41,13 @@ namespace ssm {
 namespace {
 
 constexpr int kTok = 32;    // tokens per pipeline stage (= lanes of the dt_raw stager)
+// Phase-B tokens computed between partial-readout stores, per states-per-warp
+// K (measured on B200: longer unrolled runs hide more latency until registers
+// run out; 32 for K = 4, 16 for K = 8, 4 for K = 2).
+template <int K>
+constexpr int phase_b_chunk() {
+  return K == 4 ? 32 : (K == 8 ? 16 : 4);
+}
 constexpr int kStages = 3;  // ring depth
 
 struct Maps {
@@ -410,17 +417,17 @@ struct SliceSmem {
 };
 
 // Phase B for one state slice: advance the slice's K states through kTok
-// tokens, writing the partial readouts C.h to P[slice][lane][*] eight tokens
-// at a time. The pointers do not alias (distinct shared-memory regions).
-template <int K, bool ZOH, int NPOLY>
+// tokens, writing the partial readouts C.h to P[slice][lane][*] kBChunk
+// tokens at a time (registers hold a chunk's readouts between stores). The pointers do not alias (distinct shared-memory regions).
+template <int K, bool ZOH, int NPOLY, int kBChunk = phase_b_chunk<K>()>
 __device__ __forceinline__ void slice_phase_b(const float2* __restrict__ DT, const float* __restrict__ Bs,
                                               const float* __restrict__ Cs, const float* a2, const float* Av, float* h,
                                               float* __restrict__ Pj, int lane) {
 #pragma unroll 1
-  for (int tc = 0; tc < kTok; tc += 8) {
-    float pr[8];
+  for (int tc = 0; tc < kTok; tc += kBChunk) {
+    float pr[kBChunk];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < kBChunk; ++k) {
       const int tl = tc + k;
       const float2 dd = DT[tl * 32 + lane];
       if constexpr (ZOH)
@@ -428,8 +435,9 @@ __device__ __forceinline__ void slice_phase_b(const float2* __restrict__ DT, con
       else
         pr[k] = scan_token<K / 2, NPOLY>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
     }
-    *reinterpret_cast<float4*>(Pj + tc) = make_float4(pr[0], pr[1], pr[2], pr[3]);
-    *reinterpret_cast<float4*>(Pj + tc + 4) = make_float4(pr[4], pr[5], pr[6], pr[7]);
+#pragma unroll
+    for (int k = 0; k < kBChunk; k += 4)
+      *reinterpret_cast<float4*>(Pj + tc + k) = make_float4(pr[k], pr[k + 1], pr[k + 2], pr[k + 3]);
   }
 }
 
@@ -752,14 +760,11 @@ bool prefill_shape_supported(PrefillShape sh) {
   return false;
 }
 
-// Launch shape from the parallelism b*E offers (measured on B200 for the
-// long-context, layer-shape and batched workloads): state slices of 2 when
-// b*E/32 CTAs of 2 warps still leave at most ~one warp per SM sub-partition,
-// state slices of 4 otherwise. The SFU carries every exp2 (npoly 0): the
-// FMA-pipe polynomial measured slower in every shape.
-PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int num_sms) {
-  const int64_t warps_g2 = batch * ((E + 31) / 32) * 2;
-  if (warps_g2 <= static_cast<int64_t>(num_sms) * 4 * 6 / 5) return PrefillShape{2, 32, 2, 0};
+// Default launch shape: state slices of 4 warps (measured best on B200 for the
+// long-context, layer-shape and batched workloads once phase B streams 32
+// tokens per chunk). The SFU carries every exp2 (npoly 0): the FMA-pipe
+// polynomial measured slower in every shape.
+PrefillShape choose_prefill_shape(int64_t /*batch*/, int64_t /*E*/, int64_t /*L*/, int /*num_sms*/) {
   return PrefillShape{4, 32, 2, 0};
 }
 

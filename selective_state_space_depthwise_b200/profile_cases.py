@@ -1,0 +1,59 @@
+"""Small, fixed launches of the kernels for profiler captures.
+
+    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL G N NPOLY]
+    python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
+
+prefill: three launches of the named workload's prefill (optionally shortened
+to L tokens, optionally with an explicit launch shape); decode: a 4-token
+prompt, then three decode steps at the decode workload's shape (batch 256,
+E=7680, 252 MB of state). Inputs are drawn on the GPU; a capture skips the
+first two launches (ncu -s 2 -c 1 -k regex:...).
+"""
+from __future__ import annotations
+
+import sys
+
+import torch
+
+from . import api
+from . import workloads as W
+
+
+def prefill_case(name: str, L: int = 0, shape=None):
+    w = W.WORKLOADS[name]
+    if L > 0:
+        w = w.scaled(seqlen=L)
+    tun = None
+    if shape:
+        k, g, n, p = shape
+        tun = {"kernel": k, "threads_per_channel": g, "channels_per_cta": n, "poly_pairs": p}
+    inp = W.make_inputs(w, device="cuda", gen_device="cuda")
+    args = (inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp)
+    for _ in range(3):
+        y, _, _ = api.prefill(*args, tuning=tun)
+    torch.cuda.synchronize()
+    print("prefill ok", name, w.seqlen, float(y.float().abs().mean()))
+
+
+def decode_case(batch: int = 256):
+    w = W.WORKLOADS["decode"].scaled(batch=batch, seqlen=4, decode_steps=3)
+    inp = W.make_inputs(w, device="cuda", gen_device="cuda")
+    pre = {**inp, **{k: inp[k][:, :4] for k in ("x", "z", "B", "C", "dt_raw")}}
+    _, cc, st = api.prefill(pre["x"], pre["z"], pre["B"], pre["C"], pre["dt_raw"], pre)
+    y = torch.empty((w.batch, w.d_inner), dtype=w.io_dtype, device="cuda")
+    for t in range(4, 7):
+        api.decode_step(inp["x"][:, t], inp["z"][:, t], inp["B"][:, t], inp["C"][:, t], inp["dt_raw"][:, t], inp, cc,
+                        st, y=y)
+    torch.cuda.synchronize()
+    print("decode ok", float(y.float().abs().mean()))
+
+
+if __name__ == "__main__":
+    if sys.argv[1] == "prefill":
+        L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
+        shape = tuple(int(v) for v in sys.argv[4:8]) if len(sys.argv) > 7 else None
+        prefill_case(sys.argv[2], L, shape)
+    elif sys.argv[1] == "decode":
+        decode_case(int(sys.argv[2]) if len(sys.argv) > 2 else 256)
+    else:
+        raise SystemExit(__doc__)
