@@ -101,11 +101,13 @@ typedef struct {
  * kernel 1 (channel tiles): G = threads_per_channel lanes of one warp share a
  *   channel; channels_per_cta: G=1: 32/64/128, G=2: 16/32/64, G=4 or 8: 8/16/32.
  * kernel 2 (state slices): a CTA of G warps covers 32 channels and warp j owns
- *   state slice j of each; threads_per_channel = G in {2, 4, 8}. */
+ *   state slice j of each; threads_per_channel = G in {2, 4, 8}.
+ * kernel 3 (pipelined state slices): kernel 2 with the per-token work of the
+ *   next stage overlapped with the scan of the current one; G in {4, 8}. */
 typedef struct {
   int32_t threads_per_channel; /* 0 = auto, else 1, 2, 4 or 8 */
   int32_t channels_per_cta;    /* 0 = auto (kernel 1 only) */
-  int32_t kernel;              /* 0 = auto, 1 = channel tiles, 2 = state slices */
+  int32_t kernel;              /* 0 = auto, 1 = channel tiles, 2 = state slices, 3 = pipelined slices */
   int32_t poly_pairs;          /* -1 = auto; else state pairs per thread and token whose
                                   exp2 runs as an FMA-pipe polynomial instead of on the SFU */
 } ssm_tuning;

@@ -1,10 +1,10 @@
 """Small, fixed launches of the kernels for profiler captures.
 
-    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL G N NPOLY]
+    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL G N NPOLY] [E]
     python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
 
 prefill: three launches of the named workload's prefill (optionally shortened
-to L tokens, optionally with an explicit launch shape); decode: a 4-token
+to L tokens, optionally with an explicit launch shape and E channels); decode: a 4-token
 prompt, then three decode steps at the decode workload's shape (batch 256,
 E=7680, 252 MB of state). Inputs are drawn on the GPU; a capture skips the
 first two launches (ncu -s 2 -c 1 -k regex:...).
@@ -19,10 +19,12 @@ from . import api
 from . import workloads as W
 
 
-def prefill_case(name: str, L: int = 0, shape=None):
+def prefill_case(name: str, L: int = 0, shape=None, E: int = 0):
     w = W.WORKLOADS[name]
     if L > 0:
         w = w.scaled(seqlen=L)
+    if E > 0:
+        w = w.scaled(d_inner=E)
     tun = None
     if shape:
         k, g, n, p = shape
@@ -32,7 +34,7 @@ def prefill_case(name: str, L: int = 0, shape=None):
     for _ in range(3):
         y, _, _ = api.prefill(*args, tuning=tun)
     torch.cuda.synchronize()
-    print("prefill ok", name, w.seqlen, float(y.float().abs().mean()))
+    print("prefill ok", name, w.seqlen, w.d_inner, float(y.float().abs().mean()))
 
 
 def decode_case(batch: int = 256):
@@ -52,7 +54,8 @@ if __name__ == "__main__":
     if sys.argv[1] == "prefill":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
         shape = tuple(int(v) for v in sys.argv[4:8]) if len(sys.argv) > 7 else None
-        prefill_case(sys.argv[2], L, shape)
+        E = int(sys.argv[8]) if len(sys.argv) > 8 else 0
+        prefill_case(sys.argv[2], L, shape, E)
     elif sys.argv[1] == "decode":
         decode_case(int(sys.argv[2]) if len(sys.argv) > 2 else 256)
     else:

@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 # (kernel, G, channels per CTA): kernel 1 = channel tiles, kernel 2 = state slices (32 channels per CTA)
 SHAPES = [(1, 1, 32), (1, 1, 64), (1, 1, 128), (1, 2, 16), (1, 2, 32), (1, 2, 64), (1, 4, 8), (1, 4, 16), (1, 4, 32),
-          (1, 8, 8), (1, 8, 16), (1, 8, 32), (2, 2, 0), (2, 4, 0), (2, 8, 0)]
+          (1, 8, 8), (1, 8, 16), (1, 8, 32), (2, 2, 0), (2, 4, 0), (2, 8, 0), (3, 4, 0), (3, 8, 0)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -68,9 +68,10 @@ def test_prefill_fma_pipe_exp2_variants(io_dtype, shape):
     compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"poly {shape}")
 
 
-@pytest.mark.parametrize("g", [2, 4, 8])
-def test_slice_kernel_lengths_history_and_zoh(g):
-    """The state-slice kernel on short sequences, with incoming caches, and ZOH."""
+@pytest.mark.parametrize("kg", [(2, 2), (2, 4), (2, 8), (3, 4), (3, 8)])
+def test_slice_kernel_lengths_history_and_zoh(kg):
+    """The state-slice kernels on short sequences, with incoming caches, and ZOH."""
+    kern, g = kg
     for L, E, disc in ((1, 32, "euler"), (3, 40, "euler"), (33, 64, "zoh"), (97, 32, "euler")):
         w = small_workload(torch.bfloat16, b=2, L=L, E=E, seed=90 + L)
         inp = device_inputs(w)
@@ -78,10 +79,10 @@ def test_slice_kernel_lengths_history_and_zoh(g):
         cc_in = torch.randn((2, 3, E), generator=gen).to(torch.bfloat16).cuda()
         st_in = torch.randn((2, E, 16), generator=gen).cuda()
         y, cc, st = run_prefill(inp, conv_cache_in=cc_in, ssm_state_in=st_in, discretization=disc,
-                                tuning={"kernel": 2, "threads_per_channel": g})
+                                tuning={"kernel": kern, "threads_per_channel": g})
         chans = all_channels(2, E)
         want = oracle_prefill(inp, chans, conv_cache_in=cc_in, ssm_state_in=st_in, disc=disc)
-        compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"slice G{g} L{L} {disc}")
+        compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"kernel {kern} G{g} L{L} {disc}")
 
 
 def test_tiny_workload_fp32_full():
