@@ -103,11 +103,14 @@ typedef struct {
  * kernel 2 (state slices): a CTA of G warps covers 32 channels and warp j owns
  *   state slice j of each; threads_per_channel = G in {2, 4, 8}.
  * kernel 3 (pipelined state slices): kernel 2 with the per-token work of the
- *   next stage overlapped with the scan of the current one; G in {4, 8}. */
+ *   next stage overlapped with the scan of the current one; G in {4, 8}.
+ * kernel 4: kernel 3 compiled for at most two resident CTAs per SM (a larger
+ *   register budget); G = 4. The automatic choice takes it when
+ *   batch * ceil(d_inner / 32) <= 2 * SMs, else kernel 3. */
 typedef struct {
   int32_t threads_per_channel; /* 0 = auto, else 1, 2, 4 or 8 */
   int32_t channels_per_cta;    /* 0 = auto (kernel 1 only) */
-  int32_t kernel;              /* 0 = auto, 1 = channel tiles, 2 = state slices, 3 = pipelined slices */
+  int32_t kernel;              /* 0 = auto, 1 = channel tiles, 2 = state slices, 3/4 = pipelined slices */
   int32_t poly_pairs;          /* -1 = auto; else state pairs per thread and token whose
                                   exp2 runs as an FMA-pipe polynomial instead of on the SFU */
 } ssm_tuning;

@@ -2,9 +2,10 @@
 //
 // Transcendentals go to the SFU through the PTX approximations ex2.approx and
 // rcp.approx (relative error ~2^-22). Where those lose accuracy near a
-// cancellation, the functions below use series written from the mathematics:
-//  - log1p on [0, 1] via log(1 + e) = 2 atanh(s), s = e / (2 + e) <= 1/3,
-//    with the odd Taylor series of atanh through s^15 (truncation < 2e-9 rel.);
+// cancellation, the functions below use polynomials and series instead:
+//  - log1p on [0, 1] as e * Q(e), Q a degree-8 polynomial whose maximum
+//    relative error on [0, 1] was minimised by the Remez exchange algorithm
+//    (fit_log1p_poly.py; 1.8e-7 in float32), FMA pipe only;
 //  - expm1 near 0 via its Taylor series through x^5 (|x| < 1/8: < 5e-8 rel.).
 #pragma once
 
@@ -34,18 +35,18 @@ __device__ __forceinline__ float sigmoid(float v) { return rcp_approx(1.0f + ex2
 // SiLU(v) = v * sigmoid(v).
 __device__ __forceinline__ float silu(float v) { return v * sigmoid(v); }
 
-// log(1 + e) for e in [0, 1]: 2 * atanh(e / (2 + e)) as an odd series.
+// log(1 + e) for e in [0, 1]: e * Q(e) by Horner (coefficients from
+// fit_log1p_poly.py, degree 8). No division, so no SFU work.
 __device__ __forceinline__ float log1p_unit(float e) {
-  const float s = e * rcp_approx(2.0f + e);
-  const float s2 = s * s;
-  float p = fmaf(s2, 1.0f / 15.0f, 1.0f / 13.0f);
-  p = fmaf(s2, p, 1.0f / 11.0f);
-  p = fmaf(s2, p, 1.0f / 9.0f);
-  p = fmaf(s2, p, 1.0f / 7.0f);
-  p = fmaf(s2, p, 1.0f / 5.0f);
-  p = fmaf(s2, p, 1.0f / 3.0f);
-  p = fmaf(s2, p, 1.0f);
-  return 2.0f * s * p;
+  float q = fmaf(e, 5.232694093e-03f, -2.950523980e-02f);
+  q = fmaf(e, q, 7.822595537e-02f);
+  q = fmaf(e, q, -1.366324574e-01f);
+  q = fmaf(e, q, 1.910600662e-01f);
+  q = fmaf(e, q, -2.484298199e-01f);
+  q = fmaf(e, q, 3.331909776e-01f);
+  q = fmaf(e, q, -4.999949336e-01f);
+  q = fmaf(e, q, 9.999999404e-01f);
+  return e * q;
 }
 
 // softplus(v) = log(1 + e^v) = max(v, 0) + log1p(e^-|v|), overflow-free.

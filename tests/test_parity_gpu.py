@@ -17,7 +17,7 @@ pytestmark = pytest.mark.gpu
 
 # (kernel, G, channels per CTA): kernel 1 = channel tiles, kernel 2 = state slices (32 channels per CTA)
 SHAPES = [(1, 1, 32), (1, 1, 64), (1, 1, 128), (1, 2, 16), (1, 2, 32), (1, 2, 64), (1, 4, 8), (1, 4, 16), (1, 4, 32),
-          (1, 8, 8), (1, 8, 16), (1, 8, 32), (2, 2, 0), (2, 4, 0), (2, 8, 0), (3, 4, 0), (3, 8, 0)]
+          (1, 8, 8), (1, 8, 16), (1, 8, 32), (2, 2, 0), (2, 4, 0), (2, 8, 0), (3, 4, 0), (3, 8, 0), (4, 4, 0)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -68,7 +68,7 @@ def test_prefill_fma_pipe_exp2_variants(io_dtype, shape):
     compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"poly {shape}")
 
 
-@pytest.mark.parametrize("kg", [(2, 2), (2, 4), (2, 8), (3, 4), (3, 8)])
+@pytest.mark.parametrize("kg", [(2, 2), (2, 4), (2, 8), (3, 4), (3, 8), (4, 4)])
 def test_slice_kernel_lengths_history_and_zoh(kg):
     """The state-slice kernels on short sequences, with incoming caches, and ZOH."""
     kern, g = kg
