@@ -150,6 +150,53 @@ ssm_status ssm_prefill_ex(const ssm_dims *dims, const ssm_weights *w, const void
 size_t ssm_prefill_workspace_bytes(const ssm_dims *dims);
 
 /*
+ * ssm_prefill_host -- ssm_prefill with the token tensors in HOST memory. The
+ * block core is the same, from the same pages and sections as ssm_prefill:
+ * prefill of "Axon-SSM: selective state space model", "Algorithm".
+ *
+ * What it does. x, z, B, C and dt_raw are read from host buffers, and y is
+ * written to a host buffer. L is processed in chunks of chunk_tokens tokens,
+ * and three kinds of work overlap chunk by chunk:
+ *  - the host->device copies of chunk c + 1, on an internal copy-in stream;
+ *  - the kernel of chunk c, on `stream`;
+ *  - the device->host copy of chunk c - 1's y, on an internal copy-out stream.
+ * The caches carry from chunk to chunk on the device: conv_cache_out and
+ * ssm_state_out serve as the carry. The result therefore equals one
+ * ssm_prefill over the whole sequence, bit for bit.
+ *
+ * Arguments.
+ *   x, z, B, C, dt_raw, y   HOST pointers, laid out as in ssm_prefill. The
+ *                           token and sequence strides of dims apply to them.
+ *                           Page-locked (pinned) memory lets the copies overlap;
+ *                           pageable memory gives the same result, serialised.
+ *   conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out
+ *                           device pointers, as in ssm_prefill.
+ *   workspace               device scratch of at least
+ *                           ssm_prefill_host_workspace_bytes(dims, chunk_tokens)
+ *                           bytes, 256-byte aligned. It holds two chunk buffers.
+ *   chunk_tokens            tokens per chunk, >= 1; 0 selects 2048.
+ *
+ * Ordering. The call returns once every copy and kernel is enqueued. The first
+ * copy waits for the work already queued on `stream`, and `stream` waits for
+ * the last copy. A synchronisation of `stream` therefore makes y complete on
+ * the host. The host buffers and the workspace must stay valid until then.
+ * Enqueueing from several host threads is serialised inside the library.
+ *
+ * Errors. Argument errors return SSM_ERR_INVALID_ARG before any work is
+ * queued. A CUDA error while enqueueing returns SSM_ERR_CUDA. Chunks already
+ * enqueued then still run, and `stream` is left waiting for them.
+ */
+ssm_status ssm_prefill_host(const ssm_dims *dims, const ssm_weights *w, const void *x, const void *z,
+                            const float *B, const float *C, const float *dt_raw, const void *conv_cache_in,
+                            const float *ssm_state_in, void *y, void *conv_cache_out, float *ssm_state_out,
+                            void *workspace, size_t workspace_bytes, int64_t chunk_tokens, void *stream);
+
+/* Device scratch bytes ssm_prefill_host needs for `dims` and `chunk_tokens`
+ * (0 selects 2048): two chunk buffers of x, z, y, B, C and dt_raw. Returns 0
+ * for invalid dims. */
+size_t ssm_prefill_host_workspace_bytes(const ssm_dims *dims, int64_t chunk_tokens);
+
+/*
  * ssm_decode_step -- one-token mode ("Autoregressive decoding", later calls):
  * concatenates conv_cache with the new token, runs the conv for that token and
  * exactly one scan step from ssm_state, and updates both caches IN PLACE.

@@ -21,6 +21,8 @@ EXPORTED = (
     "ssm_prefill",
     "ssm_prefill_ex",
     "ssm_prefill_workspace_bytes",
+    "ssm_prefill_host",
+    "ssm_prefill_host_workspace_bytes",
     "ssm_decode_step",
     "ssm_check_device_error",
     "ssm_status_string",
@@ -86,6 +88,10 @@ def load(path: str = LIB_PATH):
     lib.ssm_prefill_ex.restype = st
     lib.ssm_prefill_workspace_bytes.argtypes = [dims_p]
     lib.ssm_prefill_workspace_bytes.restype = sz
+    lib.ssm_prefill_host.argtypes = [dims_p, w_p] + [p] * 10 + [p, sz, ctypes.c_int64, p]
+    lib.ssm_prefill_host.restype = st
+    lib.ssm_prefill_host_workspace_bytes.argtypes = [dims_p, ctypes.c_int64]
+    lib.ssm_prefill_host_workspace_bytes.restype = sz
     lib.ssm_decode_step.argtypes = [dims_p, w_p] + [p] * 8 + [p]
     lib.ssm_decode_step.restype = st
     lib.ssm_check_device_error.argtypes = [p]

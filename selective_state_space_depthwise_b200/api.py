@@ -122,6 +122,62 @@ def prefill(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None
     return y, conv_cache_out, ssm_state_out
 
 
+def host_workspace_bytes(batch, seqlen, E, io_dtype=torch.bfloat16, chunk_tokens=0) -> int:
+    lib = _lib.load()
+    return int(lib.ssm_prefill_host_workspace_bytes(ctypes.byref(make_dims(batch, seqlen, E, io_dtype)),
+                                                    int(chunk_tokens)))
+
+
+def prefill_host(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None, y=None, conv_cache_out=None,
+                 ssm_state_out=None, dt_min=1e-4, dt_max=1.0, discretization="euler", chunk_tokens=0, workspace=None,
+                 stream=None):
+    """Full-sequence block core with the token tensors in host memory
+    (ssm_prefill_host): x, z, B, C, dt_raw and y are CPU tensors (pinned for
+    overlapped copies), shaped and strided as for `prefill`; the parameters and
+    the caches are CUDA tensors on the current device. The copies and kernels
+    are only enqueued: synchronise `stream` before reading y.
+    Returns (y [b, L, E] on the host, conv_cache_out, ssm_state_out)."""
+    lib = _lib.load()
+    b, L, E = x.shape
+    dev = params["A_log"].device
+    for n, t in (("x", x), ("z", z), ("B", B), ("C", C), ("dt_raw", dt_raw), ("y", y)):
+        if t is not None and t.is_cuda:
+            raise RuntimeError(f"{n} must be a host tensor for prefill_host (use prefill for device tensors)")
+    for n, t in (("conv_cache_in", conv_cache_in), ("ssm_state_in", ssm_state_in),
+                 ("conv_cache_out", conv_cache_out), ("ssm_state_out", ssm_state_out)):
+        _need_cuda(n, t, dev)
+    if x.dtype not in _DTYPES or z.dtype != x.dtype:
+        raise ValueError("x and z must share an io dtype (float32 or bfloat16)")
+    if z.shape != (b, L, E) or B.shape != (b, L, 16) or C.shape != (b, L, 16) or dt_raw.shape != (b, L):
+        raise ValueError("shape mismatch: z [b,L,E], B/C [b,L,16], dt_raw [b,L]")
+    if x.stride(2) != 1 or z.stride(2) != 1 or B.stride(2) != 1 or dt_raw.stride(1) != 1:
+        raise ValueError("the innermost dimension of x, z, B, C, dt_raw must be contiguous")
+    if B.stride() != C.stride():
+        raise ValueError("B and C must share strides")
+    if y is None:
+        y = torch.empty((b, L, E), dtype=x.dtype, pin_memory=True)
+    if conv_cache_out is None:
+        conv_cache_out = torch.empty((b, 3, E), dtype=x.dtype, device=dev)
+    if ssm_state_out is None:
+        ssm_state_out = torch.empty((b, E, 16), dtype=torch.float32, device=dev)
+    if y.shape != (b, L, E) or y.dtype != x.dtype or y.stride(2) != 1:
+        raise ValueError("y must be [b, L, E] in the io dtype with a contiguous last dim")
+    dims = make_dims(b, L, E, x.dtype, dt_min, dt_max, discretization,
+                     x_tok_stride=x.stride(1), x_seq_stride=x.stride(0), z_tok_stride=z.stride(1),
+                     z_seq_stride=z.stride(0), y_tok_stride=y.stride(1), y_seq_stride=y.stride(0),
+                     bc_tok_stride=B.stride(1), bc_seq_stride=B.stride(0), dt_seq_stride=dt_raw.stride(0))
+    w = _weights(params, E, dev)
+    ws = int(lib.ssm_prefill_host_workspace_bytes(ctypes.byref(dims), int(chunk_tokens)))
+    if workspace is None or workspace.numel() < ws:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+    st = lib.ssm_prefill_host(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
+                              _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(y), _ptr(conv_cache_out),
+                              _ptr(ssm_state_out), _ptr(workspace), workspace.numel(), int(chunk_tokens),
+                              _stream(stream))
+    _lib.check(st)
+    return y, conv_cache_out, ssm_state_out
+
+
 def decode_step(x, z, B, C, dt_raw, params, conv_cache, ssm_state, *, y=None, dt_min=1e-4, dt_max=1.0,
                 discretization="euler", stream=None):
     """One-token block core. x, z: [b, E] (last dim contiguous); B, C: [b, 16];

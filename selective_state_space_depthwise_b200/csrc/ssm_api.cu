@@ -12,8 +12,10 @@
 #include "ssm_internal.h"
 
 namespace {
-
 thread_local char g_last_error[512] = "";
+}  // namespace
+
+namespace ssm {
 
 ssm_status fail(ssm_status st, const char* fmt, ...) {
   va_list ap;
@@ -22,13 +24,6 @@ ssm_status fail(ssm_status st, const char* fmt, ...) {
   va_end(ap);
   return st;
 }
-
-ssm_status ok() {
-  g_last_error[0] = '\0';
-  return SSM_OK;
-}
-
-bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 // Checks shared by both modes. `prefill` selects the dense stride defaults.
 ssm_status check_dims(const ssm_dims* d, bool prefill, ssm::Strides* s) {
@@ -68,6 +63,8 @@ ssm_status check_dims(const ssm_dims* d, bool prefill, ssm::Strides* s) {
   return SSM_OK;
 }
 
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
 ssm_status check_weights(const ssm_weights* w) {
   if (!w) return fail(SSM_ERR_INVALID_ARG, "weights is NULL");
   const float* p[6] = {w->conv_w, w->conv_b, w->w_dt, w->dt_bias, w->A_log, w->D};
@@ -77,6 +74,31 @@ ssm_status check_weights(const ssm_weights* w) {
     const size_t need = (i == 0 || i == 4) ? 16 : 4;  // conv_w and A_log rows are read as 16-byte vectors
     if (!aligned(p[i], need)) return fail(SSM_ERR_INVALID_ARG, "weights.%s is not %zu-byte aligned", names[i], need);
   }
+  return SSM_OK;
+}
+
+ssm_status check_prefill_caches(const void* conv_cache_in, const float* ssm_state_in, const void* conv_cache_out,
+                                const float* ssm_state_out) {
+  if (!conv_cache_out || !aligned(conv_cache_out, 16))
+    return fail(SSM_ERR_INVALID_ARG, "conv_cache_out is NULL or not 16-byte aligned");
+  if (!ssm_state_out || !aligned(ssm_state_out, 16))
+    return fail(SSM_ERR_INVALID_ARG, "ssm_state_out is NULL or not 16-byte aligned");
+  if (conv_cache_in && !aligned(conv_cache_in, 16)) return fail(SSM_ERR_INVALID_ARG, "conv_cache_in not 16-byte aligned");
+  if (ssm_state_in && !aligned(ssm_state_in, 4)) return fail(SSM_ERR_INVALID_ARG, "ssm_state_in not 4-byte aligned");
+  return SSM_OK;
+}
+
+}  // namespace ssm
+
+namespace {
+using ssm::aligned;
+using ssm::check_dims;
+using ssm::check_prefill_caches;
+using ssm::check_weights;
+using ssm::fail;
+
+ssm_status ok() {
+  g_last_error[0] = '\0';
   return SSM_OK;
 }
 
@@ -142,10 +164,7 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
     if ((st = check_io_ptr(dt_raw, "dt_raw", 4)) != SSM_OK) return st;
     if (y == x || y == z) return fail(SSM_ERR_INVALID_ARG, "y must not alias x or z");
   }
-  if ((st = check_io_ptr(conv_cache_out, "conv_cache_out", 16)) != SSM_OK) return st;
-  if ((st = check_io_ptr(ssm_state_out, "ssm_state_out", 16)) != SSM_OK) return st;
-  if (conv_cache_in && !aligned(conv_cache_in, 16)) return fail(SSM_ERR_INVALID_ARG, "conv_cache_in not 16-byte aligned");
-  if (ssm_state_in && !aligned(ssm_state_in, 4)) return fail(SSM_ERR_INVALID_ARG, "ssm_state_in not 4-byte aligned");
+  if ((st = check_prefill_caches(conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out)) != SSM_OK) return st;
   if (workspace_bytes < ssm_prefill_workspace_bytes(dims))
     return fail(SSM_ERR_INVALID_ARG, "workspace too small");
   (void)workspace;

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "ssm.h"
+
 namespace ssm {
 
 // Element strides of every strided tensor (already resolved from the ABI's
@@ -52,5 +54,14 @@ PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t L, int num_s
 bool prefill_shape_supported(PrefillShape sh);
 cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st);
 cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStream_t st);
+
+// Shared by the entry points (ssm_api.cu): validation with the ABI's
+// "0 = dense" stride defaults, and the calling thread's last-error message.
+ssm_status check_dims(const ssm_dims* d, bool prefill, Strides* s);
+ssm_status check_weights(const ssm_weights* w);
+ssm_status check_prefill_caches(const void* conv_cache_in, const float* ssm_state_in, const void* conv_cache_out,
+                                const float* ssm_state_out);
+bool aligned(const void* p, size_t a);
+ssm_status fail(ssm_status st, const char* fmt, ...);
 
 }  // namespace ssm

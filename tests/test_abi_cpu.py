@@ -130,3 +130,55 @@ def test_binding_refuses_cpu_tensors(lib):
          for n in api.PARAM_NAMES}
     with pytest.raises(RuntimeError, match="no CPU path"):
         api.prefill(x, x, torch.zeros(1, 8, 16), torch.zeros(1, 8, 16), torch.zeros(1, 8), p)
+
+
+def test_host_workspace_bytes_cover_two_chunk_slots(lib):
+    def slot(b, T, E, es):
+        al = lambda v: (v + 255) // 256 * 256  # noqa: E731
+        return 3 * al(b * T * E * es) + 2 * al(b * T * 64) + al(b * T * 4)
+
+    d = valid_dims()  # b=2, L=64, E=32, bf16
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 16) == 2 * slot(2, 16, 32, 2)
+    # chunk 0 selects 2048 tokens, clipped to the sequence length
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 0) == 2 * slot(2, 64, 32, 2)
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 1000) == 2 * slot(2, 64, 32, 2)
+    d32 = api.make_dims(1, 5000, 64, torch.float32)
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d32), 0) == 2 * slot(1, 2048, 64, 4)
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), -1) == 0
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(valid_dims(d_state=8)), 16) == 0
+    assert lib.ssm_prefill_host_workspace_bytes(None, 16) == 0
+
+
+def call_prefill_host(lib, dims, weights, ptrs=None, ws_bytes=1 << 20, chunk=16):
+    p = dict(x=FAKE, z=FAKE, B=FAKE, C=FAKE, dt=FAKE, cin=None, sin=None, y=FAKE + 4096, cout=FAKE, sout=FAKE,
+             ws=FAKE)
+    p.update(ptrs or {})
+    return lib.ssm_prefill_host(ctypes.byref(dims) if dims is not None else None,
+                                ctypes.byref(weights) if weights is not None else None, p["x"], p["z"], p["B"], p["C"],
+                                p["dt"], p["cin"], p["sin"], p["y"], p["cout"], p["sout"], p["ws"], ws_bytes, chunk,
+                                None)
+
+
+def test_prefill_host_rejects_bad_arguments_before_any_work(lib):
+    d, w = valid_dims(), fake_weights()
+    assert call_prefill_host(lib, valid_dims(d_state=8), w) == _lib.SSM_ERR_UNSUPPORTED
+    assert call_prefill_host(lib, d, None) == _lib.SSM_ERR_INVALID_ARG
+    assert call_prefill_host(lib, d, w, chunk=-3) == _lib.SSM_ERR_INVALID_ARG
+    assert b"chunk_tokens" in lib.ssm_last_error()
+    for k in ("x", "z", "B", "C", "dt", "y", "cout", "sout", "ws"):
+        assert call_prefill_host(lib, d, w, {k: None}) == _lib.SSM_ERR_INVALID_ARG, k
+        assert b"NULL" in lib.ssm_last_error(), k
+    assert call_prefill_host(lib, d, w, {"y": FAKE}) == _lib.SSM_ERR_INVALID_ARG  # y aliases x
+    assert call_prefill_host(lib, d, w, {"ws": FAKE + 16}) == _lib.SSM_ERR_INVALID_ARG  # not 256-byte aligned
+    need = lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 16)
+    assert call_prefill_host(lib, d, w, ws_bytes=need - 1) == _lib.SSM_ERR_INVALID_ARG
+    assert b"workspace" in lib.ssm_last_error()
+
+
+def test_host_binding_refuses_host_parameters(lib):
+    x = torch.zeros(1, 8, 8, dtype=torch.bfloat16)
+    p = {n: torch.zeros(8, 4) if n == "conv_w" else torch.zeros(8, 16) if n == "A_log" else torch.zeros(8)
+         for n in api.PARAM_NAMES}
+    with pytest.raises(RuntimeError, match="CUDA tensor"):
+        api.prefill_host(x, x, torch.zeros(1, 8, 16), torch.zeros(1, 8, 16), torch.zeros(1, 8), p,
+                         conv_cache_out=torch.zeros(1, 3, 8, dtype=torch.bfloat16))
