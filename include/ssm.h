@@ -196,6 +196,37 @@ ssm_status ssm_prefill_host(const ssm_dims *dims, const ssm_weights *w, const vo
  * for invalid dims. */
 size_t ssm_prefill_host_workspace_bytes(const ssm_dims *dims, int64_t chunk_tokens);
 
+/* Bytes of the device scratch that ssm_prefill_host_static owns: a static
+ * device array of the library, one per device, reserved when the library's
+ * device code is loaded. */
+#define SSM_HOST_STATIC_SCRATCH_BYTES ((size_t)128 << 20)
+
+/*
+ * ssm_prefill_host_static -- ssm_prefill_host without a workspace and without
+ * any allocation. The computation, arguments, result (bit-identical to one
+ * ssm_prefill), ordering with `stream` and host-buffer lifetime are those of
+ * ssm_prefill_host.
+ *
+ * Scratch. The two chunk buffers live in the library's static device scratch
+ * of SSM_HOST_STATIC_SCRATCH_BYTES per device; its address is looked up once
+ * per device. The internal streams and events are created on the first call
+ * on a device and reused by every later call, so steady-state calls create
+ * nothing and allocate no memory.
+ *
+ * Chunk size. chunk_tokens 0 selects the largest chunk of at most 2048 tokens
+ * whose two buffers fit the scratch. A nonzero chunk_tokens whose buffers do
+ * not fit returns SSM_ERR_INVALID_ARG. If not even one token fits
+ * (batch * d_inner too large), the call returns SSM_ERR_UNSUPPORTED.
+ *
+ * Sharing. Calls on one device share the scratch, whatever their streams:
+ * each call's first copy waits until the previous call has finished with it,
+ * so such calls run one after another on the device.
+ */
+ssm_status ssm_prefill_host_static(const ssm_dims *dims, const ssm_weights *w, const void *x, const void *z,
+                                   const float *B, const float *C, const float *dt_raw, const void *conv_cache_in,
+                                   const float *ssm_state_in, void *y, void *conv_cache_out, float *ssm_state_out,
+                                   int64_t chunk_tokens, void *stream);
+
 /*
  * ssm_decode_step -- one-token mode ("Autoregressive decoding", later calls):
  * concatenates conv_cache with the new token, runs the conv for that token and

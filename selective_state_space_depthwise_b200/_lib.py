@@ -17,12 +17,15 @@ SSM_F32, SSM_BF16 = 0, 1
 SSM_DISC_EULER_B, SSM_DISC_ZOH = 0, 1
 
 # Every symbol include/ssm.h declares (checked by the CPU test suite).
+SSM_HOST_STATIC_SCRATCH_BYTES = 128 << 20  # include/ssm.h
+
 EXPORTED = (
     "ssm_prefill",
     "ssm_prefill_ex",
     "ssm_prefill_workspace_bytes",
     "ssm_prefill_host",
     "ssm_prefill_host_workspace_bytes",
+    "ssm_prefill_host_static",
     "ssm_decode_step",
     "ssm_check_device_error",
     "ssm_status_string",
@@ -90,6 +93,8 @@ def load(path: str = LIB_PATH):
     lib.ssm_prefill_workspace_bytes.restype = sz
     lib.ssm_prefill_host.argtypes = [dims_p, w_p] + [p] * 10 + [p, sz, ctypes.c_int64, p]
     lib.ssm_prefill_host.restype = st
+    lib.ssm_prefill_host_static.argtypes = [dims_p, w_p] + [p] * 10 + [ctypes.c_int64, p]
+    lib.ssm_prefill_host_static.restype = st
     lib.ssm_prefill_host_workspace_bytes.argtypes = [dims_p, ctypes.c_int64]
     lib.ssm_prefill_host_workspace_bytes.restype = sz
     lib.ssm_decode_step.argtypes = [dims_p, w_p] + [p] * 8 + [p]

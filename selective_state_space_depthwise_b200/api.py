@@ -130,12 +130,15 @@ def host_workspace_bytes(batch, seqlen, E, io_dtype=torch.bfloat16, chunk_tokens
 
 def prefill_host(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None, y=None, conv_cache_out=None,
                  ssm_state_out=None, dt_min=1e-4, dt_max=1.0, discretization="euler", chunk_tokens=0, workspace=None,
-                 stream=None):
+                 stream=None, static_scratch=False):
     """Full-sequence block core with the token tensors in host memory
     (ssm_prefill_host): x, z, B, C, dt_raw and y are CPU tensors (pinned for
     overlapped copies), shaped and strided as for `prefill`; the parameters and
     the caches are CUDA tensors on the current device. The copies and kernels
-    are only enqueued: synchronise `stream` before reading y.
+    are only enqueued: synchronise `stream` before reading y. With
+    static_scratch=True the call goes to ssm_prefill_host_static, which takes
+    no workspace and allocates nothing (its chunk buffers are the library's
+    static device scratch).
     Returns (y [b, L, E] on the host, conv_cache_out, ssm_state_out)."""
     lib = _lib.load()
     b, L, E = x.shape
@@ -167,6 +170,12 @@ def prefill_host(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in
                      z_seq_stride=z.stride(0), y_tok_stride=y.stride(1), y_seq_stride=y.stride(0),
                      bc_tok_stride=B.stride(1), bc_seq_stride=B.stride(0), dt_seq_stride=dt_raw.stride(0))
     w = _weights(params, E, dev)
+    if static_scratch:
+        st = lib.ssm_prefill_host_static(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C),
+                                         _ptr(dt_raw), _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(y),
+                                         _ptr(conv_cache_out), _ptr(ssm_state_out), int(chunk_tokens), _stream(stream))
+        _lib.check(st)
+        return y, conv_cache_out, ssm_state_out
     ws = int(lib.ssm_prefill_host_workspace_bytes(ctypes.byref(dims), int(chunk_tokens)))
     if workspace is None or workspace.numel() < ws:
         workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)

@@ -1,5 +1,7 @@
-// stream_prefill.cu -- ssm_prefill_host: prefill from and to host memory with
-// the copies overlapped (host code only; the kernels are prefill.cu's).
+// stream_prefill.cu -- ssm_prefill_host and ssm_prefill_host_static: prefill
+// from and to host memory with the copies overlapped (host code, plus the
+// static device scratch of the second entry point; the kernels are
+// prefill.cu's).
 //
 // The sequence is cut into chunks of T tokens and pipelined over three streams:
 //   copy-in  (internal):  H2D of chunk c's x, z, B, C, dt_raw into slot c % 2;
@@ -15,6 +17,13 @@
 // the caller's stream waits for the last copy-out. Because chunked prefill
 // with carried caches runs the same arithmetic in the same order per token,
 // the result is bit-identical to one launch over the whole sequence.
+//
+// ssm_prefill_host takes the two chunk slots from a caller-owned workspace and
+// creates its events per call. ssm_prefill_host_static allocates nothing: its
+// slots live in a file-scope static device array (one per device, address
+// taken with cudaGetSymbolAddress once per device), and its events, like the
+// internal streams, are created on the first call per device and reused.
+// Successive static calls are ordered on that scratch by a per-device event.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -26,15 +35,17 @@ namespace {
 
 constexpr int64_t kDefaultChunk = 2048;
 constexpr size_t kAlign = 256;
+constexpr size_t kStaticScratchBytes = SSM_HOST_STATIC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+// Chunk buffers of ssm_prefill_host_static, one copy per device.
+static __device__ __align__(256) unsigned char g_host_prefill_scratch[kStaticScratchBytes];
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
-int64_t chunk_of(int64_t chunk_tokens, int64_t L) {
-  const int64_t T = chunk_tokens > 0 ? chunk_tokens : kDefaultChunk;
-  return L > 0 && T > L ? L : T;
-}
+int64_t clip_chunk(int64_t T, int64_t L) { return L > 0 && T > L ? L : T; }
 
-// Byte layout of one chunk slot in the workspace (dense [b][T][...] buffers).
+// Byte layout of one chunk slot (dense [b][T][...] buffers).
 struct SlotLayout {
   size_t x, z, y, B, C, dt, bytes;
 };
@@ -52,22 +63,64 @@ SlotLayout slot_layout(int64_t b, int64_t T, int64_t E, size_t es) {
   return s;
 }
 
-// Per-device internal streams, created on first use.
-struct DeviceStreams {
-  cudaStream_t in = nullptr, out = nullptr;
+size_t io_size(const ssm_dims* d) { return d->io_dtype == SSM_BF16 ? 2 : 4; }
+
+// Pipeline events: start (on the caller's stream), per slot: inputs ready,
+// kernel done, copy-out done; end (on the copy-in stream).
+struct PipelineEvents {
+  cudaEvent_t start = nullptr, in[2] = {}, comp[2] = {}, out[2] = {}, end = nullptr;
+  cudaEvent_t* all[8] = {&start, &in[0], &in[1], &comp[0], &comp[1], &out[0], &out[1], &end};
+};
+
+cudaError_t create_events(PipelineEvents* ev) {
+  for (cudaEvent_t* e : ev->all) {
+    const cudaError_t r = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+    if (r != cudaSuccess) return r;
+  }
+  return cudaSuccess;
+}
+
+// Destroying a recorded event that has not completed is legal: its resources
+// are released when it completes.
+void destroy_events(PipelineEvents* ev) {
+  for (cudaEvent_t* e : ev->all)
+    if (*e) cudaEventDestroy(*e), *e = nullptr;
+}
+
+// Per-device state, created on first use and kept for the process.
+struct DeviceState {
+  cudaStream_t in = nullptr, out = nullptr;  // internal copy streams
+  bool static_ready = false;                 // the static entry point's members below are set
+  PipelineEvents static_ev;
+  cudaEvent_t scratch_free = nullptr;  // recorded when a static call has finished with the scratch
+  char* scratch = nullptr;             // device address of g_host_prefill_scratch
 };
 std::mutex g_mutex;  // guards the table and serialises enqueueing
-DeviceStreams g_streams[64];
+DeviceState g_dev[kMaxDevices];
 
-cudaError_t streams_for_current_device(DeviceStreams** ds) {
+cudaError_t device_state(DeviceState** out, bool with_static) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  DeviceStreams& d = g_streams[dev];
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceState& d = g_dev[dev];
   if (!d.in && (e = cudaStreamCreateWithFlags(&d.in, cudaStreamNonBlocking)) != cudaSuccess) return e;
   if (!d.out && (e = cudaStreamCreateWithFlags(&d.out, cudaStreamNonBlocking)) != cudaSuccess) return e;
-  *ds = &d;
+  if (with_static && !d.static_ready) {
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_host_prefill_scratch)) != cudaSuccess) return e;
+    if ((e = create_events(&d.static_ev)) != cudaSuccess) {
+      destroy_events(&d.static_ev);
+      return e;
+    }
+    if ((e = cudaEventCreateWithFlags(&d.scratch_free, cudaEventDisableTiming)) != cudaSuccess) {
+      destroy_events(&d.static_ev);
+      return e;
+    }
+    d.scratch = static_cast<char*>(p);
+    d.static_ready = true;
+  }
+  *out = &d;
   return cudaSuccess;
 }
 
@@ -90,48 +143,48 @@ cudaError_t copy_rows(char* dst, size_t dst_row, size_t dst_seq, const char* src
   return cudaSuccess;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t ssm_prefill_host_workspace_bytes(const ssm_dims* dims, int64_t chunk_tokens) {
+// The arguments of one host prefill, validated.
+struct HostPrefill {
+  const ssm_dims* dims;
+  const ssm_weights* w;
+  const void *x, *z;
+  const float *B, *C, *dt;
+  const void* cin;
+  const float* sin;
+  void* y;
+  void* cout;
+  float* sout;
   ssm::Strides s;
-  if (chunk_tokens < 0 || ssm::check_dims(dims, true, &s) != SSM_OK) return 0;
-  const int64_t T = chunk_of(chunk_tokens, dims->seqlen);
-  const size_t es = dims->io_dtype == SSM_BF16 ? 2 : 4;
-  return 2 * slot_layout(dims->batch, T, dims->d_inner, es).bytes;
-}
+};
 
-ssm_status ssm_prefill_host(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
-                            const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
-                            void* y, void* conv_cache_out, float* ssm_state_out, void* workspace,
-                            size_t workspace_bytes, int64_t chunk_tokens, void* stream) {
-  ssm::Strides s;
-  ssm_status st = ssm::check_dims(dims, true, &s);
+// Checks shared by both entry points, all before any CUDA call.
+ssm_status validate(HostPrefill& hp, int64_t chunk_tokens) {
+  ssm_status st = ssm::check_dims(hp.dims, true, &hp.s);
   if (st != SSM_OK) return st;
   if (chunk_tokens < 0) return ssm::fail(SSM_ERR_INVALID_ARG, "chunk_tokens=%lld must be >= 0", (long long)chunk_tokens);
-  if ((st = ssm::check_weights(w)) != SSM_OK) return st;
-  if ((st = ssm::check_prefill_caches(conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out)) != SSM_OK) return st;
-  const int64_t b = dims->batch, L = dims->seqlen, E = dims->d_inner;
-  if (L == 0)  // nothing to stream: the caches-only path of ssm_prefill
-    return ssm_prefill(dims, w, nullptr, nullptr, nullptr, nullptr, nullptr, conv_cache_in, ssm_state_in, nullptr,
-                       conv_cache_out, ssm_state_out, nullptr, 0, stream);
-  const void* host_in[5] = {x, z, B, C, dt_raw};
+  if ((st = ssm::check_weights(hp.w)) != SSM_OK) return st;
+  if ((st = ssm::check_prefill_caches(hp.cin, hp.sin, hp.cout, hp.sout)) != SSM_OK) return st;
+  if (hp.dims->seqlen == 0) return SSM_OK;  // the token tensors are not read
+  const void* host_in[5] = {hp.x, hp.z, hp.B, hp.C, hp.dt};
   const char* names[5] = {"x", "z", "B", "C", "dt_raw"};
   for (int i = 0; i < 5; ++i)
     if (!host_in[i]) return ssm::fail(SSM_ERR_INVALID_ARG, "%s is NULL", names[i]);
-  if (!y) return ssm::fail(SSM_ERR_INVALID_ARG, "y is NULL");
-  if (y == x || y == z) return ssm::fail(SSM_ERR_INVALID_ARG, "y must not alias x or z");
-  if (!workspace || !ssm::aligned(workspace, kAlign))
-    return ssm::fail(SSM_ERR_INVALID_ARG, "workspace is NULL or not %zu-byte aligned", kAlign);
-  const size_t need = ssm_prefill_host_workspace_bytes(dims, chunk_tokens);
-  if (workspace_bytes < need)
-    return ssm::fail(SSM_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  if (!hp.y) return ssm::fail(SSM_ERR_INVALID_ARG, "y is NULL");
+  if (hp.y == hp.x || hp.y == hp.z) return ssm::fail(SSM_ERR_INVALID_ARG, "y must not alias x or z");
+  return SSM_OK;
+}
 
-  const int64_t T = chunk_of(chunk_tokens, L);
-  const size_t es = dims->io_dtype == SSM_BF16 ? 2 : 4;
+// Enqueues the chunk pipeline. `after` (may be NULL) is an event the first
+// copy also waits for. On return the caller's stream waits for every copy
+// and kernel enqueued here, on success and on failure.
+ssm_status enqueue(const HostPrefill& hp, char* ws, int64_t T, cudaStream_t cs, DeviceState* ds,
+                   const PipelineEvents& ev, cudaEvent_t after) {
+  const ssm_dims* dims = hp.dims;
+  const ssm::Strides& s = hp.s;
+  const int64_t b = dims->batch, L = dims->seqlen, E = dims->d_inner;
+  const size_t es = io_size(dims);
   const SlotLayout lay = slot_layout(b, T, E, es);
-  char* slot_base[2] = {static_cast<char*>(workspace), static_cast<char*>(workspace) + lay.bytes};
+  char* slot_base[2] = {ws, ws + lay.bytes};
 
   // Chunk dims: dense device buffers, sequence pitch T tokens.
   ssm_dims cd = *dims;
@@ -141,87 +194,66 @@ ssm_status ssm_prefill_host(const ssm_dims* dims, const ssm_weights* w, const vo
   cd.bc_seq_stride = T * 16;
   cd.dt_seq_stride = T;
 
-  std::lock_guard<std::mutex> lock(g_mutex);
-  DeviceStreams* ds = nullptr;
-  cudaError_t e = streams_for_current_device(&ds);
-  if (e != cudaSuccess) return ssm::fail(SSM_ERR_CUDA, "internal streams: %s", cudaGetErrorString(e));
-  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-
-  // Events: start (on the caller's stream), per slot: inputs ready, kernel
-  // done, copy-out done. Destroying a recorded event that has not completed
-  // is legal; its resources are released when it completes.
-  cudaEvent_t ev_start, ev_in[2], ev_comp[2], ev_out[2];
-  cudaEvent_t* all[7] = {&ev_start, &ev_in[0], &ev_in[1], &ev_comp[0], &ev_comp[1], &ev_out[0], &ev_out[1]};
-  int created = 0;
-  for (; created < 7; ++created)
-    if ((e = cudaEventCreateWithFlags(all[created], cudaEventDisableTiming)) != cudaSuccess) break;
-  auto destroy_events = [&]() {
-    for (int i = 0; i < created; ++i) cudaEventDestroy(*all[i]);
-  };
-  if (e != cudaSuccess) {
-    destroy_events();
-    return ssm::fail(SSM_ERR_CUDA, "events: %s", cudaGetErrorString(e));
-  }
-
   const int64_t n_chunks = (L + T - 1) / T;
   ssm_status result = SSM_OK;
-  int64_t last_out = -1;  // index of the last chunk whose copy-out was enqueued
-  auto cuda_fail = [&](const char* what) {
-    result = ssm::fail(SSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
-  };
+  cudaError_t e = cudaSuccess;
+  int64_t last_out = -1;  // the last chunk whose copy-out was enqueued
+  auto cuda_fail = [&](const char* what) { result = ssm::fail(SSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e)); };
   do {
-    if ((e = cudaEventRecord(ev_start, cs)) != cudaSuccess) { cuda_fail("record"); break; }
-    if ((e = cudaStreamWaitEvent(ds->in, ev_start, 0)) != cudaSuccess) { cuda_fail("wait"); break; }
-    if ((e = cudaStreamWaitEvent(ds->out, ev_start, 0)) != cudaSuccess) { cuda_fail("wait"); break; }
-    for (int64_t c = 0; c < n_chunks && result == SSM_OK; ++c) {
+    if ((e = cudaEventRecord(ev.start, cs)) != cudaSuccess || (e = cudaStreamWaitEvent(ds->in, ev.start, 0)) ||
+        (e = cudaStreamWaitEvent(ds->out, ev.start, 0)) || (after && (e = cudaStreamWaitEvent(ds->in, after, 0)))) {
+      cuda_fail("start");
+      break;
+    }
+    for (int64_t c = 0; c < n_chunks; ++c) {
       const int k = static_cast<int>(c & 1);
       const int64_t t0 = c * T, Tc = (L - t0 < T) ? L - t0 : T;
       char* base = slot_base[k];
       // copy-in of chunk c (slot k was last read by the kernel of chunk c - 2)
-      if (c >= 2 && (e = cudaStreamWaitEvent(ds->in, ev_comp[k], 0)) != cudaSuccess) { cuda_fail("wait"); break; }
-      const char* hx = static_cast<const char*>(x) + static_cast<size_t>(t0 * s.x_tok) * es;
-      const char* hz = static_cast<const char*>(z) + static_cast<size_t>(t0 * s.z_tok) * es;
-      const char* hB = reinterpret_cast<const char*>(B + t0 * s.bc_tok);
-      const char* hC = reinterpret_cast<const char*>(C + t0 * s.bc_tok);
-      const char* hd = reinterpret_cast<const char*>(dt_raw + t0);
+      if (c >= 2 && (e = cudaStreamWaitEvent(ds->in, ev.comp[k], 0)) != cudaSuccess) {
+        cuda_fail("wait");
+        break;
+      }
+      const char* hx = static_cast<const char*>(hp.x) + static_cast<size_t>(t0 * s.x_tok) * es;
+      const char* hz = static_cast<const char*>(hp.z) + static_cast<size_t>(t0 * s.z_tok) * es;
+      const char* hB = reinterpret_cast<const char*>(hp.B + t0 * s.bc_tok);
+      const char* hC = reinterpret_cast<const char*>(hp.C + t0 * s.bc_tok);
+      const char* hd = reinterpret_cast<const char*>(hp.dt + t0);
       const size_t row = static_cast<size_t>(E) * es, dseq = static_cast<size_t>(T * E) * es;
-      if ((e = copy_rows(base + lay.x, row, dseq, hx, s.x_tok * es, s.x_seq * es, row, Tc, b, cudaMemcpyHostToDevice,
-                         ds->in)) != cudaSuccess ||
-          (e = copy_rows(base + lay.z, row, dseq, hz, s.z_tok * es, s.z_seq * es, row, Tc, b, cudaMemcpyHostToDevice,
-                         ds->in)) != cudaSuccess ||
-          (e = copy_rows(base + lay.B, 64, T * 64, hB, s.bc_tok * 4, s.bc_seq * 4, 64, Tc, b, cudaMemcpyHostToDevice,
-                         ds->in)) != cudaSuccess ||
-          (e = copy_rows(base + lay.C, 64, T * 64, hC, s.bc_tok * 4, s.bc_seq * 4, 64, Tc, b, cudaMemcpyHostToDevice,
-                         ds->in)) != cudaSuccess ||
-          (e = copy_rows(base + lay.dt, 4, T * 4, hd, 4, s.dt_seq * 4, 4, Tc, b, cudaMemcpyHostToDevice, ds->in)) !=
-              cudaSuccess ||
-          (e = cudaEventRecord(ev_in[k], ds->in)) != cudaSuccess) {
+      const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+      if ((e = copy_rows(base + lay.x, row, dseq, hx, s.x_tok * es, s.x_seq * es, row, Tc, b, h2d, ds->in)) ||
+          (e = copy_rows(base + lay.z, row, dseq, hz, s.z_tok * es, s.z_seq * es, row, Tc, b, h2d, ds->in)) ||
+          (e = copy_rows(base + lay.B, 64, T * 64, hB, s.bc_tok * 4, s.bc_seq * 4, 64, Tc, b, h2d, ds->in)) ||
+          (e = copy_rows(base + lay.C, 64, T * 64, hC, s.bc_tok * 4, s.bc_seq * 4, 64, Tc, b, h2d, ds->in)) ||
+          (e = copy_rows(base + lay.dt, 4, T * 4, hd, 4, s.dt_seq * 4, 4, Tc, b, h2d, ds->in)) ||
+          (e = cudaEventRecord(ev.in[k], ds->in))) {
         cuda_fail("copy-in");
         break;
       }
       // kernel of chunk c (y slot k was last read by the copy-out of chunk c - 2)
-      if ((e = cudaStreamWaitEvent(cs, ev_in[k], 0)) != cudaSuccess ||
-          (c >= 2 && (e = cudaStreamWaitEvent(cs, ev_out[k], 0)) != cudaSuccess)) {
+      if ((e = cudaStreamWaitEvent(cs, ev.in[k], 0)) || (c >= 2 && (e = cudaStreamWaitEvent(cs, ev.out[k], 0)))) {
         cuda_fail("wait");
         break;
       }
       cd.seqlen = Tc;
       const ssm_status ks = ssm_prefill(
-          &cd, w, base + lay.x, base + lay.z, reinterpret_cast<const float*>(base + lay.B),
+          &cd, hp.w, base + lay.x, base + lay.z, reinterpret_cast<const float*>(base + lay.B),
           reinterpret_cast<const float*>(base + lay.C), reinterpret_cast<const float*>(base + lay.dt),
-          c == 0 ? conv_cache_in : conv_cache_out, c == 0 ? ssm_state_in : ssm_state_out, base + lay.y,
-          conv_cache_out, ssm_state_out, nullptr, 0, stream);
+          c == 0 ? hp.cin : hp.cout, c == 0 ? hp.sin : hp.sout, base + lay.y, hp.cout, hp.sout, nullptr, 0, cs);
       if (ks != SSM_OK) {
         result = ks;  // ssm_prefill has set the message
         break;
       }
-      if ((e = cudaEventRecord(ev_comp[k], cs)) != cudaSuccess) { cuda_fail("record"); break; }
+      if ((e = cudaEventRecord(ev.comp[k], cs)) != cudaSuccess) {
+        cuda_fail("record");
+        break;
+      }
       // copy-out of chunk c
-      char* hy = static_cast<char*>(y) + static_cast<size_t>(t0 * s.y_tok) * es;
-      if ((e = cudaStreamWaitEvent(ds->out, ev_comp[k], 0)) != cudaSuccess ||
-          (e = copy_rows(hy, s.y_tok * es, s.y_seq * es, base + lay.y, row, dseq, row, Tc, b,
-                         cudaMemcpyDeviceToHost, ds->out)) != cudaSuccess ||
-          (e = cudaEventRecord(ev_out[k], ds->out)) != cudaSuccess) {
+      char* hy = static_cast<char*>(hp.y) + static_cast<size_t>(t0 * s.y_tok) * es;
+      if ((e = cudaStreamWaitEvent(ds->out, ev.comp[k], 0)) ||
+          (e = copy_rows(hy, s.y_tok * es, s.y_seq * es, base + lay.y, row, dseq, row, Tc, b, cudaMemcpyDeviceToHost,
+                         ds->out)) ||
+          (e = cudaEventRecord(ev.out[k], ds->out))) {
         cuda_fail("copy-out");
         break;
       }
@@ -229,15 +261,99 @@ ssm_status ssm_prefill_host(const ssm_dims* dims, const ssm_weights* w, const vo
     }
   } while (false);
   // The caller's stream waits for everything enqueued, on success and on failure.
-  if (last_out >= 0) cudaStreamWaitEvent(cs, ev_out[last_out & 1], 0);
-  cudaEvent_t ev_end;
-  if (cudaEventCreateWithFlags(&ev_end, cudaEventDisableTiming) == cudaSuccess) {
-    if (cudaEventRecord(ev_end, ds->in) == cudaSuccess) cudaStreamWaitEvent(cs, ev_end, 0);
-    cudaEventDestroy(ev_end);
-  }
-  destroy_events();
+  if (last_out >= 0) cudaStreamWaitEvent(cs, ev.out[last_out & 1], 0);
+  if (cudaEventRecord(ev.end, ds->in) == cudaSuccess) cudaStreamWaitEvent(cs, ev.end, 0);
   if (result == SSM_OK) ssm::fail(SSM_OK, "");
   return result;
+}
+
+// Largest chunk (at most kDefaultChunk tokens, at most L) whose two slots fit
+// `bytes`; 0 if not even one token fits.
+int64_t largest_fitting_chunk(const ssm_dims* d, size_t bytes) {
+  const size_t es = io_size(d);
+  const int64_t b = d->batch, E = d->d_inner;
+  const size_t per_token = 2 * static_cast<size_t>(b) * (3 * static_cast<size_t>(E) * es + 2 * 64 + 4);
+  int64_t T = clip_chunk(kDefaultChunk, d->seqlen);
+  const int64_t est = static_cast<int64_t>(bytes / per_token);
+  if (est < T) T = est;
+  while (T > 0 && 2 * slot_layout(b, T, E, es).bytes > bytes) --T;
+  return T;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssm_prefill_host_workspace_bytes(const ssm_dims* dims, int64_t chunk_tokens) {
+  ssm::Strides s;
+  if (chunk_tokens < 0 || ssm::check_dims(dims, true, &s) != SSM_OK) return 0;
+  const int64_t T = clip_chunk(chunk_tokens > 0 ? chunk_tokens : kDefaultChunk, dims->seqlen);
+  return 2 * slot_layout(dims->batch, T, dims->d_inner, io_size(dims)).bytes;
+}
+
+ssm_status ssm_prefill_host(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                            const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
+                            void* y, void* conv_cache_out, float* ssm_state_out, void* workspace,
+                            size_t workspace_bytes, int64_t chunk_tokens, void* stream) {
+  HostPrefill hp{dims, w, x, z, B, C, dt_raw, conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out, {}};
+  ssm_status st = validate(hp, chunk_tokens);
+  if (st != SSM_OK) return st;
+  if (dims->seqlen == 0)  // nothing to stream: the caches-only path of ssm_prefill
+    return ssm_prefill(dims, w, nullptr, nullptr, nullptr, nullptr, nullptr, conv_cache_in, ssm_state_in, nullptr,
+                       conv_cache_out, ssm_state_out, nullptr, 0, stream);
+  if (!workspace || !ssm::aligned(workspace, kAlign))
+    return ssm::fail(SSM_ERR_INVALID_ARG, "workspace is NULL or not %zu-byte aligned", kAlign);
+  const size_t need = ssm_prefill_host_workspace_bytes(dims, chunk_tokens);
+  if (workspace_bytes < need)
+    return ssm::fail(SSM_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  const int64_t T = clip_chunk(chunk_tokens > 0 ? chunk_tokens : kDefaultChunk, dims->seqlen);
+
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState* ds = nullptr;
+  cudaError_t e = device_state(&ds, false);
+  if (e != cudaSuccess) return ssm::fail(SSM_ERR_CUDA, "internal streams: %s", cudaGetErrorString(e));
+  PipelineEvents ev;
+  if ((e = create_events(&ev)) != cudaSuccess) {
+    destroy_events(&ev);
+    return ssm::fail(SSM_ERR_CUDA, "events: %s", cudaGetErrorString(e));
+  }
+  st = enqueue(hp, static_cast<char*>(workspace), T, static_cast<cudaStream_t>(stream), ds, ev, nullptr);
+  destroy_events(&ev);
+  return st;
+}
+
+ssm_status ssm_prefill_host_static(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z,
+                                   const float* B, const float* C, const float* dt_raw, const void* conv_cache_in,
+                                   const float* ssm_state_in, void* y, void* conv_cache_out, float* ssm_state_out,
+                                   int64_t chunk_tokens, void* stream) {
+  HostPrefill hp{dims, w, x, z, B, C, dt_raw, conv_cache_in, ssm_state_in, y, conv_cache_out, ssm_state_out, {}};
+  ssm_status st = validate(hp, chunk_tokens);
+  if (st != SSM_OK) return st;
+  if (dims->seqlen == 0)
+    return ssm_prefill(dims, w, nullptr, nullptr, nullptr, nullptr, nullptr, conv_cache_in, ssm_state_in, nullptr,
+                       conv_cache_out, ssm_state_out, nullptr, 0, stream);
+  int64_t T = 0;
+  if (chunk_tokens > 0) {
+    T = clip_chunk(chunk_tokens, dims->seqlen);
+    if (2 * slot_layout(dims->batch, T, dims->d_inner, io_size(dims)).bytes > kStaticScratchBytes)
+      return ssm::fail(SSM_ERR_INVALID_ARG, "chunk of %lld tokens does not fit the %zu-byte static scratch",
+                       (long long)T, kStaticScratchBytes);
+  } else if ((T = largest_fitting_chunk(dims, kStaticScratchBytes)) == 0) {
+    return ssm::fail(SSM_ERR_UNSUPPORTED, "batch * d_inner too large for the %zu-byte static scratch",
+                     kStaticScratchBytes);
+  }
+
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState* ds = nullptr;
+  cudaError_t e = device_state(&ds, true);
+  if (e != cudaSuccess) return ssm::fail(SSM_ERR_CUDA, "static scratch / streams / events: %s", cudaGetErrorString(e));
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // The first copy waits until the previous static call on this device (on
+  // any stream) has finished with the scratch; this call marks its own end.
+  st = enqueue(hp, ds->scratch, T, cs, ds, ds->static_ev, ds->scratch_free);
+  if ((e = cudaEventRecord(ds->scratch_free, cs)) != cudaSuccess && st == SSM_OK)
+    st = ssm::fail(SSM_ERR_CUDA, "record: %s", cudaGetErrorString(e));
+  return st;
 }
 
 }  // extern "C"
