@@ -282,7 +282,8 @@ def e2e_prefill(w: W.Workload, inp, steps):
 
 def decode_bench(w: W.Workload, rank: int, hbm_peak: float, peak_kind: str):
     """Prompt prefill (untimed), then the workload's one-token steps, each a
-    separate C call; per-step device time from CUDA events."""
+    separate C call; per-step device time from CUDA events. The same loop
+    replayed from a CUDA graph is reported beside it (graph_us_per_step)."""
     from selective_state_space_depthwise_b200 import api
 
     inp = make_device_inputs(w, rank)
@@ -309,11 +310,32 @@ def decode_bench(w: W.Workload, rank: int, hbm_peak: float, peak_kind: str):
     ev1.record(stream)
     torch.cuda.synchronize()
     us = ev0.elapsed_time(ev1) * 1e3 / steps
+    # The same steps captured once in a CUDA graph and replayed: no host work between launches.
+    graph = torch.cuda.CUDAGraph()
+    cc.copy_(cc0)
+    st.copy_(st0)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        for t in range(L0, L0 + steps):
+            step(t)
+    cc.copy_(cc0)
+    st.copy_(st0)
+    graph.replay()  # warm
+    cc.copy_(cc0)
+    st.copy_(st0)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    graph.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    graph_us = ev0.elapsed_time(ev1) * 1e3 / steps
+    del graph
     ct = w.batch * w.d_inner
     gbs = min_bytes_decode_step(w) / (us * 1e-6) / 1e9
     return {"workload": f"decode b={w.batch} E={w.d_inner} N=16 K=4 bf16 x/z/y, fp32 state; prompt {L0}, "
                         f"{steps} one-token steps",
-            "us_per_step": round(us, 2), "value": ct / (us * 1e-6), "unit": "channel-tokens/s",
+            "us_per_step": round(us, 2), "graph_us_per_step": round(graph_us, 2),
+            "value": ct / (us * 1e-6), "unit": "channel-tokens/s",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(gbs / hbm_peak, 4), "peak_kind": peak_kind,
                          "traffic": ncu_traffic("decode", "decode"),

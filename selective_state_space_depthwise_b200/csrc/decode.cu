@@ -65,6 +65,10 @@ struct ChannelParams {
 
 // Rows of the staged per-sequence inputs: B (16), C (16), dt_raw (1), padding.
 constexpr int kStageSeqs = 32;
+#ifndef SSM_DECODE_SETS
+#define SSM_DECODE_SETS 2
+#endif
+constexpr int kSets = SSM_DECODE_SETS;  // register sets of the sequence prefetch
 constexpr int kRow = 36;
 
 template <typename T, bool ZOH>
@@ -152,26 +156,31 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_resident_kernel(const K
   const int64_t stride = gridDim.y, s0 = blockIdx.y;
   const int64_t n = (a.batch - s0 + stride - 1) / stride;
   auto seq_of = [&](int64_t k) { return s0 + k * stride; };
-  DecodeItem A, B;
-  if (active && n > 0) decode_load<T>(a, seq_of(0), e, A);
-  for (int64_t k = 0; k < n; k += 2) {
-    if (k % kStageSeqs == 0) {  // refill the staged rows (kStageSeqs is even, so k is a multiple here)
-      __syncthreads();
-      const int nk = static_cast<int>(n - k < kStageSeqs ? n - k : kStageSeqs);
-      for (int i = threadIdx.x; i < nk * 33; i += kDecodeThreads) {
-        const int r = i / 33, j = i - r * 33;
-        const int64_t sq = seq_of(k + r);
-        rows[r][j] = j < 16 ? a.B[sq * a.s.bc_seq + j]
-                            : (j < 32 ? a.C[sq * a.s.bc_seq + j - 16] : a.dt_raw[sq * a.s.dt_seq]);
+  // kSets register sets in turn: sequence k + kSets - 1 is loaded while k runs.
+  DecodeItem it[kSets];
+#pragma unroll
+  for (int d = 0; d < kSets - 1; ++d)
+    if (active && d < n) decode_load<T>(a, seq_of(d), e, it[d]);
+  for (int64_t k = 0; k < n; k += kSets) {
+#pragma unroll
+    for (int d = 0; d < kSets; ++d) {
+      const int64_t kk = k + d;
+      if (kk >= n) break;  // block-uniform
+      if (kk % kStageSeqs == 0) {  // refill the staged rows
+        __syncthreads();
+        const int nk = static_cast<int>(n - kk < kStageSeqs ? n - kk : kStageSeqs);
+        for (int i = threadIdx.x; i < nk * 33; i += kDecodeThreads) {
+          const int r = i / 33, j = i - r * 33;
+          const int64_t sq = seq_of(kk + r);
+          rows[r][j] = j < 16 ? a.B[sq * a.s.bc_seq + j]
+                              : (j < 32 ? a.C[sq * a.s.bc_seq + j - 16] : a.dt_raw[sq * a.s.dt_seq]);
+        }
+        __syncthreads();
       }
-      __syncthreads();
+      const int64_t pf = kk + kSets - 1;
+      if (active && pf < n) decode_load<T>(a, seq_of(pf), e, it[(d + kSets - 1) % kSets]);
+      if (active) decode_step_item<T, ZOH>(a, seq_of(kk), e, p, rows[kk % kStageSeqs], it[d]);
     }
-    const int r = static_cast<int>(k % kStageSeqs);
-    if (active && k + 1 < n) decode_load<T>(a, seq_of(k + 1), e, B);
-    if (active) decode_step_item<T, ZOH>(a, seq_of(k), e, p, rows[r], A);
-    if (k + 1 >= n) break;
-    if (active && k + 2 < n) decode_load<T>(a, seq_of(k + 2), e, A);
-    if (active) decode_step_item<T, ZOH>(a, seq_of(k + 1), e, p, rows[r + 1], B);
   }
 }
 

@@ -129,18 +129,3 @@ def make_inputs(w: Workload, device="cpu", gen_device=None) -> dict:
     p.update(a)
     return p
 
-
-def sample_channels(w: Workload, n: int, seed: int = 1234) -> list:
-    """A seeded sample of (batch, channel) pairs for full-size parity checks:
-    the first and last channel of the first and last sequence, channels at the
-    edges of 8-wide groups, and the rest uniform."""
-    g = torch.Generator(device="cpu").manual_seed(seed + w.seed)
-    b, E = w.batch, w.d_inner
-    fixed = [(0, 0), (0, E - 1), (b - 1, 0), (b - 1, E - 1), (0, 7), (0, 8), (b - 1, E // 2)]
-    picks = list(dict.fromkeys(fixed))
-    while len(picks) < n:
-        bb = int(torch.randint(0, b, (1,), generator=g))
-        ee = int(torch.randint(0, E, (1,), generator=g))
-        if (bb, ee) not in picks:
-            picks.append((bb, ee))
-    return picks[:n]

@@ -72,3 +72,47 @@ def compare(io_dtype, got, want, label=""):
     assert e_h <= TOL[io_dtype], f"{label}: state rel-L2 {e_h:.3e} > {TOL[io_dtype]:.0e}"
     assert np.isfinite(ys).all() and np.isfinite(hs).all(), f"{label}: non-finite output"
     return e_y, e_h
+
+
+def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_max=1.0, max_elems=1 << 25):
+    """Every (sequence, channel) of a run against the oracle. The channels go
+    in blocks (whole sequences, or channel ranges of one long sequence) of at
+    most about `max_elems` tokens x channels, so full-size workloads fit in
+    host memory; the relative L2 of y and of the state is accumulated over the
+    whole run and the conv cache must match bit for bit. Returns (e_y, e_h)."""
+    y, cache, state = got
+    x, z = inp["x"], inp["z"]
+    b, L, E = x.shape
+    p = {k: inp[k].detach().to("cpu").double().numpy() for k in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")}
+    per_seq = L * E
+    seqs_per_block = max(1, max_elems // max(per_seq, 1))
+    ch_per_block = E if seqs_per_block > 1 or per_seq <= max_elems else max(1, max_elems // max(L, 1))
+    acc = np.zeros(4)  # |dy|^2, |y|^2, |dh|^2, |h|^2
+    for s0 in range(0, b, seqs_per_block):
+        s1 = min(b, s0 + seqs_per_block)
+        Bn = inp["B"][s0:s1].detach().to("cpu").double().numpy()
+        Cn = inp["C"][s0:s1].detach().to("cpu").double().numpy()
+        dtn = inp["dt_raw"][s0:s1].detach().to("cpu").double().numpy()
+        for e0 in range(0, E, ch_per_block):
+            e1 = min(E, e0 + ch_per_block)
+            n_e = e1 - e0
+            # (seq, channel) rows, channel fastest
+            xs = x[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, L).double().cpu().numpy()
+            zs = z[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, L).double().cpu().numpy()
+            bidx = np.repeat(np.arange(s1 - s0), n_e).tolist()
+            tile = lambda a: np.tile(a[e0:e1], (s1 - s0,) + (1,) * (a.ndim - 1))  # noqa: E731
+            out_o, h_o, c_o = oracle.channels(xs, zs, Bn, Cn, dtn, bidx, tile(p["conv_w"]), tile(p["conv_b"]),
+                                              tile(p["w_dt"]), tile(p["dt_bias"]), tile(p["A_log"]), tile(p["D"]),
+                                              lo=dt_min, hi=dt_max, disc=disc)
+            ys = y[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, L).double().cpu().numpy()
+            hs = state[s0:s1, e0:e1, :].reshape(-1, 16).double().cpu().numpy()
+            cs = cache[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, 3).double().cpu().numpy()
+            assert np.array_equal(cs, c_o), f"{label}: conv_cache differs in sequences {s0}..{s1 - 1}"
+            assert np.isfinite(ys).all() and np.isfinite(hs).all(), f"{label}: non-finite output"
+            want_y = round_io(out_o, io_dtype)
+            acc += [np.sum((ys - want_y) ** 2), np.sum(want_y ** 2), np.sum((hs - h_o) ** 2), np.sum(h_o ** 2)]
+    e_y = float(np.sqrt(acc[0] / acc[1])) if acc[1] > 0 else float(np.sqrt(acc[0]))
+    e_h = float(np.sqrt(acc[2] / acc[3])) if acc[3] > 0 else float(np.sqrt(acc[2]))
+    assert e_y <= TOL[io_dtype], f"{label}: y rel-L2 {e_y:.3e} > {TOL[io_dtype]:.0e}"
+    assert e_h <= TOL[io_dtype], f"{label}: state rel-L2 {e_h:.3e} > {TOL[io_dtype]:.0e}"
+    return e_y, e_h

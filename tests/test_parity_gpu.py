@@ -2,14 +2,15 @@
 element by element on the same seeded inputs.
 
 Small cases cover every channel and span several pipeline stages with a ragged
-tail; the five workload shapes run at full size in the launch configuration the
-benchmark uses and are compared on a seeded sample of channels.
+tail; the four GPU workload shapes run at full size in the launch configuration
+the benchmark uses and are compared on every (sequence, channel), in blocks
+that fit host memory.
 """
 import numpy as np
 import pytest
 import torch
 
-from parity_util import TOL, all_channels, compare, gather, oracle_prefill, rel_l2, round_io
+from parity_util import TOL, all_channels, compare, compare_full, gather, oracle_prefill, rel_l2, round_io
 from selective_state_space_depthwise_b200 import api
 from selective_state_space_depthwise_b200 import workloads as W
 
@@ -199,23 +200,21 @@ def test_decode_zoh():
 
 # ------------------------------------------------------------ full sizes ---
 @pytest.mark.parametrize("name", ["axon_layer", "batched", "long_context"])
-def test_full_size_prefill_sampled(name):
-    """The workload at full size, in the default launch shape, on sampled
-    channels (first/last channel of first/last sequence included)."""
+def test_full_size_prefill_all_channels(name):
+    """The workload at full size, in the default launch shape the benchmark
+    times, against the oracle on every (sequence, channel)."""
     w = W.WORKLOADS[name]
     inp = device_inputs(w, gen_device="cuda")
     y, cc, st = run_prefill(inp)
-    chans = W.sample_channels(w, 24)
-    e_y, e_h = compare(w.io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=name)
-    assert torch.isfinite(y).all()
-    print(f"{name}: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e} over {len(chans)} channels")
+    e_y, e_h = compare_full(w.io_dtype, inp, (y, cc, st), label=name)
+    print(f"{name}: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e} over all {w.batch * w.d_inner} channels")
 
 
-def test_full_size_decode_sampled():
-    """Prompt 512, then 1024 decode steps, against one oracle prefill of 1536."""
+def test_full_size_decode_all_channels():
+    """Prompt 512, then 1024 decode steps, against one oracle prefill of 1536,
+    on every (sequence, channel)."""
     w = W.WORKLOADS["decode"]
     inp = device_inputs(w, gen_device="cuda")
     y, cc, st = decode_run(inp, w, w.seqlen, w.decode_steps)
-    chans = W.sample_channels(w, 16)
-    e_y, e_h = compare(w.io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label="decode")
-    print(f"decode: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e} over {len(chans)} channels")
+    e_y, e_h = compare_full(w.io_dtype, inp, (y, cc, st), label="decode")
+    print(f"decode: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e} over all {w.batch * w.d_inner} channels")
