@@ -48,6 +48,8 @@ def _load():
         lib.oracle_channels.restype = None
         lib.oracle_causal_conv.argtypes = [i64, i32, p, p, p, d, p]
         lib.oracle_causal_conv.restype = None
+        lib.oracle_conv_silu_channels.argtypes = [i64, i64, i32, p, p, p, p, p, i32]
+        lib.oracle_conv_silu_channels.restype = None
         for name in ("oracle_silu", "oracle_softplus", "oracle_A"):
             getattr(lib, name).argtypes = [d]
             getattr(lib, name).restype = d
@@ -134,6 +136,59 @@ def channels(x, z, B, C, dt_raw, bidx, conv_w, conv_b, w_dt, dt_bias, A_log, D,
                             _ptr(bidx), _ptr(conv_w), _ptr(conv_b), _ptr(w_dt), _ptr(dt_bias), _ptr(A_log), _ptr(D),
                             _ptr(hist), _ptr(h0), _ptr(out), _ptr(h_out), _ptr(hist_out), int(threads))
     return out[:, :L], h_out, hist_out[:, : K - 1]
+
+
+def conv_silu(x, conv_w, conv_b, hist=None, threads=0):
+    """u = SiLU(causal_conv(x)) of n channels. x: [n, L]; conv_w: [n, K];
+    conv_b: [n]; hist: [n, K-1] or None (zeros). Returns u [n, L]."""
+    x, conv_w, conv_b, hist = map(_f64, (x, conv_w, conv_b, hist))
+    n, L = x.shape
+    K = conv_w.shape[1]
+    u = np.empty((n, max(L, 1)))
+    _load().oracle_conv_silu_channels(n, L, K, _ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(hist), _ptr(u), int(threads))
+    return u[:, :L]
+
+
+def block(hidden, W_in, W_x, W_out, conv_w, conv_b, w_dt, dt_bias, A_log, D, hist=None, h0=None, lo=1e-4, hi=1.0,
+          disc="euler", threads=0):
+    """The AxonSSMBlock forward of "Axon-SSM: selective state space model",
+    "Algorithm" diagram, in float64:
+
+      x, z   = split(hidden @ W_in^T)           in_proj (D -> 2E), x first, no bias
+      u      = SiLU(conv1d(x))                   depthwise causal conv, K = 4
+      B, C, dt_raw = split(u @ W_x^T)            x_proj (E -> 2N + 1), in that order, no bias
+      y      = scan core (channels(): dt_proj + softplus + clip, the scan, D skip, y * SiLU(z))
+      out    = y @ W_out^T                       out_proj (E -> D), no bias
+
+    hidden: [b, L, D]; W_in: [2E, D]; W_x: [2N + 1, E]; W_out: [D, E]
+    (projection weights are [out_features, in_features]); the scan-core
+    parameters as in channels() but per channel [E, ...]; hist: [b, K-1, E] or
+    None; h0: [b, E, N] or None. The matrix products are library matmuls (a
+    plain step each). Returns (out [b, L, D], h_out [b, E, N], hist_out [b, K-1, E])."""
+    hidden, W_in, W_x, W_out = map(_f64, (hidden, W_in, W_x, W_out))
+    conv_w, conv_b, w_dt, dt_bias, A_log, D = map(_f64, (conv_w, conv_b, w_dt, dt_bias, A_log, D))
+    b, L, Dm = hidden.shape
+    E = W_in.shape[0] // 2
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    assert W_in.shape == (2 * E, Dm) and W_x.shape == (2 * N + 1, E) and W_out.shape == (Dm, E)
+    xz = hidden @ W_in.T
+    x, z = xz[..., :E], xz[..., E:]
+    # channel-major rows (sequence s, channel e) -> row s * E + e
+    xs = np.ascontiguousarray(x.transpose(0, 2, 1).reshape(b * E, L))
+    zs = np.ascontiguousarray(z.transpose(0, 2, 1).reshape(b * E, L))
+    tile = lambda a: np.ascontiguousarray(np.tile(a, (b,) + (1,) * (a.ndim - 1)))  # noqa: E731
+    hist_rows = None if hist is None else np.ascontiguousarray(_f64(hist).transpose(0, 2, 1).reshape(b * E, K - 1))
+    h0_rows = None if h0 is None else np.ascontiguousarray(_f64(h0).reshape(b * E, N))
+    u = conv_silu(xs, tile(conv_w), tile(conv_b), hist_rows, threads).reshape(b, E, L).transpose(0, 2, 1)
+    bcd = u @ W_x.T
+    B, C, dt_raw = bcd[..., :N], bcd[..., N:2 * N], bcd[..., 2 * N]
+    out, h_out, hist_out = channels(xs, zs, np.ascontiguousarray(B), np.ascontiguousarray(C),
+                                    np.ascontiguousarray(dt_raw), np.repeat(np.arange(b), E), tile(conv_w),
+                                    tile(conv_b), tile(w_dt), tile(dt_bias), tile(A_log), tile(D), hist=hist_rows,
+                                    h0=h0_rows, lo=lo, hi=hi, disc=disc, threads=threads)
+    y = out.reshape(b, E, L).transpose(0, 2, 1)
+    return y @ W_out.T, h_out.reshape(b, E, N), hist_out.reshape(b, E, K - 1).transpose(0, 2, 1)
 
 
 def prefill_sampled(x, z, B, C, dt_raw, conv_w, conv_b, w_dt, dt_bias, A_log, D, chans,

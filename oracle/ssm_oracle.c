@@ -181,6 +181,23 @@ void oracle_channels(int64_t n_ch, int64_t L, int N, int K, int disc, double lo,
   }
 }
 
+/* [AX] "Algorithm": the x_proj input u = SiLU(conv1d(x)) of n channels (the
+ * branch that feeds x_proj in the block diagram), channel i from x[i*L..] with
+ * its own weights and history (hist may be NULL: zeros). */
+void oracle_conv_silu_channels(int64_t n_ch, int64_t L, int K, const double *x,
+                               const double *conv_w, const double *conv_b,
+                               const double *hist, double *u, int n_threads) {
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(static)
+#endif
+  for (int64_t i = 0; i < n_ch; ++i) {
+    oracle_causal_conv(L, K, hist ? hist + i * (K - 1) : NULL, x + i * L,
+                       conv_w + i * K, conv_b[i], u + i * L);
+    for (int64_t t = 0; t < L; ++t) u[i * L + t] = oracle_silu(u[i * L + t]);
+  }
+}
+
 /* Threads the OpenMP runtime would use (1 without OpenMP). */
 int oracle_max_threads(void) {
 #ifdef _OPENMP
