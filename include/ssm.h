@@ -244,6 +244,65 @@ ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const voi
                            const float *B, const float *C, const float *dt_raw, void *y, void *conv_cache,
                            float *ssm_state, void *stream);
 
+/*
+ * ssm_block_forward -- the whole AxonSSMBlock forward of "Axon-SSM: selective
+ * state space model", "Algorithm" diagram, for a prefill:
+ *
+ *   x, z         = split(hidden @ W_in^T)          in_proj  (D -> 2E), x first
+ *   u            = SiLU(conv1d(x))                  causal depthwise conv, K = 4
+ *   B, C, dt_raw = split(u @ W_x^T)                 x_proj   (E -> 2N + 1), in that order
+ *   y            = the block core of ssm_prefill    (dt_proj, softplus, clip, scan, D skip, y * SiLU(z))
+ *   out          = y @ W_out^T                      out_proj (E -> D)
+ *
+ * Implementation. in_proj and out_proj are plain GEMMs (cuBLASLt, bf16
+ * operands, fp32 accumulation). x_proj is one fused kernel: it computes u
+ * from x tile by tile straight into tensor-core operand tiles (tcgen05 MMA,
+ * TMEM accumulator), so u never reaches memory. The core is ssm_prefill's
+ * kernel, reading x and z in place from the in_proj output. No projection has
+ * a bias.
+ *
+ * Arguments.
+ *   dims      batch, seqlen, d_model (D, a multiple of 8), d_inner (E, a
+ *             multiple of 8), d_state 16, d_conv 4, dt_min / dt_max,
+ *             discretization. io_dtype must be SSM_BF16 (SSM_ERR_UNSUPPORTED
+ *             otherwise).
+ *   w         the core's per-channel parameters, as for ssm_prefill.
+ *   proj      W_in [2E, D], W_x [2N + 1, E], W_out [D, E]: row-major
+ *             [out_features, in_features], bf16, 16-byte aligned, on the device.
+ *   hidden    [b, L, D] bf16, dense;  out [b, L, D] bf16, dense.
+ *   conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out
+ *             as for ssm_prefill. The conv cache holds raw x rows (in_proj
+ *             output), so chained calls equal one call over the whole sequence.
+ *   workspace device scratch of ssm_block_workspace_bytes(dims) bytes,
+ *             256-byte aligned. It holds the in_proj output (b L 2E bf16),
+ *             B / C / dt_raw (b L 33 fp32), the gated core output (b L E bf16)
+ *             and the GEMM workspace.
+ *
+ * Ordering and errors. Everything is enqueued on `stream`, with no host
+ * synchronisation. Argument errors return before any work is queued.
+ */
+typedef struct {
+  int64_t batch, seqlen, d_model, d_inner;
+  int32_t d_state, d_conv;
+  float dt_min, dt_max;
+  ssm_dtype io_dtype;
+  ssm_discretization discretization;
+} ssm_block_dims;
+
+typedef struct {
+  const void *w_in;  /* [2E, D] */
+  const void *w_x;   /* [2N + 1, E] */
+  const void *w_out; /* [D, E] */
+} ssm_block_weights;
+
+ssm_status ssm_block_forward(const ssm_block_dims *dims, const ssm_weights *w, const ssm_block_weights *proj,
+                             const void *hidden, const void *conv_cache_in, const float *ssm_state_in, void *out,
+                             void *conv_cache_out, float *ssm_state_out, void *workspace, size_t workspace_bytes,
+                             void *stream);
+
+/* Workspace bytes of ssm_block_forward for `dims` (0 for invalid dims). */
+size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
+
 /* Reads and clears the device error word that kernels set when a bounded
  * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed. */
 ssm_status ssm_check_device_error(void *stream);

@@ -26,6 +26,8 @@ EXPORTED = (
     "ssm_prefill_host",
     "ssm_prefill_host_workspace_bytes",
     "ssm_prefill_host_static",
+    "ssm_block_forward",
+    "ssm_block_workspace_bytes",
     "ssm_decode_step",
     "ssm_check_device_error",
     "ssm_status_string",
@@ -55,6 +57,25 @@ class SsmDims(ctypes.Structure):
         ("bc_seq_stride", ctypes.c_int64),
         ("dt_seq_stride", ctypes.c_int64),
     ]
+
+
+class SsmBlockDims(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("d_model", ctypes.c_int64),
+        ("d_inner", ctypes.c_int64),
+        ("d_state", ctypes.c_int32),
+        ("d_conv", ctypes.c_int32),
+        ("dt_min", ctypes.c_float),
+        ("dt_max", ctypes.c_float),
+        ("io_dtype", ctypes.c_int32),
+        ("discretization", ctypes.c_int32),
+    ]
+
+
+class SsmBlockWeights(ctypes.Structure):
+    _fields_ = [("w_in", ctypes.c_void_p), ("w_x", ctypes.c_void_p), ("w_out", ctypes.c_void_p)]
 
 
 class SsmWeights(ctypes.Structure):
@@ -97,6 +118,11 @@ def load(path: str = LIB_PATH):
     lib.ssm_prefill_host_static.restype = st
     lib.ssm_prefill_host_workspace_bytes.argtypes = [dims_p, ctypes.c_int64]
     lib.ssm_prefill_host_workspace_bytes.restype = sz
+    bdims_p, bw_p = ctypes.POINTER(SsmBlockDims), ctypes.POINTER(SsmBlockWeights)
+    lib.ssm_block_forward.argtypes = [bdims_p, w_p, bw_p] + [p] * 6 + [p, sz, p]
+    lib.ssm_block_forward.restype = st
+    lib.ssm_block_workspace_bytes.argtypes = [bdims_p]
+    lib.ssm_block_workspace_bytes.restype = sz
     lib.ssm_decode_step.argtypes = [dims_p, w_p] + [p] * 8 + [p]
     lib.ssm_decode_step.restype = st
     lib.ssm_check_device_error.argtypes = [p]

@@ -187,6 +187,63 @@ def prefill_host(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in
     return y, conv_cache_out, ssm_state_out
 
 
+PROJ_NAMES = ("W_in", "W_x", "W_out")
+
+
+def make_block_dims(batch, seqlen, d_model, E, dt_min=1e-4, dt_max=1.0, discretization="euler"):
+    d = _lib.SsmBlockDims()
+    d.batch, d.seqlen, d.d_model, d.d_inner, d.d_state, d.d_conv = batch, seqlen, d_model, E, 16, 4
+    d.dt_min, d.dt_max = dt_min, dt_max
+    d.io_dtype = _lib.SSM_BF16
+    d.discretization = _DISC[discretization]
+    return d
+
+
+def block_workspace_bytes(batch, seqlen, d_model, E) -> int:
+    lib = _lib.load()
+    return int(lib.ssm_block_workspace_bytes(ctypes.byref(make_block_dims(batch, seqlen, d_model, E))))
+
+
+def block_forward(hidden, params, proj, *, conv_cache_in=None, ssm_state_in=None, out=None, conv_cache_out=None,
+                  ssm_state_out=None, dt_min=1e-4, dt_max=1.0, discretization="euler", workspace=None, stream=None):
+    """The whole block forward (ssm_block_forward): hidden [b, L, D] bf16 ->
+    out [b, L, D] bf16, with proj = {"W_in": [2E, D], "W_x": [33, E],
+    "W_out": [D, E]} bf16 and the core's parameters in `params`.
+    Returns (out, conv_cache_out [b, 3, E], ssm_state_out [b, E, 16])."""
+    lib = _lib.load()
+    b, L, Dm = hidden.shape
+    dev = hidden.device
+    E = proj["W_x"].shape[1]
+    for n, t in (("hidden", hidden), ("out", out), ("conv_cache_in", conv_cache_in), ("ssm_state_in", ssm_state_in),
+                 ("conv_cache_out", conv_cache_out), ("ssm_state_out", ssm_state_out)):
+        _need_cuda(n, t, dev)
+    for n in PROJ_NAMES:
+        _need_cuda(n, proj[n], dev)
+        if proj[n].dtype != torch.bfloat16 or not proj[n].is_contiguous():
+            raise ValueError(f"{n} must be a contiguous bfloat16 tensor")
+    if proj["W_in"].shape != (2 * E, Dm) or proj["W_x"].shape != (33, E) or proj["W_out"].shape != (Dm, E):
+        raise ValueError("W_in must be [2E, D], W_x [33, E] and W_out [D, E]")
+    if hidden.dtype != torch.bfloat16 or not hidden.is_contiguous():
+        raise ValueError("hidden must be a contiguous bfloat16 tensor")
+    if out is None:
+        out = torch.empty((b, L, Dm), dtype=torch.bfloat16, device=dev)
+    if conv_cache_out is None:
+        conv_cache_out = torch.empty((b, 3, E), dtype=torch.bfloat16, device=dev)
+    if ssm_state_out is None:
+        ssm_state_out = torch.empty((b, E, 16), dtype=torch.float32, device=dev)
+    dims = make_block_dims(b, L, Dm, E, dt_min, dt_max, discretization)
+    w = _weights(params, E, dev)
+    pw = _lib.SsmBlockWeights(proj["W_in"].data_ptr(), proj["W_x"].data_ptr(), proj["W_out"].data_ptr())
+    ws = int(lib.ssm_block_workspace_bytes(ctypes.byref(dims)))
+    if workspace is None or workspace.numel() < ws:
+        workspace = torch.empty(max(ws, 1), dtype=torch.uint8, device=dev)
+    st = lib.ssm_block_forward(ctypes.byref(dims), ctypes.byref(w), ctypes.byref(pw), _ptr(hidden),
+                               _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(out), _ptr(conv_cache_out),
+                               _ptr(ssm_state_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _lib.check(st)
+    return out, conv_cache_out, ssm_state_out
+
+
 def decode_step(x, z, B, C, dt_raw, params, conv_cache, ssm_state, *, y=None, dt_min=1e-4, dt_max=1.0,
                 discretization="euler", stream=None):
     """One-token block core. x, z: [b, E] (last dim contiguous); B, C: [b, 16];

@@ -1,0 +1,434 @@
+// block.cu -- the AxonSSMBlock forward around the prefill core ("Axon-SSM:
+// selective state space model", "Algorithm" diagram): in_proj and out_proj as
+// plain cuBLASLt GEMMs, x_proj as one fused tcgen05 kernel, the core as
+// prefill.cu's kernel reading x and z in place from the in_proj output.
+//
+// x_proj kernel. A CTA owns 128 tokens of one sequence (the MMA's M) and walks
+// the E channels in chunks of 64 (K). Per chunk:
+//  1. TMA brings the x tile (131 rows: 3 halo rows for the conv) and the W_x
+//     tile (48 rows = the 33 outputs padded to a multiple of 16, zero-filled by
+//     TMA past row 33; 128-byte swizzled, the MMA's B operand);
+//  2. the four warps compute u = SiLU(conv1d(x)) for their 32 tokens (lane =
+//     channel pair, a 3-row sliding window in registers) and write it as bf16
+//     straight into the MMA's A tile, in the 128-byte swizzled K-major layout;
+//  3. one thread issues four tcgen05 MMAs (K = 16 each, bf16 x bf16 -> fp32)
+//     into a 48-column TMEM accumulator and commits them to the stage's
+//     mbarrier; the stage is refilled only after that barrier completes.
+// At the end each warp reads its 32 TMEM lanes (tokens) back and writes B, C
+// ([b, L, 32] fp32) and dt_raw ([b, L] fp32). Two stages: the TMA of chunk c+1
+// and the MMAs of chunk c-1 overlap the conv/SiLU of chunk c. u never reaches
+// memory. Every mbarrier wait is bounded.
+#include <cublasLt.h>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sm100_ptx.cuh"
+#include "ssm.h"
+#include "ssm_internal.h"
+#include "ssm_math.cuh"
+
+namespace ssm {
+namespace {
+
+constexpr int kXpTok = 128;      // tokens per CTA (MMA M)
+constexpr int kXpK = 64;         // channels per chunk: 128 bytes of bf16, one swizzle row
+constexpr int kXpN = 48;         // MMA N: the 2N + 1 = 33 outputs padded to a multiple of 16
+constexpr int kXpOut = 33;
+constexpr int kXpThreads = 128;  // warp w owns TMEM lanes (tokens) 32w .. 32w + 31
+constexpr uint32_t kXpTmemCols = 64;
+
+struct XpSmem {
+  static constexpr int kABytes = kXpTok * 128;          // [128 rows][128 B], swizzled
+  static constexpr int kWBytes = kXpN * 128;            // [48 rows][128 B], swizzled by TMA
+  static constexpr int kXBytes = (kXpTok + 3) * 128;    // [131 rows][64 channels] bf16
+  static constexpr int kA = 0;                          // 2 stages, 1024-aligned
+  static constexpr int kW = 2 * kABytes;                // 2 stages, 1024-aligned
+  static constexpr int kX = kW + 2 * kWBytes;
+  static constexpr int kBar = kX + 2 * kXBytes;         // full[2], done[2]
+  static constexpr int kTmemSlot = kBar + 4 * 8;
+  static constexpr int kAbort = kTmemSlot + 4;        // set when a bounded wait gave up
+  static constexpr int kLast = kTmemSlot + 8;         // the last chunk whose MMAs were committed
+  static constexpr int kTotal = kTmemSlot + 16;
+  static constexpr uint32_t kTx = static_cast<uint32_t>(kWBytes + kXBytes);
+  static_assert(kW % 1024 == 0 && (kW + kWBytes) % 1024 == 0 && kABytes % 1024 == 0, "swizzled tiles need 1 KB");
+};
+
+// Instruction descriptor: bf16 A and B (K-major), fp32 D, M = 128, N = 48.
+constexpr uint32_t kXpIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kXpN >> 3) << 17) |
+                              (static_cast<uint32_t>(kXpTok >> 4) << 24);
+
+struct XprojArgs {
+  const float* conv_w;                  // [E][4]
+  const float* conv_b;                  // [E]
+  const __nv_bfloat16* conv_cache_in;   // [b][3][E] or null (zeros)
+  float* bc;                            // [b][L][32]: B then C
+  float* dt_raw;                        // [b][L]
+  int64_t L, E;
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+  __nv_bfloat162 v;
+  *reinterpret_cast<uint32_t*>(&v) = w;
+  return __bfloat1622float2(v);
+}
+
+__global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant__ CUtensorMap map_x,
+                                                          const __grid_constant__ CUtensorMap map_w,
+                                                          const XprojArgs a) {
+  using S = XpSmem;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sb = smem_u32(smem);
+  const int tid = threadIdx.x;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0), lane = tid & 31;
+  const int seq = blockIdx.y;
+  const int t0 = blockIdx.x * kXpTok;
+  const int nk = static_cast<int>((a.E + kXpK - 1) / kXpK);
+  auto full = [&](int s) { return sb + S::kBar + 8 * s; };
+  auto done = [&](int s) { return sb + S::kBar + 16 + 8 * s; };
+  auto issue = [&](int c) {  // thread 0
+    const int s = c & 1;
+    mbar_arrive_expect_tx(full(s), S::kTx);
+    tma_load_3d(sb + S::kX + s * S::kXBytes, &map_x, c * kXpK, t0 - 3, seq, full(s));
+    tma_load_3d(sb + S::kW + s * S::kWBytes, &map_w, c * kXpK, 0, 0, full(s));
+  };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kAbort);
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < 4; ++i) mbar_init(sb + S::kBar + 8 * i, 1);
+    mbar_fence_init();
+    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_w);
+    issue(0);
+    if (nk > 1) issue(1);
+  }
+  if (warp == 0) {
+    tmem_alloc(sb + S::kTmemSlot, kXpTmemCols);
+    tmem_relinquish();
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
+
+  int issued = -1;  // last chunk whose MMAs thread 0 committed
+  for (int c = 0; c < nk; ++c) {
+    const int s = c & 1;
+    if (!mbar_wait_bounded(full(s), static_cast<uint32_t>((c >> 1) & 1), a.err, 3)) *abort_flag = 1;
+    // this lane's channel pair and its conv weights
+    const int64_t e0 = static_cast<int64_t>(c) * kXpK + 2 * lane;
+    const bool v0 = e0 < a.E, v1 = e0 + 1 < a.E;
+    const float4 w0 = v0 ? reinterpret_cast<const float4*>(a.conv_w)[e0] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 w1 = v1 ? reinterpret_cast<const float4*>(a.conv_w)[e0 + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float b0 = v0 ? a.conv_b[e0] : 0.0f, b1 = v1 ? a.conv_b[e0 + 1] : 0.0f;
+    const uint32_t* xt = reinterpret_cast<const uint32_t*>(smem + S::kX + s * S::kXBytes);
+    unsigned char* At = smem + S::kA + s * S::kABytes;
+    // window = tile rows r, r+1, r+2 (tokens t0 + r - 3 ..); rows before token 0 are
+    // zero-filled by TMA and replaced by the incoming conv cache when there is one
+    const int r0 = 32 * warp;
+    float2 x0 = unpack_bf16x2(xt[(r0 + 0) * 32 + lane]);
+    float2 x1 = unpack_bf16x2(xt[(r0 + 1) * 32 + lane]);
+    float2 x2 = unpack_bf16x2(xt[(r0 + 2) * 32 + lane]);
+    if (t0 == 0 && warp == 0 && a.conv_cache_in) {
+      const __nv_bfloat16* h = a.conv_cache_in + static_cast<int64_t>(seq) * 3 * a.E;
+      float2 hv[3];
+#pragma unroll
+      for (int k = 0; k < 3; ++k)
+        hv[k] = make_float2(v0 ? __bfloat162float(h[k * a.E + e0]) : 0.0f,
+                            v1 ? __bfloat162float(h[k * a.E + e0 + 1]) : 0.0f);
+      x0 = hv[0], x1 = hv[1], x2 = hv[2];
+    }
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+      const int r = r0 + i;
+      const float2 x3 = unpack_bf16x2(xt[(r + 3) * 32 + lane]);
+      const float c0 = fmaf(w0.w, x3.x, fmaf(w0.z, x2.x, fmaf(w0.y, x1.x, fmaf(w0.x, x0.x, b0))));
+      const float c1 = fmaf(w1.w, x3.y, fmaf(w1.z, x2.y, fmaf(w1.y, x1.y, fmaf(w1.x, x0.y, b1))));
+      const uint32_t u = pack_bf16x2(v0 ? silu(c0) : 0.0f, v1 ? silu(c1) : 0.0f);
+      // element (row r, k = 2 lane) of the 128-byte swizzled K-major tile
+      *reinterpret_cast<uint32_t*>(At + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) + ((lane & 3) << 2)) = u;
+      x0 = x1, x1 = x2, x2 = x3;
+    }
+    fence_proxy_async_smem();  // the tile's generic-proxy writes become visible to the tensor core
+    __syncthreads();
+    if (*abort_flag) break;  // a wait gave up: stop queueing work (every thread sees the flag here)
+    if (tid == 0) {
+      tcgen05_fence_after();
+      const uint32_t a_base = sb + S::kA + s * S::kABytes, w_base = sb + S::kW + s * S::kWBytes;
+#pragma unroll
+      for (int kk = 0; kk < kXpK / 16; ++kk)
+        umma_f16_ss(tmem, umma_desc_k_sw128(a_base + 32 * kk), umma_desc_k_sw128(w_base + 32 * kk), kXpIdesc,
+                    c > 0 || kk > 0);
+      umma_commit(done(s));
+      issued = c;
+      // chunk c + 1 refills the stage chunk c - 1 used: wait for its MMAs first
+      if (c >= 1 && c + 1 < nk) {
+        if (mbar_wait_bounded(done((c - 1) & 1), static_cast<uint32_t>(((c - 1) >> 1) & 1), a.err, 4))
+          issue(c + 1);
+        else
+          *abort_flag = 1;
+      }
+    }
+  }
+  // Every thread waits (bounded) for the last MMAs thread 0 committed; thread 0
+  // publishes which chunk that was.
+  volatile int* last_slot = reinterpret_cast<volatile int*>(smem + S::kLast);
+  if (tid == 0) *last_slot = issued;
+  __syncthreads();
+  const int last = *last_slot;
+  if (last >= 0) mbar_wait_bounded(done(last & 1), static_cast<uint32_t>((last >> 1) & 1), a.err, 5);
+  tcgen05_fence_after();
+
+  float v[kXpN];
+#pragma unroll
+  for (int j = 0; j < kXpN / 16; ++j) {
+    uint32_t r[16];
+    tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 16 * j, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v[16 * j + q] = __uint_as_float(r[q]);
+  }
+  const int64_t t = t0 + 32 * warp + lane;
+  if (t < a.L) {
+    float4* bc = reinterpret_cast<float4*>(a.bc + (static_cast<int64_t>(seq) * a.L + t) * 32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) bc[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    a.dt_raw[static_cast<int64_t>(seq) * a.L + t] = v[2 * 16];
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcgen05_fence_after();
+    tmem_dealloc(tmem, kXpTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+bool bf16_map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+               uint64_t s2_bytes, uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+  auto fn = encode_tiled();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// x = the first E columns of xz [b][L][2E] (bf16); W_x [33][E] (bf16).
+cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, int64_t batch, cudaStream_t st) {
+  CUtensorMap mx, mw;
+  const uint64_t E = static_cast<uint64_t>(a.E), L = static_cast<uint64_t>(a.L);
+  if (!bf16_map3(&mx, xz, E, L, static_cast<uint64_t>(batch), 2 * E * 2, L * 2 * E * 2, kXpK, kXpTok + 3,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !bf16_map3(&mw, w_x, E, kXpOut, 1, E * 2, kXpOut * E * 2, kXpK, kXpN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const int smem = XpSmem::kTotal + 1024;
+  cudaError_t err = cudaFuncSetAttribute(xproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  const int64_t gx = (a.L + kXpTok - 1) / kXpTok;
+  if (gx > 0x7fffffff || batch > 65535) return cudaErrorInvalidConfiguration;
+  xproj_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(batch)), kXpThreads, smem, st>>>(mx, mw, a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ cuBLASLt ---
+std::mutex g_lt_mutex;
+cublasLtHandle_t g_lt[64] = {};
+
+cublasLtHandle_t lt_handle() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_lt_mutex);
+  if (!g_lt[dev] && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS) g_lt[dev] = nullptr;
+  return g_lt[dev];
+}
+
+// out[M][N] = act[M][K] . w[N][K]^T, bf16 in and out, fp32 accumulation; all
+// row-major and dense. In cuBLASLt's column-major terms: out^T = w^T' . act^T.
+ssm_status gemm_bf16_nt(const void* act, const void* w, void* out, int64_t M, int64_t N, int64_t K, void* ws,
+                        size_t ws_bytes, cudaStream_t st, const char* what) {
+  cublasLtHandle_t h = lt_handle();
+  if (!h) return fail(SSM_ERR_CUDA, "%s: no cuBLASLt handle", what);
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulPreference_t pref = nullptr;
+  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
+  cublasStatus_t s = cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F);
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, K, N, K);
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, K, M, K);
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, N, M, N);
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulPreferenceCreate(&pref);
+  if (s == CUBLAS_STATUS_SUCCESS)
+    s = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
+                                             sizeof(ws_bytes));
+  cublasLtMatmulHeuristicResult_t res{};
+  int found = 0;
+  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &found);
+  const float alpha = 1.0f, beta = 0.0f;
+  if (s == CUBLAS_STATUS_SUCCESS && found > 0)
+    s = cublasLtMatmul(h, op, &alpha, w, la, act, lb, &beta, out, lc, out, lc, &res.algo, ws, ws_bytes, st);
+  if (pref) cublasLtMatmulPreferenceDestroy(pref);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  if (s != CUBLAS_STATUS_SUCCESS) return fail(SSM_ERR_CUDA, "%s: cuBLASLt status %d", what, static_cast<int>(s));
+  if (found == 0) return fail(SSM_ERR_UNSUPPORTED, "%s: cuBLASLt found no algorithm", what);
+  return SSM_OK;
+}
+
+constexpr size_t kAlign = 256;
+constexpr size_t kLtWorkspace = 32u << 20;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct BlockLayout {
+  size_t xz, bc, dt, y, lt, bytes;
+};
+
+BlockLayout block_layout(const ssm_block_dims* d) {
+  const size_t M = static_cast<size_t>(d->batch * d->seqlen), E = static_cast<size_t>(d->d_inner);
+  BlockLayout l{};
+  size_t off = 0;
+  l.xz = off, off = align_up(off + M * 2 * E * 2);
+  l.bc = off, off = align_up(off + M * 32 * 4);
+  l.dt = off, off = align_up(off + M * 4);
+  l.y = off, off = align_up(off + M * E * 2);
+  l.lt = off, off = align_up(off + kLtWorkspace);
+  l.bytes = off;
+  return l;
+}
+
+ssm_status check_block_dims(const ssm_block_dims* d) {
+  if (!d) return fail(SSM_ERR_INVALID_ARG, "dims is NULL");
+  if (d->d_state != 16) return fail(SSM_ERR_UNSUPPORTED, "d_state=%d: only 16 is built", d->d_state);
+  if (d->d_conv != 4) return fail(SSM_ERR_UNSUPPORTED, "d_conv=%d: only 4 is built", d->d_conv);
+  if (d->io_dtype != SSM_BF16) return fail(SSM_ERR_UNSUPPORTED, "the block forward is built for bf16 only");
+  if (d->batch <= 0 || d->batch > 65535)
+    return fail(SSM_ERR_INVALID_ARG, "batch=%lld must be in 1..65535", (long long)d->batch);
+  if (d->seqlen < 0) return fail(SSM_ERR_INVALID_ARG, "seqlen=%lld must be >= 0", (long long)d->seqlen);
+  if (d->d_model <= 0 || d->d_model % 8 != 0)
+    return fail(SSM_ERR_INVALID_ARG, "d_model=%lld must be a positive multiple of 8", (long long)d->d_model);
+  if (d->d_inner <= 0 || d->d_inner % 8 != 0)
+    return fail(SSM_ERR_INVALID_ARG, "d_inner=%lld must be a positive multiple of 8", (long long)d->d_inner);
+  if (!(d->dt_min > 0.0f) || !(d->dt_max >= d->dt_min))
+    return fail(SSM_ERR_INVALID_ARG, "need 0 < dt_min <= dt_max (got %g, %g)", d->dt_min, d->dt_max);
+  if (d->discretization != SSM_DISC_EULER_B && d->discretization != SSM_DISC_ZOH)
+    return fail(SSM_ERR_INVALID_ARG, "discretization=%d unknown", d->discretization);
+  return SSM_OK;
+}
+
+ssm_dims core_dims(const ssm_block_dims* d) {
+  ssm_dims c{};
+  c.batch = d->batch, c.seqlen = d->seqlen, c.d_inner = d->d_inner, c.d_state = 16, c.d_conv = 4;
+  c.dt_min = d->dt_min, c.dt_max = d->dt_max, c.io_dtype = SSM_BF16, c.discretization = d->discretization;
+  return c;
+}
+
+}  // namespace
+}  // namespace ssm
+
+extern "C" {
+
+size_t ssm_block_workspace_bytes(const ssm_block_dims* dims) {
+  if (ssm::check_block_dims(dims) != SSM_OK) return 0;
+  return ssm::block_layout(dims).bytes;
+}
+
+ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, const ssm_block_weights* proj,
+                             const void* hidden, const void* conv_cache_in, const float* ssm_state_in, void* out,
+                             void* conv_cache_out, float* ssm_state_out, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  using ssm::fail;
+  ssm_status st = ssm::check_block_dims(dims);
+  if (st != SSM_OK) return st;
+  if ((st = ssm::check_weights(w)) != SSM_OK) return st;
+  if ((st = ssm::check_prefill_caches(conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out)) != SSM_OK)
+    return st;
+  ssm_dims cd = ssm::core_dims(dims);
+  if (dims->seqlen == 0)  // caches only
+    return ssm_prefill(&cd, w, nullptr, nullptr, nullptr, nullptr, nullptr, conv_cache_in, ssm_state_in, nullptr,
+                       conv_cache_out, ssm_state_out, nullptr, 0, stream);
+  if (!proj) return fail(SSM_ERR_INVALID_ARG, "proj is NULL");
+  const void* pw[3] = {proj->w_in, proj->w_x, proj->w_out};
+  const char* pn[3] = {"w_in", "w_x", "w_out"};
+  for (int i = 0; i < 3; ++i)
+    if (!pw[i] || !ssm::aligned(pw[i], 16)) return fail(SSM_ERR_INVALID_ARG, "proj.%s is NULL or misaligned", pn[i]);
+  if (!hidden || !ssm::aligned(hidden, 16)) return fail(SSM_ERR_INVALID_ARG, "hidden is NULL or misaligned");
+  if (!out || !ssm::aligned(out, 16)) return fail(SSM_ERR_INVALID_ARG, "out is NULL or misaligned");
+  if (out == hidden) return fail(SSM_ERR_INVALID_ARG, "out must not alias hidden");
+  const ssm::BlockLayout lay = ssm::block_layout(dims);
+  if (!workspace || !ssm::aligned(workspace, ssm::kAlign))
+    return fail(SSM_ERR_INVALID_ARG, "workspace is NULL or not %zu-byte aligned", ssm::kAlign);
+  if (workspace_bytes < lay.bytes)
+    return fail(SSM_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, lay.bytes);
+
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const int64_t b = dims->batch, L = dims->seqlen, E = dims->d_inner, Dm = dims->d_model, M = b * L;
+  void* xz = ws + lay.xz;
+  float* bc = reinterpret_cast<float*>(ws + lay.bc);
+  float* dt = reinterpret_cast<float*>(ws + lay.dt);
+  void* y = ws + lay.y;
+
+  // in_proj: xz[M][2E] = hidden[M][D] . W_in[2E][D]^T
+  if ((st = ssm::gemm_bf16_nt(hidden, proj->w_in, xz, M, 2 * E, Dm, ws + lay.lt, ssm::kLtWorkspace, cs,
+                              "in_proj")) != SSM_OK)
+    return st;
+  // x_proj (fused with conv + SiLU): B, C, dt_raw
+  ssm::XprojArgs xa{};
+  xa.conv_w = w->conv_w;
+  xa.conv_b = w->conv_b;
+  xa.conv_cache_in = static_cast<const __nv_bfloat16*>(conv_cache_in);
+  xa.bc = bc;
+  xa.dt_raw = dt;
+  xa.L = L;
+  xa.E = E;
+  xa.err = ssm::device_error_ptr();
+  if (!xa.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
+  cudaError_t err = ssm::launch_xproj(xa, xz, proj->w_x, b, cs);
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "x_proj launch: %s", cudaGetErrorString(err));
+  // the core, on x and z in place in xz
+  cd.x_tok_stride = cd.z_tok_stride = 2 * E;
+  cd.x_seq_stride = cd.z_seq_stride = L * 2 * E;
+  cd.y_tok_stride = E;
+  cd.y_seq_stride = L * E;
+  cd.bc_tok_stride = 32;
+  cd.bc_seq_stride = L * 32;
+  cd.dt_seq_stride = L;
+  const __nv_bfloat16* xzb = static_cast<const __nv_bfloat16*>(xz);
+  if ((st = ssm_prefill(&cd, w, xzb, xzb + E, bc, bc + 16, dt, conv_cache_in, ssm_state_in, y, conv_cache_out,
+                        ssm_state_out, nullptr, 0, stream)) != SSM_OK)
+    return st;
+  // out_proj: out[M][D] = y[M][E] . W_out[D][E]^T
+  if ((st = ssm::gemm_bf16_nt(y, proj->w_out, out, M, Dm, E, ws + lay.lt, ssm::kLtWorkspace, cs, "out_proj")) !=
+      SSM_OK)
+    return st;
+  return ssm::fail(SSM_OK, "");
+}
+
+}  // extern "C"

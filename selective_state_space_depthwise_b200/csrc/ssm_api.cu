@@ -125,6 +125,9 @@ void fill_weights(ssm::KernelArgs& a, const ssm_weights* w) {
 
 __device__ int g_device_error = 0;
 
+}  // namespace
+
+namespace ssm {
 // Device address of the error word on the current device (looked up once per
 // device; host code must not pass the symbol itself to a kernel).
 int* device_error_ptr() {
@@ -137,6 +140,10 @@ int* device_error_ptr() {
   if (dev >= 0 && dev < 64) cache[dev] = static_cast<int*>(p);
   return static_cast<int*>(p);
 }
+}  // namespace ssm
+
+namespace {
+using ssm::device_error_ptr;
 
 }  // namespace
 

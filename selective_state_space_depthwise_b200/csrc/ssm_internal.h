@@ -63,5 +63,6 @@ ssm_status check_prefill_caches(const void* conv_cache_in, const float* ssm_stat
                                 const float* ssm_state_out);
 bool aligned(const void* p, size_t a);
 ssm_status fail(ssm_status st, const char* fmt, ...);
+int* device_error_ptr();  // the device error word of the current device
 
 }  // namespace ssm

@@ -129,3 +129,31 @@ def make_inputs(w: Workload, device="cpu", gen_device=None) -> dict:
     p.update(a)
     return p
 
+
+
+# ------------------------------------------------------------- the block ---
+# The whole AxonSSMBlock forward at the pages' layer shape: hidden_dim D = 2560,
+# E = 7680 ("Axon-SSM: selective state space model", "Algorithm").
+BLOCK_WORKLOADS = {
+    "block_axon_layer": (Workload("block_axon_layer", batch=1, seqlen=2048, d_inner=7680, seed=5,
+                                  note="AxonSSMBlock forward at the Axon layer shape, D = 2560"), 2560),
+}
+
+
+def make_block_inputs(w: Workload, d_model: int, device="cpu", gen_device=None) -> dict:
+    """Synthetic inputs of the block forward: the core's parameters (make_params),
+    hidden [b, L, D] ~ N(0, 1) and the projection weights W_in [2E, D] ~ N(0, 1/D),
+    W_x [2N+1, E] ~ N(0, 1/E), W_out [D, E] ~ N(0, 1/E) (so x, z, B, C and dt_raw
+    come out near unit variance, like the core workloads' draws), all bf16 (RNE
+    from fp32), drawn in that order after the parameters from one seeded generator."""
+    gen_device = gen_device or device
+    p = {k: v.to(device) for k, v in make_params(w).items()}
+    g = torch.Generator(device=gen_device).manual_seed(w.seed + 1000)
+    b, L, E, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    hidden = _randn_chunked((b, L, d_model), g, gen_device, torch.bfloat16)
+    scale = lambda t, s: (t.float() * s).to(torch.bfloat16)  # noqa: E731
+    W_in = scale(_randn_chunked((2 * E, d_model), g, gen_device, torch.bfloat16), d_model ** -0.5)
+    W_x = scale(_randn_chunked((2 * N + 1, E), g, gen_device, torch.bfloat16), E ** -0.5)
+    W_out = scale(_randn_chunked((d_model, E), g, gen_device, torch.bfloat16), E ** -0.5)
+    p.update(hidden=hidden.to(device), W_in=W_in.to(device), W_x=W_x.to(device), W_out=W_out.to(device))
+    return p

@@ -182,3 +182,31 @@ def test_host_binding_refuses_host_parameters(lib):
     with pytest.raises(RuntimeError, match="CUDA tensor"):
         api.prefill_host(x, x, torch.zeros(1, 8, 16), torch.zeros(1, 8, 16), torch.zeros(1, 8), p,
                          conv_cache_out=torch.zeros(1, 3, 8, dtype=torch.bfloat16))
+
+
+def test_block_forward_rejects_bad_arguments_before_any_work(lib):
+    w = fake_weights()
+    pw = _lib.SsmBlockWeights(FAKE, FAKE, FAKE)
+    ws_need = lib.ssm_block_workspace_bytes(ctypes.byref(api.make_block_dims(2, 64, 32, 64)))
+    assert ws_need > 0
+
+    def call(dims, proj=pw, hidden=FAKE, out=FAKE + 4096, ws=FAKE, ws_bytes=ws_need):
+        return lib.ssm_block_forward(ctypes.byref(dims) if dims is not None else None, ctypes.byref(w),
+                                     ctypes.byref(proj) if proj is not None else None, hidden, None, None, out, FAKE,
+                                     FAKE, ws, ws_bytes, None)
+
+    d = api.make_block_dims(2, 64, 32, 64)
+    d32 = api.make_block_dims(2, 64, 32, 64)
+    d32.io_dtype = _lib.SSM_F32
+    assert call(d32) == _lib.SSM_ERR_UNSUPPORTED
+    assert b"bf16" in lib.ssm_last_error()
+    assert call(None) == _lib.SSM_ERR_INVALID_ARG
+    bad = api.make_block_dims(2, 64, 30, 64)  # d_model not a multiple of 8
+    assert call(bad) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, proj=None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, proj=_lib.SsmBlockWeights(FAKE, None, FAKE)) == _lib.SSM_ERR_INVALID_ARG
+    assert b"w_x" in lib.ssm_last_error()
+    assert call(d, hidden=None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, out=FAKE) == _lib.SSM_ERR_INVALID_ARG  # out aliases hidden
+    assert call(d, ws_bytes=ws_need - 1) == _lib.SSM_ERR_INVALID_ARG
+    assert lib.ssm_block_workspace_bytes(ctypes.byref(d32)) == 0
