@@ -37,6 +37,7 @@ from selective_state_space_depthwise_b200 import workloads as W  # noqa: E402
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 # SM resources used to derive the ALU roofline (B200, sm_100a): 148 SMs,
 # 16 SFU lanes and 128 FP32 lanes per SM per clock (the SFU and FFMA rates
@@ -86,6 +87,15 @@ def load_peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_bf16_peak() -> float:
+    """Measured dense bf16 GEMM throughput (burst), else the fallback figure."""
+    try:
+        with open(PEAKS_PATH) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return FALLBACK_BF16_TFLOPS
 
 
 class ClockSampler:
@@ -343,6 +353,48 @@ def decode_bench(w: W.Workload, rank: int, hbm_peak: float, peak_kind: str):
             "gpu_launches": steps}
 
 
+def block_bench(name: str, bf16_peak: float, steps: int = 10, warmup: int = 3):
+    """The whole block forward (ssm_block_forward) on device-resident inputs:
+    ms per call by CUDA events, tokens/s, and the projections' tensor FLOPs
+    (in_proj 2E*D, x_proj 33*E, out_proj D*E per token, x2) per second against
+    the measured bf16 GEMM peak."""
+    from selective_state_space_depthwise_b200 import api
+
+    w, d_model = W.BLOCK_WORKLOADS[name]
+    inp = W.make_block_inputs(w, d_model, device="cuda", gen_device="cuda")
+    proj = {k: inp[k] for k in api.PROJ_NAMES}
+    b, L, E = w.batch, w.seqlen, w.d_inner
+    out = torch.empty((b, L, d_model), dtype=torch.bfloat16, device="cuda")
+    cc = torch.empty((b, 3, E), dtype=torch.bfloat16, device="cuda")
+    st = torch.empty((b, E, 16), dtype=torch.float32, device="cuda")
+    ws = torch.empty(api.block_workspace_bytes(b, L, d_model, E), dtype=torch.uint8, device="cuda")
+
+    def call():
+        api.block_forward(inp["hidden"], inp, proj, out=out, conv_cache_out=cc, ssm_state_out=st, workspace=ws)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        call()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / steps
+    tokens = b * L
+    flops = 2.0 * tokens * (2 * E * d_model + 33 * E + d_model * E)
+    tflops = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"{name}: {w.note}; b={b} L={L} D={d_model} E={E}", "ms_per_step": round(ms, 4),
+            "value": tokens / (ms * 1e-3), "unit": "tokens/s", "steps": steps,
+            "projections": {"tflops": round(tflops, 1), "peak": bf16_peak, "unit": "TFLOP/s",
+                            "frac": round(tflops / bf16_peak, 4), "flops_per_step": flops,
+                            "note": "GEMM FLOPs of in_proj, x_proj and out_proj over the whole block time "
+                                    "(the scan core's SFU-bound time is included in the denominator)"},
+            "gpu_launches_per_step": 4}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -353,6 +405,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode sub-benchmark")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--no-block", action="store_true", help="skip the block-forward sub-benchmark")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -422,6 +475,10 @@ def main():
         torch.cuda.empty_cache()
         if not args.no_decode:
             extra["decode"] = decode_bench(W.WORKLOADS["decode"], rank, hbm_peak, peak_kind)
+        if not args.no_block:
+            torch.cuda.empty_cache()
+            bf16_peak = load_bf16_peak()
+            extra["block"] = [block_bench(n, bf16_peak) for n in W.BLOCK_WORKLOADS]
         if not args.no_cpu and world == 1:
             extra["cpu_baseline"] = cpu_baseline(w)
     if dist:

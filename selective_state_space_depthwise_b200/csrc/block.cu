@@ -3,20 +3,25 @@
 // plain cuBLASLt GEMMs, x_proj as one fused tcgen05 kernel, the core as
 // prefill.cu's kernel reading x and z in place from the in_proj output.
 //
-// x_proj kernel. A CTA owns 128 tokens of one sequence (the MMA's M) and walks
-// the E channels in chunks of 64 (K). Per chunk:
+// x_proj kernel. A CTA owns 128 tokens of one sequence (the MMA's M) and a
+// contiguous range of the E channels, walked in chunks of 64 (K). Per chunk:
 //  1. TMA brings the x tile (131 rows: 3 halo rows for the conv) and the W_x
 //     tile (48 rows = the 33 outputs padded to a multiple of 16, zero-filled by
-//     TMA past row 33; 128-byte swizzled, the MMA's B operand);
+//     TMA past row 33; 128-byte swizzled, the MMA's B operand) into a 3-slot
+//     ring, issued two chunks ahead;
 //  2. the four warps compute u = SiLU(conv1d(x)) for their 32 tokens (lane =
-//     channel pair, a 3-row sliding window in registers) and write it as bf16
-//     straight into the MMA's A tile, in the 128-byte swizzled K-major layout;
+//     channel pair, a 3-row sliding window in registers, the conv weights of
+//     the next chunk loaded one chunk ahead) and write it as bf16 straight
+//     into the MMA's A tile (2 slots), in the 128-byte swizzled K-major layout;
 //  3. one thread issues four tcgen05 MMAs (K = 16 each, bf16 x bf16 -> fp32)
-//     into a 48-column TMEM accumulator and commits them to the stage's
-//     mbarrier; the stage is refilled only after that barrier completes.
-// At the end each warp reads its 32 TMEM lanes (tokens) back and writes B, C
-// ([b, L, 32] fp32) and dt_raw ([b, L] fp32). Two stages: the TMA of chunk c+1
-// and the MMAs of chunk c-1 overlap the conv/SiLU of chunk c. u never reaches
+//     into a 48-column TMEM accumulator and commits them to the A slot's
+//     mbarrier; slots are refilled only after the MMAs that read them completed.
+// Split K: when 128-token tiles alone would not fill the GPU, a thread-block
+// cluster of S CTAs (S <= 8, along grid z) shares one tile, each CTA summing a
+// contiguous channel range in its own TMEM. The partial 128 x 48 tiles go to
+// shared memory and CTA r of the cluster adds, in the fixed order 0..S-1 over
+// distributed shared memory, the rows of tokens [r 128/S, (r+1) 128/S) and
+// writes B, C ([b, L, 32] fp32) and dt_raw ([b, L] fp32). u never reaches
 // memory. Every mbarrier wait is bounded.
 #include <cublasLt.h>
 #include <cuda.h>
@@ -39,21 +44,25 @@ constexpr int kXpN = 48;         // MMA N: the 2N + 1 = 33 outputs padded to a m
 constexpr int kXpOut = 33;
 constexpr int kXpThreads = 128;  // warp w owns TMEM lanes (tokens) 32w .. 32w + 31
 constexpr uint32_t kXpTmemCols = 64;
+constexpr int kXpStages = 3;     // x / W_x TMA ring
+constexpr int kXpMaxSplit = 8;   // portable cluster size
 
 struct XpSmem {
   static constexpr int kABytes = kXpTok * 128;          // [128 rows][128 B], swizzled
   static constexpr int kWBytes = kXpN * 128;            // [48 rows][128 B], swizzled by TMA
   static constexpr int kXBytes = (kXpTok + 3) * 128;    // [131 rows][64 channels] bf16
-  static constexpr int kA = 0;                          // 2 stages, 1024-aligned
-  static constexpr int kW = 2 * kABytes;                // 2 stages, 1024-aligned
-  static constexpr int kX = kW + 2 * kWBytes;
-  static constexpr int kBar = kX + 2 * kXBytes;         // full[2], done[2]
-  static constexpr int kTmemSlot = kBar + 4 * 8;
-  static constexpr int kAbort = kTmemSlot + 4;        // set when a bounded wait gave up
-  static constexpr int kLast = kTmemSlot + 8;         // the last chunk whose MMAs were committed
+  static constexpr int kA = 0;                          // 2 slots, 1024-aligned
+  static constexpr int kW = 2 * kABytes;                // kXpStages slots, 1024-aligned
+  static constexpr int kX = kW + kXpStages * kWBytes;   // kXpStages slots
+  static constexpr int kP = kX;                         // partial sums [128][48] fp32, after the loop
+  static constexpr int kBar = kX + kXpStages * kXBytes; // full[kXpStages], done[2]
+  static constexpr int kTmemSlot = kBar + (kXpStages + 2) * 8;
+  static constexpr int kAbort = kTmemSlot + 4;          // set when a bounded wait gave up
+  static constexpr int kLast = kTmemSlot + 8;           // the last chunk whose MMAs were committed
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr uint32_t kTx = static_cast<uint32_t>(kWBytes + kXBytes);
-  static_assert(kW % 1024 == 0 && (kW + kWBytes) % 1024 == 0 && kABytes % 1024 == 0, "swizzled tiles need 1 KB");
+  static_assert(kW % 1024 == 0 && kWBytes % 1024 == 0 && kABytes % 1024 == 0, "swizzled tiles need 1 KB");
+  static_assert(kXpTok * kXpN * 4 <= kXpStages * kXBytes, "the partial tile reuses the x ring");
 };
 
 // Instruction descriptor: bf16 A and B (K-major), fp32 D, M = 128, N = 48.
@@ -81,6 +90,21 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
   return __bfloat1622float2(v);
 }
 
+struct ConvPair {  // conv weights and biases of one lane's channel pair in one chunk
+  float4 w0, w1;
+  float b0, b1;
+};
+
+__device__ __forceinline__ ConvPair load_conv_pair(const XprojArgs& a, int64_t e0) {
+  ConvPair p;
+  const bool v0 = e0 < a.E, v1 = e0 + 1 < a.E;
+  p.w0 = v0 ? reinterpret_cast<const float4*>(a.conv_w)[e0] : make_float4(0.f, 0.f, 0.f, 0.f);
+  p.w1 = v1 ? reinterpret_cast<const float4*>(a.conv_w)[e0 + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+  p.b0 = v0 ? a.conv_b[e0] : 0.0f;
+  p.b1 = v1 ? a.conv_b[e0 + 1] : 0.0f;
+  return p;
+}
+
 __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant__ CUtensorMap map_x,
                                                           const __grid_constant__ CUtensorMap map_w,
                                                           const XprojArgs a) {
@@ -92,24 +116,25 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0), lane = tid & 31;
   const int seq = blockIdx.y;
   const int t0 = blockIdx.x * kXpTok;
+  const int split = gridDim.z, rank = blockIdx.z;  // the cluster spans grid z
   const int nk = static_cast<int>((a.E + kXpK - 1) / kXpK);
-  auto full = [&](int s) { return sb + S::kBar + 8 * s; };
-  auto done = [&](int s) { return sb + S::kBar + 16 + 8 * s; };
-  auto issue = [&](int c) {  // thread 0
-    const int s = c & 1;
-    mbar_arrive_expect_tx(full(s), S::kTx);
-    tma_load_3d(sb + S::kX + s * S::kXBytes, &map_x, c * kXpK, t0 - 3, seq, full(s));
-    tma_load_3d(sb + S::kW + s * S::kWBytes, &map_w, c * kXpK, 0, 0, full(s));
+  const int c_begin = rank * nk / split, nloc = (rank + 1) * nk / split - c_begin;
+  auto full = [&](int j) { return sb + S::kBar + 8 * (j % kXpStages); };
+  auto done = [&](int j) { return sb + S::kBar + 8 * kXpStages + 8 * (j & 1); };
+  auto issue = [&](int j) {  // thread 0: the tiles of local chunk j
+    const int slot = j % kXpStages, c = c_begin + j;
+    mbar_arrive_expect_tx(full(j), S::kTx);
+    tma_load_3d(sb + S::kX + slot * S::kXBytes, &map_x, c * kXpK, t0 - 3, seq, full(j));
+    tma_load_3d(sb + S::kW + slot * S::kWBytes, &map_w, c * kXpK, 0, 0, full(j));
   };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kAbort);
   if (tid == 0) {
     *abort_flag = 0;
-    for (int i = 0; i < 4; ++i) mbar_init(sb + S::kBar + 8 * i, 1);
+    for (int i = 0; i < kXpStages + 2; ++i) mbar_init(sb + S::kBar + 8 * i, 1);
     mbar_fence_init();
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_w);
-    issue(0);
-    if (nk > 1) issue(1);
+    for (int j = 0; j < kXpStages && j < nloc; ++j) issue(j);
   }
   if (warp == 0) {
     tmem_alloc(sb + S::kTmemSlot, kXpTmemCols);
@@ -120,18 +145,20 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
   tcgen05_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
 
-  int issued = -1;  // last chunk whose MMAs thread 0 committed
-  for (int c = 0; c < nk; ++c) {
-    const int s = c & 1;
-    if (!mbar_wait_bounded(full(s), static_cast<uint32_t>((c >> 1) & 1), a.err, 3)) *abort_flag = 1;
-    // this lane's channel pair and its conv weights
+  int issued = -1;  // the last local chunk whose MMAs thread 0 committed
+  ConvPair cw = load_conv_pair(a, static_cast<int64_t>(c_begin) * kXpK + 2 * lane);
+  for (int j = 0; j < nloc; ++j) {
+    const int c = c_begin + j;
+    // the next chunk's conv weights, one chunk ahead
+    const ConvPair cw_next =
+        j + 1 < nloc ? load_conv_pair(a, static_cast<int64_t>(c + 1) * kXpK + 2 * lane) : cw;
+    if (!mbar_wait_bounded(full(j), static_cast<uint32_t>((j / kXpStages) & 1), a.err, 3)) *abort_flag = 1;
+    if (j >= 2 && !mbar_wait_bounded(done(j), static_cast<uint32_t>(((j - 2) >> 1) & 1), a.err, 4))
+      *abort_flag = 1;  // the MMAs of chunk j - 2 have finished reading this A slot
     const int64_t e0 = static_cast<int64_t>(c) * kXpK + 2 * lane;
     const bool v0 = e0 < a.E, v1 = e0 + 1 < a.E;
-    const float4 w0 = v0 ? reinterpret_cast<const float4*>(a.conv_w)[e0] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 w1 = v1 ? reinterpret_cast<const float4*>(a.conv_w)[e0 + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float b0 = v0 ? a.conv_b[e0] : 0.0f, b1 = v1 ? a.conv_b[e0 + 1] : 0.0f;
-    const uint32_t* xt = reinterpret_cast<const uint32_t*>(smem + S::kX + s * S::kXBytes);
-    unsigned char* At = smem + S::kA + s * S::kABytes;
+    const uint32_t* xt = reinterpret_cast<const uint32_t*>(smem + S::kX + (j % kXpStages) * S::kXBytes);
+    unsigned char* At = smem + S::kA + (j & 1) * S::kABytes;
     // window = tile rows r, r+1, r+2 (tokens t0 + r - 3 ..); rows before token 0 are
     // zero-filled by TMA and replaced by the incoming conv cache when there is one
     const int r0 = 32 * warp;
@@ -151,8 +178,10 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
     for (int i = 0; i < 32; ++i) {
       const int r = r0 + i;
       const float2 x3 = unpack_bf16x2(xt[(r + 3) * 32 + lane]);
-      const float c0 = fmaf(w0.w, x3.x, fmaf(w0.z, x2.x, fmaf(w0.y, x1.x, fmaf(w0.x, x0.x, b0))));
-      const float c1 = fmaf(w1.w, x3.y, fmaf(w1.z, x2.y, fmaf(w1.y, x1.y, fmaf(w1.x, x0.y, b1))));
+      const float c0 =
+          fmaf(cw.w0.w, x3.x, fmaf(cw.w0.z, x2.x, fmaf(cw.w0.y, x1.x, fmaf(cw.w0.x, x0.x, cw.b0))));
+      const float c1 =
+          fmaf(cw.w1.w, x3.y, fmaf(cw.w1.z, x2.y, fmaf(cw.w1.y, x1.y, fmaf(cw.w1.x, x0.y, cw.b1))));
       const uint32_t u = pack_bf16x2(v0 ? silu(c0) : 0.0f, v1 ? silu(c1) : 0.0f);
       // element (row r, k = 2 lane) of the 128-byte swizzled K-major tile
       *reinterpret_cast<uint32_t*>(At + r * 128 + ((((lane >> 2) ^ (r & 7))) << 4) + ((lane & 3) << 2)) = u;
@@ -163,47 +192,71 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
     if (*abort_flag) break;  // a wait gave up: stop queueing work (every thread sees the flag here)
     if (tid == 0) {
       tcgen05_fence_after();
-      const uint32_t a_base = sb + S::kA + s * S::kABytes, w_base = sb + S::kW + s * S::kWBytes;
+      const uint32_t a_base = sb + S::kA + (j & 1) * S::kABytes;
+      const uint32_t w_base = sb + S::kW + (j % kXpStages) * S::kWBytes;
 #pragma unroll
       for (int kk = 0; kk < kXpK / 16; ++kk)
         umma_f16_ss(tmem, umma_desc_k_sw128(a_base + 32 * kk), umma_desc_k_sw128(w_base + 32 * kk), kXpIdesc,
-                    c > 0 || kk > 0);
-      umma_commit(done(s));
-      issued = c;
-      // chunk c + 1 refills the stage chunk c - 1 used: wait for its MMAs first
-      if (c >= 1 && c + 1 < nk) {
-        if (mbar_wait_bounded(done((c - 1) & 1), static_cast<uint32_t>(((c - 1) >> 1) & 1), a.err, 4))
-          issue(c + 1);
+                    j > 0 || kk > 0);
+      umma_commit(done(j));
+      issued = j;
+      // chunk j + 2 refills the ring slot chunk j - 1 used: wait for those MMAs first
+      if (j >= 1 && j + 2 < nloc) {
+        if (mbar_wait_bounded(done(j - 1), static_cast<uint32_t>(((j - 1) >> 1) & 1), a.err, 5))
+          issue(j + 2);
         else
           *abort_flag = 1;
       }
     }
+    cw = cw_next;
   }
-  // Every thread waits (bounded) for the last MMAs thread 0 committed; thread 0
-  // publishes which chunk that was.
+  // Every thread waits (bounded) for the last MMAs thread 0 committed.
   volatile int* last_slot = reinterpret_cast<volatile int*>(smem + S::kLast);
   if (tid == 0) *last_slot = issued;
   __syncthreads();
   const int last = *last_slot;
-  if (last >= 0) mbar_wait_bounded(done(last & 1), static_cast<uint32_t>((last >> 1) & 1), a.err, 5);
+  if (last >= 0) mbar_wait_bounded(done(last), static_cast<uint32_t>((last >> 1) & 1), a.err, 6);
   tcgen05_fence_after();
 
-  float v[kXpN];
+  // This CTA's partial [128 tokens][48] tile into shared memory (the x ring is free).
+  float* P = reinterpret_cast<float*>(smem + S::kP);
+  {
+    const int row = 32 * warp + lane;
 #pragma unroll
-  for (int j = 0; j < kXpN / 16; ++j) {
-    uint32_t r[16];
-    tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 16 * j, r);
-    tmem_ld_wait();
+    for (int jj = 0; jj < kXpN / 16; ++jj) {
+      uint32_t r[16];
+      if (last >= 0) {
+        tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 16 * jj, r);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-    for (int q = 0; q < 16; ++q) v[16 * j + q] = __uint_as_float(r[q]);
+        for (int q = 0; q < 16; ++q) r[q] = 0u;  // no channel range here: contributes zeros
+      }
+      float4* dst = reinterpret_cast<float4*>(P + row * kXpN + 16 * jj);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                             __uint_as_float(r[4 * q + 3]));
+    }
   }
-  const int64_t t = t0 + 32 * warp + lane;
-  if (t < a.L) {
-    float4* bc = reinterpret_cast<float4*>(a.bc + (static_cast<int64_t>(seq) * a.L + t) * 32);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) bc[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    a.dt_raw[static_cast<int64_t>(seq) * a.L + t] = v[2 * 16];
+  cluster_sync();
+  // CTA `rank` sums the cluster's partials, in rank order, for its share of the tokens.
+  const int per = kXpTok / split;
+  for (int idx = tid; idx < per * kXpOut; idx += kXpThreads) {
+    const int tl = rank * per + idx / kXpOut, o = idx % kXpOut;
+    const uint32_t addr = sb + S::kP + static_cast<uint32_t>((tl * kXpN + o) * 4);
+    float sum = 0.0f;
+    for (int q = 0; q < split; ++q) sum += ld_shared_cluster_f32(addr, static_cast<uint32_t>(q));
+    const int64_t t = t0 + tl;
+    if (t < a.L) {
+      const int64_t row = static_cast<int64_t>(seq) * a.L + t;
+      if (o < 32)
+        a.bc[row * 32 + o] = sum;
+      else
+        a.dt_raw[row] = sum;
+    }
   }
+  cluster_sync();  // the partials stay alive until every CTA of the cluster has read them
   tcgen05_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -238,7 +291,8 @@ bool bf16_map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 }
 
 // x = the first E columns of xz [b][L][2E] (bf16); W_x [33][E] (bf16).
-cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, int64_t batch, cudaStream_t st) {
+cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, int64_t batch, int num_sms,
+                         cudaStream_t st) {
   CUtensorMap mx, mw;
   const uint64_t E = static_cast<uint64_t>(a.E), L = static_cast<uint64_t>(a.L);
   if (!bf16_map3(&mx, xz, E, L, static_cast<uint64_t>(batch), 2 * E * 2, L * 2 * E * 2, kXpK, kXpTok + 3,
@@ -250,7 +304,24 @@ cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, in
   if (err != cudaSuccess) return err;
   const int64_t gx = (a.L + kXpTok - 1) / kXpTok;
   if (gx > 0x7fffffff || batch > 65535) return cudaErrorInvalidConfiguration;
-  xproj_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(batch)), kXpThreads, smem, st>>>(mx, mw, a);
+  // Split the channels over a cluster until the grid covers two CTAs per SM.
+  const int64_t tiles = gx * batch, nk = (a.E + kXpK - 1) / kXpK;
+  int split = 1;
+  while (split < kXpMaxSplit && 2 * split <= nk && tiles * split < 2 * static_cast<int64_t>(num_sms)) split *= 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(gx), static_cast<unsigned>(batch), static_cast<unsigned>(split));
+  cfg.blockDim = dim3(kXpThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(split);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, xproj_kernel, mx, mw, a);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
@@ -410,7 +481,9 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   xa.E = E;
   xa.err = ssm::device_error_ptr();
   if (!xa.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
-  cudaError_t err = ssm::launch_xproj(xa, xz, proj->w_x, b, cs);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaError_t err = ssm::launch_xproj(xa, xz, proj->w_x, b, sms, cs);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "x_proj launch: %s", cudaGetErrorString(err));
   // the core, on x and z in place in xz
   cd.x_tok_stride = cd.z_tok_stride = 2 * E;

@@ -2,12 +2,14 @@
 
     python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL G N NPOLY] [E]
     python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
+    python -m selective_state_space_depthwise_b200.profile_cases block NAME [L]
 
 prefill: three launches of the named workload's prefill (optionally shortened
 to L tokens, optionally with an explicit launch shape and E channels); decode: a 4-token
 prompt, then three decode steps at the decode workload's shape (batch 256,
-E=7680, 252 MB of state). Inputs are drawn on the GPU; a capture skips the
-first two launches (ncu -s 2 -c 1 -k regex:...).
+E=7680, 252 MB of state); block: three block forwards of the named block
+workload (optionally L tokens). Inputs are drawn on the GPU; a capture skips the
+first two launches of the kernel it selects (ncu -s 2 -c 1 -k regex:...).
 """
 from __future__ import annotations
 
@@ -50,12 +52,26 @@ def decode_case(batch: int = 256):
     print("decode ok", float(y.float().abs().mean()))
 
 
+def block_case(name: str, L: int = 0):
+    w, d_model = W.BLOCK_WORKLOADS[name]
+    if L > 0:
+        w = w.scaled(seqlen=L)
+    inp = W.make_block_inputs(w, d_model, device="cuda", gen_device="cuda")
+    proj = {k: inp[k] for k in api.PROJ_NAMES}
+    for _ in range(3):
+        out, _, _ = api.block_forward(inp["hidden"], inp, proj)
+    torch.cuda.synchronize()
+    print("block ok", name, w.seqlen, float(out.float().abs().mean()))
+
+
 if __name__ == "__main__":
     if sys.argv[1] == "prefill":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
         shape = tuple(int(v) for v in sys.argv[4:8]) if len(sys.argv) > 7 else None
         E = int(sys.argv[8]) if len(sys.argv) > 8 else 0
         prefill_case(sys.argv[2], L, shape, E)
+    elif sys.argv[1] == "block":
+        block_case(sys.argv[2], int(sys.argv[3]) if len(sys.argv) > 3 else 0)
     elif sys.argv[1] == "decode":
         decode_case(int(sys.argv[2]) if len(sys.argv) > 2 else 256)
     else:

@@ -137,6 +137,8 @@ def make_inputs(w: Workload, device="cpu", gen_device=None) -> dict:
 BLOCK_WORKLOADS = {
     "block_axon_layer": (Workload("block_axon_layer", batch=1, seqlen=2048, d_inner=7680, seed=5,
                                   note="AxonSSMBlock forward at the Axon layer shape, D = 2560"), 2560),
+    "block_long_context": (Workload("block_long_context", batch=1, seqlen=65536, d_inner=7680, seed=6,
+                                    note="AxonSSMBlock forward over a 64K-token context, D = 2560"), 2560),
 }
 
 
