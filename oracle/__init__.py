@@ -210,3 +210,38 @@ def prefill_sampled(x, z, B, C, dt_raw, conv_w, conv_b, w_dt, dt_bias, A_log, D,
     conv_w, conv_b, w_dt, dt_bias, A_log, D = map(_f64, (conv_w, conv_b, w_dt, dt_bias, A_log, D))
     return channels(cols(x), cols(z), B, C, dt_raw, bs, conv_w[es], conv_b[es], w_dt[es], dt_bias[es], A_log[es], D[es],
                     hist=hist, h0=h0, lo=lo, hi=hi, disc=disc, threads=threads)
+
+
+def ssd_chunk_scan(cb, x, dt, dA_cumsum, C, prev_states, D=None):
+    """Output of the Mamba-2 chunk scan, "What is the Mamba model?" (velog,
+    Texnee), "chunkscan" section, in float64, for every position l of chunk c
+    and head h (group g = h // (nheads / ngroups)):
+
+      out[l] = sum_{s <= l} cb[l, s] exp(dA[l] - dA[s]) dt[s] x[s]      (intra-chunk scan)
+             + exp(dA[l]) C[l] . prev_states                           (state carried into the chunk)
+             + D x[l]                                                  (skip)
+
+    cb: [b, nchunks, ngroups, cs, cs]; x: [b, L, nheads, headdim];
+    dt, dA_cumsum: [b, nheads, nchunks, cs]; C: [b, L, ngroups, dstate];
+    prev_states: [b, nchunks, nheads, headdim, dstate]; D: [nheads] or None.
+    The contractions are library einsums (a plain step each). Returns out
+    [b, L, nheads, headdim]."""
+    cb, x, dt, dA_cumsum, C, prev_states = map(_f64, (cb, x, dt, dA_cumsum, C, prev_states))
+    b, L, H, P = x.shape
+    _, nc, G, cs, _ = cb.shape
+    assert L == nc * cs and H % G == 0
+    rep = H // G
+    g_of = np.arange(H) // rep
+    cbh = cb[:, :, g_of]                                    # [b, c, h, l, s]
+    Ch = C[:, :, g_of].reshape(b, nc, cs, H, -1)            # [b, c, l, h, n]
+    xc = x.reshape(b, nc, cs, H, P)                         # [b, c, s, h, p]
+    seg = dA_cumsum[..., :, None] - dA_cumsum[..., None, :]  # [b, h, c, l, s]
+    causal = np.tril(np.ones((cs, cs), dtype=bool))
+    w = np.where(causal, cbh * np.exp(seg).transpose(0, 2, 1, 3, 4), 0.0)  # [b, c, h, l, s]
+    w = w * dt.transpose(0, 2, 1, 3)[:, :, :, None, :]      # times dt[s]
+    out = np.einsum("bchls,bcshp->bclhp", w, xc)
+    out += np.einsum("bclhn,bchpn->bclhp", Ch, prev_states) * np.exp(dA_cumsum).transpose(0, 2, 3, 1)[..., None]
+    out = out.reshape(b, L, H, P)
+    if D is not None:
+        out = out + _f64(D)[None, None, :, None] * x
+    return out
