@@ -303,6 +303,42 @@ ssm_status ssm_block_forward(const ssm_block_dims *dims, const ssm_weights *w, c
 /* Workspace bytes of ssm_block_forward for `dims` (0 for invalid dims). */
 size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
 
+/*
+ * ssm_ssd_chunk_scan -- the output of the Mamba-2 (SSD) chunk scan, "What is
+ * the Mamba model?" (velog, Texnee), "chunkscan" section. For batch b, chunk c,
+ * head h (group g = h / (nheads / ngroups)) and position l of the chunk:
+ *
+ *   out[l] = sum_{s <= l} cb[l, s] exp(dA[l] - dA[s]) dt[s] x[s]
+ *          + exp(dA[l]) C[l] . prev_states
+ *          + D[h] x[l]
+ *
+ * Arguments. Dense row-major device tensors; bf16 = SSM_BF16 storage.
+ *   cb           [b, nchunks, ngroups, cs, cs] bf16   (the chunk's C B^T scores)
+ *   x            [b, L, nheads, headdim] bf16
+ *   dt           [b, nheads, nchunks, cs] fp32
+ *   dA_cumsum    [b, nheads, nchunks, cs] fp32        (within-chunk cumulative sum of dt A)
+ *   C            [b, L, ngroups, dstate] bf16
+ *   prev_states  [b, nchunks, nheads, headdim, dstate] bf16
+ *   D            [nheads] fp32, or NULL for no skip
+ *   out          [b, L, nheads, headdim] bf16; must not overlap the inputs
+ * L = nchunks * cs. The built shape is cs = 128, headdim = 64, dstate = 128
+ * (SSM_ERR_UNSUPPORTED otherwise). nheads must be a multiple of ngroups, and
+ * every pointer 16-byte aligned.
+ *
+ * Computation. Per (b, c, h) one CTA:
+ *  - scores = masked cb * exp(dA[l] - dA[s]) * dt[s] in bf16, times x;
+ *  - exp(dA[l]) C[l] in bf16, times prev_states^T;
+ * both as tcgen05 MMAs into one fp32 TMEM accumulator, then + D x and a bf16
+ * store. The exponents are <= 0 for s <= l, so nothing overflows.
+ */
+typedef struct {
+  int64_t batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size;
+} ssm_ssd_dims;
+
+ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims *dims, const void *cb, const void *x, const float *dt,
+                              const float *dA_cumsum, const void *C, const void *prev_states, const float *D,
+                              void *out, void *stream);
+
 /* Reads and clears the device error word that kernels set when a bounded
  * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed. */
 ssm_status ssm_check_device_error(void *stream);

@@ -28,6 +28,7 @@ EXPORTED = (
     "ssm_prefill_host_static",
     "ssm_block_forward",
     "ssm_block_workspace_bytes",
+    "ssm_ssd_chunk_scan",
     "ssm_decode_step",
     "ssm_check_device_error",
     "ssm_status_string",
@@ -78,6 +79,11 @@ class SsmBlockWeights(ctypes.Structure):
     _fields_ = [("w_in", ctypes.c_void_p), ("w_x", ctypes.c_void_p), ("w_out", ctypes.c_void_p)]
 
 
+class SsmSsdDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate",
+                                             "chunk_size")]
+
+
 class SsmWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")]
 
@@ -123,6 +129,8 @@ def load(path: str = LIB_PATH):
     lib.ssm_block_forward.restype = st
     lib.ssm_block_workspace_bytes.argtypes = [bdims_p]
     lib.ssm_block_workspace_bytes.restype = sz
+    lib.ssm_ssd_chunk_scan.argtypes = [ctypes.POINTER(SsmSsdDims)] + [p] * 8 + [p]
+    lib.ssm_ssd_chunk_scan.restype = st
     lib.ssm_decode_step.argtypes = [dims_p, w_p] + [p] * 8 + [p]
     lib.ssm_decode_step.restype = st
     lib.ssm_check_device_error.argtypes = [p]

@@ -244,6 +244,38 @@ def block_forward(hidden, params, proj, *, conv_cache_in=None, ssm_state_in=None
     return out, conv_cache_out, ssm_state_out
 
 
+def ssd_chunk_scan(cb, x, dt, dA_cumsum, C, prev_states, D=None, *, out=None, stream=None):
+    """Mamba-2 chunk-scan output (ssm_ssd_chunk_scan). cb [b, nc, G, cs, cs],
+    x [b, L, H, P], C [b, L, G, N], prev_states [b, nc, H, P, N]: bf16;
+    dt, dA_cumsum [b, H, nc, cs] and D [H]: fp32. Returns out [b, L, H, P] bf16."""
+    lib = _lib.load()
+    b, L, H, P = x.shape
+    _, nc, G, cs, _ = cb.shape
+    N = C.shape[-1]
+    dev = x.device
+    for n, t in (("cb", cb), ("x", x), ("dt", dt), ("dA_cumsum", dA_cumsum), ("C", C), ("prev_states", prev_states),
+                 ("D", D), ("out", out)):
+        _need_cuda(n, t, dev)
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    for n, t in (("cb", cb), ("x", x), ("C", C), ("prev_states", prev_states)):
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{n} must be bfloat16")
+    for n, t in (("dt", dt), ("dA_cumsum", dA_cumsum), ("D", D)):
+        if t is not None and t.dtype != torch.float32:
+            raise ValueError(f"{n} must be float32")
+    if (cb.shape != (b, nc, G, cs, cs) or C.shape != (b, L, G, N) or prev_states.shape != (b, nc, H, P, N)
+            or dt.shape != (b, H, nc, cs) or dA_cumsum.shape != dt.shape or (D is not None and D.shape != (H,))):
+        raise ValueError("shape mismatch between the chunk-scan operands")
+    if out is None:
+        out = torch.empty_like(x)
+    d = _lib.SsmSsdDims(b, L, H, P, G, N, cs)
+    st = lib.ssm_ssd_chunk_scan(ctypes.byref(d), _ptr(cb), _ptr(x), _ptr(dt), _ptr(dA_cumsum), _ptr(C),
+                                _ptr(prev_states), _ptr(D), _ptr(out), _stream(stream))
+    _lib.check(st)
+    return out
+
+
 def decode_step(x, z, B, C, dt_raw, params, conv_cache, ssm_state, *, y=None, dt_min=1e-4, dt_max=1.0,
                 discretization="euler", stream=None):
     """One-token block core. x, z: [b, E] (last dim contiguous); B, C: [b, 16];

@@ -1,0 +1,304 @@
+// ssd.cu -- the output of the Mamba-2 (SSD) chunk scan for sm_100a: "What is
+// the Mamba model?" (velog, Texnee), "chunkscan" section. For batch b, chunk
+// c, head h (group g) and position l of the chunk:
+//
+//   out[l] = sum_{s <= l} cb[l, s] exp(dA[l] - dA[s]) dt[s] x[s]     (intra-chunk)
+//          + exp(dA[l]) C[l] . prev_states                          (carried state)
+//          + D[h] x[l]                                              (skip)
+//
+// Both sums are dense contractions and run on the tensor cores. One CTA per
+// (b, c, h), 128 threads, thread l owning row l of the chunk (TMEM lane l):
+//  1. TMA brings, 128-byte swizzled, the cb tile [l][s] (two 64-column
+//     atoms), the C tile [l][n] (two atoms), the x tile [s][p] and the
+//     prev_states tile [p][n] (two atoms) on one mbarrier, while the threads
+//     stage the chunk's dA and dt in shared memory;
+//  2. each thread turns row l of the cb tile, in place, into the masked and
+//     decayed scores cb[l, s] exp(dA[l] - dA[s]) dt[s] (bf16; chunks entirely
+//     above the diagonal of the warp's rows are written as zeros without any
+//     exponential) and scales row l of the C tile by exp(dA[l]): the TMA
+//     layouts are already the MMA's K-major operand layouts;
+//  3. one thread issues eight tcgen05 MMAs scores x x (x as an MN-major B
+//     operand) and eight MMAs (exp(dA) C) x prev_states^T into one 128 x 64
+//     fp32 TMEM accumulator;
+//  4. each warp reads its 32 lanes back, adds D x, and the bf16 tile leaves
+//     by TMA store from the (now free) cb buffer.
+// Every mbarrier wait is bounded; ~97 KB of shared memory lets two CTAs share
+// an SM so that one's loads overlap the other's arithmetic.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <initializer_list>
+
+#include "sm100_ptx.cuh"
+#include "ssm.h"
+#include "ssm_internal.h"
+#include "ssm_math.cuh"
+#include "tma_map.cuh"
+
+namespace ssm {
+namespace {
+
+constexpr int kCs = 128;  // chunk length: MMA M and the K of the intra-chunk term
+constexpr int kHd = 64;   // head dim: MMA N
+constexpr int kDs = 128;  // state dim: the K of the carried-state term
+constexpr int kSsdThreads = 128;
+constexpr uint32_t kSsdTmemCols = 64;
+
+struct SsdSmem {
+  static constexpr int kAtomRows128 = kCs * 128;   // one 64-column atom of a 128-row tile
+  static constexpr int kAtomRows64 = kHd * 128;    // one 64-column atom of a 64-row tile
+  static constexpr int kCb = 0;                    // cb -> scores (A of MMA 1) -> out tile
+  static constexpr int kC = 2 * kAtomRows128;      // C -> exp(dA) C (A of MMA 2)
+  static constexpr int kX = 4 * kAtomRows128;      // x [s][p] (B of MMA 1, MN-major)
+  static constexpr int kPrev = kX + kAtomRows128;  // prev_states [p][n] (B of MMA 2, K-major)
+  static constexpr int kDA = kPrev + 2 * kAtomRows64;
+  static constexpr int kDt = kDA + kCs * 4;
+  static constexpr int kBar = kDt + kCs * 4;       // full, done
+  static constexpr int kTmemSlot = kBar + 16;
+  static constexpr int kTotal = kTmemSlot + 16;
+  static constexpr uint32_t kTx = static_cast<uint32_t>(5 * kAtomRows128 + 2 * kAtomRows64);
+  static_assert(kC % 1024 == 0 && kX % 1024 == 0 && kPrev % 1024 == 0, "swizzled tiles need 1 KB");
+};
+
+// bf16 x bf16 -> fp32, M = 128, N = 64, A K-major, B K-major or MN-major.
+__host__ __device__ constexpr uint32_t ssd_idesc(bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) |
+         (static_cast<uint32_t>(kHd >> 3) << 17) | (static_cast<uint32_t>(kCs >> 4) << 24);
+}
+
+struct SsdArgs {
+  const float* dt;         // [b][H][nc][cs]
+  const float* dA;         // [b][H][nc][cs]
+  const float* D;          // [H] or null
+  int64_t nheads, nchunks, ngroups;
+  int* err;
+};
+
+// Byte offset of 16-byte chunk j (0..7) of row r in a 128-byte swizzled atom.
+__device__ __forceinline__ int sw128(int r, int j) { return r * 128 + ((j ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ void unpack8(uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 p;
+    *reinterpret_cast<uint32_t*>(&p) = w[i];
+    const float2 q = __bfloat1622float2(p);
+    f[2 * i] = q.x, f[2 * i + 1] = q.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 p = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
+    const __grid_constant__ CUtensorMap map_cb, const __grid_constant__ CUtensorMap map_x,
+    const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_prev,
+    const __grid_constant__ CUtensorMap map_out, const SsdArgs a) {
+  using S = SsdSmem;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sb = smem_u32(smem);
+  const int tid = threadIdx.x, l = tid;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
+  const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
+  const int g = static_cast<int>(h / (a.nheads / a.ngroups));
+  const uint32_t full = sb + S::kBar, done = sb + S::kBar + 8;
+  if (tid == 0) {
+    mbar_init(full, 1);
+    mbar_init(done, 1);
+    mbar_fence_init();
+    prefetch_tensormap(&map_cb);
+    prefetch_tensormap(&map_x);
+    prefetch_tensormap(&map_c);
+    prefetch_tensormap(&map_prev);
+    mbar_arrive_expect_tx(full, S::kTx);
+    const int zc = static_cast<int>((static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g);
+    const int zp = static_cast<int>((static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h);
+#pragma unroll
+    for (int at = 0; at < 2; ++at) {
+      tma_load_3d(sb + S::kCb + at * S::kAtomRows128, &map_cb, 64 * at, 0, zc, full);
+      tma_load_4d(sb + S::kC + at * S::kAtomRows128, &map_c, 64 * at, g, c * kCs, b, full);
+      tma_load_3d(sb + S::kPrev + at * S::kAtomRows64, &map_prev, 64 * at, 0, zp, full);
+    }
+    tma_load_4d(sb + S::kX, &map_x, 0, h, c * kCs, b, full);
+  }
+  if (warp == 0) {
+    tmem_alloc(sb + S::kTmemSlot, kSsdTmemCols);
+    tmem_relinquish();
+  }
+  float* sdA = reinterpret_cast<float*>(smem + S::kDA);
+  float* sdt = reinterpret_cast<float*>(smem + S::kDt);
+  {
+    const int64_t row = ((static_cast<int64_t>(b) * a.nheads + h) * a.nchunks + c) * kCs;
+    sdA[tid] = a.dA[row + tid];
+    sdt[tid] = a.dt[row + tid];
+  }
+  const float Dh = a.D ? a.D[h] : 0.0f;
+  tcgen05_fence_before();
+  __syncthreads();
+  tcgen05_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
+  mbar_wait_bounded(full, 0u, a.err, 7);
+
+  // 1. Row l of the cb tile -> masked, decayed, dt-weighted scores (in place).
+  const float dAl = sdA[l];
+  const int warp_max_l = 32 * warp + 31;
+#pragma unroll
+  for (int at = 0; at < 2; ++at) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int s0 = 64 * at + 8 * j;
+      uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
+      if (s0 > warp_max_l) {  // above the diagonal for every row of this warp
+        *p = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      float f[8];
+      unpack8(*p, f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int s = s0 + q;
+        f[q] = s <= l ? f[q] * ex2_approx((dAl - sdA[s]) * kLog2e) * sdt[s] : 0.0f;
+      }
+      *p = pack8(f);
+    }
+  }
+  // 2. Row l of the C tile times exp(dA[l]) (in place).
+  const float el = ex2_approx(dAl * kLog2e);
+#pragma unroll
+  for (int at = 0; at < 2; ++at) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint4* p = reinterpret_cast<uint4*>(smem + S::kC + at * S::kAtomRows128 + sw128(l, j));
+      float f[8];
+      unpack8(*p, f);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) f[q] *= el;
+      *p = pack8(f);
+    }
+  }
+  fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
+  __syncthreads();
+
+  // 3. The two contractions into one accumulator.
+  if (tid == 0) {
+    tcgen05_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < kCs / 16; ++kk)  // scores[l][s] x x[s][p]: s in steps of 16 rows of x
+      umma_f16_ss(tmem, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+                  umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < kDs / 16; ++kk)  // (exp(dA) C)[l][n] x prev_states[p][n]^T
+      umma_f16_ss(tmem, umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+                  umma_desc_k_sw128(sb + S::kPrev + (kk >> 2) * S::kAtomRows64 + (kk & 3) * 32), ssd_idesc(false),
+                  true);
+    umma_commit(done);
+  }
+  mbar_wait_bounded(done, 0u, a.err, 8);
+  tcgen05_fence_after();
+
+  // 4. + D x, bf16, into the out tile (the cb buffer, free now) and out by TMA.
+#pragma unroll
+  for (int jj = 0; jj < kHd / 16; ++jj) {
+    uint32_t r[16];
+    tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 16 * jj, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int j = 2 * jj + half;  // 16-byte chunk of row l: p = 8 j .. 8 j + 7
+      float xv[8], o[8];
+      unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(l, j)), xv);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o[q] = fmaf(Dh, xv[q], __uint_as_float(r[8 * half + q]));
+      *reinterpret_cast<uint4*>(smem + S::kCb + sw128(l, j)) = pack8(o);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    tma_store_4d(&map_out, sb + S::kCb, 0, h, c * kCs, b);
+    bulk_commit();
+    bulk_wait_read<0>();  // the tile stays in shared memory until the store has read it
+  }
+  tcgen05_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tcgen05_fence_after();
+    tmem_dealloc(tmem, kSsdTmemCols);
+  }
+}
+
+bool bf16_map(CUtensorMap* m, int rank, const void* base, std::initializer_list<uint64_t> dims,
+              std::initializer_list<uint64_t> strides, std::initializer_list<uint32_t> box) {
+  uint64_t d[5], s[4];
+  uint32_t bx[5];
+  int i = 0;
+  for (uint64_t v : dims) d[i++] = v;
+  i = 0;
+  for (uint64_t v : strides) s[i++] = v;
+  i = 0;
+  for (uint32_t v : box) bx[i++] = v;
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, d, s, bx, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+}  // namespace ssm
+
+extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* cb, const void* x, const float* dt,
+                                         const float* dA_cumsum, const void* C, const void* prev_states,
+                                         const float* D, void* out, void* stream) {
+  using ssm::fail;
+  if (!dims) return fail(SSM_ERR_INVALID_ARG, "dims is NULL");
+  const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim, G = dims->ngroups;
+  const int64_t N = dims->dstate, cs = dims->chunk_size;
+  if (cs != ssm::kCs || P != ssm::kHd || N != ssm::kDs)
+    return fail(SSM_ERR_UNSUPPORTED, "chunk_size %lld, headdim %lld, dstate %lld: the built shape is 128, 64, 128",
+                (long long)cs, (long long)P, (long long)N);
+  if (b <= 0 || b > 65535 || H <= 0 || H > 0x7fffffff || G <= 0 || H % G != 0)
+    return fail(SSM_ERR_INVALID_ARG, "need 0 < batch <= 65535, nheads > 0 and nheads a multiple of ngroups");
+  if (L <= 0 || L % cs != 0 || L / cs > 65535)
+    return fail(SSM_ERR_INVALID_ARG, "seqlen must be a positive multiple of chunk_size, at most 65535 chunks");
+  const void* ptrs[8] = {cb, x, dt, dA_cumsum, C, prev_states, out, D};
+  const char* names[8] = {"cb", "x", "dt", "dA_cumsum", "C", "prev_states", "out", "D"};
+  for (int i = 0; i < 8; ++i) {
+    if (!ptrs[i] && i < 7) return fail(SSM_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (ptrs[i] && !ssm::aligned(ptrs[i], 16)) return fail(SSM_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  if (out == x || out == cb || out == C || out == prev_states)
+    return fail(SSM_ERR_INVALID_ARG, "out must not alias an input");
+  const int64_t nc = L / cs;
+  CUtensorMap mcb, mx, mc, mp, mo;
+  const uint64_t e2 = 2;
+  const bool ok =
+      ssm::bf16_map(&mcb, 3, cb, {uint64_t(cs), uint64_t(cs), uint64_t(b * nc * G)}, {cs * e2, cs * cs * e2},
+                    {64, 128, 1}) &&
+      ssm::bf16_map(&mx, 4, x, {uint64_t(P), uint64_t(H), uint64_t(L), uint64_t(b)},
+                    {P * e2, H * P * e2, L * H * P * e2}, {64, 1, 128, 1}) &&
+      ssm::bf16_map(&mc, 4, C, {uint64_t(N), uint64_t(G), uint64_t(L), uint64_t(b)},
+                    {N * e2, G * N * e2, L * G * N * e2}, {64, 1, 128, 1}) &&
+      ssm::bf16_map(&mp, 3, prev_states, {uint64_t(N), uint64_t(P), uint64_t(b * nc * H)}, {N * e2, P * N * e2},
+                    {64, 64, 1}) &&
+      ssm::bf16_map(&mo, 4, out, {uint64_t(P), uint64_t(H), uint64_t(L), uint64_t(b)},
+                    {P * e2, H * P * e2, L * H * P * e2}, {64, 1, 128, 1});
+  if (!ok) return fail(SSM_ERR_CUDA, "tensor map encoding failed");
+  ssm::SsdArgs a{dt, dA_cumsum, D, H, nc, G, ssm::device_error_ptr()};
+  if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
+  const int smem = ssm::SsdSmem::kTotal + 1024;
+  cudaError_t err =
+      cudaFuncSetAttribute(ssm::ssd_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(err));
+  ssm::ssd_chunk_scan_kernel<<<dim3(static_cast<unsigned>(H), static_cast<unsigned>(nc), static_cast<unsigned>(b)),
+                               ssm::kSsdThreads, smem, static_cast<cudaStream_t>(stream)>>>(mcb, mx, mc, mp, mo, a);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "chunk-scan launch: %s", cudaGetErrorString(err));
+  return fail(SSM_OK, "");
+}

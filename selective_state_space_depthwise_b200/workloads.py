@@ -159,3 +159,41 @@ def make_block_inputs(w: Workload, d_model: int, device="cpu", gen_device=None) 
     W_out = scale(_randn_chunked((d_model, E), g, gen_device, torch.bfloat16), E ** -0.5)
     p.update(hidden=hidden.to(device), W_in=W_in.to(device), W_x=W_x.to(device), W_out=W_out.to(device))
     return p
+
+
+# ---------------------------------------------------------- chunk scan ---
+# The Mamba-2 chunk scan of "What is the Mamba model?" ("chunkscan"): the pages
+# give the operation and a chunk length of 128 as their example, no sizes; these
+# are a synthetic multi-head layout with one B/C group.
+SSD_WORKLOADS = {
+    "ssd_small": dict(batch=2, seqlen=384, nheads=4, headdim=64, ngroups=2, dstate=128, chunk_size=128, seed=7),
+    "ssd_chunk_scan": dict(batch=8, seqlen=4096, nheads=80, headdim=64, ngroups=1, dstate=128, chunk_size=128,
+                           seed=8),
+}
+
+
+def make_ssd_inputs(spec: dict, device="cpu") -> dict:
+    """Seeded chunk-scan inputs drawn from one SSD model so that the values are
+    those of a real layer: x ~ N(0,1); B, C ~ N(0,1)/sqrt(dstate) per group;
+    dt = softplus(N(-2, 1)) per (token, head); A_h = -exp(U(ln 1/16, ln 1/2))
+    (a few units of decay over a chunk, so the carried state matters);
+    dA_cumsum = the within-chunk cumulative sum of dt A_h; cb = C B^T per chunk
+    (fp32, then bf16); prev_states ~ N(0, 1/4); D ~ U(0.5, 1.5). bf16 for cb, x,
+    C, prev_states (RNE from fp32), fp32 for dt, dA_cumsum, D. Drawn on `device`."""
+    g = torch.Generator(device=device).manual_seed(spec["seed"])
+    b, L, H, P = spec["batch"], spec["seqlen"], spec["nheads"], spec["headdim"]
+    G, N, cs = spec["ngroups"], spec["dstate"], spec["chunk_size"]
+    nc = L // cs
+    f32 = dict(device=device, dtype=torch.float32, generator=g)
+    x = torch.randn((b, L, H, P), **f32).to(torch.bfloat16)
+    B = (torch.randn((b, L, G, N), **f32) * N ** -0.5).to(torch.bfloat16)
+    C = (torch.randn((b, L, G, N), **f32) * N ** -0.5).to(torch.bfloat16)
+    dt = torch.nn.functional.softplus(torch.randn((b, H, nc, cs), **f32) - 2.0)
+    A = -torch.exp(torch.rand(H, **f32) * (math.log(0.5) - math.log(1 / 16)) + math.log(1 / 16))
+    dA_cumsum = torch.cumsum(dt * A[None, :, None, None], dim=-1)
+    Bc = B.float().reshape(b, nc, cs, G, N)
+    Cc = C.float().reshape(b, nc, cs, G, N)
+    cb = torch.einsum("bclgn,bcsgn->bcgls", Cc, Bc).to(torch.bfloat16).contiguous()
+    prev = (torch.randn((b, nc, H, P, N), **f32) * 0.5).to(torch.bfloat16)
+    D = torch.rand(H, **f32) + 0.5
+    return dict(cb=cb, x=x, dt=dt.contiguous(), dA_cumsum=dA_cumsum.contiguous(), C=C, prev_states=prev, D=D)
