@@ -395,6 +395,42 @@ def block_bench(name: str, bf16_peak: float, steps: int = 10, warmup: int = 3):
             "gpu_launches_per_step": 4}
 
 
+def ssd_bench(name: str, hbm_peak: float, bf16_peak: float, steps: int = 20, warmup: int = 3):
+    """The Mamba-2 chunk scan on device-resident inputs: us per call by CUDA
+    events; HBM roofline on the algorithmic bytes (read cb, x, dt, dA_cumsum, C,
+    prev_states, D once, write out once) and the tensor FLOPs of the two
+    contractions (2 cs cs P + 2 cs N P per chunk and head)."""
+    from selective_state_space_depthwise_b200 import api
+
+    spec = W.SSD_WORKLOADS[name]
+    inp = W.make_ssd_inputs(spec, device="cuda")
+    args = [inp[k] for k in ("cb", "x", "dt", "dA_cumsum", "C", "prev_states", "D")]
+    out = torch.empty_like(inp["x"])
+    for _ in range(warmup):
+        api.ssd_chunk_scan(*args, out=out)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        api.ssd_chunk_scan(*args, out=out)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    us = ev0.elapsed_time(ev1) * 1e3 / steps
+    b, L, H, P, G, N, cs = (spec[k] for k in ("batch", "seqlen", "nheads", "headdim", "ngroups", "dstate",
+                                             "chunk_size"))
+    nc = L // cs
+    nbytes = sum(t.numel() * t.element_size() for t in args) + out.numel() * out.element_size()
+    flops = 2.0 * b * nc * H * (cs * cs * P + cs * N * P)
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"workload": f"{name}: b={b} L={L} heads={H} headdim={P} groups={G} dstate={N} chunk={cs}",
+            "us_per_step": round(us, 2), "value": b * L * H / (us * 1e-6), "unit": "token-heads/s",
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": nbytes,
+                         "tensor_tflops": round(flops / (us * 1e-6) / 1e12, 1), "tensor_peak": bf16_peak},
+            "gpu_launches_per_step": 1}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,7 +441,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the decode sub-benchmark")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
-    ap.add_argument("--no-block", action="store_true", help="skip the block-forward sub-benchmark")
+    ap.add_argument("--no-block", action="store_true",
+                    help="skip the block-forward and chunk-scan sub-benchmarks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -479,6 +516,8 @@ def main():
             torch.cuda.empty_cache()
             bf16_peak = load_bf16_peak()
             extra["block"] = [block_bench(n, bf16_peak) for n in W.BLOCK_WORKLOADS]
+            torch.cuda.empty_cache()
+            extra["ssd_chunk_scan"] = ssd_bench("ssd_chunk_scan", hbm_peak, bf16_peak)
         if not args.no_cpu and world == 1:
             extra["cpu_baseline"] = cpu_baseline(w)
     if dist:

@@ -3,6 +3,7 @@
     python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL G N NPOLY] [E]
     python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
     python -m selective_state_space_depthwise_b200.profile_cases block NAME [L]
+    python -m selective_state_space_depthwise_b200.profile_cases ssd NAME
 
 prefill: three launches of the named workload's prefill (optionally shortened
 to L tokens, optionally with an explicit launch shape and E channels); decode: a 4-token
@@ -64,12 +65,22 @@ def block_case(name: str, L: int = 0):
     print("block ok", name, w.seqlen, float(out.float().abs().mean()))
 
 
+def ssd_case(name: str):
+    inp = W.make_ssd_inputs(W.SSD_WORKLOADS[name], device="cuda")
+    for _ in range(3):
+        out = api.ssd_chunk_scan(*(inp[k] for k in ("cb", "x", "dt", "dA_cumsum", "C", "prev_states", "D")))
+    torch.cuda.synchronize()
+    print("ssd ok", name, float(out.float().abs().mean()))
+
+
 if __name__ == "__main__":
     if sys.argv[1] == "prefill":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
         shape = tuple(int(v) for v in sys.argv[4:8]) if len(sys.argv) > 7 else None
         E = int(sys.argv[8]) if len(sys.argv) > 8 else 0
         prefill_case(sys.argv[2], L, shape, E)
+    elif sys.argv[1] == "ssd":
+        ssd_case(sys.argv[2])
     elif sys.argv[1] == "block":
         block_case(sys.argv[2], int(sys.argv[3]) if len(sys.argv) > 3 else 0)
     elif sys.argv[1] == "decode":
