@@ -6,24 +6,28 @@
 //          + exp(dA[l]) C[l] . prev_states                          (carried state)
 //          + D[h] x[l]                                              (skip)
 //
-// Both sums are dense contractions and run on the tensor cores. One CTA per
-// (b, c, h), 128 threads, thread l owning row l of the chunk (TMEM lane l):
-//  1. TMA brings, 128-byte swizzled, the cb tile [l][s] (two 64-column
-//     atoms), the C tile [l][n] (two atoms), the x tile [s][p] and the
-//     prev_states tile [p][n] (two atoms) on one mbarrier, while the threads
-//     stage the chunk's dA and dt in shared memory;
-//  2. each thread turns row l of the cb tile, in place, into the masked and
-//     decayed scores cb[l, s] exp(dA[l] - dA[s]) dt[s] (bf16; chunks entirely
-//     above the diagonal of the warp's rows are written as zeros without any
-//     exponential) and scales row l of the C tile by exp(dA[l]): the TMA
-//     layouts are already the MMA's K-major operand layouts;
-//  3. one thread issues eight tcgen05 MMAs scores x x (x as an MN-major B
-//     operand) and eight MMAs (exp(dA) C) x prev_states^T into one 128 x 64
-//     fp32 TMEM accumulator;
-//  4. each warp reads its 32 lanes back, adds D x, and the bf16 tile leaves
-//     by TMA store from the (now free) cb buffer.
-// Every mbarrier wait is bounded; ~97 KB of shared memory lets two CTAs share
-// an SM so that one's loads overlap the other's arithmetic.
+// Both sums are dense contractions and run on the tensor cores, each into its
+// own TMEM accumulator, so that the carried-state term needs no rescaled copy
+// of C and starts as soon as its operands land. One CTA per (b, c, h), 256
+// threads; ~100 KB of shared memory lets two CTAs share an SM:
+//  1. TMA brings, 128-byte swizzled, the C tile [l][n] and the prev_states tile
+//     [p][n] (two 64-column atoms each) on one mbarrier, and the cb tile [l][s]
+//     (two atoms) and the x tile [s][p] on a second one, while threads stage
+//     dA and dt;
+//  2. as soon as C and prev_states are in, one thread issues eight tcgen05 MMAs
+//     C x prev_states^T into accumulator 1;
+//  3. meanwhile thread s < 128 forms F[s] = exp(dA[s0] - dA[s]) dt[s] (s0 = s
+//     rounded down to a multiple of 8), and thread t turns the 64-column atom
+//     t / 128 of row l = t mod 128 of the cb tile, in place, into the scores
+//     cb[l, s] exp(dA[l] - dA[s0]) F[s] for s <= l, zero above (one exponential
+//     per row and 8-column group; the exponents are <= 0 or small, so nothing
+//     overflows): the TMA layout is already the MMA's K-major operand;
+//  4. one thread issues eight MMAs scores x x (x as an MN-major B operand) into
+//     accumulator 0 and commits both;
+//  5. warps w and w + 4 read lanes 32 (w mod 4) .. of columns 32 (w / 4) .. of
+//     both accumulators, form acc0 + exp(dA[l]) acc1 + D x, and the bf16 tile
+//     leaves by TMA store from the (now free) cb buffer.
+// Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -42,8 +46,8 @@ namespace {
 constexpr int kCs = 128;  // chunk length: MMA M and the K of the intra-chunk term
 constexpr int kHd = 64;   // head dim: MMA N
 constexpr int kDs = 128;  // state dim: the K of the carried-state term
-constexpr int kSsdThreads = 128;
-constexpr uint32_t kSsdTmemCols = 64;
+constexpr int kSsdThreads = 256;
+constexpr uint32_t kSsdTmemCols = 128;  // accumulator 0 (intra-chunk) at column 0, 1 (carried state) at 64
 
 struct SsdSmem {
   static constexpr int kAtomRows128 = kCs * 128;   // one 64-column atom of a 128-row tile
@@ -54,10 +58,12 @@ struct SsdSmem {
   static constexpr int kPrev = kX + kAtomRows128;  // prev_states [p][n] (B of MMA 2, K-major)
   static constexpr int kDA = kPrev + 2 * kAtomRows64;
   static constexpr int kDt = kDA + kCs * 4;
-  static constexpr int kBar = kDt + kCs * 4;       // full, done
-  static constexpr int kTmemSlot = kBar + 16;
+  static constexpr int kF = kDt + kCs * 4;
+  static constexpr int kBar = kF + kCs * 4;        // full_state, full_scores, done
+  static constexpr int kTmemSlot = kBar + 24;
   static constexpr int kTotal = kTmemSlot + 16;
-  static constexpr uint32_t kTx = static_cast<uint32_t>(5 * kAtomRows128 + 2 * kAtomRows64);
+  static constexpr uint32_t kTxState = static_cast<uint32_t>(2 * kAtomRows128 + 2 * kAtomRows64);  // C, prev
+  static constexpr uint32_t kTxScores = static_cast<uint32_t>(3 * kAtomRows128);                    // cb, x
   static_assert(kC % 1024 == 0 && kX % 1024 == 0 && kPrev % 1024 == 0, "swizzled tiles need 1 KB");
 };
 
@@ -107,29 +113,33 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(smem);
-  const int tid = threadIdx.x, l = tid;
+  const int tid = threadIdx.x;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
+  const int l = tid & (kCs - 1), at = tid >> 7;  // this thread's row and 64-column atom
   const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
   const int g = static_cast<int>(h / (a.nheads / a.ngroups));
-  const uint32_t full = sb + S::kBar, done = sb + S::kBar + 8;
+  const uint32_t full_state = sb + S::kBar, full_scores = sb + S::kBar + 8, done = sb + S::kBar + 16;
   if (tid == 0) {
-    mbar_init(full, 1);
+    mbar_init(full_state, 1);
+    mbar_init(full_scores, 1);
     mbar_init(done, 1);
     mbar_fence_init();
     prefetch_tensormap(&map_cb);
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_c);
     prefetch_tensormap(&map_prev);
-    mbar_arrive_expect_tx(full, S::kTx);
     const int zc = static_cast<int>((static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g);
     const int zp = static_cast<int>((static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h);
+    mbar_arrive_expect_tx(full_state, S::kTxState);
+    mbar_arrive_expect_tx(full_scores, S::kTxScores);
 #pragma unroll
-    for (int at = 0; at < 2; ++at) {
-      tma_load_3d(sb + S::kCb + at * S::kAtomRows128, &map_cb, 64 * at, 0, zc, full);
-      tma_load_4d(sb + S::kC + at * S::kAtomRows128, &map_c, 64 * at, g, c * kCs, b, full);
-      tma_load_3d(sb + S::kPrev + at * S::kAtomRows64, &map_prev, 64 * at, 0, zp, full);
+    for (int t = 0; t < 2; ++t) {
+      tma_load_4d(sb + S::kC + t * S::kAtomRows128, &map_c, 64 * t, g, c * kCs, b, full_state);
+      tma_load_3d(sb + S::kPrev + t * S::kAtomRows64, &map_prev, 64 * t, 0, zp, full_state);
     }
-    tma_load_4d(sb + S::kX, &map_x, 0, h, c * kCs, b, full);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, 64 * t, 0, zc, full_scores);
+    tma_load_4d(sb + S::kX, &map_x, 0, h, c * kCs, b, full_scores);
   }
   if (warp == 0) {
     tmem_alloc(sb + S::kTmemSlot, kSsdTmemCols);
@@ -137,7 +147,8 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   }
   float* sdA = reinterpret_cast<float*>(smem + S::kDA);
   float* sdt = reinterpret_cast<float*>(smem + S::kDt);
-  {
+  float* F = reinterpret_cast<float*>(smem + S::kF);
+  if (tid < kCs) {
     const int64_t row = ((static_cast<int64_t>(b) * a.nheads + h) * a.nchunks + c) * kCs;
     sdA[tid] = a.dA[row + tid];
     sdt[tid] = a.dt[row + tid];
@@ -147,79 +158,77 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   __syncthreads();
   tcgen05_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
-  mbar_wait_bounded(full, 0u, a.err, 7);
-
-  // 1. Row l of the cb tile -> masked, decayed, dt-weighted scores (in place).
-  const float dAl = sdA[l];
-  const int warp_max_l = 32 * warp + 31;
+  const uint32_t acc_intra = tmem, acc_state = tmem + kHd;
+  // 2. Carried-state term, as soon as its operands are in: C[l][n] x prev_states[p][n]^T.
+  if (tid == 0) {
+    mbar_wait_bounded(full_state, 0u, a.err, 7);
+    tcgen05_fence_after();
 #pragma unroll
-  for (int at = 0; at < 2; ++at) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int s0 = 64 * at + 8 * j;
-      uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
-      if (s0 > warp_max_l) {  // above the diagonal for every row of this warp
-        *p = make_uint4(0u, 0u, 0u, 0u);
-        continue;
-      }
-      float f[8];
-      unpack8(*p, f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int s = s0 + q;
-        f[q] = s <= l ? f[q] * ex2_approx((dAl - sdA[s]) * kLog2e) * sdt[s] : 0.0f;
-      }
-      *p = pack8(f);
-    }
+    for (int kk = 0; kk < kDs / 16; ++kk)
+      umma_f16_ss(acc_state, umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+                  umma_desc_k_sw128(sb + S::kPrev + (kk >> 2) * S::kAtomRows64 + (kk & 3) * 32), ssd_idesc(false),
+                  kk > 0);
   }
-  // 2. Row l of the C tile times exp(dA[l]) (in place).
-  const float el = ex2_approx(dAl * kLog2e);
+  if (tid < kCs) F[tid] = ex2_approx((sdA[tid & ~7] - sdA[tid]) * kLog2e) * sdt[tid];
+  const float dAl = sdA[l];
+  mbar_wait_bounded(full_scores, 0u, a.err, 8);
+  __syncthreads();  // F complete
+
+  // 3. This thread's atom of row l of the cb tile -> scores (in place).
+  const int warp_max_l = 32 * (warp & 3) + 31;
 #pragma unroll
-  for (int at = 0; at < 2; ++at) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint4* p = reinterpret_cast<uint4*>(smem + S::kC + at * S::kAtomRows128 + sw128(l, j));
-      float f[8];
-      unpack8(*p, f);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) f[q] *= el;
-      *p = pack8(f);
+  for (int j = 0; j < 8; ++j) {
+    const int s0 = 64 * at + 8 * j;
+    uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
+    if (s0 > warp_max_l) {  // above the diagonal for every row of this warp
+      *p = make_uint4(0u, 0u, 0u, 0u);
+      continue;
     }
+    float f[8];
+    unpack8(*p, f);
+    const float e = s0 <= l ? ex2_approx((dAl - sdA[s0]) * kLog2e) : 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) f[q] = s0 + q <= l ? f[q] * e * F[s0 + q] : 0.0f;
+    *p = pack8(f);
   }
   fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
   __syncthreads();
 
-  // 3. The two contractions into one accumulator.
+  // 4. Intra-chunk term: scores[l][s] x x[s][p], s in steps of 16 rows of x; one commit for both.
   if (tid == 0) {
     tcgen05_fence_after();
 #pragma unroll
-    for (int kk = 0; kk < kCs / 16; ++kk)  // scores[l][s] x x[s][p]: s in steps of 16 rows of x
-      umma_f16_ss(tmem, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+    for (int kk = 0; kk < kCs / 16; ++kk)
+      umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
                   umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < kDs / 16; ++kk)  // (exp(dA) C)[l][n] x prev_states[p][n]^T
-      umma_f16_ss(tmem, umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
-                  umma_desc_k_sw128(sb + S::kPrev + (kk >> 2) * S::kAtomRows64 + (kk & 3) * 32), ssd_idesc(false),
-                  true);
     umma_commit(done);
   }
-  mbar_wait_bounded(done, 0u, a.err, 8);
+  mbar_wait_bounded(done, 0u, a.err, 9);
   tcgen05_fence_after();
 
-  // 4. + D x, bf16, into the out tile (the cb buffer, free now) and out by TMA.
+  // 5. Lanes 32 (w mod 4) .., columns 32 (w / 4) ..: acc0 + exp(dA[l]) acc1 + D x, bf16,
+  //    into the out tile (the cb buffer, free now), then out by TMA.
+  {
+    const int q4 = warp & 3, col0 = 32 * (warp >> 2);
+    const int row = 32 * q4 + (tid & 31);
+    const float el = ex2_approx(sdA[row] * kLog2e);
 #pragma unroll
-  for (int jj = 0; jj < kHd / 16; ++jj) {
-    uint32_t r[16];
-    tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 16 * jj, r);
-    tmem_ld_wait();
+    for (int jj = 0; jj < 2; ++jj) {
+      uint32_t r0[16], r1[16];
+      const uint32_t lane_col = (static_cast<uint32_t>(32 * q4) << 16) + col0 + 16 * jj;
+      tmem_ld_x16(acc_intra + lane_col, r0);
+      tmem_ld_x16(acc_state + lane_col, r1);
+      tmem_ld_wait();
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int j = 2 * jj + half;  // 16-byte chunk of row l: p = 8 j .. 8 j + 7
-      float xv[8], o[8];
-      unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(l, j)), xv);
+      for (int half = 0; half < 2; ++half) {
+        const int j = (col0 + 16 * jj) / 8 + half;  // 16-byte chunk of the row: p = 8 j .. 8 j + 7
+        float xv[8], o[8];
+        unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(row, j)), xv);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) o[q] = fmaf(Dh, xv[q], __uint_as_float(r[8 * half + q]));
-      *reinterpret_cast<uint4*>(smem + S::kCb + sw128(l, j)) = pack8(o);
+        for (int q = 0; q < 8; ++q)
+          o[q] = fmaf(Dh, xv[q], fmaf(el, __uint_as_float(r1[8 * half + q]), __uint_as_float(r0[8 * half + q])));
+        *reinterpret_cast<uint4*>(smem + S::kCb + sw128(row, j)) = pack8(o);
+      }
     }
   }
   fence_proxy_async_smem();
