@@ -158,6 +158,7 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "ssm_math.cuh", "sm100_ptx.cuh"),
     "decode": ("decode.cu", "ssm_math.cuh", "sm100_ptx.cuh"),
+    "ssd": ("ssd.cu", "ssm_math.cuh", "sm100_ptx.cuh", "tma_map.cuh"),
 }
 
 
@@ -427,7 +428,8 @@ def ssd_bench(name: str, hbm_peak: float, bf16_peak: float, steps: int = 20, war
             "us_per_step": round(us, 2), "value": b * L * H / (us * 1e-6), "unit": "token-heads/s",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                          "frac": round(gbs / hbm_peak, 4), "algorithmic_bytes_per_launch": nbytes,
-                         "tensor_tflops": round(flops / (us * 1e-6) / 1e12, 1), "tensor_peak": bf16_peak},
+                         "tensor_tflops": round(flops / (us * 1e-6) / 1e12, 1), "tensor_peak": bf16_peak,
+                         "traffic": ncu_traffic("ssd", name)},
             "gpu_launches_per_step": 1}
 
 

@@ -212,6 +212,70 @@ def prefill_sampled(x, z, B, C, dt_raw, conv_w, conv_b, w_dt, dt_bias, A_log, D,
                     hist=hist, h0=h0, lo=lo, hi=hi, disc=disc, threads=threads)
 
 
+def segment_summary(x, B, dt_raw, conv_w, conv_b, w_dt, dt_bias, A_log, hist=None, lo=1e-4, hi=1.0, disc="euler",
+                    threads=0):
+    """What one segment of a sequence hands to the segments after it, for the
+    sequence-parallel prefill: the intra-chunk step of "What is the Mamba
+    model?" (velog, Texnee), "chunkscan", with the segment as the chunk.
+
+    For every sequence s and channel e of a segment of T tokens:
+      h_zero[s, :, e] = the state after the segment's last token when the scan
+                        starts from h = 0 (the recurrence, token by token)
+      dtsum[s, e]     = sum_t dt_t, so that the segment's decay product is
+                        prod_t exp(dt_t A_n) = exp(A_n * dtsum)
+
+    x: [b, T, E]; B: [b, T, N]; dt_raw: [b, T]; parameters per channel as in
+    channels(); hist: [b, K-1, E] (the raw x rows before the segment) or None.
+    Returns [b, N + 1, E] in float64: h_zero in rows 0..N-1, dtsum in row N."""
+    x, B, dt_raw = map(_f64, (x, B, dt_raw))
+    conv_w, conv_b, w_dt, dt_bias, A_log = map(_f64, (conv_w, conv_b, w_dt, dt_bias, A_log))
+    b, T, E = x.shape
+    N, K = A_log.shape[1], conv_w.shape[1]
+    hist = None if hist is None else _f64(hist)
+    out = np.zeros((b, N + 1, E))
+    for s in range(b):
+        u = conv_silu(np.ascontiguousarray(x[s].T), conv_w, conv_b,
+                      None if hist is None else np.ascontiguousarray(hist[s].T), threads)
+        for e in range(E):
+            dt = np.array([dt_of(dt_raw[s, t], w_dt[e], dt_bias[e], lo, hi) for t in range(T)])
+            A = np.array([A_of(a) for a in A_log[e]])
+            _, h = scan(u[e], dt, A, B[s], np.zeros((T, N)), 0.0, None, disc)
+            out[s, :N, e] = h
+            out[s, N, e] = dt.sum()
+    return out
+
+
+def segment_carry(summaries, A_log, h_init=None):
+    """The state entering segment r = len(summaries): the inter-chunk step of
+    "What is the Mamba model?", "chunkscan", written as the closed form of
+    "Mamba/SSM basics" (molayo insights), "Technical details",
+    h_t = A_t ... A_1 h_0 + sum_j (A_t ... A_{j+1}) B_j x_j, at the granularity
+    of segments: segment j contributes h_zero_j and multiplies what enters it
+    by P_j = exp(A * dtsum_j), so
+
+      h_in = (prod_{j<r} P_j) h_init + sum_{j<r} (prod_{j<k<r} P_k) h_zero_j
+
+    summaries: [r, b, N + 1, E] (segment_summary's layout); A_log: [E, N];
+    h_init: [b, E, N] (the state before segment 0) or None (zeros).
+    Returns h_in [b, E, N] in float64."""
+    S = _f64(summaries)
+    A_log = _f64(A_log)
+    r, b, N1, E = S.shape  # r may be 0 (segment 0: nothing enters but h_init)
+    N = N1 - 1
+    A = np.array([[A_of(a) for a in row] for row in A_log])                  # [E, N]
+    P = [np.exp(A[None] * S[j, :, N, :][..., None]) for j in range(r)]       # [b, E, N] each
+    hz = [S[j, :, :N, :].transpose(0, 2, 1) for j in range(r)]               # [b, E, N] each
+    h = np.zeros((b, E, N)) if h_init is None else _f64(h_init).copy()
+    for j in range(r):
+        h = h * P[j]                                                         # prod_{j<r} P_j h_init
+    for j in range(r):
+        term = hz[j].copy()
+        for k in range(j + 1, r):
+            term = term * P[k]
+        h = h + term
+    return h
+
+
 def ssd_chunk_scan(cb, x, dt, dA_cumsum, C, prev_states, D=None):
     """Output of the Mamba-2 chunk scan, "What is the Mamba model?" (velog,
     Texnee), "chunkscan" section, in float64, for every position l of chunk c
