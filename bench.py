@@ -433,6 +433,75 @@ def ssd_bench(name: str, hbm_peak: float, bf16_peak: float, steps: int = 20, war
             "gpu_launches_per_step": 1}
 
 
+def seqpar_bench(w: W.Workload, R: int = 8, reps: int = 10):
+    """The sequence-parallel prefill on one GPU: the workload cut into R
+    segments as R GPUs would hold it. Times, by CUDA events, the segment
+    summary (segment 1), the carry of R-1 summaries, one segment's prefill from
+    its carried state, and the whole path run segment after segment on this
+    GPU. The per-rank kernel time of a middle rank (summary + carry + prefill)
+    gives the R-GPU figure without the exchange, which this box cannot time;
+    the exchanged bytes are reported."""
+    from selective_state_space_depthwise_b200 import api, seqpar
+
+    inp = W.make_inputs(w, device="cuda", gen_device="cuda")
+    b, L, E = w.batch, w.seqlen, w.d_inner
+    T = L // R
+    bounds = [T * r for r in range(R)] + [L]
+    x1, B1, d1 = inp["x"][:, T:2 * T], inp["B"][:, T:2 * T], inp["dt_raw"][:, T:2 * T]
+    halo = inp["x"][:, T - 3:T].contiguous()
+    ws = torch.empty(api.segment_summary_workspace_bytes(b, T, E, w.io_dtype), dtype=torch.uint8, device="cuda")
+    summ = torch.empty((b, 17, E), dtype=torch.float32, device="cuda")
+    summaries = torch.stack([api.segment_summary(inp["x"][:, bounds[r]:bounds[r + 1]], inp["B"][:, bounds[r]:bounds[r + 1]],
+                                                 inp["dt_raw"][:, bounds[r]:bounds[r + 1]], inp,
+                                                 conv_cache_in=None if r == 0 else
+                                                 inp["x"][:, bounds[r] - 3:bounds[r]].contiguous())
+                             for r in range(R - 1)]).contiguous()
+    h_in = torch.empty((b, E, 16), dtype=torch.float32, device="cuda")
+    r_last = R - 1
+    xs, zs = inp["x"][:, bounds[r_last]:], inp["z"][:, bounds[r_last]:]
+    Bs, Cs, ds = inp["B"][:, bounds[r_last]:], inp["C"][:, bounds[r_last]:], inp["dt_raw"][:, bounds[r_last]:]
+    halo_last = inp["x"][:, bounds[r_last] - 3:bounds[r_last]].contiguous()
+    y = torch.empty((b, L - bounds[r_last], E), dtype=w.io_dtype, device="cuda")
+    cc = torch.empty((b, 3, E), dtype=w.io_dtype, device="cuda")
+    st = torch.empty((b, E, 16), dtype=torch.float32, device="cuda")
+
+    def t_us(fn, n=reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / n
+
+    us_sum = t_us(lambda: api.segment_summary(x1, B1, d1, inp, conv_cache_in=halo, summary=summ, workspace=ws))
+    us_carry = t_us(lambda: api.segment_carry(summaries, inp, out=h_in))
+    us_pre = t_us(lambda: api.prefill(xs, zs, Bs, Cs, ds, inp, conv_cache_in=halo_last, ssm_state_in=h_in, y=y,
+                                      conv_cache_out=cc, ssm_state_out=st))
+    us_path = t_us(lambda: seqpar.prefill_segments(inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp, bounds),
+                   n=3)
+    ct_seg = b * T * E
+    sfu_peak = 148 * 16 * 1965e6 / 19  # 16 decays + softplus + SiLU (exp2, rcp) per channel-token on the SFU
+    per_rank = us_sum + us_carry + us_pre
+    return {"workload": f"{w.name} cut into {R} segments of {T} tokens (b={b} E={E})",
+            "summary_us": round(us_sum, 1), "carry_us": round(us_carry, 1), "segment_prefill_us": round(us_pre, 1),
+            "one_gpu_path_ms": round(us_path / 1e3, 3),
+            "summary_roofline": {"bound": "alu", "achieved": ct_seg / (us_sum * 1e-6), "peak": sfu_peak,
+                                 "unit": "channel-tokens/s", "frac": round(ct_seg / (us_sum * 1e-6) / sfu_peak, 4),
+                                 "peak_basis": "SFU 16 lanes/clk/SM x 148 SMs at 1965 MHz, 19 SFU ops per "
+                                               "channel-token"},
+            "per_rank_kernel_us": round(per_rank, 1),
+            "projected_value": b * L * E / (per_rank * 1e-6), "projected_unit": "channel-tokens/s",
+            "projected_note": f"{R} GPUs, each running summary + carry + its segment's prefill; the all-gathers are "
+                              f"not included (one GPU here)",
+            "exchange_bytes_per_rank": b * 17 * E * 4 + 3 * b * E * (2 if w.io_dtype == torch.bfloat16 else 4),
+            "gpu_launches_per_rank": 2 + 1 + 1}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -445,6 +514,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-block", action="store_true",
                     help="skip the block-forward and chunk-scan sub-benchmarks")
+    ap.add_argument("--no-seqpar", action="store_true", help="skip the sequence-parallel sub-benchmark")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -520,6 +590,9 @@ def main():
             extra["block"] = [block_bench(n, bf16_peak) for n in W.BLOCK_WORKLOADS]
             torch.cuda.empty_cache()
             extra["ssd_chunk_scan"] = ssd_bench("ssd_chunk_scan", hbm_peak, bf16_peak)
+        if not args.no_seqpar:
+            torch.cuda.empty_cache()
+            extra["sequence_parallel"] = seqpar_bench(w)
         if not args.no_cpu and world == 1:
             extra["cpu_baseline"] = cpu_baseline(w)
     if dist:

@@ -327,9 +327,9 @@ size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
  *
  * Computation. Per (b, c, h) one CTA:
  *  - scores = masked cb * exp(dA[l] - dA[s]) * dt[s] in bf16, times x;
- *  - exp(dA[l]) C[l] in bf16, times prev_states^T;
- * both as tcgen05 MMAs into one fp32 TMEM accumulator, then + D x and a bf16
- * store. The exponents are <= 0 for s <= l, so nothing overflows.
+ *  - C[l] in bf16, times prev_states^T;
+ * as tcgen05 MMAs into two fp32 TMEM accumulators, combined as
+ * acc_scores + exp(dA[l]) acc_state + D x and stored as bf16. The exponents are <= 0 for s <= l, so nothing overflows.
  */
 typedef struct {
   int64_t batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size;
@@ -338,6 +338,54 @@ typedef struct {
 ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims *dims, const void *cb, const void *x, const float *dt,
                               const float *dA_cumsum, const void *C, const void *prev_states, const float *D,
                               void *out, void *stream);
+
+/*
+ * Sequence-parallel prefill -- one sequence split into segments that are
+ * computed at the same time (one per GPU, or pieces of one long context), in
+ * the three steps of "What is the Mamba model?" (velog, Texnee), "chunkscan",
+ * with a segment as the chunk:
+ *  1. ssm_segment_summary on every segment (but the last), independently:
+ *     its final state from a zero start, h_zero, and its dt sum, dtsum;
+ *  2. the summaries are exchanged (an all-gather across GPUs; the library
+ *     does not communicate), and ssm_segment_carry folds those of segments
+ *     0..r-1 into the state entering segment r:
+ *         h <- exp(A_n dtsum_j) h + h_zero_j,   j = 0 .. r-1, from ssm_state_in,
+ *     the closed form of "Mamba/SSM basics" (molayo insights), "Technical
+ *     details" (h_t = A_t...A_1 h_0 + sum_j A_t...A_{j+1} B_j x_j), a segment
+ *     at a time;
+ *  3. ssm_prefill of segment r with ssm_state_in = that state and
+ *     conv_cache_in = the last 3 raw x rows before the segment.
+ * The result equals ssm_prefill of the whole sequence up to fp32 rounding
+ * order; the last segment's conv_cache_out and ssm_state_out are the whole
+ * sequence's.
+ *
+ * ssm_segment_summary. dims describe the segment (seqlen = its token count T,
+ * may be 0; io_dtype, discretization, dt clip and the strides of x, B and
+ * dt_raw as for ssm_prefill; z, C and y are not read).
+ *   x              [b, T, *] io_dtype          B [b, T, 16] fp32; dt_raw [b, T] fp32
+ *   conv_cache_in  [b, 3, E] io_dtype, dense: raw x rows before the segment;
+ *                  NULL = zeros (the first segment of a fresh sequence)
+ *   summary        [b, 17, E] fp32, dense: rows 0..15 h_zero (state n of
+ *                  channel e at [s][n][e]), row 16 dtsum; 16-byte aligned
+ *   workspace      ssm_segment_summary_workspace_bytes(dims) bytes of device
+ *                  scratch (b * ceil(T / 64) * 17 * E floats), 16-byte aligned
+ * Two launches: 64-token blocks reduce in parallel to (state contribution,
+ * dt total) rows, then the blocks are folded in order.
+ *
+ * ssm_segment_carry. dims give batch, d_inner and the checks of ssm_prefill
+ * (seqlen is not used).
+ *   summaries      [count, b, 17, E] fp32: the summaries of segments 0..count-1
+ *   ssm_state_in   [b, E, 16] fp32: state before segment 0, or NULL = zeros
+ *   ssm_state_out  [b, E, 16] fp32: state entering segment `count`; may alias
+ *                  ssm_state_in
+ * count = 0 copies ssm_state_in (or writes zeros).
+ */
+size_t ssm_segment_summary_workspace_bytes(const ssm_dims *dims);
+ssm_status ssm_segment_summary(const ssm_dims *dims, const ssm_weights *w, const void *x, const float *B,
+                               const float *dt_raw, const void *conv_cache_in, float *summary, void *workspace,
+                               size_t workspace_bytes, void *stream);
+ssm_status ssm_segment_carry(const ssm_dims *dims, const ssm_weights *w, const float *summaries, int64_t count,
+                             const float *ssm_state_in, float *ssm_state_out, void *stream);
 
 /* Reads and clears the device error word that kernels set when a bounded
  * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed. */

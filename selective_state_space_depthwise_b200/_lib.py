@@ -29,6 +29,9 @@ EXPORTED = (
     "ssm_block_forward",
     "ssm_block_workspace_bytes",
     "ssm_ssd_chunk_scan",
+    "ssm_segment_summary",
+    "ssm_segment_summary_workspace_bytes",
+    "ssm_segment_carry",
     "ssm_decode_step",
     "ssm_check_device_error",
     "ssm_status_string",
@@ -131,6 +134,12 @@ def load(path: str = LIB_PATH):
     lib.ssm_block_workspace_bytes.restype = sz
     lib.ssm_ssd_chunk_scan.argtypes = [ctypes.POINTER(SsmSsdDims)] + [p] * 8 + [p]
     lib.ssm_ssd_chunk_scan.restype = st
+    lib.ssm_segment_summary.argtypes = [dims_p, w_p] + [p] * 6 + [sz, p]
+    lib.ssm_segment_summary.restype = st
+    lib.ssm_segment_summary_workspace_bytes.argtypes = [dims_p]
+    lib.ssm_segment_summary_workspace_bytes.restype = sz
+    lib.ssm_segment_carry.argtypes = [dims_p, w_p, p, ctypes.c_int64, p, p, p]
+    lib.ssm_segment_carry.restype = st
     lib.ssm_decode_step.argtypes = [dims_p, w_p] + [p] * 8 + [p]
     lib.ssm_decode_step.restype = st
     lib.ssm_check_device_error.argtypes = [p]

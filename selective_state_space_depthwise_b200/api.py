@@ -187,6 +187,78 @@ def prefill_host(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in
     return y, conv_cache_out, ssm_state_out
 
 
+def segment_summary_workspace_bytes(batch, seqlen, E, io_dtype=torch.bfloat16) -> int:
+    lib = _lib.load()
+    return int(lib.ssm_segment_summary_workspace_bytes(ctypes.byref(make_dims(batch, seqlen, E, io_dtype))))
+
+
+def segment_summary(x, B, dt_raw, params, *, conv_cache_in=None, summary=None, workspace=None, dt_min=1e-4,
+                    dt_max=1.0, discretization="euler", stream=None):
+    """Summary of one segment of a sequence for the sequence-parallel prefill
+    (ssm_segment_summary): x [b, T, E] (last dim contiguous), B [b, T, 16],
+    dt_raw [b, T]; conv_cache_in [b, 3, E] = raw x rows before the segment, or
+    None for zeros. Returns summary [b, 17, E] fp32: the zero-start final
+    state in rows 0..15, the dt sum in row 16."""
+    lib = _lib.load()
+    b, T, E = x.shape
+    dev = x.device
+    for n, t in (("x", x), ("B", B), ("dt_raw", dt_raw), ("conv_cache_in", conv_cache_in), ("summary", summary),
+                 ("workspace", workspace)):
+        _need_cuda(n, t, dev)
+    if x.dtype not in _DTYPES:
+        raise ValueError("x must be float32 or bfloat16")
+    if B.shape != (b, T, 16) or dt_raw.shape != (b, T):
+        raise ValueError("shape mismatch: B [b,T,16], dt_raw [b,T]")
+    if x.stride(2) != 1 or B.stride(2) != 1 or dt_raw.stride(1) != 1:
+        raise ValueError("the innermost dimension of x, B, dt_raw must be contiguous")
+    if conv_cache_in is not None and (conv_cache_in.shape != (b, 3, E) or conv_cache_in.dtype != x.dtype
+                                      or not conv_cache_in.is_contiguous()):
+        raise ValueError("conv_cache_in must be a contiguous [b, 3, E] tensor in the io dtype")
+    if summary is None:
+        summary = torch.empty((b, 17, E), dtype=torch.float32, device=dev)
+    if summary.shape != (b, 17, E) or summary.dtype != torch.float32 or not summary.is_contiguous():
+        raise ValueError("summary must be a contiguous float32 [b, 17, E] tensor")
+    dims = make_dims(b, T, E, x.dtype, dt_min, dt_max, discretization, x_tok_stride=x.stride(1),
+                     x_seq_stride=x.stride(0), bc_tok_stride=B.stride(1), bc_seq_stride=B.stride(0),
+                     dt_seq_stride=dt_raw.stride(0))
+    ws = int(lib.ssm_segment_summary_workspace_bytes(ctypes.byref(dims)))
+    if workspace is None and ws:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    if ws and workspace.numel() * workspace.element_size() < ws:
+        raise ValueError(f"workspace needs {ws} bytes")
+    w = _weights(params, E, dev)
+    st = lib.ssm_segment_summary(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(B), _ptr(dt_raw),
+                                 _ptr(conv_cache_in), _ptr(summary), _ptr(workspace) if ws else None, ws,
+                                 _stream(stream))
+    _lib.check(st)
+    return summary
+
+
+def segment_carry(summaries, params, *, ssm_state_in=None, out=None, stream=None):
+    """State entering the segment after the summarised ones
+    (ssm_segment_carry): summaries [count, b, 17, E] fp32 (count may be 0);
+    ssm_state_in [b, E, 16] = the state before segment 0, or None for zeros.
+    Returns [b, E, 16] fp32 (out may alias ssm_state_in)."""
+    lib = _lib.load()
+    count, b, rows, E = summaries.shape
+    dev = summaries.device
+    for n, t in (("summaries", summaries), ("ssm_state_in", ssm_state_in), ("out", out)):
+        _need_cuda(n, t, dev)
+    if rows != 17 or summaries.dtype != torch.float32 or not summaries.is_contiguous():
+        raise ValueError("summaries must be a contiguous float32 [count, b, 17, E] tensor")
+    if out is None:
+        out = torch.empty((b, E, 16), dtype=torch.float32, device=dev)
+    for n, t in (("ssm_state_in", ssm_state_in), ("out", out)):
+        if t is not None and (t.shape != (b, E, 16) or t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous float32 [b, E, 16] tensor")
+    dims = make_dims(b, 0, E, torch.float32)
+    w = _weights(params, E, dev)
+    st = lib.ssm_segment_carry(ctypes.byref(dims), ctypes.byref(w), _ptr(summaries) if count else None, int(count),
+                               _ptr(ssm_state_in), _ptr(out), _stream(stream))
+    _lib.check(st)
+    return out
+
+
 PROJ_NAMES = ("W_in", "W_x", "W_out")
 
 

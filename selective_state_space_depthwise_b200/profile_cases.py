@@ -4,12 +4,15 @@
     python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
     python -m selective_state_space_depthwise_b200.profile_cases block NAME [L]
     python -m selective_state_space_depthwise_b200.profile_cases ssd NAME
+    python -m selective_state_space_depthwise_b200.profile_cases segment WORKLOAD [T]
 
 prefill: three launches of the named workload's prefill (optionally shortened
 to L tokens, optionally with an explicit launch shape and E channels); decode: a 4-token
 prompt, then three decode steps at the decode workload's shape (batch 256,
 E=7680, 252 MB of state); block: three block forwards of the named block
-workload (optionally L tokens). Inputs are drawn on the GPU; a capture skips the
+workload (optionally L tokens); segment: three segment summaries of the first
+T tokens (default L / 8) of the named workload, then three carries of 7 such
+summaries. Inputs are drawn on the GPU; a capture skips the
 first two launches of the kernel it selects (ncu -s 2 -c 1 -k regex:...).
 """
 from __future__ import annotations
@@ -73,6 +76,21 @@ def ssd_case(name: str):
     print("ssd ok", name, float(out.float().abs().mean()))
 
 
+def segment_case(name: str, T: int = 0):
+    w = W.WORKLOADS[name]
+    T = T or w.seqlen // 8
+    w = W.Workload(w.name, batch=w.batch, seqlen=T, d_inner=w.d_inner, io_dtype=w.io_dtype, seed=w.seed,
+                   clip_stress=w.clip_stress)
+    inp = W.make_inputs(w, device="cuda", gen_device="cuda")
+    for _ in range(3):
+        summ = api.segment_summary(inp["x"], inp["B"], inp["dt_raw"], inp)
+    stacked = summ.unsqueeze(0).repeat(7, 1, 1, 1).contiguous()
+    for _ in range(3):
+        h = api.segment_carry(stacked, inp)
+    torch.cuda.synchronize()
+    print("segment ok", name, T, float(summ.abs().mean()), float(h.abs().mean()))
+
+
 if __name__ == "__main__":
     if sys.argv[1] == "prefill":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
@@ -83,6 +101,8 @@ if __name__ == "__main__":
         ssd_case(sys.argv[2])
     elif sys.argv[1] == "block":
         block_case(sys.argv[2], int(sys.argv[3]) if len(sys.argv) > 3 else 0)
+    elif sys.argv[1] == "segment":
+        segment_case(sys.argv[2], int(sys.argv[3]) if len(sys.argv) > 3 else 0)
     elif sys.argv[1] == "decode":
         decode_case(int(sys.argv[2]) if len(sys.argv) > 2 else 256)
     else:

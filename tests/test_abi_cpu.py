@@ -210,3 +210,44 @@ def test_block_forward_rejects_bad_arguments_before_any_work(lib):
     assert call(d, out=FAKE) == _lib.SSM_ERR_INVALID_ARG  # out aliases hidden
     assert call(d, ws_bytes=ws_need - 1) == _lib.SSM_ERR_INVALID_ARG
     assert lib.ssm_block_workspace_bytes(ctypes.byref(d32)) == 0
+
+
+def test_segment_summary_workspace_and_argument_checks(lib):
+    d = valid_dims()  # b=2, T=64, E=32
+    assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(d)) == 2 * 1 * 17 * 32 * 4
+    d300 = valid_dims(seqlen=300)
+    assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(d300)) == 2 * 5 * 17 * 32 * 4
+    assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(valid_dims(seqlen=0))) == 0
+    assert lib.ssm_segment_summary_workspace_bytes(None) == 0
+    w = fake_weights()
+    ws = lib.ssm_segment_summary_workspace_bytes(ctypes.byref(d))
+
+    def call(dims, x=FAKE, B=FAKE, dt=FAKE, cin=None, summ=FAKE, work=FAKE + 8192, nbytes=ws):
+        return lib.ssm_segment_summary(ctypes.byref(dims) if dims else None, ctypes.byref(w), x, B, dt, cin, summ,
+                                       work, nbytes, None)
+
+    assert call(None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(valid_dims(d_state=8)) == _lib.SSM_ERR_UNSUPPORTED
+    for k in ("x", "B", "dt", "summ"):
+        assert call(d, **{k: None}) == _lib.SSM_ERR_INVALID_ARG, k
+        assert b"NULL" in lib.ssm_last_error(), k
+    assert call(d, summ=FAKE + 4) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, cin=FAKE + 2) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, nbytes=ws - 4) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, work=None) == _lib.SSM_ERR_INVALID_ARG
+    assert b"workspace" in lib.ssm_last_error()
+
+
+def test_segment_carry_argument_checks(lib):
+    d, w = valid_dims(), fake_weights()
+
+    def call(dims, summ=FAKE, count=2, sin=None, sout=FAKE):
+        return lib.ssm_segment_carry(ctypes.byref(dims) if dims else None, ctypes.byref(w), summ, count, sin, sout,
+                                     None)
+
+    assert call(None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, count=-1) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, summ=None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, sout=None) == _lib.SSM_ERR_INVALID_ARG
+    assert call(d, sin=FAKE + 2) == _lib.SSM_ERR_INVALID_ARG
+    assert call(valid_dims(d_conv=3)) == _lib.SSM_ERR_UNSUPPORTED
