@@ -32,6 +32,7 @@
 
 #include "ssm.h"
 #include "ssm_internal.h"
+#include "sm100_ptx.cuh"
 #include "ssm_math.cuh"
 
 namespace ssm {
@@ -41,6 +42,13 @@ constexpr int kN = 16;       // states
 constexpr int kSegTok = 64;  // tokens per block of the summary kernel
 constexpr int kSegCh = 128;  // channels per CTA: 4 warps, lane = channel
 constexpr int kSegThreads = 128;
+// State pairs per token whose decay exp2 runs as an FMA-pipe polynomial
+// (Euler-B): the SFU is the summary kernel's binding unit and the FMA pipe
+// has room.
+#ifndef SSM_SEG_POLY
+#define SSM_SEG_POLY 1
+#endif
+constexpr int kSegPoly = SSM_SEG_POLY;
 
 struct SegArgs {
   const void* x;
@@ -157,21 +165,34 @@ __global__ void __launch_bounds__(kSegThreads, ZOH ? 4 : 8) segment_block_kernel
     x1 = x0;
     const float u = silu(conv);
     const float dt = dt_of(fmaf(dr[t], wdt, dtb), a.dt_min, a.dt_max);
-    const float v = ZOH ? u : dt * u;
     const float4* Bt = reinterpret_cast<const float4*>(&Bs[t][0]);
+    if constexpr (ZOH) {
 #pragma unroll
-    for (int q = 0; q < kN / 4; ++q) {
-      const float4 b4 = Bt[q];
-      const float bq[4] = {b4.x, b4.y, b4.z, b4.w};
+      for (int q = 0; q < kN / 4; ++q) {
+        const float4 b4 = Bt[q];
+        const float bq[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int n = 4 * q + i;
-        float inj = v * bq[i];
-        if constexpr (ZOH) {
+        for (int i = 0; i < 4; ++i) {
+          const int n = 4 * q + i;
           const float xa = dt * An[n];
-          inj *= expm1_nonpos(xa, ex2_approx(xa * kLog2e)) / An[n];
+          const float inj = u * bq[i] * expm1_nonpos(xa, ex2_approx(xa * kLog2e)) / An[n];
+          acc[n] = fmaf(ex2_approx(a2[n] * R), inj, acc[n]);
         }
-        acc[n] = fmaf(ex2_approx(a2[n] * R), inj, acc[n]);
+      }
+    } else {
+      // Euler-B, packed in state pairs: acc += e^{A R} (dt u) B.
+      const uint64_t R2 = pk2(R, R), v2 = pk2(dt * u, dt * u);
+#pragma unroll
+      for (int p = 0; p < kN / 2; ++p) {
+        const float4 b4 = Bt[p / 2];
+        const uint64_t b2 = (p & 1) ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
+        float y0, y1;
+        upk2(fmul2(R2, pk2(a2[2 * p], a2[2 * p + 1])), y0, y1);
+        // the last kSegPoly pairs take the FMA-pipe exp2, the others the SFU
+        const uint64_t decay = p >= kN / 2 - kSegPoly ? ex2_poly2(y0, y1) : pk2(ex2_approx(y0), ex2_approx(y1));
+        uint64_t ap = pk2(acc[2 * p], acc[2 * p + 1]);
+        ap = ffma2(decay, fmul2(v2, b2), ap);
+        upk2(ap, acc[2 * p], acc[2 * p + 1]);
       }
     }
     R += dt;
@@ -223,6 +244,7 @@ __global__ void segment_carry_kernel(const CarryArgs a) {
   float h = a.h_init ? a.h_init[i] : 0.0f;
   const int64_t seg_stride = a.batch * (kN + 1) * a.E;
   const float* p = a.summaries + s * (kN + 1) * a.E + e;
+#pragma unroll 4
   for (int64_t j = 0; j < a.count; ++j) h = fmaf(ex2_approx(a2 * p[j * seg_stride + kN * a.E]), h, p[j * seg_stride + n * a.E]);
   a.h_out[i] = h;
 }
