@@ -6,24 +6,28 @@
 // caches are updated in place.
 //
 // The step is bound by the fp32 state stream: 64 B read + 64 B written per
-// (sequence, channel) against ~12 B of everything else. The kernel keeps
-// state bytes in flight without waiting on anything else:
-//  - a thread owns one channel for the whole step and walks a strided set of
-//    sequences, so the channel's parameters are read and A = -exp(A_log) is
-//    computed once;
-//  - the next sequence's state (four 16-byte loads), caches, x and z are
-//    loaded before the current sequence is computed and stored, in two
-//    register sets used in turn;
-//  - B, C and dt_raw of the block's sequences are staged in shared memory 32
-//    sequences at a time, so no item waits on an L2 round trip for them;
-//  - the grid is sized so that every block is resident at once.
-// Measured on B200 at b = 256, E = 7680: 59 us per step (4.8 TB/s), against
-// 74 us for one thread per (sequence, channel) with per-item loads.
+// (sequence, channel) against ~12 B of everything else. Two forms share the
+// per-channel arithmetic:
+//  - the TMA form (default): the state of (sequence, 128 channels) is one
+//    contiguous 8 KB tile, loaded by TMA into a ring of four shared-memory
+//    slots up to four sequences ahead and stored back by TMA from the same
+//    slot, 64-byte swizzled so that a thread's 64 B row is read and written
+//    without bank conflicts;
+//  - the register form: a thread loads the next sequence's state (four
+//    16-byte loads) into a second register set while the current one runs.
+// In both, a thread owns one channel for the whole step and walks a strided
+// set of sequences, so the channel's parameters are read and A = -exp(A_log)
+// computed once; B, C and dt_raw are staged in shared memory 32 sequences at
+// a time; the grid is sized so that every block is resident at once.
+// Measured on B200 at b = 256, E = 7680: TMA form 54.8 us per step (5.25 TB/s),
+// register form 59.3 us, one thread per (sequence, channel) with per-item
+// loads 74 us.
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
 #include "ssm_internal.h"
 #include "ssm_math.cuh"
+#include "tma_map.cuh"
 
 namespace ssm {
 namespace {
@@ -184,6 +188,170 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_resident_kernel(const K
   }
 }
 
+// ---------------------------------------------------------------------------
+// TMA form. The state of (sequence, 128 channels) is one contiguous 8 KB tile;
+// it moves by TMA in both directions (load into a ring of shared-memory slots
+// several sequences ahead, store back from the same slot), so every state
+// byte crosses DRAM in full 8 KB transfers, while a thread keeps owning one
+// channel. The tile is 64-byte swizzled, which makes the per-thread reads and
+// writes of a channel's 64 B row free of bank conflicts.
+constexpr int kTmaSlots = 4;
+constexpr int kStateTile = kDecodeThreads * 64;  // 128 channels x 16 fp32
+struct TmaSmem {
+  static constexpr int kSlots = 0;                                 // kTmaSlots x 8 KB, 1 KB aligned
+  static constexpr int kRows = kTmaSlots * kStateTile;             // staged B, C, dt_raw rows
+  static constexpr int kBar = kRows + kStageSeqs * kRow * 4;       // kTmaSlots mbarriers
+  static constexpr int kTotal = kBar + 8 * kTmaSlots;
+};
+
+// Byte offset of 16-byte chunk q of row r in a 64-byte-swizzled tile.
+__device__ __forceinline__ int sw64(int r, int q) { return r * 64 + ((q ^ ((r >> 1) & 3)) << 4); }
+
+template <typename T, bool ZOH>
+__global__ void __launch_bounds__(kDecodeThreads) decode_tma_kernel(const __grid_constant__ CUtensorMap map_h,
+                                                                     const KernelArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sb = smem_u32(smem);
+  float(*rows)[kRow] = reinterpret_cast<float(*)[kRow]>(smem + TmaSmem::kRows);
+  const uint32_t bar0 = sb + TmaSmem::kBar;
+  const int tid = threadIdx.x;
+  const int e0 = static_cast<int>(blockIdx.x) * kDecodeThreads;
+  const int64_t e = e0 + tid;
+  const bool active = e < a.E;
+  ChannelParams p;
+  if (active) {
+    const float4* Al = reinterpret_cast<const float4*>(a.A_log) + e * 4;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = Al[q];
+      const float lv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float A = -ex2_approx(lv[i] * kLog2e);  // A = -exp(A_log)
+        p.A[4 * q + i] = A;
+        p.a2[4 * q + i] = A * kLog2e;
+      }
+    }
+    p.cw = reinterpret_cast<const float4*>(a.conv_w)[e];
+    p.cb = a.conv_b[e];
+    p.wdt = a.w_dt[e];
+    p.dtb = a.dt_bias[e];
+    p.D = a.D[e];
+  }
+  const int64_t stride = gridDim.y, s0 = blockIdx.y;
+  const int64_t n = (a.batch - s0 + stride - 1) / stride;
+  auto seq_of = [&](int64_t k) { return s0 + k * stride; };
+  if (tid == 0) {
+    for (int i = 0; i < kTmaSlots; ++i) mbar_init(bar0 + 8 * i, 1);
+    mbar_fence_init();
+    prefetch_tensormap(&map_h);
+    for (int64_t k = 0; k < kTmaSlots && k < n; ++k) {
+      mbar_arrive_expect_tx(bar0 + 8 * k, kStateTile);
+      tma_load_3d(sb + static_cast<uint32_t>(k) * kStateTile, &map_h, 0, e0, static_cast<int>(seq_of(k)), bar0 + 8 * k);
+    }
+  }
+  // x, z and the conv cache of the next sequence are loaded while this one runs.
+  auto load_small = [&](int64_t seq, float (&v)[5]) {
+    const T* cache = static_cast<const T*>(a.conv_cache_out) + seq * 3 * a.E + e;
+    v[0] = IO<T>::to_f(cache[0]);
+    v[1] = IO<T>::to_f(cache[a.E]);
+    v[2] = IO<T>::to_f(cache[2 * a.E]);
+    v[3] = IO<T>::to_f(static_cast<const T*>(a.x)[seq * a.s.x_seq + e]);
+    v[4] = IO<T>::to_f(static_cast<const T*>(a.z)[seq * a.s.z_seq + e]);
+  };
+  float cur[5] = {0.f, 0.f, 0.f, 0.f, 0.f}, nxt[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+  if (active && n > 0) load_small(seq_of(0), cur);
+
+  for (int64_t k = 0; k < n; ++k) {
+    const int64_t seq = seq_of(k);
+    if (k % kStageSeqs == 0) {  // refill the staged rows (also orders the barrier init before any wait)
+      __syncthreads();
+      const int nk = static_cast<int>(n - k < kStageSeqs ? n - k : kStageSeqs);
+      for (int i = tid; i < nk * 33; i += kDecodeThreads) {
+        const int r = i / 33, j = i - r * 33;
+        const int64_t sq = seq_of(k + r);
+        rows[r][j] = j < 16 ? a.B[sq * a.s.bc_seq + j]
+                            : (j < 32 ? a.C[sq * a.s.bc_seq + j - 16] : a.dt_raw[sq * a.s.dt_seq]);
+      }
+      __syncthreads();
+    }
+    if (active && k + 1 < n) load_small(seq_of(k + 1), nxt);
+    const int slot = static_cast<int>(k % kTmaSlots);
+    unsigned char* tile = smem + slot * kStateTile;
+    mbar_wait_bounded(bar0 + 8 * slot, static_cast<uint32_t>((k / kTmaSlots) & 1), a.err, 11);
+    if (active) {
+      const float* row = rows[k % kStageSeqs];
+      const float4* Bq = reinterpret_cast<const float4*>(row);
+      const float4* Cq = reinterpret_cast<const float4*>(row + 16);
+      float4 h[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) h[q] = *reinterpret_cast<const float4*>(tile + sw64(tid, q));
+      const float conv = fmaf(p.cw.w, cur[3], fmaf(p.cw.z, cur[2], fmaf(p.cw.y, cur[1], fmaf(p.cw.x, cur[0], p.cb))));
+      const float u = silu(conv);
+      const float dt = dt_of(fmaf(row[32], p.wdt, p.dtb), a.dt_min, a.dt_max);
+      const float zg = silu(cur[4]);
+      float yl = 0.0f, yh = 0.0f;
+      if constexpr (ZOH) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 b = Bq[q], cc = Cq[q];
+          const float bv[4] = {b.x, b.y, b.z, b.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
+          float hs[4] = {h[q].x, h[q].y, h[q].z, h[q].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float A = p.A[4 * q + i];
+            const float xa = dt * A;
+            const float dA = ex2_approx(xa * kLog2e);
+            hs[i] = fmaf(dA, hs[i], expm1_nonpos(xa, dA) / A * u * bv[i]);
+            yl = fmaf(cv[i], hs[i], yl);
+          }
+          h[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
+        }
+      } else {
+        const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
+        uint64_t acc = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 b = Bq[q], cc = Cq[q];
+          float x0, x1, x2, x3;
+          upk2(fmul2(dt2, pk2(p.a2[4 * q], p.a2[4 * q + 1])), x0, x1);
+          upk2(fmul2(dt2, pk2(p.a2[4 * q + 2], p.a2[4 * q + 3])), x2, x3);
+          const uint64_t h01 = ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(h[q].x, h[q].y), fmul2(dtu2, pk2(b.x, b.y)));
+          const uint64_t h23 = ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(h[q].z, h[q].w), fmul2(dtu2, pk2(b.z, b.w)));
+          acc = q == 0 ? fmul2(pk2(cc.x, cc.y), h01) : ffma2(pk2(cc.x, cc.y), h01, acc);
+          acc = ffma2(pk2(cc.z, cc.w), h23, acc);
+          upk2(h01, h[q].x, h[q].y);
+          upk2(h23, h[q].z, h[q].w);
+        }
+        upk2(acc, yl, yh);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) *reinterpret_cast<float4*>(tile + sw64(tid, q)) = h[q];
+      static_cast<T*>(a.y)[seq * a.s.y_seq + e] = IO<T>::from_f((yl + yh + p.D * u) * zg);
+      T* cache = static_cast<T*>(a.conv_cache_out) + seq * 3 * a.E + e;  // the raw rows round-trip exactly
+      cache[0] = IO<T>::from_f(cur[1]);
+      cache[a.E] = IO<T>::from_f(cur[2]);
+      cache[2 * a.E] = IO<T>::from_f(cur[3]);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();  // the slot holds the new state of every channel
+    if (tid == 0) {
+      tma_store_3d(&map_h, sb + static_cast<uint32_t>(slot) * kStateTile, 0, e0, static_cast<int>(seq));
+      bulk_commit();
+      if (k + kTmaSlots < n) {
+        bulk_wait_read<0>();  // the store has read the slot
+        mbar_arrive_expect_tx(bar0 + 8 * slot, kStateTile);
+        tma_load_3d(sb + static_cast<uint32_t>(slot) * kStateTile, &map_h, 0, e0,
+                    static_cast<int>(seq_of(k + kTmaSlots)), bar0 + 8 * slot);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 5; ++i) cur[i] = nxt[i];
+  }
+  if (tid == 0) bulk_wait<0>();
+}
+
 template <typename T, bool ZOH>
 cudaError_t launch(const KernelArgs& a, cudaStream_t st) {
   const int64_t bx = (a.E + kDecodeThreads - 1) / kDecodeThreads;
@@ -211,9 +379,52 @@ cudaError_t launch(const KernelArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <typename T, bool ZOH>
+cudaError_t launch_tma(const KernelArgs& a, cudaStream_t st) {
+  const int64_t bx = (a.E + kDecodeThreads - 1) / kDecodeThreads;
+  if (bx > 0x7fffffff || a.batch > 0x7fffffff || a.E > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  CUtensorMap map_h;
+  const uint64_t dims[3] = {16, static_cast<uint64_t>(a.E), static_cast<uint64_t>(a.batch)};
+  const uint64_t strides[2] = {64, static_cast<uint64_t>(a.E) * 64};
+  const uint32_t box[3] = {16, kDecodeThreads, 1};
+  if (!encode_map(&map_h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.ssm_state_out, dims, strides, box,
+                  CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  auto kern = decode_tma_kernel<T, ZOH>;
+  const int smem = TmaSmem::kTotal + 1024;
+  static int resident[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  int& per_sm = resident[dev & 63];
+  if (per_sm == 0) {
+    if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return err;
+    int sms = 0, blocks = 0;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kDecodeThreads, smem)) != cudaSuccess)
+      return err;
+    per_sm = (blocks > 0 ? blocks : 1) * (sms > 0 ? sms : 148);
+  }
+  int64_t by = per_sm / bx;
+  if (by < 1) by = 1;
+  if (by > a.batch) by = a.batch;
+  if (by > 65535) by = 65535;
+  kern<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by)), kDecodeThreads, smem, st>>>(map_h, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
+// The TMA form is the default; SSM_DECODE_TMA=0 builds the register-prefetch form.
+#ifndef SSM_DECODE_TMA
+#define SSM_DECODE_TMA 1
+#endif
+
 cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStream_t st) {
+  if (SSM_DECODE_TMA) {
+    if (io_bf16) return zoh ? launch_tma<__nv_bfloat16, true>(a, st) : launch_tma<__nv_bfloat16, false>(a, st);
+    return zoh ? launch_tma<float, true>(a, st) : launch_tma<float, false>(a, st);
+  }
   if (io_bf16) return zoh ? launch<__nv_bfloat16, true>(a, st) : launch<__nv_bfloat16, false>(a, st);
   return zoh ? launch<float, true>(a, st) : launch<float, false>(a, st);
 }
