@@ -195,10 +195,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_resident_kernel(const K
 // byte crosses DRAM in full 8 KB transfers, while a thread keeps owning one
 // channel. The tile is 64-byte swizzled, which makes the per-thread reads and
 // writes of a channel's 64 B row free of bank conflicts.
-constexpr int kTmaSlots = 4;
+#ifndef SSM_DECODE_SLOTS
+#define SSM_DECODE_SLOTS 4
+#endif
+constexpr int kTmaSlots = SSM_DECODE_SLOTS;
 constexpr int kStateTile = kDecodeThreads * 64;  // 128 channels x 16 fp32
 struct TmaSmem {
-  static constexpr int kSlots = 0;                                 // kTmaSlots x 8 KB, 1 KB aligned
+  // kTmaSlots state slots of 8 KB at offset 0 (1 KB aligned), then:
   static constexpr int kRows = kTmaSlots * kStateTile;             // staged B, C, dt_raw rows
   static constexpr int kBar = kRows + kStageSeqs * kRow * 4;       // kTmaSlots mbarriers
   static constexpr int kTotal = kBar + 8 * kTmaSlots;
