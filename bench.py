@@ -502,6 +502,78 @@ def seqpar_bench(w: W.Workload, R: int = 8, reps: int = 10):
             "gpu_launches_per_rank": 2 + 1 + 1}
 
 
+def seq_parallel_main(args, w: W.Workload):
+    """--seq-parallel: one sequence split along L across the ranks (strong
+    scaling; seqpar.prefill_sequence_parallel). Rank r holds tokens
+    [L r / N, L (r + 1) / N) of the workload. A step is the whole path on every
+    rank: the all-gather of the conv tails, the segment summary (ranks
+    0..N-2), the all-gather of the summaries, the carry and the segment's
+    prefill. Timed by CUDA events between barriers, max over ranks."""
+    import datetime
+
+    from selective_state_space_depthwise_b200 import _lib, seqpar
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29531")
+    os.environ.setdefault("RANK", "0")
+    os.environ.setdefault("WORLD_SIZE", "1")
+    torch.cuda.set_device(local_rank)
+    torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                         device_id=torch.device("cuda", local_rank))
+    _lib.load()
+    inp = W.make_inputs(w, device="cuda", gen_device="cuda")  # the same seeded problem on every rank
+    b, L, E = w.batch, w.seqlen, w.d_inner
+    t0, t1 = L * rank // world, L * (rank + 1) // world
+    seg = {k: inp[k][:, t0:t1] for k in ("x", "z", "B", "C", "dt_raw")}
+    params = {k: inp[k] for k in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")}
+
+    def step():
+        return seqpar.prefill_sequence_parallel(seg["x"], seg["z"], seg["B"], seg["C"], seg["dt_raw"], params)
+
+    for _ in range(args.warmup):
+        step()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    torch.distributed.barrier()
+    t = torch.tensor([ev0.elapsed_time(ev1)], device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_step = float(t.item()) / args.steps
+    clocks = clk.summary()
+    torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    value = b * L * E / (ms_step * 1e-3)
+    peak_ct = alu_peak_ct_per_s(1965.0)
+    per_gpu = value / world
+    print(json.dumps({
+        "metric": "selective-scan channel-tokens/s (prefill); achieved HBM GB/s vs B200 peak",
+        "value": value, "unit": "channel-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "f32", "io_dtype": "bf16" if w.io_dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": f"{w.name}: {w.note}; b={b} L={L} E={E} N=16 K=4", "batch": b, "seq_len": L,
+                   "d_inner": E, "parallelism": f"sp{world} (sequence segments; all-gather of conv tails and "
+                                               f"segment summaries over NCCL)",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "roofline": {"bound": "alu", "achieved": per_gpu, "peak": peak_ct, "unit": "channel-tokens/s",
+                     "frac": round(per_gpu / peak_ct, 4), "traffic": None,
+                     "note": "per GPU; ranks 0..N-2 also run the segment summary"},
+        "gpu_launches": args.steps * (3 if world > 1 else 1),  # rank 0: summary (2) + prefill; alone: prefill
+        "clocks": clocks,
+        "e2e": None,
+    }))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -515,6 +587,9 @@ def main():
     ap.add_argument("--no-block", action="store_true",
                     help="skip the block-forward and chunk-scan sub-benchmarks")
     ap.add_argument("--no-seqpar", action="store_true", help="skip the sequence-parallel sub-benchmark")
+    ap.add_argument("--seq-parallel", action="store_true",
+                    help="split the workload's sequence across the ranks (strong scaling) instead of running "
+                         "the same workload on every rank")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -525,6 +600,9 @@ def main():
     w = W.WORKLOADS[args.workload]
     if w.decode_steps:
         ap.error("the step workload must be a prefill shape; the decode workload is reported alongside")
+
+    if args.seq_parallel and args.impl == "native":
+        return seq_parallel_main(args, w)
 
     if args.impl == "reference":
         # The oracle is the reference arm: rank 0 alone runs it on the host cores.
