@@ -368,8 +368,8 @@ ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims *dims, const void *cb, const vo
  *   summary        [b, 17, E] fp32, dense: rows 0..15 h_zero (state n of
  *                  channel e at [s][n][e]), row 16 dtsum; 16-byte aligned
  *   workspace      ssm_segment_summary_workspace_bytes(dims) bytes of device
- *                  scratch (b * ceil(T / 64) * 17 * E floats), 16-byte aligned
- * Two launches: 64-token blocks reduce in parallel to (state contribution,
+ *                  scratch (b * ceil(T / 256) * 17 * E floats), 16-byte aligned
+ * Two launches: 256-token blocks reduce in parallel to (state contribution,
  * dt total) rows, then the blocks are folded in order.
  *
  * ssm_segment_carry. dims give batch, d_inner and the checks of ssm_prefill

@@ -19,7 +19,7 @@
 //     h_zero_n = sum_t exp(A_n R_t) inj_{t,n},
 // inj = dt B u (Euler-B) or (exp(dt A)-1)/A B u (ZOH): a weighted sum over
 // tokens with no dependence between them once R_t is known. The kernel
-// computes it on 64-token blocks in parallel (R_t local to the block, so no
+// computes it on 256-token blocks in parallel (R_t local to the block, so no
 // large sums are differenced; each thread walks its block backwards, R being
 // a running sum), and a second kernel folds the blocks in order with the
 // block dt totals -- the same carry at block granularity.
@@ -39,7 +39,16 @@ namespace ssm {
 namespace {
 
 constexpr int kN = 16;       // states
-constexpr int kSegTok = 64;  // tokens per block of the summary kernel
+constexpr int kSegTok = 64;  // tokens per staged sub-block of the summary kernel
+// Measured on B200 (8192-token segment, E = 7680): 1 sub-block at 8 CTAs per
+// SM 317 us, 2 at 7 CTAs 303 us, 4 at 7 CTAs 300 us (fewer blocks to fold).
+#ifndef SSM_SEG_SUB
+#define SSM_SEG_SUB 4
+#endif
+#ifndef SSM_SEG_MINB
+#define SSM_SEG_MINB 7
+#endif
+constexpr int kSegSub = SSM_SEG_SUB;  // sub-blocks per CTA: a block (one fold step) is kSegSub x 64 tokens
 constexpr int kSegCh = 128;  // channels per CTA: 4 warps, lane = channel
 constexpr int kSegThreads = 128;
 // State pairs per token whose decay exp2 runs as an FMA-pipe polynomial
@@ -83,125 +92,131 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// One CTA per (64-token block, 128 channels, sequence). The block's raw x rows
-// (with the 3 rows before it), B rows and dt_raw are staged in shared memory;
-// then each thread walks its channel from the block's last token to its first,
-// so R, the dt mass after the current token, is one running sum.
+// One CTA per (block of kSegSub x 64 tokens, 128 channels, sequence). Each
+// 64-token sub-block's raw x rows (with the 3 rows before it), B rows and
+// dt_raw are staged in shared memory, last sub-block first; each thread walks
+// its channel backwards through them, so R, the dt mass after the current
+// token, is one running sum across the whole block.
 template <typename T, bool ZOH>
-__global__ void __launch_bounds__(kSegThreads, ZOH ? 4 : 8) segment_block_kernel(const SegArgs a) {
+__global__ void __launch_bounds__(kSegThreads, ZOH ? 4 : SSM_SEG_MINB) segment_block_kernel(const SegArgs a) {
   constexpr int kRowChunks = kSegCh * int(sizeof(T)) / 16;  // 16-byte pieces of one x row
   constexpr int kChPerChunk = 16 / int(sizeof(T));
   __shared__ __align__(16) float Bs[kSegTok][kN];
   __shared__ __align__(16) float dr[kSegTok];
-  __shared__ __align__(16) T xs[kSegTok + 3][kSegCh];  // row r = token t_blk - 3 + r
+  __shared__ __align__(16) T xs[kSegTok + 3][kSegCh];  // row r = token t_sub - 3 + r
 
   const int tid = threadIdx.x;
   const int64_t blk = blockIdx.x, s = blockIdx.z;
-  const int64_t t_blk = blk * kSegTok;
+  const int64_t t_cta = blk * kSegTok * kSegSub;
   const int64_t e0 = int64_t(blockIdx.y) * kSegCh;
-  const int nt = int(a.T - t_blk < kSegTok ? a.T - t_blk : kSegTok);  // tokens of this block (>= 1)
-
-  // Stage. Rows past the segment's end and channels past E are zero-filled.
-  {
-    const T* xseq = static_cast<const T*>(a.x) + s * a.x_seq;
-    const T* hist = static_cast<const T*>(a.conv_cache_in);
-    for (int i = tid; i < (kSegTok + 3) * kRowChunks; i += kSegThreads) {
-      const int r = i / kRowChunks, q = i % kRowChunks;
-      const int64_t t = t_blk - 3 + r, e = e0 + int64_t(q) * kChPerChunk;
-      const void* src = a.x;
-      uint32_t nb = 0;
-      if (e < a.E && t < a.T) {
-        if (t >= 0) {
-          src = xseq + t * a.x_tok + e;
-          nb = 16;
-        } else if (hist) {
-          src = hist + (s * 3 + (t + 3)) * a.E + e;
-          nb = 16;
-        }
-      }
-      cp_async_16z(smem_addr(&xs[r][q * kChPerChunk]), src, nb);
-    }
-    const float* Bseq = a.B + s * a.bc_seq;
-    for (int i = tid; i < kSegTok * (kN / 4); i += kSegThreads) {
-      const int r = i >> 2, q = i & 3;
-      const bool in = r < nt;
-      cp_async_16z(smem_addr(&Bs[r][4 * q]), in ? Bseq + (t_blk + r) * a.bc_tok + 4 * q : a.B, in ? 16 : 0);
-    }
-    if (tid < kSegTok) {
-      const bool in = tid < nt;
-      cp_async_4z(smem_addr(&dr[tid]), in ? a.dt_raw + s * a.dt_seq + t_blk + tid : a.dt_raw, in ? 4 : 0);
-    }
-    cp_async_all_done();
-  }
-  __syncthreads();
-
   const int c = tid;  // channel within the CTA
   const int64_t e = e0 + c;
-  if (e >= a.E) return;  // no barrier follows
+  const int64_t ec = e < a.E ? e : a.E - 1;  // clamped for parameter loads; idle lanes store nothing
 
-  const float4 cw = *reinterpret_cast<const float4*>(a.conv_w + e * 4);
-  const float cb = a.conv_b[e], wdt = a.w_dt[e], dtb = a.dt_bias[e];
+  const float4 cw = *reinterpret_cast<const float4*>(a.conv_w + ec * 4);
+  const float cb = a.conv_b[ec], wdt = a.w_dt[ec], dtb = a.dt_bias[ec];
   float a2[kN];  // A_n log2(e)
   float An[ZOH ? kN : 1];
 #pragma unroll
   for (int n = 0; n < kN; ++n) {
-    const float A = -expf(a.A_log[e * kN + n]);
+    const float A = -expf(a.A_log[ec * kN + n]);
     a2[n] = A * kLog2e;
     if constexpr (ZOH) An[n] = A;
   }
   float acc[kN];
 #pragma unroll
   for (int n = 0; n < kN; ++n) acc[n] = 0.0f;
-
-  // x window of token t: rows t .. t+3 (tokens t-3 .. t); slides down by one row.
-  float x3 = IO<T>::to_f(xs[nt + 2][c]), x2 = IO<T>::to_f(xs[nt + 1][c]), x1 = IO<T>::to_f(xs[nt][c]);
   float R = 0.0f;
-#pragma unroll 2
-  for (int t = nt - 1; t >= 0; --t) {
-    const float x0 = IO<T>::to_f(xs[t][c]);
-    const float conv = fmaf(cw.w, x3, fmaf(cw.z, x2, fmaf(cw.y, x1, fmaf(cw.x, x0, cb))));
-    x3 = x2;
-    x2 = x1;
-    x1 = x0;
-    const float u = silu(conv);
-    const float dt = dt_of(fmaf(dr[t], wdt, dtb), a.dt_min, a.dt_max);
-    const float4* Bt = reinterpret_cast<const float4*>(&Bs[t][0]);
-    if constexpr (ZOH) {
-#pragma unroll
-      for (int q = 0; q < kN / 4; ++q) {
-        const float4 b4 = Bt[q];
-        const float bq[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int n = 4 * q + i;
-          const float xa = dt * An[n];
-          const float inj = u * bq[i] * expm1_nonpos(xa, ex2_approx(xa * kLog2e)) / An[n];
-          acc[n] = fmaf(ex2_approx(a2[n] * R), inj, acc[n]);
+
+  const T* xseq = static_cast<const T*>(a.x) + s * a.x_seq;
+  const T* hist = static_cast<const T*>(a.conv_cache_in);
+  const float* Bseq = a.B + s * a.bc_seq;
+#pragma unroll 1
+  for (int sub = kSegSub - 1; sub >= 0; --sub) {
+    const int64_t t_sub = t_cta + int64_t(sub) * kSegTok;
+    if (t_sub >= a.T) continue;  // block-uniform
+    const int nt = int(a.T - t_sub < kSegTok ? a.T - t_sub : kSegTok);
+    __syncthreads();  // the previous sub-block's rows are no longer read
+    // Stage. Rows past the segment's end and channels past E are zero-filled.
+    for (int i = tid; i < (kSegTok + 3) * kRowChunks; i += kSegThreads) {
+      const int r = i / kRowChunks, q = i % kRowChunks;
+      const int64_t t = t_sub - 3 + r, ee = e0 + int64_t(q) * kChPerChunk;
+      const void* src = a.x;
+      uint32_t nb = 0;
+      if (ee < a.E && t < a.T) {
+        if (t >= 0) {
+          src = xseq + t * a.x_tok + ee;
+          nb = 16;
+        } else if (hist) {
+          src = hist + (s * 3 + (t + 3)) * a.E + ee;
+          nb = 16;
         }
       }
-    } else {
-      // Euler-B, packed in state pairs: acc += e^{A R} (dt u) B.
-      const uint64_t R2 = pk2(R, R), v2 = pk2(dt * u, dt * u);
-#pragma unroll
-      for (int p = 0; p < kN / 2; ++p) {
-        const float4 b4 = Bt[p / 2];
-        const uint64_t b2 = (p & 1) ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
-        float y0, y1;
-        upk2(fmul2(R2, pk2(a2[2 * p], a2[2 * p + 1])), y0, y1);
-        // the last kSegPoly pairs take the FMA-pipe exp2, the others the SFU
-        const uint64_t decay = p >= kN / 2 - kSegPoly ? ex2_poly2(y0, y1) : pk2(ex2_approx(y0), ex2_approx(y1));
-        uint64_t ap = pk2(acc[2 * p], acc[2 * p + 1]);
-        ap = ffma2(decay, fmul2(v2, b2), ap);
-        upk2(ap, acc[2 * p], acc[2 * p + 1]);
-      }
+      cp_async_16z(smem_addr(&xs[r][q * kChPerChunk]), src, nb);
     }
-    R += dt;
+    for (int i = tid; i < kSegTok * (kN / 4); i += kSegThreads) {
+      const int r = i >> 2, q = i & 3;
+      const bool in = r < nt;
+      cp_async_16z(smem_addr(&Bs[r][4 * q]), in ? Bseq + (t_sub + r) * a.bc_tok + 4 * q : a.B, in ? 16 : 0);
+    }
+    if (tid < kSegTok) {
+      const bool in = tid < nt;
+      cp_async_4z(smem_addr(&dr[tid]), in ? a.dt_raw + s * a.dt_seq + t_sub + tid : a.dt_raw, in ? 4 : 0);
+    }
+    cp_async_all_done();
+    __syncthreads();
+
+    // x window of token t: rows t .. t+3 (tokens t-3 .. t); slides down by one row.
+    float x3 = IO<T>::to_f(xs[nt + 2][c]), x2 = IO<T>::to_f(xs[nt + 1][c]), x1 = IO<T>::to_f(xs[nt][c]);
+#pragma unroll 2
+    for (int t = nt - 1; t >= 0; --t) {
+      const float x0 = IO<T>::to_f(xs[t][c]);
+      const float conv = fmaf(cw.w, x3, fmaf(cw.z, x2, fmaf(cw.y, x1, fmaf(cw.x, x0, cb))));
+      x3 = x2;
+      x2 = x1;
+      x1 = x0;
+      const float u = silu(conv);
+      const float dt = dt_of(fmaf(dr[t], wdt, dtb), a.dt_min, a.dt_max);
+      const float4* Bt = reinterpret_cast<const float4*>(&Bs[t][0]);
+      if constexpr (ZOH) {
+#pragma unroll
+        for (int q = 0; q < kN / 4; ++q) {
+          const float4 b4 = Bt[q];
+          const float bq[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int n = 4 * q + i;
+            const float xa = dt * An[n];
+            const float inj = u * bq[i] * expm1_nonpos(xa, ex2_approx(xa * kLog2e)) / An[n];
+            acc[n] = fmaf(ex2_approx(a2[n] * R), inj, acc[n]);
+          }
+        }
+      } else {
+        // Euler-B, packed in state pairs: acc += e^{A R} (dt u) B.
+        const uint64_t R2 = pk2(R, R), v2 = pk2(dt * u, dt * u);
+#pragma unroll
+        for (int p = 0; p < kN / 2; ++p) {
+          const float4 b4 = Bt[p / 2];
+          const uint64_t b2 = (p & 1) ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
+          float y0, y1;
+          upk2(fmul2(R2, pk2(a2[2 * p], a2[2 * p + 1])), y0, y1);
+          // the last kSegPoly pairs take the FMA-pipe exp2, the others the SFU
+          const uint64_t decay = p >= kN / 2 - kSegPoly ? ex2_poly2(y0, y1) : pk2(ex2_approx(y0), ex2_approx(y1));
+          uint64_t ap = pk2(acc[2 * p], acc[2 * p + 1]);
+          ap = ffma2(decay, fmul2(v2, b2), ap);
+          upk2(ap, acc[2 * p], acc[2 * p + 1]);
+        }
+      }
+      R += dt;
+    }
   }
 
-  float* out = a.part + ((s * a.nblk + blk) * (kN + 1)) * a.E + e;
+  if (e < a.E) {
+    float* out = a.part + ((s * a.nblk + blk) * (kN + 1)) * a.E + e;
 #pragma unroll
-  for (int n = 0; n < kN; ++n) out[n * a.E] = acc[n];
-  out[kN * a.E] = R;
+    for (int n = 0; n < kN; ++n) out[n * a.E] = acc[n];
+    out[kN * a.E] = R;
+  }
 }
 
 // Fold the blocks of a segment in token order: h <- exp(A_n tot_k) h + part_k.
@@ -249,7 +264,7 @@ __global__ void segment_carry_kernel(const CarryArgs a) {
   a.h_out[i] = h;
 }
 
-int64_t seg_blocks(int64_t T) { return (T + kSegTok - 1) / kSegTok; }
+int64_t seg_blocks(int64_t T) { return (T + kSegTok * kSegSub - 1) / (kSegTok * kSegSub); }
 
 }  // namespace
 }  // namespace ssm

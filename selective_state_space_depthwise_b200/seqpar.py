@@ -59,9 +59,9 @@ def cuda_ops() -> SegmentOps:
 
 
 def _as_bits(t: torch.Tensor) -> torch.Tensor:
-    """Bit-exact integer view of the same width, for the exchange (every
-    backend moves integers; bf16 is not universal)."""
-    return t.view({2: torch.int16, 4: torch.int32, 8: torch.int64}[t.element_size()])
+    """Byte view for the exchange: every backend moves uint8 bit-exactly (NCCL
+    has no 16-bit integer type, and gloo's bf16 support varies)."""
+    return t.view(torch.uint8)
 
 
 def history_before(tails: list, lengths: list, r: int, hist0: torch.Tensor) -> torch.Tensor:

@@ -216,7 +216,7 @@ def test_segment_summary_workspace_and_argument_checks(lib):
     d = valid_dims()  # b=2, T=64, E=32
     assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(d)) == 2 * 1 * 17 * 32 * 4
     d300 = valid_dims(seqlen=300)
-    assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(d300)) == 2 * 5 * 17 * 32 * 4
+    assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(d300)) == 2 * 2 * 17 * 32 * 4
     assert lib.ssm_segment_summary_workspace_bytes(ctypes.byref(valid_dims(seqlen=0))) == 0
     assert lib.ssm_segment_summary_workspace_bytes(None) == 0
     w = fake_weights()
