@@ -530,8 +530,11 @@ def seq_parallel_main(args, w: W.Workload):
     seg = {k: inp[k][:, t0:t1] for k in ("x", "z", "B", "C", "dt_raw")}
     params = {k: inp[k] for k in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")}
 
+    lengths = [L * (r + 1) // world - L * r // world for r in range(world)]
+
     def step():
-        return seqpar.prefill_sequence_parallel(seg["x"], seg["z"], seg["B"], seg["C"], seg["dt_raw"], params)
+        return seqpar.prefill_sequence_parallel(seg["x"], seg["z"], seg["B"], seg["C"], seg["dt_raw"], params,
+                                                lengths=lengths)
 
     for _ in range(args.warmup):
         step()

@@ -78,25 +78,31 @@ def history_before(tails: list, lengths: list, r: int, hist0: torch.Tensor) -> t
 
 
 def prefill_sequence_parallel(x, z, B, C, dt_raw, params, *, group=None, conv_cache_in=None, ssm_state_in=None,
-                              ops: Optional[SegmentOps] = None, **opt):
+                              lengths: Optional[list] = None, ops: Optional[SegmentOps] = None, **opt):
     """This rank's part of a sequence-parallel prefill.
 
     x, z: [b, T_r, E]; B, C: [b, T_r, 16]; dt_raw: [b, T_r] -- segment r of
     each sequence, r = this rank in `group`, segments in rank order.
     conv_cache_in [b, 3, E] and ssm_state_in [b, E, 16] describe the state
     before segment 0 and are passed identically on every rank (or None).
-    `opt` holds dt_min, dt_max, discretization. Returns (y [b, T_r, E],
-    conv_cache_out, ssm_state_out); the last rank's caches are the sequence's."""
+    `lengths` (every rank's T, in rank order) saves the exchange of the
+    segment lengths, whose read-back synchronises the host; every rank must
+    pass it or none. `opt` holds dt_min, dt_max, discretization. Returns
+    (y [b, T_r, E], conv_cache_out, ssm_state_out); the last rank's caches are
+    the sequence's."""
     ops = ops or cuda_ops()
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     b, T, E = x.shape
     dev, io = x.device, x.dtype
 
     # 0. conv history: segment lengths and last HIST raw x rows of every rank.
-    lens = torch.tensor([T], dtype=torch.int64, device=dev)
-    all_lens = [torch.empty_like(lens) for _ in range(world)]
-    dist.all_gather(all_lens, lens, group=group)
-    lengths = [int(v.item()) for v in all_lens]
+    if lengths is None:
+        lens = torch.tensor([T], dtype=torch.int64, device=dev)
+        all_lens = [torch.empty_like(lens) for _ in range(world)]
+        dist.all_gather(all_lens, lens, group=group)
+        lengths = [int(v.item()) for v in all_lens]
+    elif len(lengths) != world or lengths[rank] != T:
+        raise ValueError("lengths must list every rank's segment length, this rank's equal to x.shape[1]")
     tail = torch.zeros((b, HIST, E), dtype=io, device=dev)
     k = min(HIST, T)
     if k:

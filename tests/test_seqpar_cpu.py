@@ -98,7 +98,7 @@ def test_prefill_segments_one_device_equals_unsplit(disc):
         torch.testing.assert_close(g, w, rtol=1e-11, atol=1e-13)
 
 
-def _worker(rank, world, port, lens, with_init, result_path):
+def _worker(rank, world, port, lens, with_init, rank_knows_lengths, result_path):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -106,8 +106,9 @@ def _worker(rank, world, port, lens, with_init, result_path):
         p, inp, init = problem(7, 2, sum(lens), 8, with_init)  # every rank draws the same global problem
         s0 = sum(lens[:rank])
         seg = {k: v[:, s0:s0 + lens[rank]] for k, v in inp.items()}
+        known = lens if rank_knows_lengths else None  # both ways of learning the lengths
         y, cc, st = seqpar.prefill_sequence_parallel(seg["x"], seg["z"], seg["B"], seg["C"], seg["dt_raw"], p,
-                                                     ops=oracle_ops(), **init)
+                                                     lengths=known, ops=oracle_ops(), **init)
         m = max(lens)  # gloo gathers equal sizes: pad each segment to the longest (check only)
         pad = torch.zeros((2, m, 8), dtype=torch.float64)
         pad[:, :lens[rank]] = y
@@ -119,12 +120,13 @@ def _worker(rank, world, port, lens, with_init, result_path):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("lens,with_init", [([23, 18], False), ([11, 2, 27], True)])
-def test_ranks_exchange_summaries_and_match_unsplit(tmp_path, lens, with_init):
+@pytest.mark.parametrize("lens,with_init,known", [([23, 18], False, False), ([11, 2, 27], True, False),
+                                                  ([11, 2, 27], False, True)])
+def test_ranks_exchange_summaries_and_match_unsplit(tmp_path, lens, with_init, known):
     world = len(lens)
-    port = 29700 + (os.getpid() % 200) + 7 * world
+    port = 29700 + (os.getpid() % 200) + 7 * world + 3 * known
     result = str(tmp_path / "sp.pt")
-    mp.start_processes(_worker, args=(world, port, lens, with_init, result), nprocs=world, join=True,
+    mp.start_processes(_worker, args=(world, port, lens, with_init, known, result), nprocs=world, join=True,
                        start_method="spawn")
     got = torch.load(result)
     p, inp, init = problem(7, 2, sum(lens), 8, with_init)
