@@ -57,9 +57,10 @@ def check_summary(got, want, label):
 @pytest.mark.parametrize("disc", ["euler", "zoh"])
 @pytest.mark.parametrize("t0,t1", [(0, 300), (0, 128), (5, 6), (7, 9), (100, 233), (0, 0)])
 def test_summary_matches_oracle(io_dtype, disc, t0, t1):
-    """Segments of one, two, 128 (one whole block) and ragged block counts;
-    E = 72 leaves a ragged 32-channel group; history from the tokens before
-    the segment (or zeros at the start)."""
+    """Segments of one, two, 128 (half of one 256-token block), 300 (a whole
+    block and a ragged second) and other ragged lengths; E = 72 leaves a ragged
+    128-channel group; history from the tokens before the segment (or zeros at
+    the start)."""
     w = small(io_dtype)
     inp = W.make_inputs(w, device="cuda")
     full = torch.cat([torch.zeros((w.batch, 3, w.d_inner), dtype=io_dtype, device="cuda"), inp["x"]], dim=1)
