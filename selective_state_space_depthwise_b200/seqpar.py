@@ -78,7 +78,8 @@ def history_before(tails: list, lengths: list, r: int, hist0: torch.Tensor) -> t
 
 
 def prefill_sequence_parallel(x, z, B, C, dt_raw, params, *, group=None, conv_cache_in=None, ssm_state_in=None,
-                              lengths: Optional[list] = None, ops: Optional[SegmentOps] = None, **opt):
+                              lengths: Optional[list] = None, final_caches_to_all: bool = False,
+                              ops: Optional[SegmentOps] = None, **opt):
     """This rank's part of a sequence-parallel prefill.
 
     x, z: [b, T_r, E]; B, C: [b, T_r, 16]; dt_raw: [b, T_r] -- segment r of
@@ -89,7 +90,8 @@ def prefill_sequence_parallel(x, z, B, C, dt_raw, params, *, group=None, conv_ca
     segment lengths, whose read-back synchronises the host; every rank must
     pass it or none. `opt` holds dt_min, dt_max, discretization. Returns
     (y [b, T_r, E], conv_cache_out, ssm_state_out); the last rank's caches are
-    the sequence's."""
+    the sequence's, and with final_caches_to_all=True (on every rank) they are
+    broadcast so that every rank returns the sequence's caches."""
     ops = ops or cuda_ops()
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     b, T, E = x.shape
@@ -132,7 +134,15 @@ def prefill_sequence_parallel(x, z, B, C, dt_raw, params, *, group=None, conv_ca
         h_in = ops.carry(torch.stack(gathered[:rank]).contiguous(), params, ssm_state_in)
 
     # 4. combine: the ordinary prefill of the segment from the carried state.
-    return ops.prefill(x, z, B, C, dt_raw, params, halo, h_in, **opt)
+    y, cc, st = ops.prefill(x, z, B, C, dt_raw, params, halo, h_in, **opt)
+    if final_caches_to_all and world > 1:
+        last = dist.get_global_rank(group, world - 1) if group is not None else world - 1
+        cc_bits = _as_bits(cc.contiguous())
+        dist.broadcast(cc_bits, src=last, group=group)
+        st = st.contiguous()
+        dist.broadcast(st, src=last, group=group)
+        cc = cc_bits.view(cc.dtype).view(cc.shape)
+    return y, cc, st
 
 
 def prefill_segments(x, z, B, C, dt_raw, params, bounds, *, conv_cache_in=None, ssm_state_in=None,

@@ -98,7 +98,7 @@ def test_prefill_segments_one_device_equals_unsplit(disc):
         torch.testing.assert_close(g, w, rtol=1e-11, atol=1e-13)
 
 
-def _worker(rank, world, port, lens, with_init, rank_knows_lengths, result_path):
+def _worker(rank, world, port, lens, with_init, rank_knows_lengths, result_path, to_all=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -108,13 +108,14 @@ def _worker(rank, world, port, lens, with_init, rank_knows_lengths, result_path)
         seg = {k: v[:, s0:s0 + lens[rank]] for k, v in inp.items()}
         known = lens if rank_knows_lengths else None  # both ways of learning the lengths
         y, cc, st = seqpar.prefill_sequence_parallel(seg["x"], seg["z"], seg["B"], seg["C"], seg["dt_raw"], p,
-                                                     lengths=known, ops=oracle_ops(), **init)
+                                                     lengths=known, final_caches_to_all=to_all, ops=oracle_ops(),
+                                                     **init)
         m = max(lens)  # gloo gathers equal sizes: pad each segment to the longest (check only)
         pad = torch.zeros((2, m, 8), dtype=torch.float64)
         pad[:, :lens[rank]] = y
         ys = [torch.empty_like(pad) for _ in lens]
         dist.all_gather(ys, pad)
-        if rank == world - 1:
+        if rank == (0 if to_all else world - 1):  # with to_all, rank 0 holds the sequence's caches too
             torch.save({"y": torch.cat([t[:, :n] for t, n in zip(ys, lens)], dim=1), "cc": cc, "st": st}, result_path)
     finally:
         dist.destroy_process_group()
@@ -130,6 +131,21 @@ def test_ranks_exchange_summaries_and_match_unsplit(tmp_path, lens, with_init, k
                        start_method="spawn")
     got = torch.load(result)
     p, inp, init = problem(7, 2, sum(lens), 8, with_init)
+    y, cc, st = unsplit(p, inp, init)
+    torch.testing.assert_close(got["y"], y, rtol=1e-11, atol=1e-13)
+    torch.testing.assert_close(got["st"], st, rtol=1e-11, atol=1e-13)
+    torch.testing.assert_close(got["cc"], cc, rtol=0, atol=0)
+
+
+def test_final_caches_reach_every_rank(tmp_path):
+    lens = [9, 14, 5]
+    world = len(lens)
+    port = 29900 + (os.getpid() % 50)
+    result = str(tmp_path / "sp_all.pt")
+    mp.start_processes(_worker, args=(world, port, lens, True, True, result, True), nprocs=world, join=True,
+                       start_method="spawn")
+    got = torch.load(result)
+    p, inp, init = problem(7, 2, sum(lens), 8, True)
     y, cc, st = unsplit(p, inp, init)
     torch.testing.assert_close(got["y"], y, rtol=1e-11, atol=1e-13)
     torch.testing.assert_close(got["st"], st, rtol=1e-11, atol=1e-13)
