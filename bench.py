@@ -24,6 +24,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -108,7 +109,10 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        # The raw samples go to SSM_CLOCKS_DIR (default: the system temp directory); the
+        # bench line carries their summary.
+        out_dir = os.environ.get("SSM_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"clocks_gpu{index}.csv")
 
     def __enter__(self):
         try:
