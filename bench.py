@@ -661,10 +661,21 @@ def main():
     peak_ct = alu_peak_ct_per_s(1965.0)
 
     extra = {}
+    if not args.no_e2e:
+        # Every rank moves its own inputs through the host path at the same time;
+        # the job's time is the slowest rank's (CUDA events, max over ranks).
+        if dist:
+            torch.distributed.barrier()
+        e2e = e2e_prefill(w, inp, steps=3)
+        if dist:
+            t = torch.tensor([e2e["ms_per_step"]], device="cuda")
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e["ms_per_step"] = round(float(t.item()), 3)
+            e2e["value"] = ct_step * world / (e2e["ms_per_step"] * 1e-3)
+            e2e["h2d_bytes_per_step"] *= world
+            e2e["d2h_bytes_per_step"] *= world
+        extra["e2e"] = e2e
     if rank == 0:
-        if not args.no_e2e:
-            extra["e2e"] = e2e_prefill(w, inp, steps=3)
-            extra["e2e"]["value"] *= world
         del inp
         torch.cuda.empty_cache()
         if not args.no_decode:
