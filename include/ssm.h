@@ -236,9 +236,11 @@ ssm_status ssm_prefill_host_static(const ssm_dims *dims, const ssm_weights *w, c
  *   B, C        [b, 16] fp32 at s*bc_seq_stride (dense: 16); dt_raw [b] at s*dt_seq_stride (dense: 1)
  *   y           [b, *] io_dtype at s*y_seq_stride (dense: E)
  *   conv_cache  [b, 3, E] io_dtype, dense, in-out
- *   ssm_state   [b, E, 16] fp32, dense, in-out
+ *   ssm_state   [b, E, 16] fp32, dense, in-out, 16-byte aligned
  * dims->seqlen is ignored. Consecutive calls on one stream continue the
  * sequence: prefill(L) followed by k calls equals prefill(L + k).
+ * The state of (sequence, 128 channels) moves between HBM and shared memory
+ * as one 8 KB TMA tile in each direction; a thread owns one channel.
  */
 ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const void *x, const void *z,
                            const float *B, const float *C, const float *dt_raw, void *y, void *conv_cache,
