@@ -15,6 +15,10 @@ basics" (molayo insights), "Technical details".
       token's injection; and brute force of the closed form on tiny segments;
   Q3  the carry: nothing enters segment 0 but h_init; explicit nested
       recurrences for one and three segments.
+
+The last test restates in float64 the block decomposition the GPU summary
+computes (backward walk over 256-token blocks, then an in-order fold) and
+checks it against the oracle's recurrence.
 """
 import math
 
@@ -195,3 +199,37 @@ def test_Q3_nested_recurrence_over_segments():
                     for j in range(r):  # h <- exp(A dtsum_j) h + h_zero_j
                         h = math.exp(A * summ[j, s, N, e]) * h + summ[j, s, n, e]
                     assert got[s, e, n] == pytest.approx(h, rel=1e-13, abs=1e-15)
+
+
+def test_block_decomposition_of_the_summary_matches_the_recurrence():
+    """The segment summary as the kernels compute it, restated in float64:
+    256-token blocks, each walked backwards with R = the dt mass after the
+    token, h_blk = sum_t exp(A R_t) dt_t B_t u_t, then the blocks folded in
+    order, h <- exp(A tot_k) h + h_blk_k. It must equal the oracle's token-by-
+    token recurrence (a different algorithm), here for a segment of 3 blocks
+    with a ragged last one."""
+    rng = np.random.default_rng(41)
+    b, T, E = 1, 600, 3
+    p = params(rng, E)
+    inp = inputs(rng, b, T, E)
+    hist = rng.normal(size=(b, 3, E))
+    want = oracle.segment_summary(inp["x"], inp["B"], inp["dt_raw"], p["conv_w"], p["conv_b"], p["w_dt"],
+                                  p["dt_bias"], p["A_log"], hist=hist)
+    xh = np.concatenate([hist, inp["x"]], axis=1)[0]  # raw rows, token t at t + 3
+    blk = 256
+    for e in range(E):
+        u = [silu(p["conv_b"][e] + sum(p["conv_w"][e, k] * xh[t + k, e] for k in range(4))) for t in range(T)]
+        dt = [min(max(softplus(inp["dt_raw"][0, t] * p["w_dt"][e] + p["dt_bias"][e]), 1e-4), 1.0) for t in range(T)]
+        A = -np.exp(p["A_log"][e])
+        h = np.zeros(N)
+        dtsum = 0.0
+        for t0 in range(0, T, blk):
+            hb = np.zeros(N)
+            R = 0.0
+            for t in range(min(T, t0 + blk) - 1, t0 - 1, -1):  # backwards through the block
+                hb += np.exp(A * R) * dt[t] * inp["B"][0, t] * u[t]
+                R += dt[t]
+            h = np.exp(A * R) * h + hb  # fold: R is now the block's dt total
+            dtsum += R
+        np.testing.assert_allclose(h, want[0, :N, e], rtol=1e-11, atol=1e-14)
+        np.testing.assert_allclose(dtsum, want[0, N, e], rtol=1e-13)
