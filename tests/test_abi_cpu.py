@@ -130,6 +130,10 @@ def test_binding_refuses_cpu_tensors(lib):
          for n in api.PARAM_NAMES}
     with pytest.raises(RuntimeError, match="no CPU path"):
         api.prefill(x, x, torch.zeros(1, 8, 16), torch.zeros(1, 8, 16), torch.zeros(1, 8), p)
+    with pytest.raises(RuntimeError, match="no CPU path"):
+        api.segment_summary(x, torch.zeros(1, 8, 16), torch.zeros(1, 8), p)
+    with pytest.raises(RuntimeError, match="no CPU path"):
+        api.segment_carry(torch.zeros(1, 1, 17, 8), p)
 
 
 def test_host_workspace_bytes_cover_two_chunk_slots(lib):
