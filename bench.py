@@ -11,9 +11,14 @@ workload (prompt 512, then 1024 one-token steps at b=256, E=7680), the
 roofline of the dominant kernel, the oracle timed on the host cores, and an
 end-to-end figure through the API with host buffers.
 
-With N > 1 (torchrun, one process per GPU) every rank runs the same per-GPU
-workload on its own channels (weak scaling; channels shard with no collective
-on the data path); the time is the max over ranks.
+The default launch takes the power decay path (the workloads use the pages'
+A initialisation, A_n = (n+1) A_0); the line also reports the per-state path
+on the same inputs (decay_paths) and the layer-shape and batched workloads
+(configs).
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own independent
+sequence of the workload (batch sharding: weak scaling, no collective on the
+data path); the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -40,24 +45,34 @@ PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
+# The headline metric, printed identically by both arms (the benchmark's).
+METRIC = "selective-scan channel-tokens/s; achieved HBM GB/s vs B200 peak"
+
 # SM resources used to derive the ALU roofline (B200, sm_100a): 148 SMs,
 # 16 SFU lanes and 128 FP32 lanes per SM per clock (the SFU and FFMA rates
 # were confirmed by a throughput probe on this GPU model).
 SMS, SFU_PER_CLK, FMA_PER_CLK = 148, 16, 128
-# Per channel-token the method needs 16 exp (dA) + 2 sigmoid (exp + reciprocal)
-# + 1 softplus (exp + log1p) = 22 SFU-class evaluations, and 4 FP32 ops per
-# state (dt*A, dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 84 FP32-pipe ops.
-SFU_OPS_PER_CT, FMA_OPS_PER_CT, POLY_EXP_FMA_OPS = 22, 84, 8
+# Algorithmic work per channel-token, by decay path:
+#  per-state exponentials: 16 exp (dA) + 2 sigmoid (exp + reciprocal) + 1
+#    softplus (exp + log1p) = 22 SFU-class evaluations; 4 FP32 ops per state
+#    (dt*A, dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 84 FP32-pipe ops;
+#  powers (A_n = (n+1) A_0): 1 exp (q) + 2 sigmoid + 1 softplus = 6 SFU-class
+#    evaluations; 15 multiplies for q^2..q^16, then 3 FP32 ops per state
+#    (dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 83 FP32-pipe ops.
+ALU_MODEL = {"per_state": (22, 84), "power": (6, 83)}
+POLY_EXP_FMA_OPS = 8
 
 
-def alu_peak_ct_per_s(sm_mhz: float) -> float:
-    """Best channel-tokens/s the SM pipes allow when k of the 22 SFU
-    evaluations move to an FMA-pipe polynomial (~8 FP32 ops each): minimise
-    max((22-k)/16, (84+8k)/128) clocks per channel-token per SM."""
+def alu_peak_ct_per_s(sm_mhz: float, path: str = "per_state") -> float:
+    """Best channel-tokens/s the SM pipes allow for the path's algorithmic
+    work, when k of its SFU evaluations may move to an FMA-pipe polynomial
+    (~8 FP32 ops each): minimise max((S-k)/16, (F+8k)/128) clocks per
+    channel-token per SM."""
+    sfu, fma = ALU_MODEL[path]
     best = math.inf
-    for i in range(0, 2201):
+    for i in range(0, 100 * sfu + 1):
         k = i / 100.0
-        best = min(best, max((SFU_OPS_PER_CT - k) / SFU_PER_CLK, (FMA_OPS_PER_CT + POLY_EXP_FMA_OPS * k) / FMA_PER_CLK))
+        best = min(best, max((sfu - k) / SFU_PER_CLK, (fma + POLY_EXP_FMA_OPS * k) / FMA_PER_CLK))
     return SMS * sm_mhz * 1e6 / best
 
 
@@ -224,34 +239,112 @@ def cpu_baseline(w: W.Workload, target_s: float = 10.0):
             "seconds": round(dt_s, 3)}
 
 
+def cpu_single_core(w: W.Workload, target_s: float = 4.0):
+    """The oracle on ONE host core over n channels of the workload (its full
+    length), n sized for about `target_s`."""
+    import oracle
+
+    oracle.build()
+    params = W.make_params(w)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    L, N = w.seqlen, w.d_state
+
+    def run(n):
+        x = torch.randn((n, L), generator=g).to(w.io_dtype).double().numpy()
+        z = torch.randn((n, L), generator=g).to(w.io_dtype).double().numpy()
+        B = torch.randn((1, L, N), generator=g).double().numpy()
+        C = torch.randn((1, L, N), generator=g).double().numpy()
+        dt = torch.randn((1, L), generator=g).double().numpy()
+        p = {k: v[:n].double().numpy() for k, v in params.items()}
+        t0 = time.perf_counter()
+        oracle.channels(x, z, B, C, dt, [0] * n, p["conv_w"], p["conv_b"], p["w_dt"], p["dt_bias"], p["A_log"],
+                        p["D"], lo=w.dt_min, hi=w.dt_max, threads=1)
+        return time.perf_counter() - t0
+
+    cal = run(4)
+    n = int(min(w.d_inner, max(4, 4 * target_s / max(cal, 1e-3))))
+    dt_s = run(n)
+    return {"value": n * L / dt_s, "unit": "channel-tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} channels x L={L} of the {w.name} workload, float64, one core",
+            "seconds": round(dt_s, 3)}
+
+
 # ------------------------------------------------------------------- GPU ---
 def make_device_inputs(w: W.Workload, rank: int):
     wr = w.scaled(seed=w.seed + 1000 * rank) if rank else w
     return W.make_inputs(wr, device="cuda", gen_device="cuda")
 
 
-def timed_prefill(inp, steps, warmup, dist):
+def timed_prefill(inp, steps, warmup, dist, tuning=None, clocks=True):
     from selective_state_space_depthwise_b200 import api
 
     args = (inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp)
-    y, cc, st = api.prefill(*args)
+    y, cc, st = api.prefill(*args, tuning=tuning)
     for _ in range(warmup):
-        api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st)
+        api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st, tuning=tuning)
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(torch.cuda.current_device()) if clocks else _NoClock() as clk:
         ev0.record(stream)
         for _ in range(steps):
-            api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st)
+            api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st, tuning=tuning)
         ev1.record(stream)
         torch.cuda.synchronize()
     if dist:
         torch.distributed.barrier()
     ms = ev0.elapsed_time(ev1)
     return ms, clk.summary()
+
+
+class _NoClock:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+    def summary(self):
+        return None
+
+
+def prefill_figures(w: W.Workload, ms_step: float, hbm_peak: float, peak_kind: str, path: str) -> dict:
+    """ct/s, the HBM fraction and the ALU fraction (against the path's own
+    algorithmic bound at 1965 MHz) of one prefill of `w` taking ms_step."""
+    ct = w.batch * w.seqlen * w.d_inner
+    gbs = min_bytes_prefill(w) / (ms_step * 1e-3) / 1e9
+    peak_ct = alu_peak_ct_per_s(1965.0, path)
+    return {"ms_per_step": round(ms_step, 4), "value": ct / (ms_step * 1e-3), "unit": "channel-tokens/s",
+            "alu": {"achieved": ct / (ms_step * 1e-3), "peak": peak_ct, "frac": round(ct / (ms_step * 1e-3) / peak_ct, 4),
+                    "path": path},
+            "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s", "frac": round(gbs / hbm_peak, 4),
+                    "peak_kind": peak_kind, "algorithmic_bytes_per_launch": min_bytes_prefill(w)}}
+
+
+def decay_path_bench(w: W.Workload, inp, hbm_peak: float, peak_kind: str, steps: int = 10, warmup: int = 3):
+    """The same workload on each decay path, CUDA events, inputs resident."""
+    out = {}
+    for name, path, tun in (("power", "power", None), ("per_state", "per_state", {"decay_path": 1})):
+        ms, _ = timed_prefill(inp, steps, warmup, False, tuning=tun, clocks=False)
+        out[name] = prefill_figures(w, ms / steps, hbm_peak, peak_kind, path)
+    out["note"] = ("power: decays as powers of q = exp(dt A_0), taken automatically by every CTA whose channels "
+                   "have A_n = (n+1) A_0 (the workloads' A initialisation); per_state: one exponential per state "
+                   "(forced with decay_path = 1; the path for any other A)")
+    return out
+
+
+def config_bench(name: str, hbm_peak: float, peak_kind: str, steps: int = 20, warmup: int = 3):
+    """Another prefill workload of the pages' shapes (parity config), both decay paths."""
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, device="cuda", gen_device="cuda")
+    res = {"workload": f"{w.name}: {w.note}; b={w.batch} L={w.seqlen} E={w.d_inner} N=16 K=4"}
+    res.update(decay_path_bench(w, inp, hbm_peak, peak_kind, steps, warmup))
+    res.pop("note")
+    del inp
+    torch.cuda.empty_cache()
+    return res
 
 
 def e2e_prefill(w: W.Workload, inp, steps):
@@ -561,10 +654,10 @@ def seq_parallel_main(args, w: W.Workload):
     if rank != 0:
         return
     value = b * L * E / (ms_step * 1e-3)
-    peak_ct = alu_peak_ct_per_s(1965.0)
+    peak_ct = alu_peak_ct_per_s(1965.0, "power")
     per_gpu = value / world
     print(json.dumps({
-        "metric": "selective-scan channel-tokens/s (prefill); achieved HBM GB/s vs B200 peak",
+        "metric": METRIC,
         "value": value, "unit": "channel-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
         "dtype": "f32", "io_dtype": "bf16" if w.io_dtype == torch.bfloat16 else "f32", "data": "synthetic",
@@ -589,6 +682,8 @@ def main():
     ap.add_argument("--workload", default="long_context", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-decode", action="store_true", help="skip the decode sub-benchmark")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the layer-shape and batched prefill sub-benchmarks")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end measurement")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--no-block", action="store_true",
@@ -623,7 +718,7 @@ def main():
                 per_step.append(cb["value"])
         value = statistics.median(per_step)
         cb["value"] = value
-        print(json.dumps({"impl": "reference", "metric": "selective-scan channel-tokens/s", "value": value,
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": value,
                           "unit": "channel-tokens/s", "n_gpus": args.gpus, "steps": args.steps,
                           "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                           "dtype": "f64", "data": "synthetic", "config": {"workload": w.note, "batch": w.batch,
@@ -657,10 +752,13 @@ def main():
     value = ct_step * world / (ms_step * 1e-3)
     per_gpu = ct_step / (ms_step * 1e-3)
     gbs = min_bytes_prefill(w) / (ms_step * 1e-3) / 1e9
-    sm_mhz = clocks["sm_mhz"] if clocks else 1965.0
-    peak_ct = alu_peak_ct_per_s(1965.0)
+    # Every workload uses the pages' A initialisation, so the default launch
+    # takes the power path in every CTA; its ALU bound is the roofline.
+    peak_ct = alu_peak_ct_per_s(1965.0, "power")
 
     extra = {}
+    if rank == 0:
+        extra["decay_paths"] = decay_path_bench(w, inp, hbm_peak, peak_kind)
     if not args.no_e2e:
         # Every rank moves its own inputs through the host path at the same time;
         # the job's time is the slowest rank's (CUDA events, max over ranks).
@@ -678,6 +776,8 @@ def main():
     if rank == 0:
         del inp
         torch.cuda.empty_cache()
+        if not args.no_configs:
+            extra["configs"] = [config_bench(n, hbm_peak, peak_kind) for n in ("axon_layer", "batched")]
         if not args.no_decode:
             extra["decode"] = decode_bench(W.WORKLOADS["decode"], rank, hbm_peak, peak_kind)
         if not args.no_block:
@@ -691,6 +791,7 @@ def main():
             extra["sequence_parallel"] = seqpar_bench(w)
         if not args.no_cpu and world == 1:
             extra["cpu_baseline"] = cpu_baseline(w)
+            extra["cpu_baseline"]["single_core_layer_shape"] = cpu_single_core(W.WORKLOADS["axon_layer"])
     if dist:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -698,18 +799,20 @@ def main():
         return
 
     line = {
-        "metric": "selective-scan channel-tokens/s (prefill); achieved HBM GB/s vs B200 peak",
+        "metric": METRIC,
         "value": value, "unit": "channel-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "io_dtype": "bf16" if w.io_dtype == torch.bfloat16 else "f32", "data": "synthetic",
         "config": {"workload": f"{w.name}: {w.note}; b={w.batch} L={w.seqlen} E={w.d_inner} N=16 K=4",
                    "batch": w.batch, "seq_len": w.seqlen, "d_inner": w.d_inner, "d_state": 16, "d_conv": 4,
-                   "parallelism": f"dp{world} (channel shards, no collective)" if world > 1 else "single GPU",
+                   "parallelism": (f"dp{world}: one independent sequence of the workload per GPU (batch sharding, "
+                                   f"no collective)") if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (no flush)" if min_bytes_prefill(w) > 126e6 else "inputs fit in L2"},
         "roofline": {"bound": "alu", "achieved": per_gpu, "peak": peak_ct, "unit": "channel-tokens/s",
                      "frac": round(per_gpu / peak_ct, 4),
-                     "peak_basis": "SFU 16 + FP32 128 lanes/clk/SM x 148 SMs at 1965 MHz, 22 SFU-class + 84 FP32 "
-                                   "ops per channel-token, best SFU/FMA split",
+                     "peak_basis": "SFU 16 + FP32 128 lanes/clk/SM x 148 SMs at 1965 MHz; the power decay path's "
+                                   "algorithmic work, 6 SFU-class + 83 FP32 ops per channel-token, best SFU/FMA "
+                                   "split (the per-state path's bound, 22 + 84, is in decay_paths)",
                      "traffic": ncu_traffic("prefill", w.name),
                      "hbm": {"achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                              "frac": round(gbs / hbm_peak, 4), "peak_kind": peak_kind,

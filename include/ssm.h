@@ -97,22 +97,22 @@ typedef struct {
   const float *conv_w, *conv_b, *w_dt, *dt_bias, *A_log, *D;
 } ssm_weights;
 
-/* Launch shape overrides for tests and tuning; pass NULL for the defaults.
- * kernel 1 (channel tiles): G = threads_per_channel lanes of one warp share a
- *   channel; channels_per_cta: G=1: 32/64/128, G=2: 16/32/64, G=4 or 8: 8/16/32.
- * kernel 2 (state slices): a CTA of G warps covers 32 channels and warp j owns
- *   state slice j of each; threads_per_channel = G in {2, 4, 8}.
- * kernel 3 (pipelined state slices): kernel 2 with the per-token work of the
- *   next stage overlapped with the scan of the current one; G in {4, 8}.
- * kernel 4: kernel 3 compiled for at most two resident CTAs per SM (a larger
- *   register budget); G = 4. The automatic choice takes it when
- *   batch * ceil(d_inner / 32) <= 2 * SMs, else kernel 3. */
+/* Launch overrides for tests and tuning; pass NULL for the defaults.
+ * kernel: 0 = auto; 3 = pipelined state slices (a CTA of 4 warps covers 32
+ *   channels, warp j owns states 4j..4j+3 of each, the per-token work of the
+ *   next 32-token stage overlaps the scan of the current one), built for three
+ *   resident CTAs per SM; 4 = the same code built for two CTAs per SM (a larger
+ *   register budget). Auto takes 4 when batch * ceil(d_inner / 32) <= 2 * SMs,
+ *   else 3. Any other value returns SSM_ERR_INVALID_ARG.
+ * decay_path: 0 = auto; 1 = every decay exp(dt A_n) as its own exponential.
+ *   Auto: a CTA whose 32 channels all have A_n = (n+1) A_0 within 2^-20
+ *   relative (the "State initialization" of "Axon-SSM": diagonals -1..-16)
+ *   forms the decays as powers q^(n+1) of q = exp(dt A_0), one exponential per
+ *   channel-token instead of 16; every other CTA uses per-state exponentials.
+ *   Euler-B only (ZOH always uses per-state exponentials). */
 typedef struct {
-  int32_t threads_per_channel; /* 0 = auto, else 1, 2, 4 or 8 */
-  int32_t channels_per_cta;    /* 0 = auto (kernel 1 only) */
-  int32_t kernel;              /* 0 = auto, 1 = channel tiles, 2 = state slices, 3/4 = pipelined slices */
-  int32_t poly_pairs;          /* -1 = auto; else state pairs per thread and token whose
-                                  exp2 runs as an FMA-pipe polynomial instead of on the SFU */
+  int32_t kernel;
+  int32_t decay_path;
 } ssm_tuning;
 
 /*
@@ -167,8 +167,12 @@ size_t ssm_prefill_workspace_bytes(const ssm_dims *dims);
  * Arguments.
  *   x, z, B, C, dt_raw, y   HOST pointers, laid out as in ssm_prefill. The
  *                           token and sequence strides of dims apply to them.
- *                           Page-locked (pinned) memory lets the copies overlap;
- *                           pageable memory gives the same result, serialised.
+ *                           They must be page-locked host memory (cudaHostAlloc,
+ *                           cudaHostRegister, torch pin_memory); pageable,
+ *                           device or managed memory returns
+ *                           SSM_ERR_INVALID_ARG. (A copy from or to pageable
+ *                           memory blocks the calling thread, and the enqueue
+ *                           below holds a library-wide lock.)
  *   conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out
  *                           device pointers, as in ssm_prefill.
  *   workspace               device scratch of at least
@@ -197,8 +201,12 @@ ssm_status ssm_prefill_host(const ssm_dims *dims, const ssm_weights *w, const vo
 size_t ssm_prefill_host_workspace_bytes(const ssm_dims *dims, int64_t chunk_tokens);
 
 /* Bytes of the device scratch that ssm_prefill_host_static owns: a static
- * device array of the library, one per device, reserved when the library's
- * device code is loaded. */
+ * device array of the library, one per device. It is reserved on a device
+ * when the library's device code is loaded there (at context creation under
+ * CUDA_MODULE_LOADING=EAGER, else at the first use of any of the library's
+ * kernels), whichever entry points the process calls, and held until exit:
+ * every process that loads libssm.so pays these bytes on each device it
+ * uses the library on. */
 #define SSM_HOST_STATIC_SCRATCH_BYTES ((size_t)128 << 20)
 
 /*
@@ -331,7 +339,18 @@ size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
  *  - scores = masked cb * exp(dA[l] - dA[s]) * dt[s] in bf16, times x;
  *  - C[l] in bf16, times prev_states^T;
  * as tcgen05 MMAs into two fp32 TMEM accumulators, combined as
- * acc_scores + exp(dA[l]) acc_state + D x and stored as bf16. The exponents are <= 0 for s <= l, so nothing overflows.
+ * acc_scores + exp(dA[l]) acc_state + D x and stored as bf16.
+ *
+ * Range. Each decay exp(dA[l] - dA[s]) is formed as the product of
+ * exp(dA[l] - dA[s1]) and exp(dA[s1] - dA[s]), s1 the last position of s's
+ * 8-position group (the group that holds l: one exponential per element).
+ * When dA_cumsum does not increase along a chunk (dt >= 0 and A <= 0, what a
+ * cumulative sum of dt A gives), every exponent is <= 0: no factor exceeds 1
+ * however strong the decay, a decayed term that underflows fp32 is 0, and
+ * exp(dA[l]) <= 1 as long as dA_cumsum starts at or below 0. Any other
+ * dA_cumsum is computed by the same formula, exactly while each of those
+ * exponents and dA[l] stays below about 80 (fp32 exp range); beyond that the
+ * output may hold inf or NaN.
  */
 typedef struct {
   int64_t batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size;
@@ -390,8 +409,28 @@ ssm_status ssm_segment_carry(const ssm_dims *dims, const ssm_weights *w, const f
                              const float *ssm_state_in, float *ssm_state_out, void *stream);
 
 /* Reads and clears the device error word that kernels set when a bounded
- * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed. */
+ * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed;
+ * SSM_ERR_DEVICE with the code in ssm_last_error() otherwise. Codes: 1 the
+ * prefill's TMA ring, 3-6 the block's x_proj kernel, 7-9 the chunk scan's
+ * operand and MMA waits, 11 the decode's state ring, SSM_SELFTEST_WAIT_CODE
+ * the self-test below. Every kernel's waits give up after about 2 s. */
 ssm_status ssm_check_device_error(void *stream);
+
+/* Error-word code written by ssm_selftest_bounded_wait. */
+#define SSM_SELFTEST_WAIT_CODE 99
+
+/*
+ * ssm_selftest_bounded_wait -- exercises the failure path the kernels use
+ * when a wait cannot complete (the failure detection of the bounded mbarrier
+ * waits): one CTA arms an mbarrier that can never complete its phase, waits
+ * for at most limit_ns (1e3 .. 2e9 ns), writes SSM_SELFTEST_WAIT_CODE to the
+ * device error word and returns. Nothing faults or hangs; the context stays
+ * usable. A following ssm_check_device_error on `stream` returns
+ * SSM_ERR_DEVICE and clears the word. Enqueued on `stream`; out-of-range
+ * limit_ns returns SSM_ERR_INVALID_ARG. Not part of the computation (the
+ * pages have no counterpart): a check a caller can run on its own device.
+ */
+ssm_status ssm_selftest_bounded_wait(int64_t limit_ns, void *stream);
 
 /* Static description of a status code. */
 const char *ssm_status_string(ssm_status s);

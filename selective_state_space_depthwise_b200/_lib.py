@@ -18,6 +18,7 @@ SSM_DISC_EULER_B, SSM_DISC_ZOH = 0, 1
 
 # Every symbol include/ssm.h declares (checked by the CPU test suite).
 SSM_HOST_STATIC_SCRATCH_BYTES = 128 << 20  # include/ssm.h
+SSM_SELFTEST_WAIT_CODE = 99  # include/ssm.h
 
 EXPORTED = (
     "ssm_prefill",
@@ -34,6 +35,7 @@ EXPORTED = (
     "ssm_segment_carry",
     "ssm_decode_step",
     "ssm_check_device_error",
+    "ssm_selftest_bounded_wait",
     "ssm_status_string",
     "ssm_last_error",
     "ssm_version",
@@ -92,8 +94,7 @@ class SsmWeights(ctypes.Structure):
 
 
 class SsmTuning(ctypes.Structure):
-    _fields_ = [("threads_per_channel", ctypes.c_int32), ("channels_per_cta", ctypes.c_int32),
-                ("kernel", ctypes.c_int32), ("poly_pairs", ctypes.c_int32)]
+    _fields_ = [("kernel", ctypes.c_int32), ("decay_path", ctypes.c_int32)]
 
 
 class SsmError(RuntimeError):
@@ -144,6 +145,8 @@ def load(path: str = LIB_PATH):
     lib.ssm_decode_step.restype = st
     lib.ssm_check_device_error.argtypes = [p]
     lib.ssm_check_device_error.restype = st
+    lib.ssm_selftest_bounded_wait.argtypes = [ctypes.c_int64, p]
+    lib.ssm_selftest_bounded_wait.restype = st
     lib.ssm_status_string.argtypes = [st]
     lib.ssm_status_string.restype = ctypes.c_char_p
     lib.ssm_last_error.argtypes = []

@@ -113,8 +113,10 @@ def prefill(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None
     work = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
     tun = None
     if tuning:
-        tun = _lib.SsmTuning(int(tuning.get("threads_per_channel", 0)), int(tuning.get("channels_per_cta", 0)),
-                             int(tuning.get("kernel", 0)), int(tuning.get("poly_pairs", -1)))
+        unknown = set(tuning) - {"kernel", "decay_path"}
+        if unknown:
+            raise ValueError(f"unknown tuning keys {sorted(unknown)} (kernel, decay_path)")
+        tun = _lib.SsmTuning(int(tuning.get("kernel", 0)), int(tuning.get("decay_path", 0)))
     st = lib.ssm_prefill_ex(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
                             _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(y), _ptr(conv_cache_out),
                             _ptr(ssm_state_out), _ptr(work), ws, ctypes.byref(tun) if tun else None, _stream(stream))
@@ -132,8 +134,8 @@ def prefill_host(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in
                  ssm_state_out=None, dt_min=1e-4, dt_max=1.0, discretization="euler", chunk_tokens=0, workspace=None,
                  stream=None, static_scratch=False):
     """Full-sequence block core with the token tensors in host memory
-    (ssm_prefill_host): x, z, B, C, dt_raw and y are CPU tensors (pinned for
-    overlapped copies), shaped and strided as for `prefill`; the parameters and
+    (ssm_prefill_host): x, z, B, C, dt_raw and y are pinned CPU tensors
+    (pageable ones are refused), shaped and strided as for `prefill`; the parameters and
     the caches are CUDA tensors on the current device. The copies and kernels
     are only enqueued: synchronise `stream` before reading y. With
     static_scratch=True the call goes to ssm_prefill_host_static, which takes
@@ -379,3 +381,18 @@ def decode_step(x, z, B, C, dt_raw, params, conv_cache, ssm_state, *, y=None, dt
                              _ptr(y), _ptr(conv_cache), _ptr(ssm_state), _stream(stream))
     _lib.check(st)
     return y
+
+
+def check_device_error(stream=None):
+    """ssm_check_device_error: synchronises `stream`, then raises SsmError
+    (status SSM_ERR_DEVICE) if a kernel's bounded wait gave up since the last
+    check, clearing the device error word."""
+    lib = _lib.load()
+    _lib.check(lib.ssm_check_device_error(_stream(stream)))
+
+
+def selftest_bounded_wait(limit_ns=1_000_000, stream=None):
+    """ssm_selftest_bounded_wait: a kernel whose wait can never complete gives
+    up after limit_ns and reports through the device error word."""
+    lib = _lib.load()
+    _lib.check(lib.ssm_selftest_bounded_wait(int(limit_ns), _stream(stream)))

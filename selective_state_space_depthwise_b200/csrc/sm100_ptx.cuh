@@ -41,21 +41,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with `parity` to complete, for at most ~2 s. On timeout
-// the error word gets `code` and the caller continues (no thread ever blocks
-// forever, and control flow around CTA barriers stays uniform).
-static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* err, int code) {
+// Wait for the phase with `parity` to complete, for at most `limit_ns`. On
+// timeout the error word gets `code` and the caller continues (no thread ever
+// blocks forever, and control flow around CTA barriers stays uniform).
+static __device__ __noinline__ bool mbar_wait_bounded_ns(uint32_t bar, uint32_t parity, int* err, int code,
+                                                         uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > 2000000000ull) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       if (err) atomicExch(err, code);
       return false;
     }
   }
+}
+
+// The kernels' waits: bounded at ~2 s.
+static __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* err, int code) {
+  return mbar_wait_bounded_ns(bar, parity, err, code, 2000000000ull);
 }
 
 // ------------------------------------------------------------- cp.async ---

@@ -16,12 +16,17 @@
 //     dA and dt;
 //  2. as soon as C and prev_states are in, one thread issues eight tcgen05 MMAs
 //     C x prev_states^T into accumulator 1;
-//  3. meanwhile thread s < 128 forms F[s] = exp(dA[s0] - dA[s]) dt[s] (s0 = s
-//     rounded down to a multiple of 8), and thread t turns the 64-column atom
-//     t / 128 of row l = t mod 128 of the cb tile, in place, into the scores
-//     cb[l, s] exp(dA[l] - dA[s0]) F[s] for s <= l, zero above (one exponential
-//     per row and 8-column group; the exponents are <= 0 or small, so nothing
-//     overflows): the TMA layout is already the MMA's K-major operand;
+//  3. meanwhile thread s < 128 forms F[s] = exp(dA[s1] - dA[s]) dt[s], s1 the
+//     last column of s's 8-column group (s1 = s | 7), and thread t turns the
+//     64-column atom t / 128 of row l = t mod 128 of the cb tile, in place,
+//     into the scores cb[l, s] exp(dA[l] - dA[s]) dt[s] for s <= l, zero above:
+//     a group wholly at or below the diagonal (s1 <= l) as cb exp(dA[l] -
+//     dA[s1]) F[s], one exponential per row and group; the group that holds
+//     the diagonal with one exponential per element. Every exponent is
+//     dA[later] - dA[earlier], <= 0 when dA_cumsum does not increase along the
+//     chunk (dt >= 0, A <= 0), so no factor exceeds 1 however strong the
+//     decay, and a factor underflows to 0 only where the exact product does.
+//     The TMA layout is already the MMA's K-major operand;
 //  4. one thread issues eight MMAs scores x x (x as an MN-major B operand) into
 //     accumulator 0 and commits both;
 //  5. warps w and w + 4 read lanes 32 (w mod 4) .. of columns 32 (w / 4) .. of
@@ -189,7 +194,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
                   umma_desc_k_sw128(sb + S::kPrev + (kk >> 2) * S::kAtomRows64 + (kk & 3) * 32), ssd_idesc(false),
                   kk > 0);
   }
-  if (tid < kCs) F[tid] = ex2_approx((sdA[tid & ~7] - sdA[tid]) * kLog2e) * sdt[tid];
+  if (tid < kCs) F[tid] = ex2_approx((sdA[tid | 7] - sdA[tid]) * kLog2e) * sdt[tid];
   const float dAl = sdA[l];
   mbar_wait_bounded(full_scores, 0u, a.err, 8);
   __syncthreads();  // F complete
@@ -206,9 +211,18 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     }
     float f[8];
     unpack8(*p, f);
-    const float e = s0 <= l ? ex2_approx((dAl - sdA[s0]) * kLog2e) : 0.0f;
+    if (s0 + 7 <= l) {  // whole group at or below the diagonal: row factor x column factor, both <= 1
+      const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) f[q] = s0 + q <= l ? f[q] * e * F[s0 + q] : 0.0f;
+      for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
+    } else if (s0 <= l) {  // the diagonal group: each decay on its own
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        f[q] = s0 + q <= l ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) f[q] = 0.0f;
+    }
     *p = pack8(f);
   }
   fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core

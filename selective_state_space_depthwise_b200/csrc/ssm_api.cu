@@ -8,6 +8,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
+#include "sm100_ptx.cuh"
 #include "ssm.h"
 #include "ssm_internal.h"
 
@@ -125,19 +128,39 @@ void fill_weights(ssm::KernelArgs& a, const ssm_weights* w) {
 
 __device__ int g_device_error = 0;
 
+// One thread arms an mbarrier for two arrivals and gives it one, so the phase
+// can never complete; its bounded wait gives up after limit_ns, writes `code`
+// to the error word and the kernel returns. No memory operation is pending on
+// the barrier when the CTA exits.
+__global__ void bounded_wait_selftest_kernel(int* err, uint64_t limit_ns, int code) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = ssm::smem_u32(&bar);
+  ssm::mbar_init(b, 2);
+  ssm::mbar_fence_init();
+  ssm::mbar_arrive(b);
+  ssm::mbar_wait_bounded_ns(b, 0u, err, code, limit_ns);
+}
+
 }  // namespace
 
 namespace ssm {
 // Device address of the error word on the current device (looked up once per
 // device; host code must not pass the symbol itself to a kernel).
+// Any host thread may call this; the per-device cache entries are atomics
+// (two threads that race on an empty entry both look the address up and
+// store the same value).
 int* device_error_ptr() {
-  static int* cache[64] = {};
+  static std::atomic<int*> cache[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64 && cache[dev]) return cache[dev];
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached) {
+    int* p = cache[dev].load(std::memory_order_acquire);
+    if (p) return p;
+  }
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-  if (dev >= 0 && dev < 64) cache[dev] = static_cast<int*>(p);
+  if (cached) cache[dev].store(static_cast<int*>(p), std::memory_order_release);
   return static_cast<int*>(p);
 }
 }  // namespace ssm
@@ -177,14 +200,15 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
   (void)workspace;
 
   ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current());
+  int decay_path = 0;
   if (tuning) {
     if (tuning->kernel) sh.kernel = tuning->kernel;
-    if (tuning->poly_pairs >= 0) sh.npoly = tuning->poly_pairs;
-    if (tuning->threads_per_channel) sh.G = tuning->threads_per_channel;
-    if (tuning->channels_per_cta) sh.NCH = tuning->channels_per_cta;
-    if (sh.kernel == 1 && !tuning->channels_per_cta && sh.G > 1) sh.NCH = 32;
     if (!ssm::prefill_shape_supported(sh))
-      return fail(SSM_ERR_INVALID_ARG, "tuning: unsupported shape kernel=%d G=%d NCH=%d", sh.kernel, sh.G, sh.NCH);
+      return fail(SSM_ERR_INVALID_ARG, "tuning: kernel=%d is not built (3 or 4)", sh.kernel);
+    if (tuning->decay_path != 0 && tuning->decay_path != 1)
+      return fail(SSM_ERR_INVALID_ARG, "tuning: decay_path=%d (0 = auto, 1 = per-state exponentials)",
+                  tuning->decay_path);
+    decay_path = tuning->decay_path;
   }
 
   ssm::KernelArgs a{};
@@ -205,6 +229,7 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
   a.s = s;
   a.dt_min = dims->dt_min;
   a.dt_max = dims->dt_max;
+  a.decay_path = decay_path;
   a.err = device_error_ptr();
   if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   cudaError_t err = ssm::launch_prefill(a, dims->io_dtype == SSM_BF16, dims->discretization == SSM_DISC_ZOH, sh,
@@ -277,6 +302,18 @@ ssm_status ssm_check_device_error(void* stream) {
     cudaStreamSynchronize(st);
     return fail(SSM_ERR_DEVICE, "a kernel reported device error code %d", v);
   }
+  return ok();
+}
+
+ssm_status ssm_selftest_bounded_wait(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 2000000000LL)
+    return fail(SSM_ERR_INVALID_ARG, "limit_ns=%lld must be in [1e3, 2e9]", (long long)limit_ns);
+  int* err = device_error_ptr();
+  if (!err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
+  bounded_wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(
+      err, static_cast<uint64_t>(limit_ns), SSM_SELFTEST_WAIT_CODE);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
   return ok();
 }
 

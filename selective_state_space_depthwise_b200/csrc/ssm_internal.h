@@ -37,17 +37,14 @@ struct KernelArgs {
   int64_t batch, L, E;
   Strides s;
   float dt_min, dt_max;
-  int* err;  // device error word: a kernel whose bounded wait gave up writes a code here
+  int decay_path;  // prefill: 0 = powers of one exponential where A_n = (n+1) A_0, 1 = one exponential per state
+  int* err;        // device error word: a kernel whose bounded wait gave up writes a code here
 };
 
-// Prefill launch shape. kernel 1: G lanes of a warp per channel (each holding
-// 16/G states), NCH channels per CTA. kernel 2: CTAs of G warps over 32
-// channels, warp j holding state slice j (NCH unused).
+// Prefill launch shape: kernel 3 (pipelined state slices, register budget of
+// three CTAs per SM) or kernel 4 (the same at two CTAs per SM).
 struct PrefillShape {
-  int G;
-  int NCH;
   int kernel;
-  int npoly;  // state pairs per thread and token whose exp2 runs on the FMA pipe
 };
 
 PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t L, int num_sms);

@@ -174,6 +174,30 @@ ssm_status validate(HostPrefill& hp, int64_t chunk_tokens) {
   return SSM_OK;
 }
 
+// x, z, B, C, dt_raw and y must be page-locked host memory. A copy from or
+// to pageable memory makes the calling thread wait for it (for the kernels
+// queued before it on its stream, too) while this library's enqueue mutex is
+// held, which would stall every other thread and could deadlock one whose
+// stream waits on work queued through this library.
+ssm_status check_page_locked(const HostPrefill& hp) {
+  const void* p[6] = {hp.x, hp.z, hp.B, hp.C, hp.dt, hp.y};
+  const char* names[6] = {"x", "z", "B", "C", "dt_raw", "y"};
+  for (int i = 0; i < 6; ++i) {
+    cudaPointerAttributes at{};
+    const cudaError_t e = cudaPointerGetAttributes(&at, p[i]);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return ssm::fail(SSM_ERR_CUDA, "pointer attributes of %s: %s", names[i], cudaGetErrorString(e));
+    }
+    if (at.type != cudaMemoryTypeHost)
+      return ssm::fail(SSM_ERR_INVALID_ARG, "%s must be page-locked host memory, got %s", names[i],
+                       at.type == cudaMemoryTypeUnregistered ? "pageable host memory"
+                       : at.type == cudaMemoryTypeDevice   ? "device memory"
+                                                           : "managed memory");
+  }
+  return SSM_OK;
+}
+
 // Enqueues the chunk pipeline. `after` (may be NULL) is an event the first
 // copy also waits for. On return the caller's stream waits for every copy
 // and kernel enqueued here, on success and on failure.
@@ -307,6 +331,7 @@ ssm_status ssm_prefill_host(const ssm_dims* dims, const ssm_weights* w, const vo
   if (workspace_bytes < need)
     return ssm::fail(SSM_ERR_INVALID_ARG, "workspace of %zu bytes, need %zu", workspace_bytes, need);
   const int64_t T = clip_chunk(chunk_tokens > 0 ? chunk_tokens : kDefaultChunk, dims->seqlen);
+  if ((st = check_page_locked(hp)) != SSM_OK) return st;
 
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState* ds = nullptr;
@@ -342,6 +367,7 @@ ssm_status ssm_prefill_host_static(const ssm_dims* dims, const ssm_weights* w, c
     return ssm::fail(SSM_ERR_UNSUPPORTED, "batch * d_inner too large for the %zu-byte static scratch",
                      kStaticScratchBytes);
   }
+  if ((st = check_page_locked(hp)) != SSM_OK) return st;
 
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState* ds = nullptr;

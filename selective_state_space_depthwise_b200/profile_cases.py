@@ -1,13 +1,14 @@
 """Small, fixed launches of the kernels for profiler captures.
 
-    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL G N NPOLY] [E]
+    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL DECAY_PATH] [E]
     python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
     python -m selective_state_space_depthwise_b200.profile_cases block NAME [L]
     python -m selective_state_space_depthwise_b200.profile_cases ssd NAME
     python -m selective_state_space_depthwise_b200.profile_cases segment WORKLOAD [T]
 
 prefill: three launches of the named workload's prefill (optionally shortened
-to L tokens, optionally with an explicit launch shape and E channels); decode: a 4-token
+to L tokens, optionally with an explicit kernel (3 or 4) and decay path (0 auto,
+1 per-state exponentials), and E channels); decode: a 4-token
 prompt, then three decode steps at the decode workload's shape (batch 256,
 E=7680, 252 MB of state); block: three block forwards of the named block
 workload (optionally L tokens); segment: three segment summaries of the first
@@ -33,8 +34,8 @@ def prefill_case(name: str, L: int = 0, shape=None, E: int = 0):
         w = w.scaled(d_inner=E)
     tun = None
     if shape:
-        k, g, n, p = shape
-        tun = {"kernel": k, "threads_per_channel": g, "channels_per_cta": n, "poly_pairs": p}
+        k, dp = shape
+        tun = {"kernel": k, "decay_path": dp}
     inp = W.make_inputs(w, device="cuda", gen_device="cuda")
     args = (inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp)
     for _ in range(3):
@@ -94,8 +95,8 @@ def segment_case(name: str, T: int = 0):
 if __name__ == "__main__":
     if sys.argv[1] == "prefill":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
-        shape = tuple(int(v) for v in sys.argv[4:8]) if len(sys.argv) > 7 else None
-        E = int(sys.argv[8]) if len(sys.argv) > 8 else 0
+        shape = tuple(int(v) for v in sys.argv[4:6]) if len(sys.argv) > 5 else None
+        E = int(sys.argv[6]) if len(sys.argv) > 6 else 0
         prefill_case(sys.argv[2], L, shape, E)
     elif sys.argv[1] == "ssd":
         ssd_case(sys.argv[2])

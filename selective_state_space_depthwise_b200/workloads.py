@@ -65,6 +65,22 @@ WORKLOADS = {
 }
 
 
+def clip_stress_channels(w: Workload):
+    """(low, high): the channel indices whose dt_bias make_params pins to
+    softplus^-1(dt_min) and softplus^-1(dt_max) (empty unless clip_stress).
+    Replays the same draws, so it always agrees with make_params."""
+    if not w.clip_stress:
+        return torch.empty(0, dtype=torch.long), torch.empty(0, dtype=torch.long)
+    g = torch.Generator(device="cpu").manual_seed(w.seed)
+    E, K = w.d_inner, w.d_conv
+    torch.randn(E, K, generator=g, dtype=torch.float32)
+    torch.rand(E, generator=g, dtype=torch.float32)
+    torch.rand(E, generator=g, dtype=torch.float64)
+    perm = torch.randperm(E, generator=g)
+    n5 = E // 20
+    return perm[:n5].sort().values, perm[n5:2 * n5].sort().values
+
+
 def softplus_inv(d: torch.Tensor) -> torch.Tensor:
     """Inverse of softplus, used only to place dt_bias (an initialisation recipe)."""
     return torch.log(torch.expm1(d))

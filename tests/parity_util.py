@@ -74,20 +74,29 @@ def compare(io_dtype, got, want, label=""):
     return e_y, e_h
 
 
-def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_max=1.0, max_elems=1 << 25):
-    """Every (sequence, channel) of a run against the oracle. The channels go
-    in blocks (whole sequences, or channel ranges of one long sequence) of at
-    most about `max_elems` tokens x channels, so full-size workloads fit in
-    host memory; the relative L2 of y and of the state is accumulated over the
-    whole run and the conv cache must match bit for bit. Returns (e_y, e_h)."""
-    y, cache, state = got
+def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_max=1.0, max_elems=1 << 25,
+                 subsets=None):
+    """Every (sequence, channel) of a run against the oracle. `got` is one
+    (y, cache, state) triple or a dict {name: triple} of runs on the same
+    inputs (the oracle then runs once for all of them). The channels go in
+    blocks (whole sequences, or channel ranges of one long sequence) of at most
+    about `max_elems` tokens x channels, so full-size workloads fit in host
+    memory. Per (sequence, channel) the squared errors are kept, so besides the
+    relative L2 over the whole run this reports, and bounds by the same
+    tolerance, the worst single channel and each named channel subset
+    (`subsets`: {name: channel indices}, applied in every sequence). The conv
+    cache must match bit for bit. Returns {name: report} (or the report of the
+    single run), a report being {"y", "state", "worst_y", "worst_state",
+    "worst_channel", "subsets": {name: (y, state)}}."""
+    runs = got if isinstance(got, dict) else {"": got}
     x, z = inp["x"], inp["z"]
     b, L, E = x.shape
     p = {k: inp[k].detach().to("cpu").double().numpy() for k in ("conv_w", "conv_b", "w_dt", "dt_bias", "A_log", "D")}
     per_seq = L * E
     seqs_per_block = max(1, max_elems // max(per_seq, 1))
     ch_per_block = E if seqs_per_block > 1 or per_seq <= max_elems else max(1, max_elems // max(L, 1))
-    acc = np.zeros(4)  # |dy|^2, |y|^2, |dh|^2, |h|^2
+    # per (sequence, channel): |dy|^2, |y|^2, |dh|^2, |h|^2
+    acc = {n: np.zeros((b, E, 4)) for n in runs}
     for s0 in range(0, b, seqs_per_block):
         s1 = min(b, s0 + seqs_per_block)
         Bn = inp["B"][s0:s1].detach().to("cpu").double().numpy()
@@ -104,15 +113,47 @@ def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_
             out_o, h_o, c_o = oracle.channels(xs, zs, Bn, Cn, dtn, bidx, tile(p["conv_w"]), tile(p["conv_b"]),
                                               tile(p["w_dt"]), tile(p["dt_bias"]), tile(p["A_log"]), tile(p["D"]),
                                               lo=dt_min, hi=dt_max, disc=disc)
-            ys = y[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, L).double().cpu().numpy()
-            hs = state[s0:s1, e0:e1, :].reshape(-1, 16).double().cpu().numpy()
-            cs = cache[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, 3).double().cpu().numpy()
-            assert np.array_equal(cs, c_o), f"{label}: conv_cache differs in sequences {s0}..{s1 - 1}"
-            assert np.isfinite(ys).all() and np.isfinite(hs).all(), f"{label}: non-finite output"
             want_y = round_io(out_o, io_dtype)
-            acc += [np.sum((ys - want_y) ** 2), np.sum(want_y ** 2), np.sum((hs - h_o) ** 2), np.sum(h_o ** 2)]
-    e_y = float(np.sqrt(acc[0] / acc[1])) if acc[1] > 0 else float(np.sqrt(acc[0]))
-    e_h = float(np.sqrt(acc[2] / acc[3])) if acc[3] > 0 else float(np.sqrt(acc[2]))
-    assert e_y <= TOL[io_dtype], f"{label}: y rel-L2 {e_y:.3e} > {TOL[io_dtype]:.0e}"
-    assert e_h <= TOL[io_dtype], f"{label}: state rel-L2 {e_h:.3e} > {TOL[io_dtype]:.0e}"
-    return e_y, e_h
+            for name, (y, cache, state) in runs.items():
+                ys = y[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, L).double().cpu().numpy()
+                hs = state[s0:s1, e0:e1, :].reshape(-1, 16).double().cpu().numpy()
+                cs = cache[s0:s1, :, e0:e1].permute(0, 2, 1).reshape(-1, 3).double().cpu().numpy()
+                assert np.array_equal(cs, c_o), f"{label}{name}: conv_cache differs in sequences {s0}..{s1 - 1}"
+                assert np.isfinite(ys).all() and np.isfinite(hs).all(), f"{label}{name}: non-finite output"
+                blk = np.stack([np.sum((ys - want_y) ** 2, axis=1), np.sum(want_y ** 2, axis=1),
+                                np.sum((hs - h_o) ** 2, axis=1), np.sum(h_o ** 2, axis=1)], axis=1)
+                acc[name][s0:s1, e0:e1] = blk.reshape(s1 - s0, n_e, 4)
+
+    def rl2(a):
+        return (float(np.sqrt(a[..., 0].sum() / a[..., 1].sum())) if a[..., 1].sum() > 0 else float(np.sqrt(a[..., 0].sum())),
+                float(np.sqrt(a[..., 2].sum() / a[..., 3].sum())) if a[..., 3].sum() > 0 else float(np.sqrt(a[..., 2].sum())))
+
+    tol = TOL[io_dtype]
+    reports = {}
+    for name, a in acc.items():
+        e_y, e_h = rl2(a)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            cy = np.sqrt(np.where(a[..., 1] > 0, a[..., 0] / a[..., 1], a[..., 0]))
+            ch = np.sqrt(np.where(a[..., 3] > 0, a[..., 2] / a[..., 3], a[..., 2]))
+        wy = np.unravel_index(int(np.argmax(cy)), cy.shape)
+        rep = {"y": e_y, "state": e_h, "worst_y": float(cy.max()), "worst_state": float(ch.max()),
+               "worst_channel": (int(wy[0]), int(wy[1])), "subsets": {}}
+        for sname, idx in (subsets or {}).items():
+            idx = np.asarray(idx, dtype=np.int64)
+            if idx.size:
+                rep["subsets"][sname] = rl2(a[:, idx])
+        tag = f"{label}{' ' + name if name else ''}"
+        assert e_y <= tol, f"{tag}: y rel-L2 {e_y:.3e} > {tol:.0e}"
+        assert e_h <= tol, f"{tag}: state rel-L2 {e_h:.3e} > {tol:.0e}"
+        assert rep["worst_y"] <= tol, f"{tag}: worst channel {rep['worst_channel']} y rel-L2 {rep['worst_y']:.3e}"
+        assert rep["worst_state"] <= tol, f"{tag}: worst channel state rel-L2 {rep['worst_state']:.3e}"
+        for sname, (sy, sh) in rep["subsets"].items():
+            assert sy <= tol and sh <= tol, f"{tag}: subset {sname} rel-L2 y {sy:.3e}, state {sh:.3e}"
+        reports[name] = rep
+    return reports if isinstance(got, dict) else reports[""]
+
+
+def format_report(rep) -> str:
+    sub = ", ".join(f"{k} y {v[0]:.2e} / state {v[1]:.2e}" for k, v in rep["subsets"].items())
+    return (f"y {rep['y']:.2e}, state {rep['state']:.2e}; worst channel {rep['worst_channel']}: "
+            f"y {rep['worst_y']:.2e}, state worst {rep['worst_state']:.2e}" + (f"; {sub}" if sub else ""))

@@ -255,3 +255,8 @@ def test_segment_carry_argument_checks(lib):
     assert call(d, sout=None) == _lib.SSM_ERR_INVALID_ARG
     assert call(d, sin=FAKE + 2) == _lib.SSM_ERR_INVALID_ARG
     assert call(valid_dims(d_conv=3)) == _lib.SSM_ERR_UNSUPPORTED
+
+
+def test_selftest_rejects_bad_limits_on_the_host(lib):
+    for bad in (0, 999, 2_000_000_001):
+        assert lib.ssm_selftest_bounded_wait(bad, None) == _lib.SSM_ERR_INVALID_ARG

@@ -10,15 +10,17 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import TOL, all_channels, compare, compare_full, gather, oracle_prefill, rel_l2, round_io
+from parity_util import TOL, all_channels, compare, compare_full, format_report, gather, oracle_prefill, rel_l2
 from selective_state_space_depthwise_b200 import api
 from selective_state_space_depthwise_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
 
-# (kernel, G, channels per CTA): kernel 1 = channel tiles, kernel 2 = state slices (32 channels per CTA)
-SHAPES = [(1, 1, 32), (1, 1, 64), (1, 1, 128), (1, 2, 16), (1, 2, 32), (1, 2, 64), (1, 4, 8), (1, 4, 16), (1, 4, 32),
-          (1, 8, 8), (1, 8, 16), (1, 8, 32), (2, 2, 0), (2, 4, 0), (2, 8, 0), (3, 4, 0), (3, 8, 0), (4, 4, 0)]
+# (kernel, decay path): kernel 3 / 4 = pipelined state slices at a register
+# budget of 3 / 2 CTAs per SM; decay path 0 = auto (powers of one exponential
+# where A_n = (n+1) A_0, which the workloads' A initialisation satisfies),
+# 1 = one exponential per state.
+SHAPES = [(3, 0), (3, 1), (4, 0), (4, 1)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -43,36 +45,21 @@ def device_inputs(w, gen_device="cpu"):
 
 
 @pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("shape", SHAPES, ids=[f"k{k}_G{g}_N{n}" for k, g, n in SHAPES])
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"k{k}_d{d}" for k, d in SHAPES])
 def test_prefill_every_launch_shape(io_dtype, shape):
-    # E = 48 leaves a ragged channel tile for N >= 32; L = 200 leaves a ragged stage.
+    # E = 48 leaves a ragged channel tile; L = 200 leaves a ragged stage.
     w = small_workload(io_dtype)
     inp = device_inputs(w)
-    k, g, n = shape
-    y, cc, st = run_prefill(inp, tuning={"kernel": k, "threads_per_channel": g, "channels_per_cta": n})
+    k, d = shape
+    y, cc, st = run_prefill(inp, tuning={"kernel": k, "decay_path": d})
     chans = all_channels(w.batch, w.d_inner)
-    compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"kernel {k} G{g} N{n}")
+    compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"kernel {k} decay path {d}")
 
 
-POLY = [(1, 1, 32, 1), (1, 1, 32, 3), (1, 1, 64, 2), (1, 1, 128, 1), (2, 2, 0, 1), (2, 2, 0, 2), (2, 4, 0, 1)]
-
-
-@pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("shape", POLY, ids=[f"k{k}_G{g}_N{n}_p{p}" for k, g, n, p in POLY])
-def test_prefill_fma_pipe_exp2_variants(io_dtype, shape):
-    """Launch shapes where some decays use the FMA-pipe exp2 polynomial."""
-    w = small_workload(io_dtype, b=2, L=150, E=64, seed=13)
-    inp = device_inputs(w)
-    k, g, n, p = shape
-    y, cc, st = run_prefill(inp, tuning={"kernel": k, "threads_per_channel": g, "channels_per_cta": n, "poly_pairs": p})
-    chans = all_channels(w.batch, w.d_inner)
-    compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"poly {shape}")
-
-
-@pytest.mark.parametrize("kg", [(2, 2), (2, 4), (2, 8), (3, 4), (3, 8), (4, 4)])
-def test_slice_kernel_lengths_history_and_zoh(kg):
-    """The state-slice kernels on short sequences, with incoming caches, and ZOH."""
-    kern, g = kg
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"k{k}_d{d}" for k, d in SHAPES])
+def test_kernel_lengths_history_and_zoh(shape):
+    """Short sequences, incoming caches, and ZOH, in every launch shape."""
+    kern, d = shape
     for L, E, disc in ((1, 32, "euler"), (3, 40, "euler"), (33, 64, "zoh"), (97, 32, "euler")):
         w = small_workload(torch.bfloat16, b=2, L=L, E=E, seed=90 + L)
         inp = device_inputs(w)
@@ -80,10 +67,42 @@ def test_slice_kernel_lengths_history_and_zoh(kg):
         cc_in = torch.randn((2, 3, E), generator=gen).to(torch.bfloat16).cuda()
         st_in = torch.randn((2, E, 16), generator=gen).cuda()
         y, cc, st = run_prefill(inp, conv_cache_in=cc_in, ssm_state_in=st_in, discretization=disc,
-                                tuning={"kernel": kern, "threads_per_channel": g})
+                                tuning={"kernel": kern, "decay_path": d})
         chans = all_channels(2, E)
         want = oracle_prefill(inp, chans, conv_cache_in=cc_in, ssm_state_in=st_in, disc=disc)
-        compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"kernel {kern} G{g} L{L} {disc}")
+        compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"kernel {kern} path {d} L{L} {disc}")
+
+
+@pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
+def test_decay_paths_mixed_channels(io_dtype):
+    """A_log perturbed in some 32-channel tiles (and in one single channel of
+    another tile): those tiles must take the per-state path, the rest the
+    power path. Checked three ways: both runs (auto and forced per-state)
+    match the oracle on every channel; on the perturbed tiles auto is bit-equal
+    to forced per-state; on the untouched tiles the two differ (different
+    arithmetic), which shows the power path ran there."""
+    b, L, E = 2, 150, 160  # 5 tiles of 32 channels
+    w = small_workload(io_dtype, b=b, L=L, E=E, seed=77)
+    inp = device_inputs(w)
+    A_log = inp["A_log"].clone()
+    g = torch.Generator(device="cpu").manual_seed(3)
+    A_log[32:64] += 0.05 * torch.randn((32, 16), generator=g).cuda()  # tile 1: every channel
+    A_log[128:160] = torch.log(torch.rand((32, 16), generator=g) * 8 + 0.5).cuda()  # tile 4: random A
+    A_log[64 + 5, 7] += 1e-3  # tile 2: one state of one channel
+    inp = dict(inp, A_log=A_log.contiguous())
+    y_auto, cc_a, st_auto = run_prefill(inp)
+    y_gen, cc_g, st_gen = run_prefill(inp, tuning={"decay_path": 1})
+    chans = all_channels(b, E)
+    want = oracle_prefill(inp, chans)
+    compare(io_dtype, gather(y_auto, cc_a, st_auto, chans), want, label="mixed auto")
+    compare(io_dtype, gather(y_gen, cc_g, st_gen, chans), want, label="mixed per-state")
+    for t in (1, 2, 4):
+        sl = slice(32 * t, 32 * t + 32)
+        assert torch.equal(st_auto[:, sl], st_gen[:, sl]) and torch.equal(y_auto[..., sl], y_gen[..., sl]), \
+            f"tile {t}: perturbed A must take the per-state path"
+    for t in (0, 3):
+        sl = slice(32 * t, 32 * t + 32)
+        assert not torch.equal(st_auto[:, sl], st_gen[:, sl]), f"tile {t}: structured A must take the power path"
 
 
 def test_tiny_workload_fp32_full():
@@ -202,12 +221,21 @@ def test_decode_zoh():
 @pytest.mark.parametrize("name", ["axon_layer", "batched", "long_context"])
 def test_full_size_prefill_all_channels(name):
     """The workload at full size, in the default launch shape the benchmark
-    times, against the oracle on every (sequence, channel)."""
+    times (auto decay path: powers of one exponential, since the workloads use
+    the pages' A initialisation) and with one exponential per state, against
+    the oracle on every (sequence, channel). The long-context workload also
+    reports its two clip-stressed channel subsets on their own."""
     w = W.WORKLOADS[name]
     inp = device_inputs(w, gen_device="cuda")
-    y, cc, st = run_prefill(inp)
-    e_y, e_h = compare_full(w.io_dtype, inp, (y, cc, st), label=name)
-    print(f"{name}: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e} over all {w.batch * w.d_inner} channels")
+    runs = {"auto": run_prefill(inp), "per-state": run_prefill(inp, tuning={"decay_path": 1})}
+    lo, hi = W.clip_stress_channels(w)
+    subsets = {"dt at dt_min": lo.tolist(), "dt at dt_max": hi.tolist()} if w.clip_stress else None
+    if subsets:
+        stressed = set(subsets["dt at dt_min"]) | set(subsets["dt at dt_max"])
+        subsets["unstressed"] = [e for e in range(w.d_inner) if e not in stressed]
+    reps = compare_full(w.io_dtype, inp, runs, label=name, subsets=subsets)
+    for path, rep in reps.items():
+        print(f"{name} [{path}]: {format_report(rep)} over all {w.batch * w.d_inner} channels")
 
 
 def test_full_size_decode_all_channels():
@@ -216,5 +244,5 @@ def test_full_size_decode_all_channels():
     w = W.WORKLOADS["decode"]
     inp = device_inputs(w, gen_device="cuda")
     y, cc, st = decode_run(inp, w, w.seqlen, w.decode_steps)
-    e_y, e_h = compare_full(w.io_dtype, inp, (y, cc, st), label="decode")
-    print(f"decode: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e} over all {w.batch * w.d_inner} channels")
+    rep = compare_full(w.io_dtype, inp, (y, cc, st), label="decode")
+    print(f"decode: {format_report(rep)} over all {w.batch * w.d_inner} channels")

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from parity_util import all_channels, compare, gather, oracle_prefill
-from selective_state_space_depthwise_b200 import api
+from selective_state_space_depthwise_b200 import _lib, api
 from selective_state_space_depthwise_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -77,20 +77,20 @@ def test_host_prefill_equals_device_prefill(io_dtype, b, L, E, chunk, with_cache
     assert torch.equal(got[2], want[2]), "ssm_state_out differs"
 
 
-def test_host_prefill_strided_host_layouts_and_pageable_memory():
-    """x and z as halves of one [b, L, 2E] host buffer, B and C inside one
-    [b, L, 40] buffer, dt_raw with a padded sequence stride, y written into a
-    strided view of a wider host buffer; pageable (unpinned) memory."""
+def test_host_prefill_strided_host_layouts():
+    """x and z as halves of one [b, L, 2E] pinned host buffer, B and C inside
+    one [b, L, 40] buffer, dt_raw with a padded sequence stride, y written into
+    a strided view of a wider host buffer."""
     b, L, E = 2, 150, 64
     inp = inputs(torch.bfloat16, b, L, E, seed=7)
     want = run_device(inp)
-    xz = torch.cat([inp["x"], inp["z"]], dim=2).cpu()
-    bc = torch.zeros((b, L, 40), dtype=torch.float32)
+    xz = torch.cat([inp["x"], inp["z"]], dim=2).cpu().pin_memory()
+    bc = torch.zeros((b, L, 40), dtype=torch.float32).pin_memory()
     bc[:, :, 0:16] = inp["B"].cpu()
     bc[:, :, 16:32] = inp["C"].cpu()
-    dtb = torch.zeros((b, L + 5), dtype=torch.float32)
+    dtb = torch.zeros((b, L + 5), dtype=torch.float32).pin_memory()
     dtb[:, :L] = inp["dt_raw"].cpu()
-    out = torch.zeros((b, L, E + 16), dtype=torch.bfloat16)
+    out = torch.zeros((b, L, E + 16), dtype=torch.bfloat16).pin_memory()
     y = out[:, :, 8:8 + E]
     got = api.prefill_host(xz[:, :, :E], xz[:, :, E:], bc[:, :, 0:16], bc[:, :, 16:32], dtb[:, :L], inp, y=y,
                            chunk_tokens=48)
@@ -99,6 +99,27 @@ def test_host_prefill_strided_host_layouts_and_pageable_memory():
     assert torch.count_nonzero(out[:, :, :8]) == 0 and torch.count_nonzero(out[:, :, 8 + E:]) == 0
     assert torch.equal(y, want[0].cpu())
     assert torch.equal(got[1], want[1]) and torch.equal(got[2], want[2])
+
+
+@pytest.mark.parametrize("static", [False, True])
+@pytest.mark.parametrize("which", ["y", "x", "dt_raw"])
+def test_host_prefill_rejects_pageable_buffers(which, static):
+    """A pageable host buffer (here y, x or dt_raw) is refused with
+    SSM_ERR_INVALID_ARG before anything is enqueued, on both host entry points."""
+    b, L, E = 1, 40, 32
+    inp = inputs(torch.bfloat16, b, L, E, seed=9)
+    host = host_copy(inp)
+    y = torch.empty((b, L, E), dtype=torch.bfloat16).pin_memory()
+    if which == "y":
+        y = torch.empty((b, L, E), dtype=torch.bfloat16)
+    else:
+        host[which] = host[which].clone()  # clone of a pinned tensor is pageable
+    assert not (y if which == "y" else host[which]).is_pinned()
+    with pytest.raises(_lib.SsmError) as err:
+        api.prefill_host(host["x"], host["z"], host["B"], host["C"], host["dt_raw"], inp, y=y, chunk_tokens=16,
+                         static_scratch=static)
+    assert err.value.status == _lib.SSM_ERR_INVALID_ARG
+    assert "page-locked" in str(err.value)
 
 
 def test_host_prefill_against_the_oracle():

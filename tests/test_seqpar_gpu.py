@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import TOL, all_channels, compare, compare_full, gather, oracle_prefill, rel_l2
+from parity_util import TOL, all_channels, compare, compare_full, format_report, gather, oracle_prefill, rel_l2
 from selective_state_space_depthwise_b200 import api, seqpar
 from selective_state_space_depthwise_b200 import workloads as W
 
@@ -142,8 +142,8 @@ def test_full_size_long_context_in_eight_segments():
     bounds = [L * r // 8 for r in range(9)]
     y, cc, st = seqpar.prefill_segments(inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp, bounds)
     torch.cuda.synchronize()
-    e_y, e_h = compare_full(w.io_dtype, inp, (y, cc, st), label="long_context in 8 segments")
-    print(f"long_context / 8 segments: y rel-L2 {e_y:.2e}, state rel-L2 {e_h:.2e}")
+    rep = compare_full(w.io_dtype, inp, (y, cc, st), label="long_context in 8 segments")
+    print(f"long_context / 8 segments: {format_report(rep)}")
 
     T = bounds[1]
     summ = api.segment_summary(inp["x"][:, :T], inp["B"][:, :T], inp["dt_raw"][:, :T], inp)
