@@ -490,7 +490,42 @@ def block_bench(name: str, bf16_peak: float, steps: int = 10, warmup: int = 3):
                             "frac": round(tflops / bf16_peak, 4), "flops_per_step": flops,
                             "note": "GEMM FLOPs of in_proj, x_proj and out_proj over the whole block time "
                                     "(the scan core's SFU-bound time is included in the denominator)"},
-            "gpu_launches_per_step": 4}
+            "gpu_launches_per_step": 4,
+            "note": "in_proj and out_proj are this library's tcgen05 GEMM; no library GEMM runs"}
+
+
+def gemm_bench(bf16_peak: float, steps: int = 20, warmup: int = 3):
+    """The block's two projection GEMMs (ssm_proj_gemm, tcgen05) timed alone
+    at the layer shape (2048 tokens, D = 2560, E = 7680) and at the
+    long-context block's 65536 tokens: us per call by CUDA events, TFLOP/s
+    against the measured dense bf16 peak (burst: each is timed alone)."""
+    from selective_state_space_depthwise_b200 import api
+
+    D, E = 2560, 7680
+    out = []
+    for M in (2048, 65536):
+        for name, N, K in (("in_proj", 2 * E, D), ("out_proj", D, E)):
+            g = torch.Generator(device="cuda").manual_seed(M + N)
+            A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+            Wt = (torch.randn((N, K), device="cuda", generator=g) * K ** -0.5).to(torch.bfloat16)
+            C = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            for _ in range(warmup):
+                api.proj_gemm(A, Wt, out=C)
+            torch.cuda.synchronize()
+            stream = torch.cuda.current_stream()
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            for _ in range(steps):
+                api.proj_gemm(A, Wt, out=C)
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            us = ev0.elapsed_time(ev1) * 1e3 / steps
+            tflops = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            out.append({"gemm": name, "M": M, "N": N, "K": K, "us": round(us, 2), "tflops": round(tflops, 1),
+                        "peak": bf16_peak, "frac": round(tflops / bf16_peak, 4)})
+            del A, Wt, C
+    torch.cuda.empty_cache()
+    return out
 
 
 def ssd_bench(name: str, hbm_peak: float, bf16_peak: float, steps: int = 20, warmup: int = 3):
@@ -784,6 +819,8 @@ def main():
             torch.cuda.empty_cache()
             bf16_peak = load_bf16_peak()
             extra["block"] = [block_bench(n, bf16_peak) for n in W.BLOCK_WORKLOADS]
+            torch.cuda.empty_cache()
+            extra["projection_gemms"] = gemm_bench(bf16_peak)
             torch.cuda.empty_cache()
             extra["ssd_chunk_scan"] = ssd_bench("ssd_chunk_scan", hbm_peak, bf16_peak)
         if not args.no_seqpar:

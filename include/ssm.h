@@ -264,12 +264,13 @@ ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const voi
  *   y            = the block core of ssm_prefill    (dt_proj, softplus, clip, scan, D skip, y * SiLU(z))
  *   out          = y @ W_out^T                      out_proj (E -> D)
  *
- * Implementation. in_proj and out_proj are plain GEMMs (cuBLASLt, bf16
- * operands, fp32 accumulation). x_proj is one fused kernel: it computes u
- * from x tile by tile straight into tensor-core operand tiles (tcgen05 MMA,
- * TMEM accumulator), so u never reaches memory. The core is ssm_prefill's
- * kernel, reading x and z in place from the in_proj output. No projection has
- * a bias.
+ * Implementation. in_proj and out_proj are this library's tcgen05 GEMM
+ * (ssm_proj_gemm: bf16 operands, fp32 accumulation in TMEM, bf16 out).
+ * x_proj is one fused kernel: it computes u from x tile by tile straight into
+ * tensor-core operand tiles (tcgen05 MMA, TMEM accumulator), so u never
+ * reaches memory. The core is ssm_prefill's kernel, reading x and z in place
+ * from the in_proj output; out_proj reads the core's gated output as its A
+ * operand. No projection has a bias. No library GEMM is called.
  *
  * Arguments.
  *   dims      batch, seqlen, d_model (D, a multiple of 8), d_inner (E, a
@@ -285,8 +286,8 @@ ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const voi
  *             output), so chained calls equal one call over the whole sequence.
  *   workspace device scratch of ssm_block_workspace_bytes(dims) bytes,
  *             256-byte aligned. It holds the in_proj output (b L 2E bf16),
- *             B / C / dt_raw (b L 33 fp32), the gated core output (b L E bf16)
- *             and the GEMM workspace.
+ *             B / C / dt_raw (b L 33 fp32) and the gated core output
+ *             (b L E bf16).
  *
  * Ordering and errors. Everything is enqueued on `stream`, with no host
  * synchronisation. Argument errors return before any work is queued.
@@ -312,6 +313,19 @@ ssm_status ssm_block_forward(const ssm_block_dims *dims, const ssm_weights *w, c
 
 /* Workspace bytes of ssm_block_forward for `dims` (0 for invalid dims). */
 size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
+
+/*
+ * ssm_proj_gemm -- one projection of the block, C = A . W^T: in_proj (A =
+ * hidden [M, D], W = W_in [2E, D]) and out_proj (A = the core's gated output
+ * [M, E], W = W_out [D, E]) of "Axon-SSM: selective state space model",
+ * "Algorithm" diagram, as ssm_block_forward runs them.
+ *   A  [M, K] bf16, row-major;  W  [N, K] bf16, row-major;  C  [M, N] bf16
+ * Device pointers, 16-byte aligned; K and N multiples of 8; 0 < M, N, K <=
+ * 2^31; C must not alias A or W. fp32 accumulation, C rounded to bf16 (RNE).
+ * One persistent kernel (tcgen05 MMAs into TMEM, TMA operand ring, TMA
+ * stores) enqueued on `stream`; no workspace.
+ */
+ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64_t N, int64_t K, void *stream);
 
 /*
  * ssm_ssd_chunk_scan -- the output of the Mamba-2 (SSD) chunk scan, "What is

@@ -318,6 +318,27 @@ def block_forward(hidden, params, proj, *, conv_cache_in=None, ssm_state_in=None
     return out, conv_cache_out, ssm_state_out
 
 
+def proj_gemm(A, W, *, out=None, stream=None):
+    """One projection of the block (ssm_proj_gemm): out = A @ W^T with A [M, K]
+    and W [N, K] contiguous bf16 CUDA tensors; returns out [M, N] bf16."""
+    lib = _lib.load()
+    M, K = A.shape
+    N = W.shape[0]
+    dev = A.device
+    for n, t in (("A", A), ("W", W), ("out", out)):
+        _need_cuda(n, t, dev)
+        if t is not None and (t.dtype != torch.bfloat16 or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous bfloat16 tensor")
+    if W.shape[1] != K:
+        raise ValueError("A [M, K] and W [N, K] must share K")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if out.shape != (M, N):
+        raise ValueError("out must be [M, N]")
+    _lib.check(lib.ssm_proj_gemm(_ptr(A), _ptr(W), _ptr(out), M, N, K, _stream(stream)))
+    return out
+
+
 def ssd_chunk_scan(cb, x, dt, dA_cumsum, C, prev_states, D=None, *, out=None, stream=None):
     """Mamba-2 chunk-scan output (ssm_ssd_chunk_scan). cb [b, nc, G, cs, cs],
     x [b, L, H, P], C [b, L, G, N], prev_states [b, nc, H, P, N]: bf16;

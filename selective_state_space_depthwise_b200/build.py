@@ -20,7 +20,6 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libssm.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-CUDA_LIB = os.path.join(os.path.dirname(os.path.dirname(NVCC)), "lib64")  # cuBLASLt (in_proj / out_proj GEMMs)
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-I", INCLUDE, "-I", CSRC]
 
@@ -61,8 +60,7 @@ def build(verbose: bool = False, force: bool = False, lib: str = LIB, build_dir:
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose, build_dir, defines), srcs))
     if force or _stale(lib, objs):
-        cmd = [NVCC] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart", "-lcublasLt", "-Xlinker", "-rpath",
-                                                            "-Xlinker", CUDA_LIB]
+        cmd = [NVCC] + ARCH + ["-shared", "-o", lib] + objs + ["-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stderr}")

@@ -1,7 +1,8 @@
 // block.cu -- the AxonSSMBlock forward around the prefill core ("Axon-SSM:
 // selective state space model", "Algorithm" diagram): in_proj and out_proj as
-// plain cuBLASLt GEMMs, x_proj as one fused tcgen05 kernel, the core as
-// prefill.cu's kernel reading x and z in place from the in_proj output.
+// this library's tcgen05 GEMM (gemm.cu), x_proj as one fused tcgen05 kernel,
+// the core as prefill.cu's kernel reading x and z in place from the in_proj
+// output, and out_proj reading the core's gated output y as its A operand.
 //
 // x_proj kernel. A CTA owns 128 tokens of one sequence (the MMA's M) and a
 // contiguous range of the E channels, walked in chunks of 64 (K). Per chunk:
@@ -23,12 +24,9 @@
 // distributed shared memory, the rows of tokens [r 128/S, (r+1) 128/S) and
 // writes B, C ([b, L, 32] fp32) and dt_raw ([b, L] fp32). u never reaches
 // memory. Every mbarrier wait is bounded.
-#include <cublasLt.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
-
-#include <mutex>
 
 #include "sm100_ptx.cuh"
 #include "ssm.h"
@@ -308,60 +306,11 @@ cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, in
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------ cuBLASLt ---
-std::mutex g_lt_mutex;
-cublasLtHandle_t g_lt[64] = {};
-
-cublasLtHandle_t lt_handle() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(g_lt_mutex);
-  if (!g_lt[dev] && cublasLtCreate(&g_lt[dev]) != CUBLAS_STATUS_SUCCESS) g_lt[dev] = nullptr;
-  return g_lt[dev];
-}
-
-// out[M][N] = act[M][K] . w[N][K]^T, bf16 in and out, fp32 accumulation; all
-// row-major and dense. In cuBLASLt's column-major terms: out^T = w^T' . act^T.
-ssm_status gemm_bf16_nt(const void* act, const void* w, void* out, int64_t M, int64_t N, int64_t K, void* ws,
-                        size_t ws_bytes, cudaStream_t st, const char* what) {
-  cublasLtHandle_t h = lt_handle();
-  if (!h) return fail(SSM_ERR_CUDA, "%s: no cuBLASLt handle", what);
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  cublasStatus_t s = cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F);
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, K, N, K);
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, K, M, K);
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, N, M, N);
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulPreferenceCreate(&pref);
-  if (s == CUBLAS_STATUS_SUCCESS)
-    s = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
-                                             sizeof(ws_bytes));
-  cublasLtMatmulHeuristicResult_t res{};
-  int found = 0;
-  if (s == CUBLAS_STATUS_SUCCESS) s = cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &res, &found);
-  const float alpha = 1.0f, beta = 0.0f;
-  if (s == CUBLAS_STATUS_SUCCESS && found > 0)
-    s = cublasLtMatmul(h, op, &alpha, w, la, act, lb, &beta, out, lc, out, lc, &res.algo, ws, ws_bytes, st);
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  if (s != CUBLAS_STATUS_SUCCESS) return fail(SSM_ERR_CUDA, "%s: cuBLASLt status %d", what, static_cast<int>(s));
-  if (found == 0) return fail(SSM_ERR_UNSUPPORTED, "%s: cuBLASLt found no algorithm", what);
-  return SSM_OK;
-}
-
 constexpr size_t kAlign = 256;
-constexpr size_t kLtWorkspace = 32u << 20;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct BlockLayout {
-  size_t xz, bc, dt, y, lt, bytes;
+  size_t xz, bc, dt, y, bytes;
 };
 
 BlockLayout block_layout(const ssm_block_dims* d) {
@@ -372,7 +321,6 @@ BlockLayout block_layout(const ssm_block_dims* d) {
   l.bc = off, off = align_up(off + M * 32 * 4);
   l.dt = off, off = align_up(off + M * 4);
   l.y = off, off = align_up(off + M * E * 2);
-  l.lt = off, off = align_up(off + kLtWorkspace);
   l.bytes = off;
   return l;
 }
@@ -449,10 +397,13 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   float* dt = reinterpret_cast<float*>(ws + lay.dt);
   void* y = ws + lay.y;
 
+  int* err_word = ssm::device_error_ptr();
+  if (!err_word) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // in_proj: xz[M][2E] = hidden[M][D] . W_in[2E][D]^T
-  if ((st = ssm::gemm_bf16_nt(hidden, proj->w_in, xz, M, 2 * E, Dm, ws + lay.lt, ssm::kLtWorkspace, cs,
-                              "in_proj")) != SSM_OK)
-    return st;
+  cudaError_t err = ssm::gemm_bf16_tn(hidden, proj->w_in, xz, M, 2 * E, Dm, 0, sms, err_word, cs);
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "in_proj launch: %s", cudaGetErrorString(err));
   // x_proj (fused with conv + SiLU): B, C, dt_raw
   ssm::XprojArgs xa{};
   xa.conv_w = w->conv_w;
@@ -462,11 +413,8 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   xa.dt_raw = dt;
   xa.L = L;
   xa.E = E;
-  xa.err = ssm::device_error_ptr();
-  if (!xa.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaError_t err = ssm::launch_xproj(xa, xz, proj->w_x, b, sms, cs);
+  xa.err = err_word;
+  err = ssm::launch_xproj(xa, xz, proj->w_x, b, sms, cs);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "x_proj launch: %s", cudaGetErrorString(err));
   // the core, on x and z in place in xz
   cd.x_tok_stride = cd.z_tok_stride = 2 * E;
@@ -481,9 +429,8 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
                         ssm_state_out, nullptr, 0, stream)) != SSM_OK)
     return st;
   // out_proj: out[M][D] = y[M][E] . W_out[D][E]^T
-  if ((st = ssm::gemm_bf16_nt(y, proj->w_out, out, M, Dm, E, ws + lay.lt, ssm::kLtWorkspace, cs, "out_proj")) !=
-      SSM_OK)
-    return st;
+  err = ssm::gemm_bf16_tn(y, proj->w_out, out, M, Dm, E, 0, sms, err_word, cs);
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "out_proj launch: %s", cudaGetErrorString(err));
   return ssm::fail(SSM_OK, "");
 }
 

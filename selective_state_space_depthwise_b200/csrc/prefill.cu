@@ -16,16 +16,17 @@
 // Thread 0 re-arms a slot right after the CTA has finished with it; every
 // wait on the ring's mbarriers is bounded.
 //
-// Work split (state slices). A CTA is kG = 4 warps over 32 channels (lane =
-// channel); warp j holds states 4j..4j+3 of every channel, so B and C are
-// warp-broadcast loads and x, z, y are lane-contiguous. Each 32-token stage:
-//  A. warp j does the per-token work of tokens [8j, 8j+8) of its lane's
-//     channel (conv from a sliding window of x, SiLU, dt, D*u, SiLU(z)); the
-//     per-token decay operand and dt*u go to shared memory as token-pair rows,
-//     D*u and SiLU(z) stay in registers;
+// Work split (state slices). A CTA is G warps (G = 2 or 4) over 32 channels
+// (lane = channel); warp j holds states 16j/G .. 16(j+1)/G - 1 of every
+// channel, so B and C are warp-broadcast loads and x, z, y are lane-contiguous.
+// Each 32-token stage:
+//  A. warp j does the per-token work of tokens [32j/G, 32(j+1)/G) of its
+//     lane's channel (conv from a sliding window of x, SiLU, dt, D*u,
+//     SiLU(z)); the per-token decay operand and dt*u go to shared memory as
+//     token-pair rows, D*u and SiLU(z) stay in registers;
 //  B. every warp streams its state slice through all 32 tokens (packed f32x2
 //     multiplies and FMAs) and keeps the partial readouts C.h in registers;
-//  C. warp j sums the 4 partials of its phase-A tokens, applies the skip and
+//  C. warp j sums the G partials of its phase-A tokens, applies the skip and
 //     the gate, and fills an output tile that leaves by TMA store.
 // Phase A of stage s+1 runs inside phase B of stage s (software pipelining),
 // so every warp has two independent instruction streams.
@@ -41,9 +42,11 @@
 // other channel keeps the generic path. The power path changes each decay
 // exponent by at most that 2^-20 relative, far inside the fp32 parity bar.
 //
-// Kernels. 3: this kernel with the register budget of three CTAs per SM;
-// 4 (default when the grid needs at most two CTAs per SM): the same code built
-// for two CTAs per SM, whose larger register budget buys a deeper schedule.
+// Kernels. 3: G = 4 with the register budget of three CTAs per SM; 4: G = 4
+// built for two CTAs per SM, whose larger register budget buys a deeper
+// schedule; 5: G = 2 (8 states per thread: half the per-slice overhead of a
+// token -- the decay operand load, the power arithmetic, the partial readout
+// -- and 8 independent state chains per thread, at half the warps).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -55,10 +58,9 @@
 namespace ssm {
 namespace {
 
-constexpr int kTok = 32;        // tokens per pipeline stage (= lanes of the dt_raw stager)
-constexpr int kG = 4;           // warps per CTA = state slices
-constexpr int kK = 16 / kG;     // states per thread
-constexpr int kTA = kTok / kG;  // phase-A and phase-C tokens per warp and stage
+constexpr int kTok = 32;  // tokens per pipeline stage (= lanes of the dt_raw stager)
+// G warps per CTA = state slices; each thread holds 16 / G states of its lane's
+// channel and does the per-token work of kTok / G tokens per stage.
 #ifndef SSM_PIPE_STAGES
 #define SSM_PIPE_STAGES 3
 #endif
@@ -74,7 +76,7 @@ struct Maps {
 constexpr int align128(int v) { return (v + 127) / 128 * 128; }
 
 // Shared-memory layout (byte offsets from a 128-aligned base).
-template <typename T>
+template <typename T, int G>
 struct PipeSmem {
   static constexpr int kEs = static_cast<int>(sizeof(T));
   static constexpr int kXBytes = (kTok + 3) * 32 * kEs;  // TMA box {32, kTok + 3}
@@ -89,7 +91,7 @@ struct PipeSmem {
   static constexpr int kPR = kTok + 4;                        // partial row (padded)
   static constexpr int kDr = kDT + 2 * kTok * 32 * 8;         // dt_raw float [2][token]
   static constexpr int kP = kDr + 2 * kTok * 4;               // float [slice][channel][kPR]
-  static constexpr int kY = align128(kP + kG * 32 * kPR * 4);  // output tiles [2][token][channel]
+  static constexpr int kY = align128(kP + G * 32 * kPR * 4);  // output tiles [2][token][channel]
   static constexpr int kYBytes = align128(kTok * 32 * kEs);
   static constexpr int kBar = kY + 2 * kYBytes;
   static constexpr int kTotal = kBar + kPipeStages * 8;
@@ -97,54 +99,81 @@ struct PipeSmem {
   static_assert((32 * kEs) % 16 == 0, "TMA rows must be whole 16-byte chunks");
 };
 
-// Generic decays: advance the thread's 4 states (2 packed pairs) through one
-// token; returns C.h over them. dt2 = {dt, dt}, inj2 = {dt*u, dt*u}.
+// Generic decays: advance the thread's 2 KP states (KP packed pairs) through
+// one token; returns C.h over them. dt2 = {dt, dt}, inj2 = {dt*u, dt*u}.
+template <int KP>
 __device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const float* a2, float* h, const float* Bp,
                                             const float* Cp) {
-  const float4 bq = *reinterpret_cast<const float4*>(Bp);
-  const float4 cq = *reinterpret_cast<const float4*>(Cp);
-  float x0, x1, x2, x3;
-  upk2(fmul2(dt2, pk2(a2[0], a2[1])), x0, x1);
-  upk2(fmul2(dt2, pk2(a2[2], a2[3])), x2, x3);
-  const uint64_t hb0 = ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(h[0], h[1]), fmul2(inj2, pk2(bq.x, bq.y)));
-  const uint64_t hb1 = ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(h[2], h[3]), fmul2(inj2, pk2(bq.z, bq.w)));
-  upk2(hb0, h[0], h[1]);
-  upk2(hb1, h[2], h[3]);
+  uint64_t acc = 0;
+#pragma unroll
+  for (int q = 0; q < KP; q += 2) {
+    const float4 bq = *reinterpret_cast<const float4*>(Bp + 2 * q);
+    const float4 cq = *reinterpret_cast<const float4*>(Cp + 2 * q);
+    float x0, x1, x2, x3;
+    upk2(fmul2(dt2, pk2(a2[2 * q], a2[2 * q + 1])), x0, x1);
+    upk2(fmul2(dt2, pk2(a2[2 * q + 2], a2[2 * q + 3])), x2, x3);
+    const uint64_t hb0 =
+        ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(h[2 * q], h[2 * q + 1]), fmul2(inj2, pk2(bq.x, bq.y)));
+    const uint64_t hb1 =
+        ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(h[2 * q + 2], h[2 * q + 3]), fmul2(inj2, pk2(bq.z, bq.w)));
+    upk2(hb0, h[2 * q], h[2 * q + 1]);
+    upk2(hb1, h[2 * q + 2], h[2 * q + 3]);
+    acc = q == 0 ? fmul2(pk2(cq.x, cq.y), hb0) : ffma2(pk2(cq.x, cq.y), hb0, acc);
+    acc = ffma2(pk2(cq.z, cq.w), hb1, acc);
+  }
   float lo, hi;
-  upk2(ffma2(pk2(cq.z, cq.w), hb1, fmul2(pk2(cq.x, cq.y), hb0)), lo, hi);
+  upk2(acc, lo, hi);
   return lo + hi;
 }
 
-// Power decays: states 4j..4j+3 decay by q^(4j+1) .. q^(4j+4) =
-// base * (q, q^2, q^3, q^4) with base = q^(4j) = (q^4)^(j&1) (q^8)^(j>>1).
-// hi1 = j & 1, hi2 = j & 2 (warp-uniform). inj2 = {dt*u, dt*u}.
+// Power decays: the thread's K states K j .. K j + K - 1 decay by
+// q^(K j + 1) .. q^(K j + K) = base * (q, q^2, ..., q^K) with base = q^(K j).
+// hi1 / hi2 (warp-uniform): bits of j; base = (q^K)^(j&1) (q^2K)^(j>>1 & 1).
+// inj2 = {dt*u, dt*u}.
+template <int K>
 __device__ __forceinline__ float scan_token_pow(float q, uint64_t inj2, bool hi1, bool hi2, float* h, const float* Bp,
                                                 const float* Cp) {
-  const float4 bq = *reinterpret_cast<const float4*>(Bp);
-  const float4 cq = *reinterpret_cast<const float4*>(Cp);
+  static_assert(K == 4 || K == 8, "power decays are built for 4 or 8 states per thread");
+  uint64_t p[K / 2];  // (q, q^2), (q^3, q^4), ...
   const float q2 = q * q;
-  const uint64_t p12 = pk2(q, q2);
-  const uint64_t p34 = fmul2(p12, pk2(q2, q2));  // (q^3, q^4)
-  float q3, q4;
-  upk2(p34, q3, q4);
-  float base = hi1 ? q4 : 1.0f;
-  if (hi2) base *= q4 * q4;
+  p[0] = pk2(q, q2);
+  p[1] = fmul2(p[0], pk2(q2, q2));
+  float q3, qk;
+  upk2(p[1], q3, qk);  // qk = q^4
+  if constexpr (K == 8) {
+    const uint64_t q44 = pk2(qk, qk);
+    p[2] = fmul2(p[0], q44);
+    p[3] = fmul2(p[1], q44);
+    float q7;
+    upk2(p[3], q7, qk);  // qk = q^8
+  }
+  float base = hi1 ? qk : 1.0f;
+  if (hi2) base *= qk * qk;
   const uint64_t bb = pk2(base, base);
-  const uint64_t hb0 = ffma2(fmul2(bb, p12), pk2(h[0], h[1]), fmul2(inj2, pk2(bq.x, bq.y)));
-  const uint64_t hb1 = ffma2(fmul2(bb, p34), pk2(h[2], h[3]), fmul2(inj2, pk2(bq.z, bq.w)));
-  upk2(hb0, h[0], h[1]);
-  upk2(hb1, h[2], h[3]);
+  uint64_t acc = 0;
+#pragma unroll
+  for (int i = 0; i < K / 2; i += 2) {
+    const float4 bq = *reinterpret_cast<const float4*>(Bp + 2 * i);
+    const float4 cq = *reinterpret_cast<const float4*>(Cp + 2 * i);
+    const uint64_t hb0 = ffma2(fmul2(bb, p[i]), pk2(h[2 * i], h[2 * i + 1]), fmul2(inj2, pk2(bq.x, bq.y)));
+    const uint64_t hb1 = ffma2(fmul2(bb, p[i + 1]), pk2(h[2 * i + 2], h[2 * i + 3]), fmul2(inj2, pk2(bq.z, bq.w)));
+    upk2(hb0, h[2 * i], h[2 * i + 1]);
+    upk2(hb1, h[2 * i + 2], h[2 * i + 3]);
+    acc = i == 0 ? fmul2(pk2(cq.x, cq.y), hb0) : ffma2(pk2(cq.x, cq.y), hb0, acc);
+    acc = ffma2(pk2(cq.z, cq.w), hb1, acc);
+  }
   float lo, hi;
-  upk2(ffma2(pk2(cq.z, cq.w), hb1, fmul2(pk2(cq.x, cq.y), hb0)), lo, hi);
+  upk2(acc, lo, hi);
   return lo + hi;
 }
 
 // Zero-order-hold decays (scalar): h = e^{dt A} h + (e^{dt A} - 1)/A * u * B.
+template <int K>
 __device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* Av, float* h, const float* Bp,
                                                 const float* Cp) {
   float acc = 0.0f;
 #pragma unroll
-  for (int q = 0; q < kK; ++q) {
+  for (int q = 0; q < K; ++q) {
     const float xa = dt * Av[q];
     const float dA = ex2_approx(xa * kLog2e);
     h[q] = fmaf(dA, h[q], expm1_nonpos(xa, dA) / Av[q] * u * Bp[q]);
@@ -162,7 +191,7 @@ enum class Path { kGeneric, kPow, kZoh };
 // registers. Dr is the stage's dt_raw row. The caller stores the pairs
 // (store_rows) after the scan, so no shared-memory store sits between the
 // scan's loads in program order.
-template <typename T, Path P>
+template <typename T, Path P, int kTA>
 __device__ __forceinline__ void phase_a(const T* __restrict__ X, const T* __restrict__ Z, const float* __restrict__ Dr,
                                         int64_t t0, int64_t L, int tb, int lane, bool first, float hx0, float hx1,
                                         float hx2, float cw0, float cw1, float cw2, float cw3, float cb, float wdt,
@@ -201,6 +230,7 @@ __device__ __forceinline__ void phase_a(const T* __restrict__ X, const T* __rest
 
 // Rows as [token pair][channel] (d, inj, d', inj'): one 16-byte load per two
 // tokens in phase B.
+template <int kTA>
 __device__ __forceinline__ void store_rows(float2* DTo, int tb, int lane, const float4* rows) {
   float4* DT4 = reinterpret_cast<float4*>(DTo);
 #pragma unroll
@@ -209,7 +239,7 @@ __device__ __forceinline__ void store_rows(float2* DTo, int tb, int lane, const 
 
 // Phase B over tokens [T0, T1) of one stage: this thread's 4 states; pr gets
 // the partial readouts.
-template <Path P, int T0 = 0, int T1 = kTok>
+template <Path P, int K, int T0 = 0, int T1 = kTok>
 __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int lane, const float* Av, const float* a2,
                                            bool hi1, bool hi2, float* h, const float* __restrict__ Bs,
                                            const float* __restrict__ Cs, float* pr) {
@@ -218,19 +248,21 @@ __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int l
     const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
     const float2 dd = (tl & 1) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
     if constexpr (P == Path::kZoh)
-      pr[tl] = scan_token_zoh(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
+      pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
     else if constexpr (P == Path::kPow)
-      pr[tl] = scan_token_pow(dd.x, pk2(dd.y, dd.y), hi1, hi2, h, Bs + tl * 16, Cs + tl * 16);
+      pr[tl] = scan_token_pow<K>(dd.x, pk2(dd.y, dd.y), hi1, hi2, h, Bs + tl * 16, Cs + tl * 16);
     else
-      pr[tl] = scan_token(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
+      pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
   }
 }
 
-// The whole walk over L for one CTA, on the decay path P.
-template <typename T, Path P>
+// The whole walk over L for one CTA of G warps, on the decay path P.
+template <typename T, int G, Path P>
 __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) {
-  constexpr int NT = 32 * kG;
-  using S = PipeSmem<T>;
+  constexpr int NT = 32 * G;
+  constexpr int kK = 16 / G;     // states per thread
+  constexpr int kTA = kTok / G;  // phase-A and phase-C tokens per warp and stage
+  using S = PipeSmem<T, G>;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
@@ -306,7 +338,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + warp * kK + q] : 0.0f;
   }
   const float a20 = -expf(a.A_log[ec * 16]) * kLog2e;  // A_0 log2(e): q = 2^(dt a20) on the power path
-  const bool hi1 = (warp & 1) != 0, hi2 = (warp & 2) != 0;
+  const bool hi1 = (warp & 1) != 0, hi2 = (warp & 2) != 0;  // bits of the slice index (power path)
   const int tb = warp * kTA;
 
   // Prologue: phase A of stage 0.
@@ -314,9 +346,9 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
   {
     float4 rows0[kTA / 2];
     mbar_wait_bounded(full0, 0u, a.err, 1);
-    phase_a<T, P>(reinterpret_cast<const T*>(smem + S::kX), reinterpret_cast<const T*>(smem + S::kZ), Dr, 0, L, tb,
-                  lane, true, hx0, hx1, hx2, cw0, cw1, cw2, cw3, cb, wdt, dtb, Dd, lo, hi, a20, rows0, du, zg);
-    store_rows(DT, tb, lane, rows0);
+    phase_a<T, P, kTA>(reinterpret_cast<const T*>(smem + S::kX), reinterpret_cast<const T*>(smem + S::kZ), Dr, 0, L,
+                       tb, lane, true, hx0, hx1, hx2, cw0, cw1, cw2, cw3, cb, wdt, dtb, Dd, lo, hi, a20, rows0, du, zg);
+    store_rows<kTA>(DT, tb, lane, rows0);
   }
   named_bar_sync(1, NT);
 
@@ -342,14 +374,14 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
       // Source order: first half of the scan, the next stage's per-token work,
       // second half of the scan (measured 2% faster than either block first).
       float4 rows[kTA / 2];
-      scan_stage<P, 0, kTok / 2>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
-      phase_a<T, P>(reinterpret_cast<const T*>(nst + S::kX), reinterpret_cast<const T*>(nst + S::kZ),
-                    Dr + ((s + 1) & 1) * kTok, t0 + kTok, L, tb, lane, false, hx0, hx1, hx2, cw0, cw1, cw2, cw3, cb,
-                    wdt, dtb, Dd, lo, hi, a20, rows, duN, zgN);
-      scan_stage<P, kTok / 2, kTok>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
-      store_rows(DTn, tb, lane, rows);
+      scan_stage<P, kK, 0, kTok / 2>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      phase_a<T, P, kTA>(reinterpret_cast<const T*>(nst + S::kX), reinterpret_cast<const T*>(nst + S::kZ),
+                         Dr + ((s + 1) & 1) * kTok, t0 + kTok, L, tb, lane, false, hx0, hx1, hx2, cw0, cw1, cw2, cw3,
+                         cb, wdt, dtb, Dd, lo, hi, a20, rows, duN, zgN);
+      scan_stage<P, kK, kTok / 2, kTok>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      store_rows<kTA>(DTn, tb, lane, rows);
     } else {
-      scan_stage<P>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      scan_stage<P, kK>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
     }
     {
       float* Pj = P_ + (warp * 32 + lane) * S::kPR;
@@ -367,7 +399,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
       for (int q = 0; q < kTA; q += 4) {
         float4 acc = *reinterpret_cast<const float4*>(P_ + lane * S::kPR + tb + q);
 #pragma unroll
-        for (int jj = 1; jj < kG; ++jj) {
+        for (int jj = 1; jj < G; ++jj) {
           const float4 v = *reinterpret_cast<const float4*>(P_ + (jj * 32 + lane) * S::kPR + tb + q);
           acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
         }
@@ -423,22 +455,28 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
 }
 
 // True when every channel of this CTA has A_n = (n+1) A_0 to within kPowTol
-// (on the fp32 A = -expf(A_log) the kernel uses). Called by all threads.
+// (on the fp32 A = -expf(A_log) the kernel uses). Called by all G warps; warp
+// j checks states 16j/G .. 16(j+1)/G - 1 of its lane's channel.
+template <int G>
 __device__ __forceinline__ bool cta_has_power_decays(const KernelArgs& a) {
   const int64_t tiles = (a.E + 31) / 32;
   const int64_t e = (blockIdx.x % tiles) * 32 + (threadIdx.x & 31);
   const int64_t ec = e < a.E ? e : a.E - 1;
   const float4* row = reinterpret_cast<const float4*>(a.A_log + ec * 16);  // 16-byte aligned rows
   const float A0 = -expf(a.A_log[ec * 16]);
+  const int j = static_cast<int>(threadIdx.x >> 5);
   bool ok = true;
-  // Each warp checks a quarter of the states; the CTA vote combines them.
-  const float4 v = row[threadIdx.x >> 5];
-  const float al[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int n = 4 * static_cast<int>(threadIdx.x >> 5) + i;
-    const float An = -expf(al[i]);
-    ok = ok && fabsf(An - static_cast<float>(n + 1) * A0) <= kPowTol * fabsf(An);
+  for (int v4 = 0; v4 < 4 / G; ++v4) {
+    const int q4 = j * (4 / G) + v4;
+    const float4 v = row[q4];
+    const float al[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int n = 4 * q4 + i;
+      const float An = -expf(al[i]);
+      ok = ok && fabsf(An - static_cast<float>(n + 1) * A0) <= kPowTol * fabsf(An);
+    }
   }
   return __syncthreads_and(ok) != 0;
 }
@@ -447,17 +485,17 @@ __device__ __forceinline__ bool cta_has_power_decays(const KernelArgs& a) {
 // SM); MINB 1 lets it use up to 255 registers a thread (2 CTAs fit), which it
 // spends on a deeper schedule of the fused block: measured 7% faster when the
 // grid needs at most two CTAs per SM, slower when it needs more.
-template <typename T, bool ZOH, int MINB>
-__global__ void __launch_bounds__(32 * kG, MINB) prefill_pipe_kernel(const __grid_constant__ Maps maps,
-                                                                      const KernelArgs a) {
+template <typename T, int G, bool ZOH, int MINB>
+__global__ void __launch_bounds__(32 * G, MINB) prefill_pipe_kernel(const __grid_constant__ Maps maps,
+                                                                     const KernelArgs a) {
   if constexpr (ZOH) {
-    pipe_run<T, Path::kZoh>(maps, a);
+    pipe_run<T, G, Path::kZoh>(maps, a);
   } else {
-    const bool pw = a.decay_path == 0 && cta_has_power_decays(a);
+    const bool pw = a.decay_path == 0 && cta_has_power_decays<G>(a);
     if (pw)
-      pipe_run<T, Path::kPow>(maps, a);
+      pipe_run<T, G, Path::kPow>(maps, a);
     else
-      pipe_run<T, Path::kGeneric>(maps, a);
+      pipe_run<T, G, Path::kGeneric>(maps, a);
   }
 }
 
@@ -514,31 +552,32 @@ bool make_maps(const KernelArgs& a, Maps* m) {
          map3(&m->C, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.C, 16, L, b, a.s.bc_tok * 4, a.s.bc_seq * 4, 16, kTok);
 }
 
-template <typename T, bool ZOH, int MINB>
+template <typename T, int G, bool ZOH, int MINB>
 cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st) {
-  using S = PipeSmem<T>;
+  using S = PipeSmem<T, G>;
   Maps maps;
   if (!make_maps<T>(a, &maps)) return cudaErrorInvalidValue;
-  auto kern = prefill_pipe_kernel<T, ZOH, MINB>;
+  auto kern = prefill_pipe_kernel<T, G, ZOH, MINB>;
   const int smem = S::kTotal + 128;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   const int64_t grid = a.batch * ((a.E + 31) / 32);
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), 32 * kG, smem, st>>>(maps, a);
+  kern<<<static_cast<unsigned>(grid), 32 * G, smem, st>>>(maps, a);
   return cudaGetLastError();
 }
 
 template <typename T, bool ZOH>
 cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st) {
-  if (sh.kernel == 3) return launch_pipe<T, ZOH, 0>(a, st);
-  if (sh.kernel == 4) return launch_pipe<T, ZOH, 1>(a, st);
+  if (sh.kernel == 3) return launch_pipe<T, 4, ZOH, 0>(a, st);
+  if (sh.kernel == 4) return launch_pipe<T, 4, ZOH, 1>(a, st);
+  if (sh.kernel == 5) return launch_pipe<T, 2, ZOH, 1>(a, st);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool prefill_shape_supported(PrefillShape sh) { return sh.kernel == 3 || sh.kernel == 4; }
+bool prefill_shape_supported(PrefillShape sh) { return sh.kernel >= 3 && sh.kernel <= 5; }
 
 // Pipelined state slices; the register-rich build when the grid needs at most
 // two CTAs per SM.

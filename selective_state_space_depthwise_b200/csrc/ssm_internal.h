@@ -52,6 +52,13 @@ bool prefill_shape_supported(PrefillShape sh);
 cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st);
 cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStream_t st);
 
+// C[M][N] = A[M][K] . B[N][K]^T, bf16 operands and output, fp32 accumulation,
+// on the tensor cores (gemm.cu). bn: output tile width 256 or 128, 0 = chosen
+// from the shape. K and N multiples of 8, pointers 16-byte aligned.
+cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int bn, int num_sms,
+                         int* err, cudaStream_t st);
+int gemm_choose_bn(int64_t M, int64_t N, int num_sms);
+
 // Shared by the entry points (ssm_api.cu): validation with the ABI's
 // "0 = dense" stride defaults, and the calling thread's last-error message.
 ssm_status check_dims(const ssm_dims* d, bool prefill, Strides* s);

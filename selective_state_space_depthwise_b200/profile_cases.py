@@ -5,6 +5,7 @@
     python -m selective_state_space_depthwise_b200.profile_cases block NAME [L]
     python -m selective_state_space_depthwise_b200.profile_cases ssd NAME
     python -m selective_state_space_depthwise_b200.profile_cases segment WORKLOAD [T]
+    python -m selective_state_space_depthwise_b200.profile_cases gemm M N K
 
 prefill: three launches of the named workload's prefill (optionally shortened
 to L tokens, optionally with an explicit kernel (3 or 4) and decay path (0 auto,
@@ -13,7 +14,7 @@ prompt, then three decode steps at the decode workload's shape (batch 256,
 E=7680, 252 MB of state); block: three block forwards of the named block
 workload (optionally L tokens); segment: three segment summaries of the first
 T tokens (default L / 8) of the named workload, then three carries of 7 such
-summaries. Inputs are drawn on the GPU; a capture skips the
+summaries; gemm: three projection GEMMs C[M][N] = A[M][K] . W[N][K]^T (bf16). Inputs are drawn on the GPU; a capture skips the
 first two launches of the kernel it selects (ncu -s 2 -c 1 -k regex:...).
 """
 from __future__ import annotations
@@ -92,6 +93,16 @@ def segment_case(name: str, T: int = 0):
     print("segment ok", name, T, float(summ.abs().mean()), float(h.abs().mean()))
 
 
+def gemm_case(M: int, N: int, K: int):
+    g = torch.Generator(device="cuda").manual_seed(0)
+    A = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+    Wt = (torch.randn((N, K), device="cuda", generator=g) * K ** -0.5).to(torch.bfloat16)
+    for _ in range(3):
+        C = api.proj_gemm(A, Wt)
+    torch.cuda.synchronize()
+    print("gemm ok", M, N, K, float(C.float().abs().mean()))
+
+
 if __name__ == "__main__":
     if sys.argv[1] == "prefill":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
@@ -104,6 +115,8 @@ if __name__ == "__main__":
         block_case(sys.argv[2], int(sys.argv[3]) if len(sys.argv) > 3 else 0)
     elif sys.argv[1] == "segment":
         segment_case(sys.argv[2], int(sys.argv[3]) if len(sys.argv) > 3 else 0)
+    elif sys.argv[1] == "gemm":
+        gemm_case(int(sys.argv[2]), int(sys.argv[3]), int(sys.argv[4]))
     elif sys.argv[1] == "decode":
         decode_case(int(sys.argv[2]) if len(sys.argv) > 2 else 256)
     else:

@@ -1,0 +1,113 @@
+"""GPU tests of the block's projection GEMM (ssm_proj_gemm: C = A . W^T on
+tcgen05, bf16 operands, fp32 accumulation, bf16 output), the in_proj and
+out_proj of "Axon-SSM: selective state space model", "Algorithm" diagram.
+
+Reference: the products of the stored bf16 values summed in float64 on the
+CPU, rounded once to bf16. The kernel accumulates the same products in fp32
+(K <= 7680 terms: relative error ~1e-6, far below a bf16 step), so the two
+roundings agree except for rare one-step flips: relative L2 <= 1e-3 is asked.
+Shapes cover ragged M, N and K tails, both output tile widths (the launch
+picks 128 or 256 columns from the shape) and the block's layer shapes.
+"""
+import numpy as np
+import pytest
+import torch
+
+from selective_state_space_depthwise_b200 import _lib, api
+
+pytestmark = pytest.mark.gpu
+
+TOL_GEMM = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+def operands(M, N, K, seed):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    A = torch.randn((M, K), generator=g).to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g) * K ** -0.5).to(torch.bfloat16)
+    return A, W
+
+
+def reference(A, W, rows=None):
+    a = A.double().numpy() if rows is None else A[rows].double().numpy()
+    return torch.from_numpy(a @ W.double().numpy().T).to(torch.bfloat16).double().numpy()
+
+
+def rel_l2(got, want):
+    return float(np.linalg.norm(got - want) / np.linalg.norm(want))
+
+
+def bn_of(M, N):
+    """The tile width the launch picks (mirrors gemm_choose_bn): fewer
+    waves x width wins, ties go to 256."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tm = -(-M // 128)
+    w256 = -(-(tm * -(-N // 256)) // sms)
+    w128 = -(-(tm * -(-N // 128)) // sms)
+    return 128 if w128 * 128 < w256 * 256 else 256
+
+
+SHAPES = [(1, 8, 8), (100, 136, 72), (300, 520, 200), (129, 264, 64), (257, 1000, 1032)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"{m}x{n}x{k}" for m, n, k in SHAPES])
+def test_gemm_ragged_shapes(shape):
+    M, N, K = shape
+    A, W = operands(M, N, K, seed=M + N + K)
+    C = api.proj_gemm(A.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    e = rel_l2(C.double().cpu().numpy(), reference(A, W))
+    print(f"gemm {M}x{N}x{K} (tile width {bn_of(M, N)}): rel-L2 {e:.2e}")
+    assert e <= TOL_GEMM
+
+
+def test_gemm_both_tile_widths():
+    """One shape the launch tiles 256 columns wide and one it tiles 128 wide,
+    each with more tiles than SMs (several tiles per persistent CTA, both TMEM
+    accumulators in turn)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    # 4 row tiles x sms/4 column tiles of 256 fill the SMs once (256 wide);
+    # 5 row tiles x 4 column tiles of 128 (N = 408) tile 128 wide.
+    cases = [(512, 256 * (sms // 4), 192), (640, 408, 256)]
+    widths = set()
+    for M, N, K in cases:
+        widths.add(bn_of(M, N))
+        A, W = operands(M, N, K, seed=N)
+        C = api.proj_gemm(A.cuda(), W.cuda())
+        torch.cuda.synchronize()
+        e = rel_l2(C.double().cpu().numpy(), reference(A, W))
+        print(f"gemm {M}x{N}x{K} (tile width {bn_of(M, N)}): rel-L2 {e:.2e}")
+        assert e <= TOL_GEMM
+    assert widths == {128, 256}
+
+
+@pytest.mark.parametrize("which", ["in_proj", "out_proj"])
+def test_gemm_layer_shapes_sampled_rows(which):
+    """The block's projections at the Axon layer shape (2048 tokens, D = 2560,
+    E = 7680): every column of 96 sampled rows against the float64 reference,
+    and the full output finite."""
+    M, D, E = 2048, 2560, 7680
+    N, K = (2 * E, D) if which == "in_proj" else (D, E)
+    A, W = operands(M, N, K, seed=7 if which == "in_proj" else 8)
+    C = api.proj_gemm(A.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    assert torch.isfinite(C).all()
+    rows = np.sort(np.random.default_rng(3).choice(M, 96, replace=False))
+    rows[0], rows[-1] = 0, M - 1
+    e = rel_l2(C[torch.from_numpy(rows).cuda()].double().cpu().numpy(), reference(A, W, rows))
+    print(f"{which} {M}x{N}x{K}: rel-L2 {e:.2e} over {len(rows)} rows")
+    assert e <= TOL_GEMM
+
+
+def test_gemm_rejects_bad_arguments():
+    A = torch.zeros((16, 12), dtype=torch.bfloat16, device="cuda")  # K = 12 is not a multiple of 8
+    W = torch.zeros((8, 12), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(_lib.SsmError) as err:
+        api.proj_gemm(A, W)
+    assert err.value.status == _lib.SSM_ERR_INVALID_ARG
