@@ -357,7 +357,8 @@ ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64
  *
  * Range. Each decay exp(dA[l] - dA[s]) is formed as the product of
  * exp(dA[l] - dA[s1]) and exp(dA[s1] - dA[s]), s1 the last position of s's
- * 8-position group (the group that holds l: one exponential per element).
+ * 8-position group (in the group that holds l, when dA falls by more than 80
+ * across that group: one exponential per element).
  * When dA_cumsum does not increase along a chunk (dt >= 0 and A <= 0, what a
  * cumulative sum of dt A gives), every exponent is <= 0: no factor exceeds 1
  * however strong the decay, a decayed term that underflows fp32 is 0, and

@@ -3,9 +3,13 @@
 // model", "Algorithm" diagram, as C[M][N] = A[M][K] . B[N][K]^T with A and B
 // bf16 row-major (both K-major), fp32 accumulation and a bf16 C.
 //
-// One persistent CTA per SM walks output tiles of 128 x BN (BN = 256 or 128)
-// in a static round-robin order (tile index m-fastest, so the CTAs running at
-// the same time share B tiles in L2). Six warps with fixed roles:
+// One persistent CTA per SM walks output tiles of 128 x BN (BN = 256 or 160)
+// in a static round-robin order over a grouped raster: tiles run in groups of
+// up to 16 row blocks x every column block, row block fastest inside a group,
+// so the CTAs running at the same time share both their A row blocks and their
+// B column blocks in L2 (with a plain row-fastest order a wave of 148 tiles
+// spans 148 row blocks of one column block, and at M = 65536 every A block
+// would be read from HBM once per column block). Six warps with fixed roles:
 //   warp 0     TMA producer: the A tile [128][64] and the B tile [BN][64] of
 //              each 64-wide K chunk, 128-byte swizzled, into a STAGES-deep ring
 //              (full / empty mbarriers per slot);
@@ -16,10 +20,9 @@
 //              the 512 TMEM columns) alternate, so the next tile's MMAs run
 //              while the epilogue drains the previous one;
 //   warps 2-5  epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (its
-//              quarter of the tile's rows) 64 columns at a time, rounds to
-//              bf16, writes a 128-byte swizzled [32][64] staging tile (two per
-//              warp, alternating) and stores it with a TMA tile store, then
-//              frees the accumulator.
+//              quarter of the tile's rows) 32 columns at a time, rounds to
+//              bf16, writes a [32][32] staging tile (two per warp, alternating)
+//              and stores it with a TMA tile store, then frees the accumulator.
 // Tails: TMA loads past M, N or K read zeros; stores are clipped at M and N.
 // Every mbarrier wait is bounded; a wait that gives up sets the device error
 // word and a CTA abort flag, every role leaves its loop, the producer waits
@@ -52,20 +55,33 @@ struct GemmSmem {
   static constexpr int kABytes = kGBM * 128;
   static constexpr int kBBytes = BN * 128;
   static constexpr int kStage = kABytes + kBBytes;
-  static constexpr int kOut = STAGES * kStage;  // epilogue staging: 4 warps x 2 tiles of [32][64] bf16
-  static constexpr int kOutBytes = 32 * 128;
+  static constexpr int kOut = STAGES * kStage;  // epilogue staging: 4 warps x 2 tiles of [32][32] bf16
+  static constexpr int kOutBytes = 32 * 64;
   static constexpr int kBar = kOut + 8 * kOutBytes;  // full[S], empty[S], tfull[2], tempty[2]
   static constexpr int kTmemSlot = kBar + (2 * STAGES + 4) * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kIssued = kTmemSlot + 8;  // int64: K chunks the producer issued
   static constexpr int kTotal = kIssued + 8;
-  static_assert(kStage % 1024 == 0 && kOutBytes % 1024 == 0, "swizzled tiles need 1 KB alignment");
+  // TMEM columns: two accumulators of BN, allocated as a power of two.
+  static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256u : 512u;
+  static_assert(kStage % 1024 == 0, "swizzled operand tiles need 1 KB alignment");
 };
 
 struct GemmArgs {
   int tiles_m, tiles_n, k_chunks;
+  int group_m;  // row blocks per raster group
   int* err;
 };
+
+// Tile index -> (row block, column block) of the grouped raster.
+__device__ __forceinline__ void tile_coords(const GemmArgs& g, int tile, int& mb, int& nb) {
+  const int per_group = g.group_m * g.tiles_n;
+  const int grp = tile / per_group, r = tile - grp * per_group;
+  const int m_base = grp * g.group_m;
+  const int gm = min(g.group_m, g.tiles_m - m_base);  // the last group may be shorter
+  mb = m_base + r % gm;
+  nb = r / gm;
+}
 
 // bf16 x bf16 -> fp32, M = 128, N = BN, A and B K-major.
 template <int BN>
@@ -109,7 +125,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     prefetch_tensormap(&map_c);
   }
   if (warp == 1) {
-    tmem_alloc(sb + S::kTmemSlot, 2 * BN);
+    tmem_alloc(sb + S::kTmemSlot, S::kTmemCols);
     tmem_relinquish();
   }
   tcgen05_fence_before();
@@ -122,7 +138,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     if (lane == 0) {
       int64_t it = 0;
       for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
-        const int m0 = (tile % g.tiles_m) * kGBM, n0 = (tile / g.tiles_m) * BN;
+        int mb, nb;
+        tile_coords(g, tile, mb, nb);
+        const int m0 = mb * kGBM, n0 = nb * BN;
         for (int kc = 0; kc < g.k_chunks; ++kc, ++it) {
           const int s = static_cast<int>(it % STAGES);
           const uint32_t round = static_cast<uint32_t>(it / STAGES);
@@ -189,7 +207,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // instruction that all 32 lanes must reach together.
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
-      const int m0 = (tile % g.tiles_m) * kGBM, n0 = (tile / g.tiles_m) * BN;
+      int mb, nb;
+      tile_coords(g, tile, mb, nb);
+      const int m0 = mb * kGBM, n0 = nb * BN;
       const int buf = i & 1;
       const bool ok = mbar_wait_bounded(tfull(buf), static_cast<uint32_t>(i >> 1) & 1u, g.err, 24);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -199,30 +219,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
       tcgen05_fence_after();
       const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t r0[32], r1[32];
-        tmem_ld_x32(t_row + 64 * c, r0);
-        tmem_ld_x32(t_row + 64 * c + 32, r1);
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_x32(t_row + 32 * c, r);
         tmem_ld_wait();
-        uint32_t w[32];
+        uint32_t w[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 v0 = __floats2bfloat162_rn(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
-          const __nv_bfloat162 v1 = __floats2bfloat162_rn(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
-          w[j] = *reinterpret_cast<const uint32_t*>(&v0);
-          w[16 + j] = *reinterpret_cast<const uint32_t*>(&v1);
+          const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+          w[j] = *reinterpret_cast<const uint32_t*>(&v);
         }
         if (lane == 0) bulk_wait_read<1>();  // the store that last read staging tile `ob` is done with it
         __syncwarp();
         unsigned char* st = stage0_ptr + ob * S::kOutBytes;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)  // row `lane`, 16-byte chunk j, 128-byte swizzle
-          *reinterpret_cast<uint4*>(st + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-              make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+        for (int j = 0; j < 4; ++j)  // row `lane`: 64 bytes
+          *reinterpret_cast<uint4*>(st + lane * 64 + 16 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(&map_c, stage0 + static_cast<uint32_t>(ob * S::kOutBytes), n0 + 64 * c, m0 + 32 * q);
+          tma_store_2d(&map_c, stage0 + static_cast<uint32_t>(ob * S::kOutBytes), n0 + 32 * c, m0 + 32 * q);
           bulk_commit();
         }
         ob ^= 1;
@@ -248,15 +264,15 @@ __global__ void __launch_bounds__(kGThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tcgen05_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc(tmem, S::kTmemCols);
   }
 }
 
 bool bf16_map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-               uint32_t box_outer) {
+               uint32_t box_outer, CUtensorMapSwizzle swz) {
   const uint64_t dims[2] = {inner, outer}, strides[1] = {inner * 2};
   const uint32_t box[2] = {box_inner, box_outer};
-  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, swz);
 }
 
 template <int BN, int STAGES>
@@ -264,9 +280,9 @@ cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_
                         int* err, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
   CUtensorMap ma, mb, mc;
-  if (!bf16_map2(&ma, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kGBK, kGBM) ||
-      !bf16_map2(&mb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(N), kGBK, BN) ||
-      !bf16_map2(&mc, C, static_cast<uint64_t>(N), static_cast<uint64_t>(M), 64, 32))
+  if (!bf16_map2(&ma, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kGBK, kGBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !bf16_map2(&mb, B, static_cast<uint64_t>(K), static_cast<uint64_t>(N), kGBK, BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !bf16_map2(&mc, C, static_cast<uint64_t>(N), static_cast<uint64_t>(M), 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   GemmArgs g;
   const int64_t tm = (M + kGBM - 1) / kGBM, tn = (N + BN - 1) / BN, kc = (K + kGBK - 1) / kGBK;
@@ -274,6 +290,7 @@ cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_
   g.tiles_m = static_cast<int>(tm);
   g.tiles_n = static_cast<int>(tn);
   g.k_chunks = static_cast<int>(kc);
+  g.group_m = static_cast<int>(tm < 16 ? tm : 16);
   g.err = err;
   const int smem = S::kTotal + 1024;
   auto kern = gemm_bf16_tn_kernel<BN, STAGES>;
@@ -288,12 +305,15 @@ cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_
 }  // namespace
 
 int gemm_choose_bn(int64_t M, int64_t N, int num_sms) {
-  // Per-SM waves x tile width: the smaller finishes first (ties go to 256,
-  // which reads half the operand bytes per FLOP of 128).
+  // Waves of tiles per SM x tile width, the 160-wide tile charged 10% more per
+  // column for its lower FLOP-per-byte (measured on B200: 128-wide tiles ran
+  // at half the rate of 256-wide ones, so they are not offered). 160 wins
+  // where 256-wide tiles leave most of a last wave idle (out_proj at 2048
+  // tokens: 160 tiles on 148 SMs).
   const int64_t tm = (M + kGBM - 1) / kGBM;
   const int64_t w256 = (tm * ((N + 255) / 256) + num_sms - 1) / num_sms;
-  const int64_t w128 = (tm * ((N + 127) / 128) + num_sms - 1) / num_sms;
-  return w128 * 128 < w256 * 256 ? 128 : 256;
+  const int64_t w160 = (tm * ((N + 159) / 160) + num_sms - 1) / num_sms;
+  return 11 * w160 * 160 < 10 * w256 * 256 ? 160 : 256;
 }
 
 cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int bn,
@@ -302,7 +322,7 @@ cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64
   if (num_sms <= 0) num_sms = 148;
   if (bn == 0) bn = SSM_GEMM_FORCE_BN ? SSM_GEMM_FORCE_BN : gemm_choose_bn(M, N, num_sms);
   if (bn == 256) return launch_gemm<256, 4>(A, B, C, M, N, K, num_sms, err, st);
-  if (bn == 128) return launch_gemm<128, 6>(A, B, C, M, N, K, num_sms, err, st);
+  if (bn == 160) return launch_gemm<160, 5>(A, B, C, M, N, K, num_sms, err, st);
   return cudaErrorInvalidValue;
 }
 

@@ -75,8 +75,10 @@ struct Maps {
 
 constexpr int align128(int v) { return (v + 127) / 128 * 128; }
 
-// Shared-memory layout (byte offsets from a 128-aligned base).
-template <typename T, int G>
+// Shared-memory layout (byte offsets from a 128-aligned base). SPLIT: the
+// partial readouts alternate between two buffers by stage parity (the split
+// end-of-stage barrier needs them; see pipe_run).
+template <typename T, int G, bool SPLIT>
 struct PipeSmem {
   static constexpr int kEs = static_cast<int>(sizeof(T));
   static constexpr int kXBytes = (kTok + 3) * 32 * kEs;  // TMA box {32, kTok + 3}
@@ -90,8 +92,9 @@ struct PipeSmem {
   static constexpr int kDT = kPipeStages * kSlot;             // float4 [2][token pair][channel]
   static constexpr int kPR = kTok + 4;                        // partial row (padded)
   static constexpr int kDr = kDT + 2 * kTok * 32 * 8;         // dt_raw float [2][token]
-  static constexpr int kP = kDr + 2 * kTok * 4;               // float [slice][channel][kPR]
-  static constexpr int kY = align128(kP + G * 32 * kPR * 4);  // output tiles [2][token][channel]
+  static constexpr int kPBytes = G * 32 * kPR * 4;            // float [slice][channel][kPR]
+  static constexpr int kP = kDr + 2 * kTok * 4;               // partials, double-buffered by stage parity
+  static constexpr int kY = align128(kP + (SPLIT ? 2 : 1) * kPBytes);  // output tiles [2][token][channel]
   static constexpr int kYBytes = align128(kTok * 32 * kEs);
   static constexpr int kBar = kY + 2 * kYBytes;
   static constexpr int kTotal = kBar + kPipeStages * 8;
@@ -256,13 +259,17 @@ __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int l
   }
 }
 
-// The whole walk over L for one CTA of G warps, on the decay path P.
-template <typename T, int G, Path P>
+// The whole walk over L for one CTA of G warps, on the decay path P. Two
+// barriers per stage: barrier 1 after the scan (partials, next rows and dt_raw
+// visible; ring slot s free) and barrier 2 after phase C (output tile
+// complete). SPLIT: at barrier 2 only warp 0, which stores the tile, waits;
+// the others arrive and run on, which needs the partials double-buffered.
+template <typename T, int G, Path P, bool SPLIT>
 __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) {
   constexpr int NT = 32 * G;
   constexpr int kK = 16 / G;     // states per thread
   constexpr int kTA = kTok / G;  // phase-A and phase-C tokens per warp and stage
-  using S = PipeSmem<T, G>;
+  using S = PipeSmem<T, G, SPLIT>;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
@@ -270,7 +277,6 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
   const uint32_t full0 = sb + S::kBar;
   float2* DT = reinterpret_cast<float2*>(smem + S::kDT);
   float* Dr = reinterpret_cast<float*>(smem + S::kDr);
-  float* P_ = reinterpret_cast<float*>(smem + S::kP);
 
   const int tid = threadIdx.x;
   // A warp index the compiler can prove uniform puts the B/C row addresses of
@@ -362,6 +368,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     const int64_t t0 = s * kTok;
     const bool has_next = s + 1 < n_stages;
     float duN[kTA], zgN[kTA];
+    float* P_ = reinterpret_cast<float*>(smem + S::kP + (SPLIT ? (s & 1) * S::kPBytes : 0));
     // dt_raw of stage s + 2 into the buffer that phase A of stage s (block s - 1) has finished with
     if (warp == 0) copy_dt_raw(s + 2);
 
@@ -389,8 +396,13 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
       for (int tl = 0; tl < kTok; tl += 4)
         *reinterpret_cast<float4*>(Pj + tl) = make_float4(pr[tl], pr[tl + 1], pr[tl + 2], pr[tl + 3]);
     }
-    if (tid == 0) bulk_wait_read<1>();  // output tile (s & 1) no longer read by the store of stage s - 2
-    named_bar_sync(1, NT);              // partials of stage s and rows of stage s + 1 visible
+    if (warp == 0) cp_async_wait_all();  // dt_raw of stage s + 2 lands before the barrier
+    if (tid == 0) bulk_wait_read<1>();    // output tile (s & 1) no longer read by the store of stage s - 2
+    // Partials of stage s, rows of stage s + 1 and dt_raw of stage s + 2
+    // visible; every warp is done with ring slot s (phase A of s ran in the
+    // previous block, phase B of s just now), so it is re-armed at once.
+    named_bar_sync(1, NT);
+    if (tid == 0 && s + kPipeStages < n_stages) issue_stage(s + kPipeStages);
 
     // Phase C of stage s: tokens [tb, tb + kTA).
     {
@@ -420,12 +432,20 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
         zg[i] = zgN[i];
       }
     }
-    if (warp == 0) cp_async_wait_all();  // dt_raw of stage s + 2 lands before the barrier
-    named_bar_sync(1, NT);  // output tile complete; slot of stage s and its partials free
-    if (tid == 0) {
-      tma_store_3d(&maps.y, sb + S::kY + (s & 1) * S::kYBytes, e0, static_cast<int>(t0), seq);
-      bulk_commit();
-      if (s + kPipeStages < n_stages) issue_stage(s + kPipeStages);
+    // The output tile is complete once every warp has written its tokens.
+    // SPLIT: warp 0 waits for that and stores it; the other warps only arrive
+    // and go on to the next stage (no other buffer needs this barrier: the
+    // partials alternate by stage parity, and the next writer of any buffer
+    // read in phase C passes barrier 1 of the next stage first). Otherwise
+    // every warp waits, which also frees the single partials buffer.
+    if (!SPLIT || warp == 0) {
+      named_bar_sync(2, NT);
+      if (tid == 0) {
+        tma_store_3d(&maps.y, sb + S::kY + (s & 1) * S::kYBytes, e0, static_cast<int>(t0), seq);
+        bulk_commit();
+      }
+    } else {
+      named_bar_arrive(2, NT);
     }
   }
   if (tid == 0) bulk_wait<0>();
@@ -485,17 +505,29 @@ __device__ __forceinline__ bool cta_has_power_decays(const KernelArgs& a) {
 // SM); MINB 1 lets it use up to 255 registers a thread (2 CTAs fit), which it
 // spends on a deeper schedule of the fused block: measured 7% faster when the
 // grid needs at most two CTAs per SM, slower when it needs more.
+// The split end-of-stage barrier (double-buffered partials) is used where
+// the shared memory allows: not in the three-CTAs-per-SM build. The build
+// switch turns it off everywhere (for side-by-side measurements).
+#ifndef SSM_PREFILL_SPLIT_BARRIER
+#define SSM_PREFILL_SPLIT_BARRIER 1
+#endif
+template <int MINB>
+__host__ __device__ constexpr bool split_barrier() {
+  return MINB == 1 && SSM_PREFILL_SPLIT_BARRIER;
+}
+
 template <typename T, int G, bool ZOH, int MINB>
 __global__ void __launch_bounds__(32 * G, MINB) prefill_pipe_kernel(const __grid_constant__ Maps maps,
                                                                      const KernelArgs a) {
+  constexpr bool SPLIT = split_barrier<MINB>();
   if constexpr (ZOH) {
-    pipe_run<T, G, Path::kZoh>(maps, a);
+    pipe_run<T, G, Path::kZoh, SPLIT>(maps, a);
   } else {
     const bool pw = a.decay_path == 0 && cta_has_power_decays<G>(a);
     if (pw)
-      pipe_run<T, G, Path::kPow>(maps, a);
+      pipe_run<T, G, Path::kPow, SPLIT>(maps, a);
     else
-      pipe_run<T, G, Path::kGeneric>(maps, a);
+      pipe_run<T, G, Path::kGeneric, SPLIT>(maps, a);
   }
 }
 
@@ -554,7 +586,7 @@ bool make_maps(const KernelArgs& a, Maps* m) {
 
 template <typename T, int G, bool ZOH, int MINB>
 cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st) {
-  using S = PipeSmem<T, G>;
+  using S = PipeSmem<T, G, split_barrier<MINB>()>;
   Maps maps;
   if (!make_maps<T>(a, &maps)) return cudaErrorInvalidValue;
   auto kern = prefill_pipe_kernel<T, G, ZOH, MINB>;

@@ -233,6 +233,11 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Arrive at a named barrier without waiting for it (the waiting side uses
+// named_bar_sync with the same id and count).
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 // ----------------------------------------------------- packed f32x2 math ---
 __device__ __forceinline__ uint64_t pk2(float lo, float hi) {

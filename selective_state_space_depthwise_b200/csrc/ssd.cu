@@ -20,12 +20,14 @@
 //     last column of s's 8-column group (s1 = s | 7), and thread t turns the
 //     64-column atom t / 128 of row l = t mod 128 of the cb tile, in place,
 //     into the scores cb[l, s] exp(dA[l] - dA[s]) dt[s] for s <= l, zero above:
-//     a group wholly at or below the diagonal (s1 <= l) as cb exp(dA[l] -
-//     dA[s1]) F[s], one exponential per row and group; the group that holds
-//     the diagonal with one exponential per element. Every exponent is
-//     dA[later] - dA[earlier], <= 0 when dA_cumsum does not increase along the
-//     chunk (dt >= 0, A <= 0), so no factor exceeds 1 however strong the
-//     decay, and a factor underflows to 0 only where the exact product does.
+//     as cb exp(dA[l] - dA[s1]) F[s], one exponential per row and group. A
+//     group wholly at or below the diagonal (s1 <= l) has both exponents <= 0
+//     when dA_cumsum does not increase along the chunk (dt >= 0, A <= 0), so
+//     no factor exceeds 1 however strong the decay, and a factor underflows
+//     to 0 only where the exact product does. The group that holds the
+//     diagonal has a row factor of at most exp(dA[s0] - dA[s1]) (s0 its first
+//     column): below 80 nats it takes the same form, beyond that (where the
+//     row factor could overflow) one exponential per element.
 //     The TMA layout is already the MMA's K-major operand;
 //  4. one thread issues eight MMAs scores x x (x as an MN-major B operand) into
 //     accumulator 0 and commits both;
@@ -211,11 +213,14 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     }
     float f[8];
     unpack8(*p, f);
-    if (s0 + 7 <= l) {  // whole group at or below the diagonal: row factor x column factor, both <= 1
+    // The two-factor form also serves the diagonal group while the group's own
+    // decay range stays well inside fp32 (the same for every row of the warp).
+    const bool narrow = sdA[s0] - sdA[s0 + 7] < 80.0f;
+    if (s0 + 7 <= l || (narrow && s0 <= l)) {  // row factor x column factor
       const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
-    } else if (s0 <= l) {  // the diagonal group: each decay on its own
+      for (int q = 0; q < 8; ++q) f[q] = s0 + q <= l ? f[q] * e * F[s0 + q] : 0.0f;
+    } else if (s0 <= l) {  // the diagonal group of a strongly decaying chunk: each decay on its own
 #pragma unroll
       for (int q = 0; q < 8; ++q)
         f[q] = s0 + q <= l ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;

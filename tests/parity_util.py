@@ -87,7 +87,15 @@ def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_
     (`subsets`: {name: channel indices}, applied in every sequence). The conv
     cache must match bit for bit. Returns {name: report} (or the report of the
     single run), a report being {"y", "state", "worst_y", "worst_state",
-    "worst_channel", "subsets": {name: (y, state)}}."""
+    "worst_channel", "subsets": {name: (y, state)}}.
+
+    The run-wide and subset figures compare with the oracle rounded once to the
+    io dtype, as the other parity checks do. The worst channel's y is measured
+    against the unrounded oracle and bounded by the io dtype's unit roundoff
+    (2^-8 for bf16, 2^-24 floor plus the fp32 bar for fp32): one output that
+    sits on a rounding tie can land on either neighbour, and on a channel whose
+    largest value dominates its norm that single step alone can exceed the
+    run-wide bar even when both sides round correctly."""
     runs = got if isinstance(got, dict) else {"": got}
     x, z = inp["x"], inp["z"]
     b, L, E = x.shape
@@ -96,7 +104,7 @@ def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_
     seqs_per_block = max(1, max_elems // max(per_seq, 1))
     ch_per_block = E if seqs_per_block > 1 or per_seq <= max_elems else max(1, max_elems // max(L, 1))
     # per (sequence, channel): |dy|^2, |y|^2, |dh|^2, |h|^2
-    acc = {n: np.zeros((b, E, 4)) for n in runs}
+    acc = {n: np.zeros((b, E, 5)) for n in runs}  # + |y - unrounded oracle|^2
     for s0 in range(0, b, seqs_per_block):
         s1 = min(b, s0 + seqs_per_block)
         Bn = inp["B"][s0:s1].detach().to("cpu").double().numpy()
@@ -121,19 +129,21 @@ def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_
                 assert np.array_equal(cs, c_o), f"{label}{name}: conv_cache differs in sequences {s0}..{s1 - 1}"
                 assert np.isfinite(ys).all() and np.isfinite(hs).all(), f"{label}{name}: non-finite output"
                 blk = np.stack([np.sum((ys - want_y) ** 2, axis=1), np.sum(want_y ** 2, axis=1),
-                                np.sum((hs - h_o) ** 2, axis=1), np.sum(h_o ** 2, axis=1)], axis=1)
-                acc[name][s0:s1, e0:e1] = blk.reshape(s1 - s0, n_e, 4)
+                                np.sum((hs - h_o) ** 2, axis=1), np.sum(h_o ** 2, axis=1),
+                                np.sum((ys - out_o) ** 2, axis=1)], axis=1)
+                acc[name][s0:s1, e0:e1] = blk.reshape(s1 - s0, n_e, 5)
 
     def rl2(a):
         return (float(np.sqrt(a[..., 0].sum() / a[..., 1].sum())) if a[..., 1].sum() > 0 else float(np.sqrt(a[..., 0].sum())),
                 float(np.sqrt(a[..., 2].sum() / a[..., 3].sum())) if a[..., 3].sum() > 0 else float(np.sqrt(a[..., 2].sum())))
 
     tol = TOL[io_dtype]
+    tol_channel = 2.0 ** -8 if io_dtype == torch.bfloat16 else tol
     reports = {}
     for name, a in acc.items():
         e_y, e_h = rl2(a)
         with np.errstate(divide="ignore", invalid="ignore"):
-            cy = np.sqrt(np.where(a[..., 1] > 0, a[..., 0] / a[..., 1], a[..., 0]))
+            cy = np.sqrt(np.where(a[..., 1] > 0, a[..., 4] / a[..., 1], a[..., 4]))
             ch = np.sqrt(np.where(a[..., 3] > 0, a[..., 2] / a[..., 3], a[..., 2]))
         wy = np.unravel_index(int(np.argmax(cy)), cy.shape)
         rep = {"y": e_y, "state": e_h, "worst_y": float(cy.max()), "worst_state": float(ch.max()),
@@ -145,7 +155,8 @@ def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_
         tag = f"{label}{' ' + name if name else ''}"
         assert e_y <= tol, f"{tag}: y rel-L2 {e_y:.3e} > {tol:.0e}"
         assert e_h <= tol, f"{tag}: state rel-L2 {e_h:.3e} > {tol:.0e}"
-        assert rep["worst_y"] <= tol, f"{tag}: worst channel {rep['worst_channel']} y rel-L2 {rep['worst_y']:.3e}"
+        assert rep["worst_y"] <= tol_channel, \
+            f"{tag}: worst channel {rep['worst_channel']} y rel-L2 {rep['worst_y']:.3e} against the unrounded oracle"
         assert rep["worst_state"] <= tol, f"{tag}: worst channel state rel-L2 {rep['worst_state']:.3e}"
         for sname, (sy, sh) in rep["subsets"].items():
             assert sy <= tol and sh <= tol, f"{tag}: subset {sname} rel-L2 y {sy:.3e}, state {sh:.3e}"
@@ -156,4 +167,5 @@ def compare_full(io_dtype, inp, got, *, label="", disc="euler", dt_min=1e-4, dt_
 def format_report(rep) -> str:
     sub = ", ".join(f"{k} y {v[0]:.2e} / state {v[1]:.2e}" for k, v in rep["subsets"].items())
     return (f"y {rep['y']:.2e}, state {rep['state']:.2e}; worst channel {rep['worst_channel']}: "
-            f"y {rep['worst_y']:.2e}, state worst {rep['worst_state']:.2e}" + (f"; {sub}" if sub else ""))
+            f"y {rep['worst_y']:.2e} (against the unrounded oracle), state worst {rep['worst_state']:.2e}"
+            + (f"; {sub}" if sub else ""))
