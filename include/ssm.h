@@ -345,11 +345,13 @@ ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64
  *   prev_states  [b, nchunks, nheads, headdim, dstate] bf16
  *   D            [nheads] fp32, or NULL for no skip
  *   out          [b, L, nheads, headdim] bf16; must not overlap the inputs
- * L = nchunks * cs. The built shape is cs = 128, headdim = 64, dstate = 128
- * (SSM_ERR_UNSUPPORTED otherwise). nheads must be a multiple of ngroups, and
- * every pointer 16-byte aligned.
+ * L = nchunks * cs. The built shapes are cs = 64 or 128, headdim = 64 and
+ * dstate = 64 or 128 (SSM_ERR_UNSUPPORTED otherwise). nheads must be a
+ * multiple of ngroups, and every pointer 16-byte aligned.
  *
- * Computation. Per (b, c, h) one CTA:
+ * Computation. Per (b, h) and 128 positions -- one chunk of 128, or two
+ * consecutive chunks of 64 on the diagonal of one 128 x 128 score tile -- one
+ * CTA:
  *  - scores = masked cb * exp(dA[l] - dA[s]) * dt[s] in bf16, times x;
  *  - C[l] in bf16, times prev_states^T;
  * as tcgen05 MMAs into two fp32 TMEM accumulators, combined as

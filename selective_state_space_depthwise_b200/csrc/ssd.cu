@@ -50,11 +50,12 @@
 namespace ssm {
 namespace {
 
-constexpr int kCs = 128;  // chunk length: MMA M and the K of the intra-chunk term
+constexpr int kCs = 128;  // rows of a CTA's tile: MMA M and the K of the intra-chunk term
 constexpr int kHd = 64;   // head dim: MMA N
-constexpr int kDs = 128;  // state dim: the K of the carried-state term
+// Template parameters: the chunk length CS (64 or 128; a CTA's 128 rows hold
+// 128 / CS consecutive chunks) and the state dim DS (64 or 128: the K of the
+// carried-state term).
 constexpr int kSsdThreads = 256;
-constexpr uint32_t kSsdTmemCols = 128;
 // Load order: 1 = cb and x first (the score math starts sooner; the
 // carried-state MMAs go last), 0 = C and prev_states first (their MMAs are
 // issued on arrival). Measured on B200 at b = 8, L = 4096, 80 heads: 364 us
@@ -64,21 +65,28 @@ constexpr uint32_t kSsdTmemCols = 128;
 #endif
 constexpr bool kScoresFirst = SSM_SSD_SCORES_FIRST;  // accumulator 0 (intra-chunk) at column 0, 1 (carried state) at 64
 
+template <int CS, int DS>
 struct SsdSmem {
+  static_assert(DS == 64 || DS == 128, "state dim 64 or 128");
+  static_assert(CS == 64 || CS == 128, "chunk 64 or 128");
+  static constexpr int kNC = kCs / CS;             // chunks per CTA
+  static constexpr int kNA = DS / 64;              // 64-column atoms across the state dim
   static constexpr int kAtomRows128 = kCs * 128;   // one 64-column atom of a 128-row tile
   static constexpr int kAtomRows64 = kHd * 128;    // one 64-column atom of a 64-row tile
   static constexpr int kCb = 0;                    // cb -> scores (A of MMA 1) -> out tile
-  static constexpr int kC = 2 * kAtomRows128;      // C -> exp(dA) C (A of MMA 2)
-  static constexpr int kX = 4 * kAtomRows128;      // x [s][p] (B of MMA 1, MN-major)
-  static constexpr int kPrev = kX + kAtomRows128;  // prev_states [p][n] (B of MMA 2, K-major)
-  static constexpr int kDA = kPrev + 2 * kAtomRows64;
+  static constexpr int kC = 2 * kAtomRows128;      // C (A of MMA 2)
+  static constexpr int kX = kC + kNA * kAtomRows128;  // x [s][p] (B of MMA 1, MN-major)
+  static constexpr int kPrev = kX + kAtomRows128;  // prev_states [chunk][p][n] (B of MMA 2, K-major)
+  static constexpr int kDA = kPrev + kNC * kNA * kAtomRows64;
   static constexpr int kDt = kDA + kCs * 4;
   static constexpr int kF = kDt + kCs * 4;
   static constexpr int kBar = kF + kCs * 4;        // full_state, full_scores, done
   static constexpr int kTmemSlot = kBar + 24;
   static constexpr int kTotal = kTmemSlot + 16;
-  static constexpr uint32_t kTxState = static_cast<uint32_t>(2 * kAtomRows128 + 2 * kAtomRows64);  // C, prev
-  static constexpr uint32_t kTxScores = static_cast<uint32_t>(3 * kAtomRows128);                    // cb, x
+  static constexpr uint32_t kTxState = static_cast<uint32_t>(kNA * (kAtomRows128 + kNC * kAtomRows64));  // C, prev
+  // cb: the chunks' [CS][CS] diagonal blocks of the [128][128] score tile; x
+  static constexpr uint32_t kTxScores = static_cast<uint32_t>(kNC * CS * CS * 2 + kAtomRows128);
+  static constexpr uint32_t kTmemCols = kNC == 1 ? 128u : 256u;  // intra + one carried-state term per chunk
   static_assert(kC % 1024 == 0 && kX % 1024 == 0 && kPrev % 1024 == 0, "swizzled tiles need 1 KB");
 };
 
@@ -120,18 +128,20 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+template <int CS, int DS>
 __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     const __grid_constant__ CUtensorMap map_cb, const __grid_constant__ CUtensorMap map_x,
     const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_prev,
     const __grid_constant__ CUtensorMap map_out, const SsdArgs a) {
-  using S = SsdSmem;
+  using S = SsdSmem<CS, DS>;
+  constexpr int NC = S::kNC;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(smem);
   const int tid = threadIdx.x;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
   const int l = tid & (kCs - 1), at = tid >> 7;  // this thread's row and 64-column atom
-  const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.x, c = blockIdx.y * NC, b = blockIdx.z;  // first chunk of this CTA
   const int g = static_cast<int>(h / (a.nheads / a.ngroups));
   const uint32_t full_state = sb + S::kBar, full_scores = sb + S::kBar + 8, done = sb + S::kBar + 16;
   if (tid == 0) {
@@ -143,22 +153,35 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_c);
     prefetch_tensormap(&map_prev);
-    const int zc = static_cast<int>((static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g);
-    const int zp = static_cast<int>((static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h);
+    // A second chunk past the last one (odd chunk count) reads zeros or a
+    // neighbouring sequence's chunk; its rows lie past L and are never stored.
+    const int64_t zc0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g;
+    const int64_t zp0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h;
     mbar_arrive_expect_tx(full_state, S::kTxState);
     mbar_arrive_expect_tx(full_scores, S::kTxScores);
     auto load_state = [&] {
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        tma_load_4d(sb + S::kC + t * S::kAtomRows128, &map_c, 64 * t, g, c * kCs, b, full_state);
-        tma_load_3d(sb + S::kPrev + t * S::kAtomRows64, &map_prev, 64 * t, 0, zp, full_state);
+      for (int t = 0; t < S::kNA; ++t) {
+        tma_load_4d(sb + S::kC + t * S::kAtomRows128, &map_c, 64 * t, g, c * CS, b, full_state);
+#pragma unroll
+        for (int k = 0; k < NC; ++k)
+          tma_load_3d(sb + S::kPrev + (k * S::kNA + t) * S::kAtomRows64, &map_prev, 64 * t, 0,
+                      static_cast<int>(zp0 + k * a.nheads), full_state);
       }
     };
     auto load_scores = [&] {
+      if constexpr (NC == 1) {
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
-        tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, 64 * t, 0, zc, full_scores);
-      tma_load_4d(sb + S::kX, &map_x, 0, h, c * kCs, b, full_scores);
+        for (int t = 0; t < 2; ++t)
+          tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, 64 * t, 0, static_cast<int>(zc0), full_scores);
+      } else {
+        // chunk k's [64][64] block on the diagonal: atom k, rows 64 k ..
+#pragma unroll
+        for (int k = 0; k < NC; ++k)
+          tma_load_3d(sb + S::kCb + k * S::kAtomRows128 + k * CS * 128, &map_cb, 0, 0,
+                      static_cast<int>(zc0 + k * a.ngroups), full_scores);
+      }
+      tma_load_4d(sb + S::kX, &map_x, 0, h, c * CS, b, full_scores);
     };
     if (kScoresFirst) {
       load_scores();
@@ -169,45 +192,57 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     }
   }
   if (warp == 0) {
-    tmem_alloc(sb + S::kTmemSlot, kSsdTmemCols);
+    tmem_alloc(sb + S::kTmemSlot, S::kTmemCols);
     tmem_relinquish();
   }
   float* sdA = reinterpret_cast<float*>(smem + S::kDA);
   float* sdt = reinterpret_cast<float*>(smem + S::kDt);
   float* F = reinterpret_cast<float*>(smem + S::kF);
-  if (tid < kCs) {
-    const int64_t row = ((static_cast<int64_t>(b) * a.nheads + h) * a.nchunks + c) * kCs;
-    sdA[tid] = a.dA[row + tid];
-    sdt[tid] = a.dt[row + tid];
+  if (tid < kCs) {  // the CTA's chunks are consecutive in [b][H][nc][CS]
+    const int64_t row = ((static_cast<int64_t>(b) * a.nheads + h) * a.nchunks + c) * CS;
+    const bool in = c + tid / CS < a.nchunks;
+    sdA[tid] = in ? a.dA[row + tid] : 0.0f;
+    sdt[tid] = in ? a.dt[row + tid] : 0.0f;
   }
   const float Dh = a.D ? a.D[h] : 0.0f;
   tcgen05_fence_before();
   __syncthreads();
   tcgen05_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
-  const uint32_t acc_intra = tmem, acc_state = tmem + kHd;
+  // Accumulators: the intra-chunk term at column 0, the carried-state term of
+  // chunk k at 64 (k + 1) (C x prev_states(k)^T over all 128 rows; rows of
+  // chunk k read it).
+  const uint32_t acc_intra = tmem;
+  auto state_mmas = [&] {
+#pragma unroll
+    for (int k = 0; k < NC; ++k)
+#pragma unroll
+      for (int kk = 0; kk < DS / 16; ++kk)
+        umma_f16_ss(tmem + kHd * (k + 1),
+                    umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+                    umma_desc_k_sw128(sb + S::kPrev + (k * S::kNA + (kk >> 2)) * S::kAtomRows64 + (kk & 3) * 32),
+                    ssd_idesc(false), kk > 0);
+  };
   // 2. Carried-state term, as soon as its operands are in: C[l][n] x prev_states[p][n]^T.
   if (tid == 0 && !kScoresFirst) {
     mbar_wait_bounded(full_state, 0u, a.err, 7);
     tcgen05_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < kDs / 16; ++kk)
-      umma_f16_ss(acc_state, umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
-                  umma_desc_k_sw128(sb + S::kPrev + (kk >> 2) * S::kAtomRows64 + (kk & 3) * 32), ssd_idesc(false),
-                  kk > 0);
+    state_mmas();
   }
   if (tid < kCs) F[tid] = ex2_approx((sdA[tid | 7] - sdA[tid]) * kLog2e) * sdt[tid];
   const float dAl = sdA[l];
   mbar_wait_bounded(full_scores, 0u, a.err, 8);
   __syncthreads();  // F complete
 
-  // 3. This thread's atom of row l of the cb tile -> scores (in place).
+  // 3. This thread's atom of row l of the cb tile -> scores (in place). A
+  //    warp's 32 rows lie in one chunk, starting at column warp_min_s.
   const int warp_max_l = 32 * (warp & 3) + 31;
+  const int warp_min_s = (32 * (warp & 3)) & ~(CS - 1);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int s0 = 64 * at + 8 * j;
     uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
-    if (s0 > warp_max_l) {  // above the diagonal for every row of this warp
+    if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
       *p = make_uint4(0u, 0u, 0u, 0u);
       continue;
     }
@@ -243,11 +278,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     if (kScoresFirst) {  // carried-state term last: its operands were loaded second
       mbar_wait_bounded(full_state, 0u, a.err, 7);
       tcgen05_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kDs / 16; ++kk)
-        umma_f16_ss(acc_state, umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
-                    umma_desc_k_sw128(sb + S::kPrev + (kk >> 2) * S::kAtomRows64 + (kk & 3) * 32),
-                    ssd_idesc(false), kk > 0);
+      state_mmas();
     }
     umma_commit(done);
   }
@@ -260,6 +291,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     const int q4 = warp & 3, col0 = 32 * (warp >> 2);
     const int row = 32 * q4 + (tid & 31);
     const float el = ex2_approx(sdA[row] * kLog2e);
+    const uint32_t acc_state = tmem + kHd * (1 + (32 * q4) / CS);  // this warp's chunk
 #pragma unroll
     for (int jj = 0; jj < 2; ++jj) {
       uint32_t r0[16], r1[16];
@@ -282,7 +314,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   fence_proxy_async_smem();
   __syncthreads();
   if (tid == 0) {
-    tma_store_4d(&map_out, sb + S::kCb, 0, h, c * kCs, b);
+    tma_store_4d(&map_out, sb + S::kCb, 0, h, c * CS, b);
     bulk_commit();
     bulk_wait_read<0>();  // the tile stays in shared memory until the store has read it
   }
@@ -290,7 +322,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   __syncthreads();
   if (warp == 0) {
     tcgen05_fence_after();
-    tmem_dealloc(tmem, kSsdTmemCols);
+    tmem_dealloc(tmem, S::kTmemCols);
   }
 }
 
@@ -307,6 +339,21 @@ bool bf16_map(CUtensorMap* m, int rank, const void* base, std::initializer_list<
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, d, s, bx, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+template <int CS, int DS>
+cudaError_t launch_ssd(int64_t H, int64_t nc, int64_t b, const CUtensorMap& mcb, const CUtensorMap& mx,
+                       const CUtensorMap& mc, const CUtensorMap& mp, const CUtensorMap& mo, const SsdArgs& a,
+                       cudaStream_t st) {
+  using S = SsdSmem<CS, DS>;
+  const int smem = S::kTotal + 1024;
+  auto kern = ssd_chunk_scan_kernel<CS, DS>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>((nc + S::kNC - 1) / S::kNC),
+                  static_cast<unsigned>(b));
+  kern<<<grid, kSsdThreads, smem, st>>>(mcb, mx, mc, mp, mo, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 }  // namespace ssm
 
@@ -317,8 +364,10 @@ extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* c
   if (!dims) return fail(SSM_ERR_INVALID_ARG, "dims is NULL");
   const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim, G = dims->ngroups;
   const int64_t N = dims->dstate, cs = dims->chunk_size;
-  if (cs != ssm::kCs || P != ssm::kHd || N != ssm::kDs)
-    return fail(SSM_ERR_UNSUPPORTED, "chunk_size %lld, headdim %lld, dstate %lld: the built shape is 128, 64, 128",
+  if ((cs != 64 && cs != 128) || P != ssm::kHd || (N != 64 && N != 128))
+    return fail(SSM_ERR_UNSUPPORTED,
+                "chunk_size %lld, headdim %lld, dstate %lld: the built shapes are chunk 64 or 128, headdim 64, "
+                "dstate 64 or 128",
                 (long long)cs, (long long)P, (long long)N);
   if (b <= 0 || b > 65535 || H <= 0 || H > 0x7fffffff || G <= 0 || H % G != 0)
     return fail(SSM_ERR_INVALID_ARG, "need 0 < batch <= 65535, nheads > 0 and nheads a multiple of ngroups");
@@ -337,7 +386,7 @@ extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* c
   const uint64_t e2 = 2;
   const bool ok =
       ssm::bf16_map(&mcb, 3, cb, {uint64_t(cs), uint64_t(cs), uint64_t(b * nc * G)}, {cs * e2, cs * cs * e2},
-                    {64, 128, 1}) &&
+                    {64, uint32_t(cs), 1}) &&
       ssm::bf16_map(&mx, 4, x, {uint64_t(P), uint64_t(H), uint64_t(L), uint64_t(b)},
                     {P * e2, H * P * e2, L * H * P * e2}, {64, 1, 128, 1}) &&
       ssm::bf16_map(&mc, 4, C, {uint64_t(N), uint64_t(G), uint64_t(L), uint64_t(b)},
@@ -349,13 +398,14 @@ extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* c
   if (!ok) return fail(SSM_ERR_CUDA, "tensor map encoding failed");
   ssm::SsdArgs a{dt, dA_cumsum, D, H, nc, G, ssm::device_error_ptr()};
   if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
-  const int smem = ssm::SsdSmem::kTotal + 1024;
-  cudaError_t err =
-      cudaFuncSetAttribute(ssm::ssd_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "smem attribute: %s", cudaGetErrorString(err));
-  ssm::ssd_chunk_scan_kernel<<<dim3(static_cast<unsigned>(H), static_cast<unsigned>(nc), static_cast<unsigned>(b)),
-                               ssm::kSsdThreads, smem, static_cast<cudaStream_t>(stream)>>>(mcb, mx, mc, mp, mo, a);
-  err = cudaGetLastError();
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (cs == 128)
+    err = N == 128 ? ssm::launch_ssd<128, 128>(H, nc, b, mcb, mx, mc, mp, mo, a, st)
+                   : ssm::launch_ssd<128, 64>(H, nc, b, mcb, mx, mc, mp, mo, a, st);
+  else
+    err = N == 128 ? ssm::launch_ssd<64, 128>(H, nc, b, mcb, mx, mc, mp, mo, a, st)
+                   : ssm::launch_ssd<64, 64>(H, nc, b, mcb, mx, mc, mp, mo, a, st);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "chunk-scan launch: %s", cudaGetErrorString(err));
   return fail(SSM_OK, "");
 }

@@ -75,6 +75,37 @@ def test_ssd_two_groups_many_chunks():
     assert e <= TOL_SSD
 
 
+def test_ssd_state_dim_64():
+    """d_state 64 (one 64-column operand atom for C and prev_states), two
+    groups, every output against the oracle."""
+    spec = dict(batch=2, seqlen=512, nheads=6, headdim=64, ngroups=2, dstate=64, chunk_size=128, seed=43)
+    inp = W.make_ssd_inputs(spec, device="cuda")
+    out = run(inp).double().cpu().numpy()
+    f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
+    want = oracle.ssd_chunk_scan(*(f(inp[k]) for k in ARGS))
+    e = rel_l2(out, want)
+    print(f"ssd dstate 64: rel-L2 {e:.2e}")
+    assert e <= TOL_SSD
+
+
+@pytest.mark.parametrize("dstate", [64, 128])
+@pytest.mark.parametrize("seqlen", [512, 448])
+def test_ssd_chunk_64(dstate, seqlen):
+    """Chunk length 64: two consecutive chunks share a CTA's 128-row tiles
+    (block-diagonal scores, one carried-state term per chunk); 448 tokens give
+    an odd chunk count, so the last CTA holds one chunk. Every output against
+    the oracle."""
+    spec = dict(batch=2, seqlen=seqlen, nheads=4, headdim=64, ngroups=2, dstate=dstate, chunk_size=64,
+                seed=47 + dstate + seqlen)
+    inp = W.make_ssd_inputs(spec, device="cuda")
+    out = run(inp).double().cpu().numpy()
+    f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
+    want = oracle.ssd_chunk_scan(*(f(inp[k]) for k in ARGS))
+    e = rel_l2(out, want)
+    print(f"ssd chunk 64, dstate {dstate}, L {seqlen}: rel-L2 {e:.2e}")
+    assert e <= TOL_SSD
+
+
 def test_ssd_full_size_every_chunk():
     """b=8, L=4096, 80 heads: every (sequence, chunk) pair, every head and
     position, against the oracle one sequence at a time; the rel-L2 is pooled
