@@ -528,14 +528,15 @@ def gemm_bench(bf16_peak: float, steps: int = 20, warmup: int = 3):
     return out
 
 
-def ssd_bench(name: str, hbm_peak: float, bf16_peak: float, steps: int = 20, warmup: int = 3):
+def ssd_bench(name: str, hbm_peak: float, bf16_peak: float, steps: int = 20, warmup: int = 3, spec_over=None):
     """The Mamba-2 chunk scan on device-resident inputs: us per call by CUDA
     events; HBM roofline on the algorithmic bytes (read cb, x, dt, dA_cumsum, C,
     prev_states, D once, write out once) and the tensor FLOPs of the two
-    contractions (2 cs cs P + 2 cs N P per chunk and head)."""
+    contractions (2 cs cs P + 2 cs N P per chunk and head). spec_over replaces
+    fields of the named workload (another built chunk length or state dim)."""
     from selective_state_space_depthwise_b200 import api
 
-    spec = W.SSD_WORKLOADS[name]
+    spec = dict(W.SSD_WORKLOADS[name], **(spec_over or {}))
     inp = W.make_ssd_inputs(spec, device="cuda")
     args = [inp[k] for k in ("cb", "x", "dt", "dA_cumsum", "C", "prev_states", "D")]
     out = torch.empty_like(inp["x"])
@@ -823,6 +824,9 @@ def main():
             extra["projection_gemms"] = gemm_bench(bf16_peak)
             torch.cuda.empty_cache()
             extra["ssd_chunk_scan"] = ssd_bench("ssd_chunk_scan", hbm_peak, bf16_peak)
+            extra["ssd_chunk_scan_shapes"] = [
+                ssd_bench("ssd_chunk_scan", hbm_peak, bf16_peak, spec_over={"chunk_size": cs, "dstate": ds})
+                for cs, ds in ((64, 128), (256, 128), (128, 64))]
         if not args.no_seqpar:
             torch.cuda.empty_cache()
             extra["sequence_parallel"] = seqpar_bench(w)

@@ -286,8 +286,9 @@ ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const voi
  *             output), so chained calls equal one call over the whole sequence.
  *   workspace device scratch of ssm_block_workspace_bytes(dims) bytes,
  *             256-byte aligned. It holds the in_proj output (b L 2E bf16),
- *             B / C / dt_raw (b L 33 fp32) and the gated core output
- *             (b L E bf16).
+ *             B / C / dt_raw (b L 33 fp32), the gated core output
+ *             (b L E bf16) and the projections' split-K scratch (see
+ *             ssm_proj_gemm).
  *
  * Ordering and errors. Everything is enqueued on `stream`, with no host
  * synchronisation. Argument errors return before any work is queued.
@@ -323,9 +324,18 @@ size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
  * Device pointers, 16-byte aligned; K and N multiples of 8; 0 < M, N, K <=
  * 2^31; C must not alias A or W. fp32 accumulation, C rounded to bf16 (RNE).
  * One persistent kernel (tcgen05 MMAs into TMEM, TMA operand ring, TMA
- * stores) enqueued on `stream`; no workspace.
+ * stores) enqueued on `stream`, after a memset of the workspace's tile
+ * counters when the shape runs split-K.
+ *   workspace  ssm_proj_gemm_workspace_bytes(M, N, K) bytes of device scratch,
+ *              256-byte aligned, or NULL when that is 0. Shapes whose 128 x 256
+ *              output tiles would leave most SMs idle in a last wave split K
+ *              into up to 4 slices; the slices' fp32 partial tiles and a
+ *              counter per tile live here. Calls that overlap on the GPU need
+ *              separate workspaces.
  */
-ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64_t N, int64_t K, void *stream);
+size_t ssm_proj_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64_t N, int64_t K, void *workspace,
+                         size_t workspace_bytes, void *stream);
 
 /*
  * ssm_ssd_chunk_scan -- the output of the Mamba-2 (SSD) chunk scan, "What is
@@ -345,13 +355,15 @@ ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64
  *   prev_states  [b, nchunks, nheads, headdim, dstate] bf16
  *   D            [nheads] fp32, or NULL for no skip
  *   out          [b, L, nheads, headdim] bf16; must not overlap the inputs
- * L = nchunks * cs. The built shapes are cs = 64 or 128, headdim = 64 and
- * dstate = 64 or 128 (SSM_ERR_UNSUPPORTED otherwise). nheads must be a
- * multiple of ngroups, and every pointer 16-byte aligned.
+ * L = nchunks * cs. The built shapes are cs = 64, 128 or 256, headdim = 64
+ * and dstate = 64 or 128 (SSM_ERR_UNSUPPORTED otherwise); at most 32767
+ * chunks. nheads must be a multiple of ngroups, and every pointer 16-byte
+ * aligned.
  *
- * Computation. Per (b, h) and 128 positions -- one chunk of 128, or two
- * consecutive chunks of 64 on the diagonal of one 128 x 128 score tile -- one
- * CTA:
+ * Computation. Per (b, h) and 128 positions -- one chunk of 128, two
+ * consecutive chunks of 64 on the diagonal of one 128 x 128 score tile, or
+ * one half of a chunk of 256 (the second half contracting over all 256
+ * positions) -- one CTA:
  *  - scores = masked cb * exp(dA[l] - dA[s]) * dt[s] in bf16, times x;
  *  - C[l] in bf16, times prev_states^T;
  * as tcgen05 MMAs into two fp32 TMEM accumulators, combined as

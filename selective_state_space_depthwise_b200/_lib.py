@@ -30,6 +30,7 @@ EXPORTED = (
     "ssm_block_forward",
     "ssm_block_workspace_bytes",
     "ssm_proj_gemm",
+    "ssm_proj_gemm_workspace_bytes",
     "ssm_ssd_chunk_scan",
     "ssm_segment_summary",
     "ssm_segment_summary_workspace_bytes",
@@ -135,8 +136,10 @@ def load(path: str = LIB_PATH):
     lib.ssm_block_workspace_bytes.argtypes = [bdims_p]
     lib.ssm_block_workspace_bytes.restype = sz
     i64 = ctypes.c_int64
-    lib.ssm_proj_gemm.argtypes = [p, p, p, i64, i64, i64, p]
+    lib.ssm_proj_gemm.argtypes = [p, p, p, i64, i64, i64, p, sz, p]
     lib.ssm_proj_gemm.restype = st
+    lib.ssm_proj_gemm_workspace_bytes.argtypes = [i64, i64, i64]
+    lib.ssm_proj_gemm_workspace_bytes.restype = sz
     lib.ssm_ssd_chunk_scan.argtypes = [ctypes.POINTER(SsmSsdDims)] + [p] * 8 + [p]
     lib.ssm_ssd_chunk_scan.restype = st
     lib.ssm_segment_summary.argtypes = [dims_p, w_p] + [p] * 6 + [sz, p]

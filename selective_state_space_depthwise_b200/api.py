@@ -318,9 +318,15 @@ def block_forward(hidden, params, proj, *, conv_cache_in=None, ssm_state_in=None
     return out, conv_cache_out, ssm_state_out
 
 
-def proj_gemm(A, W, *, out=None, stream=None):
+def proj_gemm_workspace_bytes(M, N, K) -> int:
+    lib = _lib.load()
+    return int(lib.ssm_proj_gemm_workspace_bytes(int(M), int(N), int(K)))
+
+
+def proj_gemm(A, W, *, out=None, workspace=None, stream=None):
     """One projection of the block (ssm_proj_gemm): out = A @ W^T with A [M, K]
-    and W [N, K] contiguous bf16 CUDA tensors; returns out [M, N] bf16."""
+    and W [N, K] contiguous bf16 CUDA tensors; returns out [M, N] bf16. The
+    split-K scratch, when the shape needs one, is `workspace` or allocated."""
     lib = _lib.load()
     M, K = A.shape
     N = W.shape[0]
@@ -335,7 +341,11 @@ def proj_gemm(A, W, *, out=None, stream=None):
         out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     if out.shape != (M, N):
         raise ValueError("out must be [M, N]")
-    _lib.check(lib.ssm_proj_gemm(_ptr(A), _ptr(W), _ptr(out), M, N, K, _stream(stream)))
+    ws = int(lib.ssm_proj_gemm_workspace_bytes(M, N, K))
+    if ws and (workspace is None or workspace.numel() * workspace.element_size() < ws):
+        workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+    _lib.check(lib.ssm_proj_gemm(_ptr(A), _ptr(W), _ptr(out), M, N, K, _ptr(workspace) if ws else None, ws,
+                                 _stream(stream)))
     return out
 
 

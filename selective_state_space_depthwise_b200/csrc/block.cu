@@ -310,8 +310,15 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct BlockLayout {
-  size_t xz, bc, dt, y, bytes;
+  size_t xz, bc, dt, y, gemm, gemm_bytes, bytes;
 };
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();  // no device: the default SM count
+  return sms > 0 ? sms : 148;
+}
 
 BlockLayout block_layout(const ssm_block_dims* d) {
   const size_t M = static_cast<size_t>(d->batch * d->seqlen), E = static_cast<size_t>(d->d_inner);
@@ -321,6 +328,12 @@ BlockLayout block_layout(const ssm_block_dims* d) {
   l.bc = off, off = align_up(off + M * 32 * 4);
   l.dt = off, off = align_up(off + M * 4);
   l.y = off, off = align_up(off + M * E * 2);
+  // split-K scratch of whichever projection needs more (in_proj and out_proj run one after the other)
+  const int sms = sm_count();
+  const int64_t Mi = static_cast<int64_t>(M), Ei = static_cast<int64_t>(E), Dm = d->d_model;
+  const size_t g_in = gemm_workspace_bytes(Mi, 2 * Ei, Dm, sms), g_out = gemm_workspace_bytes(Mi, Dm, Ei, sms);
+  l.gemm_bytes = g_in > g_out ? g_in : g_out;
+  l.gemm = off, off = align_up(off + l.gemm_bytes);
   l.bytes = off;
   return l;
 }
@@ -402,7 +415,8 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // in_proj: xz[M][2E] = hidden[M][D] . W_in[2E][D]^T
-  cudaError_t err = ssm::gemm_bf16_tn(hidden, proj->w_in, xz, M, 2 * E, Dm, 0, sms, err_word, cs);
+  cudaError_t err =
+      ssm::gemm_bf16_tn(hidden, proj->w_in, xz, M, 2 * E, Dm, ws + lay.gemm, lay.gemm_bytes, sms, err_word, cs);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "in_proj launch: %s", cudaGetErrorString(err));
   // x_proj (fused with conv + SiLU): B, C, dt_raw
   ssm::XprojArgs xa{};
@@ -429,7 +443,7 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
                         ssm_state_out, nullptr, 0, stream)) != SSM_OK)
     return st;
   // out_proj: out[M][D] = y[M][E] . W_out[D][E]^T
-  err = ssm::gemm_bf16_tn(y, proj->w_out, out, M, Dm, E, 0, sms, err_word, cs);
+  err = ssm::gemm_bf16_tn(y, proj->w_out, out, M, Dm, E, ws + lay.gemm, lay.gemm_bytes, sms, err_word, cs);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "out_proj launch: %s", cudaGetErrorString(err));
   return ssm::fail(SSM_OK, "");
 }

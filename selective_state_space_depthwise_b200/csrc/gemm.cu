@@ -3,7 +3,7 @@
 // model", "Algorithm" diagram, as C[M][N] = A[M][K] . B[N][K]^T with A and B
 // bf16 row-major (both K-major), fp32 accumulation and a bf16 C.
 //
-// One persistent CTA per SM walks output tiles of 128 x BN (BN = 256 or 160)
+// One persistent CTA per SM walks output tiles of 128 x BN (BN = 256)
 // in a static round-robin order over a grouped raster: tiles run in groups of
 // up to 16 row blocks x every column block, row block fastest inside a group,
 // so the CTAs running at the same time share both their A row blocks and their
@@ -61,7 +61,10 @@ struct GemmSmem {
   static constexpr int kTmemSlot = kBar + (2 * STAGES + 4) * 8;
   static constexpr int kAbort = kTmemSlot + 4;
   static constexpr int kIssued = kTmemSlot + 8;  // int64: K chunks the producer issued
-  static constexpr int kTotal = kIssued + 8;
+  static constexpr int kSplitFlag = kIssued + 8;  // int: this unit finished its tile (split K)
+  static constexpr int kPartBar = kSplitFlag + 8;  // split K: the 4 epilogue warps published their rows
+  static constexpr int kDecBar = kPartBar + 8;     // split K: the unit's tile counter was read
+  static constexpr int kTotal = kDecBar + 8;
   // TMEM columns: two accumulators of BN, allocated as a power of two.
   static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256u : 512u;
   static_assert(kStage % 1024 == 0, "swizzled operand tiles need 1 KB alignment");
@@ -69,9 +72,21 @@ struct GemmSmem {
 
 struct GemmArgs {
   int tiles_m, tiles_n, k_chunks;
-  int group_m;  // row blocks per raster group
+  int group_m;      // row blocks per raster group
+  int nsplit;       // K slices per tile (work units = tiles x nsplit)
+  float* partial;   // nsplit > 1: [tiles][nsplit][128][BN] fp32 partial tiles
+  int* counters;    // nsplit > 1: [tiles], zero on entry: slices of each tile finished
   int* err;
 };
+
+// Work unit -> its tile and K-chunk range: the nsplit slices of a tile are
+// consecutive units, so consecutive CTAs run them at the same time.
+__device__ __forceinline__ void unit_range(const GemmArgs& g, int unit, int& tile, int& split, int& k0, int& k1) {
+  tile = unit / g.nsplit;
+  split = unit - tile * g.nsplit;
+  k0 = static_cast<int>(static_cast<int64_t>(split) * g.k_chunks / g.nsplit);
+  k1 = static_cast<int>(static_cast<int64_t>(split + 1) * g.k_chunks / g.nsplit);
+}
 
 // Tile index -> (row block, column block) of the grouped raster.
 __device__ __forceinline__ void tile_coords(const GemmArgs& g, int tile, int& mb, int& nb) {
@@ -106,7 +121,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
   auto tempty = [&](int b) { return sb + S::kBar + 8 * (2 * STAGES + 2 + b); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kAbort);
   volatile int64_t* issued_slot = reinterpret_cast<volatile int64_t*>(smem + S::kIssued);
-  const int ntiles = g.tiles_m * g.tiles_n;
+  volatile int* split_flag = reinterpret_cast<volatile int*>(smem + S::kSplitFlag);
+  const uint32_t part_bar = sb + S::kPartBar, dec_bar = sb + S::kDecBar;
+  const int nunits = g.tiles_m * g.tiles_n * g.nsplit;
 
   if (tid == 0) {
     *abort_flag = 0;
@@ -119,6 +136,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
       mbar_init(tfull(b), 1);
       mbar_init(tempty(b), 4);  // one arrival per epilogue warp
     }
+    mbar_init(part_bar, 4);
+    mbar_init(dec_bar, 1);
     mbar_fence_init();
     prefetch_tensormap(&map_a);
     prefetch_tensormap(&map_b);
@@ -137,11 +156,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // ---------------------------------------------------------- producer ---
     if (lane == 0) {
       int64_t it = 0;
-      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
-        int mb, nb;
+      for (int unit = blockIdx.x; unit < nunits && !*abort_flag; unit += gridDim.x) {
+        int tile, split, k0, k1, mb, nb;
+        unit_range(g, unit, tile, split, k0, k1);
         tile_coords(g, tile, mb, nb);
         const int m0 = mb * kGBM, n0 = nb * BN;
-        for (int kc = 0; kc < g.k_chunks; ++kc, ++it) {
+        for (int kc = k0; kc < k1; ++kc, ++it) {
           const int s = static_cast<int>(it % STAGES);
           const uint32_t round = static_cast<uint32_t>(it / STAGES);
           if (!mbar_wait_bounded(empty(s), (round & 1u) ^ 1u, g.err, 21) || *abort_flag) {
@@ -162,7 +182,9 @@ __global__ void __launch_bounds__(kGThreads, 1)
       int last_slot = -1;
       uint32_t last_round = 0;
       int i = 0;
-      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++i) {
+      for (int unit = blockIdx.x; unit < nunits && !*abort_flag; unit += gridDim.x, ++i) {
+        int tile, split, k0, k1;
+        unit_range(g, unit, tile, split, k0, k1);
         const int buf = i & 1;
         if (!mbar_wait_bounded(tempty(buf), (static_cast<uint32_t>(i >> 1) & 1u) ^ 1u, g.err, 22)) {
           *abort_flag = 1;
@@ -171,7 +193,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         tcgen05_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
         bool ok = true;
-        for (int kc = 0; kc < g.k_chunks; ++kc, ++it) {
+        for (int kc = k0; kc < k1; ++kc, ++it) {
           const int s = static_cast<int>(it % STAGES);
           const uint32_t round = static_cast<uint32_t>(it / STAGES);
           if (!mbar_wait_bounded(full(s), round & 1u, g.err, 23) || *abort_flag) {
@@ -184,7 +206,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < kGBK / 16; ++kk)
             umma_f16_ss(d, umma_desc_k_sw128(a + 32 * kk), umma_desc_k_sw128(b + 32 * kk), gemm_idesc<BN>(),
-                        kc > 0 || kk > 0);
+                        kc > k0 || kk > 0);
           umma_commit(empty(s));  // the slot is free once these MMAs have read it
           last_slot = s;
           last_round = round;
@@ -205,9 +227,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
     int ob = 0, i = 0;
     // Every decision below is warp-uniform: tcgen05.ld is a .sync.aligned
     // instruction that all 32 lanes must reach together.
-    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+    for (int unit = blockIdx.x; unit < nunits; unit += gridDim.x, ++i) {
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
-      int mb, nb;
+      int tile, split, k0, k1, mb, nb;
+      unit_range(g, unit, tile, split, k0, k1);
       tile_coords(g, tile, mb, nb);
       const int m0 = mb * kGBM, n0 = nb * BN;
       const int buf = i & 1;
@@ -218,30 +241,83 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
       tcgen05_fence_after();
       const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
+      const int row = 32 * q + lane;  // this thread's row of the tile
+      bool store = true;              // this unit writes the bf16 tile
+      if (g.nsplit > 1) {
+        // Every slice publishes its fp32 partial; the slice that finishes the
+        // tile last adds the others to its own and writes the output.
+        float* mine = g.partial + ((static_cast<int64_t>(tile) * g.nsplit + split) * kGBM + row) * BN;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld_x32(t_row + 32 * c, r);
-        tmem_ld_wait();
-        uint32_t w[16];
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_x32(t_row + 32 * c, r);
+          tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-          w[j] = *reinterpret_cast<const uint32_t*>(&v);
+          for (int j = 0; j < 8; ++j)
+            reinterpret_cast<float4*>(mine + 32 * c)[j] =
+                make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
+                            __uint_as_float(r[4 * j + 3]));
         }
-        if (lane == 0) bulk_wait_read<1>();  // the store that last read staging tile `ob` is done with it
+        // Handshake of the four epilogue warps on two mbarriers (bounded
+        // waits, so a warp that left on an abort cannot strand the others):
+        // all four publish their rows, then one thread counts the slice in.
+        __threadfence();
         __syncwarp();
-        unsigned char* st = stage0_ptr + ob * S::kOutBytes;
+        if (lane == 0) mbar_arrive(part_bar);
+        if (warp == 2 && lane == 0) {
+          const bool okp = mbar_wait_bounded(part_bar, static_cast<uint32_t>(i) & 1u, g.err, 27);
+          if (!okp) *abort_flag = 1;
+          *split_flag = okp && atomicAdd(g.counters + tile, 1) == g.nsplit - 1;
+          mbar_arrive(dec_bar);  // also after a timeout, so the others do not wait in vain
+        }
+        const bool okd = mbar_wait_bounded(dec_bar, static_cast<uint32_t>(i) & 1u, g.err, 28);
+        if (!__all_sync(0xffffffffu, okd)) {
+          if (lane == 0) *abort_flag = 1;
+          break;
+        }
+        store = *split_flag != 0;
+        if (store) __threadfence();  // the other slices' partials, published before their increments
+      }
+      if (store) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_x32(t_row + 32 * c, r);
+          tmem_ld_wait();
+          float v[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)  // row `lane`: 64 bytes
-          *reinterpret_cast<uint4*>(st + lane * 64 + 16 * j) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&map_c, stage0 + static_cast<uint32_t>(ob * S::kOutBytes), n0 + 32 * c, m0 + 32 * q);
-          bulk_commit();
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          for (int o = 0; o < g.nsplit; ++o) {
+            if (o == split) continue;
+            const float4* other = reinterpret_cast<const float4*>(
+                g.partial + ((static_cast<int64_t>(tile) * g.nsplit + o) * kGBM + row) * BN + 32 * c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 p = __ldcg(other + j);
+              v[4 * j] += p.x, v[4 * j + 1] += p.y, v[4 * j + 2] += p.z, v[4 * j + 3] += p.w;
+            }
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const __nv_bfloat162 bv = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+            w[j] = *reinterpret_cast<const uint32_t*>(&bv);
+          }
+          if (lane == 0) bulk_wait_read<1>();  // the store that last read staging tile `ob` is done with it
+          __syncwarp();
+          unsigned char* st = stage0_ptr + ob * S::kOutBytes;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)  // row `lane`: 64 bytes
+            *reinterpret_cast<uint4*>(st + lane * 64 + 16 * j) =
+                make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_c, stage0 + static_cast<uint32_t>(ob * S::kOutBytes), n0 + 32 * c, m0 + 32 * q);
+            bulk_commit();
+          }
+          ob ^= 1;
         }
-        ob ^= 1;
       }
       tcgen05_fence_before();
       __syncwarp();
@@ -276,8 +352,8 @@ bool bf16_map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
 }
 
 template <int BN, int STAGES>
-cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int num_sms,
-                        int* err, cudaStream_t st) {
+cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int nsplit,
+                        void* ws, int num_sms, int* err, cudaStream_t st) {
   using S = GemmSmem<BN, STAGES>;
   CUtensorMap ma, mb, mc;
   if (!bf16_map2(&ma, A, static_cast<uint64_t>(K), static_cast<uint64_t>(M), kGBK, kGBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
@@ -286,50 +362,88 @@ cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_
     return cudaErrorInvalidValue;
   GemmArgs g;
   const int64_t tm = (M + kGBM - 1) / kGBM, tn = (N + BN - 1) / BN, kc = (K + kGBK - 1) / kGBK;
-  if (tm * tn > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  const int64_t units = tm * tn * nsplit;
+  if (units > 0x7fffffff) return cudaErrorInvalidConfiguration;
   g.tiles_m = static_cast<int>(tm);
   g.tiles_n = static_cast<int>(tn);
   g.k_chunks = static_cast<int>(kc);
   g.group_m = static_cast<int>(tm < 16 ? tm : 16);
+  g.nsplit = nsplit;
+  g.partial = nullptr;
+  g.counters = nullptr;
   g.err = err;
+  if (nsplit > 1) {
+    if (!ws) return cudaErrorInvalidValue;
+    g.partial = static_cast<float*>(ws);
+    g.counters = reinterpret_cast<int*>(static_cast<char*>(ws) + static_cast<size_t>(tm * tn * nsplit) * kGBM * BN * 4);
+    cudaError_t e = cudaMemsetAsync(g.counters, 0, static_cast<size_t>(tm * tn) * sizeof(int), st);
+    if (e != cudaSuccess) return e;
+  }
   const int smem = S::kTotal + 1024;
   auto kern = gemm_bf16_tn_kernel<BN, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const int64_t tiles = tm * tn;
-  const unsigned grid = static_cast<unsigned>(tiles < num_sms ? tiles : num_sms);
+  const unsigned grid = static_cast<unsigned>(units < num_sms ? units : num_sms);
   kern<<<grid, kGThreads, smem, st>>>(ma, mb, mc, g);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-int gemm_choose_bn(int64_t M, int64_t N, int num_sms) {
-  // Waves of tiles per SM x tile width, the 160-wide tile charged 10% more per
-  // column for its lower FLOP-per-byte (measured on B200: 128-wide tiles ran
-  // at half the rate of 256-wide ones, so they are not offered). 160 wins
-  // where 256-wide tiles leave most of a last wave idle (out_proj at 2048
-  // tokens: 160 tiles on 148 SMs).
-  const int64_t tm = (M + kGBM - 1) / kGBM;
-  const int64_t w256 = (tm * ((N + 255) / 256) + num_sms - 1) / num_sms;
-  const int64_t w160 = (tm * ((N + 159) / 160) + num_sms - 1) / num_sms;
-  return 11 * w160 * 160 < 10 * w256 * 256 ? 160 : 256;
+int gemm_choose_bn(int64_t /*M*/, int64_t /*N*/, int /*num_sms*/) {
+  // 256 columns: measured on B200, narrower tiles (160, 128) ran at 0.5 - 0.9
+  // of its rate on every projection shape, even where they left fewer SMs idle
+  // in the last wave (they read more operand bytes per FLOP).
+  return 256;
 }
 
-cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int bn,
-                         int num_sms, int* err, cudaStream_t st) {
+int gemm_choose_split(int64_t M, int64_t N, int64_t K, int num_sms) {
+  // K slices per tile when whole tiles would leave most of a last wave idle:
+  // minimise waves / slices, each extra slice charged 4% for its fp32 partial
+  // (written once, read once by the slice that finishes the tile); at least 8
+  // K chunks per slice. out_proj at 2048 tokens: 160 tiles on 148 SMs -> 4
+  // slices (5 waves of quarter tiles instead of 2 of whole ones).
+  if (num_sms <= 0) num_sms = 148;
+  const int64_t tiles = ((M + kGBM - 1) / kGBM) * ((N + 255) / 256), kc = (K + kGBK - 1) / kGBK;
+  int best = 1;
+  double best_cost = static_cast<double>((tiles + num_sms - 1) / num_sms);
+  for (int ns = 2; ns <= 4 && kc / ns >= 8; ++ns) {
+    const double cost = static_cast<double>((tiles * ns + num_sms - 1) / num_sms) / ns * (1.0 + 0.04 * ns);
+    if (cost < best_cost) best = ns, best_cost = cost;
+  }
+  return best;
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  const int ns = gemm_choose_split(M, N, K, num_sms);
+  if (ns == 1) return 0;
+  const int64_t tiles = ((M + kGBM - 1) / kGBM) * ((N + 255) / 256);
+  return static_cast<size_t>(tiles * ns) * kGBM * 256 * 4 + static_cast<size_t>(tiles) * sizeof(int);
+}
+
+cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* ws,
+                         size_t ws_bytes, int num_sms, int* err, cudaStream_t st) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0 || N % 8 != 0) return cudaErrorInvalidValue;
   if (num_sms <= 0) num_sms = 148;
-  if (bn == 0) bn = SSM_GEMM_FORCE_BN ? SSM_GEMM_FORCE_BN : gemm_choose_bn(M, N, num_sms);
-  if (bn == 256) return launch_gemm<256, 4>(A, B, C, M, N, K, num_sms, err, st);
-  if (bn == 160) return launch_gemm<160, 5>(A, B, C, M, N, K, num_sms, err, st);
+  const int bn = SSM_GEMM_FORCE_BN ? SSM_GEMM_FORCE_BN : gemm_choose_bn(M, N, num_sms);
+  int ns = gemm_choose_split(M, N, K, num_sms);
+  if (ns > 1 && (!ws || ws_bytes < gemm_workspace_bytes(M, N, K, num_sms))) return cudaErrorInvalidValue;
+  if (bn == 256) return launch_gemm<256, 4>(A, B, C, M, N, K, ns, ws, num_sms, err, st);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace ssm
 
+extern "C" size_t ssm_proj_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();  // no device: the default SM count
+  return ssm::gemm_workspace_bytes(M, N, K, sms);
+}
+
 extern "C" ssm_status ssm_proj_gemm(const void* A, const void* W, void* C, int64_t M, int64_t N, int64_t K,
-                                    void* stream) {
+                                    void* workspace, size_t workspace_bytes, void* stream) {
   using ssm::fail;
   if (M <= 0 || N <= 0 || K <= 0) return fail(SSM_ERR_INVALID_ARG, "M, N, K must be positive");
   if (K % 8 != 0 || N % 8 != 0) return fail(SSM_ERR_INVALID_ARG, "K and N must be multiples of 8");
@@ -340,11 +454,15 @@ extern "C" ssm_status ssm_proj_gemm(const void* A, const void* W, void* C, int64
   for (int i = 0; i < 3; ++i)
     if (!p[i] || !ssm::aligned(p[i], 16)) return fail(SSM_ERR_INVALID_ARG, "%s is NULL or not 16-byte aligned", names[i]);
   if (C == A || C == W) return fail(SSM_ERR_INVALID_ARG, "C must not alias A or W");
+  const size_t need = ssm_proj_gemm_workspace_bytes(M, N, K);
+  if (need && (!workspace || !ssm::aligned(workspace, 256) || workspace_bytes < need))
+    return fail(SSM_ERR_INVALID_ARG, "workspace: need %zu bytes, 256-byte aligned (got %zu)", need, workspace_bytes);
   int* err = ssm::device_error_ptr();
   if (!err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const cudaError_t e = ssm::gemm_bf16_tn(A, W, C, M, N, K, 0, sms, err, static_cast<cudaStream_t>(stream));
+  const cudaError_t e =
+      ssm::gemm_bf16_tn(A, W, C, M, N, K, workspace, workspace_bytes, sms, err, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(SSM_ERR_CUDA, "projection GEMM launch: %s", cudaGetErrorString(e));
   return fail(SSM_OK, "");
 }

@@ -68,24 +68,30 @@ constexpr bool kScoresFirst = SSM_SSD_SCORES_FIRST;  // accumulator 0 (intra-chu
 template <int CS, int DS>
 struct SsdSmem {
   static_assert(DS == 64 || DS == 128, "state dim 64 or 128");
-  static_assert(CS == 64 || CS == 128, "chunk 64 or 128");
-  static constexpr int kNC = kCs / CS;             // chunks per CTA
-  static constexpr int kNA = DS / 64;              // 64-column atoms across the state dim
-  static constexpr int kAtomRows128 = kCs * 128;   // one 64-column atom of a 128-row tile
-  static constexpr int kAtomRows64 = kHd * 128;    // one 64-column atom of a 64-row tile
-  static constexpr int kCb = 0;                    // cb -> scores (A of MMA 1) -> out tile
-  static constexpr int kC = 2 * kAtomRows128;      // C (A of MMA 2)
-  static constexpr int kX = kC + kNA * kAtomRows128;  // x [s][p] (B of MMA 1, MN-major)
-  static constexpr int kPrev = kX + kAtomRows128;  // prev_states [chunk][p][n] (B of MMA 2, K-major)
+  static_assert(CS == 64 || CS == 128 || CS == 256, "chunk 64, 128 or 256");
+  static constexpr int kNC = CS < kCs ? kCs / CS : 1;  // chunks per CTA (stacked on the tile diagonal)
+  static constexpr int kHalves = CS > kCs ? CS / kCs : 1;  // CTAs per chunk (128-row halves)
+  static constexpr int kKS = CS > kCs ? CS : kCs;      // most score columns = rows of x = K of the intra term
+  static constexpr int kNA = DS / 64;                  // 64-column atoms across the state dim
+  static constexpr int kAtomRows128 = kCs * 128;       // one 64-column atom of a 128-row tile
+  static constexpr int kAtomRows64 = kHd * 128;        // one 64-column atom of a 64-row tile
+  static constexpr int kCb = 0;                        // cb -> scores [128][kKS] (A of MMA 1) -> out tile
+  static constexpr int kC = kCb + (kKS / 64) * kAtomRows128;  // C [128][DS] (A of MMA 2)
+  static constexpr int kX = kC + kNA * kAtomRows128;   // x [kKS][p] (B of MMA 1, MN-major)
+  static constexpr int kPrev = kX + kKS * 128;         // prev_states [chunk][p][n] (B of MMA 2, K-major)
   static constexpr int kDA = kPrev + kNC * kNA * kAtomRows64;
-  static constexpr int kDt = kDA + kCs * 4;
-  static constexpr int kF = kDt + kCs * 4;
-  static constexpr int kBar = kF + kCs * 4;        // full_state, full_scores, done
+  static constexpr int kDt = kDA + kKS * 4;
+  static constexpr int kF = kDt + kKS * 4;
+  static constexpr int kBar = kF + kKS * 4;            // full_state, full_scores, done
   static constexpr int kTmemSlot = kBar + 24;
   static constexpr int kTotal = kTmemSlot + 16;
   static constexpr uint32_t kTxState = static_cast<uint32_t>(kNA * (kAtomRows128 + kNC * kAtomRows64));  // C, prev
-  // cb: the chunks' [CS][CS] diagonal blocks of the [128][128] score tile; x
-  static constexpr uint32_t kTxScores = static_cast<uint32_t>(kNC * CS * CS * 2 + kAtomRows128);
+  // cb and x of a CTA whose score tile is ks columns wide (ks = 128, or 256 for
+  // the second half of a 256-chunk): stacked chunks load their [CS][CS]
+  // diagonal blocks, otherwise 128 rows x ks columns; x has ks rows.
+  static __host__ __device__ constexpr uint32_t tx_scores(int ks) {
+    return static_cast<uint32_t>((kNC > 1 ? kNC * CS * CS * 2 : kCs * ks * 2) + ks * 128);
+  }
   static constexpr uint32_t kTmemCols = kNC == 1 ? 128u : 256u;  // intra + one carried-state term per chunk
   static_assert(kC % 1024 == 0 && kX % 1024 == 0 && kPrev % 1024 == 0, "swizzled tiles need 1 KB");
 };
@@ -140,8 +146,14 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   const uint32_t sb = smem_u32(smem);
   const int tid = threadIdx.x;
   const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0);
-  const int l = tid & (kCs - 1), at = tid >> 7;  // this thread's row and 64-column atom
-  const int h = blockIdx.x, c = blockIdx.y * NC, b = blockIdx.z;  // first chunk of this CTA
+  const int l = tid & (kCs - 1), at = tid >> 7;  // this thread's tile row and first 64-column atom
+  const int h = blockIdx.x, b = blockIdx.z;
+  // This CTA: chunk c (the first of NC stacked ones), rows r0 .. r0 + 127 of
+  // it (r0 > 0 only for the second half of a 256-chunk), ks score columns.
+  const int c = S::kHalves > 1 ? static_cast<int>(blockIdx.y) / S::kHalves : static_cast<int>(blockIdx.y) * NC;
+  const int r0 = S::kHalves > 1 ? (static_cast<int>(blockIdx.y) % S::kHalves) * kCs : 0;
+  const int ks = r0 + kCs;
+  const int64_t t_chunk = static_cast<int64_t>(c) * CS;  // first token of chunk c
   const int g = static_cast<int>(h / (a.nheads / a.ngroups));
   const uint32_t full_state = sb + S::kBar, full_scores = sb + S::kBar + 8, done = sb + S::kBar + 16;
   if (tid == 0) {
@@ -153,16 +165,17 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_c);
     prefetch_tensormap(&map_prev);
-    // A second chunk past the last one (odd chunk count) reads zeros or a
-    // neighbouring sequence's chunk; its rows lie past L and are never stored.
+    // A second stacked chunk past the last one (odd chunk count) reads zeros
+    // or a neighbouring sequence's chunk; its rows lie past L and are never stored.
     const int64_t zc0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g;
     const int64_t zp0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h;
     mbar_arrive_expect_tx(full_state, S::kTxState);
-    mbar_arrive_expect_tx(full_scores, S::kTxScores);
+    mbar_arrive_expect_tx(full_scores, S::tx_scores(ks));
     auto load_state = [&] {
 #pragma unroll
       for (int t = 0; t < S::kNA; ++t) {
-        tma_load_4d(sb + S::kC + t * S::kAtomRows128, &map_c, 64 * t, g, c * CS, b, full_state);
+        tma_load_4d(sb + S::kC + t * S::kAtomRows128, &map_c, 64 * t, g, static_cast<int>(t_chunk + r0), b,
+                    full_state);
 #pragma unroll
         for (int k = 0; k < NC; ++k)
           tma_load_3d(sb + S::kPrev + (k * S::kNA + t) * S::kAtomRows64, &map_prev, 64 * t, 0,
@@ -171,17 +184,17 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     };
     auto load_scores = [&] {
       if constexpr (NC == 1) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-          tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, 64 * t, 0, static_cast<int>(zc0), full_scores);
+        for (int t = 0; t < ks / 64; ++t)  // rows r0 .. r0 + 127, columns 64 t ..
+          tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, 64 * t, r0, static_cast<int>(zc0), full_scores);
       } else {
-        // chunk k's [64][64] block on the diagonal: atom k, rows 64 k ..
+        // chunk k's [CS][CS] block on the diagonal: atom k, rows CS k ..
 #pragma unroll
         for (int k = 0; k < NC; ++k)
           tma_load_3d(sb + S::kCb + k * S::kAtomRows128 + k * CS * 128, &map_cb, 0, 0,
                       static_cast<int>(zc0 + k * a.ngroups), full_scores);
       }
-      tma_load_4d(sb + S::kX, &map_x, 0, h, c * CS, b, full_scores);
+      for (int t = 0; t < ks / kCs; ++t)  // x rows 128 t .. of the chunk
+        tma_load_4d(sb + S::kX + t * kCs * 128, &map_x, 0, h, static_cast<int>(t_chunk + kCs * t), b, full_scores);
     };
     if (kScoresFirst) {
       load_scores();
@@ -198,11 +211,13 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   float* sdA = reinterpret_cast<float*>(smem + S::kDA);
   float* sdt = reinterpret_cast<float*>(smem + S::kDt);
   float* F = reinterpret_cast<float*>(smem + S::kF);
-  if (tid < kCs) {  // the CTA's chunks are consecutive in [b][H][nc][CS]
+  {  // the score columns' dA and dt: positions 0 .. ks - 1 from chunk c on ([b][H][nc][CS], chunks adjacent)
     const int64_t row = ((static_cast<int64_t>(b) * a.nheads + h) * a.nchunks + c) * CS;
-    const bool in = c + tid / CS < a.nchunks;
-    sdA[tid] = in ? a.dA[row + tid] : 0.0f;
-    sdt[tid] = in ? a.dt[row + tid] : 0.0f;
+    for (int i = tid; i < ks; i += kSsdThreads) {
+      const bool in = c + i / CS < a.nchunks;
+      sdA[i] = in ? a.dA[row + i] : 0.0f;
+      sdt[i] = in ? a.dt[row + i] : 0.0f;
+    }
   }
   const float Dh = a.D ? a.D[h] : 0.0f;
   tcgen05_fence_before();
@@ -210,8 +225,8 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   tcgen05_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
   // Accumulators: the intra-chunk term at column 0, the carried-state term of
-  // chunk k at 64 (k + 1) (C x prev_states(k)^T over all 128 rows; rows of
-  // chunk k read it).
+  // stacked chunk k at 64 (k + 1) (C x prev_states(k)^T over all 128 rows;
+  // rows of chunk k read it).
   const uint32_t acc_intra = tmem;
   auto state_mmas = [&] {
 #pragma unroll
@@ -229,41 +244,49 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     tcgen05_fence_after();
     state_mmas();
   }
-  if (tid < kCs) F[tid] = ex2_approx((sdA[tid | 7] - sdA[tid]) * kLog2e) * sdt[tid];
-  const float dAl = sdA[l];
+  for (int i = tid; i < ks; i += kSsdThreads) F[i] = ex2_approx((sdA[i | 7] - sdA[i]) * kLog2e) * sdt[i];
+  const int lg = r0 + l;  // this thread's row within its chunk pair / chunk
+  const float dAl = sdA[lg];
   mbar_wait_bounded(full_scores, 0u, a.err, 8);
   __syncthreads();  // F complete
 
-  // 3. This thread's atom of row l of the cb tile -> scores (in place). A
-  //    warp's 32 rows lie in one chunk, starting at column warp_min_s.
-  const int warp_max_l = 32 * (warp & 3) + 31;
-  const int warp_min_s = (32 * (warp & 3)) & ~(CS - 1);
+  // 3. Row l of the cb tile -> scores (in place), atoms at, at + 2, .. of the
+  //    ks columns. A warp's 32 rows lie in one chunk, starting at column warp_min_s.
+  const int warp_max_l = r0 + 32 * (warp & 3) + 31;
+  const int warp_min_s = CS < kCs ? (32 * (warp & 3)) & ~(CS - 1) : 0;
+  for (int aa = at; aa < ks / 64; aa += 2) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int s0 = 64 * at + 8 * j;
-    uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
-    if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
-      *p = make_uint4(0u, 0u, 0u, 0u);
-      continue;
+    for (int j = 0; j < 8; ++j) {
+      const int s0 = 64 * aa + 8 * j;
+      uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + aa * S::kAtomRows128 + sw128(l, j));
+      if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
+        *p = make_uint4(0u, 0u, 0u, 0u);
+        continue;
+      }
+      float f[8];
+      unpack8(*p, f);
+      if (s0 + 7 <= lg) {  // wholly at or below the diagonal: row factor x column factor
+        const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
+      } else if (s0 <= lg) {  // the diagonal group
+        // The two-factor form while the group's own decay range stays well
+        // inside fp32, else each decay on its own.
+        if (sdA[s0] - sdA[s0 + 7] < 80.0f) {
+          const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) f[q] = 0.0f;
+      }
+      *p = pack8(f);
     }
-    float f[8];
-    unpack8(*p, f);
-    // The two-factor form also serves the diagonal group while the group's own
-    // decay range stays well inside fp32 (the same for every row of the warp).
-    const bool narrow = sdA[s0] - sdA[s0 + 7] < 80.0f;
-    if (s0 + 7 <= l || (narrow && s0 <= l)) {  // row factor x column factor
-      const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) f[q] = s0 + q <= l ? f[q] * e * F[s0 + q] : 0.0f;
-    } else if (s0 <= l) {  // the diagonal group of a strongly decaying chunk: each decay on its own
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        f[q] = s0 + q <= l ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) f[q] = 0.0f;
-    }
-    *p = pack8(f);
   }
   fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
   __syncthreads();
@@ -271,8 +294,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   // 4. Intra-chunk term: scores[l][s] x x[s][p], s in steps of 16 rows of x; one commit for both.
   if (tid == 0) {
     tcgen05_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < kCs / 16; ++kk)
+    for (int kk = 0; kk < ks / 16; ++kk)
       umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
                   umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), kk > 0);
     if (kScoresFirst) {  // carried-state term last: its operands were loaded second
@@ -290,23 +312,23 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   {
     const int q4 = warp & 3, col0 = 32 * (warp >> 2);
     const int row = 32 * q4 + (tid & 31);
-    const float el = ex2_approx(sdA[row] * kLog2e);
-    const uint32_t acc_state = tmem + kHd * (1 + (32 * q4) / CS);  // this warp's chunk
+    const float el = ex2_approx(sdA[r0 + row] * kLog2e);
+    const uint32_t acc_state = tmem + kHd * (1 + (CS < kCs ? (32 * q4) / CS : 0));  // this warp's chunk
 #pragma unroll
     for (int jj = 0; jj < 2; ++jj) {
-      uint32_t r0[16], r1[16];
+      uint32_t r0v[16], r1v[16];
       const uint32_t lane_col = (static_cast<uint32_t>(32 * q4) << 16) + col0 + 16 * jj;
-      tmem_ld_x16(acc_intra + lane_col, r0);
-      tmem_ld_x16(acc_state + lane_col, r1);
+      tmem_ld_x16(acc_intra + lane_col, r0v);
+      tmem_ld_x16(acc_state + lane_col, r1v);
       tmem_ld_wait();
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const int j = (col0 + 16 * jj) / 8 + half;  // 16-byte chunk of the row: p = 8 j .. 8 j + 7
         float xv[8], o[8];
-        unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(row, j)), xv);
+        unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(r0 + row, j)), xv);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          o[q] = fmaf(Dh, xv[q], fmaf(el, __uint_as_float(r1[8 * half + q]), __uint_as_float(r0[8 * half + q])));
+          o[q] = fmaf(Dh, xv[q], fmaf(el, __uint_as_float(r1v[8 * half + q]), __uint_as_float(r0v[8 * half + q])));
         *reinterpret_cast<uint4*>(smem + S::kCb + sw128(row, j)) = pack8(o);
       }
     }
@@ -314,7 +336,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   fence_proxy_async_smem();
   __syncthreads();
   if (tid == 0) {
-    tma_store_4d(&map_out, sb + S::kCb, 0, h, c * CS, b);
+    tma_store_4d(&map_out, sb + S::kCb, 0, h, static_cast<int>(t_chunk + r0), b);
     bulk_commit();
     bulk_wait_read<0>();  // the tile stays in shared memory until the store has read it
   }
@@ -348,7 +370,7 @@ cudaError_t launch_ssd(int64_t H, int64_t nc, int64_t b, const CUtensorMap& mcb,
   auto kern = ssd_chunk_scan_kernel<CS, DS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
-  const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>((nc + S::kNC - 1) / S::kNC),
+  const dim3 grid(static_cast<unsigned>(H), static_cast<unsigned>((nc + S::kNC - 1) / S::kNC * S::kHalves),
                   static_cast<unsigned>(b));
   kern<<<grid, kSsdThreads, smem, st>>>(mcb, mx, mc, mp, mo, a);
   return cudaGetLastError();
@@ -364,15 +386,15 @@ extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* c
   if (!dims) return fail(SSM_ERR_INVALID_ARG, "dims is NULL");
   const int64_t b = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim, G = dims->ngroups;
   const int64_t N = dims->dstate, cs = dims->chunk_size;
-  if ((cs != 64 && cs != 128) || P != ssm::kHd || (N != 64 && N != 128))
+  if ((cs != 64 && cs != 128 && cs != 256) || P != ssm::kHd || (N != 64 && N != 128))
     return fail(SSM_ERR_UNSUPPORTED,
-                "chunk_size %lld, headdim %lld, dstate %lld: the built shapes are chunk 64 or 128, headdim 64, "
+                "chunk_size %lld, headdim %lld, dstate %lld: the built shapes are chunk 64, 128 or 256, headdim 64, "
                 "dstate 64 or 128",
                 (long long)cs, (long long)P, (long long)N);
   if (b <= 0 || b > 65535 || H <= 0 || H > 0x7fffffff || G <= 0 || H % G != 0)
     return fail(SSM_ERR_INVALID_ARG, "need 0 < batch <= 65535, nheads > 0 and nheads a multiple of ngroups");
-  if (L <= 0 || L % cs != 0 || L / cs > 65535)
-    return fail(SSM_ERR_INVALID_ARG, "seqlen must be a positive multiple of chunk_size, at most 65535 chunks");
+  if (L <= 0 || L % cs != 0 || L / cs > 32767)
+    return fail(SSM_ERR_INVALID_ARG, "seqlen must be a positive multiple of chunk_size, at most 32767 chunks");
   const void* ptrs[8] = {cb, x, dt, dA_cumsum, C, prev_states, out, D};
   const char* names[8] = {"cb", "x", "dt", "dA_cumsum", "C", "prev_states", "out", "D"};
   for (int i = 0; i < 8; ++i) {
@@ -386,7 +408,7 @@ extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* c
   const uint64_t e2 = 2;
   const bool ok =
       ssm::bf16_map(&mcb, 3, cb, {uint64_t(cs), uint64_t(cs), uint64_t(b * nc * G)}, {cs * e2, cs * cs * e2},
-                    {64, uint32_t(cs), 1}) &&
+                    {64, uint32_t(cs < 128 ? cs : 128), 1}) &&
       ssm::bf16_map(&mx, 4, x, {uint64_t(P), uint64_t(H), uint64_t(L), uint64_t(b)},
                     {P * e2, H * P * e2, L * H * P * e2}, {64, 1, 128, 1}) &&
       ssm::bf16_map(&mc, 4, C, {uint64_t(N), uint64_t(G), uint64_t(L), uint64_t(b)},
@@ -400,7 +422,10 @@ extern "C" ssm_status ssm_ssd_chunk_scan(const ssm_ssd_dims* dims, const void* c
   if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t err;
-  if (cs == 128)
+  if (cs == 256)
+    err = N == 128 ? ssm::launch_ssd<256, 128>(H, nc, b, mcb, mx, mc, mp, mo, a, st)
+                   : ssm::launch_ssd<256, 64>(H, nc, b, mcb, mx, mc, mp, mo, a, st);
+  else if (cs == 128)
     err = N == 128 ? ssm::launch_ssd<128, 128>(H, nc, b, mcb, mx, mc, mp, mo, a, st)
                    : ssm::launch_ssd<128, 64>(H, nc, b, mcb, mx, mc, mp, mo, a, st);
   else

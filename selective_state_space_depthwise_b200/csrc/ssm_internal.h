@@ -53,10 +53,13 @@ cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillS
 cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStream_t st);
 
 // C[M][N] = A[M][K] . B[N][K]^T, bf16 operands and output, fp32 accumulation,
-// on the tensor cores (gemm.cu). bn: output tile width 256 or 128, 0 = chosen
-// from the shape. K and N multiples of 8, pointers 16-byte aligned.
-cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, int bn, int num_sms,
-                         int* err, cudaStream_t st);
+// on the tensor cores (gemm.cu). K and N multiples of 8, pointers 16-byte
+// aligned. ws: gemm_workspace_bytes() of device scratch (split-K partials and
+// tile counters; 0 bytes when the shape runs unsplit).
+cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* ws,
+                         size_t ws_bytes, int num_sms, int* err, cudaStream_t st);
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+int gemm_choose_split(int64_t M, int64_t N, int64_t K, int num_sms);
 int gemm_choose_bn(int64_t M, int64_t N, int num_sms);
 
 // Shared by the entry points (ssm_api.cu): validation with the ABI's

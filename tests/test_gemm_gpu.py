@@ -6,8 +6,10 @@ Reference: the products of the stored bf16 values summed in float64 on the
 CPU, rounded once to bf16. The kernel accumulates the same products in fp32
 (K <= 7680 terms: relative error ~1e-6, far below a bf16 step), so the two
 roundings agree except for rare one-step flips: relative L2 <= 1e-3 is asked.
-Shapes cover ragged M, N and K tails, both output tile widths (the launch
-picks 160 or 256 columns from the shape) and the block's layer shapes.
+Shapes cover ragged M, N and K tails, more tiles than SMs (each persistent
+CTA taking several, alternating its two accumulators), split K (few tiles,
+long K: fp32 partials added by the slice that finishes each tile) and the
+block's layer shapes (out_proj at 2048 tokens runs split).
 """
 import numpy as np
 import pytest
@@ -43,16 +45,6 @@ def rel_l2(got, want):
     return float(np.linalg.norm(got - want) / np.linalg.norm(want))
 
 
-def bn_of(M, N):
-    """The tile width the launch picks (mirrors gemm_choose_bn): waves x width,
-    the 160-wide tile charged 10% more per column; ties go to 256."""
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    tm = -(-M // 128)
-    w256 = -(-(tm * -(-N // 256)) // sms)
-    w160 = -(-(tm * -(-N // 160)) // sms)
-    return 160 if 11 * w160 * 160 < 10 * w256 * 256 else 256
-
-
 SHAPES = [(1, 8, 8), (100, 136, 72), (300, 520, 200), (129, 264, 64), (257, 1000, 1032)]
 
 
@@ -63,28 +55,40 @@ def test_gemm_ragged_shapes(shape):
     C = api.proj_gemm(A.cuda(), W.cuda())
     torch.cuda.synchronize()
     e = rel_l2(C.double().cpu().numpy(), reference(A, W))
-    print(f"gemm {M}x{N}x{K} (tile width {bn_of(M, N)}): rel-L2 {e:.2e}")
+    print(f"gemm {M}x{N}x{K}: rel-L2 {e:.2e}")
     assert e <= TOL_GEMM
 
 
-def test_gemm_both_tile_widths():
-    """One shape the launch tiles 256 columns wide and one it tiles 128 wide,
-    each with more tiles than SMs (several tiles per persistent CTA, both TMEM
-    accumulators in turn)."""
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    # 4 row tiles x sms/4 column tiles of 256 fill the SMs once (256 wide);
-    # 5 row tiles x 3 column tiles (N = 408) tile 160 wide.
-    cases = [(512, 256 * (sms // 4), 192), (640, 408, 256)]
-    widths = set()
-    for M, N, K in cases:
-        widths.add(bn_of(M, N))
-        A, W = operands(M, N, K, seed=N)
-        C = api.proj_gemm(A.cuda(), W.cuda())
+def test_gemm_many_tiles_per_cta():
+    """More output tiles than SMs: each persistent CTA takes several tiles, so
+    both TMEM accumulators alternate and the grouped raster wraps (8 row
+    blocks x 40 column blocks)."""
+    M, N, K = 1000, 256 * 40 - 24, 200
+    A, W = operands(M, N, K, seed=N)
+    C = api.proj_gemm(A.cuda(), W.cuda())
+    torch.cuda.synchronize()
+    e = rel_l2(C.double().cpu().numpy(), reference(A, W))
+    print(f"gemm {M}x{N}x{K}: rel-L2 {e:.2e}")
+    assert e <= TOL_GEMM
+
+
+@pytest.mark.parametrize("shape", [(256, 512, 4096), (200, 264, 1000)], ids=["4_slices", "2_slices_ragged"])
+def test_gemm_split_k(shape):
+    """Few output tiles and a long K: the launch splits K into slices whose
+    fp32 partials the last-finishing slice adds up. Every element against the
+    reference, twice with the same workspace (its tile counters are zeroed by
+    each call)."""
+    M, N, K = shape
+    assert api.proj_gemm_workspace_bytes(M, N, K) > 0  # this shape runs split
+    A, W = operands(M, N, K, seed=K)
+    ws = torch.empty(api.proj_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    want = reference(A, W)
+    for _ in range(2):
+        C = api.proj_gemm(A.cuda(), W.cuda(), workspace=ws)
         torch.cuda.synchronize()
-        e = rel_l2(C.double().cpu().numpy(), reference(A, W))
-        print(f"gemm {M}x{N}x{K} (tile width {bn_of(M, N)}): rel-L2 {e:.2e}")
+        e = rel_l2(C.double().cpu().numpy(), want)
+        print(f"gemm split K {M}x{N}x{K}: rel-L2 {e:.2e}")
         assert e <= TOL_GEMM
-    assert widths == {160, 256}
 
 
 @pytest.mark.parametrize("which", ["in_proj", "out_proj"])

@@ -106,6 +106,21 @@ def test_ssd_chunk_64(dstate, seqlen):
     assert e <= TOL_SSD
 
 
+@pytest.mark.parametrize("dstate", [64, 128])
+def test_ssd_chunk_256(dstate):
+    """Chunk length 256: each chunk is two CTAs of 128 rows, the second with
+    a 256-wide intra-chunk contraction. Every output against the oracle."""
+    spec = dict(batch=2, seqlen=768, nheads=4, headdim=64, ngroups=2, dstate=dstate, chunk_size=256,
+                seed=53 + dstate)
+    inp = W.make_ssd_inputs(spec, device="cuda")
+    out = run(inp).double().cpu().numpy()
+    f = lambda t: t.detach().double().cpu().numpy()  # noqa: E731
+    want = oracle.ssd_chunk_scan(*(f(inp[k]) for k in ARGS))
+    e = rel_l2(out, want)
+    print(f"ssd chunk 256, dstate {dstate}: rel-L2 {e:.2e}")
+    assert e <= TOL_SSD
+
+
 def test_ssd_full_size_every_chunk():
     """b=8, L=4096, 80 heads: every (sequence, chunk) pair, every head and
     position, against the oracle one sequence at a time; the rel-L2 is pooled
