@@ -74,10 +74,20 @@ struct GemmArgs {
   int tiles_m, tiles_n, k_chunks;
   int group_m;      // row blocks per raster group
   int nsplit;       // K slices per tile (work units = tiles x nsplit)
-  float* partial;   // nsplit > 1: [tiles][nsplit][128][BN] fp32 partial tiles
+  float* partial;   // nsplit > 1: [tiles][nsplit] fp32 partial tiles of 128 x BN, each stored
+                    // [warp quarter][32-column chunk][float4 slot][lane] so every warp
+                    // instruction moves 512 contiguous bytes
   int* counters;    // nsplit > 1: [tiles], zero on entry: slices of each tile finished
   int* err;
 };
+
+// Float4 index of (tile, slice, warp quarter q, 32-column chunk c, slot j,
+// lane) in the split-K partials: a warp's 32 lanes are adjacent.
+__device__ __forceinline__ int64_t partial_index(const GemmArgs& g, int tile, int split, int q, int c, int j,
+                                                int lane) {
+  constexpr int kChunks = 256 / 32;  // BN / 32 at the only built width
+  return ((((static_cast<int64_t>(tile) * g.nsplit + split) * 4 + q) * kChunks + c) * 8 + j) * 32 + lane;
+}
 
 // Work unit -> its tile and K-chunk range: the nsplit slices of a tile are
 // consecutive units, so consecutive CTAs run them at the same time.
@@ -110,6 +120,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     gemm_bf16_tn_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                         const __grid_constant__ CUtensorMap map_c, const GemmArgs g) {
   using S = GemmSmem<BN, STAGES>;
+  static_assert(BN == 256, "the split-K partial layout (partial_index) is built for 256-wide tiles");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(smem);
@@ -241,12 +252,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
       }
       tcgen05_fence_after();
       const uint32_t t_row = tmem + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf * BN);
-      const int row = 32 * q + lane;  // this thread's row of the tile
-      bool store = true;              // this unit writes the bf16 tile
+      bool store = true;  // this unit writes the bf16 tile
       if (g.nsplit > 1) {
         // Every slice publishes its fp32 partial; the slice that finishes the
         // tile last adds the others to its own and writes the output.
-        float* mine = g.partial + ((static_cast<int64_t>(tile) * g.nsplit + split) * kGBM + row) * BN;
+        float4* mine = reinterpret_cast<float4*>(g.partial) + partial_index(g, tile, split, q, 0, 0, lane);
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -254,9 +264,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            reinterpret_cast<float4*>(mine + 32 * c)[j] =
-                make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]), __uint_as_float(r[4 * j + 2]),
-                            __uint_as_float(r[4 * j + 3]));
+            mine[(c * 8 + j) * 32] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
         }
         // Handshake of the four epilogue warps on two mbarriers (bounded
         // waits, so a warp that left on an abort cannot strand the others):
@@ -289,11 +298,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           for (int o = 0; o < g.nsplit; ++o) {
             if (o == split) continue;
-            const float4* other = reinterpret_cast<const float4*>(
-                g.partial + ((static_cast<int64_t>(tile) * g.nsplit + o) * kGBM + row) * BN + 32 * c);
+            const float4* other = reinterpret_cast<const float4*>(g.partial) + partial_index(g, tile, o, q, c, 0, lane);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float4 p = __ldcg(other + j);
+              const float4 p = __ldcg(other + j * 32);
               v[4 * j] += p.x, v[4 * j + 1] += p.y, v[4 * j + 2] += p.z, v[4 * j + 3] += p.w;
             }
           }
