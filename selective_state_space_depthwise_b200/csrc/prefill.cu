@@ -44,9 +44,12 @@
 //
 // Kernels. 3: G = 4 with the register budget of three CTAs per SM; 4: G = 4
 // built for two CTAs per SM, whose larger register budget buys a deeper
-// schedule. (G = 2, 8 states per thread, executes ~13% fewer instructions per
-// channel-token but measured 1.28x slower at the long-context shape: with one
-// warp per SM sub-partition its dependency latencies are not hidden.)
+// schedule. Measured alternatives at the long-context shape: G = 2 (8 states
+// a thread) executes ~13% fewer instructions per channel-token but runs 1.28x
+// slower (one warp per SM sub-partition leaves dependency latencies exposed);
+// G = 8 (2 states a thread, 16 warps per SM) runs 1.36x slower: with two
+// states a thread the power path saves nothing, and the 16 per-state
+// exponentials and the B/C loads then saturate the shared MIO queue.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -107,17 +110,6 @@ struct PipeSmem {
 template <int KP>
 __device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const float* a2, float* h, const float* Bp,
                                             const float* Cp) {
-  if constexpr (KP == 1) {  // two states: 8-byte B and C loads
-    const float2 b = *reinterpret_cast<const float2*>(Bp);
-    const float2 c = *reinterpret_cast<const float2*>(Cp);
-    float x0, x1;
-    upk2(fmul2(dt2, pk2(a2[0], a2[1])), x0, x1);
-    const uint64_t hb = ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(h[0], h[1]), fmul2(inj2, pk2(b.x, b.y)));
-    upk2(hb, h[0], h[1]);
-    float lo, hi;
-    upk2(fmul2(pk2(c.x, c.y), hb), lo, hi);
-    return lo + hi;
-  }
   uint64_t acc = 0;
 #pragma unroll
   for (int q = 0; q < KP; q += 2) {
@@ -533,10 +525,6 @@ __global__ void __launch_bounds__(32 * G, MINB) prefill_pipe_kernel(const __grid
   constexpr bool SPLIT = split_barrier<MINB>();
   if constexpr (ZOH) {
     pipe_run<T, G, Path::kZoh, SPLIT>(maps, a);
-  } else if constexpr (G == 8) {
-    // Two states a thread: a power decay would cost as much as the two
-    // exponentials it replaces, so every channel takes the generic path.
-    pipe_run<T, G, Path::kGeneric, SPLIT>(maps, a);
   } else {
     const bool pw = a.decay_path == 0 && cta_has_power_decays<G>(a);
     if (pw)
@@ -618,13 +606,12 @@ template <typename T, bool ZOH>
 cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st) {
   if (sh.kernel == 3) return launch_pipe<T, 4, ZOH, 0>(a, st);
   if (sh.kernel == 4) return launch_pipe<T, 4, ZOH, 1>(a, st);
-  if (sh.kernel == 5) return launch_pipe<T, 8, ZOH, 2>(a, st);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool prefill_shape_supported(PrefillShape sh) { return sh.kernel >= 3 && sh.kernel <= 5; }
+bool prefill_shape_supported(PrefillShape sh) { return sh.kernel == 3 || sh.kernel == 4; }
 
 // Pipelined state slices; the register-rich build when the grid needs at most
 // two CTAs per SM.
