@@ -287,7 +287,7 @@ ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const voi
  *   workspace device scratch of ssm_block_workspace_bytes(dims) bytes,
  *             256-byte aligned. It holds the in_proj output (b L 2E bf16),
  *             B / C / dt_raw (b L 33 fp32), the gated core output
- *             (b L E bf16) and the projections' split-K scratch (see
+ *             (b L E bf16) and the projections' cut-tile scratch (see
  *             ssm_proj_gemm).
  *
  * Ordering and errors. Everything is enqueued on `stream`, with no host
@@ -323,15 +323,17 @@ size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
  *   A  [M, K] bf16, row-major;  W  [N, K] bf16, row-major;  C  [M, N] bf16
  * Device pointers, 16-byte aligned; K and N multiples of 8; 0 < M, N, K <=
  * 2^31; C must not alias A or W. fp32 accumulation, C rounded to bf16 (RNE).
- * One persistent kernel (tcgen05 MMAs into TMEM, TMA operand ring, TMA
- * stores) enqueued on `stream`, after a memset of the workspace's tile
- * counters when the shape runs split-K.
+ * One persistent kernel of CTA pairs (two-SM tcgen05 MMAs into TMEM, TMA
+ * operand rings, TMA stores) enqueued on `stream`, after a memset of the
+ * workspace's tile counters when some tile is cut between pairs.
  *   workspace  ssm_proj_gemm_workspace_bytes(M, N, K) bytes of device scratch,
- *              256-byte aligned, or NULL when that is 0. Shapes whose 128 x 256
- *              output tiles would leave most SMs idle in a last wave split K
- *              into up to 4 slices; the slices' fp32 partial tiles and a
- *              counter per tile live here. Calls that overlap on the GPU need
- *              separate workspaces.
+ *              256-byte aligned, or NULL when that is 0. Whole 256 x 256 output
+ *              tiles go round-robin to the pairs; the last one to two tiles a
+ *              pair are instead cut along K into equal runs, one per pair, and
+ *              the fp32 partials of the cut tiles (512 KB a pair) and a
+ *              counter per tile live here. The partials of a cut tile are
+ *              summed in a fixed order, so results do not depend on timing.
+ *              Calls that overlap on the GPU need separate workspaces.
  */
 size_t ssm_proj_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64_t N, int64_t K, void *workspace,
@@ -441,8 +443,11 @@ ssm_status ssm_segment_carry(const ssm_dims *dims, const ssm_weights *w, const f
  * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed;
  * SSM_ERR_DEVICE with the code in ssm_last_error() otherwise. Codes: 1 the
  * prefill's TMA ring, 3-6 the block's x_proj kernel, 7-9 the chunk scan's
- * operand and MMA waits, 11 the decode's state ring, SSM_SELFTEST_WAIT_CODE
- * the self-test below. Every kernel's waits give up after about 2 s. */
+ * operand and MMA waits, 11 the decode's state ring, 21-29 the projection
+ * GEMM (21 ring slot free, 22 accumulator free, 23 operands landed, 24
+ * accumulator full, 25 and 29 drains, 27-28 the cut-tile handshake),
+ * SSM_SELFTEST_WAIT_CODE the self-test below. Every kernel's waits give up
+ * after about 2 s. */
 ssm_status ssm_check_device_error(void *stream);
 
 /* Error-word code written by ssm_selftest_bounded_wait. */

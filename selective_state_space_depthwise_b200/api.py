@@ -326,7 +326,7 @@ def proj_gemm_workspace_bytes(M, N, K) -> int:
 def proj_gemm(A, W, *, out=None, workspace=None, stream=None):
     """One projection of the block (ssm_proj_gemm): out = A @ W^T with A [M, K]
     and W [N, K] contiguous bf16 CUDA tensors; returns out [M, N] bf16. The
-    split-K scratch, when the shape needs one, is `workspace` or allocated."""
+    cut-tile scratch, when the shape needs one, is `workspace` or allocated."""
     lib = _lib.load()
     M, K = A.shape
     N = W.shape[0]

@@ -328,7 +328,7 @@ BlockLayout block_layout(const ssm_block_dims* d) {
   l.bc = off, off = align_up(off + M * 32 * 4);
   l.dt = off, off = align_up(off + M * 4);
   l.y = off, off = align_up(off + M * E * 2);
-  // split-K scratch of whichever projection needs more (in_proj and out_proj run one after the other)
+  // cut-tile scratch of whichever projection needs more (in_proj and out_proj run one after the other)
   const int sms = sm_count();
   const int64_t Mi = static_cast<int64_t>(M), Ei = static_cast<int64_t>(E), Dm = d->d_model;
   const size_t g_in = gemm_workspace_bytes(Mi, 2 * Ei, Dm, sms), g_out = gemm_workspace_bytes(Mi, Dm, Ei, sms);

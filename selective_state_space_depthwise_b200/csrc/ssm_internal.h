@@ -54,13 +54,11 @@ cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStrea
 
 // C[M][N] = A[M][K] . B[N][K]^T, bf16 operands and output, fp32 accumulation,
 // on the tensor cores (gemm.cu). K and N multiples of 8, pointers 16-byte
-// aligned. ws: gemm_workspace_bytes() of device scratch (split-K partials and
-// tile counters; 0 bytes when the shape runs unsplit).
+// aligned. ws: gemm_workspace_bytes() of device scratch (the fp32 partials of
+// tiles cut between CTA pairs and their counters; 0 bytes when none is cut).
 cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* ws,
                          size_t ws_bytes, int num_sms, int* err, cudaStream_t st);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
-int gemm_choose_split(int64_t M, int64_t N, int64_t K, int num_sms);
-int gemm_choose_bn(int64_t M, int64_t N, int num_sms);
 
 // Shared by the entry points (ssm_api.cu): validation with the ABI's
 // "0 = dense" stride defaults, and the calling thread's last-error message.
