@@ -27,7 +27,8 @@
 //     to 0 only where the exact product does. The group that holds the
 //     diagonal has a row factor of at most exp(dA[s0] - dA[s1]) (s0 its first
 //     column): below 80 nats it takes the same form, beyond that (where the
-//     row factor could overflow) one exponential per element.
+//     row factor could overflow) one exponential per element. The choice is
+//     made per warp (over its 32 rows), so no branch diverges.
 //     The TMA layout is already the MMA's K-major operand;
 //  4. one thread issues eight MMAs scores x x (x as an MN-major B operand) into
 //     accumulator 0 and commits both;
@@ -251,9 +252,18 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   __syncthreads();  // F complete
 
   // 3. Row l of the cb tile -> scores (in place), atoms at, at + 2, .. of the
-  //    ks columns. A warp's 32 rows lie in one chunk, starting at column warp_min_s.
-  const int warp_max_l = r0 + 32 * (warp & 3) + 31;
+  //    ks columns. A warp's 32 rows lie in one chunk, starting at column
+  //    warp_min_s. Groups are classified against the warp's whole row span,
+  //    so every branch below is warp-uniform: groups wholly at or below all 32
+  //    rows take the two-factor product with no masking; the four groups the
+  //    span straddles mask per element, in the two-factor form unless the
+  //    diagonal group of some row of the warp decays by 80 nats or more
+  //    across its 8 columns (then its row factor could overflow, and each
+  //    decay is formed on its own).
+  const int warp_min_l = r0 + 32 * (warp & 3), warp_max_l = warp_min_l + 31;
   const int warp_min_s = CS < kCs ? (32 * (warp & 3)) & ~(CS - 1) : 0;
+  const int sd = lg & ~7;
+  const bool strong = __any_sync(0xffffffffu, sdA[sd] - sdA[sd + 7] >= 80.0f);
   for (int aa = at; aa < ks / 64; aa += 2) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -265,25 +275,18 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
       }
       float f[8];
       unpack8(*p, f);
-      if (s0 + 7 <= lg) {  // wholly at or below the diagonal: row factor x column factor
+      if (s0 + 7 <= warp_min_l) {  // wholly at or below the diagonal for every row: row factor x column factor
         const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
 #pragma unroll
         for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
-      } else if (s0 <= lg) {  // the diagonal group
-        // The two-factor form while the group's own decay range stays well
-        // inside fp32, else each decay on its own.
-        if (sdA[s0] - sdA[s0 + 7] < 80.0f) {
-          const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+      } else if (!strong) {  // straddled by the warp's rows: masked two-factor form
+        const float e = s0 <= lg ? ex2_approx((dAl - sdA[s0 + 7]) * kLog2e) : 0.0f;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
-        } else {
+        for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
+      } else {  // masked, each decay on its own
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
-        }
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] = 0.0f;
+        for (int q = 0; q < 8; ++q)
+          f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
       }
       *p = pack8(f);
     }

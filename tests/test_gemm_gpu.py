@@ -6,11 +6,11 @@ Reference: the products of the stored bf16 values summed in float64 on the
 CPU, rounded once to bf16. The kernel accumulates the same products in fp32
 (K <= 7680 terms: relative error ~1e-6, far below a bf16 step), so the two
 roundings agree except for rare one-step flips: relative L2 <= 1e-3 is asked.
-Shapes cover ragged M, N and K tails, more tiles than CTA pairs (each pair
-taking several whole tiles, alternating its two accumulators, then a run of
-K chunks), tiles cut along K between pairs (few tiles, long K: fp32 partials
-summed in pair order by the contributor that completes the count, so the
-output is the same on every call) and the block's layer shapes.
+Shapes cover ragged M, N and K tails, more tiles than SMs (each persistent
+CTA taking several whole tiles, alternating its two accumulators, then a run
+of K chunks), tiles cut along K between CTAs (few tiles, long K: fp32
+partials summed in CTA order by the contributor that completes the count, so
+the output is the same on every call) and the block's layer shapes.
 """
 import numpy as np
 import pytest
@@ -60,10 +60,11 @@ def test_gemm_ragged_shapes(shape):
     assert e <= TOL_GEMM
 
 
-def test_gemm_many_tiles_per_pair():
-    """More output tiles than CTA pairs: each pair takes three rounds of whole
-    tiles, then its run of cut tiles, so both TMEM accumulators alternate and
-    the grouped raster wraps (8 row blocks x 40 column blocks)."""
+def test_gemm_many_tiles_per_cta():
+    """More output tiles than SMs: each persistent CTA takes three rounds of
+    whole tiles, then its run of cut tiles, so both TMEM accumulators
+    alternate and the grouped raster wraps (16 row blocks x 40 column
+    blocks)."""
     M, N, K = 2000, 256 * 40 - 24, 200
     A, W = operands(M, N, K, seed=N)
     C = api.proj_gemm(A.cuda(), W.cuda())
@@ -75,9 +76,9 @@ def test_gemm_many_tiles_per_pair():
 
 @pytest.mark.parametrize("shape", [(256, 512, 4096), (200, 264, 1000)], ids=["16_way", "4_way_ragged"])
 def test_gemm_tiles_cut_along_k(shape):
-    """Few output tiles and a long K: every tile is cut along K between CTA
-    pairs (16 and 4 contributors a tile) whose fp32 partials the last
-    contributor sums. Every element against the reference, twice with the
+    """Few output tiles and a long K: every tile is cut along K between CTAs
+    (16 and 4 contributors a tile) whose fp32 partials the last contributor
+    sums. Every element against the reference, twice with the
     same workspace (its tile counters are zeroed by each call), and the two
     outputs bit-equal (the sum runs in pair order whoever finishes last)."""
     M, N, K = shape
