@@ -80,7 +80,7 @@ def test_gemm_tiles_cut_along_k(shape):
     (16 and 4 contributors a tile) whose fp32 partials the last contributor
     sums. Every element against the reference, twice with the
     same workspace (its tile counters are zeroed by each call), and the two
-    outputs bit-equal (the sum runs in pair order whoever finishes last)."""
+    outputs bit-equal (the sum runs in CTA order whoever finishes last)."""
     M, N, K = shape
     assert api.proj_gemm_workspace_bytes(M, N, K) > 0  # this shape cuts tiles
     A, W = operands(M, N, K, seed=K)
