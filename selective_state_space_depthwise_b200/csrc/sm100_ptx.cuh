@@ -59,9 +59,10 @@ static __device__ __noinline__ bool mbar_wait_bounded_ns(uint32_t bar, uint32_t 
   }
 }
 
-// The kernels' waits: bounded at ~2 s.
+// The kernels' waits: bounded at ~2 s. The first test is inline, so a phase
+// that has already completed costs no call.
 static __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* err, int code) {
-  return mbar_wait_bounded_ns(bar, parity, err, code, 2000000000ull);
+  return mbar_try_wait(bar, parity) || mbar_wait_bounded_ns(bar, parity, err, code, 2000000000ull);
 }
 
 // ------------------------------------------------------------- cp.async ---

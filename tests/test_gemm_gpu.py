@@ -60,12 +60,16 @@ def test_gemm_ragged_shapes(shape):
     assert e <= TOL_GEMM
 
 
-def test_gemm_many_tiles_per_cta():
-    """More output tiles than SMs: each persistent CTA takes three rounds of
-    whole tiles, then its run of cut tiles, so both TMEM accumulators
-    alternate and the grouped raster wraps (16 row blocks x 40 column
-    blocks)."""
-    M, N, K = 2000, 256 * 40 - 24, 200
+@pytest.mark.parametrize("shape", [(2000, 256 * 29 - 24, 200), (2000, 256 * 26 - 24, 200)],
+                         ids=["whole_then_cut", "whole_only"])
+def test_gemm_many_tiles_per_cta(shape):
+    """More output tiles than SMs: each persistent CTA takes several whole
+    tiles, so both TMEM accumulators alternate and the grouped raster wraps
+    (16 row blocks x 29 or 26 column blocks). 464 tiles (3.1 a CTA): two
+    rounds of whole tiles, then a run of tiles cut along K; 416 tiles (2.8 a
+    CTA): three rounds of whole tiles, the last one partly idle."""
+    M, N, K = shape
+    assert (api.proj_gemm_workspace_bytes(M, N, K) > 0) == (N == 256 * 29 - 24)
     A, W = operands(M, N, K, seed=N)
     C = api.proj_gemm(A.cuda(), W.cuda())
     torch.cuda.synchronize()
