@@ -16,14 +16,14 @@
 // Thread 0 re-arms a slot right after the CTA has finished with it; every
 // wait on the ring's mbarriers is bounded.
 //
-// Work split (state slices). A CTA is G = 4 warps over 32 channels
+// Work split (state slices). A CTA is G warps (G = 2 or 4) over 32 channels
 // (lane = channel); warp j holds states 16j/G .. 16(j+1)/G - 1 of every
 // channel, so B and C are warp-broadcast loads and x, z, y are lane-contiguous.
 // Each 32-token stage:
 //  A. warp j does the per-token work of tokens [32j/G, 32(j+1)/G) of its
 //     lane's channel (conv from a sliding window of x, SiLU, dt, D*u,
-//     SiLU(z)); the per-token decay operands and dt*u go to shared memory as
-//     rows, D*u and SiLU(z) stay in registers;
+//     SiLU(z)); the per-token decay operand and dt*u go to shared memory as
+//     token-pair rows, D*u and SiLU(z) stay in registers;
 //  B. every warp streams its state slice through all 32 tokens (packed f32x2
 //     multiplies and FMAs) and keeps the partial readouts C.h in registers;
 //  C. warp j sums the G partials of its phase-A tokens, applies the skip and
@@ -35,16 +35,12 @@
 // 2^(dt A_n log2 e): 16 exponentials per channel-token. "Axon-SSM", "State
 // initialization" sets A_log so that the diagonal of A is -1, -2, ..., -16,
 // i.e. A_n = (n+1) A_0. For such a channel exp(dt A_n) = q^(n+1) with
-// q = 2^l, l = dt A_0 log2(e). Phase A writes each token's row as
-// (dt u, dt u, q^2, l), so the scan loads its operands as ready register
-// pairs; slice j forms q^(4j+1) and q^(4j+2) as 2^(l (4j+1)) and
-// 2^(l (4j+2)) and the other two decays as those times q^2: 2 exponentials
-// per slice and token (8 per channel-token instead of 16) and no packing
-// moves. At the start each CTA tests its channels' A (|A_n - (n+1) A_0| <=
-// 2^-20 |A_n| for every n, on the fp32 values the kernel computes); it takes
-// the power path only if all 32 pass, so every other channel keeps the
-// generic path. The power path changes each decay exponent by at most that
-// 2^-20 relative, far inside the fp32 parity bar.
+// q = exp(dt A_0): one exponential per channel-token (in phase A) and a few
+// multiplications per state slice. At the start each CTA tests its channels'
+// A (|A_n - (n+1) A_0| <= 2^-20 |A_n| for every n, on the fp32 values the
+// kernel computes); it takes the power path only if all 32 pass, so every
+// other channel keeps the generic path. The power path changes each decay
+// exponent by at most that 2^-20 relative, far inside the fp32 parity bar.
 //
 // Kernels. 3: G = 4 with the register budget of three CTAs per SM; 4: G = 4
 // built for two CTAs per SM, whose larger register budget buys a deeper
@@ -68,6 +64,11 @@ namespace {
 constexpr int kTok = 32;  // tokens per pipeline stage (= lanes of the dt_raw stager)
 // G warps per CTA = state slices; each thread holds 16 / G states of its lane's
 // channel and does the per-token work of kTok / G tokens per stage.
+#ifndef SSM_PIPE_STAGES
+#define SSM_PIPE_STAGES 3
+#endif
+// Ring depth (depths 3 to 5 time the same on long sequences).
+constexpr int kPipeStages = SSM_PIPE_STAGES;
 // Power-path test: |A_n - (n+1) A_0| <= kPowTol |A_n|.
 constexpr float kPowTol = 9.5367431640625e-07f;  // 2^-20
 
@@ -79,8 +80,8 @@ constexpr int align128(int v) { return (v + 127) / 128 * 128; }
 
 // Shared-memory layout (byte offsets from a 128-aligned base). SPLIT: the
 // partial readouts alternate between two buffers by stage parity (the split
-// end-of-stage barrier needs them; see pipe_run). NS: ring depth.
-template <typename T, int G, bool SPLIT, int NS>
+// end-of-stage barrier needs them; see pipe_run).
+template <typename T, int G, bool SPLIT>
 struct PipeSmem {
   static constexpr int kEs = static_cast<int>(sizeof(T));
   static constexpr int kXBytes = (kTok + 3) * 32 * kEs;  // TMA box {32, kTok + 3}
@@ -91,18 +92,15 @@ struct PipeSmem {
   static constexpr int kB = align128(kZ + kZBytes);
   static constexpr int kC = kB + kBCBytes;
   static constexpr int kSlot = kC + kBCBytes;
-  // Per-token rows, two buffers by stage parity: float4 [token][channel] on
-  // the power path, float4 [token pair][channel] (8 bytes a token) otherwise.
-  static constexpr int kDT = NS * kSlot;
-  static constexpr int kDTBuf = kTok * 32 * 16;
+  static constexpr int kDT = kPipeStages * kSlot;             // float4 [2][token pair][channel]
   static constexpr int kPR = kTok + 4;                        // partial row (padded)
-  static constexpr int kDr = kDT + 2 * kDTBuf;                // dt_raw float [2][token]
+  static constexpr int kDr = kDT + 2 * kTok * 32 * 8;         // dt_raw float [2][token]
   static constexpr int kPBytes = G * 32 * kPR * 4;            // float [slice][channel][kPR]
   static constexpr int kP = kDr + 2 * kTok * 4;               // partials, double-buffered by stage parity
   static constexpr int kY = align128(kP + (SPLIT ? 2 : 1) * kPBytes);  // output tiles [2][token][channel]
   static constexpr int kYBytes = align128(kTok * 32 * kEs);
   static constexpr int kBar = kY + 2 * kYBytes;
-  static constexpr int kTotal = kBar + NS * 8;
+  static constexpr int kTotal = kBar + kPipeStages * 8;
   static constexpr uint32_t kTxBytes = static_cast<uint32_t>(kXBytes + kZBytes + 2 * kBCBytes);
   static_assert((32 * kEs) % 16 == 0, "TMA rows must be whole 16-byte chunks");
 };
@@ -134,22 +132,42 @@ __device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const f
   return lo + hi;
 }
 
-// Power decays: the thread's states 4j .. 4j + 3 decay by q^(4j+1) ..
-// q^(4j+4) with q = 2^l. The token's row r = (dt u, dt u, q^2, l) is loaded
-// as ready register pairs; the first two decays are exponentials of
-// l (4j + 1) and l (4j + 2) (c1, c2), the other two those times q^2.
-__device__ __forceinline__ float scan_token_pow(float4 r, float c1, float c2, float* h, const float* Bp,
+// Power decays: the thread's K states K j .. K j + K - 1 decay by
+// q^(K j + 1) .. q^(K j + K) = base * (q, q^2, ..., q^K) with base = q^(K j).
+// hi1 / hi2 (warp-uniform): bits of j; base = (q^K)^(j&1) (q^2K)^(j>>1 & 1).
+// inj2 = {dt*u, dt*u}.
+template <int K>
+__device__ __forceinline__ float scan_token_pow(float q, uint64_t inj2, bool hi1, bool hi2, float* h, const float* Bp,
                                                 const float* Cp) {
-  const uint64_t inj2 = pk2(r.x, r.y);
-  const float d1 = ex2_approx(r.w * c1), d2 = ex2_approx(r.w * c2);
-  const float4 bq = *reinterpret_cast<const float4*>(Bp);
-  const float4 cq = *reinterpret_cast<const float4*>(Cp);
-  const uint64_t hb0 = ffma2(pk2(d1, d2), pk2(h[0], h[1]), fmul2(inj2, pk2(bq.x, bq.y)));
-  const uint64_t hb1 = ffma2(pk2(d1 * r.z, d2 * r.z), pk2(h[2], h[3]), fmul2(inj2, pk2(bq.z, bq.w)));
-  upk2(hb0, h[0], h[1]);
-  upk2(hb1, h[2], h[3]);
-  uint64_t acc = fmul2(pk2(cq.x, cq.y), hb0);
-  acc = ffma2(pk2(cq.z, cq.w), hb1, acc);
+  static_assert(K == 4 || K == 8, "power decays are built for 4 or 8 states per thread");
+  uint64_t p[K / 2];  // (q, q^2), (q^3, q^4), ...
+  const float q2 = q * q;
+  p[0] = pk2(q, q2);
+  p[1] = fmul2(p[0], pk2(q2, q2));
+  float q3, qk;
+  upk2(p[1], q3, qk);  // qk = q^4
+  if constexpr (K == 8) {
+    const uint64_t q44 = pk2(qk, qk);
+    p[2] = fmul2(p[0], q44);
+    p[3] = fmul2(p[1], q44);
+    float q7;
+    upk2(p[3], q7, qk);  // qk = q^8
+  }
+  float base = hi1 ? qk : 1.0f;
+  if (hi2) base *= qk * qk;
+  const uint64_t bb = pk2(base, base);
+  uint64_t acc = 0;
+#pragma unroll
+  for (int i = 0; i < K / 2; i += 2) {
+    const float4 bq = *reinterpret_cast<const float4*>(Bp + 2 * i);
+    const float4 cq = *reinterpret_cast<const float4*>(Cp + 2 * i);
+    const uint64_t hb0 = ffma2(fmul2(bb, p[i]), pk2(h[2 * i], h[2 * i + 1]), fmul2(inj2, pk2(bq.x, bq.y)));
+    const uint64_t hb1 = ffma2(fmul2(bb, p[i + 1]), pk2(h[2 * i + 2], h[2 * i + 3]), fmul2(inj2, pk2(bq.z, bq.w)));
+    upk2(hb0, h[2 * i], h[2 * i + 1]);
+    upk2(hb1, h[2 * i + 2], h[2 * i + 3]);
+    acc = i == 0 ? fmul2(pk2(cq.x, cq.y), hb0) : ffma2(pk2(cq.x, cq.y), hb0, acc);
+    acc = ffma2(pk2(cq.z, cq.w), hb1, acc);
+  }
   float lo, hi;
   upk2(acc, lo, hi);
   return lo + hi;
@@ -170,16 +188,15 @@ __device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* 
   return acc;
 }
 
-// Rows stored per token: (dt, dt*u) in token pairs (generic); (dt, u) in
-// token pairs (ZOH); (dt*u, dt*u, q^2, l) with l = dt A_0 log2(e), q = 2^l
-// (power path).
+// Decay operand stored per token: dt (generic), q = e^{dt A_0} (power path),
+// dt (ZOH, with u instead of dt*u as the second value).
 enum class Path { kGeneric, kPow, kZoh };
 
 // Per-token work of kTA tokens [tb, tb+kTA) of this lane's channel for one
-// stage: the rows (kTA float4 on the power path, kTA / 2 otherwise), D*u and
-// SiLU(z) to registers. Dr is the stage's dt_raw row. The caller stores the
-// rows (store_rows) after the scan, so no shared-memory store sits between
-// the scan's loads in program order.
+// stage: the (decay operand, injection) of token pairs, D*u and SiLU(z) to
+// registers. Dr is the stage's dt_raw row. The caller stores the pairs
+// (store_rows) after the scan, so no shared-memory store sits between the
+// scan's loads in program order.
 template <typename T, Path P, int kTA>
 __device__ __forceinline__ void phase_a(const T* __restrict__ X, const T* __restrict__ Z, const float* __restrict__ Dr,
                                         int64_t t0, int64_t L, int tb, int lane, bool first, float hx0, float hx1,
@@ -205,60 +222,43 @@ __device__ __forceinline__ void phase_a(const T* __restrict__ X, const T* __rest
     const float conv = fmaf(cw3, xw[i + 3], fmaf(cw2, xw[i + 2], fmaf(cw1, xw[i + 1], fmaf(cw0, xw[i], cb))));
     const float u = silu(conv);
     float dt = dt_of(fmaf(dr[i], wdt, dtb), lo, hi);
-    if (t0 + tb + i >= L) dt = 0.0f;  // past the end: keep the state (decay 1, no injection)
-    if constexpr (P == Path::kPow) {
-      const float l = dt * a20, inj = dt * u;
-      rows[i] = make_float4(inj, inj, ex2_approx(l + l), l);
-    } else {
+    if (t0 + tb + i >= L) dt = 0.0f;  // past the end: keep the state (q = 1, no injection)
+    if constexpr (P == Path::kPow)
+      dtv[i] = make_float2(ex2_approx(dt * a20), dt * u);
+    else
       dtv[i] = make_float2(dt, P == Path::kZoh ? u : dt * u);
-    }
     du[i] = Dd * u;
     zg[i] = silu(zr[i]);
   }
-  if constexpr (P != Path::kPow) {
 #pragma unroll
-    for (int i = 0; i < kTA; i += 2) rows[i / 2] = make_float4(dtv[i].x, dtv[i].y, dtv[i + 1].x, dtv[i + 1].y);
-  }
+  for (int i = 0; i < kTA; i += 2) rows[i / 2] = make_float4(dtv[i].x, dtv[i].y, dtv[i + 1].x, dtv[i + 1].y);
 }
 
-// Rows a warp's phase A produces per stage.
-template <Path P, int kTA>
-__host__ __device__ constexpr int row_count() {
-  return P == Path::kPow ? kTA : kTA / 2;
-}
-
-// Rows as [token][channel] (power path) or [token pair][channel] (d, inj,
-// d', inj'): one 16-byte load per token, or per two tokens, in phase B.
-template <Path P, int kTA>
-__device__ __forceinline__ void store_rows(float4* DT4, int tb, int lane, const float4* rows) {
-  if constexpr (P == Path::kPow) {
+// Rows as [token pair][channel] (d, inj, d', inj'): one 16-byte load per two
+// tokens in phase B.
+template <int kTA>
+__device__ __forceinline__ void store_rows(float2* DTo, int tb, int lane, const float4* rows) {
+  float4* DT4 = reinterpret_cast<float4*>(DTo);
 #pragma unroll
-    for (int i = 0; i < kTA; ++i) DT4[(tb + i) * 32 + lane] = rows[i];
-  } else {
-#pragma unroll
-    for (int i = 0; i < kTA; i += 2) DT4[((tb + i) >> 1) * 32 + lane] = rows[i / 2];
-  }
+  for (int i = 0; i < kTA; i += 2) DT4[((tb + i) >> 1) * 32 + lane] = rows[i / 2];
 }
 
 // Phase B over tokens [T0, T1) of one stage: this thread's 4 states; pr gets
 // the partial readouts.
 template <Path P, int K, int T0 = 0, int T1 = kTok>
-__device__ __forceinline__ void scan_stage(const float4* __restrict__ DTc, int lane, const float* Av, const float* a2,
-                                           float c1, float c2, float* h, const float* __restrict__ Bs,
+__device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int lane, const float* Av, const float* a2,
+                                           bool hi1, bool hi2, float* h, const float* __restrict__ Bs,
                                            const float* __restrict__ Cs, float* pr) {
 #pragma unroll
   for (int tl = T0; tl < T1; ++tl) {
-    if constexpr (P == Path::kPow) {
-      static_assert(K == 4, "power decays are built for 4 states per thread");
-      pr[tl] = scan_token_pow(DTc[tl * 32 + lane], c1, c2, h, Bs + tl * 16, Cs + tl * 16);
-    } else {
-      const float4 d4 = DTc[(tl >> 1) * 32 + lane];
-      const float2 dd = (tl & 1) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
-      if constexpr (P == Path::kZoh)
-        pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
-      else
-        pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
-    }
+    const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
+    const float2 dd = (tl & 1) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+    if constexpr (P == Path::kZoh)
+      pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
+    else if constexpr (P == Path::kPow)
+      pr[tl] = scan_token_pow<K>(dd.x, pk2(dd.y, dd.y), hi1, hi2, h, Bs + tl * 16, Cs + tl * 16);
+    else
+      pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
   }
 }
 
@@ -267,20 +267,18 @@ __device__ __forceinline__ void scan_stage(const float4* __restrict__ DTc, int l
 // visible; ring slot s free) and barrier 2 after phase C (output tile
 // complete). SPLIT: at barrier 2 only warp 0, which stores the tile, waits;
 // the others arrive and run on, which needs the partials double-buffered.
-template <typename T, int G, Path P, bool SPLIT, int NS>
+template <typename T, int G, Path P, bool SPLIT>
 __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) {
   constexpr int NT = 32 * G;
   constexpr int kK = 16 / G;     // states per thread
   constexpr int kTA = kTok / G;  // phase-A and phase-C tokens per warp and stage
-  using S = PipeSmem<T, G, SPLIT, NS>;
-  constexpr int kRows = row_count<P, kTA>();
-  constexpr int kDTStride = S::kDTBuf / 16;  // float4 per row buffer
+  using S = PipeSmem<T, G, SPLIT>;
 
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
   const uint32_t sb = smem_u32(smem);
   const uint32_t full0 = sb + S::kBar;
-  float4* DT = reinterpret_cast<float4*>(smem + S::kDT);
+  float2* DT = reinterpret_cast<float2*>(smem + S::kDT);
   float* Dr = reinterpret_cast<float*>(smem + S::kDr);
 
   const int tid = threadIdx.x;
@@ -295,7 +293,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
   const float* dtr = a.dt_raw + static_cast<int64_t>(seq) * a.s.dt_seq;
 
   auto issue_stage = [&](int64_t st_idx) {  // thread 0 only
-    const int slot = static_cast<int>(st_idx % NS);
+    const int slot = static_cast<int>(st_idx % kPipeStages);
     const uint32_t base = sb + slot * S::kSlot, bar = full0 + 8 * slot;
     const int t0 = static_cast<int>(st_idx * kTok);
     mbar_arrive_expect_tx(bar, S::kTxBytes);
@@ -305,13 +303,13 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     tma_load_3d(base + S::kC, &maps.C, 0, t0, seq, bar);
   };
   if (tid == 0) {
-    for (int i = 0; i < NS; ++i) mbar_init(full0 + 8 * i, 1);
+    for (int i = 0; i < kPipeStages; ++i) mbar_init(full0 + 8 * i, 1);
     mbar_fence_init();
     prefetch_tensormap(&maps.x);
     prefetch_tensormap(&maps.z);
     prefetch_tensormap(&maps.B);
     prefetch_tensormap(&maps.C);
-    for (int64_t i = 0; i < NS && i < n_stages; ++i) issue_stage(i);
+    for (int64_t i = 0; i < kPipeStages && i < n_stages; ++i) issue_stage(i);
   }
   // dt_raw of stage st_idx (one token per lane of warp 0) into its buffer; zero past the end
   auto copy_dt_raw = [&](int64_t st_idx) {
@@ -349,28 +347,27 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + warp * kK + q] : 0.0f;
   }
   const float a20 = -expf(a.A_log[ec * 16]) * kLog2e;  // A_0 log2(e): q = 2^(dt a20) on the power path
-  // Power path: this slice's first two decays are 2^(l c1) and 2^(l c2).
-  const float c1 = static_cast<float>(warp * kK + 1), c2 = static_cast<float>(warp * kK + 2);
+  const bool hi1 = (warp & 1) != 0, hi2 = (warp & 2) != 0;  // bits of the slice index (power path)
   const int tb = warp * kTA;
 
   // Prologue: phase A of stage 0.
   float du[kTA], zg[kTA];
   {
-    float4 rows0[kRows];
+    float4 rows0[kTA / 2];
     mbar_wait_bounded(full0, 0u, a.err, 1);
     phase_a<T, P, kTA>(reinterpret_cast<const T*>(smem + S::kX), reinterpret_cast<const T*>(smem + S::kZ), Dr, 0, L,
                        tb, lane, true, hx0, hx1, hx2, cw0, cw1, cw2, cw3, cb, wdt, dtb, Dd, lo, hi, a20, rows0, du, zg);
-    store_rows<P, kTA>(DT, tb, lane, rows0);
+    store_rows<kTA>(DT, tb, lane, rows0);
   }
   named_bar_sync(1, NT);
 
   for (int64_t s = 0; s < n_stages; ++s) {
-    const int slot = static_cast<int>(s % NS);
+    const int slot = static_cast<int>(s % kPipeStages);
     const unsigned char* st = smem + slot * S::kSlot;
     const float* Bs = reinterpret_cast<const float*>(st + S::kB) + warp * kK;
     const float* Cs = reinterpret_cast<const float*>(st + S::kC) + warp * kK;
-    const float4* DTc = DT + (s & 1) * kDTStride;
-    float4* DTn = DT + ((s + 1) & 1) * kDTStride;
+    const float2* DTc = DT + (s & 1) * kTok * 32;
+    float2* DTn = DT + ((s + 1) & 1) * kTok * 32;
     const int64_t t0 = s * kTok;
     const bool has_next = s + 1 < n_stages;
     float duN[kTA], zgN[kTA];
@@ -381,20 +378,20 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     // Phase B of stage s fused with phase A of stage s + 1.
     float pr[kTok];
     if (has_next) {
-      const int nslot = static_cast<int>((s + 1) % NS);
-      mbar_wait_bounded(full0 + 8 * nslot, static_cast<uint32_t>(((s + 1) / NS) & 1), a.err, 1);
+      const int nslot = static_cast<int>((s + 1) % kPipeStages);
+      mbar_wait_bounded(full0 + 8 * nslot, static_cast<uint32_t>(((s + 1) / kPipeStages) & 1), a.err, 1);
       const unsigned char* nst = smem + nslot * S::kSlot;
       // Source order: first half of the scan, the next stage's per-token work,
       // second half of the scan (measured 2% faster than either block first).
-      float4 rows[kRows];
-      scan_stage<P, kK, 0, kTok / 2>(DTc, lane, Av, a2, c1, c2, h, Bs, Cs, pr);
+      float4 rows[kTA / 2];
+      scan_stage<P, kK, 0, kTok / 2>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
       phase_a<T, P, kTA>(reinterpret_cast<const T*>(nst + S::kX), reinterpret_cast<const T*>(nst + S::kZ),
                          Dr + ((s + 1) & 1) * kTok, t0 + kTok, L, tb, lane, false, hx0, hx1, hx2, cw0, cw1, cw2, cw3,
                          cb, wdt, dtb, Dd, lo, hi, a20, rows, duN, zgN);
-      scan_stage<P, kK, kTok / 2, kTok>(DTc, lane, Av, a2, c1, c2, h, Bs, Cs, pr);
-      store_rows<P, kTA>(DTn, tb, lane, rows);
+      scan_stage<P, kK, kTok / 2, kTok>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      store_rows<kTA>(DTn, tb, lane, rows);
     } else {
-      scan_stage<P, kK>(DTc, lane, Av, a2, c1, c2, h, Bs, Cs, pr);
+      scan_stage<P, kK>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
     }
     {
       float* Pj = P_ + (warp * 32 + lane) * S::kPR;
@@ -408,7 +405,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     // visible; every warp is done with ring slot s (phase A of s ran in the
     // previous block, phase B of s just now), so it is re-armed at once.
     named_bar_sync(1, NT);
-    if (tid == 0 && s + NS < n_stages) issue_stage(s + NS);
+    if (tid == 0 && s + kPipeStages < n_stages) issue_stage(s + kPipeStages);
 
     // Phase C of stage s: tokens [tb, tb + kTA).
     {
@@ -521,28 +518,19 @@ template <int MINB>
 __host__ __device__ constexpr bool split_barrier() {
   return MINB == 1 && SSM_PREFILL_SPLIT_BARRIER;
 }
-// Ring depth: 3 stages where two CTAs share an SM; 2 in the three-CTAs-per-SM
-// build, whose shared memory (three CTAs in 227 KB) has no room for a third
-// slot next to the power path's 16-byte-a-token rows (a stage lasts several
-// microseconds there, far longer than a TMA load).
-template <int MINB>
-__host__ __device__ constexpr int ring_depth() {
-  return MINB == 1 ? 3 : 2;
-}
 
 template <typename T, int G, bool ZOH, int MINB>
 __global__ void __launch_bounds__(32 * G, MINB) prefill_pipe_kernel(const __grid_constant__ Maps maps,
                                                                      const KernelArgs a) {
   constexpr bool SPLIT = split_barrier<MINB>();
-  constexpr int NS = ring_depth<MINB>();
   if constexpr (ZOH) {
-    pipe_run<T, G, Path::kZoh, SPLIT, NS>(maps, a);
+    pipe_run<T, G, Path::kZoh, SPLIT>(maps, a);
   } else {
     const bool pw = a.decay_path == 0 && cta_has_power_decays<G>(a);
     if (pw)
-      pipe_run<T, G, Path::kPow, SPLIT, NS>(maps, a);
+      pipe_run<T, G, Path::kPow, SPLIT>(maps, a);
     else
-      pipe_run<T, G, Path::kGeneric, SPLIT, NS>(maps, a);
+      pipe_run<T, G, Path::kGeneric, SPLIT>(maps, a);
   }
 }
 
@@ -601,7 +589,7 @@ bool make_maps(const KernelArgs& a, Maps* m) {
 
 template <typename T, int G, bool ZOH, int MINB>
 cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st) {
-  using S = PipeSmem<T, G, split_barrier<MINB>(), ring_depth<MINB>()>;
+  using S = PipeSmem<T, G, split_barrier<MINB>()>;
   Maps maps;
   if (!make_maps<T>(a, &maps)) return cudaErrorInvalidValue;
   auto kern = prefill_pipe_kernel<T, G, ZOH, MINB>;
