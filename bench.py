@@ -178,6 +178,7 @@ KERNEL_SOURCES = {
     "prefill": ("prefill.cu", "ssm_math.cuh", "sm100_ptx.cuh"),
     "decode": ("decode.cu", "ssm_math.cuh", "sm100_ptx.cuh"),
     "ssd": ("ssd.cu", "ssm_math.cuh", "sm100_ptx.cuh", "tma_map.cuh"),
+    "gemm": ("gemm.cu", "sm100_ptx.cuh", "tma_map.cuh"),
 }
 
 
