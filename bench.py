@@ -205,6 +205,15 @@ def ncu_traffic(kernel: str, workload: str):
         return None
 
 
+def step_config(w: W.Workload, world: int) -> dict:
+    """The `config` of the step workload, the same in both arms' lines."""
+    return {"workload": f"{w.name}: {w.note}; b={w.batch} L={w.seqlen} E={w.d_inner} N=16 K=4",
+            "batch": w.batch, "seq_len": w.seqlen, "d_inner": w.d_inner, "d_state": 16, "d_conv": 4,
+            "parallelism": (f"dp{world}: one independent sequence of the workload per GPU (batch sharding, "
+                            f"no collective)") if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (no flush)" if min_bytes_prefill(w) > 126e6 else "inputs fit in L2"}
+
+
 # ----------------------------------------------------------------- oracle ---
 def cpu_baseline(w: W.Workload, target_s: float = 10.0):
     """The oracle, as it stands, on the host cores: n channels of sequence 0
@@ -758,8 +767,7 @@ def main():
         print(json.dumps({"impl": "reference", "metric": METRIC, "value": value,
                           "unit": "channel-tokens/s", "n_gpus": args.gpus, "steps": args.steps,
                           "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                          "dtype": "f64", "data": "synthetic", "config": {"workload": w.note, "batch": w.batch,
-                                                                          "seq_len": w.seqlen, "d_inner": w.d_inner},
+                          "dtype": "f64", "data": "synthetic", "config": step_config(w, args.gpus),
                           "cpu_baseline": cb,
                           "e2e": {"value": value, "unit": "channel-tokens/s", "h2d_bytes_per_step": 0,
                                   "d2h_bytes_per_step": 0}}))
@@ -845,11 +853,7 @@ def main():
         "value": value, "unit": "channel-tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "io_dtype": "bf16" if w.io_dtype == torch.bfloat16 else "f32", "data": "synthetic",
-        "config": {"workload": f"{w.name}: {w.note}; b={w.batch} L={w.seqlen} E={w.d_inner} N=16 K=4",
-                   "batch": w.batch, "seq_len": w.seqlen, "d_inner": w.d_inner, "d_state": 16, "d_conv": 4,
-                   "parallelism": (f"dp{world}: one independent sequence of the workload per GPU (batch sharding, "
-                                   f"no collective)") if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (no flush)" if min_bytes_prefill(w) > 126e6 else "inputs fit in L2"},
+        "config": step_config(w, world),
         "roofline": {"bound": "alu", "achieved": per_gpu, "peak": peak_ct, "unit": "channel-tokens/s",
                      "frac": round(per_gpu / peak_ct, 4),
                      "peak_basis": "SFU 16 + FP32 128 lanes/clk/SM x 148 SMs at 1965 MHz; the power decay path's "

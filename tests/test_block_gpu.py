@@ -1,6 +1,7 @@
-"""GPU parity of the whole block forward (ssm_block_forward: cuBLASLt in_proj,
-the fused tcgen05 x_proj kernel, the prefill core, cuBLASLt out_proj) against
-the block oracle, on seeded synthetic inputs.
+"""GPU parity of the whole block forward (ssm_block_forward: the library's
+tcgen05 GEMM for in_proj, the fused tcgen05 x_proj kernel, the prefill core,
+the same GEMM for out_proj) against the block oracle, on seeded synthetic
+inputs.
 
 Tolerance. The GPU path stores four intermediate quantities in bf16: x and z
 (the in_proj output), u (the x_proj operand), the gated core output, and the
