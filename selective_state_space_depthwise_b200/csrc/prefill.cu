@@ -402,9 +402,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
         *reinterpret_cast<float4*>(Pj + tl) = make_float4(pr[tl], pr[tl + 1], pr[tl + 2], pr[tl + 3]);
     }
     if (warp == 0) cp_async_wait_all();  // dt_raw of stage s + 2 lands before the barrier
-    // Output tile (s & 1) no longer read by the store of stage s - 2, which
-    // lane 0 of warp (s - 2) mod G issued (bulk groups are per thread).
-    if (s >= 2 && lane == 0 && warp == static_cast<int>((s - 2) & (G - 1))) bulk_wait_read<0>();
+    if (tid == 0) bulk_wait_read<1>();    // output tile (s & 1) no longer read by the store of stage s - 2
     // Partials of stage s, rows of stage s + 1 and dt_raw of stage s + 2
     // visible; every warp is done with ring slot s (phase A of s ran in the
     // previous block, phase B of s just now), so it is re-armed at once.
@@ -439,18 +437,15 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
         zg[i] = zgN[i];
       }
     }
-    // The output tile is complete once every warp has written its tokens. The
-    // store rotates over the warps by stage (warp s mod G), so the extra wait
-    // and the store do not always fall on the same warp. SPLIT: the storing
-    // warp waits for the tile and stores it; the other warps only arrive and
-    // go on to the next stage (no other buffer needs this barrier: the
+    // The output tile is complete once every warp has written its tokens.
+    // SPLIT: warp 0 waits for that and stores it; the other warps only arrive
+    // and go on to the next stage (no other buffer needs this barrier: the
     // partials alternate by stage parity, and the next writer of any buffer
     // read in phase C passes barrier 1 of the next stage first). Otherwise
     // every warp waits, which also frees the single partials buffer.
-    const int storer = static_cast<int>(s & (G - 1));
-    if (!SPLIT || warp == storer) {
+    if (!SPLIT || warp == 0) {
       named_bar_sync(2, NT);
-      if (warp == storer && lane == 0) {
+      if (tid == 0) {
         tma_store_3d(&maps.y, sb + S::kY + (s & 1) * S::kYBytes, e0, static_cast<int>(t0), seq);
         bulk_commit();
       }
@@ -458,7 +453,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
       named_bar_arrive(2, NT);
     }
   }
-  if (lane == 0) bulk_wait<0>();  // every warp's stores have completed
+  if (tid == 0) bulk_wait<0>();
 
   if (ch_ok) {
 #pragma unroll
