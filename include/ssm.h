@@ -323,15 +323,15 @@ size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
  *   A  [M, K] bf16, row-major;  W  [N, K] bf16, row-major;  C  [M, N] bf16
  * Device pointers, 16-byte aligned; K and N multiples of 8; 0 < M, N, K <=
  * 2^31; C must not alias A or W. fp32 accumulation, C rounded to bf16 (RNE).
- * One persistent kernel (tcgen05 MMAs into TMEM, TMA operand ring, TMA
- * stores) enqueued on `stream`, after a memset of the workspace's tile
- * counters when some tile is cut between CTAs.
+ * One persistent kernel of CTA pairs (two-SM tcgen05 MMAs into TMEM, TMA
+ * operand rings, TMA stores) enqueued on `stream`, after a memset of the
+ * workspace's tile counters when some tile is cut between pairs.
  *   workspace  ssm_proj_gemm_workspace_bytes(M, N, K) bytes of device scratch,
- *              256-byte aligned, or NULL when that is 0. Whole 128 x 256 output
- *              tiles go round-robin to one CTA per SM; the last one to two
- *              tiles a CTA are instead cut along K into equal runs, one per
- *              CTA, and the fp32 partials of the cut tiles (256 KB a CTA) and
- *              a counter per tile live here. The partials of a cut tile are
+ *              256-byte aligned, or NULL when that is 0. Whole 256 x 256 output
+ *              tiles go round-robin to the pairs. Where a last wave would leave
+ *              most pairs idle, the final one to two tiles a pair are instead
+ *              cut along K into equal runs, one per pair; the fp32 partials of
+ *              the cut tiles (512 KB a pair) and a counter per tile live here. The partials of a cut tile are
  *              summed in a fixed order, so results do not depend on timing.
  *              Calls that overlap on the GPU need separate workspaces.
  */

@@ -59,8 +59,7 @@ static __device__ __noinline__ bool mbar_wait_bounded_ns(uint32_t bar, uint32_t 
   }
 }
 
-// The kernels' waits: bounded at ~2 s. The first test is inline, so a phase
-// that has already completed costs no call.
+// The kernels' waits: bounded at ~2 s.
 static __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int* err, int code) {
   return mbar_try_wait(bar, parity) || mbar_wait_bounded_ns(bar, parity, err, code, 2000000000ull);
 }
@@ -165,7 +164,69 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr, uint32_t r
   return v;
 }
 
+// Shared::cluster address of the object at local shared address `addr` in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  return remote;
+}
+// One arrival on an mbarrier anywhere in the cluster (shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Busy-wait for `ns` nanoseconds.
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) {
+  }
+}
+
+// ------------------------------------------------------ tcgen05, CTA pair ---
+// The same operations issued for a pair of CTAs (cluster ranks 0 and 1): the
+// allocation is made by one warp of each CTA and gives both the same TMEM
+// address; the MMA is issued by one thread of rank 0 and reads A (M rows split
+// 128 / 128) and B (N rows split in halves) from the same shared-memory
+// offsets in both CTAs, each CTA's TMEM receiving its own 128 rows of D.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t smem_dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_dst), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma_f16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 bool accumulate) {
+  const uint32_t acc = accumulate ? 1u : 0u;
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// One arrival on the mbarrier at local offset `mbar` in every CTA of
+// `cta_mask` once all MMAs issued so far have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t mbar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(mbar),
+      "h"(cta_mask)
+      : "memory");
+}
+
 // ------------------------------------------------------------------ TMA ---
+// Tile load into this CTA's shared memory whose completion is counted on an
+// mbarrier of either CTA of the pair (`bar`: shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int32_t c0, int32_t c1, int32_t c2,
                                             int32_t c3, uint32_t bar) {
   asm volatile(

@@ -6,11 +6,13 @@ Reference: the products of the stored bf16 values summed in float64 on the
 CPU, rounded once to bf16. The kernel accumulates the same products in fp32
 (K <= 7680 terms: relative error ~1e-6, far below a bf16 step), so the two
 roundings agree except for rare one-step flips: relative L2 <= 1e-3 is asked.
-Shapes cover ragged M, N and K tails, more tiles than SMs (each persistent
-CTA taking several whole tiles, alternating its two accumulators, then a run
-of K chunks), tiles cut along K between CTAs (few tiles, long K: fp32
-partials summed in CTA order by the contributor that completes the count, so
-the output is the same on every call) and the block's layer shapes.
+The kernel runs on CTA pairs (256 x 256 tiles, two-SM MMAs). Shapes cover
+ragged M, N and K tails (the second CTA of a pair past M), more tiles than
+pairs (each persistent pair taking several whole tiles, alternating its two
+accumulators, then a run of K chunks), tiles cut along K between pairs (few
+tiles, long K: fp32 partials summed in pair order by the contributor that
+completes the count, so the output is the same on every call) and the
+block's layer shapes.
 """
 import numpy as np
 import pytest
@@ -63,11 +65,11 @@ def test_gemm_ragged_shapes(shape):
 @pytest.mark.parametrize("shape", [(2000, 256 * 29 - 24, 200), (2000, 256 * 26 - 24, 200)],
                          ids=["whole_then_cut", "whole_only"])
 def test_gemm_many_tiles_per_cta(shape):
-    """More output tiles than SMs: each persistent CTA takes several whole
-    tiles, so both TMEM accumulators alternate and the grouped raster wraps
-    (16 row blocks x 29 or 26 column blocks). 464 tiles (3.1 a CTA): two
-    rounds of whole tiles, then a run of tiles cut along K; 416 tiles (2.8 a
-    CTA): three rounds of whole tiles, the last one partly idle."""
+    """More output tiles than CTA pairs: each persistent pair takes several
+    whole tiles, so both TMEM accumulators alternate and the grouped raster
+    wraps (8 row blocks x 29 or 26 column blocks). 232 tiles (3.1 a pair):
+    two rounds of whole tiles, then a run of tiles cut along K; 208 tiles
+    (2.8 a pair): three rounds of whole tiles, the last one partly idle."""
     M, N, K = shape
     assert (api.proj_gemm_workspace_bytes(M, N, K) > 0) == (N == 256 * 29 - 24)
     A, W = operands(M, N, K, seed=N)
@@ -80,11 +82,11 @@ def test_gemm_many_tiles_per_cta(shape):
 
 @pytest.mark.parametrize("shape", [(256, 512, 4096), (200, 264, 1000)], ids=["16_way", "4_way_ragged"])
 def test_gemm_tiles_cut_along_k(shape):
-    """Few output tiles and a long K: every tile is cut along K between CTAs
-    (16 and 4 contributors a tile) whose fp32 partials the last contributor
-    sums. Every element against the reference, twice with the
+    """Few output tiles and a long K: every tile is cut along K between CTA
+    pairs (16 and 4 contributors a tile) whose fp32 partials the last
+    contributor sums. Every element against the reference, twice with the
     same workspace (its tile counters are zeroed by each call), and the two
-    outputs bit-equal (the sum runs in CTA order whoever finishes last)."""
+    outputs bit-equal (the sum runs in pair order whoever finishes last)."""
     M, N, K = shape
     assert api.proj_gemm_workspace_bytes(M, N, K) > 0  # this shape cuts tiles
     A, W = operands(M, N, K, seed=K)
