@@ -74,19 +74,26 @@ struct SsdSmem {
   static constexpr int kHalves = CS > kCs ? CS / kCs : 1;  // CTAs per chunk (128-row halves)
   static constexpr int kKS = CS > kCs ? CS : kCs;      // most score columns = rows of x = K of the intra term
   static constexpr int kNA = DS / 64;                  // 64-column atoms across the state dim
+  // State dim 128 at chunk 64 or 128: the carried-state operands are loaded
+  // one 64-column atom at a time into one buffer (the first atom's MMAs free
+  // it for the second). That brings a chunk-128 CTA to ~75 KB (three CTAs per
+  // SM instead of two) and a chunk-64 CTA to ~84 KB (two instead of one).
+  static constexpr bool kReload = kNA == 2 && CS <= kCs;
+  static constexpr int kSA = kReload ? 1 : kNA;        // state atoms resident at once
   static constexpr int kAtomRows128 = kCs * 128;       // one 64-column atom of a 128-row tile
   static constexpr int kAtomRows64 = kHd * 128;        // one 64-column atom of a 64-row tile
   static constexpr int kCb = 0;                        // cb -> scores [128][kKS] (A of MMA 1) -> out tile
   static constexpr int kC = kCb + (kKS / 64) * kAtomRows128;  // C [128][DS] (A of MMA 2)
-  static constexpr int kX = kC + kNA * kAtomRows128;   // x [kKS][p] (B of MMA 1, MN-major)
+  static constexpr int kX = kC + kSA * kAtomRows128;   // x [kKS][p] (B of MMA 1, MN-major)
   static constexpr int kPrev = kX + kKS * 128;         // prev_states [chunk][p][n] (B of MMA 2, K-major)
-  static constexpr int kDA = kPrev + kNC * kNA * kAtomRows64;
+  static constexpr int kDA = kPrev + kNC * kSA * kAtomRows64;
   static constexpr int kDt = kDA + kKS * 4;
   static constexpr int kF = kDt + kKS * 4;
-  static constexpr int kBar = kF + kKS * 4;            // full_state, full_scores, done
-  static constexpr int kTmemSlot = kBar + 24;
+  static constexpr int kBar = kF + kKS * 4;            // full_state, full_scores, done, state_free
+  static constexpr int kTmemSlot = kBar + 32;
   static constexpr int kTotal = kTmemSlot + 16;
-  static constexpr uint32_t kTxState = static_cast<uint32_t>(kNA * (kAtomRows128 + kNC * kAtomRows64));  // C, prev
+  // C and prev_states bytes of one load round (all atoms, or one when reloading)
+  static constexpr uint32_t kTxState = static_cast<uint32_t>(kSA * (kAtomRows128 + kNC * kAtomRows64));
   // cb and x of a CTA whose score tile is ks columns wide (ks = 128, or 256 for
   // the second half of a 256-chunk): stacked chunks load their [CS][CS]
   // diagonal blocks, otherwise 128 rows x ks columns; x has ks rows.
@@ -157,10 +164,25 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   const int64_t t_chunk = static_cast<int64_t>(c) * CS;  // first token of chunk c
   const int g = static_cast<int>(h / (a.nheads / a.ngroups));
   const uint32_t full_state = sb + S::kBar, full_scores = sb + S::kBar + 8, done = sb + S::kBar + 16;
+  const uint32_t state_free = sb + S::kBar + 24;
+  const int64_t zp0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h;
+  // State atoms [t0, t0 + kSA) of C and prev_states into the state buffers.
+  auto load_state = [&](int t0) {
+#pragma unroll
+    for (int i = 0; i < S::kSA; ++i) {
+      const int t = t0 + i;
+      tma_load_4d(sb + S::kC + i * S::kAtomRows128, &map_c, 64 * t, g, static_cast<int>(t_chunk + r0), b, full_state);
+#pragma unroll
+      for (int k = 0; k < NC; ++k)
+        tma_load_3d(sb + S::kPrev + (k * S::kSA + i) * S::kAtomRows64, &map_prev, 64 * t, 0,
+                    static_cast<int>(zp0 + k * a.nheads), full_state);
+    }
+  };
   if (tid == 0) {
     mbar_init(full_state, 1);
     mbar_init(full_scores, 1);
     mbar_init(done, 1);
+    mbar_init(state_free, 1);
     mbar_fence_init();
     prefetch_tensormap(&map_cb);
     prefetch_tensormap(&map_x);
@@ -169,20 +191,8 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     // A second stacked chunk past the last one (odd chunk count) reads zeros
     // or a neighbouring sequence's chunk; its rows lie past L and are never stored.
     const int64_t zc0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g;
-    const int64_t zp0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h;
     mbar_arrive_expect_tx(full_state, S::kTxState);
     mbar_arrive_expect_tx(full_scores, S::tx_scores(ks));
-    auto load_state = [&] {
-#pragma unroll
-      for (int t = 0; t < S::kNA; ++t) {
-        tma_load_4d(sb + S::kC + t * S::kAtomRows128, &map_c, 64 * t, g, static_cast<int>(t_chunk + r0), b,
-                    full_state);
-#pragma unroll
-        for (int k = 0; k < NC; ++k)
-          tma_load_3d(sb + S::kPrev + (k * S::kNA + t) * S::kAtomRows64, &map_prev, 64 * t, 0,
-                      static_cast<int>(zp0 + k * a.nheads), full_state);
-      }
-    };
     auto load_scores = [&] {
       if constexpr (NC == 1) {
         for (int t = 0; t < ks / 64; ++t)  // rows r0 .. r0 + 127, columns 64 t ..
@@ -199,9 +209,9 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     };
     if (kScoresFirst) {
       load_scores();
-      load_state();
+      load_state(0);
     } else {
-      load_state();
+      load_state(0);
       load_scores();
     }
   }
@@ -229,21 +239,31 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   // stacked chunk k at 64 (k + 1) (C x prev_states(k)^T over all 128 rows;
   // rows of chunk k read it).
   const uint32_t acc_intra = tmem;
-  auto state_mmas = [&] {
+  // MMAs of the resident state atoms, the first of which is state atom t0
+  // (a K of 16 per MMA, four per 64-column atom).
+  auto state_mmas = [&](int t0) {
 #pragma unroll
     for (int k = 0; k < NC; ++k)
 #pragma unroll
-      for (int kk = 0; kk < DS / 16; ++kk)
+      for (int kk = 0; kk < 4 * S::kSA; ++kk)
         umma_f16_ss(tmem + kHd * (k + 1),
                     umma_desc_k_sw128(sb + S::kC + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
-                    umma_desc_k_sw128(sb + S::kPrev + (k * S::kNA + (kk >> 2)) * S::kAtomRows64 + (kk & 3) * 32),
-                    ssd_idesc(false), kk > 0);
+                    umma_desc_k_sw128(sb + S::kPrev + (k * S::kSA + (kk >> 2)) * S::kAtomRows64 + (kk & 3) * 32),
+                    ssd_idesc(false), t0 > 0 || kk > 0);
   };
   // 2. Carried-state term, as soon as its operands are in: C[l][n] x prev_states[p][n]^T.
-  if (tid == 0 && !kScoresFirst) {
+  //    Reloading: the first atom here, then the buffer is refilled with the
+  //    second while the scores are formed.
+  if (tid == 0 && (S::kReload || !kScoresFirst)) {
     mbar_wait_bounded(full_state, 0u, a.err, 7);
     tcgen05_fence_after();
-    state_mmas();
+    state_mmas(0);
+    if constexpr (S::kReload) {
+      umma_commit(state_free);
+      mbar_wait_bounded(state_free, 0u, a.err, 10);  // the MMAs have read the buffer
+      mbar_arrive_expect_tx(full_state, S::kTxState);
+      load_state(1);
+    }
   }
   for (int i = tid; i < ks; i += kSsdThreads) F[i] = ex2_approx((sdA[i | 7] - sdA[i]) * kLog2e) * sdt[i];
   const int lg = r0 + l;  // this thread's row within its chunk pair / chunk
@@ -300,10 +320,14 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     for (int kk = 0; kk < ks / 16; ++kk)
       umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
                   umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), kk > 0);
-    if (kScoresFirst) {  // carried-state term last: its operands were loaded second
+    if constexpr (S::kReload) {  // the second state atom
+      mbar_wait_bounded(full_state, 1u, a.err, 7);
+      tcgen05_fence_after();
+      state_mmas(1);
+    } else if (kScoresFirst) {  // carried-state term last: its operands were loaded second
       mbar_wait_bounded(full_state, 0u, a.err, 7);
       tcgen05_fence_after();
-      state_mmas();
+      state_mmas(0);
     }
     umma_commit(done);
   }
