@@ -442,7 +442,7 @@ ssm_status ssm_segment_carry(const ssm_dims *dims, const ssm_weights *w, const f
 /* Reads and clears the device error word that kernels set when a bounded
  * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed;
  * SSM_ERR_DEVICE with the code in ssm_last_error() otherwise. Codes: 1 the
- * prefill's TMA ring, 3-6 the block's x_proj kernel, 7-10 the chunk scan's
+ * prefill's TMA ring, 3-6 the block's x_proj kernel, 7-11 the chunk scan's
  * operand and MMA waits, 11 the decode's state ring, 21-29 the projection
  * GEMM (21 ring slot free, 22 accumulator free, 23 operands landed, 24
  * accumulator full, 25 and 29 drains, 27-28 the cut-tile handshake),

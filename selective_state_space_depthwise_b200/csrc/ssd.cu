@@ -8,14 +8,17 @@
 //
 // Both sums are dense contractions and run on the tensor cores, each into its
 // own TMEM accumulator, so that the carried-state term needs no rescaled copy
-// of C and starts as soon as its operands land. One CTA per (b, c, h), 256
-// threads; ~100 KB of shared memory lets two CTAs share an SM:
-//  1. TMA brings, 128-byte swizzled, the C tile [l][n] and the prev_states tile
-//     [p][n] (two 64-column atoms each) on one mbarrier, and the cb tile [l][s]
-//     (two atoms) and the x tile [s][p] on a second one, while threads stage
-//     dA and dt;
-//  2. as soon as C and prev_states are in, one thread issues eight tcgen05 MMAs
-//     C x prev_states^T into accumulator 1;
+// of C and starts as soon as its operands land. One CTA per (b, c, h) (two
+// per chunk of 256, one per two chunks of 64), 256 threads; ~75 KB of shared
+// memory at chunk 128 lets three CTAs share an SM:
+//  1. TMA brings, 128-byte swizzled, the cb tile [l][s] (128 columns, two
+//     atoms) and the x tile [s][p] on one mbarrier, and the first 64-column
+//     atom of the C tile [l][n] and of the prev_states tile [p][n] on a
+//     second, while threads stage dA and dt;
+//  2. as soon as that state atom is in, one thread issues its four tcgen05
+//     MMAs C x prev_states^T into accumulator 1; their commit frees the
+//     buffer, which takes the second atom (state dim 128) while the scores
+//     are formed;
 //  3. meanwhile thread s < 128 forms F[s] = exp(dA[s1] - dA[s]) dt[s], s1 the
 //     last column of s's 8-column group (s1 = s | 7), and thread t turns the
 //     64-column atom t / 128 of row l = t mod 128 of the cb tile, in place,
@@ -31,7 +34,10 @@
 //     made per warp (over its 32 rows), so no branch diverges.
 //     The TMA layout is already the MMA's K-major operand;
 //  4. one thread issues eight MMAs scores x x (x as an MN-major B operand) into
-//     accumulator 0 and commits both;
+//     accumulator 0. The second half of a 256-chunk has 256 score columns: it
+//     runs steps 3-4 twice, on columns 0..127 then 128..255, the buffers
+//     refilled once the first pass's MMAs have read them. Then the last state
+//     atom's MMAs, and one commit for all;
 //  5. warps w and w + 4 read lanes 32 (w mod 4) .. of columns 32 (w / 4) .. of
 //     both accumulators, form acc0 + exp(dA[l]) acc1 + D x, and the bf16 tile
 //     leaves by TMA store from the (now free) cb buffer.
@@ -72,13 +78,15 @@ struct SsdSmem {
   static_assert(CS == 64 || CS == 128 || CS == 256, "chunk 64, 128 or 256");
   static constexpr int kNC = CS < kCs ? kCs / CS : 1;  // chunks per CTA (stacked on the tile diagonal)
   static constexpr int kHalves = CS > kCs ? CS / kCs : 1;  // CTAs per chunk (128-row halves)
-  static constexpr int kKS = CS > kCs ? CS : kCs;      // most score columns = rows of x = K of the intra term
+  static constexpr int kCols = CS > kCs ? CS : kCs;    // most score columns = rows of x = K of the intra term
+  static constexpr int kKS = kCs;                      // score columns (and rows of x) staged per pass
   static constexpr int kNA = DS / 64;                  // 64-column atoms across the state dim
-  // State dim 128 at chunk 64 or 128: the carried-state operands are loaded
-  // one 64-column atom at a time into one buffer (the first atom's MMAs free
-  // it for the second). That brings a chunk-128 CTA to ~75 KB (three CTAs per
-  // SM instead of two) and a chunk-64 CTA to ~84 KB (two instead of one).
-  static constexpr bool kReload = kNA == 2 && CS <= kCs;
+  // State dim 128: the carried-state operands are loaded one 64-column atom
+  // at a time into one buffer (the first atom's MMAs free it for the
+  // second). With the 128-column score passes below, that brings a chunk-128
+  // or chunk-256 CTA to ~75 KB (three CTAs per SM) and a chunk-64 CTA to
+  // ~84 KB (two).
+  static constexpr bool kReload = kNA == 2;
   static constexpr int kSA = kReload ? 1 : kNA;        // state atoms resident at once
   static constexpr int kAtomRows128 = kCs * 128;       // one 64-column atom of a 128-row tile
   static constexpr int kAtomRows64 = kHd * 128;        // one 64-column atom of a 64-row tile
@@ -87,19 +95,17 @@ struct SsdSmem {
   static constexpr int kX = kC + kSA * kAtomRows128;   // x [kKS][p] (B of MMA 1, MN-major)
   static constexpr int kPrev = kX + kKS * 128;         // prev_states [chunk][p][n] (B of MMA 2, K-major)
   static constexpr int kDA = kPrev + kNC * kSA * kAtomRows64;
-  static constexpr int kDt = kDA + kKS * 4;
-  static constexpr int kF = kDt + kKS * 4;
-  static constexpr int kBar = kF + kKS * 4;            // full_state, full_scores, done, state_free
-  static constexpr int kTmemSlot = kBar + 32;
+  static constexpr int kDt = kDA + kCols * 4;
+  static constexpr int kF = kDt + kCols * 4;
+  static constexpr int kBar = kF + kCols * 4;          // full_state, full_scores, done, state_free, pass_free
+  static constexpr int kTmemSlot = kBar + 40;
   static constexpr int kTotal = kTmemSlot + 16;
   // C and prev_states bytes of one load round (all atoms, or one when reloading)
   static constexpr uint32_t kTxState = static_cast<uint32_t>(kSA * (kAtomRows128 + kNC * kAtomRows64));
-  // cb and x of a CTA whose score tile is ks columns wide (ks = 128, or 256 for
-  // the second half of a 256-chunk): stacked chunks load their [CS][CS]
-  // diagonal blocks, otherwise 128 rows x ks columns; x has ks rows.
-  static __host__ __device__ constexpr uint32_t tx_scores(int ks) {
-    return static_cast<uint32_t>((kNC > 1 ? kNC * CS * CS * 2 : kCs * ks * 2) + ks * 128);
-  }
+  // cb and x of one score pass: stacked chunks load their [CS][CS] diagonal
+  // blocks, otherwise 128 rows x 128 columns; x has 128 rows.
+  static constexpr uint32_t kTxScores =
+      static_cast<uint32_t>((kNC > 1 ? kNC * CS * CS * 2 : kCs * kKS * 2) + kKS * 128);
   static constexpr uint32_t kTmemCols = kNC == 1 ? 128u : 256u;  // intra + one carried-state term per chunk
   static_assert(kC % 1024 == 0 && kX % 1024 == 0 && kPrev % 1024 == 0, "swizzled tiles need 1 KB");
 };
@@ -164,7 +170,8 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   const int64_t t_chunk = static_cast<int64_t>(c) * CS;  // first token of chunk c
   const int g = static_cast<int>(h / (a.nheads / a.ngroups));
   const uint32_t full_state = sb + S::kBar, full_scores = sb + S::kBar + 8, done = sb + S::kBar + 16;
-  const uint32_t state_free = sb + S::kBar + 24;
+  const uint32_t state_free = sb + S::kBar + 24, pass_free = sb + S::kBar + 32;
+  const int np = ks / kCs;  // score passes: 2 for the second half of a 256-chunk, else 1
   const int64_t zp0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.nheads + h;
   // State atoms [t0, t0 + kSA) of C and prev_states into the state buffers.
   auto load_state = [&](int t0) {
@@ -178,41 +185,45 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
                     static_cast<int>(zp0 + k * a.nheads), full_state);
     }
   };
+  // A second stacked chunk past the last one (odd chunk count) reads zeros
+  // or a neighbouring sequence's chunk; its rows lie past L and are never stored.
+  const int64_t zc0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g;
+  // Score pass p: cb columns 128 p .. 128 p + 127 of this CTA's 128 rows and
+  // x rows 128 p .. of the chunk into the score buffers.
+  auto load_scores = [&](int p) {
+    if constexpr (NC == 1) {
+#pragma unroll
+      for (int t = 0; t < S::kKS / 64; ++t)  // rows r0 .. r0 + 127, columns 128 p + 64 t ..
+        tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, kCs * p + 64 * t, r0, static_cast<int>(zc0),
+                    full_scores);
+    } else {
+      // chunk k's [CS][CS] block on the diagonal: atom k, rows CS k ..
+#pragma unroll
+      for (int k = 0; k < NC; ++k)
+        tma_load_3d(sb + S::kCb + k * S::kAtomRows128 + k * CS * 128, &map_cb, 0, 0,
+                    static_cast<int>(zc0 + k * a.ngroups), full_scores);
+    }
+    tma_load_4d(sb + S::kX, &map_x, 0, h, static_cast<int>(t_chunk + kCs * p), b, full_scores);
+  };
   if (tid == 0) {
     mbar_init(full_state, 1);
     mbar_init(full_scores, 1);
     mbar_init(done, 1);
     mbar_init(state_free, 1);
+    mbar_init(pass_free, 1);
     mbar_fence_init();
     prefetch_tensormap(&map_cb);
     prefetch_tensormap(&map_x);
     prefetch_tensormap(&map_c);
     prefetch_tensormap(&map_prev);
-    // A second stacked chunk past the last one (odd chunk count) reads zeros
-    // or a neighbouring sequence's chunk; its rows lie past L and are never stored.
-    const int64_t zc0 = (static_cast<int64_t>(b) * a.nchunks + c) * a.ngroups + g;
     mbar_arrive_expect_tx(full_state, S::kTxState);
-    mbar_arrive_expect_tx(full_scores, S::tx_scores(ks));
-    auto load_scores = [&] {
-      if constexpr (NC == 1) {
-        for (int t = 0; t < ks / 64; ++t)  // rows r0 .. r0 + 127, columns 64 t ..
-          tma_load_3d(sb + S::kCb + t * S::kAtomRows128, &map_cb, 64 * t, r0, static_cast<int>(zc0), full_scores);
-      } else {
-        // chunk k's [CS][CS] block on the diagonal: atom k, rows CS k ..
-#pragma unroll
-        for (int k = 0; k < NC; ++k)
-          tma_load_3d(sb + S::kCb + k * S::kAtomRows128 + k * CS * 128, &map_cb, 0, 0,
-                      static_cast<int>(zc0 + k * a.ngroups), full_scores);
-      }
-      for (int t = 0; t < ks / kCs; ++t)  // x rows 128 t .. of the chunk
-        tma_load_4d(sb + S::kX + t * kCs * 128, &map_x, 0, h, static_cast<int>(t_chunk + kCs * t), b, full_scores);
-    };
+    mbar_arrive_expect_tx(full_scores, S::kTxScores);
     if (kScoresFirst) {
-      load_scores();
+      load_scores(0);
       load_state(0);
     } else {
       load_state(0);
-      load_scores();
+      load_scores(0);
     }
   }
   if (warp == 0) {
@@ -271,8 +282,9 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   mbar_wait_bounded(full_scores, 0u, a.err, 8);
   __syncthreads();  // F complete
 
-  // 3. Row l of the cb tile -> scores (in place), atoms at, at + 2, .. of the
-  //    ks columns. A warp's 32 rows lie in one chunk, starting at column
+  // 3. Row l of the cb tile -> scores (in place), one pass of 128 columns at a
+  //    time (two passes only for the second half of a 256-chunk), this
+  //    thread's 64-column atom `at` of each. A warp's 32 rows lie in one chunk, starting at column
   //    warp_min_s. Groups are classified against the warp's whole row span,
   //    so every branch below is warp-uniform: groups wholly at or below all 32
   //    rows take the two-factor product with no masking; the four groups the
@@ -284,42 +296,59 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   const int warp_min_s = CS < kCs ? (32 * (warp & 3)) & ~(CS - 1) : 0;
   const int sd = lg & ~7;
   const bool strong = __any_sync(0xffffffffu, sdA[sd] - sdA[sd + 7] >= 80.0f);
-  for (int aa = at; aa < ks / 64; aa += 2) {
+  for (int pass = 0; pass < np; ++pass) {
+    if (pass > 0) mbar_wait_bounded(full_scores, static_cast<uint32_t>(pass) & 1u, a.err, 8);
+    // This thread's 64-column atom of the pass: columns 128 pass + 64 at ..
+    {
+      const int aa = 2 * pass + at;  // atom index over the chunk's columns
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int s0 = 64 * aa + 8 * j;
-      uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + aa * S::kAtomRows128 + sw128(l, j));
-      if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
-        *p = make_uint4(0u, 0u, 0u, 0u);
-        continue;
+      for (int j = 0; j < 8; ++j) {
+        const int s0 = 64 * aa + 8 * j;
+        uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
+        if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
+          *p = make_uint4(0u, 0u, 0u, 0u);
+          continue;
+        }
+        float f[8];
+        unpack8(*p, f);
+        if (s0 + 7 <= warp_min_l) {  // wholly at or below the diagonal for every row: row factor x column factor
+          const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
+        } else if (!strong) {  // straddled by the warp's rows: masked two-factor form
+          const float e = s0 <= lg ? ex2_approx((dAl - sdA[s0 + 7]) * kLog2e) : 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
+        } else {  // masked, each decay on its own
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
+        }
+        *p = pack8(f);
       }
-      float f[8];
-      unpack8(*p, f);
-      if (s0 + 7 <= warp_min_l) {  // wholly at or below the diagonal for every row: row factor x column factor
-        const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+    }
+    fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
+    __syncthreads();
+
+    // 4. Intra-chunk term of the pass: scores[l][s] x x[s][p], s in steps of
+    //    16 rows of x. Before a second pass the buffers are refilled once
+    //    these MMAs have read them.
+    if (tid == 0) {
+      tcgen05_fence_after();
 #pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
-      } else if (!strong) {  // straddled by the warp's rows: masked two-factor form
-        const float e = s0 <= lg ? ex2_approx((dAl - sdA[s0 + 7]) * kLog2e) : 0.0f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
-      } else {  // masked, each decay on its own
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
+      for (int kk = 0; kk < S::kKS / 16; ++kk)
+        umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+                    umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), pass > 0 || kk > 0);
+      if (pass + 1 < np) {
+        umma_commit(pass_free);
+        mbar_wait_bounded(pass_free, static_cast<uint32_t>(pass) & 1u, a.err, 11);
+        mbar_arrive_expect_tx(full_scores, S::kTxScores);
+        load_scores(pass + 1);
       }
-      *p = pack8(f);
     }
   }
-  fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
-  __syncthreads();
-
-  // 4. Intra-chunk term: scores[l][s] x x[s][p], s in steps of 16 rows of x; one commit for both.
+  // The carried-state term (its last atom) and one commit for everything.
   if (tid == 0) {
-    tcgen05_fence_after();
-    for (int kk = 0; kk < ks / 16; ++kk)
-      umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
-                  umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), kk > 0);
     if constexpr (S::kReload) {  // the second state atom
       mbar_wait_bounded(full_state, 1u, a.err, 7);
       tcgen05_fence_after();
@@ -352,7 +381,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
       for (int half = 0; half < 2; ++half) {
         const int j = (col0 + 16 * jj) / 8 + half;  // 16-byte chunk of the row: p = 8 j .. 8 j + 7
         float xv[8], o[8];
-        unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(r0 + row, j)), xv);
+        unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(row, j)), xv);  // the last pass's x rows
 #pragma unroll
         for (int q = 0; q < 8; ++q)
           o[q] = fmaf(Dh, xv[q], fmaf(el, __uint_as_float(r1v[8 * half + q]), __uint_as_float(r0v[8 * half + q])));
