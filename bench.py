@@ -802,7 +802,11 @@ def main():
     peak_ct = alu_peak_ct_per_s(1965.0, "power")
 
     extra = {}
-    if rank == 0:
+    # The sub-benchmarks (decay paths, configs, decode, block, GEMMs, chunk
+    # scan, sequence-parallel pieces, CPU baseline) run only in a 1-GPU run:
+    # with N ranks they would hold every GPU while rank 0 alone works.
+    subs = world == 1
+    if subs:
         extra["decay_paths"] = decay_path_bench(w, inp, hbm_peak, peak_kind)
     if not args.no_e2e:
         # Every rank moves its own inputs through the host path at the same time;
@@ -818,7 +822,7 @@ def main():
             e2e["h2d_bytes_per_step"] *= world
             e2e["d2h_bytes_per_step"] *= world
         extra["e2e"] = e2e
-    if rank == 0:
+    if subs:
         del inp
         torch.cuda.empty_cache()
         if not args.no_configs:
@@ -839,7 +843,7 @@ def main():
         if not args.no_seqpar:
             torch.cuda.empty_cache()
             extra["sequence_parallel"] = seqpar_bench(w)
-        if not args.no_cpu and world == 1:
+        if not args.no_cpu:
             extra["cpu_baseline"] = cpu_baseline(w)
             extra["cpu_baseline"]["single_core_layer_shape"] = cpu_single_core(W.WORKLOADS["axon_layer"])
     if dist:
