@@ -24,6 +24,8 @@
 // loads 74 us.
 #include <cuda_bf16.h>
 
+#include <atomic>
+
 #include "sm100_ptx.cuh"
 #include "ssm_internal.h"
 #include "ssm_math.cuh"
@@ -222,6 +224,12 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_tma_kernel(const __grid
   const int e0 = static_cast<int>(blockIdx.x) * kDecodeThreads;
   const int64_t e = e0 + tid;
   const bool active = e < a.E;
+  // Launched with programmatic stream serialisation: everything global is
+  // read after the previous grid on the stream (typically the last step,
+  // which wrote the state and caches) has completed; the next step may be
+  // scheduled at once, so its launch overlaps this one.
+  griddep_wait();
+  griddep_launch_dependents();
   ChannelParams p;
   if (active) {
     const float4* Al = reinterpret_cast<const float4*>(a.A_log) + e * 4;
@@ -360,11 +368,11 @@ cudaError_t launch(const KernelArgs& a, cudaStream_t st) {
   const int64_t bx = (a.E + kDecodeThreads - 1) / kDecodeThreads;
   if (bx > 0x7fffffff) return cudaErrorInvalidConfiguration;
   // Every block resident at once: gridDim.y = resident blocks / channel blocks.
-  static int resident[64] = {};
+  static std::atomic<int> resident[64] = {};  // per device: blocks resident at once (0 = not yet known)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  int& per_sm = resident[dev & 63];
+  int per_sm = resident[dev & 63].load();
   if (per_sm == 0) {
     int sms = 0;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
@@ -373,6 +381,7 @@ cudaError_t launch(const KernelArgs& a, cudaStream_t st) {
                                                              0)) != cudaSuccess)
       return err;
     per_sm = (blocks > 0 ? blocks : 1) * (sms > 0 ? sms : 148);
+    resident[dev & 63].store(per_sm);
   }
   int64_t by = per_sm / bx;
   if (by < 1) by = 1;
@@ -395,11 +404,11 @@ cudaError_t launch_tma(const KernelArgs& a, cudaStream_t st) {
     return cudaErrorInvalidValue;
   auto kern = decode_tma_kernel<T, ZOH>;
   const int smem = TmaSmem::kTotal + 1024;
-  static int resident[64] = {};
+  static std::atomic<int> resident[64] = {};  // per device: blocks resident at once (0 = not yet known)
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
-  int& per_sm = resident[dev & 63];
+  int per_sm = resident[dev & 63].load();
   if (per_sm == 0) {
     if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return err;
     int sms = 0, blocks = 0;
@@ -407,12 +416,24 @@ cudaError_t launch_tma(const KernelArgs& a, cudaStream_t st) {
     if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kDecodeThreads, smem)) != cudaSuccess)
       return err;
     per_sm = (blocks > 0 ? blocks : 1) * (sms > 0 ? sms : 148);
+    resident[dev & 63].store(per_sm);
   }
   int64_t by = per_sm / bx;
   if (by < 1) by = 1;
   if (by > a.batch) by = a.batch;
   if (by > 65535) by = 65535;
-  kern<<<dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by)), kDecodeThreads, smem, st>>>(map_h, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(bx), static_cast<unsigned>(by));
+  cfg.blockDim = dim3(kDecodeThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the launch with the previous step
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, map_h, a);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
