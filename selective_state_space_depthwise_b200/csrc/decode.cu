@@ -19,9 +19,12 @@
 // set of sequences, so the channel's parameters are read and A = -exp(A_log)
 // computed once; B, C and dt_raw are staged in shared memory 32 sequences at
 // a time; the grid is sized so that every block is resident at once.
+// The TMA form is launched with programmatic stream serialisation, so each
+// step is scheduled while the previous one runs (it waits for it before its
+// first global read).
 // Measured on B200 at b = 256, E = 7680: TMA form 54.8 us per step (5.25 TB/s),
-// register form 59.3 us, one thread per (sequence, channel) with per-item
-// loads 74 us.
+// 53.0 us with the overlapped launch; register form 59.3 us; one thread per
+// (sequence, channel) with per-item loads 74 us.
 #include <cuda_bf16.h>
 
 #include <atomic>
