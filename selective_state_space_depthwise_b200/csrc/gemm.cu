@@ -33,9 +33,10 @@
 // waves), the final one to two tiles a pair are instead cut along K into
 // equal runs of K chunks, one per pair (stream-K):
 // a tile cut between pairs has every contributing CTA write its fp32 partial
-// and count itself in; the one that completes the count sums all partials in
-// pair order (so the result does not depend on who came last) and stores the
-// tile. No CTA waits on another pair.
+// and count itself in; the one that completes the count adds the other's
+// partial to its own accumulator (two contributors) or sums all partials in
+// pair order (more), so the result does not depend on who came last, and
+// stores the tile. No CTA waits on another pair.
 // Tails: TMA loads past M, N or K read zeros; stores are clipped at M and N.
 // Every mbarrier wait is bounded; a wait that gives up sets the device error
 // word and the CTA's abort flag, every role leaves its loop, the waits that
@@ -365,16 +366,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          } else {
+          } else if (p_hi - p_lo == 1) {
+            // Two contributors: this CTA's own accumulator plus the other's
+            // partial (a + b == b + a, so the sum does not depend on which
+            // contributor came last), one partial read instead of two.
+            const int other = pair == p_lo ? p_hi : p_lo;
+            const float4* src = reinterpret_cast<const float4*>(g.partial) +
+                                partial_index(other, sk_slot(g, other, tl), half, q, c, 0, lane);
+            float4 pv[8];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-            for (int p = p_lo; p <= p_hi; ++p) {
+            for (int j = 0; j < 8; ++j) pv[j] = __ldcg(src + j * 32);
+            uint32_t r[32];
+            tmem_ld_x32(t_row + 32 * c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              v[4 * j] = __uint_as_float(r[4 * j]) + pv[j].x;
+              v[4 * j + 1] = __uint_as_float(r[4 * j + 1]) + pv[j].y;
+              v[4 * j + 2] = __uint_as_float(r[4 * j + 2]) + pv[j].z;
+              v[4 * j + 3] = __uint_as_float(r[4 * j + 3]) + pv[j].w;
+            }
+          } else {
+            // Three or more: every partial, in pair order; the next
+            // contributor's loads are in flight while the current one is added.
+            auto fetch = [&](int p, float4 (&dst)[8]) {
               const float4* src =
                   reinterpret_cast<const float4*>(g.partial) + partial_index(p, sk_slot(g, p, tl), half, q, c, 0, lane);
 #pragma unroll
+              for (int j = 0; j < 8; ++j) dst[j] = __ldcg(src + j * 32);
+            };
+            float4 cur[8], nxt[8];
+            fetch(p_lo, cur);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+            for (int p = p_lo; p <= p_hi; ++p) {
+              if (p < p_hi) fetch(p + 1, nxt);
+#pragma unroll
               for (int j = 0; j < 8; ++j) {
-                const float4 pv = __ldcg(src + j * 32);
-                v[4 * j] += pv.x, v[4 * j + 1] += pv.y, v[4 * j + 2] += pv.z, v[4 * j + 3] += pv.w;
+                v[4 * j] += cur[j].x, v[4 * j + 1] += cur[j].y, v[4 * j + 2] += cur[j].z, v[4 * j + 3] += cur[j].w;
+                cur[j] = nxt[j];
               }
             }
           }

@@ -107,13 +107,17 @@ def test_gemm_tiles_cut_along_k(shape):
 def test_gemm_layer_shapes_sampled_rows(which):
     """The block's projections at the Axon layer shape (2048 tokens, D = 2560,
     E = 7680): every column of 96 sampled rows against the float64 reference,
-    and the full output finite."""
+    the full output finite, and two calls bit-equal (out_proj cuts its tiles
+    between two CTA pairs; the one that finishes last adds the other's partial
+    to its own accumulator, which gives the same sum either way)."""
     M, D, E = 2048, 2560, 7680
     N, K = (2 * E, D) if which == "in_proj" else (D, E)
     A, W = operands(M, N, K, seed=7 if which == "in_proj" else 8)
     C = api.proj_gemm(A.cuda(), W.cuda())
+    C2 = api.proj_gemm(A.cuda(), W.cuda())
     torch.cuda.synchronize()
     assert torch.isfinite(C).all()
+    assert torch.equal(C, C2)
     rows = np.sort(np.random.default_rng(3).choice(M, 96, replace=False))
     rows[0], rows[-1] = 0, M - 1
     e = rel_l2(C[torch.from_numpy(rows).cuda()].double().cpu().numpy(), reference(A, W, rows))

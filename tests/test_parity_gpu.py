@@ -209,6 +209,32 @@ def test_decode_continues_prefill(L0, io_dtype):
     compare(io_dtype, gather(y, cc, st, chans), oracle_prefill(inp, chans), label=f"decode L0={L0}")
 
 
+def test_decode_inputs_written_just_before_each_step():
+    """Each decode step is launched so that it may be scheduled while the
+    kernel before it runs; it must still read its inputs only after that
+    kernel finished. Here a long matmul and then a kernel that writes the
+    step's x, z, B, C and dt_raw run right before every step; the outputs and
+    caches must equal, bit for bit, those of decoding straight from the source
+    tensors."""
+    w = small_workload(torch.bfloat16, b=64, L=4 + 24, E=512, seed=73)
+    inp = device_inputs(w)
+    L0, steps = 4, 24
+    y_ref, cc_ref, st_ref = decode_run(inp, w, L0, steps)
+    pre = {**inp, **{k: inp[k][:, :L0] for k in ("x", "z", "B", "C", "dt_raw")}}
+    _, cc, st = api.prefill(pre["x"], pre["z"], pre["B"], pre["C"], pre["dt_raw"], pre)
+    y = torch.empty_like(y_ref)
+    y[:, :L0] = y_ref[:, :L0]
+    big = torch.randn((4096, 4096), device="cuda", dtype=torch.bfloat16)
+    bufs = {k: torch.empty_like(inp[k][:, 0]) for k in ("x", "z", "B", "C", "dt_raw")}
+    for t in range(L0, L0 + steps):
+        zero = (big @ big).float().sum() * 0.0  # a long kernel, then the writes depend on it
+        for k, v in bufs.items():
+            v.copy_(inp[k][:, t] + zero.to(v.dtype))
+        api.decode_step(bufs["x"], bufs["z"], bufs["B"], bufs["C"], bufs["dt_raw"], inp, cc, st, y=y[:, t])
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref) and torch.equal(cc, cc_ref) and torch.equal(st, st_ref)
+
+
 def test_decode_zoh():
     w = small_workload(torch.bfloat16, b=2, L=20, E=16, seed=71)
     inp = device_inputs(w)
