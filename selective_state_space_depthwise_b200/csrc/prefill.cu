@@ -22,12 +22,14 @@
 // Each 32-token stage:
 //  A. warp j does the per-token work of tokens [32j/G, 32(j+1)/G) of its
 //     lane's channel (conv from a sliding window of x, SiLU, dt, D*u,
-//     SiLU(z)); the per-token decay operand and dt*u go to shared memory as
-//     token-pair rows, D*u and SiLU(z) stay in registers;
+//     SiLU(z)) two tokens at a time on f32x2 operations; the per-token decay
+//     operand and dt*u go to shared memory as token-pair rows, D*u and
+//     SiLU(z) stay in registers;
 //  B. every warp streams its state slice through all 32 tokens (packed f32x2
 //     multiplies and FMAs) and keeps the partial readouts C.h in registers;
 //  C. warp j sums the G partials of its phase-A tokens, applies the skip and
-//     the gate, and fills an output tile that leaves by TMA store.
+//     the gate (again two tokens per f32x2 operation), and fills an output
+//     tile that leaves by TMA store.
 // Phase A of stage s+1 runs inside phase B of stage s (software pipelining),
 // so every warp has two independent instruction streams.
 //
@@ -52,6 +54,13 @@
 // exponentials and the B/C loads then saturate the shared MIO queue. A power
 // path forming each slice's first two decays as exponentials (two per slice
 // and token, no power chain) ran 1.14x slower: SFU latency on the scan chain.
+// Doing phases A and C on token pairs (f32x2) cut the executed instructions
+// by 12%: 8% off the batched shape and 5% off the per-state path, but under 1%
+// off the long-context power path, which is bound by dependency latency at
+// two warps per SM sub-partition, not by issue slots. One-warp CTAs over 8
+// channels (960 CTAs for E = 7680, six or seven warps on every SM instead of
+// kernel 4's eight or four) ran 5% slower there: per-lane slice arithmetic
+// adds 9% instructions and the warps' latency is no better hidden.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -194,55 +203,107 @@ __device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* 
 // dt (ZOH, with u instead of dt*u as the second value).
 enum class Path { kGeneric, kPow, kZoh };
 
-// Per-token work of kTA tokens [tb, tb+kTA) of this lane's channel for one
-// stage: the (decay operand, injection) of token pairs, D*u and SiLU(z) to
-// registers. Dr is the stage's dt_raw row. The caller stores the pairs
-// (store_rows) after the scan, so no shared-memory store sits between the
-// scan's loads in program order.
+// Two tokens per f32x2 operation. The packed forms round exactly as the scalar
+// ones (same operations in the same order), so both give the same bits.
+__device__ __forceinline__ uint64_t splat2(float v) { return pk2(v, v); }
+
+__device__ __forceinline__ uint64_t ex2_pair(uint64_t x) {
+  float x0, x1;
+  upk2(x, x0, x1);
+  return pk2(ex2_approx(x0), ex2_approx(x1));
+}
+
+// SiLU of both halves: v / (1 + 2^(-v log2 e)).
+__device__ __forceinline__ uint64_t silu_pair(uint64_t v) {
+  const uint64_t e = ex2_pair(fmul2(v, splat2(-kLog2e)));
+  float d0, d1;
+  upk2(fadd2(e, splat2(1.0f)), d0, d1);
+  return fmul2(v, pk2(rcp_approx(d0), rcp_approx(d1)));
+}
+
+// clip(softplus(v), lo, hi) of both halves (softplus as in dt_of).
+__device__ __forceinline__ uint64_t dt_pair(uint64_t v, float lo, float hi) {
+  float v0, v1;
+  upk2(v, v0, v1);
+  const uint64_t e = pk2(ex2_approx(-fabsf(v0) * kLog2e), ex2_approx(-fabsf(v1) * kLog2e));
+  uint64_t q = ffma2(e, splat2(log1p_q(0)), splat2(log1p_q(1)));
+#pragma unroll
+  for (int k = 2; k <= kLog1pDeg; ++k) q = ffma2(e, q, splat2(log1p_q(k)));
+  float s0, s1;
+  upk2(fadd2(pk2(fmaxf(v0, 0.0f), fmaxf(v1, 0.0f)), fmul2(e, q)), s0, s1);
+  return pk2(fminf(fmaxf(s0, lo), hi), fminf(fmaxf(s1, lo), hi));
+}
+
+// Rows of tokens at or past L (last stage only) become the row of a token that
+// keeps the state: decay 1 (or dt 0) and no injection.
+template <Path P, int kTA>
+__device__ __forceinline__ void fix_rows(float4* rows, int64_t t0, int64_t L, int tb) {
+  if (t0 + tb + kTA > L) {
+    constexpr float kKeep = P == Path::kPow ? 1.0f : 0.0f;  // q = 1, or dt = 0
+#pragma unroll
+    for (int p = 0; p < kTA / 2; ++p) {
+      const int64_t t = t0 + tb + 2 * p;
+      if (t >= L) rows[p].x = kKeep, rows[p].z = 0.0f;
+      if (t + 1 >= L) rows[p].y = kKeep, rows[p].w = 0.0f;
+    }
+  }
+}
+
+// Per-token work of tokens [tb, tb + kTA) of this lane's channel for one
+// stage, as kTA / 2 token pairs that share each f32x2 operation. Outputs per
+// pair: the row (d, d', inj, inj') of decay operands and injections, D*u and
+// SiLU(z). Dr is the stage's dt_raw row. Tokens at or past L get the row of a
+// token that changes nothing (decay 1, no injection). The caller stores the
+// rows (store_rows) after the scan, so no shared-memory store sits between
+// the scan's loads in program order.
 template <typename T, Path P, int kTA>
 __device__ __forceinline__ void phase_a(const T* __restrict__ X, const T* __restrict__ Z, const float* __restrict__ Dr,
                                         int64_t t0, int64_t L, int tb, int lane, bool first, float hx0, float hx1,
                                         float hx2, float cw0, float cw1, float cw2, float cw3, float cb, float wdt,
-                                        float dtb, float Dd, float lo, float hi, float a20, float4* rows, float* du,
-                                        float* zg) {
-  float xw[kTA + 3], zr[kTA], dr[kTA];
+                                        float dtb, float Dd, float lo, float hi, float a20, float4* rows, uint64_t* du2,
+                                        uint64_t* zg2) {
+  float xw[kTA + 3];
 #pragma unroll
   for (int i = 0; i < kTA + 3; ++i) {
     const int r = tb + i;
     xw[i] = (first && r < 3) ? (r == 0 ? hx0 : (r == 1 ? hx1 : hx2)) : IO<T>::to_f(X[r * 32 + lane]);
   }
 #pragma unroll
-  for (int i = 0; i < kTA; ++i) zr[i] = IO<T>::to_f(Z[(tb + i) * 32 + lane]);
-#pragma unroll
-  for (int i = 0; i < kTA; i += 4) {
-    const float4 v = *reinterpret_cast<const float4*>(Dr + tb + i);  // broadcast
-    dr[i] = v.x, dr[i + 1] = v.y, dr[i + 2] = v.z, dr[i + 3] = v.w;
-  }
-  float2 dtv[kTA];
-#pragma unroll
-  for (int i = 0; i < kTA; ++i) {
-    const float conv = fmaf(cw3, xw[i + 3], fmaf(cw2, xw[i + 2], fmaf(cw1, xw[i + 1], fmaf(cw0, xw[i], cb))));
-    const float u = silu(conv);
-    float dt = dt_of(fmaf(dr[i], wdt, dtb), lo, hi);
-    if (t0 + tb + i >= L) dt = 0.0f;  // past the end: keep the state (q = 1, no injection)
+  for (int p = 0; p < kTA / 2; ++p) {
+    const int t = tb + 2 * p;  // first token of the pair, from the stage start
+    const float* x = xw + 2 * p;
+    const float c0 = fmaf(cw3, x[3], fmaf(cw2, x[2], fmaf(cw1, x[1], fmaf(cw0, x[0], cb))));
+    const float c1 = fmaf(cw3, x[4], fmaf(cw2, x[3], fmaf(cw1, x[2], fmaf(cw0, x[1], cb))));
+    const float2 dr = *reinterpret_cast<const float2*>(Dr + t);  // broadcast
+    const float z0 = IO<T>::to_f(Z[t * 32 + lane]), z1 = IO<T>::to_f(Z[(t + 1) * 32 + lane]);
+    const uint64_t u2 = silu_pair(pk2(c0, c1));
+    const uint64_t dt2 = dt_pair(ffma2(pk2(dr.x, dr.y), splat2(wdt), splat2(dtb)), lo, hi);
+    uint64_t r1, r2;
     if constexpr (P == Path::kPow)
-      dtv[i] = make_float2(ex2_approx(dt * a20), dt * u);
+      r1 = ex2_pair(fmul2(dt2, splat2(a20)));
     else
-      dtv[i] = make_float2(dt, P == Path::kZoh ? u : dt * u);
-    du[i] = Dd * u;
-    zg[i] = silu(zr[i]);
+      r1 = dt2;
+    if constexpr (P == Path::kZoh)
+      r2 = u2;
+    else
+      r2 = fmul2(dt2, u2);
+    float a0, a1, b0, b1;
+    upk2(r1, a0, a1);
+    upk2(r2, b0, b1);
+    rows[p] = make_float4(a0, a1, b0, b1);
+    du2[p] = fmul2(splat2(Dd), u2);
+    zg2[p] = silu_pair(pk2(z0, z1));
   }
-#pragma unroll
-  for (int i = 0; i < kTA; i += 2) rows[i / 2] = make_float4(dtv[i].x, dtv[i].y, dtv[i + 1].x, dtv[i + 1].y);
+  fix_rows<P, kTA>(rows, t0, L, tb);
 }
 
-// Rows as [token pair][channel] (d, inj, d', inj'): one 16-byte load per two
+// Rows as [token pair][channel] (d, d', inj, inj'): one 16-byte load per two
 // tokens in phase B.
 template <int kTA>
 __device__ __forceinline__ void store_rows(float2* DTo, int tb, int lane, const float4* rows) {
   float4* DT4 = reinterpret_cast<float4*>(DTo);
 #pragma unroll
-  for (int i = 0; i < kTA; i += 2) DT4[((tb + i) >> 1) * 32 + lane] = rows[i / 2];
+  for (int p = 0; p < kTA / 2; ++p) DT4[((tb >> 1) + p) * 32 + lane] = rows[p];
 }
 
 // Phase B over tokens [T0, T1) of one stage: this thread's 4 states; pr gets
@@ -254,7 +315,7 @@ __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int l
 #pragma unroll
   for (int tl = T0; tl < T1; ++tl) {
     const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
-    const float2 dd = (tl & 1) ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+    const float2 dd = (tl & 1) ? make_float2(d4.y, d4.w) : make_float2(d4.x, d4.z);
     if constexpr (P == Path::kZoh)
       pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
     else if constexpr (P == Path::kPow)
@@ -262,6 +323,22 @@ __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int l
     else
       pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
   }
+}
+
+// Phase C for 4 consecutive tokens of one channel: the sum of the NS slices'
+// partial readouts (slice j at Pj + j * stride), plus D*u, times SiLU(z).
+template <int NS, int stride>
+__device__ __forceinline__ void gate_pairs(const float* Pj, const uint64_t* du, const uint64_t* zg, float* ys) {
+  const float4 a4 = *reinterpret_cast<const float4*>(Pj);
+  uint64_t lo = pk2(a4.x, a4.y), hi = pk2(a4.z, a4.w);
+#pragma unroll
+  for (int j = 1; j < NS; ++j) {
+    const float4 v = *reinterpret_cast<const float4*>(Pj + j * stride);
+    lo = fadd2(lo, pk2(v.x, v.y));
+    hi = fadd2(hi, pk2(v.z, v.w));
+  }
+  upk2(fmul2(fadd2(lo, du[0]), zg[0]), ys[0], ys[1]);
+  upk2(fmul2(fadd2(hi, du[1]), zg[1]), ys[2], ys[3]);
 }
 
 // The whole walk over L for one CTA of G warps, on the decay path P. Two
@@ -353,7 +430,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
   const int tb = warp * kTA;
 
   // Prologue: phase A of stage 0.
-  float du[kTA], zg[kTA];
+  uint64_t du[kTA / 2], zg[kTA / 2];  // D*u and SiLU(z) of token pairs
   {
     float4 rows0[kTA / 2];
     mbar_wait_bounded(full0, 0u, a.err, 1);
@@ -372,13 +449,14 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     float2* DTn = DT + ((s + 1) & 1) * kTok * 32;
     const int64_t t0 = s * kTok;
     const bool has_next = s + 1 < n_stages;
-    float duN[kTA], zgN[kTA];
+    uint64_t duN[kTA / 2], zgN[kTA / 2];
     float* P_ = reinterpret_cast<float*>(smem + S::kP + (SPLIT ? (s & 1) * S::kPBytes : 0));
     // dt_raw of stage s + 2 into the buffer that phase A of stage s (block s - 1) has finished with
     if (warp == 0) copy_dt_raw(s + 2);
 
     // Phase B of stage s fused with phase A of stage s + 1.
     float pr[kTok];
+    float* Pj = P_ + (warp * 32 + lane) * S::kPR;  // this thread's partial readouts
     if (has_next) {
       const int nslot = static_cast<int>((s + 1) % kPipeStages);
       mbar_wait_bounded(full0 + 8 * nslot, static_cast<uint32_t>(((s + 1) / kPipeStages) & 1), a.err, 1);
@@ -395,12 +473,9 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     } else {
       scan_stage<P, kK>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
     }
-    {
-      float* Pj = P_ + (warp * 32 + lane) * S::kPR;
 #pragma unroll
-      for (int tl = 0; tl < kTok; tl += 4)
-        *reinterpret_cast<float4*>(Pj + tl) = make_float4(pr[tl], pr[tl + 1], pr[tl + 2], pr[tl + 3]);
-    }
+    for (int tl = 0; tl < kTok; tl += 4)
+      *reinterpret_cast<float4*>(Pj + tl) = make_float4(pr[tl], pr[tl + 1], pr[tl + 2], pr[tl + 3]);
     if (warp == 0) cp_async_wait_all();  // dt_raw of stage s + 2 lands before the barrier
     if (tid == 0) bulk_wait_read<1>();    // output tile (s & 1) no longer read by the store of stage s - 2
     // Partials of stage s, rows of stage s + 1 and dt_raw of stage s + 2
@@ -413,18 +488,8 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     {
       float ys[kTA];
 #pragma unroll
-      for (int q = 0; q < kTA; q += 4) {
-        float4 acc = *reinterpret_cast<const float4*>(P_ + lane * S::kPR + tb + q);
-#pragma unroll
-        for (int jj = 1; jj < G; ++jj) {
-          const float4 v = *reinterpret_cast<const float4*>(P_ + (jj * 32 + lane) * S::kPR + tb + q);
-          acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
-        }
-        ys[q + 0] = (acc.x + du[q + 0]) * zg[q + 0];
-        ys[q + 1] = (acc.y + du[q + 1]) * zg[q + 1];
-        ys[q + 2] = (acc.z + du[q + 2]) * zg[q + 2];
-        ys[q + 3] = (acc.w + du[q + 3]) * zg[q + 3];
-      }
+      for (int q = 0; q < kTA; q += 4)
+        gate_pairs<G, 32 * S::kPR>(P_ + lane * S::kPR + tb + q, du + q / 2, zg + q / 2, ys + q);
       T* Y = reinterpret_cast<T*>(smem + S::kY + (s & 1) * S::kYBytes);
 #pragma unroll
       for (int i = 0; i < kTA; ++i) Y[(tb + i) * 32 + lane] = IO<T>::from_f(ys[i]);
@@ -432,7 +497,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     }
     if (has_next) {
 #pragma unroll
-      for (int i = 0; i < kTA; ++i) {
+      for (int i = 0; i < kTA / 2; ++i) {
         du[i] = duN[i];
         zg[i] = zgN[i];
       }

@@ -35,17 +35,26 @@ __device__ __forceinline__ float sigmoid(float v) { return rcp_approx(1.0f + ex2
 // SiLU(v) = v * sigmoid(v).
 __device__ __forceinline__ float silu(float v) { return v * sigmoid(v); }
 
-// log(1 + e) for e in [0, 1]: e * Q(e) by Horner (coefficients from
-// fit_log1p_poly.py, degree 8). No division, so no SFU work.
+// Coefficients of Q, highest degree first (fit_log1p_poly.py, degree 8):
+// log(1 + e) ~ e * Q(e) on [0, 1].
+constexpr int kLog1pDeg = 8;
+__host__ __device__ constexpr float log1p_q(int k) {
+  return k == 0   ? 5.232694093e-03f
+         : k == 1 ? -2.950523980e-02f
+         : k == 2 ? 7.822595537e-02f
+         : k == 3 ? -1.366324574e-01f
+         : k == 4 ? 1.910600662e-01f
+         : k == 5 ? -2.484298199e-01f
+         : k == 6 ? 3.331909776e-01f
+         : k == 7 ? -4.999949336e-01f
+                  : 9.999999404e-01f;
+}
+
+// log(1 + e) for e in [0, 1]: e * Q(e) by Horner. No division, so no SFU work.
 __device__ __forceinline__ float log1p_unit(float e) {
-  float q = fmaf(e, 5.232694093e-03f, -2.950523980e-02f);
-  q = fmaf(e, q, 7.822595537e-02f);
-  q = fmaf(e, q, -1.366324574e-01f);
-  q = fmaf(e, q, 1.910600662e-01f);
-  q = fmaf(e, q, -2.484298199e-01f);
-  q = fmaf(e, q, 3.331909776e-01f);
-  q = fmaf(e, q, -4.999949336e-01f);
-  q = fmaf(e, q, 9.999999404e-01f);
+  float q = fmaf(e, log1p_q(0), log1p_q(1));
+#pragma unroll
+  for (int k = 2; k <= kLog1pDeg; ++k) q = fmaf(e, q, log1p_q(k));
   return e * q;
 }
 

@@ -73,8 +73,9 @@ def test_kernel_lengths_history_and_zoh(shape):
         compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"kernel {kern} path {d} L{L} {disc}")
 
 
+@pytest.mark.parametrize("kernel", [3, 4])
 @pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
-def test_decay_paths_mixed_channels(io_dtype):
+def test_decay_paths_mixed_channels(io_dtype, kernel):
     """A_log perturbed in some 32-channel tiles (and in one single channel of
     another tile): those tiles must take the per-state path, the rest the
     power path. Checked three ways: both runs (auto and forced per-state)
@@ -90,12 +91,12 @@ def test_decay_paths_mixed_channels(io_dtype):
     A_log[128:160] = torch.log(torch.rand((32, 16), generator=g) * 8 + 0.5).cuda()  # tile 4: random A
     A_log[64 + 5, 7] += 1e-3  # tile 2: one state of one channel
     inp = dict(inp, A_log=A_log.contiguous())
-    y_auto, cc_a, st_auto = run_prefill(inp)
-    y_gen, cc_g, st_gen = run_prefill(inp, tuning={"decay_path": 1})
+    y_auto, cc_a, st_auto = run_prefill(inp, tuning={"kernel": kernel, "decay_path": 0})
+    y_gen, cc_g, st_gen = run_prefill(inp, tuning={"kernel": kernel, "decay_path": 1})
     chans = all_channels(b, E)
     want = oracle_prefill(inp, chans)
-    compare(io_dtype, gather(y_auto, cc_a, st_auto, chans), want, label="mixed auto")
-    compare(io_dtype, gather(y_gen, cc_g, st_gen, chans), want, label="mixed per-state")
+    compare(io_dtype, gather(y_auto, cc_a, st_auto, chans), want, label=f"mixed auto, kernel {kernel}")
+    compare(io_dtype, gather(y_gen, cc_g, st_gen, chans), want, label=f"mixed per-state, kernel {kernel}")
     for t in (1, 2, 4):
         sl = slice(32 * t, 32 * t + 32)
         assert torch.equal(st_auto[:, sl], st_gen[:, sl]) and torch.equal(y_auto[..., sl], y_gen[..., sl]), \
