@@ -291,7 +291,11 @@ ssm_status ssm_decode_step(const ssm_dims *dims, const ssm_weights *w, const voi
  *             ssm_proj_gemm).
  *
  * Ordering and errors. Everything is enqueued on `stream`, with no host
- * synchronisation. Argument errors return before any work is queued.
+ * synchronisation: a memset of the projections' tile counters (when a tile is
+ * cut), then in_proj, x_proj, the core and out_proj. Each of the last three is
+ * launched overlapped with the kernel before it (programmatic dependent
+ * launch), and reads nothing that kernel writes before it has finished.
+ * Argument errors return before any work is queued.
  */
 typedef struct {
   int64_t batch, seqlen, d_model, d_inner;
@@ -330,10 +334,11 @@ size_t ssm_block_workspace_bytes(const ssm_block_dims *dims);
  *              256-byte aligned, or NULL when that is 0. Whole 256 x 256 output
  *              tiles go round-robin to the pairs. Where a last wave would leave
  *              most pairs idle, the final one to two tiles a pair are instead
- *              cut along K into equal runs, one per pair; the fp32 partials of
- *              the cut tiles (512 KB a pair) and a counter per tile live here. The partials of a cut tile are
- *              summed in a fixed order, so results do not depend on timing.
- *              Calls that overlap on the GPU need separate workspaces.
+ *              cut along K into equal runs, one per pair; a counter per tile
+ *              (first) and the fp32 partials of the cut tiles (512 KB a pair)
+ *              live here. The partials of a cut tile are summed in a fixed
+ *              order, so results do not depend on timing. Calls that overlap
+ *              on the GPU need separate workspaces.
  */
 size_t ssm_proj_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 ssm_status ssm_proj_gemm(const void *A, const void *W, void *C, int64_t M, int64_t N, int64_t K, void *workspace,

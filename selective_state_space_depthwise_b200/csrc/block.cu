@@ -108,6 +108,9 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
                                                           const __grid_constant__ CUtensorMap map_w,
                                                           const XprojArgs a) {
   using S = XpSmem;
+  // Launched overlapped with in_proj (programmatic dependent launch): nothing
+  // in global memory is touched before it has finished.
+  griddep_wait();
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(smem);
@@ -257,6 +260,10 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
   }
   cluster_sync();  // the partials stay alive until every CTA of the cluster has read them
   tcgen05_fence_before();
+  // The next kernel may now be launched (it waits for this one to finish
+  // before it reads anything); signalling this late, not at the start, keeps
+  // its waiting CTAs off the SMs while this kernel still runs.
+  griddep_launch_dependents();
   __syncthreads();
   if (warp == 0) {
     tcgen05_fence_after();
@@ -273,7 +280,7 @@ bool bf16_map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint6
 
 // x = the first E columns of xz [b][L][2E] (bf16); W_x [33][E] (bf16).
 cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, int64_t batch, int num_sms,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool pdl) {
   CUtensorMap mx, mw;
   const uint64_t E = static_cast<uint64_t>(a.E), L = static_cast<uint64_t>(a.L);
   if (!bf16_map3(&mx, xz, E, L, static_cast<uint64_t>(batch), 2 * E * 2, L * 2 * E * 2, kXpK, kXpTok + 3,
@@ -294,13 +301,15 @@ cudaError_t launch_xproj(const XprojArgs& a, const void* xz, const void* w_x, in
   cfg.blockDim = dim3(kXpThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = static_cast<unsigned>(split);
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   err = cudaLaunchKernelEx(&cfg, xproj_kernel, mx, mw, a);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
@@ -414,9 +423,18 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   if (!err_word) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // The four kernels run back to back; each after the first is launched
+  // overlapped with the one before it (programmatic dependent launch), so its
+  // launch and setup hide under that kernel's tail. The GEMMs' cut-tile
+  // counters lead their shared scratch: zeroed once here (a memset between
+  // two kernels would break the overlap), they are zero again after each GEMM.
+  const size_t cnt_in = ssm::gemm_counter_bytes(M, 2 * E, Dm, sms), cnt_out = ssm::gemm_counter_bytes(M, Dm, E, sms);
+  const size_t cnt = cnt_in > cnt_out ? cnt_in : cnt_out;
+  cudaError_t err = cnt ? cudaMemsetAsync(ws + lay.gemm, 0, cnt, cs) : cudaSuccess;
+  if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "projection scratch: %s", cudaGetErrorString(err));
   // in_proj: xz[M][2E] = hidden[M][D] . W_in[2E][D]^T
-  cudaError_t err =
-      ssm::gemm_bf16_tn(hidden, proj->w_in, xz, M, 2 * E, Dm, ws + lay.gemm, lay.gemm_bytes, sms, err_word, cs);
+  err = ssm::gemm_bf16_tn(hidden, proj->w_in, xz, M, 2 * E, Dm, ws + lay.gemm, lay.gemm_bytes, sms, err_word, cs,
+                          false, true);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "in_proj launch: %s", cudaGetErrorString(err));
   // x_proj (fused with conv + SiLU): B, C, dt_raw
   ssm::XprojArgs xa{};
@@ -428,7 +446,7 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   xa.L = L;
   xa.E = E;
   xa.err = err_word;
-  err = ssm::launch_xproj(xa, xz, proj->w_x, b, sms, cs);
+  err = ssm::launch_xproj(xa, xz, proj->w_x, b, sms, cs, true);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "x_proj launch: %s", cudaGetErrorString(err));
   // the core, on x and z in place in xz
   cd.x_tok_stride = cd.z_tok_stride = 2 * E;
@@ -439,11 +457,12 @@ ssm_status ssm_block_forward(const ssm_block_dims* dims, const ssm_weights* w, c
   cd.bc_seq_stride = L * 32;
   cd.dt_seq_stride = L;
   const __nv_bfloat16* xzb = static_cast<const __nv_bfloat16*>(xz);
-  if ((st = ssm_prefill(&cd, w, xzb, xzb + E, bc, bc + 16, dt, conv_cache_in, ssm_state_in, y, conv_cache_out,
-                        ssm_state_out, nullptr, 0, stream)) != SSM_OK)
+  if ((st = ssm::prefill_entry(&cd, w, xzb, xzb + E, bc, bc + 16, dt, conv_cache_in, ssm_state_in, y,
+                               conv_cache_out, ssm_state_out, nullptr, true, stream)) != SSM_OK)
     return st;
   // out_proj: out[M][D] = y[M][E] . W_out[D][E]^T
-  err = ssm::gemm_bf16_tn(y, proj->w_out, out, M, Dm, E, ws + lay.gemm, lay.gemm_bytes, sms, err_word, cs);
+  err = ssm::gemm_bf16_tn(y, proj->w_out, out, M, Dm, E, ws + lay.gemm, lay.gemm_bytes, sms, err_word, cs, true,
+                          true);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "out_proj launch: %s", cudaGetErrorString(err));
   return ssm::fail(SSM_OK, "");
 }

@@ -92,7 +92,8 @@ struct GemmArgs {
   float* partial;     // [pairs][2 slots][2 halves] fp32 half tiles of 128 x 256, each stored
                       // [warp quarter][32-column chunk][float4 slot][lane]: every warp
                       // instruction moves 512 contiguous bytes
-  int* counters;      // [tiles][2 halves]: contributions counted so far, zero on entry
+  int* counters;      // [tiles][2 halves]: contributions counted so far, zero on entry; the
+                      // contributor that completes a count sets it back to zero
   int* err;
 };
 
@@ -213,6 +214,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
   cluster_sync();  // barriers of both CTAs initialised before any remote arrival
   tcgen05_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + S::kTmemSlot);
+  // Launched overlapped with the kernel before it (programmatic dependent
+  // launch): the setup above ran during its tail; global memory is touched
+  // only after it has finished. Without that launch attribute it returns at
+  // once.
+  griddep_wait();
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer ---
@@ -344,7 +350,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
         if (warp == 2 && lane == 0) {
           const bool okp = mbar_wait_bounded(part_bar, static_cast<uint32_t>(np) & 1u, g.err, 27);
           if (!okp) *abort_flag = 1;
-          *split_flag = okp && atomicAdd(g.counters + 2 * sg.tile + half, 1) == p_hi - p_lo;
+          const bool last = okp && atomicAdd(g.counters + 2 * sg.tile + half, 1) == p_hi - p_lo;
+          if (last) g.counters[2 * sg.tile + half] = 0;  // every contributor has counted: ready for the next launch
+          *split_flag = last;
           mbar_arrive(dec_bar);  // also after a timeout, so the others do not wait in vain
         }
         const bool okd = mbar_wait_bounded(dec_bar, static_cast<uint32_t>(np) & 1u, g.err, 28);
@@ -438,6 +446,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     if (lane == 0) bulk_wait<0>();
   }
 
+  // The next kernel may now be launched (it waits for this one to finish
+  // before it reads anything); signalled at the end, not the start, so its
+  // waiting CTAs do not sit on the SMs while this kernel still runs (measured:
+  // the block at 2048 tokens 1.3% faster than without the overlap, 2.8% slower
+  // with the signal at the start).
+  griddep_launch_dependents();
   __syncwarp();  // the single-thread roles rejoin their warps before the CTA barrier
   __syncthreads();
   // After an abort, loads issued by either CTA may still be landing and cannot
@@ -497,9 +511,12 @@ GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
 }
 
 size_t partial_bytes(const GemmPlan& pl) { return static_cast<size_t>(pl.pairs) * 4 * kHalfM * kTileN * 4; }
+// The counters lead the workspace (so every GEMM finds its own at offset 0),
+// the partials follow on a 512-byte boundary.
+size_t counter_bytes(const GemmPlan& pl) { return (static_cast<size_t>(pl.tiles) * 2 * sizeof(int) + 511) / 512 * 512; }
 
 cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* ws,
-                        size_t ws_bytes, int num_sms, int* err, cudaStream_t st) {
+                        size_t ws_bytes, int num_sms, int* err, bool pdl, bool counters_zeroed, cudaStream_t st) {
   using S = GemmSmem;
   const GemmPlan pl = gemm_plan(M, N, K, num_sms);
   if (pl.tiles >= (int64_t(1) << 30)) return cudaErrorInvalidConfiguration;
@@ -523,15 +540,28 @@ cudaError_t launch_gemm(const void* A, const void* B, void* C, int64_t M, int64_
   g.err = err;
   if (pl.partials) {
     if (!ws || ws_bytes < gemm_workspace_bytes(M, N, K, num_sms)) return cudaErrorInvalidValue;
-    g.partial = static_cast<float*>(ws);
-    g.counters = reinterpret_cast<int*>(static_cast<char*>(ws) + partial_bytes(pl));
-    cudaError_t e = cudaMemsetAsync(g.counters, 0, static_cast<size_t>(pl.tiles) * 2 * sizeof(int), st);
-    if (e != cudaSuccess) return e;
+    g.counters = static_cast<int*>(ws);
+    g.partial = reinterpret_cast<float*>(static_cast<char*>(ws) + counter_bytes(pl));
+    if (!counters_zeroed) {
+      cudaError_t e = cudaMemsetAsync(g.counters, 0, counter_bytes(pl), st);
+      if (e != cudaSuccess) return e;
+    }
   }
   const int smem = S::kTotal + 1024;
   cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  gemm_bf16_tn_kernel<<<static_cast<unsigned>(2 * pl.pairs), kGThreads, smem, st>>>(ma, mb, mc, g);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pl.pairs), 1, 1);
+  cfg.blockDim = dim3(kGThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, gemm_bf16_tn_kernel, ma, mb, mc, g);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -541,14 +571,20 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   const GemmPlan pl = gemm_plan(M, N, K, num_sms);
   if (!pl.partials) return 0;
-  return partial_bytes(pl) + static_cast<size_t>(pl.tiles) * 2 * sizeof(int);
+  return counter_bytes(pl) + partial_bytes(pl);
+}
+
+size_t gemm_counter_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  const GemmPlan pl = gemm_plan(M, N, K, num_sms);
+  return pl.partials ? counter_bytes(pl) : 0;
 }
 
 cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* ws,
-                         size_t ws_bytes, int num_sms, int* err, cudaStream_t st) {
+                         size_t ws_bytes, int num_sms, int* err, cudaStream_t st, bool pdl, bool counters_zeroed) {
   if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0 || N % 8 != 0) return cudaErrorInvalidValue;
   if (num_sms <= 1) num_sms = 148;
-  return launch_gemm(A, B, C, M, N, K, ws, ws_bytes, num_sms, err, st);
+  return launch_gemm(A, B, C, M, N, K, ws, ws_bytes, num_sms, err, pdl, counters_zeroed, st);
 }
 
 }  // namespace ssm

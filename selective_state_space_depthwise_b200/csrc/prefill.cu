@@ -518,6 +518,7 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
       named_bar_arrive(2, NT);
     }
   }
+  griddep_launch_dependents();  // the next kernel may be launched (it waits for this one to finish)
   if (tid == 0) bulk_wait<0>();
 
   if (ch_ok) {
@@ -590,6 +591,10 @@ template <typename T, int G, bool ZOH, int MINB>
 __global__ void __launch_bounds__(32 * G, MINB) prefill_pipe_kernel(const __grid_constant__ Maps maps,
                                                                      const KernelArgs a) {
   constexpr bool SPLIT = split_barrier<MINB>();
+  // Launched overlapped with the kernel before it (programmatic dependent
+  // launch, in the block forward): nothing in global memory is touched before
+  // that kernel has finished. Without that launch attribute it returns at once.
+  griddep_wait();
   if constexpr (ZOH) {
     pipe_run<T, G, Path::kZoh, SPLIT>(maps, a);
   } else {
@@ -655,7 +660,7 @@ bool make_maps(const KernelArgs& a, Maps* m) {
 }
 
 template <typename T, int G, bool ZOH, int MINB>
-cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st) {
+cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st, bool pdl) {
   using S = PipeSmem<T, G, split_barrier<MINB>()>;
   Maps maps;
   if (!make_maps<T>(a, &maps)) return cudaErrorInvalidValue;
@@ -665,14 +670,25 @@ cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st) {
   if (err != cudaSuccess) return err;
   const int64_t grid = a.batch * ((a.E + 31) / 32);
   if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  kern<<<static_cast<unsigned>(grid), 32 * G, smem, st>>>(maps, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(32 * G, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  err = cudaLaunchKernelEx(&cfg, kern, maps, a);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
 template <typename T, bool ZOH>
-cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st) {
-  if (sh.kernel == 3) return launch_pipe<T, 4, ZOH, 0>(a, st);
-  if (sh.kernel == 4) return launch_pipe<T, 4, ZOH, 1>(a, st);
+cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st, bool pdl) {
+  if (sh.kernel == 3) return launch_pipe<T, 4, ZOH, 0>(a, st, pdl);
+  if (sh.kernel == 4) return launch_pipe<T, 4, ZOH, 1>(a, st, pdl);
   return cudaErrorInvalidValue;
 }
 
@@ -687,7 +703,7 @@ PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int n
   return PrefillShape{ctas <= 2 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148) ? 4 : 3};
 }
 
-cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st) {
+cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st, bool pdl) {
   if (a.L == 0) {
     const int64_t n = a.batch * a.E;
     const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
@@ -698,8 +714,9 @@ cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillS
     return cudaGetLastError();
   }
   if (!prefill_shape_supported(sh)) return cudaErrorInvalidValue;
-  if (io_bf16) return zoh ? dispatch<__nv_bfloat16, true>(a, sh, st) : dispatch<__nv_bfloat16, false>(a, sh, st);
-  return zoh ? dispatch<float, true>(a, sh, st) : dispatch<float, false>(a, sh, st);
+  if (io_bf16)
+    return zoh ? dispatch<__nv_bfloat16, true>(a, sh, st, pdl) : dispatch<__nv_bfloat16, false>(a, sh, st, pdl);
+  return zoh ? dispatch<float, true>(a, sh, st, pdl) : dispatch<float, false>(a, sh, st, pdl);
 }
 
 }  // namespace ssm

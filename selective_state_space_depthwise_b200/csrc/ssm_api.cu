@@ -170,17 +170,12 @@ using ssm::device_error_ptr;
 
 }  // namespace
 
-extern "C" {
+namespace ssm {
 
-size_t ssm_prefill_workspace_bytes(const ssm_dims* dims) {
-  (void)dims;
-  return 0;
-}
-
-ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
-                          const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
-                          void* y, void* conv_cache_out, float* ssm_state_out, void* workspace, size_t workspace_bytes,
-                          const ssm_tuning* tuning, void* stream) {
+ssm_status prefill_entry(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                         const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
+                         void* y, void* conv_cache_out, float* ssm_state_out, const ssm_tuning* tuning, bool pdl,
+                         void* stream) {
   ssm::Strides s;
   ssm_status st = check_dims(dims, true, &s);
   if (st != SSM_OK) return st;
@@ -195,9 +190,6 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
     if (y == x || y == z) return fail(SSM_ERR_INVALID_ARG, "y must not alias x or z");
   }
   if ((st = check_prefill_caches(conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out)) != SSM_OK) return st;
-  if (workspace_bytes < ssm_prefill_workspace_bytes(dims))
-    return fail(SSM_ERR_INVALID_ARG, "workspace too small");
-  (void)workspace;
 
   ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current());
   int decay_path = 0;
@@ -233,9 +225,28 @@ ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void
   a.err = device_error_ptr();
   if (!a.err) return fail(SSM_ERR_CUDA, "device error word: %s", cudaGetErrorString(cudaGetLastError()));
   cudaError_t err = ssm::launch_prefill(a, dims->io_dtype == SSM_BF16, dims->discretization == SSM_DISC_ZOH, sh,
-                                        static_cast<cudaStream_t>(stream));
+                                        static_cast<cudaStream_t>(stream), pdl);
   if (err != cudaSuccess) return fail(SSM_ERR_CUDA, "prefill launch: %s", cudaGetErrorString(err));
   return ok();
+}
+
+}  // namespace ssm
+
+extern "C" {
+
+size_t ssm_prefill_workspace_bytes(const ssm_dims* dims) {
+  (void)dims;
+  return 0;
+}
+
+ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                          const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
+                          void* y, void* conv_cache_out, float* ssm_state_out, void* workspace, size_t workspace_bytes,
+                          const ssm_tuning* tuning, void* stream) {
+  if (workspace_bytes < ssm_prefill_workspace_bytes(dims)) return fail(SSM_ERR_INVALID_ARG, "workspace too small");
+  (void)workspace;
+  return ssm::prefill_entry(dims, w, x, z, B, C, dt_raw, conv_cache_in, ssm_state_in, y, conv_cache_out,
+                            ssm_state_out, tuning, false, stream);
 }
 
 ssm_status ssm_prefill(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,

@@ -49,16 +49,26 @@ struct PrefillShape {
 
 PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t L, int num_sms);
 bool prefill_shape_supported(PrefillShape sh);
-cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st);
+// pdl: overlap the launch with the kernel before it on the stream (that must
+// be a kernel, not a copy or memset); the kernel reads its inputs only after
+// that kernel has finished.
+cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st,
+                           bool pdl = false);
 cudaError_t launch_decode(const KernelArgs& a, bool io_bf16, bool zoh, cudaStream_t st);
 
 // C[M][N] = A[M][K] . B[N][K]^T, bf16 operands and output, fp32 accumulation,
 // on the tensor cores (gemm.cu). K and N multiples of 8, pointers 16-byte
-// aligned. ws: gemm_workspace_bytes() of device scratch (the fp32 partials of
-// tiles cut between CTA pairs and their counters; 0 bytes when none is cut).
+// aligned. ws: gemm_workspace_bytes() of device scratch (the counters of tiles
+// cut between CTA pairs, first, then their fp32 partials; 0 bytes when none is
+// cut). The counters must be zero on entry and are zero again after a launch
+// that completed: counters_zeroed skips the memset that ensures it. pdl: the
+// launch may overlap the kernel before it on the stream (programmatic
+// dependent launch), which must be a kernel, not a copy or memset.
 cudaError_t gemm_bf16_tn(const void* A, const void* B, void* C, int64_t M, int64_t N, int64_t K, void* ws,
-                         size_t ws_bytes, int num_sms, int* err, cudaStream_t st);
+                         size_t ws_bytes, int num_sms, int* err, cudaStream_t st, bool pdl = false,
+                         bool counters_zeroed = false);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+size_t gemm_counter_bytes(int64_t M, int64_t N, int64_t K, int num_sms);  // leading part of the workspace
 
 // Shared by the entry points (ssm_api.cu): validation with the ABI's
 // "0 = dense" stride defaults, and the calling thread's last-error message.
@@ -66,6 +76,12 @@ ssm_status check_dims(const ssm_dims* d, bool prefill, Strides* s);
 ssm_status check_weights(const ssm_weights* w);
 ssm_status check_prefill_caches(const void* conv_cache_in, const float* ssm_state_in, const void* conv_cache_out,
                                 const float* ssm_state_out);
+// ssm_prefill_ex with the launch overlapped with the kernel before it (pdl, as
+// for launch_prefill); the block forward's core step.
+ssm_status prefill_entry(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,
+                         const float* C, const float* dt_raw, const void* conv_cache_in, const float* ssm_state_in,
+                         void* y, void* conv_cache_out, float* ssm_state_out, const ssm_tuning* tuning, bool pdl,
+                         void* stream);
 bool aligned(const void* p, size_t a);
 ssm_status fail(ssm_status st, const char* fmt, ...);
 int* device_error_ptr();  // the device error word of the current device
