@@ -102,8 +102,8 @@ typedef struct {
  *   channels, warp j owns states 4j..4j+3 of each, the per-token work of the
  *   next 32-token stage overlaps the scan of the current one), built for three
  *   resident CTAs per SM; 4 = the same code built for two CTAs per SM (a larger
- *   register budget). Auto takes 4 when batch * ceil(d_inner / 32) <= 2 * SMs,
- *   else 3. Any other value returns SSM_ERR_INVALID_ARG.
+ *   register budget). Auto takes 4 when batch * ceil(d_inner / 32) <= 64 *
+ *   SMs, else 3. Any other value returns SSM_ERR_INVALID_ARG.
  * decay_path: 0 = auto; 1 = every decay exp(dt A_n) as its own exponential.
  *   Auto: a CTA whose 32 channels all have A_n = (n+1) A_0 within 2^-20
  *   relative (the "State initialization" of "Axon-SSM": diagonals -1..-16)

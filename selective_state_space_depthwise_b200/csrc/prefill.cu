@@ -574,8 +574,7 @@ __device__ __forceinline__ bool cta_has_power_decays(const KernelArgs& a) {
 
 // MINB 0 leaves the register budget to the compiler (3 CTAs of 4 warps fit an
 // SM); MINB 1 lets it use up to 255 registers a thread (2 CTAs fit), which it
-// spends on a deeper schedule of the fused block: measured 7% faster when the
-// grid needs at most two CTAs per SM, slower when it needs more.
+// spends on a deeper schedule of the fused block (see choose_prefill_shape).
 // The split end-of-stage barrier (double-buffered partials) is used where
 // the shared memory allows: not in the three-CTAs-per-SM build. The build
 // switch turns it off everywhere (for side-by-side measurements).
@@ -696,11 +695,13 @@ cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st, bool
 
 bool prefill_shape_supported(PrefillShape sh) { return sh.kernel == 3 || sh.kernel == 4; }
 
-// Pipelined state slices; the register-rich build when the grid needs at most
-// two CTAs per SM.
+// Pipelined state slices: the register-rich build (two CTAs per SM), except
+// for grids of many waves. Measured on B200: kernel 4 matched or beat kernel 3
+// from 80 to 5120 CTAs (by 1-27%); at 61440 CTAs (256 sequences of 7680
+// channels) kernel 3 was 2.6% faster.
 PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int num_sms) {
   const int64_t ctas = batch * ((E + 31) / 32);
-  return PrefillShape{ctas <= 2 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148) ? 4 : 3};
+  return PrefillShape{ctas <= 64 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148) ? 4 : 3};
 }
 
 cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st, bool pdl) {
