@@ -143,47 +143,6 @@ __device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const f
   return lo + hi;
 }
 
-// Power decays: the thread's K states K j .. K j + K - 1 decay by
-// q^(K j + 1) .. q^(K j + K) = base * (q, q^2, ..., q^K) with base = q^(K j).
-// hi1 / hi2 (warp-uniform): bits of j; base = (q^K)^(j&1) (q^2K)^(j>>1 & 1).
-// inj2 = {dt*u, dt*u}.
-template <int K>
-__device__ __forceinline__ float scan_token_pow(float q, uint64_t inj2, bool hi1, bool hi2, float* h, const float* Bp,
-                                                const float* Cp) {
-  static_assert(K == 4 || K == 8, "power decays are built for 4 or 8 states per thread");
-  uint64_t p[K / 2];  // (q, q^2), (q^3, q^4), ...
-  const float q2 = q * q;
-  p[0] = pk2(q, q2);
-  p[1] = fmul2(p[0], pk2(q2, q2));
-  float q3, qk;
-  upk2(p[1], q3, qk);  // qk = q^4
-  if constexpr (K == 8) {
-    const uint64_t q44 = pk2(qk, qk);
-    p[2] = fmul2(p[0], q44);
-    p[3] = fmul2(p[1], q44);
-    float q7;
-    upk2(p[3], q7, qk);  // qk = q^8
-  }
-  float base = hi1 ? qk : 1.0f;
-  if (hi2) base *= qk * qk;
-  const uint64_t bb = pk2(base, base);
-  uint64_t acc = 0;
-#pragma unroll
-  for (int i = 0; i < K / 2; i += 2) {
-    const float4 bq = *reinterpret_cast<const float4*>(Bp + 2 * i);
-    const float4 cq = *reinterpret_cast<const float4*>(Cp + 2 * i);
-    const uint64_t hb0 = ffma2(fmul2(bb, p[i]), pk2(h[2 * i], h[2 * i + 1]), fmul2(inj2, pk2(bq.x, bq.y)));
-    const uint64_t hb1 = ffma2(fmul2(bb, p[i + 1]), pk2(h[2 * i + 2], h[2 * i + 3]), fmul2(inj2, pk2(bq.z, bq.w)));
-    upk2(hb0, h[2 * i], h[2 * i + 1]);
-    upk2(hb1, h[2 * i + 2], h[2 * i + 3]);
-    acc = i == 0 ? fmul2(pk2(cq.x, cq.y), hb0) : ffma2(pk2(cq.x, cq.y), hb0, acc);
-    acc = ffma2(pk2(cq.z, cq.w), hb1, acc);
-  }
-  float lo, hi;
-  upk2(acc, lo, hi);
-  return lo + hi;
-}
-
 // Zero-order-hold decays (scalar): h = e^{dt A} h + (e^{dt A} - 1)/A * u * B.
 template <int K>
 __device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* Av, float* h, const float* Bp,
@@ -306,22 +265,80 @@ __device__ __forceinline__ void store_rows(float2* DTo, int tb, int lane, const 
   for (int p = 0; p < kTA / 2; ++p) DT4[((tb >> 1) + p) * 32 + lane] = rows[p];
 }
 
+// Power decays, 4 states a thread: states 4j .. 4j + 3 decay by q^(4j+1) ..
+// q^(4j+4) = base * (q, q^2, q^3, q^4) with base = q^(4j); hi1 / hi2
+// (warp-uniform) are the bits of j, so base = (q^4)^(j&1) (q^8)^(j>>1 & 1).
+// pow_prep forms everything of token tl that does not depend on the state:
+// its decays, its injections dt*u*B (row values q and dt*u) and its C.
+struct PowPrep {
+  uint64_t d01, d23, b01, b23, c01, c23;
+};
+__device__ __forceinline__ PowPrep pow_prep(const float2* __restrict__ DTc, int lane, int tl, bool hi1, bool hi2,
+                                            const float* __restrict__ Bs, const float* __restrict__ Cs) {
+  const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
+  const float q = (tl & 1) ? d4.y : d4.x, inj = (tl & 1) ? d4.w : d4.z;
+  const float4 bq = *reinterpret_cast<const float4*>(Bs + tl * 16);
+  const float4 cq = *reinterpret_cast<const float4*>(Cs + tl * 16);
+  const float q2 = q * q;
+  const uint64_t p0 = pk2(q, q2);
+  const uint64_t p1 = fmul2(p0, pk2(q2, q2));
+  float q3, q4;
+  upk2(p1, q3, q4);
+  float base = hi1 ? q4 : 1.0f;
+  if (hi2) base *= q4 * q4;
+  const uint64_t bb = pk2(base, base), i2 = pk2(inj, inj);
+  PowPrep r;
+  r.d01 = fmul2(bb, p0);
+  r.d23 = fmul2(bb, p1);
+  r.b01 = fmul2(i2, pk2(bq.x, bq.y));
+  r.b23 = fmul2(i2, pk2(bq.z, bq.w));
+  r.c01 = pk2(cq.x, cq.y);
+  r.c23 = pk2(cq.z, cq.w);
+  return r;
+}
+
+// The power path's phase B with token tl + 1 prepared while token tl updates
+// the state (measured ~1% faster than preparing each token just before its
+// update).
+template <int T0, int T1>
+__device__ __forceinline__ void scan_stage_pow_la(const float2* __restrict__ DTc, int lane, bool hi1, bool hi2,
+                                                  float* h, const float* __restrict__ Bs, const float* __restrict__ Cs,
+                                                  float* pr) {
+  uint64_t h01 = pk2(h[0], h[1]), h23 = pk2(h[2], h[3]);
+  PowPrep nx = pow_prep(DTc, lane, T0, hi1, hi2, Bs, Cs);
+#pragma unroll
+  for (int tl = T0; tl < T1; ++tl) {
+    const PowPrep cu = nx;
+    if (tl + 1 < T1) nx = pow_prep(DTc, lane, tl + 1, hi1, hi2, Bs, Cs);
+    h01 = ffma2(cu.d01, h01, cu.b01);
+    h23 = ffma2(cu.d23, h23, cu.b23);
+    float lo, hi;
+    upk2(ffma2(cu.c23, h23, fmul2(cu.c01, h01)), lo, hi);
+    pr[tl] = lo + hi;
+  }
+  upk2(h01, h[0], h[1]);
+  upk2(h23, h[2], h[3]);
+}
+
 // Phase B over tokens [T0, T1) of one stage: this thread's 4 states; pr gets
 // the partial readouts.
 template <Path P, int K, int T0 = 0, int T1 = kTok>
 __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int lane, const float* Av, const float* a2,
                                            bool hi1, bool hi2, float* h, const float* __restrict__ Bs,
                                            const float* __restrict__ Cs, float* pr) {
+  if constexpr (P == Path::kPow) {
+    static_assert(K == 4, "power decays are built for 4 states per thread");
+    scan_stage_pow_la<T0, T1>(DTc, lane, hi1, hi2, h, Bs, Cs, pr);
+  } else {
 #pragma unroll
-  for (int tl = T0; tl < T1; ++tl) {
-    const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
-    const float2 dd = (tl & 1) ? make_float2(d4.y, d4.w) : make_float2(d4.x, d4.z);
-    if constexpr (P == Path::kZoh)
-      pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
-    else if constexpr (P == Path::kPow)
-      pr[tl] = scan_token_pow<K>(dd.x, pk2(dd.y, dd.y), hi1, hi2, h, Bs + tl * 16, Cs + tl * 16);
-    else
-      pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
+    for (int tl = T0; tl < T1; ++tl) {
+      const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
+      const float2 dd = (tl & 1) ? make_float2(d4.y, d4.w) : make_float2(d4.x, d4.z);
+      if constexpr (P == Path::kZoh)
+        pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
+      else
+        pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
+    }
   }
 }
 
