@@ -9,8 +9,11 @@
 // Both sums are dense contractions and run on the tensor cores, each into its
 // own TMEM accumulator, so that the carried-state term needs no rescaled copy
 // of C and starts as soon as its operands land. One CTA per (b, c, h) (two
-// per chunk of 256, one per two chunks of 64), 256 threads; ~75 KB of shared
-// memory at chunk 128 lets three CTAs share an SM:
+// per chunk of 256, one per two chunks of 64): eight math warps (scores and
+// epilogue) and a control warp, whose first thread issues the TMA loads and
+// every MMA and waits on their barriers, so that the math warps wait only
+// for their own data; ~75 KB of shared memory at chunk 128 lets three CTAs
+// share an SM:
 //  1. TMA brings, 128-byte swizzled, the cb tile [l][s] (128 columns, two
 //     atoms) and the x tile [s][p] on one mbarrier, and the first 64-column
 //     atom of the C tile [l][n] and of the prev_states tile [p][n] on a
@@ -33,7 +36,8 @@
 //     row factor could overflow) one exponential per element. The choice is
 //     made per warp (over its 32 rows), so no branch diverges.
 //     The TMA layout is already the MMA's K-major operand;
-//  4. one thread issues eight MMAs scores x x (x as an MN-major B operand) into
+//  4. once the math warps have arrived at a named barrier, the control
+//     thread issues eight MMAs scores x x (x as an MN-major B operand) into
 //     accumulator 0. The second half of a 256-chunk has 256 score columns: it
 //     runs steps 3-4 twice, on columns 0..127 then 128..255, the buffers
 //     refilled once the first pass's MMAs have read them. Then the last state
@@ -62,7 +66,11 @@ constexpr int kHd = 64;   // head dim: MMA N
 // Template parameters: the chunk length CS (64 or 128; a CTA's 128 rows hold
 // 128 / CS consecutive chunks) and the state dim DS (64 or 128: the K of the
 // carried-state term).
-constexpr int kSsdThreads = 256;
+constexpr int kSsdMath = 256;                  // warps 0-7: scores and epilogue (a thread per row and atom)
+constexpr int kSsdThreads = kSsdMath + 32;     // warp 8: TMA loads, TMEM, and every MMA issue and wait
+constexpr int kCtlWarp = kSsdMath / 32;
+constexpr int kBarScores = 1;                  // named barrier: the math warps' scores are in (arrive) -> MMAs (sync)
+constexpr int kBarMath = 2;                    // named barrier among the math warps only
 // Load order: 1 = cb and x first (the score math starts sooner; the
 // carried-state MMAs go last), 0 = C and prev_states first (their MMAs are
 // issued on arrival). Measured on B200 at b = 8, L = 4096, 80 heads: 364 us
@@ -205,7 +213,8 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
     }
     tma_load_4d(sb + S::kX, &map_x, 0, h, static_cast<int>(t_chunk + kCs * p), b, full_scores);
   };
-  if (tid == 0) {
+  const bool ctl = tid == kSsdMath;  // the control thread: lane 0 of warp 8
+  if (ctl) {
     mbar_init(full_state, 1);
     mbar_init(full_scores, 1);
     mbar_init(done, 1);
@@ -226,7 +235,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
       load_scores(0);
     }
   }
-  if (warp == 0) {
+  if (warp == kCtlWarp) {
     tmem_alloc(sb + S::kTmemSlot, S::kTmemCols);
     tmem_relinquish();
   }
@@ -262,133 +271,147 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
                     umma_desc_k_sw128(sb + S::kPrev + (k * S::kSA + (kk >> 2)) * S::kAtomRows64 + (kk & 3) * 32),
                     ssd_idesc(false), t0 > 0 || kk > 0);
   };
-  // 2. Carried-state term, as soon as its operands are in: C[l][n] x prev_states[p][n]^T.
-  //    Reloading: the first atom here, then the buffer is refilled with the
-  //    second while the scores are formed.
-  if (tid == 0 && (S::kReload || !kScoresFirst)) {
-    mbar_wait_bounded(full_state, 0u, a.err, 7);
-    tcgen05_fence_after();
-    state_mmas(0);
-    if constexpr (S::kReload) {
-      umma_commit(state_free);
-      mbar_wait_bounded(state_free, 0u, a.err, 10);  // the MMAs have read the buffer
-      mbar_arrive_expect_tx(full_state, S::kTxState);
-      load_state(1);
-    }
-  }
-  for (int i = tid; i < ks; i += kSsdThreads) F[i] = ex2_approx((sdA[i | 7] - sdA[i]) * kLog2e) * sdt[i];
-  const int lg = r0 + l;  // this thread's row within its chunk pair / chunk
-  const float dAl = sdA[lg];
-  mbar_wait_bounded(full_scores, 0u, a.err, 8);
-  __syncthreads();  // F complete
-
-  // 3. Row l of the cb tile -> scores (in place), one pass of 128 columns at a
-  //    time (two passes only for the second half of a 256-chunk), this
-  //    thread's 64-column atom `at` of each. A warp's 32 rows lie in one chunk, starting at column
-  //    warp_min_s. Groups are classified against the warp's whole row span,
-  //    so every branch below is warp-uniform: groups wholly at or below all 32
-  //    rows take the two-factor product with no masking; the four groups the
-  //    span straddles mask per element, in the two-factor form unless the
-  //    diagonal group of some row of the warp decays by 80 nats or more
-  //    across its 8 columns (then its row factor could overflow, and each
-  //    decay is formed on its own).
-  const int warp_min_l = r0 + 32 * (warp & 3), warp_max_l = warp_min_l + 31;
-  const int warp_min_s = CS < kCs ? (32 * (warp & 3)) & ~(CS - 1) : 0;
-  const int sd = lg & ~7;
-  const bool strong = __any_sync(0xffffffffu, sdA[sd] - sdA[sd + 7] >= 80.0f);
-  for (int pass = 0; pass < np; ++pass) {
-    if (pass > 0) mbar_wait_bounded(full_scores, static_cast<uint32_t>(pass) & 1u, a.err, 8);
-    // This thread's 64-column atom of the pass: columns 128 pass + 64 at ..
-    {
-      const int aa = 2 * pass + at;  // atom index over the chunk's columns
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int s0 = 64 * aa + 8 * j;
-        uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
-        if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
-          *p = make_uint4(0u, 0u, 0u, 0u);
-          continue;
+  if (warp == kCtlWarp) {
+    // The control warp: the MMAs and the waits they need, so that the math
+    // warps wait only for their data.
+    if (ctl) {
+      // 2. Carried-state term, as soon as its operands are in: C[l][n] x prev_states[p][n]^T.
+      //    Reloading: the first atom here, then the buffer is refilled with the
+      //    second while the scores are formed.
+      if (S::kReload || !kScoresFirst) {
+        mbar_wait_bounded(full_state, 0u, a.err, 7);
+        tcgen05_fence_after();
+        state_mmas(0);
+        if constexpr (S::kReload) {
+          umma_commit(state_free);
+          mbar_wait_bounded(state_free, 0u, a.err, 10);  // the MMAs have read the buffer
+          mbar_arrive_expect_tx(full_state, S::kTxState);
+          load_state(1);
         }
-        float f[8];
-        unpack8(*p, f);
-        if (s0 + 7 <= warp_min_l) {  // wholly at or below the diagonal for every row: row factor x column factor
-          const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+      }
+    }
+    // 4. Intra-chunk term of each pass: scores[l][s] x x[s][p], s in steps of
+    //    16 rows of x, once the math warps have formed the pass's scores.
+    //    Before a second pass the buffers are refilled once these MMAs have
+    //    read them. (The warp reconverges before each barrier: bar.sync is
+    //    executed by whole warps.)
+    for (int pass = 0; pass < np; ++pass) {
+      __syncwarp();
+      named_bar_sync(kBarScores, kSsdThreads);
+      if (ctl) {
+        tcgen05_fence_after();
 #pragma unroll
-          for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
-        } else if (!strong) {  // straddled by the warp's rows: masked two-factor form
-          const float e = s0 <= lg ? ex2_approx((dAl - sdA[s0 + 7]) * kLog2e) : 0.0f;
+        for (int kk = 0; kk < S::kKS / 16; ++kk)
+          umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
+                      umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), pass > 0 || kk > 0);
+        if (pass + 1 < np) {
+          umma_commit(pass_free);
+          mbar_wait_bounded(pass_free, static_cast<uint32_t>(pass) & 1u, a.err, 11);
+          mbar_arrive_expect_tx(full_scores, S::kTxScores);
+          load_scores(pass + 1);
+        }
+      }
+    }
+    // The carried-state term (its last atom) and one commit for everything.
+    if (ctl) {
+      if constexpr (S::kReload) {  // the second state atom
+        mbar_wait_bounded(full_state, 1u, a.err, 7);
+        tcgen05_fence_after();
+        state_mmas(1);
+      } else if (kScoresFirst) {  // carried-state term last: its operands were loaded second
+        mbar_wait_bounded(full_state, 0u, a.err, 7);
+        tcgen05_fence_after();
+        state_mmas(0);
+      }
+      umma_commit(done);
+    }
+    __syncwarp();
+  } else {
+    for (int i = tid; i < ks; i += kSsdMath) F[i] = ex2_approx((sdA[i | 7] - sdA[i]) * kLog2e) * sdt[i];
+    const int lg = r0 + l;  // this thread's row within its chunk pair / chunk
+    const float dAl = sdA[lg];
+    mbar_wait_bounded(full_scores, 0u, a.err, 8);
+    named_bar_sync(kBarMath, kSsdMath);  // F complete
+
+    // 3. Row l of the cb tile -> scores (in place), one pass of 128 columns at a
+    //    time (two passes only for the second half of a 256-chunk), this
+    //    thread's 64-column atom `at` of each. A warp's 32 rows lie in one chunk, starting at column
+    //    warp_min_s. Groups are classified against the warp's whole row span,
+    //    so every branch below is warp-uniform: groups wholly at or below all 32
+    //    rows take the two-factor product with no masking; the four groups the
+    //    span straddles mask per element, in the two-factor form unless the
+    //    diagonal group of some row of the warp decays by 80 nats or more
+    //    across its 8 columns (then its row factor could overflow, and each
+    //    decay is formed on its own).
+    const int warp_min_l = r0 + 32 * (warp & 3), warp_max_l = warp_min_l + 31;
+    const int warp_min_s = CS < kCs ? (32 * (warp & 3)) & ~(CS - 1) : 0;
+    const int sd = lg & ~7;
+    const bool strong = __any_sync(0xffffffffu, sdA[sd] - sdA[sd + 7] >= 80.0f);
+    for (int pass = 0; pass < np; ++pass) {
+      if (pass > 0) mbar_wait_bounded(full_scores, static_cast<uint32_t>(pass) & 1u, a.err, 8);
+      // This thread's 64-column atom of the pass: columns 128 pass + 64 at ..
+      {
+        const int aa = 2 * pass + at;  // atom index over the chunk's columns
 #pragma unroll
-          for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
-        } else {  // masked, each decay on its own
+        for (int j = 0; j < 8; ++j) {
+          const int s0 = 64 * aa + 8 * j;
+          uint4* p = reinterpret_cast<uint4*>(smem + S::kCb + at * S::kAtomRows128 + sw128(l, j));
+          if (s0 > warp_max_l || s0 < warp_min_s) {  // above the diagonal or outside the chunk, every row
+            *p = make_uint4(0u, 0u, 0u, 0u);
+            continue;
+          }
+          float f[8];
+          unpack8(*p, f);
+          if (s0 + 7 <= warp_min_l) {  // wholly at or below the diagonal for every row: row factor x column factor
+            const float e = ex2_approx((dAl - sdA[s0 + 7]) * kLog2e);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) f[q] *= e * F[s0 + q];
+          } else if (!strong) {  // straddled by the warp's rows: masked two-factor form
+            const float e = s0 <= lg ? ex2_approx((dAl - sdA[s0 + 7]) * kLog2e) : 0.0f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) f[q] = s0 + q <= lg ? f[q] * e * F[s0 + q] : 0.0f;
+          } else {  // masked, each decay on its own
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
+          }
+          *p = pack8(f);
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
+      tcgen05_fence_before();
+      named_bar_arrive(kBarScores, kSsdThreads);  // the pass's scores are in: the control warp issues its MMAs
+    }
+    mbar_wait_bounded(done, 0u, a.err, 9);
+    tcgen05_fence_after();
+
+    // 5. Lanes 32 (w mod 4) .., columns 32 (w / 4) ..: acc0 + exp(dA[l]) acc1 + D x, bf16,
+    //    into the out tile (the cb buffer, free now), then out by TMA.
+    {
+      const int q4 = warp & 3, col0 = 32 * (warp >> 2);
+      const int row = 32 * q4 + (tid & 31);
+      const float el = ex2_approx(sdA[r0 + row] * kLog2e);
+      const uint32_t acc_state = tmem + kHd * (1 + (CS < kCs ? (32 * q4) / CS : 0));  // this warp's chunk
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        uint32_t r0v[16], r1v[16];
+        const uint32_t lane_col = (static_cast<uint32_t>(32 * q4) << 16) + col0 + 16 * jj;
+        tmem_ld_x16(acc_intra + lane_col, r0v);
+        tmem_ld_x16(acc_state + lane_col, r1v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int j = (col0 + 16 * jj) / 8 + half;  // 16-byte chunk of the row: p = 8 j .. 8 j + 7
+          float xv[8], o[8];
+          unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(row, j)), xv);  // the last pass's x rows
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            f[q] = s0 + q <= lg ? f[q] * ex2_approx((dAl - sdA[s0 + q]) * kLog2e) * sdt[s0 + q] : 0.0f;
+            o[q] = fmaf(Dh, xv[q], fmaf(el, __uint_as_float(r1v[8 * half + q]), __uint_as_float(r0v[8 * half + q])));
+          *reinterpret_cast<uint4*>(smem + S::kCb + sw128(row, j)) = pack8(o);
         }
-        *p = pack8(f);
       }
     }
-    fence_proxy_async_smem();  // generic-proxy writes become visible to the tensor core
-    __syncthreads();
-
-    // 4. Intra-chunk term of the pass: scores[l][s] x x[s][p], s in steps of
-    //    16 rows of x. Before a second pass the buffers are refilled once
-    //    these MMAs have read them.
-    if (tid == 0) {
-      tcgen05_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < S::kKS / 16; ++kk)
-        umma_f16_ss(acc_intra, umma_desc_k_sw128(sb + S::kCb + (kk >> 2) * S::kAtomRows128 + (kk & 3) * 32),
-                    umma_desc_k_sw128(sb + S::kX + kk * 16 * 128), ssd_idesc(true), pass > 0 || kk > 0);
-      if (pass + 1 < np) {
-        umma_commit(pass_free);
-        mbar_wait_bounded(pass_free, static_cast<uint32_t>(pass) & 1u, a.err, 11);
-        mbar_arrive_expect_tx(full_scores, S::kTxScores);
-        load_scores(pass + 1);
-      }
-    }
-  }
-  // The carried-state term (its last atom) and one commit for everything.
-  if (tid == 0) {
-    if constexpr (S::kReload) {  // the second state atom
-      mbar_wait_bounded(full_state, 1u, a.err, 7);
-      tcgen05_fence_after();
-      state_mmas(1);
-    } else if (kScoresFirst) {  // carried-state term last: its operands were loaded second
-      mbar_wait_bounded(full_state, 0u, a.err, 7);
-      tcgen05_fence_after();
-      state_mmas(0);
-    }
-    umma_commit(done);
-  }
-  mbar_wait_bounded(done, 0u, a.err, 9);
-  tcgen05_fence_after();
-
-  // 5. Lanes 32 (w mod 4) .., columns 32 (w / 4) ..: acc0 + exp(dA[l]) acc1 + D x, bf16,
-  //    into the out tile (the cb buffer, free now), then out by TMA.
-  {
-    const int q4 = warp & 3, col0 = 32 * (warp >> 2);
-    const int row = 32 * q4 + (tid & 31);
-    const float el = ex2_approx(sdA[r0 + row] * kLog2e);
-    const uint32_t acc_state = tmem + kHd * (1 + (CS < kCs ? (32 * q4) / CS : 0));  // this warp's chunk
-#pragma unroll
-    for (int jj = 0; jj < 2; ++jj) {
-      uint32_t r0v[16], r1v[16];
-      const uint32_t lane_col = (static_cast<uint32_t>(32 * q4) << 16) + col0 + 16 * jj;
-      tmem_ld_x16(acc_intra + lane_col, r0v);
-      tmem_ld_x16(acc_state + lane_col, r1v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int j = (col0 + 16 * jj) / 8 + half;  // 16-byte chunk of the row: p = 8 j .. 8 j + 7
-        float xv[8], o[8];
-        unpack8(*reinterpret_cast<const uint4*>(smem + S::kX + sw128(row, j)), xv);  // the last pass's x rows
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          o[q] = fmaf(Dh, xv[q], fmaf(el, __uint_as_float(r1v[8 * half + q]), __uint_as_float(r0v[8 * half + q])));
-        *reinterpret_cast<uint4*>(smem + S::kCb + sw128(row, j)) = pack8(o);
-      }
-    }
-  }
+  }  // math warps
   fence_proxy_async_smem();
   __syncthreads();
   if (tid == 0) {
@@ -398,7 +421,7 @@ __global__ void __launch_bounds__(kSsdThreads) ssd_chunk_scan_kernel(
   }
   tcgen05_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kCtlWarp) {
     tcgen05_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
   }
