@@ -77,6 +77,31 @@ def test_block_small_against_the_oracle(b, L, Dm, E):
     print(f"block b={b} L={L} D={Dm} E={E}: out {e[0]:.2e} state {e[1]:.2e} cache {e[2]:.2e}")
 
 
+def test_block_both_projections_cut_along_k():
+    """b=1, L=64, D=128, E=1088: in_proj (64 x 2176 x 128) and out_proj
+    (64 x 128 x 1088) both cut tiles along K between CTA pairs. Their tile
+    counters lead the shared GEMM scratch and are zeroed once per block call;
+    in_proj's completing contributors set theirs back to zero, so out_proj
+    starts from zero (else out_proj's tiles would never be stored). The output
+    must match the oracle and be bit-equal over repeated calls on one
+    workspace, also when that workspace holds garbage (every counter -1, every
+    partial NaN) before the call."""
+    b, L, Dm, E = 1, 64, 128, 1088
+    M = b * L
+    assert api.proj_gemm_workspace_bytes(M, 2 * E, Dm) > 0 and api.proj_gemm_workspace_bytes(M, Dm, E) > 0
+    inp = inputs(b, L, Dm, E, seed=17)
+    ws = torch.empty(api.block_workspace_bytes(b, L, Dm, E), dtype=torch.uint8, device="cuda")
+    first = run_gpu(inp, workspace=ws)
+    e = check(first, run_oracle(inp), "block, both projections cut")
+    print(f"block b={b} L={L} D={Dm} E={E} (both projections cut): out {e[0]:.2e} state {e[1]:.2e} cache {e[2]:.2e}")
+    for i in range(3):
+        again = run_gpu(inp, workspace=ws)
+        assert all(torch.equal(x, y) for x, y in zip(first, again)), f"call {i + 2} differs"
+    ws.fill_(0xFF)  # garbage scratch: the call zeroes the counters it needs
+    again = run_gpu(inp, workspace=ws)
+    assert all(torch.equal(x, y) for x, y in zip(first, again)), "block on a garbage-filled workspace differs"
+
+
 def test_block_chained_calls_with_caches():
     b, L, Dm, E = 2, 260, 64, 128
     inp = inputs(b, L, Dm, E, seed=77)
