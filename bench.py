@@ -45,7 +45,7 @@ PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
-# The headline metric, printed identically by both arms (the benchmark's).
+# The headline metric, printed identically by both arms (the benchmark's stated metric).
 METRIC = "selective-scan channel-tokens/s; achieved HBM GB/s vs B200 peak"
 
 # SM resources used to derive the ALU roofline (B200, sm_100a): 148 SMs,
