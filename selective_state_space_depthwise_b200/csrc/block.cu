@@ -176,7 +176,10 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
                             v1 ? __bfloat162float(h[k * a.E + e0 + 1]) : 0.0f);
       x0 = hv[0], x1 = hv[1], x2 = hv[2];
     }
-#pragma unroll 8
+    // Fully unrolled: with one warp per SM sub-partition at the layer shape,
+    // the compiler needs the whole run to hide the window loads and the SFU
+    // latency (the 2048-token block measured 4.6% faster than with 8 rows).
+#pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int r = r0 + i;
       const float2 x3 = unpack_bf16x2(xt[(r + 3) * 32 + lane]);
