@@ -10,7 +10,7 @@
 //     tile (48 rows = the 33 outputs padded to a multiple of 16, zero-filled by
 //     TMA past row 33; 128-byte swizzled, the MMA's B operand) into a 3-slot
 //     ring, issued two chunks ahead;
-//  2. the four warps compute u = SiLU(conv1d(x)) for their 32 tokens (lane =
+//  2. the eight warps compute u = SiLU(conv1d(x)) for their 16 tokens (lane =
 //     channel pair, a 3-row sliding window in registers, the conv weights of
 //     the next chunk loaded one chunk ahead) and write it as bf16 straight
 //     into the MMA's A tile (2 slots), in the 128-byte swizzled K-major layout;
@@ -41,7 +41,13 @@ constexpr int kXpTok = 128;      // tokens per CTA (MMA M)
 constexpr int kXpK = 64;         // channels per chunk: 128 bytes of bf16, one swizzle row
 constexpr int kXpN = 48;         // MMA N: the 2N + 1 = 33 outputs padded to a multiple of 16
 constexpr int kXpOut = 33;
-constexpr int kXpThreads = 128;  // warp w owns TMEM lanes (tokens) 32w .. 32w + 31
+// Eight warps: warp w forms token rows 16w .. 16w + 15 of each A tile; in the
+// epilogue warps w and w + 4 read TMEM lanes (tokens) 32 (w mod 4) ..,
+// columns 0-31 and 32-47. Four warps of 32 rows left one warp per SM
+// sub-partition at the layer shape (one CTA per SM): x_proj alone took 49.0
+// against 40.9 us at 2048 tokens, 185 against 153 us at 16384.
+constexpr int kXpThreads = 256;
+constexpr int kXpRows = kXpTok / (kXpThreads / 32);  // A-tile rows per warp
 constexpr uint32_t kXpTmemCols = 64;
 constexpr int kXpStages = 3;     // x / W_x TMA ring
 constexpr int kXpMaxSplit = 8;   // portable cluster size
@@ -163,7 +169,7 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
     unsigned char* At = smem + S::kA + (j & 1) * S::kABytes;
     // window = tile rows r, r+1, r+2 (tokens t0 + r - 3 ..); rows before token 0 are
     // zero-filled by TMA and replaced by the incoming conv cache when there is one
-    const int r0 = 32 * warp;
+    const int r0 = kXpRows * warp;
     float2 x0 = unpack_bf16x2(xt[(r0 + 0) * 32 + lane]);
     float2 x1 = unpack_bf16x2(xt[(r0 + 1) * 32 + lane]);
     float2 x2 = unpack_bf16x2(xt[(r0 + 2) * 32 + lane]);
@@ -176,11 +182,11 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
                             v1 ? __bfloat162float(h[k * a.E + e0 + 1]) : 0.0f);
       x0 = hv[0], x1 = hv[1], x2 = hv[2];
     }
-    // Fully unrolled: with one warp per SM sub-partition at the layer shape,
-    // the compiler needs the whole run to hide the window loads and the SFU
-    // latency (the 2048-token block measured 4.6% faster than with 8 rows).
+    // Fully unrolled, so the compiler can hide the window loads and the SFU
+    // latency across the whole run (four warps with 8 of their 32 rows
+    // unrolled: 53 us at 2048 tokens).
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
+    for (int i = 0; i < kXpRows; ++i) {
       const int r = r0 + i;
       const float2 x3 = unpack_bf16x2(xt[(r + 3) * 32 + lane]);
       const float c0 =
@@ -226,12 +232,13 @@ __global__ void __launch_bounds__(kXpThreads) xproj_kernel(const __grid_constant
   // This CTA's partial [128 tokens][48] tile into shared memory (the x ring is free).
   float* P = reinterpret_cast<float*>(smem + S::kP);
   {
-    const int row = 32 * warp + lane;
-#pragma unroll
-    for (int jj = 0; jj < kXpN / 16; ++jj) {
+    const int q = warp & 3, row = 32 * q + lane;
+    // 16-column groups of the accumulator: warps 0-3 read groups 0 and 1, warps 4-7 group 2
+    const int jj0 = warp < 4 ? 0 : 2, jj1 = warp < 4 ? 2 : kXpN / 16;
+    for (int jj = jj0; jj < jj1; ++jj) {
       uint32_t r[16];
       if (last >= 0) {
-        tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 16 * jj, r);
+        tmem_ld_x16(tmem + (static_cast<uint32_t>(32 * q) << 16) + 16 * jj, r);
         tmem_ld_wait();
       } else {
 #pragma unroll
