@@ -265,6 +265,20 @@ def test_full_size_prefill_all_channels(name):
         print(f"{name} [{path}]: {format_report(rep)} over all {w.batch * w.d_inner} channels")
 
 
+@pytest.mark.parametrize("L", [2051, 4093])
+def test_layer_shape_ragged_tail_every_channel(L):
+    """E = 7680 (the benchmark's 240-CTA launch) with L not a multiple of the
+    32-token stage: the last stage's tokens past L must leave the state alone
+    (decay 1, no injection) and their outputs must not be stored. Both decay
+    paths and both kernels, against the oracle on every channel."""
+    w = W.WORKLOADS["axon_layer"].scaled(seqlen=L)
+    inp = device_inputs(w, gen_device="cuda")
+    runs = {f"k{k} d{d}": run_prefill(inp, tuning={"kernel": k, "decay_path": d}) for k in (3, 4) for d in (0, 1)}
+    reps = compare_full(w.io_dtype, inp, runs, label=f"L={L}")
+    for path, rep in reps.items():
+        print(f"axon_layer L={L} [{path}]: {format_report(rep)} over all {w.d_inner} channels")
+
+
 def test_full_size_decode_all_channels():
     """Prompt 512, then 1024 decode steps, against one oracle prefill of 1536,
     on every (sequence, channel)."""
