@@ -102,8 +102,11 @@ typedef struct {
  *   channels, warp j owns states 4j..4j+3 of each, the per-token work of the
  *   next 32-token stage overlaps the scan of the current one), built for three
  *   resident CTAs per SM; 4 = the same code built for two CTAs per SM (a larger
- *   register budget). Auto takes 4 when batch * ceil(d_inner / 32) <= 64 *
- *   SMs, else 3. Any other value returns SSM_ERR_INVALID_ARG.
+ *   register budget); 5 = warp-specialised: the same state slices in 4 warps
+ *   and the per-token work (conv, SiLU, dt, gate) of the next stage in 4 more,
+ *   handing over through mbarriers (two CTAs of 8 warps per SM). With
+ *   ctas = batch * ceil(d_inner / 32), auto takes 5 when ctas <= SMs, 4 when
+ *   ctas <= 64 * SMs, else 3. Any other value returns SSM_ERR_INVALID_ARG.
  * decay_path: 0 = auto; 1 = every decay exp(dt A_n) as its own exponential.
  *   Auto: a CTA whose 32 channels all have A_n = (n+1) A_0 within 2^-20
  *   relative (the "State initialization" of "Axon-SSM": diagonals -1..-16)
@@ -447,7 +450,7 @@ ssm_status ssm_segment_carry(const ssm_dims *dims, const ssm_weights *w, const f
 /* Reads and clears the device error word that kernels set when a bounded
  * wait gives up (synchronises `stream` first). SSM_OK if no kernel failed;
  * SSM_ERR_DEVICE with the code in ssm_last_error() otherwise. Codes: 1 the
- * prefill's TMA ring, 3-6 the block's x_proj kernel, 7-11 the chunk scan's
+ * prefill's TMA ring, 2 the hand-overs of prefill kernel 5, 3-6 the block's x_proj kernel, 7-11 the chunk scan's
  * operand and MMA waits, 11 the decode's state ring, 21-29 the projection
  * GEMM (21 ring slot free, 22 accumulator free, 23 operands landed, 24
  * accumulator full, 25 and 29 drains, 27-28 the cut-tile handshake),

@@ -46,7 +46,8 @@
 //
 // Kernels. 3: G = 4 with the register budget of three CTAs per SM; 4: G = 4
 // built for two CTAs per SM, whose larger register budget buys a deeper
-// schedule. Measured alternatives at the long-context shape: G = 2 (8 states
+// schedule; 5: the same state slices with phases A and C in four more warps
+// of the CTA, handing over through mbarriers (ws_run). Measured alternatives at the long-context shape: G = 2 (8 states
 // a thread) executes ~13% fewer instructions per channel-token but runs 1.28x
 // slower (one warp per SM sub-partition leaves dependency latencies exposed);
 // G = 8 (2 states a thread, 16 warps per SM) runs 1.36x slower: with two
@@ -211,7 +212,7 @@ __device__ __forceinline__ void fix_rows(float4* rows, int64_t t0, int64_t L, in
 // Per-token work of tokens [tb, tb + kTA) of this lane's channel for one
 // stage, as kTA / 2 token pairs that share each f32x2 operation. Outputs per
 // pair: the row (d, d', inj, inj') of decay operands and injections, D*u and
-// SiLU(z). Dr is the stage's dt_raw row. Tokens at or past L get the row of a
+// SiLU(z). Tokens at or past L get the row of a
 // token that changes nothing (decay 1, no injection). The caller stores the
 // rows (store_rows) after the scan, so no shared-memory store sits between
 // the scan's loads in program order.
@@ -234,12 +235,10 @@ __device__ __forceinline__ void phase_a_window(const T* __restrict__ X, int tb, 
 
 // Token pair t, t + 1 (t from the stage start; x = its conv window, 5 rows).
 template <typename T, Path P>
-__device__ __forceinline__ void phase_a_pair(const float* x, const T* __restrict__ Z, const float* __restrict__ Dr,
-                                             int t, int lane, const PhaseAConsts& k, float4& row, uint64_t& du2,
-                                             uint64_t& zg2) {
+__device__ __forceinline__ void phase_a_pair(const float* x, const T* __restrict__ Z, float2 dr, int t, int lane,
+                                             const PhaseAConsts& k, float4& row, uint64_t& du2, uint64_t& zg2) {
   const float c0 = fmaf(k.cw3, x[3], fmaf(k.cw2, x[2], fmaf(k.cw1, x[1], fmaf(k.cw0, x[0], k.cb))));
   const float c1 = fmaf(k.cw3, x[4], fmaf(k.cw2, x[3], fmaf(k.cw1, x[2], fmaf(k.cw0, x[1], k.cb))));
-  const float2 dr = *reinterpret_cast<const float2*>(Dr + t);  // broadcast
   const float z0 = IO<T>::to_f(Z[t * 32 + lane]), z1 = IO<T>::to_f(Z[(t + 1) * 32 + lane]);
   const uint64_t u2 = silu_pair(pk2(c0, c1));
   const uint64_t dt2 = dt_pair(ffma2(pk2(dr.x, dr.y), splat2(k.wdt), splat2(k.dtb)), k.lo, k.hi);
@@ -270,7 +269,9 @@ __device__ __forceinline__ void phase_a(const T* __restrict__ X, const T* __rest
   phase_a_window<T, kTA>(X, tb, lane, first, hx0, hx1, hx2, xw);
   const PhaseAConsts k{cw0, cw1, cw2, cw3, cb, wdt, dtb, Dd, lo, hi, a20};
 #pragma unroll
-  for (int p = 0; p < kTA / 2; ++p) phase_a_pair<T, P>(xw + 2 * p, Z, Dr, tb + 2 * p, lane, k, rows[p], du2[p], zg2[p]);
+  for (int p = 0; p < kTA / 2; ++p)
+    phase_a_pair<T, P>(xw + 2 * p, Z, *reinterpret_cast<const float2*>(Dr + tb + 2 * p), tb + 2 * p, lane, k, rows[p],
+                       du2[p], zg2[p]);  // dt_raw: a broadcast load
   fix_rows<P, kTA>(rows, t0, L, tb);
 }
 
@@ -588,10 +589,238 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
   }
 }
 
+// ------------------------------------------- warp-specialised CTA (kernel 5) ---
+// The same state slices as pipe_run (state warp j holds states 4j .. 4j + 3 of
+// its lane's channel), with the per-token work moved to four more warps of the
+// CTA: token warp k does phase A of tokens [8k, 8k + 8) of stage s + 1 and then
+// phase C of the same tokens of stage s, while the state warps scan stage s.
+// The two groups hand over through mbarriers, each a double buffer: rows of
+// decay operands and injections (token -> state warps) and partial readouts
+// (state -> token warps). No warp waits at a CTA-wide barrier, and with two
+// CTAs of eight warps every SM sub-partition holds four warps instead of two.
+// Token warp 0's lane 0 keeps the TMA ring of x, z, B and C filled; the gated
+// outputs leave by direct stores (each token a 32-channel row, one per lane).
+constexpr int kWsSlots = 4;     // ring depth (stage s + 4 is loaded once stage s is scanned)
+constexpr int kWsThreads = 256;  // 4 state warps, then 4 token warps
+constexpr int kWsTA = kTok / 4;  // phase-A and phase-C tokens per token warp and stage
+
+template <typename T>
+struct WsSmem {
+  static constexpr int kEs = static_cast<int>(sizeof(T));
+  static constexpr int kXBytes = (kTok + 3) * 32 * kEs;  // TMA box {32, kTok + 3}
+  static constexpr int kZBytes = kTok * 32 * kEs;        // TMA box {32, kTok}
+  static constexpr int kBCBytes = kTok * 16 * 4;         // TMA box {16, kTok}
+  static constexpr int kX = 0;
+  static constexpr int kZ = align128(kX + kXBytes);
+  static constexpr int kB = align128(kZ + kZBytes);
+  static constexpr int kC = kB + kBCBytes;
+  static constexpr int kSlot = align128(kC + kBCBytes);
+  static constexpr int kRowBytes = (kTok / 2) * 32 * 16;  // float4 [token pair][channel]
+  static constexpr int kRows = kWsSlots * kSlot;         // [2] row buffers
+  static constexpr int kPR = kTok + 4;                   // partial row (padded)
+  static constexpr int kPBytes = 4 * 32 * kPR * 4;       // float [slice][channel][kPR]
+  static constexpr int kP = kRows + 2 * kRowBytes;       // [2] partial buffers
+  static constexpr int kBar = kP + 2 * kPBytes;          // full[kWsSlots], then 4 pairs (below)
+  static constexpr int kTotal = kBar + (kWsSlots + 8) * 8;
+  static constexpr uint32_t kTxBytes = static_cast<uint32_t>(kXBytes + kZBytes + 2 * kBCBytes);
+};
+
+template <typename T, Path P>
+__device__ __forceinline__ void ws_run(const Maps& maps, const KernelArgs& a) {
+  using S = WsSmem<T>;
+  constexpr int kTA = kWsTA;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t full0 = sb + S::kBar;                 // ring slot landed (TMA transaction count)
+  const uint32_t rows_full = full0 + 8 * kWsSlots;     // rows of a stage written (128 token threads)
+  const uint32_t rows_free = rows_full + 16;           // rows of a stage read (128 state threads)
+  const uint32_t part_full = rows_free + 16;           // partials of a stage written (state threads)
+  const uint32_t part_free = part_full + 16;           // partials of a stage read (token threads)
+  float4* R = reinterpret_cast<float4*>(smem + S::kRows);
+  float* PB = reinterpret_cast<float*>(smem + S::kP);
+
+  const int tid = threadIdx.x;
+  const int warp = __shfl_sync(0xffffffffu, tid >> 5, 0), lane = tid & 31;
+  const int64_t tiles = (a.E + 31) / 32;
+  const int seq = static_cast<int>(blockIdx.x / tiles);
+  const int e0 = static_cast<int>(blockIdx.x % tiles) * 32;
+  const int64_t L = a.L;
+  const int64_t n_stages = (L + kTok - 1) / kTok;
+  const int e = e0 + lane;
+  const bool ch_ok = e < a.E;
+  const int64_t ec = ch_ok ? e : a.E - 1;
+  // A thread whose wait gave up (error word set) waits no more, so a broken
+  // hand-over ends the kernel after one time-out per thread, not one per stage.
+  bool live = true;
+  auto wait = [&](uint32_t bar, uint32_t parity) {
+    if (live) live = mbar_wait_bounded(bar, parity, a.err, 2);
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kWsSlots; ++i) mbar_init(full0 + 8 * i, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(rows_full + 8 * i, 128);
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp >= 4) {
+    // ---------------- token warps: phases A and C, and the TMA ring.
+    const int k = warp - 4, tb = k * kTA;
+    const bool issuer = tid == 128;
+    auto issue_stage = [&](int64_t st_idx) {
+      const int slot = static_cast<int>(st_idx % kWsSlots);
+      const uint32_t base = sb + slot * S::kSlot, bar = full0 + 8 * slot;
+      const int t0 = static_cast<int>(st_idx * kTok);
+      mbar_arrive_expect_tx(bar, S::kTxBytes);
+      tma_load_3d(base + S::kX, &maps.x, e0, t0 - 3, seq, bar);
+      tma_load_3d(base + S::kZ, &maps.z, e0, t0, seq, bar);
+      tma_load_3d(base + S::kB, &maps.B, 0, t0, seq, bar);
+      tma_load_3d(base + S::kC, &maps.C, 0, t0, seq, bar);
+    };
+    if (issuer) {
+      prefetch_tensormap(&maps.x);
+      prefetch_tensormap(&maps.z);
+      prefetch_tensormap(&maps.B);
+      prefetch_tensormap(&maps.C);
+      for (int64_t i = 0; i < kWsSlots && i < n_stages; ++i) issue_stage(i);
+    }
+    const PhaseAConsts kc{a.conv_w[ec * 4 + 0], a.conv_w[ec * 4 + 1], a.conv_w[ec * 4 + 2], a.conv_w[ec * 4 + 3],
+                          a.conv_b[ec], a.w_dt[ec], a.dt_bias[ec], a.D[ec], a.dt_min, a.dt_max,
+                          -expf(a.A_log[ec * 16]) * kLog2e};
+    float hx0 = 0.0f, hx1 = 0.0f, hx2 = 0.0f;
+    if (a.conv_cache_in) {
+      const T* hist = static_cast<const T*>(a.conv_cache_in) + static_cast<int64_t>(seq) * 3 * a.E + ec;
+      hx0 = IO<T>::to_f(hist[0]);
+      hx1 = IO<T>::to_f(hist[a.E]);
+      hx2 = IO<T>::to_f(hist[2 * a.E]);
+    }
+    // dt_raw: lane i holds token tb + (i & 7) of a stage, loaded a stage before its use.
+    const float* dtr = a.dt_raw + static_cast<int64_t>(seq) * a.s.dt_seq;
+    auto load_dr = [&](int64_t st_idx) -> float {
+      const int64_t t = st_idx * kTok + tb + (lane & 7);
+      return t < L ? __ldg(dtr + t) : 0.0f;
+    };
+    // Phase A of stage st_idx: rows to row buffer (st_idx & 1) once the state
+    // warps have read its previous contents (stage st_idx - 2).
+    auto phase_a_ws = [&](int64_t st_idx, float dr, uint64_t* du2, uint64_t* zg2) {
+      const int slot = static_cast<int>(st_idx % kWsSlots);
+      wait(full0 + 8 * slot, static_cast<uint32_t>((st_idx / kWsSlots) & 1));
+      const unsigned char* st = smem + slot * S::kSlot;
+      float xw[kTA + 3];
+      phase_a_window<T, kTA>(reinterpret_cast<const T*>(st + S::kX), tb, lane, st_idx == 0, hx0, hx1, hx2, xw);
+      float4 rows[kTA / 2];
+#pragma unroll
+      for (int p = 0; p < kTA / 2; ++p) {
+        const float2 d2 = make_float2(__shfl_sync(0xffffffffu, dr, 2 * p), __shfl_sync(0xffffffffu, dr, 2 * p + 1));
+        phase_a_pair<T, P>(xw + 2 * p, reinterpret_cast<const T*>(st + S::kZ), d2, tb + 2 * p, lane, kc, rows[p],
+                           du2[p], zg2[p]);
+      }
+      fix_rows<P, kTA>(rows, st_idx * kTok, L, tb);
+      const int b = static_cast<int>(st_idx & 1);
+      if (st_idx >= 2) wait(rows_free + 8 * b, static_cast<uint32_t>(((st_idx - 2) >> 1) & 1));
+      store_rows<kTA>(reinterpret_cast<float2*>(R + b * (kTok / 2) * 32), tb, lane, rows);
+      mbar_arrive(rows_full + 8 * b);
+    };
+
+    uint64_t du[kTA / 2], zg[kTA / 2], duN[kTA / 2], zgN[kTA / 2];
+    float dr_next = load_dr(0);
+    {
+      const float dr = dr_next;
+      dr_next = load_dr(1);
+      phase_a_ws(0, dr, du, zg);
+    }
+    T* Y = static_cast<T*>(a.y) + static_cast<int64_t>(seq) * a.s.y_seq + e;
+    for (int64_t s = 0; s < n_stages; ++s) {
+      const bool has_next = s + 1 < n_stages;
+      if (has_next) {
+        const float dr = dr_next;
+        dr_next = load_dr(s + 2);
+        phase_a_ws(s + 1, dr, duN, zgN);
+      }
+      // Phase C of stage s.
+      const int b = static_cast<int>(s & 1);
+      wait(part_full + 8 * b, static_cast<uint32_t>((s >> 1) & 1));
+      // Stage s is scanned and its phase A is long done: its slot takes stage s + kWsSlots.
+      if (issuer && s + kWsSlots < n_stages) issue_stage(s + kWsSlots);
+      float ys[kTA];
+      const float* Pp = PB + b * (S::kPBytes / 4) + lane * S::kPR + tb;
+#pragma unroll
+      for (int q = 0; q < kTA; q += 4) gate_pairs<4, 32 * S::kPR>(Pp + q, du + q / 2, zg + q / 2, ys + q);
+      mbar_arrive(part_free + 8 * b);
+      const int64_t t0 = s * kTok + tb;
+#pragma unroll
+      for (int i = 0; i < kTA; ++i)
+        if (ch_ok && t0 + i < L) Y[(t0 + i) * a.s.y_tok] = IO<T>::from_f(ys[i]);
+      if (has_next) {
+#pragma unroll
+        for (int i = 0; i < kTA / 2; ++i) {
+          du[i] = duN[i];
+          zg[i] = zgN[i];
+        }
+      }
+    }
+    if (k == 0 && ch_ok) {
+      // conv_cache_out = last 3 raw rows of [history, x]; read all before
+      // writing (the output may alias conv_cache_in).
+      const T* x = static_cast<const T*>(a.x);
+      const T* hist = static_cast<const T*>(a.conv_cache_in);
+      T keep[3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int64_t t = L - 3 + j;
+        if (t >= 0)
+          keep[j] = x[seq * a.s.x_seq + t * a.s.x_tok + e];
+        else
+          keep[j] = hist ? hist[(static_cast<int64_t>(seq) * 3 + (3 + t)) * a.E + e] : IO<T>::from_f(0.0f);
+      }
+      T* out = static_cast<T*>(a.conv_cache_out);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) out[(static_cast<int64_t>(seq) * 3 + j) * a.E + e] = keep[j];
+    }
+  } else {
+    // ---------------- state warps: phase B.
+    float a2[4], Av[4], h[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float A = -expf(a.A_log[ec * 16 + warp * 4 + q]);
+      Av[q] = A;
+      a2[q] = A * kLog2e;
+      h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + warp * 4 + q] : 0.0f;
+    }
+    const bool hi1 = (warp & 1) != 0, hi2 = (warp & 2) != 0;
+    float* Pj = PB + (warp * 32 + lane) * S::kPR;
+    for (int64_t s = 0; s < n_stages; ++s) {
+      const int slot = static_cast<int>(s % kWsSlots), b = static_cast<int>(s & 1);
+      wait(full0 + 8 * slot, static_cast<uint32_t>((s / kWsSlots) & 1));
+      wait(rows_full + 8 * b, static_cast<uint32_t>((s >> 1) & 1));
+      const unsigned char* st = smem + slot * S::kSlot;
+      const float* Bs = reinterpret_cast<const float*>(st + S::kB) + warp * 4;
+      const float* Cs = reinterpret_cast<const float*>(st + S::kC) + warp * 4;
+      float pr[kTok];
+      scan_stage<P, 4>(reinterpret_cast<const float2*>(R + b * (kTok / 2) * 32), lane, Av, a2, hi1, hi2, h, Bs, Cs,
+                       pr);
+      mbar_arrive(rows_free + 8 * b);
+      if (s >= 2) wait(part_free + 8 * b, static_cast<uint32_t>(((s - 2) >> 1) & 1));
+      float* Pw = Pj + b * (S::kPBytes / 4);
+#pragma unroll
+      for (int tl = 0; tl < kTok; tl += 4)
+        *reinterpret_cast<float4*>(Pw + tl) = make_float4(pr[tl], pr[tl + 1], pr[tl + 2], pr[tl + 3]);
+      mbar_arrive(part_full + 8 * b);
+    }
+    if (ch_ok) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) a.ssm_state_out[(static_cast<int64_t>(seq) * a.E + e) * 16 + warp * 4 + q] = h[q];
+    }
+  }
+  griddep_launch_dependents();  // the next kernel may be launched (it waits for this one to finish)
+}
+
 // True when every channel of this CTA has A_n = (n+1) A_0 to within kPowTol
-// (on the fp32 A = -expf(A_log) the kernel uses). Called by all G warps; warp
-// j checks states 16j/G .. 16(j+1)/G - 1 of its lane's channel.
-template <int G>
+// (on the fp32 A = -expf(A_log) the kernel uses). Called by all NT threads of
+// the CTA; warp j < G checks states 16j/G .. 16(j+1)/G - 1 of its lane's
+// channel (warps past G only vote).
+template <int G, int NT = 32 * G>
 __device__ __forceinline__ bool cta_has_power_decays(const KernelArgs& a) {
   const int64_t tiles = (a.E + 31) / 32;
   const int64_t e = (blockIdx.x % tiles) * 32 + (threadIdx.x & 31);
@@ -602,6 +831,7 @@ __device__ __forceinline__ bool cta_has_power_decays(const KernelArgs& a) {
   bool ok = true;
 #pragma unroll
   for (int v4 = 0; v4 < 4 / G; ++v4) {
+    if (NT > 32 * G && j >= G) break;
     const int q4 = j * (4 / G) + v4;
     const float4 v = row[q4];
     const float al[4] = {v.x, v.y, v.z, v.w};
@@ -645,6 +875,21 @@ __global__ void __launch_bounds__(32 * G, MINB) prefill_pipe_kernel(const __grid
       pipe_run<T, G, Path::kPow, SPLIT>(maps, a);
     else
       pipe_run<T, G, Path::kGeneric, SPLIT>(maps, a);
+  }
+}
+
+template <typename T, bool ZOH>
+__global__ void __launch_bounds__(kWsThreads, 2) prefill_ws_kernel(const __grid_constant__ Maps maps,
+                                                                    const KernelArgs a) {
+  griddep_wait();  // as in prefill_pipe_kernel
+  if constexpr (ZOH) {
+    ws_run<T, Path::kZoh>(maps, a);
+  } else {
+    const bool pw = a.decay_path == 0 && cta_has_power_decays<4, kWsThreads>(a);
+    if (pw)
+      ws_run<T, Path::kPow>(maps, a);
+    else
+      ws_run<T, Path::kGeneric>(maps, a);
   }
 }
 
@@ -728,23 +973,53 @@ cudaError_t launch_pipe(const KernelArgs& a, cudaStream_t st, bool pdl) {
 }
 
 template <typename T, bool ZOH>
+cudaError_t launch_ws(const KernelArgs& a, cudaStream_t st, bool pdl) {
+  Maps maps;
+  if (!make_maps<T>(a, &maps)) return cudaErrorInvalidValue;
+  auto kern = prefill_ws_kernel<T, ZOH>;
+  const int smem = WsSmem<T>::kTotal + 128;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  const int64_t grid = a.batch * ((a.E + 31) / 32);
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kWsThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  err = cudaLaunchKernelEx(&cfg, kern, maps, a);
+  if (err != cudaSuccess) return err;
+  return cudaGetLastError();
+}
+
+template <typename T, bool ZOH>
 cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st, bool pdl) {
   if (sh.kernel == 3) return launch_pipe<T, 4, ZOH, 0>(a, st, pdl);
   if (sh.kernel == 4) return launch_pipe<T, 4, ZOH, 1>(a, st, pdl);
+  if (sh.kernel == 5) return launch_ws<T, ZOH>(a, st, pdl);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool prefill_shape_supported(PrefillShape sh) { return sh.kernel == 3 || sh.kernel == 4; }
+bool prefill_shape_supported(PrefillShape sh) { return sh.kernel >= 3 && sh.kernel <= 5; }
 
-// Pipelined state slices: the register-rich build (two CTAs per SM), except
-// for grids of many waves. Measured on B200: kernel 4 matched or beat kernel 3
-// from 80 to 5120 CTAs (by 1-27%); at 61440 CTAs (256 sequences of 7680
-// channels) kernel 3 was 2.6% faster.
+// Measured on B200 at L = 16384: with at most one CTA per SM the
+// warp-specialised kernel 5 was 4% faster than kernel 4 on the power path and
+// 20% faster on the per-state path (32 to 148 CTAs); from two CTAs per SM on
+// it was 8% slower on the power path (160 to 296 CTAs), so the register-rich
+// kernel 4 takes those grids. Kernel 4 matched or beat kernel 3 from 80 to
+// 5120 CTAs (by 1-27%); at 61440 CTAs (256 sequences of 7680 channels)
+// kernel 3 was 2.6% faster.
 PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int num_sms) {
-  const int64_t ctas = batch * ((E + 31) / 32);
-  return PrefillShape{ctas <= 64 * static_cast<int64_t>(num_sms > 0 ? num_sms : 148) ? 4 : 3};
+  const int64_t ctas = batch * ((E + 31) / 32), sms = num_sms > 0 ? num_sms : 148;
+  if (ctas <= sms) return PrefillShape{5};
+  return PrefillShape{ctas <= 64 * sms ? 4 : 3};
 }
 
 cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st, bool pdl) {

@@ -196,7 +196,7 @@ ssm_status prefill_entry(const ssm_dims* dims, const ssm_weights* w, const void*
   if (tuning) {
     if (tuning->kernel) sh.kernel = tuning->kernel;
     if (!ssm::prefill_shape_supported(sh))
-      return fail(SSM_ERR_INVALID_ARG, "tuning: kernel=%d is not built (3 or 4)", sh.kernel);
+      return fail(SSM_ERR_INVALID_ARG, "tuning: kernel=%d is not built (3, 4 or 5)", sh.kernel);
     if (tuning->decay_path != 0 && tuning->decay_path != 1)
       return fail(SSM_ERR_INVALID_ARG, "tuning: decay_path=%d (0 = auto, 1 = per-state exponentials)",
                   tuning->decay_path);

@@ -42,7 +42,8 @@ struct KernelArgs {
 };
 
 // Prefill launch shape: kernel 3 (pipelined state slices, register budget of
-// three CTAs per SM) or kernel 4 (the same at two CTAs per SM).
+// three CTAs per SM), kernel 4 (the same at two CTAs per SM) or kernel 5 (the
+// state slices and the per-token work in separate warps of one CTA).
 struct PrefillShape {
   int kernel;
 };

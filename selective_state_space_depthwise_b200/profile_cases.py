@@ -8,7 +8,7 @@
     python -m selective_state_space_depthwise_b200.profile_cases gemm M N K
 
 prefill: three launches of the named workload's prefill (optionally shortened
-to L tokens, optionally with an explicit kernel (3 or 4) and decay path (0 auto,
+to L tokens, optionally with an explicit kernel (3, 4 or 5) and decay path (0 auto,
 1 per-state exponentials), and E channels); decode: a 4-token
 prompt, then three decode steps at the decode workload's shape (batch 256,
 E=7680, 252 MB of state); block: three block forwards of the named block

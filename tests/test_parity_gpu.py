@@ -17,10 +17,12 @@ from selective_state_space_depthwise_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 # (kernel, decay path): kernel 3 / 4 = pipelined state slices, 4 warps per 32
-# channels, at a register budget of 3 / 2 CTAs per SM; decay path 0 = auto
-# (powers of one exponential where A_n = (n+1) A_0, which the workloads' A
-# initialisation satisfies), 1 = one exponential per state.
-SHAPES = [(3, 0), (3, 1), (4, 0), (4, 1)]
+# channels, at a register budget of 3 / 2 CTAs per SM; kernel 5 = the same
+# slices with the per-token work in 4 more warps (warp-specialised); decay
+# path 0 = auto (powers of one exponential where A_n = (n+1) A_0, which the
+# workloads' A initialisation satisfies), 1 = one exponential per state.
+KERNELS = (3, 4, 5)
+SHAPES = [(k, d) for k in KERNELS for d in (0, 1)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -73,7 +75,7 @@ def test_kernel_lengths_history_and_zoh(shape):
         compare(torch.bfloat16, gather(y, cc, st, chans), want, label=f"kernel {kern} path {d} L{L} {disc}")
 
 
-@pytest.mark.parametrize("kernel", [3, 4])
+@pytest.mark.parametrize("kernel", KERNELS)
 @pytest.mark.parametrize("io_dtype", [torch.float32, torch.bfloat16])
 def test_decay_paths_mixed_channels(io_dtype, kernel):
     """A_log perturbed in some 32-channel tiles (and in one single channel of
@@ -248,13 +250,15 @@ def test_decode_zoh():
 @pytest.mark.parametrize("name", ["axon_layer", "batched", "long_context"])
 def test_full_size_prefill_all_channels(name):
     """The workload at full size, in the default launch shape the benchmark
-    times (auto decay path: powers of one exponential, since the workloads use
+    times and in the warp-specialised kernel 5 (auto decay path: powers of one exponential, since the workloads use
     the pages' A initialisation) and with one exponential per state, against
     the oracle on every (sequence, channel). The long-context workload also
     reports its two clip-stressed channel subsets on their own."""
     w = W.WORKLOADS[name]
     inp = device_inputs(w, gen_device="cuda")
-    runs = {"auto": run_prefill(inp), "per-state": run_prefill(inp, tuning={"decay_path": 1})}
+    runs = {"auto": run_prefill(inp), "per-state": run_prefill(inp, tuning={"decay_path": 1}),
+            "k5 auto": run_prefill(inp, tuning={"kernel": 5}),
+            "k5 per-state": run_prefill(inp, tuning={"kernel": 5, "decay_path": 1})}
     lo, hi = W.clip_stress_channels(w)
     subsets = {"dt at dt_min": lo.tolist(), "dt at dt_max": hi.tolist()} if w.clip_stress else None
     if subsets:
@@ -273,7 +277,7 @@ def test_layer_shape_ragged_tail_every_channel(L):
     paths and both kernels, against the oracle on every channel."""
     w = W.WORKLOADS["axon_layer"].scaled(seqlen=L)
     inp = device_inputs(w, gen_device="cuda")
-    runs = {f"k{k} d{d}": run_prefill(inp, tuning={"kernel": k, "decay_path": d}) for k in (3, 4) for d in (0, 1)}
+    runs = {f"k{k} d{d}": run_prefill(inp, tuning={"kernel": k, "decay_path": d}) for k in KERNELS for d in (0, 1)}
     reps = compare_full(w.io_dtype, inp, runs, label=f"L={L}")
     for path, rep in reps.items():
         print(f"axon_layer L={L} [{path}]: {format_report(rep)} over all {w.d_inner} channels")
