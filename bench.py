@@ -58,8 +58,11 @@ SMS, SFU_PER_CLK, FMA_PER_CLK = 148, 16, 128
 #    (dt*A, dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 84 FP32-pipe ops;
 #  powers (A_n = (n+1) A_0): 1 exp (q) + 2 sigmoid + 1 softplus = 6 SFU-class
 #    evaluations; 15 multiplies for q^2..q^16, then 3 FP32 ops per state
-#    (dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 83 FP32-pipe ops.
-ALU_MODEL = {"per_state": (22, 84), "power": (6, 83)}
+#    (dt*u*B, h FMA, readout FMA) + ~20 scalar ops = 83 FP32-pipe ops;
+#  zero-order hold: the per-state SFU work (22); 7 FP32 ops per state (dt*A,
+#    e^{dt A} - 1, times 1/A, times u, times B, h FMA, readout FMA) + ~20
+#    scalar ops = 132 FP32-pipe ops.
+ALU_MODEL = {"per_state": (22, 84), "power": (6, 83), "zoh": (22, 132)}
 POLY_EXP_FMA_OPS = 8
 
 
@@ -285,13 +288,13 @@ def make_device_inputs(w: W.Workload, rank: int):
     return W.make_inputs(wr, device="cuda", gen_device="cuda")
 
 
-def timed_prefill(inp, steps, warmup, dist, tuning=None, clocks=True):
+def timed_prefill(inp, steps, warmup, dist, tuning=None, clocks=True, disc="euler"):
     from selective_state_space_depthwise_b200 import api
 
     args = (inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp)
-    y, cc, st = api.prefill(*args, tuning=tuning)
+    y, cc, st = api.prefill(*args, tuning=tuning, discretization=disc)
     for _ in range(warmup):
-        api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st, tuning=tuning)
+        api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st, tuning=tuning, discretization=disc)
     stream = torch.cuda.current_stream()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
@@ -300,7 +303,7 @@ def timed_prefill(inp, steps, warmup, dist, tuning=None, clocks=True):
     with ClockSampler(torch.cuda.current_device()) if clocks else _NoClock() as clk:
         ev0.record(stream)
         for _ in range(steps):
-            api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st, tuning=tuning)
+            api.prefill(*args, y=y, conv_cache_out=cc, ssm_state_out=st, tuning=tuning, discretization=disc)
         ev1.record(stream)
         torch.cuda.synchronize()
     if dist:
@@ -333,15 +336,21 @@ def prefill_figures(w: W.Workload, ms_step: float, hbm_peak: float, peak_kind: s
                     "peak_kind": peak_kind, "algorithmic_bytes_per_launch": min_bytes_prefill(w)}}
 
 
-def decay_path_bench(w: W.Workload, inp, hbm_peak: float, peak_kind: str, steps: int = 10, warmup: int = 3):
-    """The same workload on each decay path, CUDA events, inputs resident."""
+def decay_path_bench(w: W.Workload, inp, hbm_peak: float, peak_kind: str, steps: int = 10, warmup: int = 3,
+                     zoh: bool = False):
+    """The same workload on each decay path (and, with zoh, the zero-order-hold
+    discretisation), CUDA events, inputs resident."""
     out = {}
-    for name, path, tun in (("power", "power", None), ("per_state", "per_state", {"decay_path": 1})):
-        ms, _ = timed_prefill(inp, steps, warmup, False, tuning=tun, clocks=False)
+    runs = [("power", "power", None, "euler"), ("per_state", "per_state", {"decay_path": 1}, "euler")]
+    if zoh:
+        runs.append(("zoh", "zoh", None, "zoh"))
+    for name, path, tun, disc in runs:
+        ms, _ = timed_prefill(inp, steps, warmup, False, tuning=tun, clocks=False, disc=disc)
         out[name] = prefill_figures(w, ms / steps, hbm_peak, peak_kind, path)
     out["note"] = ("power: decays as powers of q = exp(dt A_0), taken automatically by every CTA whose channels "
                    "have A_n = (n+1) A_0 (the workloads' A initialisation); per_state: one exponential per state "
-                   "(forced with decay_path = 1; the path for any other A)")
+                   "(forced with decay_path = 1; the path for any other A)" +
+                   ("; zoh: zero-order-hold discretisation (per-state exponentials)" if zoh else ""))
     return out
 
 
@@ -807,7 +816,7 @@ def main():
     # with N ranks they would hold every GPU while rank 0 alone works.
     subs = world == 1
     if subs:
-        extra["decay_paths"] = decay_path_bench(w, inp, hbm_peak, peak_kind)
+        extra["decay_paths"] = decay_path_bench(w, inp, hbm_peak, peak_kind, zoh=True)
     if not args.no_e2e:
         # Every rank moves its own inputs through the host path at the same time;
         # the job's time is the slowest rank's (CUDA events, max over ranks).

@@ -105,8 +105,10 @@ typedef struct {
  *   register budget); 5 = warp-specialised: the same state slices in 4 warps
  *   and the per-token work (conv, SiLU, dt, gate) of the next stage in 4 more,
  *   handing over through mbarriers (two CTAs of 8 warps per SM). With
- *   ctas = batch * ceil(d_inner / 32), auto takes 5 when ctas <= SMs, 4 when
- *   ctas <= 64 * SMs, else 3. Any other value returns SSM_ERR_INVALID_ARG.
+ *   ctas = batch * ceil(d_inner / 32), auto takes 5 when ctas <= SMs; else,
+ *   up to 64 * SMs, 5 when every CTA runs per-state exponentials (ZOH, or
+ *   decay_path = 1) and 4 otherwise; else 3. Any other value returns
+ *   SSM_ERR_INVALID_ARG.
  * decay_path: 0 = auto; 1 = every decay exp(dt A_n) as its own exponential.
  *   Auto: a CTA whose 32 channels all have A_n = (n+1) A_0 within 2^-20
  *   relative (the "State initialization" of "Axon-SSM": diagonals -1..-16)

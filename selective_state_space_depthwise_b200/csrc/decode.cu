@@ -70,6 +70,7 @@ struct ChannelParams {
   float cb, wdt, dtb, D;
   float a2[16];  // A * log2(e)
   float A[16];   // A itself (ZOH only)
+  float rA[16];  // 1 / A (ZOH only)
 };
 
 // Rows of the staged per-sequence inputs: B (16), C (16), dt_raw (1), padding.
@@ -101,7 +102,7 @@ __device__ __forceinline__ void decode_step_item(const KernelArgs& a, int64_t se
         const float A = p.A[4 * q + i];
         const float xa = dt * A;
         const float dA = ex2_approx(xa * kLog2e);
-        hs[i] = fmaf(dA, hs[i], expm1_nonpos(xa, dA) / A * u * bv[i]);
+        hs[i] = fmaf(dA, hs[i], zoh_scale(xa, dt, dA, p.rA[4 * q + i]) * u * bv[i]);
         yl = fmaf(cv[i], hs[i], yl);
       }
       it.h[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
@@ -152,6 +153,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_resident_kernel(const K
       for (int i = 0; i < 4; ++i) {
         const float A = -ex2_approx(lv[i] * kLog2e);  // A = -exp(A_log)
         p.A[4 * q + i] = A;
+        p.rA[4 * q + i] = 1.0f / A;
         p.a2[4 * q + i] = A * kLog2e;
       }
     }
@@ -244,6 +246,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_tma_kernel(const __grid
       for (int i = 0; i < 4; ++i) {
         const float A = -ex2_approx(lv[i] * kLog2e);  // A = -exp(A_log)
         p.A[4 * q + i] = A;
+        p.rA[4 * q + i] = 1.0f / A;
         p.a2[4 * q + i] = A * kLog2e;
       }
     }
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_tma_kernel(const __grid
             const float A = p.A[4 * q + i];
             const float xa = dt * A;
             const float dA = ex2_approx(xa * kLog2e);
-            hs[i] = fmaf(dA, hs[i], expm1_nonpos(xa, dA) / A * u * bv[i]);
+            hs[i] = fmaf(dA, hs[i], zoh_scale(xa, dt, dA, p.rA[4 * q + i]) * u * bv[i]);
             yl = fmaf(cv[i], hs[i], yl);
           }
           h[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);

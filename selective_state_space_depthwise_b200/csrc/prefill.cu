@@ -144,19 +144,48 @@ __device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const f
   return lo + hi;
 }
 
-// Zero-order-hold decays (scalar): h = e^{dt A} h + (e^{dt A} - 1)/A * u * B.
+// Zero-order-hold decays, in state pairs: h = e^{dt A} h + (e^{dt A} - 1)/A
+// * u * B, the input scale as zoh_scale forms it (rA = 1 / A), each half of a
+// packed operation rounding as the scalar form does.
+__device__ __forceinline__ uint64_t zoh_scale_pair(uint64_t x, uint64_t dt2, uint64_t ex, uint64_t rA) {
+  uint64_t p = ffma2(x, pk2(1.0f / 120.0f, 1.0f / 120.0f), pk2(1.0f / 24.0f, 1.0f / 24.0f));
+  p = ffma2(x, p, pk2(1.0f / 6.0f, 1.0f / 6.0f));
+  p = ffma2(x, p, pk2(0.5f, 0.5f));
+  p = ffma2(x, p, pk2(1.0f, 1.0f));
+  float s0, s1, l0, l1, x0, x1;
+  upk2(fmul2(dt2, p), s0, s1);
+  upk2(fmul2(fadd2(ex, pk2(-1.0f, -1.0f)), rA), l0, l1);
+  upk2(x, x0, x1);
+  return pk2(x0 > -0.125f ? s0 : l0, x1 > -0.125f ? s1 : l1);
+}
 template <int K>
-__device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* Av, float* h, const float* Bp,
-                                                const float* Cp) {
-  float acc = 0.0f;
+__device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* Av, const float* rA, float* h,
+                                                const float* Bp, const float* Cp) {
+  static_assert(K % 4 == 0, "states in groups of 4");
+  const uint64_t dt2 = pk2(dt, dt), u2 = pk2(u, u);
+  uint64_t acc = 0;
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
-    const float xa = dt * Av[q];
-    const float dA = ex2_approx(xa * kLog2e);
-    h[q] = fmaf(dA, h[q], expm1_nonpos(xa, dA) / Av[q] * u * Bp[q]);
-    acc = fmaf(Cp[q], h[q], acc);
+  for (int q = 0; q < K; q += 4) {
+    const float4 bq = *reinterpret_cast<const float4*>(Bp + q);
+    const float4 cq = *reinterpret_cast<const float4*>(Cp + q);
+#pragma unroll
+    for (int r = 0; r < 4; r += 2) {
+      const int i = q + r;
+      const uint64_t x = fmul2(dt2, pk2(Av[i], Av[i + 1]));
+      float l0, l1;
+      upk2(fmul2(x, pk2(kLog2e, kLog2e)), l0, l1);
+      const uint64_t ex = pk2(ex2_approx(l0), ex2_approx(l1));
+      const uint64_t c = zoh_scale_pair(x, dt2, ex, pk2(rA[i], rA[i + 1]));
+      const uint64_t b2 = r == 0 ? pk2(bq.x, bq.y) : pk2(bq.z, bq.w);
+      const uint64_t c2 = r == 0 ? pk2(cq.x, cq.y) : pk2(cq.z, cq.w);
+      const uint64_t hh = ffma2(ex, pk2(h[i], h[i + 1]), fmul2(fmul2(c, u2), b2));
+      upk2(hh, h[i], h[i + 1]);
+      acc = i == 0 ? fmul2(c2, hh) : ffma2(c2, hh, acc);
+    }
   }
-  return acc;
+  float lo, hi;
+  upk2(acc, lo, hi);
+  return lo + hi;
 }
 
 // Decay operand stored per token: dt (generic), q = e^{dt A_0} (power path),
@@ -348,8 +377,8 @@ __device__ __forceinline__ void scan_stage_la(Prep prep, float* h, float* pr) {
 // Phase B over tokens [T0, T1) of one stage: this thread's 4 states; pr gets
 // the partial readouts.
 template <Path P, int K, int T0 = 0, int T1 = kTok>
-__device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int lane, const float* Av, const float* a2,
-                                           bool hi1, bool hi2, float* h, const float* __restrict__ Bs,
+__device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int lane, const float* Av, const float* rA,
+                                           const float* a2, bool hi1, bool hi2, float* h, const float* __restrict__ Bs,
                                            const float* __restrict__ Cs, float* pr) {
   if constexpr (P == Path::kPow) {
     static_assert(K == 4, "power decays are built for 4 states per thread");
@@ -360,7 +389,7 @@ __device__ __forceinline__ void scan_stage(const float2* __restrict__ DTc, int l
       const float4 d4 = reinterpret_cast<const float4*>(DTc)[(tl >> 1) * 32 + lane];
       const float2 dd = (tl & 1) ? make_float2(d4.y, d4.w) : make_float2(d4.x, d4.z);
       if constexpr (P == Path::kZoh)
-        pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, h, Bs + tl * 16, Cs + tl * 16);
+        pr[tl] = scan_token_zoh<K>(dd.x, dd.y, Av, rA, h, Bs + tl * 16, Cs + tl * 16);
       else
         pr[tl] = scan_token<K / 2>(pk2(dd.x, dd.x), pk2(dd.y, dd.y), a2, h, Bs + tl * 16, Cs + tl * 16);
     }
@@ -459,11 +488,12 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
     hx1 = IO<T>::to_f(hist[a.E]);
     hx2 = IO<T>::to_f(hist[2 * a.E]);
   }
-  float a2[kK], Av[kK], h[kK];
+  float a2[kK], Av[kK], rA[kK], h[kK];
 #pragma unroll
   for (int q = 0; q < kK; ++q) {
     const float A = -expf(a.A_log[ec * 16 + warp * kK + q]);
     Av[q] = A;
+    rA[q] = 1.0f / A;  // ZOH only
     a2[q] = A * kLog2e;
     h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + warp * kK + q] : 0.0f;
   }
@@ -508,14 +538,14 @@ __device__ __forceinline__ void pipe_run(const Maps& maps, const KernelArgs& a) 
       // and 5% faster on the power path than one token pair of the next
       // stage after every 8 tokens of the scan).
       float4 rows[kTA / 2];
-      scan_stage<P, kK, 0, kTok / 2>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      scan_stage<P, kK, 0, kTok / 2>(DTc, lane, Av, rA, a2, hi1, hi2, h, Bs, Cs, pr);
       phase_a<T, P, kTA>(reinterpret_cast<const T*>(nst + S::kX), reinterpret_cast<const T*>(nst + S::kZ),
                          Dr + ((s + 1) & 1) * kTok, t0 + kTok, L, tb, lane, false, hx0, hx1, hx2, cw0, cw1, cw2, cw3,
                          cb, wdt, dtb, Dd, lo, hi, a20, rows, duN, zgN);
-      scan_stage<P, kK, kTok / 2, kTok>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      scan_stage<P, kK, kTok / 2, kTok>(DTc, lane, Av, rA, a2, hi1, hi2, h, Bs, Cs, pr);
       store_rows<kTA>(DTn, tb, lane, rows);
     } else {
-      scan_stage<P, kK>(DTc, lane, Av, a2, hi1, hi2, h, Bs, Cs, pr);
+      scan_stage<P, kK>(DTc, lane, Av, rA, a2, hi1, hi2, h, Bs, Cs, pr);
     }
 #pragma unroll
     for (int tl = 0; tl < kTok; tl += 4)
@@ -780,11 +810,12 @@ __device__ __forceinline__ void ws_run(const Maps& maps, const KernelArgs& a) {
     }
   } else {
     // ---------------- state warps: phase B.
-    float a2[4], Av[4], h[4];
+    float a2[4], Av[4], rA[4], h[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float A = -expf(a.A_log[ec * 16 + warp * 4 + q]);
       Av[q] = A;
+      rA[q] = 1.0f / A;  // ZOH only
       a2[q] = A * kLog2e;
       h[q] = a.ssm_state_in ? a.ssm_state_in[(static_cast<int64_t>(seq) * a.E + ec) * 16 + warp * 4 + q] : 0.0f;
     }
@@ -798,8 +829,8 @@ __device__ __forceinline__ void ws_run(const Maps& maps, const KernelArgs& a) {
       const float* Bs = reinterpret_cast<const float*>(st + S::kB) + warp * 4;
       const float* Cs = reinterpret_cast<const float*>(st + S::kC) + warp * 4;
       float pr[kTok];
-      scan_stage<P, 4>(reinterpret_cast<const float2*>(R + b * (kTok / 2) * 32), lane, Av, a2, hi1, hi2, h, Bs, Cs,
-                       pr);
+      scan_stage<P, 4>(reinterpret_cast<const float2*>(R + b * (kTok / 2) * 32), lane, Av, rA, a2, hi1, hi2, h, Bs,
+                       Cs, pr);
       mbar_arrive(rows_free + 8 * b);
       if (s >= 2) wait(part_free + 8 * b, static_cast<uint32_t>(((s - 2) >> 1) & 1));
       float* Pw = Pj + b * (S::kPBytes / 4);
@@ -1009,17 +1040,20 @@ cudaError_t dispatch(const KernelArgs& a, PrefillShape sh, cudaStream_t st, bool
 
 bool prefill_shape_supported(PrefillShape sh) { return sh.kernel >= 3 && sh.kernel <= 5; }
 
-// Measured on B200 at L = 16384: with at most one CTA per SM the
-// warp-specialised kernel 5 was 4% faster than kernel 4 on the power path and
-// 20% faster on the per-state path (32 to 148 CTAs); from two CTAs per SM on
-// it was 8% slower on the power path (160 to 296 CTAs), so the register-rich
-// kernel 4 takes those grids. Kernel 4 matched or beat kernel 3 from 80 to
-// 5120 CTAs (by 1-27%); at 61440 CTAs (256 sequences of 7680 channels)
-// kernel 3 was 2.6% faster.
-PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int num_sms) {
+// Measured on B200 (L = 16384 unless stated): with at most one CTA per SM
+// the warp-specialised kernel 5 was 4% faster than kernel 4 on the power path
+// and 20% faster on the per-state path (32 to 148 CTAs). From two CTAs per SM
+// on it was 8% slower on the power path (160 to 296 CTAs), so the
+// register-rich kernel 4 takes those grids, unless every CTA is known to run
+// per-state exponentials (ZOH, or per-state decays forced): there kernel 5
+// was level at 240 CTAs and 2-8% faster from 480 to 15360 CTAs. Kernel 4
+// matched or beat kernel 3 from 80 to 5120 CTAs (by 1-27%); at 61440 CTAs
+// (256 sequences of 7680 channels) kernel 3 was 2.6% faster.
+PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t /*L*/, int num_sms, bool per_state) {
   const int64_t ctas = batch * ((E + 31) / 32), sms = num_sms > 0 ? num_sms : 148;
   if (ctas <= sms) return PrefillShape{5};
-  return PrefillShape{ctas <= 64 * sms ? 4 : 3};
+  if (ctas > 64 * sms) return PrefillShape{3};
+  return PrefillShape{per_state ? 5 : 4};
 }
 
 cudaError_t launch_prefill(const KernelArgs& a, bool io_bf16, bool zoh, PrefillShape sh, cudaStream_t st, bool pdl) {

@@ -116,12 +116,15 @@ __global__ void __launch_bounds__(kSegThreads, ZOH ? 4 : SSM_SEG_MINB) segment_b
   const float4 cw = *reinterpret_cast<const float4*>(a.conv_w + ec * 4);
   const float cb = a.conv_b[ec], wdt = a.w_dt[ec], dtb = a.dt_bias[ec];
   float a2[kN];  // A_n log2(e)
-  float An[ZOH ? kN : 1];
+  float An[ZOH ? kN : 1], rAn[ZOH ? kN : 1];  // A_n and 1 / A_n (ZOH only)
 #pragma unroll
   for (int n = 0; n < kN; ++n) {
     const float A = -expf(a.A_log[ec * kN + n]);
     a2[n] = A * kLog2e;
-    if constexpr (ZOH) An[n] = A;
+    if constexpr (ZOH) {
+      An[n] = A;
+      rAn[n] = 1.0f / A;
+    }
   }
   float acc[kN];
 #pragma unroll
@@ -187,7 +190,7 @@ __global__ void __launch_bounds__(kSegThreads, ZOH ? 4 : SSM_SEG_MINB) segment_b
           for (int i = 0; i < 4; ++i) {
             const int n = 4 * q + i;
             const float xa = dt * An[n];
-            const float inj = u * bq[i] * expm1_nonpos(xa, ex2_approx(xa * kLog2e)) / An[n];
+            const float inj = u * bq[i] * zoh_scale(xa, dt, ex2_approx(xa * kLog2e), rAn[n]);
             acc[n] = fmaf(ex2_approx(a2[n] * R), inj, acc[n]);
           }
         }

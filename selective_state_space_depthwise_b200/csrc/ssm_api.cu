@@ -191,7 +191,9 @@ ssm_status prefill_entry(const ssm_dims* dims, const ssm_weights* w, const void*
   }
   if ((st = check_prefill_caches(conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out)) != SSM_OK) return st;
 
-  ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current());
+  const bool per_state = dims->discretization == SSM_DISC_ZOH || (tuning && tuning->decay_path == 1);
+  ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current(),
+                                                   per_state);
   int decay_path = 0;
   if (tuning) {
     if (tuning->kernel) sh.kernel = tuning->kernel;

@@ -48,7 +48,9 @@ struct PrefillShape {
   int kernel;
 };
 
-PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t L, int num_sms);
+// per_state: every CTA will run per-state exponentials (ZOH, or per-state
+// decays forced), as opposed to the per-CTA choice of the auto decay path.
+PrefillShape choose_prefill_shape(int64_t batch, int64_t E, int64_t L, int num_sms, bool per_state);
 bool prefill_shape_supported(PrefillShape sh);
 // pdl: overlap the launch with the kernel before it on the stream (that must
 // be a kernel, not a copy or memset); the kernel reads its inputs only after

@@ -67,14 +67,16 @@ __device__ __forceinline__ float softplus(float v) {
 // dt = clip(softplus(v), lo, hi).
 __device__ __forceinline__ float dt_of(float v, float lo, float hi) { return fminf(fmaxf(softplus(v), lo), hi); }
 
-// e^x - 1 for x <= 0, given ex = e^x: Taylor series near 0, ex - 1 elsewhere.
-__device__ __forceinline__ float expm1_nonpos(float x, float ex) {
+// The zero-order-hold input scale (e^x - 1) / A for x = dt A <= 0, given
+// ex = e^x and rA = 1 / A: near 0 as dt (e^x - 1) / x by its Taylor series
+// (dt (1 + x/2 + x^2/6 + x^3/24 + x^4/120), no cancellation, no division),
+// elsewhere (ex - 1) * rA.
+__device__ __forceinline__ float zoh_scale(float x, float dt, float ex, float rA) {
   float p = fmaf(x, 1.0f / 120.0f, 1.0f / 24.0f);
   p = fmaf(x, p, 1.0f / 6.0f);
   p = fmaf(x, p, 0.5f);
   p = fmaf(x, p, 1.0f);
-  const float series = x * p;
-  return x > -0.125f ? series : ex - 1.0f;
+  return x > -0.125f ? dt * p : (ex - 1.0f) * rA;
 }
 
 // 2^x for x <= 0 on the FMA pipe, for a pair of arguments (packed f32x2):
