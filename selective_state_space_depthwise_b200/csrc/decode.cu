@@ -92,21 +92,31 @@ __device__ __forceinline__ void decode_step_item(const KernelArgs& a, int64_t se
   const float zg = silu(it.z);
   float yl = 0.0f, yh = 0.0f;
   if constexpr (ZOH) {
+    const uint64_t dt2 = pk2(dt, dt), u2 = pk2(u, u);
+    uint64_t acc = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 b = Bq[q], cc = Cq[q];
-      const float bv[4] = {b.x, b.y, b.z, b.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-      float hs[4] = {it.h[q].x, it.h[q].y, it.h[q].z, it.h[q].w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float A = p.A[4 * q + i];
-        const float xa = dt * A;
-        const float dA = ex2_approx(xa * kLog2e);
-        hs[i] = fmaf(dA, hs[i], zoh_scale(xa, dt, dA, p.rA[4 * q + i]) * u * bv[i]);
-        yl = fmaf(cv[i], hs[i], yl);
+      for (int r = 0; r < 4; r += 2) {
+        const int i = 4 * q + r;
+        const uint64_t x = fmul2(dt2, pk2(p.A[i], p.A[i + 1]));
+        float l0, l1;
+        upk2(fmul2(x, pk2(kLog2e, kLog2e)), l0, l1);
+        const uint64_t ex = pk2(ex2_approx(l0), ex2_approx(l1));
+        const uint64_t sc = zoh_scale_pair(x, dt2, ex, pk2(p.rA[i], p.rA[i + 1]));
+        const uint64_t b2 = r == 0 ? pk2(b.x, b.y) : pk2(b.z, b.w);
+        const uint64_t c2 = r == 0 ? pk2(cc.x, cc.y) : pk2(cc.z, cc.w);
+        const uint64_t h2 = r == 0 ? pk2(it.h[q].x, it.h[q].y) : pk2(it.h[q].z, it.h[q].w);
+        const uint64_t hh = ffma2(ex, h2, fmul2(fmul2(sc, u2), b2));
+        acc = i == 0 ? fmul2(c2, hh) : ffma2(c2, hh, acc);
+        if (r == 0)
+          upk2(hh, it.h[q].x, it.h[q].y);
+        else
+          upk2(hh, it.h[q].z, it.h[q].w);
       }
-      it.h[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
     }
+    upk2(acc, yl, yh);
   } else {
     const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
     uint64_t acc = 0;
@@ -311,20 +321,31 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_tma_kernel(const __grid
       float yl = 0.0f, yh = 0.0f;
       if constexpr (ZOH) {
 #pragma unroll
+        const uint64_t dt2 = pk2(dt, dt), u2 = pk2(u, u);
+        uint64_t acc = 0;
+#pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float4 b = Bq[q], cc = Cq[q];
-          const float bv[4] = {b.x, b.y, b.z, b.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
-          float hs[4] = {h[q].x, h[q].y, h[q].z, h[q].w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float A = p.A[4 * q + i];
-            const float xa = dt * A;
-            const float dA = ex2_approx(xa * kLog2e);
-            hs[i] = fmaf(dA, hs[i], zoh_scale(xa, dt, dA, p.rA[4 * q + i]) * u * bv[i]);
-            yl = fmaf(cv[i], hs[i], yl);
+          for (int r = 0; r < 4; r += 2) {
+            const int i = 4 * q + r;
+            const uint64_t x = fmul2(dt2, pk2(p.A[i], p.A[i + 1]));
+            float l0, l1;
+            upk2(fmul2(x, pk2(kLog2e, kLog2e)), l0, l1);
+            const uint64_t ex = pk2(ex2_approx(l0), ex2_approx(l1));
+            const uint64_t sc = zoh_scale_pair(x, dt2, ex, pk2(p.rA[i], p.rA[i + 1]));
+            const uint64_t b2 = r == 0 ? pk2(b.x, b.y) : pk2(b.z, b.w);
+            const uint64_t c2 = r == 0 ? pk2(cc.x, cc.y) : pk2(cc.z, cc.w);
+            const uint64_t h2 = r == 0 ? pk2(h[q].x, h[q].y) : pk2(h[q].z, h[q].w);
+            const uint64_t hh = ffma2(ex, h2, fmul2(fmul2(sc, u2), b2));
+            acc = i == 0 ? fmul2(c2, hh) : ffma2(c2, hh, acc);
+            if (r == 0)
+              upk2(hh, h[q].x, h[q].y);
+            else
+              upk2(hh, h[q].z, h[q].w);
           }
-          h[q] = make_float4(hs[0], hs[1], hs[2], hs[3]);
         }
+        upk2(acc, yl, yh);
       } else {
         const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
         uint64_t acc = 0;

@@ -145,19 +145,7 @@ __device__ __forceinline__ float scan_token(uint64_t dt2, uint64_t inj2, const f
 }
 
 // Zero-order-hold decays, in state pairs: h = e^{dt A} h + (e^{dt A} - 1)/A
-// * u * B, the input scale as zoh_scale forms it (rA = 1 / A), each half of a
-// packed operation rounding as the scalar form does.
-__device__ __forceinline__ uint64_t zoh_scale_pair(uint64_t x, uint64_t dt2, uint64_t ex, uint64_t rA) {
-  uint64_t p = ffma2(x, pk2(1.0f / 120.0f, 1.0f / 120.0f), pk2(1.0f / 24.0f, 1.0f / 24.0f));
-  p = ffma2(x, p, pk2(1.0f / 6.0f, 1.0f / 6.0f));
-  p = ffma2(x, p, pk2(0.5f, 0.5f));
-  p = ffma2(x, p, pk2(1.0f, 1.0f));
-  float s0, s1, l0, l1, x0, x1;
-  upk2(fmul2(dt2, p), s0, s1);
-  upk2(fmul2(fadd2(ex, pk2(-1.0f, -1.0f)), rA), l0, l1);
-  upk2(x, x0, x1);
-  return pk2(x0 > -0.125f ? s0 : l0, x1 > -0.125f ? s1 : l1);
-}
+// * u * B, the input scale as zoh_scale_pair forms it (rA = 1 / A).
 template <int K>
 __device__ __forceinline__ float scan_token_zoh(float dt, float u, const float* Av, const float* rA, float* h,
                                                 const float* Bp, const float* Cp) {

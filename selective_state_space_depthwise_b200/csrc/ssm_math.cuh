@@ -6,11 +6,14 @@
 //  - log1p on [0, 1] as e * Q(e), Q a degree-8 polynomial whose maximum
 //    relative error on [0, 1] was minimised by the Remez exchange algorithm
 //    (fit_log1p_poly.py; 1.8e-7 in float32), FMA pipe only;
-//  - expm1 near 0 via its Taylor series through x^5 (|x| < 1/8: < 5e-8 rel.).
+//  - the zero-order-hold input scale (e^x - 1)/A near 0 as dt times the
+//    Taylor series of expm1(x)/x through x^4 (|x| < 1/8: < 5e-8 rel.).
 #pragma once
 
 #include <cuda_bf16.h>
 #include <stdint.h>
+
+#include "sm100_ptx.cuh"
 
 namespace ssm {
 
@@ -77,6 +80,20 @@ __device__ __forceinline__ float zoh_scale(float x, float dt, float ex, float rA
   p = fmaf(x, p, 0.5f);
   p = fmaf(x, p, 1.0f);
   return x > -0.125f ? dt * p : (ex - 1.0f) * rA;
+}
+
+// zoh_scale of two states at once (packed f32x2; each half rounds as the
+// scalar form does).
+__device__ __forceinline__ uint64_t zoh_scale_pair(uint64_t x, uint64_t dt2, uint64_t ex, uint64_t rA) {
+  uint64_t p = ffma2(x, pk2(1.0f / 120.0f, 1.0f / 120.0f), pk2(1.0f / 24.0f, 1.0f / 24.0f));
+  p = ffma2(x, p, pk2(1.0f / 6.0f, 1.0f / 6.0f));
+  p = ffma2(x, p, pk2(0.5f, 0.5f));
+  p = ffma2(x, p, pk2(1.0f, 1.0f));
+  float s0, s1, l0, l1, x0, x1;
+  upk2(fmul2(dt2, p), s0, s1);
+  upk2(fmul2(fadd2(ex, pk2(-1.0f, -1.0f)), rA), l0, l1);
+  upk2(x, x0, x1);
+  return pk2(x0 > -0.125f ? s0 : l0, x1 > -0.125f ? s1 : l1);
 }
 
 // 2^x for x <= 0 on the FMA pipe, for a pair of arguments (packed f32x2):
