@@ -73,6 +73,61 @@ struct ChannelParams {
   float rA[16];  // 1 / A (ZOH only)
 };
 
+// One channel's 16 states through one token: h = dA h + (input) B with dA =
+// e^{dt A}, the readout C.h returned in two halves (yl + yh). Euler-B: input
+// dt u; ZOH: input (e^{dt A} - 1)/A u (zoh_scale_pair). State pairs share
+// packed f32x2 operations.
+template <bool ZOH>
+__device__ __forceinline__ void channel_states(const ChannelParams& p, float dt, float u, const float4* Bq,
+                                               const float4* Cq, float4 (&h)[4], float& yl, float& yh) {
+  if constexpr (ZOH) {
+    const uint64_t dt2 = pk2(dt, dt), u2 = pk2(u, u);
+    uint64_t acc = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 b = Bq[q], cc = Cq[q];
+#pragma unroll
+      for (int r = 0; r < 4; r += 2) {
+        const int i = 4 * q + r;
+        const uint64_t x = fmul2(dt2, pk2(p.A[i], p.A[i + 1]));
+        float l0, l1;
+        upk2(fmul2(x, pk2(kLog2e, kLog2e)), l0, l1);
+        const uint64_t ex = pk2(ex2_approx(l0), ex2_approx(l1));
+        const uint64_t sc = zoh_scale_pair(x, dt2, ex, pk2(p.rA[i], p.rA[i + 1]));
+        const uint64_t b2 = r == 0 ? pk2(b.x, b.y) : pk2(b.z, b.w);
+        const uint64_t c2 = r == 0 ? pk2(cc.x, cc.y) : pk2(cc.z, cc.w);
+        const uint64_t h2 = r == 0 ? pk2(h[q].x, h[q].y) : pk2(h[q].z, h[q].w);
+        const uint64_t hh = ffma2(ex, h2, fmul2(fmul2(sc, u2), b2));
+        acc = i == 0 ? fmul2(c2, hh) : ffma2(c2, hh, acc);
+        if (r == 0)
+          upk2(hh, h[q].x, h[q].y);
+        else
+          upk2(hh, h[q].z, h[q].w);
+      }
+    }
+    upk2(acc, yl, yh);
+  } else {
+    const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
+    uint64_t acc = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 b = Bq[q], cc = Cq[q];
+      float x0, x1, x2, x3;
+      upk2(fmul2(dt2, pk2(p.a2[4 * q], p.a2[4 * q + 1])), x0, x1);
+      upk2(fmul2(dt2, pk2(p.a2[4 * q + 2], p.a2[4 * q + 3])), x2, x3);
+      const uint64_t h01 =
+          ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(h[q].x, h[q].y), fmul2(dtu2, pk2(b.x, b.y)));
+      const uint64_t h23 =
+          ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(h[q].z, h[q].w), fmul2(dtu2, pk2(b.z, b.w)));
+      acc = q == 0 ? fmul2(pk2(cc.x, cc.y), h01) : ffma2(pk2(cc.x, cc.y), h01, acc);
+      acc = ffma2(pk2(cc.z, cc.w), h23, acc);
+      upk2(h01, h[q].x, h[q].y);
+      upk2(h23, h[q].z, h[q].w);
+    }
+    upk2(acc, yl, yh);
+  }
+}
+
 // Rows of the staged per-sequence inputs: B (16), C (16), dt_raw (1), padding.
 constexpr int kStageSeqs = 32;
 #ifndef SSM_DECODE_SETS
@@ -91,52 +146,7 @@ __device__ __forceinline__ void decode_step_item(const KernelArgs& a, int64_t se
   const float dt = dt_of(fmaf(row[32], p.wdt, p.dtb), a.dt_min, a.dt_max);
   const float zg = silu(it.z);
   float yl = 0.0f, yh = 0.0f;
-  if constexpr (ZOH) {
-    const uint64_t dt2 = pk2(dt, dt), u2 = pk2(u, u);
-    uint64_t acc = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 b = Bq[q], cc = Cq[q];
-#pragma unroll
-      for (int r = 0; r < 4; r += 2) {
-        const int i = 4 * q + r;
-        const uint64_t x = fmul2(dt2, pk2(p.A[i], p.A[i + 1]));
-        float l0, l1;
-        upk2(fmul2(x, pk2(kLog2e, kLog2e)), l0, l1);
-        const uint64_t ex = pk2(ex2_approx(l0), ex2_approx(l1));
-        const uint64_t sc = zoh_scale_pair(x, dt2, ex, pk2(p.rA[i], p.rA[i + 1]));
-        const uint64_t b2 = r == 0 ? pk2(b.x, b.y) : pk2(b.z, b.w);
-        const uint64_t c2 = r == 0 ? pk2(cc.x, cc.y) : pk2(cc.z, cc.w);
-        const uint64_t h2 = r == 0 ? pk2(it.h[q].x, it.h[q].y) : pk2(it.h[q].z, it.h[q].w);
-        const uint64_t hh = ffma2(ex, h2, fmul2(fmul2(sc, u2), b2));
-        acc = i == 0 ? fmul2(c2, hh) : ffma2(c2, hh, acc);
-        if (r == 0)
-          upk2(hh, it.h[q].x, it.h[q].y);
-        else
-          upk2(hh, it.h[q].z, it.h[q].w);
-      }
-    }
-    upk2(acc, yl, yh);
-  } else {
-    const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
-    uint64_t acc = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 b = Bq[q], cc = Cq[q];
-      float x0, x1, x2, x3;
-      upk2(fmul2(dt2, pk2(p.a2[4 * q], p.a2[4 * q + 1])), x0, x1);
-      upk2(fmul2(dt2, pk2(p.a2[4 * q + 2], p.a2[4 * q + 3])), x2, x3);
-      const uint64_t h01 =
-          ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(it.h[q].x, it.h[q].y), fmul2(dtu2, pk2(b.x, b.y)));
-      const uint64_t h23 =
-          ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(it.h[q].z, it.h[q].w), fmul2(dtu2, pk2(b.z, b.w)));
-      acc = q == 0 ? fmul2(pk2(cc.x, cc.y), h01) : ffma2(pk2(cc.x, cc.y), h01, acc);
-      acc = ffma2(pk2(cc.z, cc.w), h23, acc);
-      upk2(h01, it.h[q].x, it.h[q].y);
-      upk2(h23, it.h[q].z, it.h[q].w);
-    }
-    upk2(acc, yl, yh);
-  }
+  channel_states<ZOH>(p, dt, u, Bq, Cq, it.h, yl, yh);
   float4* hp = reinterpret_cast<float4*>(a.ssm_state_out) + (seq * a.E + e) * 4;
 #pragma unroll
   for (int q = 0; q < 4; ++q) hp[q] = it.h[q];
@@ -319,51 +329,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_tma_kernel(const __grid
       const float dt = dt_of(fmaf(row[32], p.wdt, p.dtb), a.dt_min, a.dt_max);
       const float zg = silu(cur[4]);
       float yl = 0.0f, yh = 0.0f;
-      if constexpr (ZOH) {
-#pragma unroll
-        const uint64_t dt2 = pk2(dt, dt), u2 = pk2(u, u);
-        uint64_t acc = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 b = Bq[q], cc = Cq[q];
-#pragma unroll
-          for (int r = 0; r < 4; r += 2) {
-            const int i = 4 * q + r;
-            const uint64_t x = fmul2(dt2, pk2(p.A[i], p.A[i + 1]));
-            float l0, l1;
-            upk2(fmul2(x, pk2(kLog2e, kLog2e)), l0, l1);
-            const uint64_t ex = pk2(ex2_approx(l0), ex2_approx(l1));
-            const uint64_t sc = zoh_scale_pair(x, dt2, ex, pk2(p.rA[i], p.rA[i + 1]));
-            const uint64_t b2 = r == 0 ? pk2(b.x, b.y) : pk2(b.z, b.w);
-            const uint64_t c2 = r == 0 ? pk2(cc.x, cc.y) : pk2(cc.z, cc.w);
-            const uint64_t h2 = r == 0 ? pk2(h[q].x, h[q].y) : pk2(h[q].z, h[q].w);
-            const uint64_t hh = ffma2(ex, h2, fmul2(fmul2(sc, u2), b2));
-            acc = i == 0 ? fmul2(c2, hh) : ffma2(c2, hh, acc);
-            if (r == 0)
-              upk2(hh, h[q].x, h[q].y);
-            else
-              upk2(hh, h[q].z, h[q].w);
-          }
-        }
-        upk2(acc, yl, yh);
-      } else {
-        const uint64_t dt2 = pk2(dt, dt), dtu2 = pk2(dt * u, dt * u);
-        uint64_t acc = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 b = Bq[q], cc = Cq[q];
-          float x0, x1, x2, x3;
-          upk2(fmul2(dt2, pk2(p.a2[4 * q], p.a2[4 * q + 1])), x0, x1);
-          upk2(fmul2(dt2, pk2(p.a2[4 * q + 2], p.a2[4 * q + 3])), x2, x3);
-          const uint64_t h01 = ffma2(pk2(ex2_approx(x0), ex2_approx(x1)), pk2(h[q].x, h[q].y), fmul2(dtu2, pk2(b.x, b.y)));
-          const uint64_t h23 = ffma2(pk2(ex2_approx(x2), ex2_approx(x3)), pk2(h[q].z, h[q].w), fmul2(dtu2, pk2(b.z, b.w)));
-          acc = q == 0 ? fmul2(pk2(cc.x, cc.y), h01) : ffma2(pk2(cc.x, cc.y), h01, acc);
-          acc = ffma2(pk2(cc.z, cc.w), h23, acc);
-          upk2(h01, h[q].x, h[q].y);
-          upk2(h23, h[q].z, h[q].w);
-        }
-        upk2(acc, yl, yh);
-      }
+      channel_states<ZOH>(p, dt, u, Bq, Cq, h, yl, yh);
 #pragma unroll
       for (int q = 0; q < 4; ++q) *reinterpret_cast<float4*>(tile + sw64(tid, q)) = h[q];
       static_cast<T*>(a.y)[seq * a.s.y_seq + e] = IO<T>::from_f((yl + yh + p.D * u) * zg);

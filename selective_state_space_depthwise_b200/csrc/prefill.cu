@@ -16,7 +16,7 @@
 // Thread 0 re-arms a slot right after the CTA has finished with it; every
 // wait on the ring's mbarriers is bounded.
 //
-// Work split (state slices). A CTA is G warps (G = 2 or 4) over 32 channels
+// Work split (state slices). A CTA is G = 4 warps over 32 channels
 // (lane = channel); warp j holds states 16j/G .. 16(j+1)/G - 1 of every
 // channel, so B and C are warp-broadcast loads and x, z, y are lane-contiguous.
 // Each 32-token stage:
@@ -47,9 +47,9 @@
 // Kernels. 3: G = 4 with the register budget of three CTAs per SM; 4: G = 4
 // built for two CTAs per SM, whose larger register budget buys a deeper
 // schedule; 5: the same state slices with phases A and C in four more warps
-// of the CTA, handing over through mbarriers (ws_run). Measured alternatives at the long-context shape: G = 2 (8 states
-// a thread) executes ~13% fewer instructions per channel-token but runs 1.28x
-// slower (one warp per SM sub-partition leaves dependency latencies exposed);
+// of the CTA, handing over through mbarriers (ws_run). Measured alternatives
+// at the long-context shape: G = 2 (8 states a thread) executes ~13% fewer
+// instructions per channel-token but runs 1.28x slower (one warp per SM sub-partition leaves dependency latencies exposed);
 // G = 8 (2 states a thread, 16 warps per SM) runs 1.36x slower: with two
 // states a thread the power path saves nothing, and the 16 per-state
 // exponentials and the B/C loads then saturate the shared MIO queue. A power
