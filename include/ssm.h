@@ -154,6 +154,12 @@ ssm_status ssm_prefill_ex(const ssm_dims *dims, const ssm_weights *w, const void
  * single-pass kernel covers). Returns 0 for invalid dims as well. */
 size_t ssm_prefill_workspace_bytes(const ssm_dims *dims);
 
+/* The prefill kernel (3, 4 or 5; see ssm_tuning) that ssm_prefill launches
+ * for `dims` and `tuning` (NULL = defaults) on a GPU of `num_sms` SMs
+ * (<= 0: the current device's). Host-only: with num_sms > 0 it makes no CUDA
+ * call. Returns 0 where ssm_prefill would reject the dims or the tuning. */
+int32_t ssm_prefill_kernel(const ssm_dims *dims, const ssm_tuning *tuning, int32_t num_sms);
+
 /*
  * ssm_prefill_host -- ssm_prefill with the token tensors in HOST memory. The
  * block core is the same, from the same pages and sections as ssm_prefill:

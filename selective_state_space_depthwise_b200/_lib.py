@@ -24,6 +24,7 @@ EXPORTED = (
     "ssm_prefill",
     "ssm_prefill_ex",
     "ssm_prefill_workspace_bytes",
+    "ssm_prefill_kernel",
     "ssm_prefill_host",
     "ssm_prefill_host_workspace_bytes",
     "ssm_prefill_host_static",
@@ -124,6 +125,8 @@ def load(path: str = LIB_PATH):
     lib.ssm_prefill_ex.restype = st
     lib.ssm_prefill_workspace_bytes.argtypes = [dims_p]
     lib.ssm_prefill_workspace_bytes.restype = sz
+    lib.ssm_prefill_kernel.argtypes = [dims_p, tun_p, ctypes.c_int32]
+    lib.ssm_prefill_kernel.restype = ctypes.c_int32
     lib.ssm_prefill_host.argtypes = [dims_p, w_p] + [p] * 10 + [p, sz, ctypes.c_int64, p]
     lib.ssm_prefill_host.restype = st
     lib.ssm_prefill_host_static.argtypes = [dims_p, w_p] + [p] * 10 + [ctypes.c_int64, p]

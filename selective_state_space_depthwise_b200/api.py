@@ -54,6 +54,16 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _tuning_ref(tuning):
+    """ssm_tuning from a dict {"kernel": k, "decay_path": d} (None: defaults)."""
+    if not tuning:
+        return None
+    unknown = set(tuning) - {"kernel", "decay_path"}
+    if unknown:
+        raise ValueError(f"unknown tuning keys {sorted(unknown)} (kernel, decay_path)")
+    return ctypes.byref(_lib.SsmTuning(int(tuning.get("kernel", 0)), int(tuning.get("decay_path", 0))))
+
+
 def make_dims(batch, seqlen, E, io_dtype, dt_min=1e-4, dt_max=1.0, discretization="euler", **strides):
     d = _lib.SsmDims()
     d.batch, d.seqlen, d.d_inner, d.d_state, d.d_conv = batch, seqlen, E, 16, 4
@@ -68,6 +78,16 @@ def make_dims(batch, seqlen, E, io_dtype, dt_min=1e-4, dt_max=1.0, discretizatio
 def workspace_bytes(batch, seqlen, E, io_dtype=torch.bfloat16) -> int:
     lib = _lib.load()
     return int(lib.ssm_prefill_workspace_bytes(ctypes.byref(make_dims(batch, seqlen, E, io_dtype))))
+
+
+def prefill_kernel(batch, seqlen, E, io_dtype=torch.bfloat16, discretization="euler", tuning=None,
+                   num_sms=0) -> int:
+    """The prefill kernel (3, 4 or 5) `prefill` launches for this shape and
+    tuning on a GPU of num_sms SMs (0: the current device's); 0 where the call
+    would be rejected. Host-only for num_sms > 0."""
+    lib = _lib.load()
+    dims = make_dims(batch, seqlen, E, io_dtype, discretization=discretization)
+    return int(lib.ssm_prefill_kernel(ctypes.byref(dims), _tuning_ref(tuning), int(num_sms)))
 
 
 def prefill(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None, y=None, conv_cache_out=None,
@@ -111,15 +131,9 @@ def prefill(x, z, B, C, dt_raw, params, *, conv_cache_in=None, ssm_state_in=None
     w = _weights(params, E, dev)
     ws = int(lib.ssm_prefill_workspace_bytes(ctypes.byref(dims)))
     work = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
-    tun = None
-    if tuning:
-        unknown = set(tuning) - {"kernel", "decay_path"}
-        if unknown:
-            raise ValueError(f"unknown tuning keys {sorted(unknown)} (kernel, decay_path)")
-        tun = _lib.SsmTuning(int(tuning.get("kernel", 0)), int(tuning.get("decay_path", 0)))
     st = lib.ssm_prefill_ex(ctypes.byref(dims), ctypes.byref(w), _ptr(x), _ptr(z), _ptr(B), _ptr(C), _ptr(dt_raw),
                             _ptr(conv_cache_in), _ptr(ssm_state_in), _ptr(y), _ptr(conv_cache_out),
-                            _ptr(ssm_state_out), _ptr(work), ws, ctypes.byref(tun) if tun else None, _stream(stream))
+                            _ptr(ssm_state_out), _ptr(work), ws, _tuning_ref(tuning), _stream(stream))
     _lib.check(st)
     return y, conv_cache_out, ssm_state_out
 

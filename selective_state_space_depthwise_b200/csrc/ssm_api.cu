@@ -168,6 +168,26 @@ int* device_error_ptr() {
 namespace {
 using ssm::device_error_ptr;
 
+// The prefill launch shape for `dims` and `tuning` on a GPU of `num_sms` SMs:
+// the automatic choice, or the one `tuning` names; the tuning's fields are
+// checked here. Host-only.
+ssm_status resolve_prefill_shape(const ssm_dims* dims, const ssm_tuning* tuning, int num_sms,
+                                 ssm::PrefillShape* sh, int* decay_path) {
+  const bool per_state = dims->discretization == SSM_DISC_ZOH || (tuning && tuning->decay_path == 1);
+  *sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms, per_state);
+  *decay_path = 0;
+  if (tuning) {
+    if (tuning->kernel) sh->kernel = tuning->kernel;
+    if (!ssm::prefill_shape_supported(*sh))
+      return fail(SSM_ERR_INVALID_ARG, "tuning: kernel=%d is not built (3, 4 or 5)", sh->kernel);
+    if (tuning->decay_path != 0 && tuning->decay_path != 1)
+      return fail(SSM_ERR_INVALID_ARG, "tuning: decay_path=%d (0 = auto, 1 = per-state exponentials)",
+                  tuning->decay_path);
+    *decay_path = tuning->decay_path;
+  }
+  return SSM_OK;
+}
+
 }  // namespace
 
 namespace ssm {
@@ -191,19 +211,9 @@ ssm_status prefill_entry(const ssm_dims* dims, const ssm_weights* w, const void*
   }
   if ((st = check_prefill_caches(conv_cache_in, ssm_state_in, conv_cache_out, ssm_state_out)) != SSM_OK) return st;
 
-  const bool per_state = dims->discretization == SSM_DISC_ZOH || (tuning && tuning->decay_path == 1);
-  ssm::PrefillShape sh = ssm::choose_prefill_shape(dims->batch, dims->d_inner, dims->seqlen, num_sms_current(),
-                                                   per_state);
+  ssm::PrefillShape sh;
   int decay_path = 0;
-  if (tuning) {
-    if (tuning->kernel) sh.kernel = tuning->kernel;
-    if (!ssm::prefill_shape_supported(sh))
-      return fail(SSM_ERR_INVALID_ARG, "tuning: kernel=%d is not built (3, 4 or 5)", sh.kernel);
-    if (tuning->decay_path != 0 && tuning->decay_path != 1)
-      return fail(SSM_ERR_INVALID_ARG, "tuning: decay_path=%d (0 = auto, 1 = per-state exponentials)",
-                  tuning->decay_path);
-    decay_path = tuning->decay_path;
-  }
+  if ((st = resolve_prefill_shape(dims, tuning, num_sms_current(), &sh, &decay_path)) != SSM_OK) return st;
 
   ssm::KernelArgs a{};
   a.x = x;
@@ -239,6 +249,16 @@ extern "C" {
 size_t ssm_prefill_workspace_bytes(const ssm_dims* dims) {
   (void)dims;
   return 0;
+}
+
+int32_t ssm_prefill_kernel(const ssm_dims* dims, const ssm_tuning* tuning, int32_t num_sms) {
+  ssm::Strides s;
+  if (check_dims(dims, true, &s) != SSM_OK) return 0;
+  ssm::PrefillShape sh;
+  int decay_path = 0;
+  if (resolve_prefill_shape(dims, tuning, num_sms > 0 ? num_sms : num_sms_current(), &sh, &decay_path) != SSM_OK)
+    return 0;
+  return sh.kernel;
 }
 
 ssm_status ssm_prefill_ex(const ssm_dims* dims, const ssm_weights* w, const void* x, const void* z, const float* B,

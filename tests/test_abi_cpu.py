@@ -260,3 +260,24 @@ def test_segment_carry_argument_checks(lib):
 def test_selftest_rejects_bad_limits_on_the_host(lib):
     for bad in (0, 999, 2_000_000_001):
         assert lib.ssm_selftest_bounded_wait(bad, None) == _lib.SSM_ERR_INVALID_ARG
+
+
+def test_prefill_kernel_choice_on_the_host(lib):
+    """The automatic launch shape, on the host for a 148-SM GPU: kernel 5 up
+    to one CTA (32 channels of one sequence) per SM; kernel 4 up to 64 CTAs
+    per SM, unless every CTA runs per-state exponentials (ZOH, or decay_path
+    1), where kernel 5 stays; kernel 3 beyond; an explicit kernel wins; a
+    rejected tuning or shape gives 0."""
+    k = lambda b, E, **kw: api.prefill_kernel(b, 1024, E, num_sms=148, **kw)
+    assert k(1, 32) == 5 and k(1, 4736) == 5 and k(2, 2368) == 5  # 1, 148, 148 CTAs
+    assert k(1, 4768) == 4 and k(1, 7680) == 4 and k(8, 5120) == 4  # 149, 240, 1280 CTAs
+    assert k(1, 7680, discretization="zoh") == 5
+    assert k(1, 7680, tuning={"decay_path": 1}) == 5
+    assert k(64 * 148, 32) == 4 and k(64 * 148 + 1, 32) == 3
+    assert k(64 * 148 + 1, 32, discretization="zoh") == 3
+    assert k(256, 7680) == 3  # the decode prompt's 61440 CTAs
+    assert k(1, 7680, tuning={"kernel": 3}) == 3 and k(1, 32, tuning={"kernel": 4}) == 4
+    assert k(1, 7680, tuning={"kernel": 2}) == 0
+    assert k(1, 7680, tuning={"decay_path": 2}) == 0
+    assert k(1, 7684) == 0  # E not a multiple of 8
+    assert api.prefill_kernel(1, 1024, 7680, num_sms=74) == 4 and api.prefill_kernel(1, 1024, 2368, num_sms=74) == 5
