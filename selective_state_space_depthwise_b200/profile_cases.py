@@ -1,6 +1,6 @@
 """Small, fixed launches of the kernels for profiler captures.
 
-    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL DECAY_PATH] [E]
+    python -m selective_state_space_depthwise_b200.profile_cases prefill WORKLOAD [L] [KERNEL DECAY_PATH] [E] [DISC]
     python -m selective_state_space_depthwise_b200.profile_cases decode [BATCH]
     python -m selective_state_space_depthwise_b200.profile_cases block NAME [L]
     python -m selective_state_space_depthwise_b200.profile_cases ssd NAME
@@ -9,7 +9,7 @@
 
 prefill: three launches of the named workload's prefill (optionally shortened
 to L tokens, optionally with an explicit kernel (3, 4 or 5) and decay path (0 auto,
-1 per-state exponentials), and E channels); decode: a 4-token
+1 per-state exponentials), E channels and the discretisation, euler or zoh); decode: a 4-token
 prompt, then three decode steps at the decode workload's shape (batch 256,
 E=7680, 252 MB of state); block: three block forwards of the named block
 workload (optionally L tokens); segment: three segment summaries of the first
@@ -27,7 +27,7 @@ from . import api
 from . import workloads as W
 
 
-def prefill_case(name: str, L: int = 0, shape=None, E: int = 0):
+def prefill_case(name: str, L: int = 0, shape=None, E: int = 0, disc: str = "euler"):
     w = W.WORKLOADS[name]
     if L > 0:
         w = w.scaled(seqlen=L)
@@ -40,7 +40,7 @@ def prefill_case(name: str, L: int = 0, shape=None, E: int = 0):
     inp = W.make_inputs(w, device="cuda", gen_device="cuda")
     args = (inp["x"], inp["z"], inp["B"], inp["C"], inp["dt_raw"], inp)
     for _ in range(3):
-        y, _, _ = api.prefill(*args, tuning=tun)
+        y, _, _ = api.prefill(*args, tuning=tun, discretization=disc)
     torch.cuda.synchronize()
     print("prefill ok", name, w.seqlen, w.d_inner, float(y.float().abs().mean()))
 
@@ -108,7 +108,7 @@ if __name__ == "__main__":
         L = int(sys.argv[3]) if len(sys.argv) > 3 else 0
         shape = tuple(int(v) for v in sys.argv[4:6]) if len(sys.argv) > 5 else None
         E = int(sys.argv[6]) if len(sys.argv) > 6 else 0
-        prefill_case(sys.argv[2], L, shape, E)
+        prefill_case(sys.argv[2], L, shape, E, sys.argv[7] if len(sys.argv) > 7 else "euler")
     elif sys.argv[1] == "ssd":
         ssd_case(sys.argv[2])
     elif sys.argv[1] == "block":
