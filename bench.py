@@ -404,7 +404,8 @@ def e2e_prefill(w: W.Workload, inp, steps):
     ms = ev0.elapsed_time(ev1) / steps
     return {"value": b * L * E / (ms * 1e-3), "unit": "channel-tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3),
-            "path": "ssm_prefill_host: 2048-token chunks, H2D / kernel / D2H overlapped on three streams"}
+            "path": ("ssm_prefill_host: 4096-token chunks (the last 4096 tokens as quarters), H2D / kernel / D2H "
+                     "overlapped on three streams")}
 
 
 def decode_bench(w: W.Workload, rank: int, hbm_peak: float, peak_kind: str):

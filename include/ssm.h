@@ -166,8 +166,10 @@ int32_t ssm_prefill_kernel(const ssm_dims *dims, const ssm_tuning *tuning, int32
  * prefill of "Axon-SSM: selective state space model", "Algorithm".
  *
  * What it does. x, z, B, C and dt_raw are read from host buffers, and y is
- * written to a host buffer. L is processed in chunks of chunk_tokens tokens,
- * and three kinds of work overlap chunk by chunk:
+ * written to a host buffer. L is processed in chunks of chunk_tokens tokens
+ * (when L is longer than one chunk, its last chunk_tokens tokens go as four
+ * quarter chunks, so that the pipeline drains after a short kernel and
+ * copy-out), and three kinds of work overlap chunk by chunk:
  *  - the host->device copies of chunk c + 1, on an internal copy-in stream;
  *  - the kernel of chunk c, on `stream`;
  *  - the device->host copy of chunk c - 1's y, on an internal copy-out stream.
@@ -189,7 +191,7 @@ int32_t ssm_prefill_kernel(const ssm_dims *dims, const ssm_tuning *tuning, int32
  *   workspace               device scratch of at least
  *                           ssm_prefill_host_workspace_bytes(dims, chunk_tokens)
  *                           bytes, 256-byte aligned. It holds two chunk buffers.
- *   chunk_tokens            tokens per chunk, >= 1; 0 selects 2048.
+ *   chunk_tokens            tokens per chunk, >= 1; 0 selects 4096.
  *
  * Ordering. The call returns once every copy and kernel is enqueued. The first
  * copy waits for the work already queued on `stream`, and `stream` waits for
@@ -207,7 +209,7 @@ ssm_status ssm_prefill_host(const ssm_dims *dims, const ssm_weights *w, const vo
                             void *workspace, size_t workspace_bytes, int64_t chunk_tokens, void *stream);
 
 /* Device scratch bytes ssm_prefill_host needs for `dims` and `chunk_tokens`
- * (0 selects 2048): two chunk buffers of x, z, y, B, C and dt_raw. Returns 0
+ * (0 selects 4096): two chunk buffers of x, z, y, B, C and dt_raw. Returns 0
  * for invalid dims. */
 size_t ssm_prefill_host_workspace_bytes(const ssm_dims *dims, int64_t chunk_tokens);
 

@@ -3,7 +3,8 @@
 // static device scratch of the second entry point; the kernels are
 // prefill.cu's).
 //
-// The sequence is cut into chunks of T tokens and pipelined over three streams:
+// The sequence is cut into chunks of at most T tokens (the last T tokens of a
+// longer sequence as quarters) and pipelined over three streams:
 //   copy-in  (internal):  H2D of chunk c's x, z, B, C, dt_raw into slot c % 2;
 //   compute  (caller's):  the prefill kernel of chunk c on slot c % 2, its
 //                         caches chained from chunk c - 1 (conv_cache_out and
@@ -33,7 +34,8 @@
 
 namespace {
 
-constexpr int64_t kDefaultChunk = 2048;
+constexpr int64_t kDefaultChunk = 4096;        // ssm_prefill_host's chunk (chunk_tokens 0)
+constexpr int64_t kStaticChunkCap = 2048;      // the static variant's largest automatic chunk
 constexpr size_t kAlign = 256;
 constexpr size_t kStaticScratchBytes = SSM_HOST_STATIC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
@@ -218,7 +220,18 @@ ssm_status enqueue(const HostPrefill& hp, char* ws, int64_t T, cudaStream_t cs, 
   cd.bc_seq_stride = T * 16;
   cd.dt_seq_stride = T;
 
-  const int64_t n_chunks = (L + T - 1) / T;
+  // Chunk lengths: T tokens at a time, except that a sequence longer than one
+  // chunk sends its last T tokens as quarters, so the pipeline drains after a
+  // short kernel and copy-out (the caches carry across any cut, so the result
+  // does not depend on where the chunks fall).
+  const int64_t quarter = (T + 3) / 4;
+  auto chunk_len = [&](int64_t t0) -> int64_t {
+    const int64_t rem = L - t0;
+    if (L <= T) return rem;
+    if (rem > 2 * T) return T;
+    if (rem > T) return rem - T;  // leaves exactly T tokens for the quarters
+    return rem < quarter ? rem : quarter;
+  };
   ssm_status result = SSM_OK;
   cudaError_t e = cudaSuccess;
   int64_t last_out = -1;  // the last chunk whose copy-out was enqueued
@@ -229,9 +242,10 @@ ssm_status enqueue(const HostPrefill& hp, char* ws, int64_t T, cudaStream_t cs, 
       cuda_fail("start");
       break;
     }
-    for (int64_t c = 0; c < n_chunks; ++c) {
+    int64_t t0 = 0, Tc = 0;
+    for (int64_t c = 0; t0 < L; ++c, t0 += Tc) {
       const int k = static_cast<int>(c & 1);
-      const int64_t t0 = c * T, Tc = (L - t0 < T) ? L - t0 : T;
+      Tc = chunk_len(t0);
       char* base = slot_base[k];
       // copy-in of chunk c (slot k was last read by the kernel of chunk c - 2)
       if (c >= 2 && (e = cudaStreamWaitEvent(ds->in, ev.comp[k], 0)) != cudaSuccess) {
@@ -291,13 +305,13 @@ ssm_status enqueue(const HostPrefill& hp, char* ws, int64_t T, cudaStream_t cs, 
   return result;
 }
 
-// Largest chunk (at most kDefaultChunk tokens, at most L) whose two slots fit
+// Largest chunk (at most kStaticChunkCap tokens, at most L) whose two slots fit
 // `bytes`; 0 if not even one token fits.
 int64_t largest_fitting_chunk(const ssm_dims* d, size_t bytes) {
   const size_t es = io_size(d);
   const int64_t b = d->batch, E = d->d_inner;
   const size_t per_token = 2 * static_cast<size_t>(b) * (3 * static_cast<size_t>(E) * es + 2 * 64 + 4);
-  int64_t T = clip_chunk(kDefaultChunk, d->seqlen);
+  int64_t T = clip_chunk(kStaticChunkCap, d->seqlen);
   const int64_t est = static_cast<int64_t>(bytes / per_token);
   if (est < T) T = est;
   while (T > 0 && 2 * slot_layout(b, T, E, es).bytes > bytes) --T;

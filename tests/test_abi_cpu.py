@@ -143,11 +143,11 @@ def test_host_workspace_bytes_cover_two_chunk_slots(lib):
 
     d = valid_dims()  # b=2, L=64, E=32, bf16
     assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 16) == 2 * slot(2, 16, 32, 2)
-    # chunk 0 selects 2048 tokens, clipped to the sequence length
+    # chunk 0 selects 4096 tokens, clipped to the sequence length
     assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 0) == 2 * slot(2, 64, 32, 2)
     assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), 1000) == 2 * slot(2, 64, 32, 2)
     d32 = api.make_dims(1, 5000, 64, torch.float32)
-    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d32), 0) == 2 * slot(1, 2048, 64, 4)
+    assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d32), 0) == 2 * slot(1, 4096, 64, 4)
     assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(d), -1) == 0
     assert lib.ssm_prefill_host_workspace_bytes(ctypes.byref(valid_dims(d_state=8)), 16) == 0
     assert lib.ssm_prefill_host_workspace_bytes(None, 16) == 0
