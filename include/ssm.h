@@ -157,7 +157,9 @@ size_t ssm_prefill_workspace_bytes(const ssm_dims *dims);
 /* The prefill kernel (3, 4 or 5; see ssm_tuning) that ssm_prefill launches
  * for `dims` and `tuning` (NULL = defaults) on a GPU of `num_sms` SMs
  * (<= 0: the current device's). Host-only: with num_sms > 0 it makes no CUDA
- * call. Returns 0 where ssm_prefill would reject the dims or the tuning. */
+ * call. Returns 0 where ssm_prefill would reject the dims or the tuning. With
+ * seqlen 0 ssm_prefill runs no scan kernel (it only passes the caches on);
+ * the value is then the shape the same call would take with tokens. */
 int32_t ssm_prefill_kernel(const ssm_dims *dims, const ssm_tuning *tuning, int32_t num_sms);
 
 /*
